@@ -1,0 +1,148 @@
+/*
+ * gdn.h -- C ABI of the looped gated delta-rule (GDN) mixer library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation ("LT2: Linear-Time Looped Transformers", §2, "LT2."
+ * paragraph): a looped transformer applies its shared block stack T times; in
+ * LT2 the block's token mixer is a linear-attention recurrence with queries and
+ * keys q_t, k_t in R^{dk}, values v_t in R^{dv} and a recurrent state
+ * S_t in R^{dk x dv}.  The mixer used here is Gated DeltaNet (named among the
+ * LT2 mixers, Appendix C).  In the page's dk x dv orientation the state update
+ * and readout are
+ *
+ *     S_t = a_t (I - b_t k_t k_t^T) S_{t-1} + b_t k_t v_t^T,   o_t = scale * S_t^T q_t
+ *
+ * (a rank-1, diagonal-plus-low-rank update, §2 and Appendix B.1), and the
+ * per-loop residual across iterations is h^(tau) = h~^(tau) + rho_tau (.) h^(tau-1)
+ * with a per-channel gate rho_tau in R^d (§2, "LT2." paragraph).
+ *
+ * Conventions for every entry point
+ *   - All pointers passed to the compute calls are DEVICE pointers unless a
+ *     parameter says otherwise; the caller owns every buffer.  The compute calls
+ *     never allocate, free or synchronise; they enqueue work on `stream` and
+ *     return.
+ *   - Tensors are dense and row-major in the layouts given below; every
+ *     pointer must be 16-byte aligned.
+ *   - Argument errors are detected on the host and returned before anything is
+ *     launched (GDN_ERR_INVALID, GDN_ERR_UNSUPPORTED).  A failed launch returns
+ *     GDN_ERR_CUDA.  A device-side wait that exceeds its iteration limit records
+ *     GDN_ERR_TIMEOUT in a device status word, read (and cleared) by
+ *     gdn_get_device_status().
+ *   - Thread safety: calls on different streams may run concurrently; they share
+ *     only read-only launch constants and the device status word.
+ */
+#ifndef LOOPED_GDN_H
+#define LOOPED_GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID = 1,     /* null pointer, bad size, misaligned pointer      */
+    GDN_ERR_UNSUPPORTED = 2, /* shape/dtype combination this build does not run */
+    GDN_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed     */
+    GDN_ERR_TIMEOUT = 4,     /* a device-side wait hit its iteration limit      */
+    GDN_ERR_WORKSPACE = 5    /* workspace pointer/size below the queried need   */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Flags for gdn_fwd_params.flags and gdn_decode_step(). */
+#define GDN_QK_L2NORM 0x1u /* normalise q and k per head in fp32 before use:
+                              x / sqrt(sum x^2 + 1e-6), then round to io dtype */
+#define GDN_PRECISE   0x2u /* prefill: use the fp32 CUDA-core chunk kernel even
+                              for bf16 inputs (slower, fp32 operands)          */
+
+/*
+ * Prefill over packed or variable-length sequences.
+ *
+ *   q, k       [total_tokens][H][dk]   io_dtype
+ *   v          [total_tokens][H][dv]   io_dtype
+ *   a, b       [total_tokens][H]       fp32.  a_t in (0, 1] is the decay gate,
+ *                                      b_t the write strength (any finite value;
+ *                                      b in [0, 2] keeps ||I - b k k^T|| <= 1 for
+ *                                      unit keys, Appendix B.1).
+ *   S0         [n_seq][H][dk][dv]      fp32, or NULL for a zero initial state
+ *   o          [total_tokens][H][dv]   io_dtype, written
+ *   S_T        [n_seq][H][dk][dv]      fp32 final state, or NULL to skip; may
+ *                                      alias S0 exactly (in-place update)
+ *   cu_seqlens device int32 [n_seq+1] token offsets (0 = cu[0] <= ... <= cu[n_seq]
+ *              = total_tokens), or NULL: n_seq sequences of seq_len tokens each
+ *              (total_tokens = n_seq * seq_len).
+ *   scale      multiplies every output (1.0 reproduces the recurrence as written).
+ * Each (sequence, head) chain starts from its S0 and runs the recurrence over its
+ * own tokens; a sequence of length 0 writes no output and S_T = S0.
+ * o must not overlap q, k, v, a, b, S0 or S_T.
+ *
+ * Supported: dk in {64, 128}; dv a multiple of 64, at most 512; H >= 1.
+ * bf16 with dk = 128 and dv a multiple of 128 runs on the tensor-core (tcgen05)
+ * kernel; fp32, or any other supported shape, or GDN_PRECISE, runs on the fp32
+ * CUDA-core chunk kernel.
+ */
+typedef struct {
+    const void *q, *k, *v;
+    const float *a, *b;
+    const float *S0;
+    void *o;
+    float *S_T;
+    const int32_t *cu_seqlens;
+    int n_seq, seq_len, total_tokens, H, dk, dv;
+    gdn_dtype io_dtype;
+    float scale;
+    unsigned flags;
+} gdn_fwd_params;
+
+/* Bytes of device workspace gdn_chunk_fwd needs for these parameters (may be 0).
+ * Returns (size_t)-1 if the parameters are invalid. */
+size_t gdn_chunk_fwd_workspace(const gdn_fwd_params *p);
+
+/* Chunkwise prefill (chunks of 64 tokens).  ws/ws_bytes: device workspace of at
+ * least gdn_chunk_fwd_workspace(p) bytes (NULL/0 allowed when that is 0). */
+gdn_status gdn_chunk_fwd(const gdn_fwd_params *p, void *ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/*
+ * One decode step: one new token for each of N independent state slots (a slot
+ * is one sequence x layer x loop state), H heads each.
+ *   q, k [N][H][dk], v [N][H][dv], o [N][H][dv]  io_dtype
+ *   a, b [N][H] fp32
+ *   S    [N][H][dk][dv] fp32, read and overwritten in place with S_t.
+ * flags: GDN_QK_L2NORM as above.  Supported: dk in {64, 128}, dv a multiple of
+ * 64 up to 512.  o must not overlap S or the inputs.
+ */
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const float *a, const float *b, float *S, void *o,
+                           int N, int H, int dk, int dv, gdn_dtype io_dtype,
+                           float scale, unsigned flags, cudaStream_t stream);
+
+/*
+ * Loop residual h_out = h_tilde + rho (.) h_prev, computed in fp32 and rounded
+ * to nearest-even in io_dtype.
+ *   h_tilde, h_prev, h_out [rows][d] io_dtype; rho [d] fp32.
+ * h_out may alias h_tilde or h_prev exactly.  d must be a multiple of 8.
+ */
+gdn_status loop_residual(const void *h_tilde, const void *h_prev, const float *rho,
+                         void *h_out, int64_t rows, int d, gdn_dtype io_dtype,
+                         cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char *gdn_status_string(gdn_status s);
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device (GDN_OK if no kernel recorded an error since the last call). */
+gdn_status gdn_get_device_status(cudaStream_t stream);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOOPED_GDN_H */

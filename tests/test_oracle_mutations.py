@@ -1,0 +1,47 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case copies the oracle to a temporary directory, plants one mistake in its
+C source (CPU only), and runs the pin suite against the copy in a subprocess:
+the suite has to fail.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "decay_misplaced": ("row[j] = a * (row[j] - b * ki * y[j]) + b * ki * v[j];",
+                        "row[j] = a * row[j] - b * ki * y[j] + b * ki * v[j];"),
+    "write_strength_dropped": ("+ b * ki * v[j];", "+ ki * v[j];"),
+    "erase_sign_flipped": ("(row[j] - b * ki * y[j])", "(row[j] + b * ki * y[j])"),
+    "readout_before_update": ("    /* Sigma_t = a (Sigma - b k y) + b k v^T */",
+                              "    if (o) { for (int j = 0; j < dv; ++j) { o[j] = 0.0;"
+                              " for (int i = 0; i < dk; ++i) o[j] += q[i] * sig[(size_t)i * dv + j];"
+                              " o[j] *= scale; } o = 0; }\n"
+                              "    /* Sigma_t = a (Sigma - b k y) + b k v^T */"),
+    "key_transposed_with_query": ("const double ki = k[i];\n        double *row",
+                                  "const double ki = q[i];\n        double *row"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(tmp_path, name):
+    src, dst = MUTATIONS[name]
+    shutil.copytree(os.path.join(ROOT, "oracle"), tmp_path / "oracle",
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    shutil.copytree(os.path.join(ROOT, "tests"), tmp_path / "tests",
+                    ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutations.py"))
+    cfile = tmp_path / "oracle" / "gdn_oracle.c"
+    text = cfile.read_text()
+    assert text.count(src) == 1, f"mutation anchor not found once: {src!r}"
+    cfile.write_text(text.replace(src, dst))
+    env = dict(os.environ, PYTHONPATH=str(tmp_path))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        str(tmp_path / "tests" / "test_oracle_pins.py")],
+                       cwd=tmp_path, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout

@@ -1,0 +1,503 @@
+#!/usr/bin/env python
+"""Benchmark of the looped GDN mixer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the looped-prefill workload: T = 4 loops of (q/k/v projection ->
+GDN chunkwise prefill with in-kernel q/k L2 norm -> loop residual) over one
+sequence of 4096 tokens, d = 2048 (16 heads x 128).  Inputs are resident in
+HBM when the timed region starts; L2 is flushed between steps (256 MiB write).
+`value` is whole-job tokens/s (sequence tokens through all T loops).  The same
+JSON line carries the roofline of the prefill kernel, the CPU oracle baseline,
+the end-to-end figure through host buffers, and the other workloads (long
+prefill, variable-length prefill, decode state streaming) measured on their
+own.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
+the workload (weak scaling, no collective on the data path); the timed region
+is bracketed by a barrier + synchronize and the time is the max over ranks.
+
+--impl reference times the CPU oracle (rank 0 only) on a bounded sample of
+the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "looped GDN prefill tokens/s (T=4) and decode state-HBM GB/s vs B200 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    """Hash of the prefill kernel sources: ncu traffic figures are reported only
+    while they were taken on the kernel as it stands."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "looped_linear_attention_b200", "csrc")
+    for name in ("common.cuh", "gdn_prefill_tc.cu"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """Per-launch DRAM traffic of the prefill kernel from the committed ncu summary,
+    if it was captured on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "gdn_prefill_tc_looped_prefill.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("kernel_source_hash") == kernel_source_hash():
+            return d.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ byte / flop accounting
+def prefill_bytes_per_token_head(dk, dv, io_bytes=2):
+    """Algorithmic HBM bytes of one token of one head in one prefill launch:
+    q, k (dk each), v and o (dv each) in the io dtype, a and b in fp32."""
+    return io_bytes * (2 * dk + 2 * dv) + 8
+
+
+def prefill_state_bytes(n_seq, H, dk, dv, s0, st):
+    return n_seq * H * dk * dv * 4 * ((1 if s0 else 0) + (1 if st else 0))
+
+
+def decode_bytes_per_head_state(dk, dv, io_bytes=2):
+    """State read + write (fp32) plus q, k, v, o and a, b."""
+    return 2 * dk * dv * 4 + io_bytes * (2 * dk + 2 * dv) + 8
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local):
+    import numpy as np
+    import torch
+
+    import looped_linear_attention_b200 as lla
+    from looped_linear_attention_b200 import build as lib_build
+    from looped_linear_attention_b200 import workloads as W
+
+    if rank == 0 and not os.path.exists(lib_build.LIB_PATH):
+        lib_build.build()
+    barrier(world)
+    lla.library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    wl = W.WORKLOADS["looped_prefill"]
+    inp = W.looped_inputs(wl, dev)
+    L, d = inp["L"], inp["d"]
+    runner = lla.LoopedPrefill(L, wl.H, wl.dk, wl.dv, wl.loops, dev, time_mixer=True)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    out = torch.empty(L, d, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        runner.run(inp["h0"], inp["Wq"], inp["Wk"], inp["Wv"], inp["a"], inp["b"], inp["rho"],
+                   out=out)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    runner.mixer_events.clear()
+    step_events = []
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for _ in range(args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            step_events.append((e0, e1))
+        torch.cuda.synchronize()
+    barrier(world)
+    gdn_events = list(runner.mixer_events)
+    runner.time_mixer = False
+    step_ms = [a.elapsed_time(b) for a, b in step_events]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, world)
+    tokens_per_step = L
+    value = world * tokens_per_step * args.steps / total_s
+    gdn_ms = [a.elapsed_time(b) for a, b in gdn_events]
+    gdn_avg_s = statistics.mean(gdn_ms) / 1e3
+    gdn_bytes = prefill_bytes_per_token_head(wl.dk, wl.dv) * L * wl.H
+    achieved = gdn_bytes / gdn_avg_s / 1e9
+    hbm_peak = peaks["hbm_gbs"]
+    launches = args.steps * wl.loops * 2
+
+    # ---- end to end through host buffers (pinned), same step
+    e2e = run_e2e(args, runner, inp, wl, dev, stream, world)
+
+    # ---- other workloads, each on its own
+    extras = {}
+    if not args.no_extras:
+        del flush
+        torch.cuda.empty_cache()
+        extras["long_prefill"] = bench_prefill_workload(W.WORKLOADS["long_prefill"], dev, args,
+                                                        peaks, world)
+        torch.cuda.empty_cache()
+        extras["decode"] = bench_decode(W.WORKLOADS["decode"], dev, args, peaks, world)
+        torch.cuda.empty_cache()
+        extras["varlen"] = bench_prefill_workload(W.WORKLOADS["varlen"], dev, args, peaks, world)
+        torch.cuda.empty_cache()
+
+    st = lla.gdn_get_device_status()
+    if st != lla.GDN_OK:
+        raise RuntimeError(f"device status after the benchmark: {lla.status_string(st)}")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_seconds)
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_s * 1e3 / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; random-init projection weights)",
+        "config": {"workload": "looped_prefill", "batch": 1, "seq_len": L, "d_model": d,
+                   "heads": wl.H, "dk": wl.dk, "dv": wl.dv, "loops": wl.loops, "chunk": 64,
+                   "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)"},
+        "roofline": {"kernel": "gdn_prefill_tc", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "peak_source": peak_kind, "traffic": profiled_traffic(),
+                     "algorithmic_bytes_per_launch": gdn_bytes,
+                     "avg_launch_ms": gdn_avg_s * 1e3},
+        "gpu_launches": launches,
+        "e2e": e2e,
+        "clocks": clocks.summary(),
+        "workloads": extras,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, runner, inp, wl, dev, stream, world):
+    """Same step through the public API with the inputs in pinned host memory:
+    h0, a, b copied in, h^(T) copied out, inside the timed region."""
+    import torch
+    h_host = inp["h0"].cpu().pin_memory()
+    a_host = inp["a"].cpu().pin_memory()
+    b_host = inp["b"].cpu().pin_memory()
+    out_host = torch.empty(inp["L"], inp["d"], dtype=torch.bfloat16).pin_memory()
+    h_dev = torch.empty_like(inp["h0"])
+    a_dev = torch.empty_like(inp["a"])
+    b_dev = torch.empty_like(inp["b"])
+    out_dev = torch.empty_like(inp["h0"])
+
+    def step():
+        h_dev.copy_(h_host, non_blocking=True)
+        a_dev.copy_(a_host, non_blocking=True)
+        b_dev.copy_(b_host, non_blocking=True)
+        runner.run(h_dev, inp["Wq"], inp["Wk"], inp["Wv"], a_dev, b_dev, inp["rho"], out=out_dev)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    h2d = h_host.numel() * 2 + a_host.numel() * 4 + b_host.numel() * 4
+    d2h = out_host.numel() * 2
+    return {"value": world * inp["L"] * args.steps / t, "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def bench_prefill_workload(wl, dev, args, peaks, world):
+    """T = wl.loops prefill launches per step over the same inputs (each loop from
+    its S0); returns tokens/s, GB/s and fraction of the HBM roof."""
+    import torch
+    import looped_linear_attention_b200 as lla
+    from looped_linear_attention_b200 import workloads as W
+    inp = W.prefill_inputs(wl, dev)
+    cu = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).to(dev)
+    o = torch.empty(inp["total_tokens"], wl.H, wl.dv, dtype=wl.dtype, device=dev)
+    ST = torch.empty(inp["n_seq"], wl.H, wl.dk, wl.dv, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for _ in range(wl.loops):
+            lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S0"], cu,
+                              n_seq=inp["n_seq"], o=o, S_T=ST)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n = max(1, args.steps)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n
+    tokens = inp["total_tokens"]
+    bytes_launch = (prefill_bytes_per_token_head(wl.dk, wl.dv) * tokens * wl.H
+                    + prefill_state_bytes(inp["n_seq"], wl.H, wl.dk, wl.dv, inp["S0"] is not None, True))
+    launch_s = t / wl.loops
+    gbs = bytes_launch / launch_s / 1e9
+    res = {"tokens_per_s": world * tokens / t, "ms_per_step": t * 1e3, "loops": wl.loops,
+           "tokens": tokens, "heads": wl.H, "dk": wl.dk, "dv": wl.dv,
+           "achieved_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+           "algorithmic_bytes_per_launch": bytes_launch}
+    del inp, o, ST
+    return res
+
+
+def bench_decode(wl, dev, args, peaks, world):
+    """One decode launch over every (slot, head) state per step, in place."""
+    import torch
+    import looped_linear_attention_b200 as lla
+    from looped_linear_attention_b200 import workloads as W
+    inp = W.decode_inputs(wl, dev)
+    o = torch.empty(wl.n_seq, wl.H, wl.dv, dtype=wl.dtype, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lla.gdn_decode_step(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S"], o=o)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    n = max(1, args.steps)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n
+    nbytes = decode_bytes_per_head_state(wl.dk, wl.dv) * wl.n_seq * wl.H
+    gbs = nbytes / t / 1e9
+    res = {"state_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"], "ms_per_step": t * 1e3,
+           "seq_tokens_per_s": world * 256 / t * 1.0, "slots": wl.n_seq, "heads": wl.H,
+           "bytes_per_step": nbytes,
+           "note": "one step = one token for 256 sequences x 24 layers x 4 loops (all slots)"}
+    del inp, o
+    return res
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_baseline(seconds_target: float = 15.0, sample_tokens: int = 1024):
+    """The oracle as it stands, on the first `sample_tokens` tokens of the
+    looped-prefill workload (all 4 loops, full width), on this host's cores."""
+    import torch
+    import oracle
+    from looped_linear_attention_b200 import workloads as W
+    wl = W.WORKLOADS["looped_prefill"]
+    inp = W.looped_inputs(wl, "cpu")
+    Ls = sample_tokens
+    t0 = time.perf_counter()
+    runs = 0
+    while True:
+        oracle.looped_forward(inp["h0"][:Ls], inp["Wq"], inp["Wk"], inp["Wv"],
+                              inp["a"][:, :Ls], inp["b"][:, :Ls], inp["rho"], wl.H, wl.dk, wl.dv)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el > seconds_target or runs >= 3:
+            break
+    value = Ls * runs / el
+    try:
+        model = next(l.split(":", 1)[1].strip() for l in open("/proc/cpuinfo") if "model name" in l)
+    except Exception:
+        model = "unknown"
+    return {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {Ls} of {wl.seq_len} tokens, all {wl.loops} loops, d={wl.H * wl.dk}, "
+                      f"{runs} run(s), {el:.1f} s; fp64 C oracle (OpenMP) + numpy projections",
+            "cpu": model}
+
+
+def run_reference(args, rank, world):
+    """CPU oracle arm: rank 0 only, bounded samples of the looped-prefill workload."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    for _ in range(max(0, min(args.warmup, 1))):
+        cpu_baseline(0.0, sample_tokens=256)
+    times = []
+    Ls = 512
+    for _ in range(args.steps):
+        r = cpu_baseline(0.0, sample_tokens=Ls)
+        times.append(Ls / r["value"])
+    total = sum(times)
+    value = Ls * args.steps / total
+    from looped_linear_attention_b200 import workloads as W
+    wl = W.WORKLOADS["looped_prefill"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": "looped_prefill", "batch": 1, "seq_len": wl.seq_len,
+                   "d_model": wl.H * wl.dk, "heads": wl.H, "dk": wl.dk, "dv": wl.dv,
+                   "loops": wl.loops, "parallelism": "cpu oracle, rank 0"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: first {Ls} of {wl.seq_len} tokens, all {wl.loops} loops"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        # the CPU oracle arm: rank 0 alone, no process group
+        run_reference(args, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,25 @@
+"""Looped gated delta-rule (GDN) mixer for NVIDIA B200 (sm_100a).
+
+The library is the C-ABI shared object ``libgdn.so`` (declared in
+``include/gdn.h``), built from ``csrc/`` by ``looped_linear_attention_b200.build``.
+This package is its thin Python binding plus the seeded workload generators:
+
+    gdn_chunk_fwd    chunkwise prefill over packed / variable-length sequences
+    gdn_decode_step  one token per state slot, in-place state update
+    loop_residual    h = h_tilde + rho (.) h_prev
+    LoopedPrefill    T loops of projection -> GDN -> loop residual
+
+No compute runs in Python: if the library is missing, every entry point raises.
+"""
+from ._binding import (GDN_BF16, GDN_ERR_CUDA, GDN_ERR_INVALID, GDN_ERR_TIMEOUT,
+                       GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_F32, GDN_OK, GDN_PRECISE,
+                       GDN_QK_L2NORM, GdnError, gdn_chunk_fwd, gdn_decode_step,
+                       gdn_get_device_status, library, loop_residual, status_string, version)
+from .looped import LoopedPrefill
+
+__all__ = [
+    "gdn_chunk_fwd", "gdn_decode_step", "loop_residual", "gdn_get_device_status",
+    "LoopedPrefill", "GdnError", "library", "status_string", "version",
+    "GDN_OK", "GDN_ERR_INVALID", "GDN_ERR_UNSUPPORTED", "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT",
+    "GDN_ERR_WORKSPACE", "GDN_F32", "GDN_BF16", "GDN_QK_L2NORM", "GDN_PRECISE",
+]

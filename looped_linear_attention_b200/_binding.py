@@ -1,0 +1,218 @@
+"""ctypes binding of libgdn.so: argument marshalling only.
+
+Every compute step runs in the library's CUDA kernels; this module checks
+tensor dtypes/shapes/devices, allocates outputs with torch when the caller does
+not pass them, and forwards raw device pointers and the current CUDA stream.
+If the library is missing the import of any entry point raises -- there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_OK = 0
+GDN_ERR_INVALID = 1
+GDN_ERR_UNSUPPORTED = 2
+GDN_ERR_CUDA = 3
+GDN_ERR_TIMEOUT = 4
+GDN_ERR_WORKSPACE = 5
+
+GDN_F32 = 0
+GDN_BF16 = 1
+
+GDN_QK_L2NORM = 0x1
+GDN_PRECISE = 0x2
+
+_DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class gdn_fwd_params(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("a", ctypes.c_void_p), ("b", ctypes.c_void_p), ("S0", ctypes.c_void_p),
+        ("o", ctypes.c_void_p), ("S_T", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p),
+        ("n_seq", ctypes.c_int), ("seq_len", ctypes.c_int), ("total_tokens", ctypes.c_int),
+        ("H", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
+        ("io_dtype", ctypes.c_int), ("scale", ctypes.c_float), ("flags", ctypes.c_uint),
+    ]
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libgdn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library {LIB_PATH} is missing; build it with "
+                "`python -m looped_linear_attention_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i32, u32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_float
+        lib.gdn_chunk_fwd_workspace.argtypes = [ctypes.POINTER(gdn_fwd_params)]
+        lib.gdn_chunk_fwd_workspace.restype = ctypes.c_size_t
+        lib.gdn_chunk_fwd.argtypes = [ctypes.POINTER(gdn_fwd_params), vp, ctypes.c_size_t, vp]
+        lib.gdn_chunk_fwd.restype = i32
+        lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                        f32, u32, vp]
+        lib.gdn_decode_step.restype = i32
+        lib.loop_residual.argtypes = [vp, vp, vp, vp, ctypes.c_int64, i32, i32, vp]
+        lib.loop_residual.restype = i32
+        lib.gdn_status_string.argtypes = [i32]
+        lib.gdn_status_string.restype = ctypes.c_char_p
+        lib.gdn_get_device_status.argtypes = [vp]
+        lib.gdn_get_device_status.restype = i32
+        lib.gdn_version.argtypes = []
+        lib.gdn_version.restype = i32
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return library().gdn_status_string(int(status)).decode()
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,
+                  b: torch.Tensor, S0: Optional[torch.Tensor] = None,
+                  cu_seqlens: Optional[torch.Tensor] = None, *, n_seq: Optional[int] = None,
+                  scale: float = 1.0, flags: int = 0, o: Optional[torch.Tensor] = None,
+                  S_T: Optional[torch.Tensor] = None, return_state: bool = True,
+                  stream: Optional[torch.cuda.Stream] = None):
+    """Chunkwise prefill (see gdn_chunk_fwd in include/gdn.h).
+
+    q, k: [T, H, dk]; v: [T, H, dv] (fp32 or bf16); a, b: [T, H] fp32;
+    S0: [n_seq, H, dk, dv] fp32 or None; cu_seqlens: int32 [n_seq+1] on the device,
+    or None with n_seq sequences of T // n_seq tokens (n_seq defaults to 1).
+    Returns (o, S_T) (S_T is None when return_state is False)."""
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    _check(q, "q", q.dtype)
+    _check(k, "k", q.dtype, (T, H, dk))
+    _check(v, "v", q.dtype, (T, H, dv))
+    _check(a, "a", torch.float32, (T, H))
+    _check(b, "b", torch.float32, (T, H))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        ns = cu_seqlens.numel() - 1
+        seq_len = 0
+    else:
+        ns = 1 if n_seq is None else int(n_seq)
+        if ns <= 0 or T % ns != 0:
+            raise ValueError("without cu_seqlens, the token count must be n_seq * seq_len")
+        seq_len = T // ns
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (ns, H, dk, dv))
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=q.dtype, device=q.device)
+    else:
+        _check(o, "o", q.dtype, (T, H, dv))
+    if S_T is None and return_state:
+        S_T = torch.empty(ns, H, dk, dv, dtype=torch.float32, device=q.device)
+    elif S_T is not None:
+        _check(S_T, "S_T", torch.float32, (ns, H, dk, dv))
+    p = gdn_fwd_params(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0), _ptr(o),
+                       _ptr(S_T), _ptr(cu_seqlens), ns, seq_len, T, H, dk, dv,
+                       _DTYPES[q.dtype], float(scale), int(flags))
+    lib = library()
+    ws = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
+    if ws == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_INVALID, "gdn_chunk_fwd")
+    work = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
+    st = lib.gdn_chunk_fwd(ctypes.byref(p), _ptr(work), ctypes.c_size_t(ws), _stream_ptr(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd")
+    return o, S_T
+
+
+def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,
+                    b: torch.Tensor, S: torch.Tensor, *, scale: float = 1.0, flags: int = 0,
+                    o: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One token per slot; S [N, H, dk, dv] fp32 is updated in place. Returns o [N, H, dv]."""
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    _check(q, "q", q.dtype)
+    _check(k, "k", q.dtype, (N, H, dk))
+    _check(v, "v", q.dtype, (N, H, dv))
+    _check(a, "a", torch.float32, (N, H))
+    _check(b, "b", torch.float32, (N, H))
+    _check(S, "S", torch.float32, (N, H, dk, dv))
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
+    else:
+        _check(o, "o", q.dtype, (N, H, dv))
+    st = library().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S), _ptr(o),
+                                   N, H, dk, dv, _DTYPES[q.dtype], float(scale), int(flags),
+                                   _stream_ptr(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode_step")
+    return o
+
+
+def loop_residual(h_tilde: torch.Tensor, h_prev: torch.Tensor, rho: torch.Tensor,
+                  out: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """h = h_tilde + rho (.) h_prev over the last dimension; out may alias an input."""
+    if h_tilde.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {h_tilde.dtype}")
+    d = h_tilde.shape[-1]
+    rows = h_tilde.numel() // d if d else 0
+    _check(h_tilde, "h_tilde", h_tilde.dtype)
+    _check(h_prev, "h_prev", h_tilde.dtype, h_tilde.shape)
+    _check(rho, "rho", torch.float32, (d,))
+    if out is None:
+        out = torch.empty_like(h_tilde)
+    else:
+        _check(out, "out", h_tilde.dtype, h_tilde.shape)
+    st = library().loop_residual(_ptr(h_tilde), _ptr(h_prev), _ptr(rho), _ptr(out), rows, d,
+                                 _DTYPES[h_tilde.dtype], _stream_ptr(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "loop_residual")
+    return out
+
+
+def gdn_get_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronises the stream and returns/clears the device status word."""
+    return int(library().gdn_get_device_status(_stream_ptr(stream)))
+
+
+def version() -> int:
+    return int(library().gdn_version())

@@ -1,0 +1,203 @@
+// C ABI of the looped GDN mixer library: argument validation, dispatch to the
+// kernels, the device status word.  See include/gdn.h for the contract of each
+// entry point.
+#include <string.h>
+
+#include "common.cuh"
+
+namespace gdn {
+bool prefill_tc_supported(const gdn_fwd_params* p);
+gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
+gdn_status launch_prefill_simt(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
+                          const float* b, float* S, void* o, int N, int H, int dk, int dv,
+                          gdn_dtype dt, float scale, unsigned flags, cudaStream_t stream);
+cudaError_t launch_loop_residual(const void* h_tilde, const void* h_prev, const float* rho,
+                                 void* h_out, int64_t rows, int d, gdn_dtype dt, int num_sms,
+                                 cudaStream_t stream);
+}  // namespace gdn
+
+// Device status word: kernels record the first error they hit (atomicCAS from 0).
+__device__ unsigned g_gdn_device_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+// Address of the status word on the current device (looked up once per device).
+unsigned* status_ptr() {
+  static void* cache[kMaxDevices] = {nullptr};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_gdn_device_status) != cudaSuccess) return nullptr;
+    cache[dev] = ptr;
+  }
+  return static_cast<unsigned*>(cache[dev]);
+}
+
+int sm_count() {
+  static int cache[kMaxDevices] = {0};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+bool dtype_ok(gdn_dtype t) { return t == GDN_F32 || t == GDN_BF16; }
+
+size_t elem_bytes(gdn_dtype t) { return t == GDN_BF16 ? 2 : 4; }
+
+// Shape/pointer checks shared by the workspace query and the launch.
+gdn_status validate_fwd(const gdn_fwd_params* p) {
+  if (!p) return GDN_ERR_INVALID;
+  if (!dtype_ok(p->io_dtype)) return GDN_ERR_INVALID;
+  if (p->n_seq < 0 || p->H <= 0 || p->dk <= 0 || p->dv <= 0 || p->total_tokens < 0)
+    return GDN_ERR_INVALID;
+  if (p->flags & ~(GDN_QK_L2NORM | GDN_PRECISE)) return GDN_ERR_INVALID;
+  if (!p->cu_seqlens) {
+    if (p->seq_len < 0) return GDN_ERR_INVALID;
+    if ((long long)p->n_seq * p->seq_len != (long long)p->total_tokens) return GDN_ERR_INVALID;
+  }
+  if (p->dk != 64 && p->dk != 128) return GDN_ERR_UNSUPPORTED;
+  if (p->dv % 64 != 0 || p->dv > 512) return GDN_ERR_UNSUPPORTED;
+  const bool any_tokens = p->total_tokens > 0;
+  if (any_tokens && (!p->q || !p->k || !p->v || !p->a || !p->b || !p->o)) return GDN_ERR_INVALID;
+  const void* ptrs[] = {p->q, p->k, p->v, p->a, p->b, p->S0, p->o, p->S_T, p->cu_seqlens};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return GDN_ERR_INVALID;
+  if (p->S_T && p->S0 && p->S_T != p->S0) {
+    // partial overlap of S0 and S_T is not allowed (exact aliasing is)
+    const size_t bytes = (size_t)p->n_seq * p->H * p->dk * p->dv * sizeof(float);
+    const char* a0 = reinterpret_cast<const char*>(p->S0);
+    const char* b0 = reinterpret_cast<const char*>(p->S_T);
+    if (a0 < b0 + bytes && b0 < a0 + bytes) return GDN_ERR_INVALID;
+  }
+  if (any_tokens && p->o) {
+    // the output may not overlap any input
+    const size_t ob = (size_t)p->total_tokens * p->H * p->dv * elem_bytes(p->io_dtype);
+    const char* o0 = reinterpret_cast<const char*>(p->o);
+    struct R { const void* ptr; size_t bytes; } ins[] = {
+        {p->q, (size_t)p->total_tokens * p->H * p->dk * elem_bytes(p->io_dtype)},
+        {p->k, (size_t)p->total_tokens * p->H * p->dk * elem_bytes(p->io_dtype)},
+        {p->v, (size_t)p->total_tokens * p->H * p->dv * elem_bytes(p->io_dtype)},
+        {p->a, (size_t)p->total_tokens * p->H * sizeof(float)},
+        {p->b, (size_t)p->total_tokens * p->H * sizeof(float)},
+    };
+    for (const R& r : ins) {
+      const char* s = reinterpret_cast<const char*>(r.ptr);
+      if (s && s < o0 + ob && o0 < s + r.bytes) return GDN_ERR_INVALID;
+    }
+  }
+  return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_version(void) { return 100; }
+
+const char* gdn_status_string(gdn_status s) {
+  switch (s) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_INVALID: return "invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case GDN_ERR_CUDA: return "CUDA error";
+    case GDN_ERR_TIMEOUT: return "device-side wait timed out";
+    case GDN_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+size_t gdn_chunk_fwd_workspace(const gdn_fwd_params* p) {
+  if (validate_fwd(p) != GDN_OK) return (size_t)-1;
+  return 0;
+}
+
+gdn_status gdn_chunk_fwd(const gdn_fwd_params* p, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  const gdn_status v = validate_fwd(p);
+  if (v != GDN_OK) return v;
+  (void)ws;
+  (void)ws_bytes;
+  if (p->n_seq == 0) return GDN_OK;
+  if (p->total_tokens == 0) {
+    // every sequence is empty: S_T = S0 (or zero)
+    if (!p->S_T) return GDN_OK;
+    const size_t bytes = (size_t)p->n_seq * p->H * p->dk * p->dv * sizeof(float);
+    cudaError_t e = p->S0 ? (p->S0 == p->S_T ? cudaSuccess
+                                             : cudaMemcpyAsync(p->S_T, p->S0, bytes,
+                                                               cudaMemcpyDeviceToDevice, stream))
+                          : cudaMemsetAsync(p->S_T, 0, bytes, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  }
+  unsigned* st = status_ptr();
+  if (!st) return GDN_ERR_CUDA;
+  if (gdn::prefill_tc_supported(p)) return gdn::launch_prefill_tc(p, st, stream);
+  return gdn::launch_prefill_simt(p, st, stream);
+}
+
+gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* a,
+                           const float* b, float* S, void* o, int N, int H, int dk, int dv,
+                           gdn_dtype io_dtype, float scale, unsigned flags,
+                           cudaStream_t stream) {
+  if (!dtype_ok(io_dtype) || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return GDN_ERR_INVALID;
+  if (flags & ~GDN_QK_L2NORM) return GDN_ERR_INVALID;
+  if (dk != 64 && dk != 128) return GDN_ERR_UNSUPPORTED;
+  if (dv % 64 != 0 || dv > 512) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  if (!q || !k || !v || !a || !b || !S || !o) return GDN_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, a, b, S, o};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return GDN_ERR_INVALID;
+  {
+    const size_t ob = (size_t)N * H * dv * elem_bytes(io_dtype);
+    const size_t sb = (size_t)N * H * dk * dv * sizeof(float);
+    const char* o0 = reinterpret_cast<const char*>(o);
+    const char* s0 = reinterpret_cast<const char*>(S);
+    if (o0 < s0 + sb && s0 < o0 + ob) return GDN_ERR_INVALID;
+  }
+  const cudaError_t e =
+      gdn::launch_decode(q, k, v, a, b, S, o, N, H, dk, dv, io_dtype, scale, flags, stream);
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status loop_residual(const void* h_tilde, const void* h_prev, const float* rho, void* h_out,
+                         int64_t rows, int d, gdn_dtype io_dtype, cudaStream_t stream) {
+  if (!dtype_ok(io_dtype) || rows < 0 || d <= 0 || d % 8 != 0) return GDN_ERR_INVALID;
+  if (rows == 0) return GDN_OK;
+  if (!h_tilde || !h_prev || !rho || !h_out) return GDN_ERR_INVALID;
+  if (!aligned16(h_tilde) || !aligned16(h_prev) || !aligned16(rho) || !aligned16(h_out))
+    return GDN_ERR_INVALID;
+  const cudaError_t e = gdn::launch_loop_residual(h_tilde, h_prev, rho, h_out, rows, d, io_dtype,
+                                                  sm_count(), stream);
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_get_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
+  unsigned host = 0;
+  if (cudaMemcpyFromSymbol(&host, g_gdn_device_status, sizeof(host)) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  const unsigned zero = 0;
+  if (host != 0 && cudaMemcpyToSymbol(g_gdn_device_status, &zero, sizeof(zero)) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  return static_cast<gdn_status>(host);
+}
+
+}  // extern "C"

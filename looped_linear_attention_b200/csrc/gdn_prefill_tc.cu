@@ -1,0 +1,612 @@
+// Chunkwise prefill of the gated delta rule on the 5th-generation tensor cores
+// (tcgen05 MMA with tensor-memory accumulators, TMA-fed shared memory), sm_100a.
+//
+// The recurrence ("LT2: Linear-Time Looped Transformers", §2, "LT2." paragraph;
+// Gated DeltaNet mixer, Appendix C), with the state Sigma in R^{dk x dv}:
+//     Sigma_t = a_t (I - b_t k_t k_t^T) Sigma_{t-1} + b_t k_t v_t^T,  o_t = scale Sigma_t^T q_t.
+// The page reports that LT2's GDN layers run as a fused chunkwise kernel
+// (§3.2).  This file is this library's own chunked form: for a chunk of C = 64
+// tokens with start state Sigma_0, g_i = sum_{j<=i} log a_j, gamma_i = exp(g_i),
+// D_ij = exp(g_i - g_j) (j <= i, all <= 1):
+//     A   = strict_lower(diag(b) (D o K K^T)),     T = (I + A)^{-1}
+//     W   = T diag(b gamma) K,   U~ = T diag(b) V,   U = U~ - W Sigma_0
+//     O   = scale (diag(gamma) Q Sigma_0 + tril(D o Q K^T) U)
+//     Sigma_C = gamma_C Sigma_0 + K^T diag(gamma_C / gamma) U
+// U holds the per-token corrections u_t = b_t (v_t - a_t Sigma_{t-1}^T k_t), so
+// Sigma_t = a_t Sigma_{t-1} + k_t u_t^T, and the three lines above follow by
+// unrolling that inside the chunk.
+//
+// Data path (one CTA per (sequence, head, 128-wide slice of dv)):
+//   * every product is issued TRANSPOSED so its M dimension is 128 (dv rows of
+//     Sigma^T, dk rows of W^T, or the stacked [K; Q] rows) and lands in tensor
+//     memory with lane = row: G = [K;Q] K^T, U^T = V^T T2^T - Sigma^T W^T,
+//     W^T = K^T T1^T, O_A^T = Sigma^T Q^T, O_B^T = U^T P^T,
+//     Sigma^T += (U^T diag(gamma_C/gamma)) K.
+//   * q, k, v tiles arrive by TMA (128-byte swizzle) into a 2-stage ring filled
+//     by a producer warp; operands computed in the CTA (T1, T2, P, W, U^T,
+//     Sigma^T) are rounded to bf16 and written in the same swizzled layout.
+//   * the fp32 master state stays in tensor memory for the whole sequence; its
+//     bf16 copy in shared memory feeds the next chunk's MMAs.
+//   * every wait is bounded (GDN_ERR_TIMEOUT) so a fault in the schedule cannot
+//     hang the GPU.
+#include "common.cuh"
+
+namespace gdn {
+namespace tc {
+
+constexpr int C = 64;            // chunk length
+constexpr int DK = 128;          // key/query width (this kernel)
+constexpr int DVS = 128;         // dv slice per CTA
+constexpr int STAGES = 2;
+constexpr int CW = 128;          // compute warpgroup: warps 0-3 (tensor-memory lanes 0-127)
+constexpr int THREADS = CW + 32; // + producer warp 4
+
+// tensor-memory columns (fp32 accumulators, lane = row)
+constexpr uint32_t COL_G = 0;     // [K;Q] K^T      128 x 64
+constexpr uint32_t COL_W = 64;    // W^T            128 x 64
+constexpr uint32_t COL_U = 128;   // U^T            128 x 64
+constexpr uint32_t COL_OA = 192;  // Sigma^T Q^T    128 x 64
+constexpr uint32_t COL_OB = 256;  // U^T P^T        128 x 64
+constexpr uint32_t COL_S = 384;   // Sigma^T fp32   128 x 128
+constexpr uint32_t TMEM_COLS = 512;
+
+// Shared-memory plan (offsets from a 1024-byte aligned base).
+constexpr uint32_t OFF_KQ = 0;                          // STAGES x 32 KB: [K0|Q0|K1|Q1] 8 KB slabs
+constexpr uint32_t KQ_BYTES = 32768;
+constexpr uint32_t OFF_V = OFF_KQ + STAGES * KQ_BYTES;  // STAGES x 16 KB: [V0|V1]
+constexpr uint32_t V_BYTES = 16384;
+constexpr uint32_t OFF_SIG = OFF_V + STAGES * V_BYTES;  // Sigma^T bf16 [128 dv][128 dk], 2 x 16 KB slabs
+constexpr uint32_t OFF_W = OFF_SIG + 32768;             // W bf16 [64 tok][128 dk], 2 x 8 KB slabs
+constexpr uint32_t OFF_UT = OFF_W + 16384;              // U^T bf16 [128 dv][64 tok]
+constexpr uint32_t OFF_UTP = OFF_UT + 16384;            // U^T diag(gamma_C/gamma) bf16
+constexpr uint32_t OFF_P = OFF_UTP + 16384;             // P bf16 [64][64]
+constexpr uint32_t OFF_T1 = OFF_P + 8192;               // T diag(b gamma) bf16 [64][64]
+constexpr uint32_t OFF_T2 = OFF_T1 + 8192;              // T diag(b) bf16 [64][64]
+constexpr uint32_t OFF_A = OFF_T2 + 8192;               // A fp32 [64][65] (padded rows)
+constexpr int A_LD = 65;
+constexpr uint32_t OFF_GATE = OFF_A + 64 * A_LD * 4;    // g, gamma, b: 3 x 64 fp32
+constexpr uint32_t OFF_BAR = OFF_GATE + 3 * 256;        // mbarriers
+constexpr uint32_t OFF_MISC = OFF_BAR + 64;             // tmem base, abort, scan carry
+constexpr uint32_t SMEM_USED = OFF_MISC + 64;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;       // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
+
+struct Params {
+  const float* a;
+  const float* b;
+  const float* S0;
+  float* S_T;
+  __nv_bfloat16* o;
+  const int32_t* cu_seqlens;
+  unsigned* status;
+  int n_seq, seq_len, total_tokens, H, dv, n_slices;
+  float scale;
+  unsigned flags;
+};
+
+// Named barrier of the four compute warps (the warp is reconverged first: the
+// barrier is warp-aligned and the bounded waits exit lane by lane).
+__device__ __forceinline__ void cw_sync() {
+  __syncwarp();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// K-major, 128-byte swizzled operand: rows of 128 bytes, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return smem_desc(saddr, 16, 1024); }
+// MN-major, 128-byte swizzled operand: 64 contiguous MN elements per 128-byte row,
+// rows along K 128 B apart (8-row atoms 1024 B apart), next 64 MN elements `lbo` bytes on.
+__device__ __forceinline__ uint64_t mndesc(uint32_t saddr, uint32_t lbo) {
+  return smem_desc(saddr, lbo, 1024);
+}
+
+// All compute-warpgroup threads wait on `bar`; the outcome is made uniform
+// through the abort flag so that no thread leaves the schedule alone.
+__device__ __forceinline__ bool cw_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                        unsigned* status) {
+  mbar_wait_bounded(bar, parity, abort, status);
+  cw_sync();
+  return *abort == 0;
+}
+
+// Normalise one 128-element bf16 row of a [K0|Q0|K1|Q1] stage tile in place:
+// x / sqrt(sum x^2 + eps) in fp32, rounded to bf16.
+__device__ __forceinline__ void l2norm_row(uint8_t* kq, int row_in_tile, uint32_t tile_off) {
+  float ss = 0.f;
+  uint4 v[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t off = tile_off + (c >> 3) * 16384 + sw128_offset(row_in_tile, (c & 7) * 8);
+    v[c] = *reinterpret_cast<const uint4*>(kq + off);
+    const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = bf16_lo(w[e]), hi = bf16_hi(w[e]);
+      ss = fmaf(lo, lo, ss);
+      ss = fmaf(hi, hi, ss);
+    }
+  }
+  const float inv = 1.0f / sqrtf(ss + kQkNormEps);
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t off = tile_off + (c >> 3) * 16384 + sw128_offset(row_in_tile, (c & 7) * 8);
+    uint4 o;
+    o.x = pack_bf16x2(bf16_lo(v[c].x) * inv, bf16_hi(v[c].x) * inv);
+    o.y = pack_bf16x2(bf16_lo(v[c].y) * inv, bf16_hi(v[c].y) * inv);
+    o.z = pack_bf16x2(bf16_lo(v[c].z) * inv, bf16_hi(v[c].z) * inv);
+    o.w = pack_bf16x2(bf16_lo(v[c].w) * inv, bf16_hi(v[c].w) * inv);
+    *reinterpret_cast<uint4*>(kq + off) = o;
+  }
+}
+
+// Writes 64 fp32 values (one tensor-memory row over 64 columns) as a bf16 row of
+// a 128-byte-swizzled K-major tile.
+__device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int row, const float (&x)[64]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 o;
+    o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
+    o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
+    o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
+    o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
+    *reinterpret_cast<uint4*>(tile + sw128_offset(row, c * 8)) = o;
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  float* s_g = reinterpret_cast<float*>(sm + OFF_GATE);
+  float* s_gamma = s_g + 64;
+  float* s_b = s_g + 128;
+  uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* bar_empty = bar_full + STAGES;
+  uint64_t* bar_mma = bar_empty + STAGES;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+  float* s_carry = reinterpret_cast<float*>(sm + OFF_MISC + 8);
+  float* s_A = reinterpret_cast<float*>(sm + OFF_A);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // work unit
+  const int slice = blockIdx.x % p.n_slices;
+  const int chain = blockIdx.x / p.n_slices;
+  const int h = chain % p.H;
+  const int seq = chain / p.H;
+  int seq_start, seq_end;
+  if (p.cu_seqlens) {
+    seq_start = p.cu_seqlens[seq];
+    seq_end = p.cu_seqlens[seq + 1];
+  } else {
+    seq_start = seq * p.seq_len;
+    seq_end = seq_start + p.seq_len;
+  }
+  {
+    // offsets outside [0, total_tokens] or decreasing: clamp, and report
+    const int s0 = min(max(seq_start, 0), p.total_tokens);
+    const int s1 = min(max(seq_end, s0), p.total_tokens);
+    if ((s0 != seq_start || s1 != seq_end) && threadIdx.x == 0) record_status(p.status, GDN_ERR_INVALID);
+    seq_start = s0;
+    seq_end = s1;
+  }
+  const int len = seq_end - seq_start;
+  const int n_chunks = (len + C - 1) / C;
+  const int H = p.H, dv = p.dv;
+  const int col0 = slice * DVS;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bar_full[s], 1);
+      mbar_init(&bar_empty[s], 1);
+    }
+    mbar_init(bar_mma, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued[STAGES] = {0, 0};
+      for (int c = 0; c < n_chunks; ++c) {
+        const int s = c % STAGES;
+        const int use = c / STAGES;
+        if (use > 0 && !mbar_wait_bounded(&bar_empty[s], (use - 1) & 1, s_abort, p.status)) break;
+        uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
+        uint8_t* vv = sm + OFF_V + s * V_BYTES;
+        const int tok0 = seq_start + c * C;
+        mbar_arrive_expect_tx(&bar_full[s], KQ_BYTES + V_BYTES);
+        tma_load_3d(kq + 0, &tm_k, &bar_full[s], 0, h, tok0);
+        tma_load_3d(kq + 16384, &tm_k, &bar_full[s], 64, h, tok0);
+        tma_load_3d(kq + 8192, &tm_q, &bar_full[s], 0, h, tok0);
+        tma_load_3d(kq + 24576, &tm_q, &bar_full[s], 64, h, tok0);
+        tma_load_3d(vv + 0, &tm_v, &bar_full[s], col0, h, tok0);
+        tma_load_3d(vv + 8192, &tm_v, &bar_full[s], col0 + 64, h, tok0);
+        issued[s] = use + 1;
+      }
+      // never leave the block with bulk copies still landing in its shared memory
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s] > 0) mbar_wait_bounded(&bar_full[s], (issued[s] - 1) & 1, nullptr, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------ compute warpgroup
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;   // this warp's tensor-memory lanes
+    const int j = tid;                                        // dv row (or dk row) owned
+    const size_t state_base = ((size_t)seq * H + h) * DK * (size_t)dv + col0 + j;
+    uint32_t mma_phase = 0;
+
+    // initial state: Sigma^T row j = column (col0 + j) of S0, fp32 into tensor memory,
+    // bf16 into the Sigma^T operand tile.
+#pragma unroll 1
+    for (int piece = 0; piece < 4; ++piece) {
+      float x[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        x[e] = p.S0 ? __ldg(p.S0 + state_base + (size_t)(piece * 32 + e) * dv) : 0.f;
+      tmem_st32(tmem + lane_off + COL_S + piece * 32, x);
+      uint8_t* slab = sm + OFF_SIG + (piece >> 1) * 16384;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint4 o;
+        o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
+        o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
+        o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
+        o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
+        *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + c * 8)) = o;
+      }
+    }
+    tmem_wait_st();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    cw_sync();
+
+    const uint32_t sbase = smem_u32(sm);
+    bool ok = true;
+#pragma unroll 1
+    for (int c = 0; c < n_chunks && ok; ++c) {
+      const int s = c % STAGES;
+      const int use = c / STAGES;
+      const int tok0 = seq_start + c * C;
+      const int valid = min(C, seq_end - tok0);
+      uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
+      const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
+      const uint32_t v_a = sbase + OFF_V + s * V_BYTES;
+
+      // ---- gates: g = inclusive prefix sum of log a over the chunk (rows past the
+      // sequence end get log a = 0, b = 0, which removes them from every product)
+      if (tid < C) {
+        float la = 0.f, bb = 0.f;
+        if (tid < valid) {
+          const size_t ti = (size_t)(tok0 + tid) * H + h;
+          la = logf(__ldg(p.a + ti));
+          bb = __ldg(p.b + ti);
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, la, off);
+          if (lane >= off) la += y;
+        }
+        if (tid == 31) *s_carry = la;
+        s_b[tid] = bb;
+        s_g[tid] = la;   // partial (warp 1 adds the carry below)
+      }
+      cw_sync();
+      if (tid >= 32 && tid < C) s_g[tid] += *s_carry;
+      cw_sync();
+      if (tid < C) s_gamma[tid] = expf(s_g[tid]);
+
+      if (!cw_wait(&bar_full[s], use & 1, s_abort, p.status)) { ok = false; break; }
+      if (p.flags & GDN_QK_L2NORM) {
+        // rows 0-63: K (tile offset 0), rows 64-127: Q (tile offset 8192)
+        l2norm_row(kq, tid & 63, tid < 64 ? 0u : 8192u);
+        fence_proxy_async_smem();
+      }
+      cw_sync();
+
+      // ---- G = [K; Q] K^T   (M = 128, N = 64, K = dk)
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16(tmem + COL_G, kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
+                   kk > 0);
+        }
+        mma_commit(bar_mma);
+      }
+      if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
+      mma_phase ^= 1;
+      tc_fence_after();
+      {
+        float gr[64];
+        tmem_ld32(tmem + lane_off + COL_G, *reinterpret_cast<float(*)[32]>(&gr[0]));
+        tmem_ld32(tmem + lane_off + COL_G + 32, *reinterpret_cast<float(*)[32]>(&gr[32]));
+        tmem_wait_ld();
+        if (tid < C) {
+          const int i = tid;
+          const float gi = s_g[i], bi = s_b[i];
+#pragma unroll
+          for (int jj = 0; jj < C; ++jj)
+            s_A[i * A_LD + jj] = (jj < i) ? bi * expf(gi - s_g[jj]) * gr[jj] : 0.f;
+        } else {
+          const int i = tid - C;
+          const float gi = s_g[i];
+#pragma unroll
+          for (int jj = 0; jj < C; ++jj) gr[jj] = (jj <= i) ? expf(gi - s_g[jj]) * gr[jj] : 0.f;
+          store_row64_bf16(sm + OFF_P, i, gr);
+        }
+      }
+      cw_sync();
+
+      // ---- T = (I + A)^{-1} by forward substitution, one column per thread
+      if (tid < C) {
+        const int col = tid;
+        float x[C];
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+          float acc = (i == col) ? 1.f : 0.f;
+#pragma unroll
+          for (int m = 0; m < i; ++m) acc = fmaf(-s_A[i * A_LD + m], x[m], acc);
+          x[i] = acc;
+        }
+        const float bj = s_b[col], bgj = s_b[col] * s_gamma[col];
+        uint8_t* t1 = sm + OFF_T1;
+        uint8_t* t2 = sm + OFF_T2;
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+          *reinterpret_cast<__nv_bfloat16*>(t1 + sw128_offset(i, col)) = __float2bfloat16_rn(x[i] * bgj);
+          *reinterpret_cast<__nv_bfloat16*>(t2 + sw128_offset(i, col)) = __float2bfloat16_rn(x[i] * bj);
+        }
+      }
+      fence_proxy_async_smem();
+      cw_sync();
+
+      // ---- U~^T = V^T T2^T  and  W^T = K^T T1^T   (M = 128, N = 64, K = 64 tokens)
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          mma_bf16(tmem + COL_U, mndesc(v_a + kk * 2048, 8192), kdesc(sbase + OFF_T2 + kk * 32),
+                   idesc_bf16(128, 64, 1, 0), kk > 0);
+          mma_bf16(tmem + COL_W, mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
+                   idesc_bf16(128, 64, 1, 0), kk > 0);
+        }
+        mma_commit(bar_mma);
+      }
+      if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
+      mma_phase ^= 1;
+      tc_fence_after();
+      {
+        // W^T row d = tid -> column d of W ([64 tok][128 dk] tile, 2 slabs)
+        float wr[64];
+        tmem_ld32(tmem + lane_off + COL_W, *reinterpret_cast<float(*)[32]>(&wr[0]));
+        tmem_ld32(tmem + lane_off + COL_W + 32, *reinterpret_cast<float(*)[32]>(&wr[32]));
+        tmem_wait_ld();
+        uint8_t* slab = sm + OFF_W + (tid >> 6) * 8192;
+        const int dcol = tid & 63;
+#pragma unroll
+        for (int i = 0; i < C; ++i)
+          *reinterpret_cast<__nv_bfloat16*>(slab + sw128_offset(i, dcol)) = __float2bfloat16_rn(wr[i]);
+      }
+      fence_proxy_async_smem();
+      cw_sync();
+
+      // ---- U^T -= Sigma^T W^T  and  O_A^T = Sigma^T Q^T   (M = 128, N = 64, K = dk)
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint64_t a_sig = kdesc(sbase + OFF_SIG + (kk >> 2) * 16384 + (kk & 3) * 32);
+          mma_bf16(tmem + COL_U, a_sig, kdesc(sbase + OFF_W + (kk >> 2) * 8192 + (kk & 3) * 32),
+                   idesc_bf16(128, 64, 0, 0, /*neg_b=*/1), 1);
+          mma_bf16(tmem + COL_OA, a_sig,
+                   kdesc(kq_a + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32),
+                   idesc_bf16(128, 64, 0, 0), kk > 0);
+        }
+        mma_commit(bar_mma);
+      }
+      if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
+      mma_phase ^= 1;
+      tc_fence_after();
+      const float gC = s_gamma[C - 1];
+      {
+        // U^T row j (dv) over 64 tokens -> operand tiles U^T and U^T diag(gamma_C / gamma)
+        float ur[64];
+        tmem_ld32(tmem + lane_off + COL_U, *reinterpret_cast<float(*)[32]>(&ur[0]));
+        tmem_ld32(tmem + lane_off + COL_U + 32, *reinterpret_cast<float(*)[32]>(&ur[32]));
+        tmem_wait_ld();
+        store_row64_bf16(sm + OFF_UT, j, ur);
+#pragma unroll
+        for (int i = 0; i < C; ++i) ur[i] *= gC / s_gamma[i];
+        store_row64_bf16(sm + OFF_UTP, j, ur);
+        // decay the fp32 master state in place: Sigma^T <- gamma_C Sigma^T
+#pragma unroll 1
+        for (int piece = 0; piece < 4; ++piece) {
+          float x[32];
+          tmem_ld32(tmem + lane_off + COL_S + piece * 32, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= gC;
+          tmem_st32(tmem + lane_off + COL_S + piece * 32, x);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      cw_sync();
+
+      // ---- O_B^T = U^T P^T (N = 64)  and  Sigma^T += U'^T K (N = dk), K = 64 tokens
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          mma_bf16(tmem + COL_OB, kdesc(sbase + OFF_UT + kk * 32), kdesc(sbase + OFF_P + kk * 32),
+                   idesc_bf16(128, 64, 0, 0), kk > 0);
+          mma_bf16(tmem + COL_S, kdesc(sbase + OFF_UTP + kk * 32), mndesc(kq_a + kk * 2048, 16384),
+                   idesc_bf16(128, 128, 0, 1), 1);
+        }
+        mma_commit(bar_mma);
+      }
+      if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
+      mma_phase ^= 1;
+      tc_fence_after();
+      if (tid == 0) mbar_arrive(&bar_empty[s]);   // every read of stage s has completed
+
+      // ---- outputs: o[tok0 + i][h][col0 + j] = scale (gamma_i O_A + O_B)
+      {
+        float oa[32], ob[32];
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          tmem_ld32(tmem + lane_off + COL_OA + half * 32, oa);
+          tmem_ld32(tmem + lane_off + COL_OB + half * 32, ob);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int i = half * 32 + e;
+            if (i < valid) {
+              const float val = p.scale * fmaf(s_gamma[i], oa[e], ob[e]);
+              p.o[((size_t)(tok0 + i) * H + h) * dv + col0 + j] = __float2bfloat16_rn(val);
+            }
+          }
+        }
+      }
+      // ---- next chunk's Sigma^T operand (bf16) and, at the end, S_T (fp32)
+      const bool last = (c == n_chunks - 1);
+#pragma unroll 1
+      for (int piece = 0; piece < 4; ++piece) {
+        float x[32];
+        tmem_ld32(tmem + lane_off + COL_S + piece * 32, x);
+        tmem_wait_ld();
+        uint8_t* slab = sm + OFF_SIG + (piece >> 1) * 16384;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint4 o;
+          o.x = pack_bf16x2(x[cc * 8 + 0], x[cc * 8 + 1]);
+          o.y = pack_bf16x2(x[cc * 8 + 2], x[cc * 8 + 3]);
+          o.z = pack_bf16x2(x[cc * 8 + 4], x[cc * 8 + 5]);
+          o.w = pack_bf16x2(x[cc * 8 + 6], x[cc * 8 + 7]);
+          *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + cc * 8)) = o;
+        }
+        if (last && p.S_T) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) p.S_T[state_base + (size_t)(piece * 32 + e) * dv] = x[e];
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      cw_sync();
+    }
+    if (n_chunks == 0 && p.S_T) {
+      // empty sequence: S_T = S0 (or zero)
+      for (int d = 0; d < DK; ++d)
+        p.S_T[state_base + (size_t)d * dv] = p.S0 ? p.S0[state_base + (size_t)d * dv] : 0.f;
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace tc
+
+// Host launcher: builds the TMA descriptors (3-D views [tokens][H][width] of
+// q, k, v with 64 x 1 x 64 boxes) and launches one CTA per (sequence, head,
+// 128-wide dv slice).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
+            cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, const void* base, int width, int H, int total_tokens) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)total_tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)width * 2 * H};
+  cuuint32_t box[3] = {64, 1, 64};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool prefill_tc_supported(const gdn_fwd_params* p) {
+  return p->io_dtype == GDN_BF16 && p->dk == tc::DK && p->dv % tc::DVS == 0 &&
+         !(p->flags & GDN_PRECISE);
+}
+
+gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(tc::gdn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc::SMEM_BYTES) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    attr_set = true;
+  }
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, p->q, p->dk, p->H, p->total_tokens) ||
+      !make_map(&mk, p->k, p->dk, p->H, p->total_tokens) ||
+      !make_map(&mv, p->v, p->dv, p->H, p->total_tokens))
+    return GDN_ERR_CUDA;
+  tc::Params kp;
+  kp.a = p->a;
+  kp.b = p->b;
+  kp.S0 = p->S0;
+  kp.S_T = p->S_T;
+  kp.o = static_cast<__nv_bfloat16*>(p->o);
+  kp.cu_seqlens = p->cu_seqlens;
+  kp.status = status;
+  kp.n_seq = p->n_seq;
+  kp.seq_len = p->seq_len;
+  kp.total_tokens = p->total_tokens;
+  kp.H = p->H;
+  kp.dv = p->dv;
+  kp.n_slices = p->dv / tc::DVS;
+  kp.scale = p->scale;
+  kp.flags = p->flags;
+  const long long blocks = (long long)p->n_seq * p->H * kp.n_slices;
+  if (blocks <= 0) return GDN_OK;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  tc::gdn_prefill_tc_kernel<<<(unsigned)blocks, tc::THREADS, tc::SMEM_BYTES, stream>>>(mq, mk, mv,
+                                                                                      kp);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace gdn

@@ -1,0 +1,132 @@
+"""The C-ABI library builds, loads without a GPU, exports every entry point its
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import looped_linear_attention_b200 as lla
+from looped_linear_attention_b200 import _binding as B
+from looped_linear_attention_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.library()
+
+
+def _declared_functions():
+    names = []
+    for fname in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fname.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fname)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s+\**\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                             text, flags=re.M):
+            names.append(m.group(1))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace", "gdn_decode_step",
+                     "loop_residual", "gdn_status_string", "gdn_get_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), f"libgdn.so does not export {name}"
+
+
+def test_version_and_status_strings(lib):
+    assert lla.version() >= 100
+    assert lla.status_string(B.GDN_OK) == "ok"
+    assert "invalid" in lla.status_string(B.GDN_ERR_INVALID)
+    assert "timed out" in lla.status_string(B.GDN_ERR_TIMEOUT)
+    assert lla.status_string(99) == "unknown status"
+
+
+def _params(**kw):
+    p = B.gdn_fwd_params()
+    base = dict(q=16, k=32, v=48, a=64, b=80, o=1 << 28, n_seq=1, seq_len=64, total_tokens=64,
+                H=2, dk=128, dv=128, io_dtype=B.GDN_BF16, scale=1.0, flags=0)
+    base.update(kw)
+    for f, val in base.items():
+        setattr(p, f, val)
+    return p
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(dk=96), B.GDN_ERR_UNSUPPORTED),
+    (dict(dv=100), B.GDN_ERR_UNSUPPORTED),
+    (dict(dv=1024), B.GDN_ERR_UNSUPPORTED),
+    (dict(H=0), B.GDN_ERR_INVALID),
+    (dict(io_dtype=7), B.GDN_ERR_INVALID),
+    (dict(flags=0x100), B.GDN_ERR_INVALID),
+    (dict(total_tokens=65), B.GDN_ERR_INVALID),          # != n_seq * seq_len
+    (dict(q=8), B.GDN_ERR_INVALID),                      # misaligned
+    (dict(q=0), B.GDN_ERR_INVALID),                      # null input with tokens
+    (dict(S0=1 << 20, S_T=(1 << 20) + 64), B.GDN_ERR_INVALID),   # partial state overlap
+    (dict(o=16), B.GDN_ERR_INVALID),                     # output overlaps q
+])
+def test_prefill_rejects_bad_arguments_on_host(lib, bad, expect):
+    p = _params(**bad)
+    assert lib.gdn_chunk_fwd(ctypes.byref(p), None, 0, None) == expect
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == ctypes.c_size_t(-1).value
+
+
+def test_prefill_null_params(lib):
+    assert lib.gdn_chunk_fwd(None, None, 0, None) == B.GDN_ERR_INVALID
+
+
+def test_workspace_query_is_zero_for_valid_shapes(lib):
+    p = _params(S0=1 << 20, S_T=1 << 20)     # exact aliasing is allowed
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
+
+
+@pytest.mark.parametrize("args,expect", [
+    (dict(dk=96), B.GDN_ERR_UNSUPPORTED),
+    (dict(dv=40), B.GDN_ERR_UNSUPPORTED),
+    (dict(N=-1), B.GDN_ERR_INVALID),
+    (dict(flags=B.GDN_PRECISE), B.GDN_ERR_INVALID),
+    (dict(q=8), B.GDN_ERR_INVALID),
+    (dict(o=1 << 20), B.GDN_ERR_INVALID),                # output inside the state
+])
+def test_decode_rejects_bad_arguments_on_host(lib, args, expect):
+    base = dict(q=16, k=32, v=48, a=64, b=80, S=1 << 20, o=1 << 30, N=4, H=2, dk=128, dv=128,
+                dt=B.GDN_BF16, scale=1.0, flags=0)
+    base.update(args)
+    st = lib.gdn_decode_step(base["q"], base["k"], base["v"], base["a"], base["b"], base["S"],
+                             base["o"], base["N"], base["H"], base["dk"], base["dv"], base["dt"],
+                             base["scale"], base["flags"], None)
+    assert st == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    (dict(d=7), B.GDN_ERR_INVALID),
+    (dict(rows=-1), B.GDN_ERR_INVALID),
+    (dict(h_tilde=0), B.GDN_ERR_INVALID),
+    (dict(rho=4), B.GDN_ERR_INVALID),
+    (dict(dt=5), B.GDN_ERR_INVALID),
+])
+def test_residual_rejects_bad_arguments_on_host(lib, args, expect):
+    base = dict(h_tilde=16, h_prev=32, rho=48, out=64, rows=4, d=16, dt=B.GDN_BF16)
+    base.update(args)
+    st = lib.loop_residual(base["h_tilde"], base["h_prev"], base["rho"], base["out"],
+                           base["rows"], base["d"], base["dt"], None)
+    assert st == expect
+
+
+def test_empty_work_is_a_no_op(lib):
+    assert lib.loop_residual(None, None, None, None, 0, 16, B.GDN_BF16, None) == B.GDN_OK
+    assert lib.gdn_decode_step(None, None, None, None, None, None, None, 0, 2, 128, 128,
+                               B.GDN_BF16, 1.0, 0, None) == B.GDN_OK
+    p = _params(n_seq=0, seq_len=0, total_tokens=0)
+    assert lib.gdn_chunk_fwd(ctypes.byref(p), None, 0, None) == B.GDN_OK

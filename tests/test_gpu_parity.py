@@ -1,0 +1,324 @@
+"""Parity of the CUDA kernels (through the C ABI) with the CPU oracle.
+
+Small cases span several 64-token chunks with ragged tails and every edge case
+the ABI admits; the full-size workloads run on the GPU exactly as the benchmark
+launches them and are checked on sampled (sequence, head) chains that the
+oracle recomputes one by one.  Bars: relative L2 error 1e-4 for fp32 inputs,
+1e-2 on outputs and 5e-3 on final states for bf16 inputs; the loop residual
+within one bf16 ulp element-wise.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import looped_linear_attention_b200 as lla
+from looped_linear_attention_b200 import workloads as W
+from gpu_util import TOL_BF16_O, TOL_BF16_S, TOL_F32, bf16_ulp, host, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    from looped_linear_attention_b200 import build
+    build.build()
+    lla.library()
+    torch.cuda.init()
+    yield
+    assert lla.gdn_get_device_status() == lla.GDN_OK
+
+
+def _status_ok():
+    st = lla.gdn_get_device_status()
+    assert st == lla.GDN_OK, lla.status_string(st)
+
+
+def _wl(name, **kw):
+    return dataclasses.replace(W.WORKLOADS[name], **kw)
+
+
+def _gpu_prefill(inp, scale=1.0, flags=0, S0="inp", alias=False):
+    q, k, v, a, b = (inp[n].cuda() for n in ("q", "k", "v", "a", "b"))
+    s0 = inp["S0"] if S0 == "inp" else S0
+    s0 = None if s0 is None else s0.cuda()
+    cu = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).cuda()
+    kw = {}
+    if alias:
+        assert s0 is not None
+        kw["S_T"] = s0
+    o, ST = lla.gdn_chunk_fwd(q, k, v, a, b, s0, cu, n_seq=inp["n_seq"], scale=scale,
+                              flags=flags, **kw)
+    torch.cuda.synchronize()
+    return host(o), host(ST)
+
+
+def _oracle_prefill(inp, scale=1.0, normalize=False, S0="inp"):
+    q, k = inp["q"], inp["k"]
+    if normalize:
+        q, k = oracle.qk_l2norm(q), oracle.qk_l2norm(k)
+    s0 = inp["S0"] if S0 == "inp" else S0
+    cu = inp["cu_seqlens"]
+    if cu is None:
+        L = inp["seq_len"]
+        cu = np.arange(inp["n_seq"] + 1, dtype=np.int32) * L
+    return oracle.gdn_fwd(q, k, inp["v"], inp["a"], inp["b"], s0, cu, scale)
+
+
+def _check(o, ST, o_ref, S_ref, fp32):
+    eo, es = rel_l2(o, o_ref), rel_l2(ST, S_ref)
+    if fp32:
+        assert eo < TOL_F32 and es < TOL_F32, (eo, es)
+    else:
+        assert eo < TOL_BF16_O and es < TOL_BF16_S, (eo, es)
+    return eo, es
+
+
+# ------------------------------------------------------------------ residual
+@pytest.mark.parametrize("alias", [False, True])
+def test_loop_residual_bf16_within_one_ulp(alias):
+    g = torch.Generator().manual_seed(W.seed_for("test", "residual"))
+    rows, d = 4099, 2048
+    ht = torch.randn(rows, d, generator=g).bfloat16()
+    hp = torch.randn(rows, d, generator=g).bfloat16()
+    rho = torch.rand(d, generator=g) * 0.5
+    ht_d, hp_d = ht.cuda(), hp.cuda()
+    out = lla.loop_residual(ht_d, hp_d, rho.cuda(), out=hp_d if alias else None)
+    torch.cuda.synchronize()
+    ref = oracle.loop_residual(ht, hp, rho)
+    got = host(out).double().numpy()
+    err = np.abs(got - ref)
+    assert np.all(err <= bf16_ulp(ref) + 1e-30)
+    assert np.mean(got == oracle.round_bf16(ref)) > 0.99
+    _status_ok()
+
+
+def test_loop_residual_f32():
+    g = torch.Generator().manual_seed(W.seed_for("test", "residual32"))
+    ht, hp = torch.randn(37, 24, generator=g), torch.randn(37, 24, generator=g)
+    rho = torch.rand(24, generator=g)
+    out = lla.loop_residual(ht.cuda(), hp.cuda(), rho.cuda())
+    np.testing.assert_allclose(host(out).double().numpy(), oracle.loop_residual(ht, hp, rho),
+                               rtol=1e-6, atol=1e-6)
+
+
+# ------------------------------------------------------------------ decode
+@pytest.mark.parametrize("dk,dv,dtype,flags", [
+    (128, 128, torch.bfloat16, lla.GDN_QK_L2NORM),
+    (128, 128, torch.bfloat16, 0),
+    (64, 64, torch.float32, 0),
+    (128, 192, torch.bfloat16, 0),
+    (64, 256, torch.float32, lla.GDN_QK_L2NORM),
+])
+def test_decode_step(dk, dv, dtype, flags):
+    wl = _wl("decode", dk=dk, dv=dv, dtype=dtype, H=3, normalize_qk=not flags)
+    inp = W.decode_inputs(wl, "cpu", n_slots=37)
+    S = inp["S"].cuda()
+    o = lla.gdn_decode_step(inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda(), inp["a"].cuda(),
+                            inp["b"].cuda(), S, scale=0.75, flags=flags)
+    torch.cuda.synchronize()
+    q, k = inp["q"], inp["k"]
+    if flags & lla.GDN_QK_L2NORM:
+        q, k = oracle.qk_l2norm(q), oracle.qk_l2norm(k)
+    o_ref, S_ref = oracle.gdn_decode(q, k, inp["v"], inp["a"], inp["b"], inp["S"], 0.75)
+    tol_o = TOL_F32 if dtype == torch.float32 else 4e-3   # bf16 output rounding
+    assert rel_l2(host(o), o_ref) < tol_o
+    assert rel_l2(host(S), S_ref) < TOL_F32
+    _status_ok()
+
+
+# ------------------------------------------------------------------ prefill, precise path
+def test_prefill_tiny_workload_fp32():
+    """B=1, H=2, L=256, dk=dv=64, fp32, zero initial state."""
+    inp = W.prefill_inputs(W.WORKLOADS["tiny"], "cpu")
+    o, ST = _gpu_prefill(inp)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o, ST, o_ref, S_ref, fp32=True)
+    _status_ok()
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 192), (64, 64)])
+def test_prefill_precise_varlen_edges(dk, dv):
+    """Empty, 1-token, 63/64/65-token and longer sequences, random S0, q/k
+    normalised in-kernel, scale != 1."""
+    wl = _wl("varlen", dk=dk, dv=dv, H=3, dtype=torch.float32, normalize_qk=False)
+    inp = W.prefill_inputs(wl, "cpu", lengths=[0, 1, 63, 64, 65, 200])
+    o, ST = _gpu_prefill(inp, scale=0.5, flags=lla.GDN_QK_L2NORM)
+    o_ref, S_ref = _oracle_prefill(inp, scale=0.5, normalize=True)
+    _check(o, ST, o_ref, S_ref, fp32=True)
+    np.testing.assert_allclose(ST[0].numpy(), inp["S0"][0].numpy(), rtol=0, atol=0)
+    _status_ok()
+
+
+# ------------------------------------------------------------------ prefill, tensor-core path
+def test_prefill_tc_fixed_length_ragged():
+    wl = _wl("long_prefill", n_seq=2, H=3, seq_len=300, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu")
+    o, ST = _gpu_prefill(inp)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+    _status_ok()
+
+
+def test_prefill_tc_zero_initial_state():
+    wl = _wl("long_prefill", n_seq=1, H=2, seq_len=192)
+    inp = W.prefill_inputs(wl, "cpu")
+    o, ST = _gpu_prefill(inp)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+
+
+def test_prefill_tc_varlen_dv256_l2norm():
+    wl = _wl("varlen", H=2, normalize_qk=False)
+    inp = W.prefill_inputs(wl, "cpu", lengths=[0, 1, 63, 64, 65, 129, 700])
+    o, ST = _gpu_prefill(inp, scale=0.125, flags=lla.GDN_QK_L2NORM)
+    o_ref, S_ref = _oracle_prefill(inp, scale=0.125, normalize=True)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+    np.testing.assert_array_equal(ST[0].numpy(), inp["S0"][0].numpy())
+    _status_ok()
+
+
+def test_prefill_tc_in_place_state():
+    wl = _wl("long_prefill", n_seq=2, H=2, seq_len=130, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu")
+    o, ST = _gpu_prefill(inp, alias=True)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+
+
+def test_prefill_tc_matches_precise_path_and_oracle():
+    wl = _wl("long_prefill", n_seq=1, H=2, seq_len=640, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu")
+    o_tc, S_tc = _gpu_prefill(inp)
+    o_pr, S_pr = _gpu_prefill(inp, flags=lla.GDN_PRECISE)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o_tc, S_tc, o_ref, S_ref, fp32=False)
+    # the fp32 path only sees bf16 rounding of its outputs
+    assert rel_l2(o_pr, o_ref) < 4e-3 and rel_l2(S_pr, S_ref) < TOL_F32
+
+
+def test_prefill_tc_is_deterministic():
+    wl = _wl("long_prefill", n_seq=2, H=2, seq_len=257, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu")
+    o1, S1 = _gpu_prefill(inp)
+    o2, S2 = _gpu_prefill(inp)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_prefill_split_and_resume():
+    """[0, m) then [m, L) with the state carried equals one pass (m not a
+    multiple of the chunk)."""
+    wl = _wl("long_prefill", n_seq=1, H=2, seq_len=1000)
+    inp = W.prefill_inputs(wl, "cpu")
+    m = 333
+    first = {k: (v[:m] if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    first.update(seq_len=m, total_tokens=m)
+    second = {k: (v[m:] if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    second.update(seq_len=1000 - m, total_tokens=1000 - m)
+    o1, S1 = _gpu_prefill(first)
+    o2, S2 = _gpu_prefill(second, S0=S1)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(torch.cat([o1, o2]), S2, o_ref, S_ref, fp32=False)
+
+
+def test_decode_continues_prefill():
+    wl = _wl("long_prefill", n_seq=1, H=2, seq_len=201)
+    inp = W.prefill_inputs(wl, "cpu")
+    L = 200
+    pre = {k: (v[:L] if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    pre.update(seq_len=L, total_tokens=L)
+    _, S_L = _gpu_prefill(pre)
+    S = S_L.cuda()
+    o_d = lla.gdn_decode_step(*(inp[n][L:].cuda() for n in ("q", "k", "v", "a", "b")), S)
+    torch.cuda.synchronize()
+    o_ref, S_ref = _oracle_prefill(inp)
+    assert rel_l2(host(o_d)[0], o_ref[L]) < TOL_BF16_O
+    assert rel_l2(host(S), S_ref) < TOL_BF16_S
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+def _sample_chain_check(inp, o, ST, chains):
+    cu = inp["cu_seqlens"]
+    for s, h in chains:
+        if cu is None:
+            t0, t1 = s * inp["seq_len"], (s + 1) * inp["seq_len"]
+        else:
+            t0, t1 = int(cu[s]), int(cu[s + 1])
+        sl = slice(t0, t1)
+        s0 = None if inp["S0"] is None else host(inp["S0"][s:s + 1, h:h + 1])
+        o_ref, S_ref = oracle.gdn_fwd(host(inp["q"][sl, h:h + 1]), host(inp["k"][sl, h:h + 1]),
+                                      host(inp["v"][sl, h:h + 1]), host(inp["a"][sl, h:h + 1]),
+                                      host(inp["b"][sl, h:h + 1]), s0)
+        _check(host(o[sl, h:h + 1]), host(ST[s:s + 1, h:h + 1]), o_ref, S_ref, fp32=False)
+
+
+def test_full_long_prefill_sampled():
+    """B=8, H=16, L=16384, dk=dv=128 bf16, one loop launched as the benchmark does."""
+    wl = W.WORKLOADS["long_prefill"]
+    inp = W.prefill_inputs(wl, "cuda")
+    o, ST = lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], None, None,
+                              n_seq=wl.n_seq)
+    torch.cuda.synchronize()
+    _status_ok()
+    _sample_chain_check(inp, o, ST, [(0, 0), (7, 15), (3, 9)])
+
+
+def test_full_varlen_sampled():
+    """64 sequences, lengths U[512, 32768], H=16, dk=128, dv=256, random S0."""
+    wl = W.WORKLOADS["varlen"]
+    inp = W.prefill_inputs(wl, "cuda")
+    cu = torch.from_numpy(inp["cu_seqlens"]).cuda()
+    o, ST = lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S0"], cu)
+    torch.cuda.synchronize()
+    _status_ok()
+    lens = np.diff(inp["cu_seqlens"])
+    chains = [(int(np.argmin(lens)), 0), (int(np.argmax(lens)), 5), (17, 11)]
+    _sample_chain_check(inp, o, ST, chains)
+    del inp, o, ST
+    torch.cuda.empty_cache()
+
+
+def test_full_decode_sampled():
+    """24576 slots x 16 heads, 128 x 128 fp32 states, in place."""
+    wl = W.WORKLOADS["decode"]
+    inp = W.decode_inputs(wl, "cuda")
+    rng = np.random.default_rng(0)
+    slots = np.sort(rng.choice(wl.n_seq, 24, replace=False))
+    S_before = host(inp["S"][slots])
+    o = lla.gdn_decode_step(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S"])
+    torch.cuda.synchronize()
+    _status_ok()
+    o_ref, S_ref = oracle.gdn_decode(host(inp["q"][slots]), host(inp["k"][slots]),
+                                     host(inp["v"][slots]), host(inp["a"][slots]),
+                                     host(inp["b"][slots]), S_before)
+    assert rel_l2(host(o[slots]), o_ref) < 4e-3
+    assert rel_l2(host(inp["S"][slots]), S_ref) < TOL_F32
+    del inp
+    torch.cuda.empty_cache()
+
+
+def test_looped_prefill_end_to_end():
+    """B=1, L=4096, d=2048 (16 heads x 128), T=4 loops of projection -> GDN
+    (q, k normalised in-kernel) -> loop residual, against the oracle's own chain."""
+    wl = W.WORKLOADS["looped_prefill"]
+    inp = W.looped_inputs(wl, "cpu")
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    runner = lla.LoopedPrefill(inp["L"], wl.H, wl.dk, wl.dv, wl.loops, "cuda")
+    hT = runner.run(dev["h0"], dev["Wq"], dev["Wk"], dev["Wv"], dev["a"], dev["b"], dev["rho"])
+    torch.cuda.synchronize()
+    _status_ok()
+    ref = oracle.looped_forward(inp["h0"], inp["Wq"], inp["Wk"], inp["Wv"], inp["a"], inp["b"],
+                                inp["rho"], wl.H, wl.dk, wl.dv)
+    assert rel_l2(host(hT), ref) < TOL_BF16_O
+    # first loop's mixer on identical projections
+    L, d = inp["L"], inp["d"]
+    q = (dev["h0"] @ dev["Wq"]).view(L, wl.H, wl.dk)
+    k = (dev["h0"] @ dev["Wk"]).view(L, wl.H, wl.dk)
+    v = (dev["h0"] @ dev["Wv"]).view(L, wl.H, wl.dv)
+    o, _ = lla.gdn_chunk_fwd(q, k, v, dev["a"][0].contiguous(), dev["b"][0].contiguous(),
+                             flags=lla.GDN_QK_L2NORM)
+    o_ref, _ = oracle.gdn_fwd(oracle.qk_l2norm(host(q)), oracle.qk_l2norm(host(k)), host(v),
+                              inp["a"][0], inp["b"][0])
+    assert rel_l2(host(o), o_ref) < TOL_BF16_O

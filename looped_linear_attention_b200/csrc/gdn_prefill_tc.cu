@@ -138,17 +138,63 @@ __device__ __forceinline__ void l2norm_row(uint8_t* kq, int row_in_tile, uint32_
   }
 }
 
-// Writes 64 fp32 values (one tensor-memory row over 64 columns) as a bf16 row of
-// a 128-byte-swizzled K-major tile.
-__device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int row, const float (&x)[64]) {
+// Writes 32 fp32 values as bf16 into columns [col0, col0 + 32) of one row of a
+// 128-byte-swizzled K-major tile (four 16-byte chunks).
+__device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int row, int col0, const float (&x)[32]) {
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < 4; ++c) {
     uint4 o;
     o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
     o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
     o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
     o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
-    *reinterpret_cast<uint4*>(tile + sw128_offset(row, c * 8)) = o;
+    *reinterpret_cast<uint4*>(tile + sw128_offset(row, col0 + c * 8)) = o;
+  }
+}
+
+// T = (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32, row stride
+// A_LD), written to s_T (fp32, row stride A_LD; its upper block triangle is left
+// unset).  Blocked by 16: the four diagonal blocks are inverted by forward
+// substitution (one column per thread), then the off-diagonal blocks follow by
+// increasing block distance d: T_{b+d,b} = -T_{b+d,b+d} sum_{m=b}^{b+d-1} A_{b+d,m} T_{m,b}.
+// All 128 compute threads take part; s_Y is 3 x 16 x 17 fp32 scratch.
+__device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_T, float* s_Y, int tid) {
+  if (tid < 64) {
+    const int r0 = (tid >> 4) * 16, c = tid & 15;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float acc = (i == c) ? 1.f : 0.f;
+#pragma unroll
+      for (int m = 0; m < i; ++m) acc = fmaf(-s_A[(r0 + i) * A_LD + r0 + m], x[m], acc);
+      x[i] = acc;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s_T[(r0 + i) * A_LD + r0 + c] = x[i];
+  }
+  cw_sync();
+#pragma unroll 1
+  for (int d = 1; d < 4; ++d) {
+    const int nb = 4 - d;
+    for (int e = tid; e < nb * 256; e += CW) {
+      const int bb = e >> 8, r = (e >> 4) & 15, c = e & 15;
+      const int rowA = (bb + d) * 16 + r;
+      float acc = 0.f;
+      for (int kk = bb * 16; kk < (bb + d) * 16; ++kk)
+        acc = fmaf(s_A[rowA * A_LD + kk], s_T[kk * A_LD + bb * 16 + c], acc);
+      s_Y[(bb * 16 + r) * 17 + c] = acc;
+    }
+    cw_sync();
+    for (int e = tid; e < nb * 256; e += CW) {
+      const int bb = e >> 8, r = (e >> 4) & 15, c = e & 15;
+      const int rowT = (bb + d) * 16 + r;
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        acc = fmaf(s_T[rowT * A_LD + (bb + d) * 16 + k], s_Y[(bb * 16 + k) * 17 + c], acc);
+      s_T[rowT * A_LD + bb * 16 + c] = -acc;
+    }
+    cw_sync();
   }
 }
 
@@ -338,44 +384,49 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_phase ^= 1;
       tc_fence_after();
       {
-        float gr[64];
-        tmem_ld32(tmem + lane_off + COL_G, *reinterpret_cast<float(*)[32]>(&gr[0]));
-        tmem_ld32(tmem + lane_off + COL_G + 32, *reinterpret_cast<float(*)[32]>(&gr[32]));
-        tmem_wait_ld();
-        if (tid < C) {
-          const int i = tid;
-          const float gi = s_g[i], bi = s_b[i];
+        // A (rows 0-63, fp32, for the solve) and P (rows 64-127 -> bf16 operand),
+        // 32 columns of G at a time
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float gr[32];
+          tmem_ld32(tmem + lane_off + COL_G + half * 32, gr);
+          if (tid < C) {
+            const int i = tid;
+            const float gi = s_g[i], bi = s_b[i];
 #pragma unroll
-          for (int jj = 0; jj < C; ++jj)
-            s_A[i * A_LD + jj] = (jj < i) ? bi * expf(gi - s_g[jj]) * gr[jj] : 0.f;
-        } else {
-          const int i = tid - C;
-          const float gi = s_g[i];
+            for (int e = 0; e < 32; ++e) {
+              const int jj = half * 32 + e;
+              s_A[i * A_LD + jj] = (jj < i) ? bi * expf(gi - s_g[jj]) * gr[e] : 0.f;
+            }
+          } else {
+            const int i = tid - C;
+            const float gi = s_g[i];
 #pragma unroll
-          for (int jj = 0; jj < C; ++jj) gr[jj] = (jj <= i) ? expf(gi - s_g[jj]) * gr[jj] : 0.f;
-          store_row64_bf16(sm + OFF_P, i, gr);
+            for (int e = 0; e < 32; ++e) {
+              const int jj = half * 32 + e;
+              gr[e] = (jj <= i) ? expf(gi - s_g[jj]) * gr[e] : 0.f;
+            }
+            store_row32_bf16(sm + OFF_P, i, half * 32, gr);
+          }
         }
       }
+      tc_fence_before();
       cw_sync();
 
-      // ---- T = (I + A)^{-1} by forward substitution, one column per thread
-      if (tid < C) {
-        const int col = tid;
-        float x[C];
-#pragma unroll
-        for (int i = 0; i < C; ++i) {
-          float acc = (i == col) ? 1.f : 0.f;
-#pragma unroll
-          for (int m = 0; m < i; ++m) acc = fmaf(-s_A[i * A_LD + m], x[m], acc);
-          x[i] = acc;
-        }
-        const float bj = s_b[col], bgj = s_b[col] * s_gamma[col];
+      // ---- T = (I + A)^{-1} (blocked, scratch in the U^T tiles, which are free here),
+      // then T1 = T diag(b gamma) and T2 = T diag(b) as bf16 operands
+      {
+        float* s_T = reinterpret_cast<float*>(sm + OFF_UT);
+        float* s_Y = s_T + 64 * A_LD;
+        invert_unit_lower_64(s_A, s_T, s_Y, tid);
         uint8_t* t1 = sm + OFF_T1;
         uint8_t* t2 = sm + OFF_T2;
-#pragma unroll
-        for (int i = 0; i < C; ++i) {
-          *reinterpret_cast<__nv_bfloat16*>(t1 + sw128_offset(i, col)) = __float2bfloat16_rn(x[i] * bgj);
-          *reinterpret_cast<__nv_bfloat16*>(t2 + sw128_offset(i, col)) = __float2bfloat16_rn(x[i] * bj);
+        for (int e = tid; e < C * C; e += CW) {
+          const int i = e >> 6, jc = e & 63;
+          const float t = ((jc >> 4) > (i >> 4)) ? 0.f : s_T[i * A_LD + jc];
+          const float bj = s_b[jc];
+          *reinterpret_cast<__nv_bfloat16*>(t1 + sw128_offset(i, jc)) = __float2bfloat16_rn(t * bj * s_gamma[jc]);
+          *reinterpret_cast<__nv_bfloat16*>(t2 + sw128_offset(i, jc)) = __float2bfloat16_rn(t * bj);
         }
       }
       fence_proxy_async_smem();
@@ -397,17 +448,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_phase ^= 1;
       tc_fence_after();
       {
-        // W^T row d = tid -> column d of W ([64 tok][128 dk] tile, 2 slabs)
-        float wr[64];
-        tmem_ld32(tmem + lane_off + COL_W, *reinterpret_cast<float(*)[32]>(&wr[0]));
-        tmem_ld32(tmem + lane_off + COL_W + 32, *reinterpret_cast<float(*)[32]>(&wr[32]));
-        tmem_wait_ld();
+        // W^T row d = tid -> column d of W ([64 tok][128 dk] tile, 2 slabs), 32 tokens at a time
         uint8_t* slab = sm + OFF_W + (tid >> 6) * 8192;
         const int dcol = tid & 63;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float wr[32];
+          tmem_ld32(tmem + lane_off + COL_W + half * 32, wr);
 #pragma unroll
-        for (int i = 0; i < C; ++i)
-          *reinterpret_cast<__nv_bfloat16*>(slab + sw128_offset(i, dcol)) = __float2bfloat16_rn(wr[i]);
+          for (int e = 0; e < 32; ++e)
+            *reinterpret_cast<__nv_bfloat16*>(slab + sw128_offset(half * 32 + e, dcol)) =
+                __float2bfloat16_rn(wr[e]);
+        }
       }
+      tc_fence_before();
       fence_proxy_async_smem();
       cw_sync();
 
@@ -431,20 +485,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float gC = s_gamma[C - 1];
       {
         // U^T row j (dv) over 64 tokens -> operand tiles U^T and U^T diag(gamma_C / gamma)
-        float ur[64];
-        tmem_ld32(tmem + lane_off + COL_U, *reinterpret_cast<float(*)[32]>(&ur[0]));
-        tmem_ld32(tmem + lane_off + COL_U + 32, *reinterpret_cast<float(*)[32]>(&ur[32]));
-        tmem_wait_ld();
-        store_row64_bf16(sm + OFF_UT, j, ur);
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float ur[32];
+          tmem_ld32(tmem + lane_off + COL_U + half * 32, ur);
+          store_row32_bf16(sm + OFF_UT, j, half * 32, ur);
 #pragma unroll
-        for (int i = 0; i < C; ++i) ur[i] *= gC / s_gamma[i];
-        store_row64_bf16(sm + OFF_UTP, j, ur);
+          for (int e = 0; e < 32; ++e) ur[e] *= gC / s_gamma[half * 32 + e];
+          store_row32_bf16(sm + OFF_UTP, j, half * 32, ur);
+        }
         // decay the fp32 master state in place: Sigma^T <- gamma_C Sigma^T
 #pragma unroll 1
         for (int piece = 0; piece < 4; ++piece) {
           float x[32];
           tmem_ld32(tmem + lane_off + COL_S + piece * 32, x);
-          tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) x[e] *= gC;
           tmem_st32(tmem + lane_off + COL_S + piece * 32, x);
@@ -479,7 +533,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int half = 0; half < 2; ++half) {
           tmem_ld32(tmem + lane_off + COL_OA + half * 32, oa);
           tmem_ld32(tmem + lane_off + COL_OB + half * 32, ob);
-          tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int i = half * 32 + e;
@@ -496,7 +549,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int piece = 0; piece < 4; ++piece) {
         float x[32];
         tmem_ld32(tmem + lane_off + COL_S + piece * 32, x);
-        tmem_wait_ld();
         uint8_t* slab = sm + OFF_SIG + (piece >> 1) * 16384;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {

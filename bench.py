@@ -474,6 +474,36 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """Small fixed case for profiler captures: `--profile WORKLOAD` runs only that
+    workload's kernel (warm-up + steps launches) with `--n-seq` sequences/slots."""
+    import torch
+    import looped_linear_attention_b200 as lla
+    from looped_linear_attention_b200 import workloads as W
+    import dataclasses
+    torch.cuda.set_device(0)
+    wl = W.WORKLOADS[args.profile]
+    if args.n_seq:
+        wl = dataclasses.replace(wl, n_seq=args.n_seq)
+    dev = torch.device("cuda", 0)
+    if args.profile == "decode":
+        inp = W.decode_inputs(wl, dev)
+        run = lambda: lla.gdn_decode_step(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S"])
+    else:
+        inp = W.prefill_inputs(wl, dev)
+        cu = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).to(dev)
+        run = lambda: lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S0"], cu,
+                                        n_seq=inp["n_seq"])
+    for _ in range(args.warmup + args.steps):
+        run()
+    torch.cuda.synchronize()
+    st = lla.gdn_get_device_status()
+    print(json.dumps({"profile_case": args.profile, "n_seq": wl.n_seq, "launches": args.warmup + args.steps,
+                      "status": lla.status_string(st)}))
+    if st != lla.GDN_OK:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -483,7 +513,13 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile", choices=["tiny", "long_prefill", "varlen", "decode"], default=None,
+                    help="run only this workload's kernel (for profiler captures)")
+    ap.add_argument("--n-seq", type=int, default=0, help="sequences (or decode slots) for --profile")
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

@@ -48,14 +48,42 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         return LIB_PATH
     tmp = LIB_PATH + f".tmp{os.getpid()}"
     cmd = [_nvcc(), "-O3", "-std=c++17", *ARCH_FLAGS, "-lineinfo", "-Xcompiler", "-fPIC",
-           "-shared", "-cudart", "static", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
-    if ptxas_info:
-        cmd.insert(1, "-Xptxas=-v")
+           "-shared", "-cudart", "static", "-Xptxas=-v", "-I", INCLUDE, "-I", CSRC, "-o", tmp,
+           *sources()]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if ptxas_info or r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+    if r.returncode != 0:
+        raise RuntimeError("nvcc failed")
+    spills = check_no_spills(r.stdout + r.stderr)
+    if spills:
+        os.remove(tmp)
+        raise RuntimeError("register spills in " + ", ".join(spills) +
+                           " (the tensor-core kernels are kept spill-free)")
     os.replace(tmp, LIB_PATH)
     return LIB_PATH
+
+
+# Kernels that drive tcgen05 / tensor memory must not spill registers: spills
+# around asynchronously written tensor-memory load registers were the one
+# difference between faulting and clean builds of the prefill kernel.
+SPILL_FREE_KERNELS = ("gdn_prefill_tc_kernel",)
+
+
+def check_no_spills(ptxas_log: str):
+    """Names of the tensor-core kernels for which ptxas reports spill stores or loads."""
+    bad, current = [], None
+    for line in ptxas_log.splitlines():
+        if "Compiling entry function" in line:
+            current = line.split("'")[1] if "'" in line else line
+        elif "spill stores" in line and current:
+            nums = [int(t) for t in line.replace(",", " ").split() if t.isdigit()]
+            if len(nums) >= 3 and (nums[1] or nums[2]) and any(
+                    k in current for k in SPILL_FREE_KERNELS):
+                bad.append(current)
+    return bad
 
 
 def main():

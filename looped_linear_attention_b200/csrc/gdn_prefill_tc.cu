@@ -23,10 +23,17 @@
 //     W^T = K^T T1^T, O_A^T = Sigma^T Q^T, O_B^T = U^T P^T,
 //     Sigma^T += (U^T diag(gamma_C/gamma)) K.
 //   * q, k, v tiles arrive by TMA (128-byte swizzle) into a 2-stage ring filled
-//     by a producer warp; operands computed in the CTA (T1, T2, P, W, U^T,
-//     Sigma^T) are rounded to bf16 and written in the same swizzled layout.
-//   * the fp32 master state stays in tensor memory for the whole sequence; its
-//     bf16 copy in shared memory feeds the next chunk's MMAs.
+//     by a producer warp; K and V are read straight from their tiles as
+//     MN-major operands.  Operands computed in the CTA (T1, T2, P, W^T, U^T,
+//     Sigma^T) are rounded to bf16 and written as whole 16-byte chunks in the
+//     same swizzled layout (W^T is an MN-major B operand, so every thread
+//     writes one contiguous row).
+//   * the fp32 master state stays in tensor memory for the whole sequence,
+//     kept pre-multiplied by the next chunk's gamma_C so that the carry MMA
+//     accumulates straight onto it; its bf16 copy in shared memory feeds the
+//     next chunk's MMAs.
+//   * T = (I + A)^{-1} is inverted in 16 x 16 blocks on the CUDA cores; gate
+//     vectors (gamma, b gamma, gamma_C / gamma) are computed once per token.
 //   * every wait is bounded (GDN_ERR_TIMEOUT) so a fault in the schedule cannot
 //     hang the GPU.
 #include "common.cuh"
@@ -47,7 +54,7 @@ constexpr uint32_t COL_W = 64;    // W^T            128 x 64
 constexpr uint32_t COL_U = 128;   // U^T            128 x 64
 constexpr uint32_t COL_OA = 192;  // Sigma^T Q^T    128 x 64
 constexpr uint32_t COL_OB = 256;  // U^T P^T        128 x 64
-constexpr uint32_t COL_S = 384;   // Sigma^T fp32   128 x 128
+constexpr uint32_t COL_S = 384;   // Sigma^T fp32   128 x 128 (kept pre-decayed by gamma_C)
 constexpr uint32_t TMEM_COLS = 512;
 
 // Shared-memory plan (offsets from a 1024-byte aligned base).
@@ -56,20 +63,22 @@ constexpr uint32_t KQ_BYTES = 32768;
 constexpr uint32_t OFF_V = OFF_KQ + STAGES * KQ_BYTES;  // STAGES x 16 KB: [V0|V1]
 constexpr uint32_t V_BYTES = 16384;
 constexpr uint32_t OFF_SIG = OFF_V + STAGES * V_BYTES;  // Sigma^T bf16 [128 dv][128 dk], 2 x 16 KB slabs
-constexpr uint32_t OFF_W = OFF_SIG + 32768;             // W bf16 [64 tok][128 dk], 2 x 8 KB slabs
-constexpr uint32_t OFF_UT = OFF_W + 16384;              // U^T bf16 [128 dv][64 tok]
-constexpr uint32_t OFF_UTP = OFF_UT + 16384;            // U^T diag(gamma_C/gamma) bf16
+constexpr uint32_t OFF_WT = OFF_SIG + 32768;            // W^T bf16 [128 dk][64 tok] (MN-major B operand)
+constexpr uint32_t OFF_UT = OFF_WT + 16384;             // U^T bf16 [128 dv][64 tok]; solve scratch
+constexpr uint32_t OFF_UTP = OFF_UT + 16384;            // U^T diag(gamma_C/gamma) bf16; output staging
 constexpr uint32_t OFF_P = OFF_UTP + 16384;             // P bf16 [64][64]
 constexpr uint32_t OFF_T1 = OFF_P + 8192;               // T diag(b gamma) bf16 [64][64]
 constexpr uint32_t OFF_T2 = OFF_T1 + 8192;              // T diag(b) bf16 [64][64]
 constexpr uint32_t OFF_A = OFF_T2 + 8192;               // A fp32 [64][65] (padded rows)
 constexpr int A_LD = 65;
-constexpr uint32_t OFF_GATE = OFF_A + 64 * A_LD * 4;    // g, gamma, b: 3 x 64 fp32
-constexpr uint32_t OFF_BAR = OFF_GATE + 3 * 256;        // mbarriers
+constexpr uint32_t OFF_GATE = OFF_A + 64 * A_LD * 4;    // 2 buffers x {g, gamma, b, b*gamma, gamma_C/gamma}
+constexpr uint32_t GATE_BYTES = 5 * 64 * 4;
+constexpr uint32_t OFF_BAR = OFF_GATE + 2 * GATE_BYTES; // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 64;             // tmem base, abort, scan carry
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;       // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
+static_assert(64 * A_LD * 4 + 48 * 17 * 4 <= 32768, "solve scratch exceeds the U^T tiles");
 
 struct Params {
   const float* a;
@@ -83,6 +92,20 @@ struct Params {
   float scale;
   unsigned flags;
 };
+
+// Per-chunk gate vectors (one buffer).
+struct Gates {
+  float* g;      // prefix sum of log a
+  float* gamma;  // exp(g)
+  float* b;      // write strength (0 past the sequence end)
+  float* bg;     // b * gamma
+  float* r;      // gamma_C / gamma = exp(g_C - g)
+};
+
+__device__ __forceinline__ Gates gates_at(uint8_t* sm, int buf) {
+  float* base = reinterpret_cast<float*>(sm + OFF_GATE + buf * GATE_BYTES);
+  return Gates{base, base + 64, base + 128, base + 192, base + 256};
+}
 
 // Named barrier of the four compute warps (the warp is reconverged first: the
 // barrier is warp-aligned and the bounded waits exit lane by lane).
@@ -139,7 +162,7 @@ __device__ __forceinline__ void l2norm_row(uint8_t* kq, int row_in_tile, uint32_
 }
 
 // Writes 32 fp32 values as bf16 into columns [col0, col0 + 32) of one row of a
-// 128-byte-swizzled K-major tile (four 16-byte chunks).
+// 128-byte-swizzled tile with 128-byte rows (four 16-byte chunks).
 __device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int row, int col0, const float (&x)[32]) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -152,12 +175,84 @@ __device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int row, int col
   }
 }
 
+// Gate vectors of one chunk (all 128 compute threads call this; threads 0-63
+// own one token each).  Rows past the sequence end get log a = 0 and b = 0.
+__device__ __forceinline__ void compute_gates(const Params& p, Gates G, float* s_carry, int tok0,
+                                              int valid, int h, int tid) {
+  const int lane = tid & 31;
+  float la = 0.f;
+  if (tid < C) {
+    float bb = 0.f;
+    if (tid < valid) {
+      const size_t ti = (size_t)(tok0 + tid) * p.H + h;
+      la = logf(__ldg(p.a + ti));
+      bb = __ldg(p.b + ti);
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, la, off);
+      if (lane >= off) la += y;
+    }
+    if (tid == 31) *s_carry = la;
+    G.b[tid] = bb;
+  }
+  cw_sync();
+  if (tid < C) {
+    if (tid >= 32) la += *s_carry;
+    G.g[tid] = la;
+  }
+  cw_sync();
+  if (tid < C) {
+    const float gC = G.g[C - 1];
+    const float gam = __expf(la);
+    G.gamma[tid] = gam;
+    G.bg[tid] = G.b[tid] * gam;
+    G.r[tid] = __expf(gC - la);
+  }
+}
+
 // T = (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32, row stride
-// A_LD), written to s_T (fp32, row stride A_LD; its upper block triangle is left
-// unset).  Blocked by 16: the four diagonal blocks are inverted by forward
-// substitution (one column per thread), then the off-diagonal blocks follow by
-// increasing block distance d: T_{b+d,b} = -T_{b+d,b+d} sum_{m=b}^{b+d-1} A_{b+d,m} T_{m,b}.
-// All 128 compute threads take part; s_Y is 3 x 16 x 17 fp32 scratch.
+// A_LD), blocked by 16.  The diagonal blocks are inverted by forward
+// substitution (one column per thread); the off-diagonal blocks follow by
+// block distance D: T_{b+D,b} = -T_{b+D,b+D} sum_{m=b}^{b+D-1} A_{b+D,m} T_{m,b}.
+// s_T receives T (its upper block triangle is left unset); s_Y is 3 x 16 x 17
+// fp32 scratch.  Every compute thread takes part (the barriers are inside).
+template <int D>
+__device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, float* s_Y, int tid) {
+  constexpr int NB = 4 - D;
+  constexpr int ITEMS = NB * 128;   // (block, row, column pair c / c+8)
+  for (int it = tid; it < ITEMS; it += CW) {
+    const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
+    const float* arow = s_A + ((bb + D) * 16 + r) * A_LD + bb * 16;
+    const float* tcol = s_T + (bb * 16) * A_LD + bb * 16 + c;
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16 * D; ++k) {
+      const float av = arow[k];
+      y0 = fmaf(av, tcol[k * A_LD], y0);
+      y1 = fmaf(av, tcol[k * A_LD + 8], y1);
+    }
+    s_Y[(bb * 16 + r) * 17 + c] = y0;
+    s_Y[(bb * 16 + r) * 17 + c + 8] = y1;
+  }
+  cw_sync();
+  for (int it = tid; it < ITEMS; it += CW) {
+    const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
+    const float* trow = s_T + ((bb + D) * 16 + r) * A_LD + (bb + D) * 16;
+    const float* ycol = s_Y + (bb * 16) * 17 + c;
+    float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float tv = trow[k];
+      t0 = fmaf(tv, ycol[k * 17], t0);
+      t1 = fmaf(tv, ycol[k * 17 + 8], t1);
+    }
+    s_T[((bb + D) * 16 + r) * A_LD + bb * 16 + c] = -t0;
+    s_T[((bb + D) * 16 + r) * A_LD + bb * 16 + c + 8] = -t1;
+  }
+  cw_sync();
+}
+
 __device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_T, float* s_Y, int tid) {
   if (tid < 64) {
     const int r0 = (tid >> 4) * 16, c = tid & 15;
@@ -173,29 +268,42 @@ __device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_
     for (int i = 0; i < 16; ++i) s_T[(r0 + i) * A_LD + r0 + c] = x[i];
   }
   cw_sync();
+  offdiag_level<1>(s_A, s_T, s_Y, tid);
+  offdiag_level<2>(s_A, s_T, s_Y, tid);
+  offdiag_level<3>(s_A, s_T, s_Y, tid);
+}
+
+// Sigma^T row j (fp32, in tensor memory) -> bf16 operand tile for the next
+// chunk; the tensor-memory copy is scaled by `decay` (gamma_C of the next
+// chunk) so that the next carry MMA accumulates onto gamma_C Sigma.  With
+// `st_out`, the unscaled fp32 row is also written as column j of S_T.
+__device__ __forceinline__ void refresh_state(uint32_t taddr, uint8_t* sig, int j, float decay,
+                                              bool scale_tmem, float* st_out, int dv) {
 #pragma unroll 1
-  for (int d = 1; d < 4; ++d) {
-    const int nb = 4 - d;
-    for (int e = tid; e < nb * 256; e += CW) {
-      const int bb = e >> 8, r = (e >> 4) & 15, c = e & 15;
-      const int rowA = (bb + d) * 16 + r;
-      float acc = 0.f;
-      for (int kk = bb * 16; kk < (bb + d) * 16; ++kk)
-        acc = fmaf(s_A[rowA * A_LD + kk], s_T[kk * A_LD + bb * 16 + c], acc);
-      s_Y[(bb * 16 + r) * 17 + c] = acc;
-    }
-    cw_sync();
-    for (int e = tid; e < nb * 256; e += CW) {
-      const int bb = e >> 8, r = (e >> 4) & 15, c = e & 15;
-      const int rowT = (bb + d) * 16 + r;
-      float acc = 0.f;
+  for (int piece = 0; piece < 4; ++piece) {
+    float x[32];
+    tmem_ld32(taddr + piece * 32, x);
+    uint8_t* slab = sig + (piece >> 1) * 16384;
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        acc = fmaf(s_T[rowT * A_LD + (bb + d) * 16 + k], s_Y[(bb * 16 + k) * 17 + c], acc);
-      s_T[rowT * A_LD + bb * 16 + c] = -acc;
+    for (int cc = 0; cc < 4; ++cc) {
+      uint4 o;
+      o.x = pack_bf16x2(x[cc * 8 + 0], x[cc * 8 + 1]);
+      o.y = pack_bf16x2(x[cc * 8 + 2], x[cc * 8 + 3]);
+      o.z = pack_bf16x2(x[cc * 8 + 4], x[cc * 8 + 5]);
+      o.w = pack_bf16x2(x[cc * 8 + 6], x[cc * 8 + 7]);
+      *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + cc * 8)) = o;
     }
-    cw_sync();
+    if (st_out) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) st_out[(size_t)(piece * 32 + e) * dv] = x[e];
+    }
+    if (scale_tmem) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] *= decay;
+      tmem_st32(taddr + piece * 32, x);
+    }
   }
+  tmem_wait_st();
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -205,9 +313,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  float* s_g = reinterpret_cast<float*>(sm + OFF_GATE);
-  float* s_gamma = s_g + 64;
-  float* s_b = s_g + 128;
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint64_t* bar_empty = bar_full + STAGES;
   uint64_t* bar_mma = bar_empty + STAGES;
@@ -273,7 +378,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued[STAGES] = {0, 0};
+      int issued0 = 0, issued1 = 0;
       for (int c = 0; c < n_chunks; ++c) {
         const int s = c % STAGES;
         const int use = c / STAGES;
@@ -288,45 +393,56 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_3d(kq + 24576, &tm_q, &bar_full[s], 64, h, tok0);
         tma_load_3d(vv + 0, &tm_v, &bar_full[s], col0, h, tok0);
         tma_load_3d(vv + 8192, &tm_v, &bar_full[s], col0 + 64, h, tok0);
-        issued[s] = use + 1;
+        if (s == 0) issued0 = use + 1; else issued1 = use + 1;
       }
       // never leave the block with bulk copies still landing in its shared memory
-      for (int s = 0; s < STAGES; ++s)
-        if (issued[s] > 0) mbar_wait_bounded(&bar_full[s], (issued[s] - 1) & 1, nullptr, p.status);
+      if (issued0 > 0) mbar_wait_bounded(&bar_full[0], (issued0 - 1) & 1, nullptr, p.status);
+      if (issued1 > 0) mbar_wait_bounded(&bar_full[1], (issued1 - 1) & 1, nullptr, p.status);
     }
   } else {
     // ------------------------------------------------------------ compute warpgroup
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;   // this warp's tensor-memory lanes
     const int j = tid;                                        // dv row (or dk row) owned
     const size_t state_base = ((size_t)seq * H + h) * DK * (size_t)dv + col0 + j;
+    const uint32_t sbase = smem_u32(sm);
     uint32_t mma_phase = 0;
 
-    // initial state: Sigma^T row j = column (col0 + j) of S0, fp32 into tensor memory,
-    // bf16 into the Sigma^T operand tile.
+    // gates of chunk 0, then the initial state: Sigma^T row j = column (col0 + j)
+    // of S0; tensor memory holds gamma_C(0) * S0, the bf16 operand holds S0.
+    if (n_chunks > 0) compute_gates(p, gates_at(sm, 0), s_carry, seq_start, min(C, len), h, tid);
+    cw_sync();
+    {
+      const float decay0 = (n_chunks > 0) ? gates_at(sm, 0).gamma[C - 1] : 1.f;
 #pragma unroll 1
-    for (int piece = 0; piece < 4; ++piece) {
-      float x[32];
+      for (int piece = 0; piece < 4; ++piece) {
+        float x[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        x[e] = p.S0 ? __ldg(p.S0 + state_base + (size_t)(piece * 32 + e) * dv) : 0.f;
-      tmem_st32(tmem + lane_off + COL_S + piece * 32, x);
-      uint8_t* slab = sm + OFF_SIG + (piece >> 1) * 16384;
+        for (int e = 0; e < 32; ++e)
+          x[e] = p.S0 ? __ldg(p.S0 + state_base + (size_t)(piece * 32 + e) * dv) : 0.f;
+        uint8_t* slab = sm + OFF_SIG + (piece >> 1) * 16384;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 o;
-        o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
-        o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
-        o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
-        o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
-        *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + c * 8)) = o;
+        for (int c = 0; c < 4; ++c) {
+          uint4 o;
+          o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
+          o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
+          o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
+          o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
+          *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + c * 8)) = o;
+        }
+        if (n_chunks == 0 && p.S_T) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) p.S_T[state_base + (size_t)(piece * 32 + e) * dv] = x[e];
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] *= decay0;
+        tmem_st32(tmem + lane_off + COL_S + piece * 32, x);
       }
+      tmem_wait_st();
     }
-    tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
     cw_sync();
 
-    const uint32_t sbase = smem_u32(sm);
     bool ok = true;
 #pragma unroll 1
     for (int c = 0; c < n_chunks && ok; ++c) {
@@ -337,29 +453,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
       const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
       const uint32_t v_a = sbase + OFF_V + s * V_BYTES;
-
-      // ---- gates: g = inclusive prefix sum of log a over the chunk (rows past the
-      // sequence end get log a = 0, b = 0, which removes them from every product)
-      if (tid < C) {
-        float la = 0.f, bb = 0.f;
-        if (tid < valid) {
-          const size_t ti = (size_t)(tok0 + tid) * H + h;
-          la = logf(__ldg(p.a + ti));
-          bb = __ldg(p.b + ti);
-        }
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, la, off);
-          if (lane >= off) la += y;
-        }
-        if (tid == 31) *s_carry = la;
-        s_b[tid] = bb;
-        s_g[tid] = la;   // partial (warp 1 adds the carry below)
-      }
-      cw_sync();
-      if (tid >= 32 && tid < C) s_g[tid] += *s_carry;
-      cw_sync();
-      if (tid < C) s_gamma[tid] = expf(s_g[tid]);
+      const Gates G = gates_at(sm, c & 1);
 
       if (!cw_wait(&bar_full[s], use & 1, s_abort, p.status)) { ok = false; break; }
       if (p.flags & GDN_QK_L2NORM) {
@@ -384,27 +478,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_phase ^= 1;
       tc_fence_after();
       {
-        // A (rows 0-63, fp32, for the solve) and P (rows 64-127 -> bf16 operand),
-        // 32 columns of G at a time
+        // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32, for the solve) and
+        // P = tril(D o Q K^T) (rows 64-127, bf16 operand), 32 columns of G at a time
+        const int i = tid & 63;
+        const float gi = G.g[i], bi = G.b[i];
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           float gr[32];
           tmem_ld32(tmem + lane_off + COL_G + half * 32, gr);
           if (tid < C) {
-            const int i = tid;
-            const float gi = s_g[i], bi = s_b[i];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int jj = half * 32 + e;
-              s_A[i * A_LD + jj] = (jj < i) ? bi * expf(gi - s_g[jj]) * gr[e] : 0.f;
+              s_A[i * A_LD + jj] = (jj < i) ? bi * __expf(gi - G.g[jj]) * gr[e] : 0.f;
             }
           } else {
-            const int i = tid - C;
-            const float gi = s_g[i];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int jj = half * 32 + e;
-              gr[e] = (jj <= i) ? expf(gi - s_g[jj]) * gr[e] : 0.f;
+              gr[e] = (jj <= i) ? __expf(gi - G.g[jj]) * gr[e] : 0.f;
             }
             store_row32_bf16(sm + OFF_P, i, half * 32, gr);
           }
@@ -413,20 +505,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       cw_sync();
 
-      // ---- T = (I + A)^{-1} (blocked, scratch in the U^T tiles, which are free here),
-      // then T1 = T diag(b gamma) and T2 = T diag(b) as bf16 operands
+      // ---- T = (I + A)^{-1} (scratch in the U^T tiles, free here), then
+      // T1 = T diag(b gamma) and T2 = T diag(b) as bf16 operands (8 columns per store)
       {
         float* s_T = reinterpret_cast<float*>(sm + OFF_UT);
         float* s_Y = s_T + 64 * A_LD;
         invert_unit_lower_64(s_A, s_T, s_Y, tid);
-        uint8_t* t1 = sm + OFF_T1;
-        uint8_t* t2 = sm + OFF_T2;
-        for (int e = tid; e < C * C; e += CW) {
-          const int i = e >> 6, jc = e & 63;
-          const float t = ((jc >> 4) > (i >> 4)) ? 0.f : s_T[i * A_LD + jc];
-          const float bj = s_b[jc];
-          *reinterpret_cast<__nv_bfloat16*>(t1 + sw128_offset(i, jc)) = __float2bfloat16_rn(t * bj * s_gamma[jc]);
-          *reinterpret_cast<__nv_bfloat16*>(t2 + sw128_offset(i, jc)) = __float2bfloat16_rn(t * bj);
+#pragma unroll 1
+        for (int it = tid; it < C * 8; it += CW) {
+          const int i = it >> 3, q8 = (it & 7) * 8;
+          const bool zero = ((q8 >> 4) > (i >> 4));
+          float t1v[8], t2v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float t = zero ? 0.f : s_T[i * A_LD + q8 + e];
+            t1v[e] = t * G.bg[q8 + e];
+            t2v[e] = t * G.b[q8 + e];
+          }
+          uint4 o1, o2;
+          o1.x = pack_bf16x2(t1v[0], t1v[1]); o1.y = pack_bf16x2(t1v[2], t1v[3]);
+          o1.z = pack_bf16x2(t1v[4], t1v[5]); o1.w = pack_bf16x2(t1v[6], t1v[7]);
+          o2.x = pack_bf16x2(t2v[0], t2v[1]); o2.y = pack_bf16x2(t2v[2], t2v[3]);
+          o2.z = pack_bf16x2(t2v[4], t2v[5]); o2.w = pack_bf16x2(t2v[6], t2v[7]);
+          *reinterpret_cast<uint4*>(sm + OFF_T1 + sw128_offset(i, q8)) = o1;
+          *reinterpret_cast<uint4*>(sm + OFF_T2 + sw128_offset(i, q8)) = o2;
         }
       }
       fence_proxy_async_smem();
@@ -448,17 +550,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_phase ^= 1;
       tc_fence_after();
       {
-        // W^T row d = tid -> column d of W ([64 tok][128 dk] tile, 2 slabs), 32 tokens at a time
-        uint8_t* slab = sm + OFF_W + (tid >> 6) * 8192;
-        const int dcol = tid & 63;
+        // W^T row d = tid -> row d of the W^T operand tile ([128 dk][64 tok], MN-major B)
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           float wr[32];
           tmem_ld32(tmem + lane_off + COL_W + half * 32, wr);
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            *reinterpret_cast<__nv_bfloat16*>(slab + sw128_offset(half * 32 + e, dcol)) =
-                __float2bfloat16_rn(wr[e]);
+          store_row32_bf16(sm + OFF_WT, tid, half * 32, wr);
         }
       }
       tc_fence_before();
@@ -471,8 +568,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint64_t a_sig = kdesc(sbase + OFF_SIG + (kk >> 2) * 16384 + (kk & 3) * 32);
-          mma_bf16(tmem + COL_U, a_sig, kdesc(sbase + OFF_W + (kk >> 2) * 8192 + (kk & 3) * 32),
-                   idesc_bf16(128, 64, 0, 0, /*neg_b=*/1), 1);
+          mma_bf16(tmem + COL_U, a_sig, mndesc(sbase + OFF_WT + kk * 2048, 8192),
+                   idesc_bf16(128, 64, 0, 1, /*neg_b=*/1), 1);
           mma_bf16(tmem + COL_OA, a_sig,
                    kdesc(kq_a + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32),
                    idesc_bf16(128, 64, 0, 0), kk > 0);
@@ -482,7 +579,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
       mma_phase ^= 1;
       tc_fence_after();
-      const float gC = s_gamma[C - 1];
       {
         // U^T row j (dv) over 64 tokens -> operand tiles U^T and U^T diag(gamma_C / gamma)
 #pragma unroll 1
@@ -491,19 +587,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(tmem + lane_off + COL_U + half * 32, ur);
           store_row32_bf16(sm + OFF_UT, j, half * 32, ur);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ur[e] *= gC / s_gamma[half * 32 + e];
+          for (int e = 0; e < 32; ++e) ur[e] *= G.r[half * 32 + e];
           store_row32_bf16(sm + OFF_UTP, j, half * 32, ur);
         }
-        // decay the fp32 master state in place: Sigma^T <- gamma_C Sigma^T
-#pragma unroll 1
-        for (int piece = 0; piece < 4; ++piece) {
-          float x[32];
-          tmem_ld32(tmem + lane_off + COL_S + piece * 32, x);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] *= gC;
-          tmem_st32(tmem + lane_off + COL_S + piece * 32, x);
-        }
-        tmem_wait_st();
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -521,13 +607,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         mma_commit(bar_mma);
       }
+      // gates of the next chunk (global loads and exponentials) while the MMAs run
+      const bool last = (c == n_chunks - 1);
+      if (!last) {
+        const int ntok0 = tok0 + C;
+        compute_gates(p, gates_at(sm, (c + 1) & 1), s_carry, ntok0, min(C, seq_end - ntok0), h, tid);
+      }
       if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
       mma_phase ^= 1;
       tc_fence_after();
       if (tid == 0) mbar_arrive(&bar_empty[s]);   // every read of stage s has completed
 
-      // ---- outputs: o[tok0 + i][h][col0 + j] = scale (gamma_i O_A + O_B)
+      // ---- next chunk's Sigma^T operand (bf16) and pre-decayed fp32 state; S_T at the end
+      refresh_state(tmem + lane_off + COL_S, sm + OFF_SIG, j,
+                    last ? 1.f : gates_at(sm, (c + 1) & 1).gamma[C - 1], !last,
+                    (last && p.S_T) ? p.S_T + state_base : nullptr, dv);
+
+      // ---- outputs: o[tok0 + i][h][col0 + j] = scale (gamma_i O_A + O_B), staged
+      // through shared memory ([64 tok][128 dv] bf16) for 16-byte coalesced stores
       {
+        uint8_t* stage = sm + OFF_UTP;
         float oa[32], ob[32];
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
@@ -536,42 +635,28 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int i = half * 32 + e;
-            if (i < valid) {
-              const float val = p.scale * fmaf(s_gamma[i], oa[e], ob[e]);
-              p.o[((size_t)(tok0 + i) * H + h) * dv + col0 + j] = __float2bfloat16_rn(val);
-            }
+            *reinterpret_cast<__nv_bfloat16*>(stage + i * 256 + j * 2) =
+                __float2bfloat16_rn(p.scale * fmaf(G.gamma[i], oa[e], ob[e]));
           }
         }
       }
-      // ---- next chunk's Sigma^T operand (bf16) and, at the end, S_T (fp32)
-      const bool last = (c == n_chunks - 1);
-#pragma unroll 1
-      for (int piece = 0; piece < 4; ++piece) {
-        float x[32];
-        tmem_ld32(tmem + lane_off + COL_S + piece * 32, x);
-        uint8_t* slab = sm + OFF_SIG + (piece >> 1) * 16384;
+      tc_fence_before();
+      cw_sync();
+      {
+        const uint8_t* stage = sm + OFF_UTP;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint4 o;
-          o.x = pack_bf16x2(x[cc * 8 + 0], x[cc * 8 + 1]);
-          o.y = pack_bf16x2(x[cc * 8 + 2], x[cc * 8 + 3]);
-          o.z = pack_bf16x2(x[cc * 8 + 4], x[cc * 8 + 5]);
-          o.w = pack_bf16x2(x[cc * 8 + 6], x[cc * 8 + 7]);
-          *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + cc * 8)) = o;
-        }
-        if (last && p.S_T) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) p.S_T[state_base + (size_t)(piece * 32 + e) * dv] = x[e];
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const int it = tid + k8 * CW;
+          const int i = it >> 4, q = it & 15;
+          if (i < valid) {
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
+            __nv_bfloat16* dst = p.o + ((size_t)(tok0 + i) * H + h) * dv + col0 + q * 8;
+            __stcs(reinterpret_cast<uint4*>(dst), v);
+          }
         }
       }
       fence_proxy_async_smem();
-      tc_fence_before();
       cw_sync();
-    }
-    if (n_chunks == 0 && p.S_T) {
-      // empty sequence: S_T = S0 (or zero)
-      for (int d = 0; d < DK; ++d)
-        p.S_T[state_base + (size_t)d * dv] = p.S0 ? p.S0[state_base + (size_t)d * dv] : 0.f;
     }
   }
 

@@ -16,7 +16,13 @@
 // Sigma_t = a_t Sigma_{t-1} + k_t u_t^T, and the three lines above follow by
 // unrolling that inside the chunk.
 //
-// Data path (one CTA per (sequence, head, 128-wide slice of dv)):
+// Data path (one CTA per (sequence, head, 128-wide slice of dv); three roles:
+// a prep warpgroup builds the state-independent operands of chunk c+1 -- gates,
+// G, A, P, T, T1, T2, U~, W^T -- while a state warpgroup runs chunk c -- the
+// Sigma-dependent MMAs, the U^T operands, the state refresh and the outputs --
+// and a producer warp streams K, Q (2 stages) and V (1 stage) in by TMA.  Each
+// warpgroup issues its own MMAs; the hand-offs are mbarriers indexed by buffer
+// slot, so no waiter can fall two phases behind):
 //   * every product is issued TRANSPOSED so its M dimension is 128 (dv rows of
 //     Sigma^T, dk rows of W^T, or the stacked [K; Q] rows) and lands in tensor
 //     memory with lane = row: G = [K;Q] K^T, U^T = V^T T2^T - Sigma^T W^T,
@@ -44,41 +50,61 @@ namespace tc {
 constexpr int C = 64;            // chunk length
 constexpr int DK = 128;          // key/query width (this kernel)
 constexpr int DVS = 128;         // dv slice per CTA
-constexpr int STAGES = 2;
-constexpr int CW = 128;          // compute warpgroup: warps 0-3 (tensor-memory lanes 0-127)
-constexpr int THREADS = CW + 32; // + producer warp 4
+constexpr int WG = 128;          // one warpgroup (tensor-memory lanes 0-127)
+// warps 0-3: prep warpgroup (state-independent part of chunk c+1)
+// warps 4-7: state warpgroup (state-dependent part of chunk c)
+// warp 8   : TMA producer
+constexpr int THREADS = 2 * WG + 32;
+constexpr int BAR_PREP = 1;      // named barriers of the two warpgroups
+constexpr int BAR_STATE = 2;
 
 // tensor-memory columns (fp32 accumulators, lane = row)
-constexpr uint32_t COL_G = 0;     // [K;Q] K^T      128 x 64
-constexpr uint32_t COL_W = 64;    // W^T            128 x 64
-constexpr uint32_t COL_U = 128;   // U^T            128 x 64
-constexpr uint32_t COL_OA = 192;  // Sigma^T Q^T    128 x 64
-constexpr uint32_t COL_OB = 256;  // U^T P^T        128 x 64
-constexpr uint32_t COL_S = 384;   // Sigma^T fp32   128 x 128 (kept pre-decayed by gamma_C)
+constexpr uint32_t COL_GW = 0;    // [K;Q] K^T, then W^T, of the prep chunk    128 x 64
+constexpr uint32_t COL_U = 64;    // U^T, two buffers (chunk parity)           2 x 128 x 64
+constexpr uint32_t COL_OA = 192;  // Sigma^T Q^T                                128 x 64
+constexpr uint32_t COL_OB = 256;  // U^T P^T                                    128 x 64
+constexpr uint32_t COL_S = 384;   // Sigma^T fp32 (kept pre-decayed by gamma_C) 128 x 128
 constexpr uint32_t TMEM_COLS = 512;
 
 // Shared-memory plan (offsets from a 1024-byte aligned base).
-constexpr uint32_t OFF_KQ = 0;                          // STAGES x 32 KB: [K0|Q0|K1|Q1] 8 KB slabs
+constexpr uint32_t OFF_KQ = 0;            // 2 stages x 32 KB: [K0|Q0|K1|Q1] 8 KB slabs
 constexpr uint32_t KQ_BYTES = 32768;
-constexpr uint32_t OFF_V = OFF_KQ + STAGES * KQ_BYTES;  // STAGES x 16 KB: [V0|V1]
+constexpr uint32_t OFF_V = 65536;         // 1 stage x 16 KB: [V0|V1]
 constexpr uint32_t V_BYTES = 16384;
-constexpr uint32_t OFF_SIG = OFF_V + STAGES * V_BYTES;  // Sigma^T bf16 [128 dv][128 dk], 2 x 16 KB slabs
-constexpr uint32_t OFF_WT = OFF_SIG + 32768;            // W^T bf16 [128 dk][64 tok] (MN-major B operand)
-constexpr uint32_t OFF_UT = OFF_WT + 16384;             // U^T bf16 [128 dv][64 tok]; solve scratch
-constexpr uint32_t OFF_UTP = OFF_UT + 16384;            // U^T diag(gamma_C/gamma) bf16; output staging
-constexpr uint32_t OFF_P = OFF_UTP + 16384;             // P bf16 [64][64]
-constexpr uint32_t OFF_T1 = OFF_P + 8192;               // T diag(b gamma) bf16 [64][64]
-constexpr uint32_t OFF_T2 = OFF_T1 + 8192;              // T diag(b) bf16 [64][64]
-constexpr uint32_t OFF_A = OFF_T2 + 8192;               // A fp32 [64][65] (padded rows)
+constexpr uint32_t OFF_SIG = 81920;       // Sigma^T bf16 [128 dv][128 dk], 2 x 16 KB slabs
+constexpr uint32_t OFF_WT = 114688;       // W^T bf16 [128 dk][64 tok] (MN-major B operand)
+constexpr uint32_t OFF_UT = 131072;       // U^T bf16 [128 dv][64 tok]
+constexpr uint32_t OFF_UTP = 147456;      // U^T diag(gamma_C/gamma) bf16; output staging
+constexpr uint32_t OFF_P = 163840;        // P bf16 [64][64], two buffers (chunk parity)
+constexpr uint32_t OFF_T1 = 180224;       // T diag(b gamma) bf16 [64][64] (T fp32 scratch overlays T1|T2)
+constexpr uint32_t OFF_T2 = 188416;       // T diag(b) bf16 [64][64]
+constexpr uint32_t OFF_A = 196608;        // A fp32 [64][65] (padded rows)
 constexpr int A_LD = 65;
-constexpr uint32_t OFF_GATE = OFF_A + 64 * A_LD * 4;    // 2 buffers x {g, gamma, b, b*gamma, gamma_C/gamma}
+constexpr int T_LD = 64;
+constexpr uint32_t OFF_Y = OFF_A + 64 * A_LD * 4;     // solve scratch 48 x 17 fp32
+constexpr uint32_t OFF_GATE = OFF_Y + 48 * 17 * 4;    // 3 buffers x {g, gamma, b, b*gamma, gamma_C/gamma}
 constexpr uint32_t GATE_BYTES = 5 * 64 * 4;
-constexpr uint32_t OFF_BAR = OFF_GATE + 2 * GATE_BYTES; // mbarriers
-constexpr uint32_t OFF_MISC = OFF_BAR + 64;             // tmem base, abort, scan carry
+constexpr uint32_t OFF_BAR = OFF_GATE + 3 * GATE_BYTES;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;          // tmem base, abort flag, scan carry
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;       // + alignment slack
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
-static_assert(64 * A_LD * 4 + 48 * 17 * 4 <= 32768, "solve scratch exceeds the U^T tiles");
+static_assert(OFF_T1 + 64 * T_LD * 4 <= OFF_A, "T scratch must fit over T1|T2");
+
+// mbarriers (index into the barrier array)
+enum : int {
+  B_KQ_FULL = 0,      // [2] TMA K, Q landed
+  B_KQ_EMPTY = 2,     // [2] state: last read of the K, Q stage done (carry MMA)
+  B_V_FULL = 4,       //     TMA V landed
+  B_V_EMPTY = 5,      //     prep: U~ MMA done, V stage free
+  B_GATES = 6,        // [3] prep: gate vectors of a chunk written
+  B_W_READY = 9,      //     prep: W^T tile written, U~ in tensor memory
+  B_W_CONSUMED = 10,  //     state: U MMA done, W^T tile free
+  B_CHUNK_DONE = 11,  // [2] state: chunk finished (U and P buffers free)
+  B_PREP_MMA = 13,    //     commits of the prep warpgroup
+  B_STATE_MMA = 14,   //     commits of the state warpgroup
+  NBAR = 15
+};
 
 struct Params {
   const float* a;
@@ -107,11 +133,22 @@ __device__ __forceinline__ Gates gates_at(uint8_t* sm, int buf) {
   return Gates{base, base + 64, base + 128, base + 192, base + 256};
 }
 
-// Named barrier of the four compute warps (the warp is reconverged first: the
-// barrier is warp-aligned and the bounded waits exit lane by lane).
-__device__ __forceinline__ void cw_sync() {
+// Named barrier of one warpgroup (the warp is reconverged first: the barrier is
+// warp-aligned and the bounded waits exit lane by lane).
+template <int ID>
+__device__ __forceinline__ void wg_sync() {
   __syncwarp();
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync %0, 128;" ::"n"(ID) : "memory");
+}
+
+// All threads of a warpgroup wait on `bar`; the outcome is made uniform through
+// the abort flag so that no thread leaves the schedule alone.
+template <int ID>
+__device__ __forceinline__ bool wg_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                        unsigned* status) {
+  mbar_wait_bounded(bar, parity, abort, status);
+  wg_sync<ID>();
+  return *abort == 0;
 }
 
 // K-major, 128-byte swizzled operand: rows of 128 bytes, 8-row groups 1024 B apart.
@@ -120,15 +157,6 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return smem_desc(sad
 // rows along K 128 B apart (8-row atoms 1024 B apart), next 64 MN elements `lbo` bytes on.
 __device__ __forceinline__ uint64_t mndesc(uint32_t saddr, uint32_t lbo) {
   return smem_desc(saddr, lbo, 1024);
-}
-
-// All compute-warpgroup threads wait on `bar`; the outcome is made uniform
-// through the abort flag so that no thread leaves the schedule alone.
-__device__ __forceinline__ bool cw_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                        unsigned* status) {
-  mbar_wait_bounded(bar, parity, abort, status);
-  cw_sync();
-  return *abort == 0;
 }
 
 // Normalise one 128-element bf16 row of a [K0|Q0|K1|Q1] stage tile in place:
@@ -175,16 +203,16 @@ __device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int row, int col
   }
 }
 
-// Gate vectors of one chunk (all 128 compute threads call this; threads 0-63
-// own one token each).  Rows past the sequence end get log a = 0 and b = 0.
+// Gate vectors of one chunk (all 128 prep threads call this; threads 0-63 own
+// one token each).  Rows past the sequence end get log a = 0 and b = 0.
 __device__ __forceinline__ void compute_gates(const Params& p, Gates G, float* s_carry, int tok0,
-                                              int valid, int h, int tid) {
-  const int lane = tid & 31;
+                                              int valid, int h, int t) {
+  const int lane = t & 31;
   float la = 0.f;
-  if (tid < C) {
+  if (t < C) {
     float bb = 0.f;
-    if (tid < valid) {
-      const size_t ti = (size_t)(tok0 + tid) * p.H + h;
+    if (t < valid) {
+      const size_t ti = (size_t)(tok0 + t) * p.H + h;
       la = logf(__ldg(p.a + ti));
       bb = __ldg(p.b + ti);
     }
@@ -193,21 +221,21 @@ __device__ __forceinline__ void compute_gates(const Params& p, Gates G, float* s
       const float y = __shfl_up_sync(0xffffffffu, la, off);
       if (lane >= off) la += y;
     }
-    if (tid == 31) *s_carry = la;
-    G.b[tid] = bb;
+    if (t == 31) *s_carry = la;
+    G.b[t] = bb;
   }
-  cw_sync();
-  if (tid < C) {
-    if (tid >= 32) la += *s_carry;
-    G.g[tid] = la;
+  wg_sync<BAR_PREP>();
+  if (t < C) {
+    if (t >= 32) la += *s_carry;
+    G.g[t] = la;
   }
-  cw_sync();
-  if (tid < C) {
+  wg_sync<BAR_PREP>();
+  if (t < C) {
     const float gC = G.g[C - 1];
     const float gam = __expf(la);
-    G.gamma[tid] = gam;
-    G.bg[tid] = G.b[tid] * gam;
-    G.r[tid] = __expf(gC - la);
+    G.gamma[t] = gam;
+    G.bg[t] = G.b[t] * gam;
+    G.r[t] = __expf(gC - la);
   }
 }
 
@@ -215,30 +243,30 @@ __device__ __forceinline__ void compute_gates(const Params& p, Gates G, float* s
 // A_LD), blocked by 16.  The diagonal blocks are inverted by forward
 // substitution (one column per thread); the off-diagonal blocks follow by
 // block distance D: T_{b+D,b} = -T_{b+D,b+D} sum_{m=b}^{b+D-1} A_{b+D,m} T_{m,b}.
-// s_T receives T (its upper block triangle is left unset); s_Y is 3 x 16 x 17
-// fp32 scratch.  Every compute thread takes part (the barriers are inside).
+// s_T receives T (row stride T_LD; its upper block triangle is left unset);
+// s_Y is 3 x 16 x 17 fp32 scratch.  All prep threads take part.
 template <int D>
-__device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, float* s_Y, int tid) {
+__device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, float* s_Y, int t) {
   constexpr int NB = 4 - D;
   constexpr int ITEMS = NB * 128;   // (block, row, column pair c / c+8)
-  for (int it = tid; it < ITEMS; it += CW) {
+  for (int it = t; it < ITEMS; it += WG) {
     const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
     const float* arow = s_A + ((bb + D) * 16 + r) * A_LD + bb * 16;
-    const float* tcol = s_T + (bb * 16) * A_LD + bb * 16 + c;
+    const float* tcol = s_T + (bb * 16) * T_LD + bb * 16 + c;
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
     for (int k = 0; k < 16 * D; ++k) {
       const float av = arow[k];
-      y0 = fmaf(av, tcol[k * A_LD], y0);
-      y1 = fmaf(av, tcol[k * A_LD + 8], y1);
+      y0 = fmaf(av, tcol[k * T_LD], y0);
+      y1 = fmaf(av, tcol[k * T_LD + 8], y1);
     }
     s_Y[(bb * 16 + r) * 17 + c] = y0;
     s_Y[(bb * 16 + r) * 17 + c + 8] = y1;
   }
-  cw_sync();
-  for (int it = tid; it < ITEMS; it += CW) {
+  wg_sync<BAR_PREP>();
+  for (int it = t; it < ITEMS; it += WG) {
     const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
-    const float* trow = s_T + ((bb + D) * 16 + r) * A_LD + (bb + D) * 16;
+    const float* trow = s_T + ((bb + D) * 16 + r) * T_LD + (bb + D) * 16;
     const float* ycol = s_Y + (bb * 16) * 17 + c;
     float t0 = 0.f, t1 = 0.f;
 #pragma unroll
@@ -247,15 +275,15 @@ __device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, floa
       t0 = fmaf(tv, ycol[k * 17], t0);
       t1 = fmaf(tv, ycol[k * 17 + 8], t1);
     }
-    s_T[((bb + D) * 16 + r) * A_LD + bb * 16 + c] = -t0;
-    s_T[((bb + D) * 16 + r) * A_LD + bb * 16 + c + 8] = -t1;
+    s_T[((bb + D) * 16 + r) * T_LD + bb * 16 + c] = -t0;
+    s_T[((bb + D) * 16 + r) * T_LD + bb * 16 + c + 8] = -t1;
   }
-  cw_sync();
+  wg_sync<BAR_PREP>();
 }
 
-__device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_T, float* s_Y, int tid) {
-  if (tid < 64) {
-    const int r0 = (tid >> 4) * 16, c = tid & 15;
+__device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_T, float* s_Y, int t) {
+  if (t < 64) {
+    const int r0 = (t >> 4) * 16, c = t & 15;
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -265,12 +293,12 @@ __device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_
       x[i] = acc;
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s_T[(r0 + i) * A_LD + r0 + c] = x[i];
+    for (int i = 0; i < 16; ++i) s_T[(r0 + i) * T_LD + r0 + c] = x[i];
   }
-  cw_sync();
-  offdiag_level<1>(s_A, s_T, s_Y, tid);
-  offdiag_level<2>(s_A, s_T, s_Y, tid);
-  offdiag_level<3>(s_A, s_T, s_Y, tid);
+  wg_sync<BAR_PREP>();
+  offdiag_level<1>(s_A, s_T, s_Y, t);
+  offdiag_level<2>(s_A, s_T, s_Y, t);
+  offdiag_level<3>(s_A, s_T, s_Y, t);
 }
 
 // Sigma^T row j (fp32, in tensor memory) -> bf16 operand tile for the next
@@ -306,20 +334,17 @@ __device__ __forceinline__ void refresh_state(uint32_t taddr, uint8_t* sig, int 
   tmem_wait_st();
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __maxnreg__(224)
     gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* bar_empty = bar_full + STAGES;
-  uint64_t* bar_mma = bar_empty + STAGES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
   float* s_carry = reinterpret_cast<float*>(sm + OFF_MISC + 8);
-  float* s_A = reinterpret_cast<float*>(sm + OFF_A);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -342,7 +367,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // offsets outside [0, total_tokens] or decreasing: clamp, and report
     const int s0 = min(max(seq_start, 0), p.total_tokens);
     const int s1 = min(max(seq_end, s0), p.total_tokens);
-    if ((s0 != seq_start || s1 != seq_end) && threadIdx.x == 0) record_status(p.status, GDN_ERR_INVALID);
+    if ((s0 != seq_start || s1 != seq_end) && tid == 0) record_status(p.status, GDN_ERR_INVALID);
     seq_start = s0;
     seq_end = s1;
   }
@@ -352,11 +377,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int col0 = slice * DVS;
 
   if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_empty[s], 1);
-    }
-    mbar_init(bar_mma, 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -364,7 +385,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(s_tmem, TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -374,45 +395,194 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  const uint32_t sbase = smem_u32(sm);
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  if (warp == 8) {
+    // ================================================================ producer
     if (lane == 0) {
-      int issued0 = 0, issued1 = 0;
+      int kq_issued0 = 0, kq_issued1 = 0, v_issued = 0;
       for (int c = 0; c < n_chunks; ++c) {
-        const int s = c % STAGES;
-        const int use = c / STAGES;
-        if (use > 0 && !mbar_wait_bounded(&bar_empty[s], (use - 1) & 1, s_abort, p.status)) break;
-        uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
-        uint8_t* vv = sm + OFF_V + s * V_BYTES;
+        const int s = c & 1;
         const int tok0 = seq_start + c * C;
-        mbar_arrive_expect_tx(&bar_full[s], KQ_BYTES + V_BYTES);
-        tma_load_3d(kq + 0, &tm_k, &bar_full[s], 0, h, tok0);
-        tma_load_3d(kq + 16384, &tm_k, &bar_full[s], 64, h, tok0);
-        tma_load_3d(kq + 8192, &tm_q, &bar_full[s], 0, h, tok0);
-        tma_load_3d(kq + 24576, &tm_q, &bar_full[s], 64, h, tok0);
-        tma_load_3d(vv + 0, &tm_v, &bar_full[s], col0, h, tok0);
-        tma_load_3d(vv + 8192, &tm_v, &bar_full[s], col0 + 64, h, tok0);
-        if (s == 0) issued0 = use + 1; else issued1 = use + 1;
+        if (c >= 2 &&
+            !mbar_wait_bounded(&bars[B_KQ_EMPTY + s], ((c >> 1) - 1) & 1, s_abort, p.status))
+          break;
+        uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
+        mbar_arrive_expect_tx(&bars[B_KQ_FULL + s], KQ_BYTES);
+        tma_load_3d(kq + 0, &tm_k, &bars[B_KQ_FULL + s], 0, h, tok0);
+        tma_load_3d(kq + 16384, &tm_k, &bars[B_KQ_FULL + s], 64, h, tok0);
+        tma_load_3d(kq + 8192, &tm_q, &bars[B_KQ_FULL + s], 0, h, tok0);
+        tma_load_3d(kq + 24576, &tm_q, &bars[B_KQ_FULL + s], 64, h, tok0);
+        if (s == 0) kq_issued0 = (c >> 1) + 1; else kq_issued1 = (c >> 1) + 1;
+        if (c >= 1 && !mbar_wait_bounded(&bars[B_V_EMPTY], (c - 1) & 1, s_abort, p.status)) break;
+        mbar_arrive_expect_tx(&bars[B_V_FULL], V_BYTES);
+        tma_load_3d(sm + OFF_V, &tm_v, &bars[B_V_FULL], col0, h, tok0);
+        tma_load_3d(sm + OFF_V + 8192, &tm_v, &bars[B_V_FULL], col0 + 64, h, tok0);
+        v_issued = c + 1;
       }
       // never leave the block with bulk copies still landing in its shared memory
-      if (issued0 > 0) mbar_wait_bounded(&bar_full[0], (issued0 - 1) & 1, nullptr, p.status);
-      if (issued1 > 0) mbar_wait_bounded(&bar_full[1], (issued1 - 1) & 1, nullptr, p.status);
+      if (kq_issued0 > 0) mbar_wait_bounded(&bars[B_KQ_FULL], (kq_issued0 - 1) & 1, nullptr, p.status);
+      if (kq_issued1 > 0) mbar_wait_bounded(&bars[B_KQ_FULL + 1], (kq_issued1 - 1) & 1, nullptr, p.status);
+      if (v_issued > 0) mbar_wait_bounded(&bars[B_V_FULL], (v_issued - 1) & 1, nullptr, p.status);
+    }
+  } else if (warp < 4) {
+    // ================================================================ prep warpgroup
+    const int t = tid;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    float* s_A = reinterpret_cast<float*>(sm + OFF_A);
+    float* s_T = reinterpret_cast<float*>(sm + OFF_T1);
+    float* s_Y = reinterpret_cast<float*>(sm + OFF_Y);
+    uint32_t pphase = 0;
+#pragma unroll 1
+    for (int c = 0; c < n_chunks; ++c) {
+      const int s = c & 1;
+      const int tok0 = seq_start + c * C;
+      const int valid = min(C, seq_end - tok0);
+      const Gates G = gates_at(sm, c % 3);
+      uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
+      const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
+
+      // ---- gates of chunk c (the buffer's previous user, chunk c-3, is finished)
+      compute_gates(p, G, s_carry, tok0, valid, h, t);
+      wg_sync<BAR_PREP>();
+      if (t == 0) mbar_arrive(&bars[B_GATES + c % 3]);
+
+      // ---- K, Q of chunk c; optional in-place L2 norm
+      if (!wg_wait<BAR_PREP>(&bars[B_KQ_FULL + s], (c >> 1) & 1, s_abort, p.status)) break;
+      if (p.flags & GDN_QK_L2NORM) {
+        l2norm_row(kq, t & 63, t < 64 ? 0u : 8192u);   // rows 0-63: K, rows 64-127: Q
+        fence_proxy_async_smem();
+        wg_sync<BAR_PREP>();
+      }
+
+      // ---- G = [K; Q] K^T   (M = 128, N = 64, K = dk)
+      if (t == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16(tmem + COL_GW, kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
+                   kk > 0);
+        }
+        mma_commit(&bars[B_PREP_MMA]);
+      }
+      if (!wg_wait<BAR_PREP>(&bars[B_PREP_MMA], pphase, s_abort, p.status)) break;
+      pphase ^= 1;
+      tc_fence_after();
+
+      // ---- P buffer s and U buffer s are free once chunk c-2 is finished
+      if (c >= 2 &&
+          !wg_wait<BAR_PREP>(&bars[B_CHUNK_DONE + s], ((c >> 1) - 1) & 1, s_abort, p.status))
+        break;
+      {
+        // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32) and
+        // P = tril(D o Q K^T) (rows 64-127, bf16 operand), 32 columns of G at a time
+        const int i = t & 63;
+        const float gi = G.g[i], bi = G.b[i];
+        uint8_t* pt = sm + OFF_P + s * 8192;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float gr[32];
+          tmem_ld32(tmem + lane_off + COL_GW + half * 32, gr);
+          if (t < C) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int jj = half * 32 + e;
+              s_A[i * A_LD + jj] = (jj < i) ? bi * __expf(gi - G.g[jj]) * gr[e] : 0.f;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int jj = half * 32 + e;
+              gr[e] = (jj <= i) ? __expf(gi - G.g[jj]) * gr[e] : 0.f;
+            }
+            store_row32_bf16(pt, i, half * 32, gr);
+          }
+        }
+      }
+      tc_fence_before();
+      wg_sync<BAR_PREP>();
+
+      // ---- T = (I + A)^{-1}, then T1 = T diag(b gamma), T2 = T diag(b) (bf16, over the T scratch)
+      invert_unit_lower_64(s_A, s_T, s_Y, t);
+      {
+        float tv[4][8];
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int it = t + k4 * WG;
+          const int i = it >> 3, q8 = (it & 7) * 8;
+          const bool zero = ((q8 >> 4) > (i >> 4));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) tv[k4][e] = zero ? 0.f : s_T[i * T_LD + q8 + e];
+        }
+        wg_sync<BAR_PREP>();
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int it = t + k4 * WG;
+          const int i = it >> 3, q8 = (it & 7) * 8;
+          uint4 o1, o2;
+          o1.x = pack_bf16x2(tv[k4][0] * G.bg[q8 + 0], tv[k4][1] * G.bg[q8 + 1]);
+          o1.y = pack_bf16x2(tv[k4][2] * G.bg[q8 + 2], tv[k4][3] * G.bg[q8 + 3]);
+          o1.z = pack_bf16x2(tv[k4][4] * G.bg[q8 + 4], tv[k4][5] * G.bg[q8 + 5]);
+          o1.w = pack_bf16x2(tv[k4][6] * G.bg[q8 + 6], tv[k4][7] * G.bg[q8 + 7]);
+          o2.x = pack_bf16x2(tv[k4][0] * G.b[q8 + 0], tv[k4][1] * G.b[q8 + 1]);
+          o2.y = pack_bf16x2(tv[k4][2] * G.b[q8 + 2], tv[k4][3] * G.b[q8 + 3]);
+          o2.z = pack_bf16x2(tv[k4][4] * G.b[q8 + 4], tv[k4][5] * G.b[q8 + 5]);
+          o2.w = pack_bf16x2(tv[k4][6] * G.b[q8 + 6], tv[k4][7] * G.b[q8 + 7]);
+          *reinterpret_cast<uint4*>(sm + OFF_T1 + sw128_offset(i, q8)) = o1;
+          *reinterpret_cast<uint4*>(sm + OFF_T2 + sw128_offset(i, q8)) = o2;
+        }
+      }
+      fence_proxy_async_smem();
+      wg_sync<BAR_PREP>();
+
+      // ---- U~^T = V^T T2^T (into U buffer s) and W^T = K^T T1^T (M = 128, N = 64, K = 64 tokens)
+      if (!wg_wait<BAR_PREP>(&bars[B_V_FULL], c & 1, s_abort, p.status)) break;
+      if (t == 0) {
+        tc_fence_after();
+        const uint32_t v_a = sbase + OFF_V;
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          mma_bf16(tmem + COL_U + s * 64, mndesc(v_a + kk * 2048, 8192),
+                   kdesc(sbase + OFF_T2 + kk * 32), idesc_bf16(128, 64, 1, 0), kk > 0);
+          mma_bf16(tmem + COL_GW, mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
+                   idesc_bf16(128, 64, 1, 0), kk > 0);
+        }
+        mma_commit(&bars[B_PREP_MMA]);
+      }
+      if (!wg_wait<BAR_PREP>(&bars[B_PREP_MMA], pphase, s_abort, p.status)) break;
+      pphase ^= 1;
+      tc_fence_after();
+      if (t == 0) mbar_arrive(&bars[B_V_EMPTY]);
+
+      // ---- W^T tile (row d = t): free once the state warpgroup's U MMA of chunk c-1 is done
+      if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        float wr[32];
+        tmem_ld32(tmem + lane_off + COL_GW + half * 32, wr);
+        store_row32_bf16(sm + OFF_WT, t, half * 32, wr);
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      wg_sync<BAR_PREP>();
+      if (t == 0) mbar_arrive(&bars[B_W_READY]);
     }
   } else {
-    // ------------------------------------------------------------ compute warpgroup
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;   // this warp's tensor-memory lanes
-    const int j = tid;                                        // dv row (or dk row) owned
+    // ================================================================ state warpgroup
+    const int j = tid - WG;                                   // dv row owned
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const size_t state_base = ((size_t)seq * H + h) * DK * (size_t)dv + col0 + j;
-    const uint32_t sbase = smem_u32(sm);
-    uint32_t mma_phase = 0;
+    uint32_t sphase = 0;
+    bool ok = true;
 
-    // gates of chunk 0, then the initial state: Sigma^T row j = column (col0 + j)
-    // of S0; tensor memory holds gamma_C(0) * S0, the bf16 operand holds S0.
-    if (n_chunks > 0) compute_gates(p, gates_at(sm, 0), s_carry, seq_start, min(C, len), h, tid);
-    cw_sync();
-    {
-      const float decay0 = (n_chunks > 0) ? gates_at(sm, 0).gamma[C - 1] : 1.f;
+    // initial state: tensor memory holds gamma_C(0) * S0, the bf16 operand holds S0
+    float decay0 = 1.f;
+    if (n_chunks > 0) {
+      ok = wg_wait<BAR_STATE>(&bars[B_GATES + 0], 0, s_abort, p.status);
+      decay0 = gates_at(sm, 0).gamma[C - 1];
+    }
+    if (ok) {
 #pragma unroll 1
       for (int piece = 0; piece < 4; ++piece) {
         float x[32];
@@ -421,13 +591,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           x[e] = p.S0 ? __ldg(p.S0 + state_base + (size_t)(piece * 32 + e) * dv) : 0.f;
         uint8_t* slab = sm + OFF_SIG + (piece >> 1) * 16384;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint4 o;
-          o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
-          o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
-          o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
-          o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
-          *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + c * 8)) = o;
+          o.x = pack_bf16x2(x[cc * 8 + 0], x[cc * 8 + 1]);
+          o.y = pack_bf16x2(x[cc * 8 + 2], x[cc * 8 + 3]);
+          o.z = pack_bf16x2(x[cc * 8 + 4], x[cc * 8 + 5]);
+          o.w = pack_bf16x2(x[cc * 8 + 6], x[cc * 8 + 7]);
+          *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + cc * 8)) = o;
         }
         if (n_chunks == 0 && p.S_T) {
 #pragma unroll
@@ -441,186 +611,74 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    cw_sync();
+    wg_sync<BAR_STATE>();
 
-    bool ok = true;
 #pragma unroll 1
     for (int c = 0; c < n_chunks && ok; ++c) {
-      const int s = c % STAGES;
-      const int use = c / STAGES;
+      const int s = c & 1;
       const int tok0 = seq_start + c * C;
       const int valid = min(C, seq_end - tok0);
-      uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
+      const bool last = (c == n_chunks - 1);
+      const Gates G = gates_at(sm, c % 3);
       const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
-      const uint32_t v_a = sbase + OFF_V + s * V_BYTES;
-      const Gates G = gates_at(sm, c & 1);
 
-      if (!cw_wait(&bar_full[s], use & 1, s_abort, p.status)) { ok = false; break; }
-      if (p.flags & GDN_QK_L2NORM) {
-        // rows 0-63: K (tile offset 0), rows 64-127: Q (tile offset 8192)
-        l2norm_row(kq, tid & 63, tid < 64 ? 0u : 8192u);
-        fence_proxy_async_smem();
-      }
-      cw_sync();
-
-      // ---- G = [K; Q] K^T   (M = 128, N = 64, K = dk)
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + COL_G, kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
-                   kk > 0);
-        }
-        mma_commit(bar_mma);
-      }
-      if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
-      mma_phase ^= 1;
-      tc_fence_after();
-      {
-        // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32, for the solve) and
-        // P = tril(D o Q K^T) (rows 64-127, bf16 operand), 32 columns of G at a time
-        const int i = tid & 63;
-        const float gi = G.g[i], bi = G.b[i];
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float gr[32];
-          tmem_ld32(tmem + lane_off + COL_G + half * 32, gr);
-          if (tid < C) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int jj = half * 32 + e;
-              s_A[i * A_LD + jj] = (jj < i) ? bi * __expf(gi - G.g[jj]) * gr[e] : 0.f;
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int jj = half * 32 + e;
-              gr[e] = (jj <= i) ? __expf(gi - G.g[jj]) * gr[e] : 0.f;
-            }
-            store_row32_bf16(sm + OFF_P, i, half * 32, gr);
-          }
-        }
-      }
-      tc_fence_before();
-      cw_sync();
-
-      // ---- T = (I + A)^{-1} (scratch in the U^T tiles, free here), then
-      // T1 = T diag(b gamma) and T2 = T diag(b) as bf16 operands (8 columns per store)
-      {
-        float* s_T = reinterpret_cast<float*>(sm + OFF_UT);
-        float* s_Y = s_T + 64 * A_LD;
-        invert_unit_lower_64(s_A, s_T, s_Y, tid);
-#pragma unroll 1
-        for (int it = tid; it < C * 8; it += CW) {
-          const int i = it >> 3, q8 = (it & 7) * 8;
-          const bool zero = ((q8 >> 4) > (i >> 4));
-          float t1v[8], t2v[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float t = zero ? 0.f : s_T[i * A_LD + q8 + e];
-            t1v[e] = t * G.bg[q8 + e];
-            t2v[e] = t * G.b[q8 + e];
-          }
-          uint4 o1, o2;
-          o1.x = pack_bf16x2(t1v[0], t1v[1]); o1.y = pack_bf16x2(t1v[2], t1v[3]);
-          o1.z = pack_bf16x2(t1v[4], t1v[5]); o1.w = pack_bf16x2(t1v[6], t1v[7]);
-          o2.x = pack_bf16x2(t2v[0], t2v[1]); o2.y = pack_bf16x2(t2v[2], t2v[3]);
-          o2.z = pack_bf16x2(t2v[4], t2v[5]); o2.w = pack_bf16x2(t2v[6], t2v[7]);
-          *reinterpret_cast<uint4*>(sm + OFF_T1 + sw128_offset(i, q8)) = o1;
-          *reinterpret_cast<uint4*>(sm + OFF_T2 + sw128_offset(i, q8)) = o2;
-        }
-      }
-      fence_proxy_async_smem();
-      cw_sync();
-
-      // ---- U~^T = V^T T2^T  and  W^T = K^T T1^T   (M = 128, N = 64, K = 64 tokens)
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          mma_bf16(tmem + COL_U, mndesc(v_a + kk * 2048, 8192), kdesc(sbase + OFF_T2 + kk * 32),
-                   idesc_bf16(128, 64, 1, 0), kk > 0);
-          mma_bf16(tmem + COL_W, mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
-                   idesc_bf16(128, 64, 1, 0), kk > 0);
-        }
-        mma_commit(bar_mma);
-      }
-      if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
-      mma_phase ^= 1;
-      tc_fence_after();
-      {
-        // W^T row d = tid -> row d of the W^T operand tile ([128 dk][64 tok], MN-major B)
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float wr[32];
-          tmem_ld32(tmem + lane_off + COL_W + half * 32, wr);
-          store_row32_bf16(sm + OFF_WT, tid, half * 32, wr);
-        }
-      }
-      tc_fence_before();
-      fence_proxy_async_smem();
-      cw_sync();
-
-      // ---- U^T -= Sigma^T W^T  and  O_A^T = Sigma^T Q^T   (M = 128, N = 64, K = dk)
-      if (tid == 0) {
+      // ---- U^T -= Sigma^T W^T (onto U~^T in buffer s)  and  O_A^T = Sigma^T Q^T
+      if (!wg_wait<BAR_STATE>(&bars[B_W_READY], c & 1, s_abort, p.status)) break;
+      if (j == 0) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint64_t a_sig = kdesc(sbase + OFF_SIG + (kk >> 2) * 16384 + (kk & 3) * 32);
-          mma_bf16(tmem + COL_U, a_sig, mndesc(sbase + OFF_WT + kk * 2048, 8192),
+          mma_bf16(tmem + COL_U + s * 64, a_sig, mndesc(sbase + OFF_WT + kk * 2048, 8192),
                    idesc_bf16(128, 64, 0, 1, /*neg_b=*/1), 1);
-          mma_bf16(tmem + COL_OA, a_sig,
-                   kdesc(kq_a + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32),
+          mma_bf16(tmem + COL_OA, a_sig, kdesc(kq_a + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32),
                    idesc_bf16(128, 64, 0, 0), kk > 0);
         }
-        mma_commit(bar_mma);
+        mma_commit(&bars[B_STATE_MMA]);
       }
-      if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
-      mma_phase ^= 1;
+      if (!wg_wait<BAR_STATE>(&bars[B_STATE_MMA], sphase, s_abort, p.status)) break;
+      sphase ^= 1;
       tc_fence_after();
-      {
-        // U^T row j (dv) over 64 tokens -> operand tiles U^T and U^T diag(gamma_C / gamma)
+      if (j == 0) mbar_arrive(&bars[B_W_CONSUMED]);
+
+      // ---- U^T row j -> operand tiles U^T and U^T diag(gamma_C / gamma)
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float ur[32];
-          tmem_ld32(tmem + lane_off + COL_U + half * 32, ur);
-          store_row32_bf16(sm + OFF_UT, j, half * 32, ur);
+      for (int half = 0; half < 2; ++half) {
+        float ur[32];
+        tmem_ld32(tmem + lane_off + COL_U + s * 64 + half * 32, ur);
+        store_row32_bf16(sm + OFF_UT, j, half * 32, ur);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ur[e] *= G.r[half * 32 + e];
-          store_row32_bf16(sm + OFF_UTP, j, half * 32, ur);
-        }
+        for (int e = 0; e < 32; ++e) ur[e] *= G.r[half * 32 + e];
+        store_row32_bf16(sm + OFF_UTP, j, half * 32, ur);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      cw_sync();
+      wg_sync<BAR_STATE>();
 
       // ---- O_B^T = U^T P^T (N = 64)  and  Sigma^T += U'^T K (N = dk), K = 64 tokens
-      if (tid == 0) {
+      if (j == 0) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
-          mma_bf16(tmem + COL_OB, kdesc(sbase + OFF_UT + kk * 32), kdesc(sbase + OFF_P + kk * 32),
-                   idesc_bf16(128, 64, 0, 0), kk > 0);
+          mma_bf16(tmem + COL_OB, kdesc(sbase + OFF_UT + kk * 32),
+                   kdesc(sbase + OFF_P + s * 8192 + kk * 32), idesc_bf16(128, 64, 0, 0), kk > 0);
           mma_bf16(tmem + COL_S, kdesc(sbase + OFF_UTP + kk * 32), mndesc(kq_a + kk * 2048, 16384),
                    idesc_bf16(128, 128, 0, 1), 1);
         }
-        mma_commit(bar_mma);
+        mma_commit(&bars[B_STATE_MMA]);
       }
-      // gates of the next chunk (global loads and exponentials) while the MMAs run
-      const bool last = (c == n_chunks - 1);
-      if (!last) {
-        const int ntok0 = tok0 + C;
-        compute_gates(p, gates_at(sm, (c + 1) & 1), s_carry, ntok0, min(C, seq_end - ntok0), h, tid);
-      }
-      if (!cw_wait(bar_mma, mma_phase, s_abort, p.status)) { ok = false; break; }
-      mma_phase ^= 1;
+      if (!wg_wait<BAR_STATE>(&bars[B_STATE_MMA], sphase, s_abort, p.status)) break;
+      sphase ^= 1;
       tc_fence_after();
-      if (tid == 0) mbar_arrive(&bar_empty[s]);   // every read of stage s has completed
+      if (j == 0) mbar_arrive(&bars[B_KQ_EMPTY + s]);   // last read of the K, Q stage is done
 
       // ---- next chunk's Sigma^T operand (bf16) and pre-decayed fp32 state; S_T at the end
-      refresh_state(tmem + lane_off + COL_S, sm + OFF_SIG, j,
-                    last ? 1.f : gates_at(sm, (c + 1) & 1).gamma[C - 1], !last,
+      float decay = 1.f;
+      if (!last) {
+        if (!wg_wait<BAR_STATE>(&bars[B_GATES + (c + 1) % 3], ((c + 1) / 3) & 1, s_abort, p.status)) break;
+        decay = gates_at(sm, (c + 1) % 3).gamma[C - 1];
+      }
+      refresh_state(tmem + lane_off + COL_S, sm + OFF_SIG, j, decay, !last,
                     (last && p.S_T) ? p.S_T + state_base : nullptr, dv);
 
       // ---- outputs: o[tok0 + i][h][col0 + j] = scale (gamma_i O_A + O_B), staged
@@ -641,12 +699,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       tc_fence_before();
-      cw_sync();
+      wg_sync<BAR_STATE>();
       {
         const uint8_t* stage = sm + OFF_UTP;
 #pragma unroll
         for (int k8 = 0; k8 < 8; ++k8) {
-          const int it = tid + k8 * CW;
+          const int it = j + k8 * WG;
           const int i = it >> 4, q = it & 15;
           if (i < valid) {
             const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
@@ -656,7 +714,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       fence_proxy_async_smem();
-      cw_sync();
+      wg_sync<BAR_STATE>();
+      if (j == 0) mbar_arrive(&bars[B_CHUNK_DONE + s]);
     }
   }
 

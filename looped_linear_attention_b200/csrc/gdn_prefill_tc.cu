@@ -51,10 +51,12 @@ constexpr int C = 64;            // chunk length
 constexpr int DK = 128;          // key/query width (this kernel)
 constexpr int DVS = 128;         // dv slice per CTA
 constexpr int WG = 128;          // one warpgroup (tensor-memory lanes 0-127)
-// warps 0-3: prep warpgroup (state-independent part of chunk c+1)
-// warps 4-7: state warpgroup (state-dependent part of chunk c)
-// warp 8   : TMA producer
-constexpr int THREADS = 2 * WG + 32;
+// warps 0-3: prep warpgroup (state-independent part of chunk c+1); its thread 0
+//            also issues the TMA loads of V (one stage)
+// warps 4-7: state warpgroup (state-dependent part of chunk c); its thread 0
+//            also issues the TMA loads of K and Q (two stages)
+// Two warps per SM sub-partition leave room for 224 registers per thread.
+constexpr int THREADS = 2 * WG;
 constexpr int BAR_PREP = 1;      // named barriers of the two warpgroups
 constexpr int BAR_STATE = 2;
 
@@ -94,16 +96,14 @@ static_assert(OFF_T1 + 64 * T_LD * 4 <= OFF_A, "T scratch must fit over T1|T2");
 // mbarriers (index into the barrier array)
 enum : int {
   B_KQ_FULL = 0,      // [2] TMA K, Q landed
-  B_KQ_EMPTY = 2,     // [2] state: last read of the K, Q stage done (carry MMA)
-  B_V_FULL = 4,       //     TMA V landed
-  B_V_EMPTY = 5,      //     prep: U~ MMA done, V stage free
-  B_GATES = 6,        // [3] prep: gate vectors of a chunk written
-  B_W_READY = 9,      //     prep: W^T tile written, U~ in tensor memory
-  B_W_CONSUMED = 10,  //     state: U MMA done, W^T tile free
-  B_CHUNK_DONE = 11,  // [2] state: chunk finished (U and P buffers free)
-  B_PREP_MMA = 13,    //     commits of the prep warpgroup
-  B_STATE_MMA = 14,   //     commits of the state warpgroup
-  NBAR = 15
+  B_V_FULL = 2,       //     TMA V landed
+  B_GATES = 3,        // [3] prep: gate vectors of a chunk written
+  B_W_READY = 6,      //     prep: W^T tile written, U~ in tensor memory
+  B_W_CONSUMED = 7,   //     state: U MMA done, W^T tile free
+  B_CHUNK_DONE = 8,   // [2] state: chunk finished (U and P buffers free)
+  B_PREP_MMA = 10,    //     commits of the prep warpgroup
+  B_STATE_MMA = 11,   //     commits of the state warpgroup
+  NBAR = 12
 };
 
 struct Params {
@@ -334,6 +334,23 @@ __device__ __forceinline__ void refresh_state(uint32_t taddr, uint8_t* sig, int 
   tmem_wait_st();
 }
 
+// TMA loads of one chunk: K and Q into stage s, or the V slice.
+__device__ __forceinline__ void load_kq(uint8_t* sm, uint64_t* bar, const CUtensorMap* tq,
+                                        const CUtensorMap* tk, int s, int h, int tok0) {
+  uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
+  mbar_arrive_expect_tx(bar, KQ_BYTES);
+  tma_load_3d(kq + 0, tk, bar, 0, h, tok0);
+  tma_load_3d(kq + 16384, tk, bar, 64, h, tok0);
+  tma_load_3d(kq + 8192, tq, bar, 0, h, tok0);
+  tma_load_3d(kq + 24576, tq, bar, 64, h, tok0);
+}
+__device__ __forceinline__ void load_v(uint8_t* sm, uint64_t* bar, const CUtensorMap* tv, int col0,
+                                       int h, int tok0) {
+  mbar_arrive_expect_tx(bar, V_BYTES);
+  tma_load_3d(sm + OFF_V, tv, bar, col0, h, tok0);
+  tma_load_3d(sm + OFF_V + 8192, tv, bar, col0 + 64, h, tok0);
+}
+
 __global__ void __maxnreg__(224)
     gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -345,6 +362,8 @@ __global__ void __maxnreg__(224)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
   float* s_carry = reinterpret_cast<float*>(sm + OFF_MISC + 8);
+  // loads issued so far: K/Q per stage, V (read back to drain in-flight copies on exit)
+  volatile int* s_issued = reinterpret_cast<volatile int*>(sm + OFF_MISC + 16);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -379,16 +398,12 @@ __global__ void __maxnreg__(224)
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], 1);
     *s_abort = 0;
+    s_issued[0] = s_issued[1] = s_issued[2] = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
     tmem_alloc(s_tmem, TMEM_COLS);
     tmem_relinquish();
-  }
-  if (warp == 8 && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
   }
   __syncwarp();
   tc_fence_before();
@@ -396,36 +411,22 @@ __global__ void __maxnreg__(224)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = smem_u32(sm);
-
-  if (warp == 8) {
-    // ================================================================ producer
-    if (lane == 0) {
-      int kq_issued0 = 0, kq_issued1 = 0, v_issued = 0;
-      for (int c = 0; c < n_chunks; ++c) {
-        const int s = c & 1;
-        const int tok0 = seq_start + c * C;
-        if (c >= 2 &&
-            !mbar_wait_bounded(&bars[B_KQ_EMPTY + s], ((c >> 1) - 1) & 1, s_abort, p.status))
-          break;
-        uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
-        mbar_arrive_expect_tx(&bars[B_KQ_FULL + s], KQ_BYTES);
-        tma_load_3d(kq + 0, &tm_k, &bars[B_KQ_FULL + s], 0, h, tok0);
-        tma_load_3d(kq + 16384, &tm_k, &bars[B_KQ_FULL + s], 64, h, tok0);
-        tma_load_3d(kq + 8192, &tm_q, &bars[B_KQ_FULL + s], 0, h, tok0);
-        tma_load_3d(kq + 24576, &tm_q, &bars[B_KQ_FULL + s], 64, h, tok0);
-        if (s == 0) kq_issued0 = (c >> 1) + 1; else kq_issued1 = (c >> 1) + 1;
-        if (c >= 1 && !mbar_wait_bounded(&bars[B_V_EMPTY], (c - 1) & 1, s_abort, p.status)) break;
-        mbar_arrive_expect_tx(&bars[B_V_FULL], V_BYTES);
-        tma_load_3d(sm + OFF_V, &tm_v, &bars[B_V_FULL], col0, h, tok0);
-        tma_load_3d(sm + OFF_V + 8192, &tm_v, &bars[B_V_FULL], col0 + 64, h, tok0);
-        v_issued = c + 1;
-      }
-      // never leave the block with bulk copies still landing in its shared memory
-      if (kq_issued0 > 0) mbar_wait_bounded(&bars[B_KQ_FULL], (kq_issued0 - 1) & 1, nullptr, p.status);
-      if (kq_issued1 > 0) mbar_wait_bounded(&bars[B_KQ_FULL + 1], (kq_issued1 - 1) & 1, nullptr, p.status);
-      if (v_issued > 0) mbar_wait_bounded(&bars[B_V_FULL], (v_issued - 1) & 1, nullptr, p.status);
+  if (tid == 0 && n_chunks > 0) {
+    // first loads: K/Q of chunks 0 and 1, V of chunk 0
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    load_kq(sm, &bars[B_KQ_FULL + 0], &tm_q, &tm_k, 0, h, seq_start);
+    s_issued[0] = 1;
+    if (n_chunks > 1) {
+      load_kq(sm, &bars[B_KQ_FULL + 1], &tm_q, &tm_k, 1, h, seq_start + C);
+      s_issued[1] = 1;
     }
-  } else if (warp < 4) {
+    load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, seq_start);
+    s_issued[2] = 1;
+  }
+
+  if (warp < 4) {
     // ================================================================ prep warpgroup
     const int t = tid;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
@@ -553,7 +554,10 @@ __global__ void __maxnreg__(224)
       if (!wg_wait<BAR_PREP>(&bars[B_PREP_MMA], pphase, s_abort, p.status)) break;
       pphase ^= 1;
       tc_fence_after();
-      if (t == 0) mbar_arrive(&bars[B_V_EMPTY]);
+      if (t == 0 && c + 1 < n_chunks) {   // the V stage is free: load V of chunk c+1
+        load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, tok0 + C);
+        s_issued[2] = c + 2;
+      }
 
       // ---- W^T tile (row d = t): free once the state warpgroup's U MMA of chunk c-1 is done
       if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
@@ -670,7 +674,10 @@ __global__ void __maxnreg__(224)
       if (!wg_wait<BAR_STATE>(&bars[B_STATE_MMA], sphase, s_abort, p.status)) break;
       sphase ^= 1;
       tc_fence_after();
-      if (j == 0) mbar_arrive(&bars[B_KQ_EMPTY + s]);   // last read of the K, Q stage is done
+      if (j == 0 && c + 2 < n_chunks) {   // last read of the K, Q stage is done: load chunk c+2
+        load_kq(sm, &bars[B_KQ_FULL + s], &tm_q, &tm_k, s, h, tok0 + 2 * C);
+        s_issued[s] = (c >> 1) + 2;
+      }
 
       // ---- next chunk's Sigma^T operand (bf16) and pre-decayed fp32 state; S_T at the end
       float decay = 1.f;
@@ -722,6 +729,12 @@ __global__ void __maxnreg__(224)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  if (tid == 0) {
+    // never leave the block with bulk copies still landing in its shared memory
+    if (s_issued[0] > 0) mbar_wait_bounded(&bars[B_KQ_FULL + 0], (s_issued[0] - 1) & 1, nullptr, p.status);
+    if (s_issued[1] > 0) mbar_wait_bounded(&bars[B_KQ_FULL + 1], (s_issued[1] - 1) & 1, nullptr, p.status);
+    if (s_issued[2] > 0) mbar_wait_bounded(&bars[B_V_FULL], (s_issued[2] - 1) & 1, nullptr, p.status);
+  }
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);

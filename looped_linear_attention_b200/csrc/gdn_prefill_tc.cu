@@ -203,19 +203,40 @@ __device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int row, int col
   }
 }
 
+__device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int row, const float (&x)[64]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 o;
+    o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
+    o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
+    o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
+    o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
+    *reinterpret_cast<uint4*>(tile + sw128_offset(row, c * 8)) = o;
+  }
+}
+
+// Gate inputs of one token (threads 0-63 of the prep warpgroup): log a and b,
+// or 0 past the sequence end.  Issued one chunk ahead so the global-memory
+// latency is hidden behind the current chunk.
+__device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int valid, int h, int t,
+                                                 float& la, float& bb) {
+  la = 0.f;
+  bb = 0.f;
+  if (t < valid) {
+    const size_t ti = (size_t)(tok0 + t) * p.H + h;
+    la = __ldg(p.a + ti);
+    bb = __ldg(p.b + ti);
+  }
+}
+
 // Gate vectors of one chunk (all 128 prep threads call this; threads 0-63 own
 // one token each).  Rows past the sequence end get log a = 0 and b = 0.
-__device__ __forceinline__ void compute_gates(const Params& p, Gates G, float* s_carry, int tok0,
-                                              int valid, int h, int t) {
+__device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid, int t,
+                                              float a_in, float bb) {
   const int lane = t & 31;
   float la = 0.f;
   if (t < C) {
-    float bb = 0.f;
-    if (t < valid) {
-      const size_t ti = (size_t)(tok0 + t) * p.H + h;
-      la = logf(__ldg(p.a + ti));
-      bb = __ldg(p.b + ti);
-    }
+    la = (t < valid) ? logf(a_in) : 0.f;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const float y = __shfl_up_sync(0xffffffffu, la, off);
@@ -253,30 +274,34 @@ __device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, floa
     const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
     const float* arow = s_A + ((bb + D) * 16 + r) * A_LD + bb * 16;
     const float* tcol = s_T + (bb * 16) * T_LD + bb * 16 + c;
-    float y0 = 0.f, y1 = 0.f;
+    float y0 = 0.f, y1 = 0.f, z0 = 0.f, z1 = 0.f;
 #pragma unroll
-    for (int k = 0; k < 16 * D; ++k) {
-      const float av = arow[k];
+    for (int k = 0; k < 16 * D; k += 2) {
+      const float av = arow[k], aw = arow[k + 1];
       y0 = fmaf(av, tcol[k * T_LD], y0);
       y1 = fmaf(av, tcol[k * T_LD + 8], y1);
+      z0 = fmaf(aw, tcol[(k + 1) * T_LD], z0);
+      z1 = fmaf(aw, tcol[(k + 1) * T_LD + 8], z1);
     }
-    s_Y[(bb * 16 + r) * 17 + c] = y0;
-    s_Y[(bb * 16 + r) * 17 + c + 8] = y1;
+    s_Y[(bb * 16 + r) * 17 + c] = y0 + z0;
+    s_Y[(bb * 16 + r) * 17 + c + 8] = y1 + z1;
   }
   wg_sync<BAR_PREP>();
   for (int it = t; it < ITEMS; it += WG) {
     const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
     const float* trow = s_T + ((bb + D) * 16 + r) * T_LD + (bb + D) * 16;
     const float* ycol = s_Y + (bb * 16) * 17 + c;
-    float t0 = 0.f, t1 = 0.f;
+    float t0 = 0.f, t1 = 0.f, u0 = 0.f, u1 = 0.f;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float tv = trow[k];
+    for (int k = 0; k < 16; k += 2) {
+      const float tv = trow[k], tw = trow[k + 1];
       t0 = fmaf(tv, ycol[k * 17], t0);
       t1 = fmaf(tv, ycol[k * 17 + 8], t1);
+      u0 = fmaf(tw, ycol[(k + 1) * 17], u0);
+      u1 = fmaf(tw, ycol[(k + 1) * 17 + 8], u1);
     }
-    s_T[((bb + D) * 16 + r) * T_LD + bb * 16 + c] = -t0;
-    s_T[((bb + D) * 16 + r) * T_LD + bb * 16 + c + 8] = -t1;
+    s_T[((bb + D) * 16 + r) * T_LD + bb * 16 + c] = -(t0 + u0);
+    s_T[((bb + D) * 16 + r) * T_LD + bb * 16 + c + 8] = -(t1 + u1);
   }
   wg_sync<BAR_PREP>();
 }
@@ -287,10 +312,14 @@ __device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      float acc = (i == c) ? 1.f : 0.f;
+      float acc0 = (i == c) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int m = 0; m < i; ++m) acc = fmaf(-s_A[(r0 + i) * A_LD + r0 + m], x[m], acc);
-      x[i] = acc;
+      for (int m = 0; m + 1 < i; m += 2) {
+        acc0 = fmaf(-s_A[(r0 + i) * A_LD + r0 + m], x[m], acc0);
+        acc1 = fmaf(-s_A[(r0 + i) * A_LD + r0 + m + 1], x[m + 1], acc1);
+      }
+      if (i & 1) acc0 = fmaf(-s_A[(r0 + i) * A_LD + r0 + i - 1], x[i - 1], acc0);
+      x[i] = acc0 + acc1;
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) s_T[(r0 + i) * T_LD + r0 + c] = x[i];
@@ -308,27 +337,22 @@ __device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_
 __device__ __forceinline__ void refresh_state(uint32_t taddr, uint8_t* sig, int j, float decay,
                                               bool scale_tmem, float* st_out, int dv) {
 #pragma unroll 1
-  for (int piece = 0; piece < 4; ++piece) {
-    float x[32];
-    tmem_ld32(taddr + piece * 32, x);
-    uint8_t* slab = sig + (piece >> 1) * 16384;
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      uint4 o;
-      o.x = pack_bf16x2(x[cc * 8 + 0], x[cc * 8 + 1]);
-      o.y = pack_bf16x2(x[cc * 8 + 2], x[cc * 8 + 3]);
-      o.z = pack_bf16x2(x[cc * 8 + 4], x[cc * 8 + 5]);
-      o.w = pack_bf16x2(x[cc * 8 + 6], x[cc * 8 + 7]);
-      *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + cc * 8)) = o;
-    }
+  for (int piece = 0; piece < 2; ++piece) {
+    float x[64];
+    tmem_ld64(taddr + piece * 64, x);
+    store_row64_bf16(sig + piece * 16384, j, x);
     if (st_out) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) st_out[(size_t)(piece * 32 + e) * dv] = x[e];
+      for (int e = 0; e < 64; ++e) st_out[(size_t)(piece * 64 + e) * dv] = x[e];
     }
     if (scale_tmem) {
+      float y[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) x[e] *= decay;
-      tmem_st32(taddr + piece * 32, x);
+      for (int e = 0; e < 32; ++e) y[e] = x[e] * decay;
+      tmem_st32(taddr + piece * 64, y);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) y[e] = x[32 + e] * decay;
+      tmem_st32(taddr + piece * 64 + 32, y);
     }
   }
   tmem_wait_st();
@@ -355,9 +379,12 @@ __global__ void __maxnreg__(224)
     gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
+  if (smem_u32(sm) & 1023u) {   // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) record_status(p.status, GDN_ERR_CUDA);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
@@ -434,6 +461,8 @@ __global__ void __maxnreg__(224)
     float* s_T = reinterpret_cast<float*>(sm + OFF_T1);
     float* s_Y = reinterpret_cast<float*>(sm + OFF_Y);
     uint32_t pphase = 0;
+    float a_in = 1.f, b_in = 0.f;
+    if (n_chunks > 0) load_gate_inputs(p, seq_start, min(C, len), h, t, a_in, b_in);
 #pragma unroll 1
     for (int c = 0; c < n_chunks; ++c) {
       const int s = c & 1;
@@ -443,8 +472,10 @@ __global__ void __maxnreg__(224)
       uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
       const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
 
-      // ---- gates of chunk c (the buffer's previous user, chunk c-3, is finished)
-      compute_gates(p, G, s_carry, tok0, valid, h, t);
+      // ---- gates of chunk c (the buffer's previous user, chunk c-3, is finished);
+      // the next chunk's inputs are fetched now and used one iteration later
+      compute_gates(G, s_carry, valid, t, a_in, b_in);
+      if (c + 1 < n_chunks) load_gate_inputs(p, tok0 + C, min(C, seq_end - tok0 - C), h, t, a_in, b_in);
       wg_sync<BAR_PREP>();
       if (t == 0) mbar_arrive(&bars[B_GATES + c % 3]);
 
@@ -481,24 +512,16 @@ __global__ void __maxnreg__(224)
         const int i = t & 63;
         const float gi = G.g[i], bi = G.b[i];
         uint8_t* pt = sm + OFF_P + s * 8192;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float gr[32];
-          tmem_ld32(tmem + lane_off + COL_GW + half * 32, gr);
-          if (t < C) {
+        float gr[64];
+        tmem_ld64(tmem + lane_off + COL_GW, gr);
+        if (t < C) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int jj = half * 32 + e;
-              s_A[i * A_LD + jj] = (jj < i) ? bi * __expf(gi - G.g[jj]) * gr[e] : 0.f;
-            }
-          } else {
+          for (int jj = 0; jj < C; ++jj)
+            s_A[i * A_LD + jj] = (jj < i) ? bi * __expf(gi - G.g[jj]) * gr[jj] : 0.f;
+        } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int jj = half * 32 + e;
-              gr[e] = (jj <= i) ? __expf(gi - G.g[jj]) * gr[e] : 0.f;
-            }
-            store_row32_bf16(pt, i, half * 32, gr);
-          }
+          for (int jj = 0; jj < C; ++jj) gr[jj] = (jj <= i) ? __expf(gi - G.g[jj]) * gr[jj] : 0.f;
+          store_row64_bf16(pt, i, gr);
         }
       }
       tc_fence_before();
@@ -561,11 +584,10 @@ __global__ void __maxnreg__(224)
 
       // ---- W^T tile (row d = t): free once the state warpgroup's U MMA of chunk c-1 is done
       if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        float wr[32];
-        tmem_ld32(tmem + lane_off + COL_GW + half * 32, wr);
-        store_row32_bf16(sm + OFF_WT, t, half * 32, wr);
+      {
+        float wr[64];
+        tmem_ld64(tmem + lane_off + COL_GW, wr);
+        store_row64_bf16(sm + OFF_WT, t, wr);
       }
       tc_fence_before();
       fence_proxy_async_smem();
@@ -646,14 +668,13 @@ __global__ void __maxnreg__(224)
       if (j == 0) mbar_arrive(&bars[B_W_CONSUMED]);
 
       // ---- U^T row j -> operand tiles U^T and U^T diag(gamma_C / gamma)
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        float ur[32];
-        tmem_ld32(tmem + lane_off + COL_U + s * 64 + half * 32, ur);
-        store_row32_bf16(sm + OFF_UT, j, half * 32, ur);
+      {
+        float ur[64];
+        tmem_ld64(tmem + lane_off + COL_U + s * 64, ur);
+        store_row64_bf16(sm + OFF_UT, j, ur);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) ur[e] *= G.r[half * 32 + e];
-        store_row32_bf16(sm + OFF_UTP, j, half * 32, ur);
+        for (int e = 0; e < C; ++e) ur[e] *= G.r[e];
+        store_row64_bf16(sm + OFF_UTP, j, ur);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -692,18 +713,20 @@ __global__ void __maxnreg__(224)
       // through shared memory ([64 tok][128 dv] bf16) for 16-byte coalesced stores
       {
         uint8_t* stage = sm + OFF_UTP;
-        float oa[32], ob[32];
-#pragma unroll 1
+        float oo[64];
+        tmem_ld64(tmem + lane_off + COL_OA, oo);
+#pragma unroll
+        for (int i = 0; i < C; ++i) oo[i] *= G.gamma[i];
+#pragma unroll
         for (int half = 0; half < 2; ++half) {
-          tmem_ld32(tmem + lane_off + COL_OA + half * 32, oa);
+          float ob[32];
           tmem_ld32(tmem + lane_off + COL_OB + half * 32, ob);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = half * 32 + e;
-            *reinterpret_cast<__nv_bfloat16*>(stage + i * 256 + j * 2) =
-                __float2bfloat16_rn(p.scale * fmaf(G.gamma[i], oa[e], ob[e]));
-          }
+          for (int e = 0; e < 32; ++e) oo[half * 32 + e] = p.scale * (oo[half * 32 + e] + ob[e]);
         }
+#pragma unroll
+        for (int i = 0; i < C; ++i)
+          *reinterpret_cast<__nv_bfloat16*>(stage + i * 256 + j * 2) = __float2bfloat16_rn(oo[i]);
       }
       tc_fence_before();
       wg_sync<BAR_STATE>();

@@ -82,7 +82,9 @@ constexpr uint32_t OFF_T1 = 180224;       // T diag(b gamma) bf16 [64][64] (T fp
 constexpr uint32_t OFF_T2 = 188416;       // T diag(b) bf16 [64][64]
 constexpr uint32_t OFF_A = 196608;        // A fp32 [64][65] (padded rows)
 constexpr int A_LD = 65;
-constexpr int T_LD = 64;
+// T scratch: 64 x 64 fp32 with the column XOR-swizzled by (row mod 4) * 8, so
+// that column reads across four consecutive rows hit distinct banks.
+__device__ __forceinline__ int tix(int row, int col) { return row * 64 + (col ^ ((row & 3) << 3)); }
 constexpr uint32_t OFF_Y = OFF_A + 64 * A_LD * 4;     // solve scratch 48 x 17 fp32
 constexpr uint32_t OFF_GATE = OFF_Y + 48 * 17 * 4;    // 3 buffers x {g, gamma, b, b*gamma, gamma_C/gamma}
 constexpr uint32_t GATE_BYTES = 5 * 64 * 4;
@@ -91,7 +93,7 @@ constexpr uint32_t OFF_MISC = OFF_BAR + 256;          // tmem base, abort flag, 
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
-static_assert(OFF_T1 + 64 * T_LD * 4 <= OFF_A, "T scratch must fit over T1|T2");
+static_assert(OFF_T1 + 64 * 64 * 4 <= OFF_A, "T scratch must fit over T1|T2");
 
 // mbarriers (index into the barrier array)
 enum : int {
@@ -264,7 +266,7 @@ __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid
 // A_LD), blocked by 16.  The diagonal blocks are inverted by forward
 // substitution (one column per thread); the off-diagonal blocks follow by
 // block distance D: T_{b+D,b} = -T_{b+D,b+D} sum_{m=b}^{b+D-1} A_{b+D,m} T_{m,b}.
-// s_T receives T (row stride T_LD; its upper block triangle is left unset);
+// s_T receives T (swizzled by tix(); its upper block triangle is left unset);
 // s_Y is 3 x 16 x 17 fp32 scratch.  All prep threads take part.
 template <int D>
 __device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, float* s_Y, int t) {
@@ -273,15 +275,15 @@ __device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, floa
   for (int it = t; it < ITEMS; it += WG) {
     const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
     const float* arow = s_A + ((bb + D) * 16 + r) * A_LD + bb * 16;
-    const float* tcol = s_T + (bb * 16) * T_LD + bb * 16 + c;
     float y0 = 0.f, y1 = 0.f, z0 = 0.f, z1 = 0.f;
 #pragma unroll
     for (int k = 0; k < 16 * D; k += 2) {
       const float av = arow[k], aw = arow[k + 1];
-      y0 = fmaf(av, tcol[k * T_LD], y0);
-      y1 = fmaf(av, tcol[k * T_LD + 8], y1);
-      z0 = fmaf(aw, tcol[(k + 1) * T_LD], z0);
-      z1 = fmaf(aw, tcol[(k + 1) * T_LD + 8], z1);
+      const int r0 = bb * 16 + k, c0 = bb * 16 + c;
+      y0 = fmaf(av, s_T[tix(r0, c0)], y0);
+      y1 = fmaf(av, s_T[tix(r0, c0 + 8)], y1);
+      z0 = fmaf(aw, s_T[tix(r0 + 1, c0)], z0);
+      z1 = fmaf(aw, s_T[tix(r0 + 1, c0 + 8)], z1);
     }
     s_Y[(bb * 16 + r) * 17 + c] = y0 + z0;
     s_Y[(bb * 16 + r) * 17 + c + 8] = y1 + z1;
@@ -289,19 +291,19 @@ __device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, floa
   wg_sync<BAR_PREP>();
   for (int it = t; it < ITEMS; it += WG) {
     const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
-    const float* trow = s_T + ((bb + D) * 16 + r) * T_LD + (bb + D) * 16;
+    const int rowT = (bb + D) * 16 + r;
     const float* ycol = s_Y + (bb * 16) * 17 + c;
     float t0 = 0.f, t1 = 0.f, u0 = 0.f, u1 = 0.f;
 #pragma unroll
     for (int k = 0; k < 16; k += 2) {
-      const float tv = trow[k], tw = trow[k + 1];
+      const float tv = s_T[tix(rowT, (bb + D) * 16 + k)], tw = s_T[tix(rowT, (bb + D) * 16 + k + 1)];
       t0 = fmaf(tv, ycol[k * 17], t0);
       t1 = fmaf(tv, ycol[k * 17 + 8], t1);
       u0 = fmaf(tw, ycol[(k + 1) * 17], u0);
       u1 = fmaf(tw, ycol[(k + 1) * 17 + 8], u1);
     }
-    s_T[((bb + D) * 16 + r) * T_LD + bb * 16 + c] = -(t0 + u0);
-    s_T[((bb + D) * 16 + r) * T_LD + bb * 16 + c + 8] = -(t1 + u1);
+    s_T[tix(rowT, bb * 16 + c)] = -(t0 + u0);
+    s_T[tix(rowT, bb * 16 + c + 8)] = -(t1 + u1);
   }
   wg_sync<BAR_PREP>();
 }
@@ -322,7 +324,7 @@ __device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_
       x[i] = acc0 + acc1;
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s_T[(r0 + i) * T_LD + r0 + c] = x[i];
+    for (int i = 0; i < 16; ++i) s_T[tix(r0 + i, r0 + c)] = x[i];
   }
   wg_sync<BAR_PREP>();
   offdiag_level<1>(s_A, s_T, s_Y, t);
@@ -537,7 +539,7 @@ __global__ void __maxnreg__(224)
           const int i = it >> 3, q8 = (it & 7) * 8;
           const bool zero = ((q8 >> 4) > (i >> 4));
 #pragma unroll
-          for (int e = 0; e < 8; ++e) tv[k4][e] = zero ? 0.f : s_T[i * T_LD + q8 + e];
+          for (int e = 0; e < 8; ++e) tv[k4][e] = zero ? 0.f : s_T[tix(i, q8 + e)];
         }
         wg_sync<BAR_PREP>();
 #pragma unroll

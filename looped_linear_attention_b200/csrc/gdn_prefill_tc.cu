@@ -88,7 +88,12 @@ __device__ __forceinline__ int tix(int row, int col) { return row * 64 + (col ^ 
 constexpr uint32_t OFF_Y = OFF_A + 64 * A_LD * 4;     // solve scratch 48 x 17 fp32
 constexpr uint32_t OFF_GATE = OFF_Y + 48 * 17 * 4;    // 3 buffers x {g, gamma, b, b*gamma, gamma_C/gamma}
 constexpr uint32_t GATE_BYTES = 5 * 64 * 4;
-constexpr uint32_t OFF_BAR = OFF_GATE + 3 * GATE_BYTES;
+// prep-only decay tables of the current chunk: row factors e_i = exp(g_i - g_16I),
+// column factors F[I-1][j] = exp(g_16I - g_j) (j < 16I, I = 1..3), and the
+// in-block decays Dd[I][r][c] = exp(g_{16I+r} - g_{16I+c}) (c <= r, else 0)
+constexpr uint32_t OFF_DEC = OFF_GATE + 3 * GATE_BYTES;
+constexpr uint32_t DEC_BYTES = (64 + 3 * 64 + 4 * 256) * 4;
+constexpr uint32_t OFF_BAR = OFF_DEC + DEC_BYTES;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;          // tmem base, abort flag, scan carry
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
@@ -217,6 +222,45 @@ __device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int row, const f
   }
 }
 
+// exp(x) for x <= 0 as 2^(x log2 e) with the hardware base-2 exponential
+// (relative error about 2^-22; results below 2^-126 flush to zero).
+constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float exp_nonpos(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * kLog2e));
+  return y;
+}
+
+// Warp-level m16n8k8 tf32 MMA (fp32 accumulate) for the 16 x 16 blocks of the
+// solve, with each operand split into a tf32 high part and a tf32 remainder:
+// a b ~= ah bh + ah bl + al bh, which keeps the products close to fp32.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = to_tf32(x);
+  lo = to_tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void mma_3xtf32(float (&d)[4], const float (&a)[4], const float (&b)[2]) {
+  uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) split_tf32(a[i], ah[i], al[i]);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) split_tf32(b[i], bh[i], bl[i]);
+  mma_tf32(d, al, bh);
+  mma_tf32(d, ah, bl);
+  mma_tf32(d, ah, bh);
+}
+
 // Gate inputs of one token (threads 0-63 of the prep warpgroup): log a and b,
 // or 0 past the sequence end.  Issued one chunk ahead so the global-memory
 // latency is hidden behind the current chunk.
@@ -233,8 +277,8 @@ __device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int 
 
 // Gate vectors of one chunk (all 128 prep threads call this; threads 0-63 own
 // one token each).  Rows past the sequence end get log a = 0 and b = 0.
-__device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid, int t,
-                                              float a_in, float bb) {
+__device__ __forceinline__ void compute_gates(Gates G, float* s_carry, float* s_dec, int valid,
+                                              int t, float a_in, float bb) {
   const int lane = t & 31;
   float la = 0.f;
   if (t < C) {
@@ -255,10 +299,24 @@ __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid
   wg_sync<BAR_PREP>();
   if (t < C) {
     const float gC = G.g[C - 1];
-    const float gam = __expf(la);
+    const float gam = exp_nonpos(la);
     G.gamma[t] = gam;
     G.bg[t] = G.b[t] * gam;
-    G.r[t] = __expf(gC - la);
+    G.r[t] = exp_nonpos(gC - la);
+    s_dec[t] = exp_nonpos(la - G.g[t & ~15]);                         // e_i
+  }
+  // F[I-1][j] = exp(g_16I - g_j) for j < 16I: 96 entries
+  for (int u = t; u < 96; u += WG) {
+    const int I = (u < 16) ? 1 : (u < 48 ? 2 : 3);
+    const int jj = u - (I == 1 ? 0 : (I == 2 ? 16 : 48));
+    s_dec[64 + (I - 1) * 64 + jj] = exp_nonpos(G.g[16 * I] - G.g[jj]);
+  }
+  // Dd[I][r][c] = exp(g_{16I+r} - g_{16I+c}) for c <= r
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int u = t + k * WG;
+    const int I = u >> 8, r = (u >> 4) & 15, cc = u & 15;
+    s_dec[256 + u] = (cc <= r) ? exp_nonpos(G.g[16 * I + r] - G.g[16 * I + cc]) : 0.f;
   }
 }
 
@@ -271,39 +329,54 @@ __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid
 template <int D>
 __device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, float* s_Y, int t) {
   constexpr int NB = 4 - D;
-  constexpr int ITEMS = NB * 128;   // (block, row, column pair c / c+8)
-  for (int it = t; it < ITEMS; it += WG) {
-    const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
-    const float* arow = s_A + ((bb + D) * 16 + r) * A_LD + bb * 16;
-    float y0 = 0.f, y1 = 0.f, z0 = 0.f, z1 = 0.f;
+  const int warp = t >> 5, lane = t & 31;
+  const int g = lane >> 2, q = lane & 3;   // mma fragment coordinates
+  if (warp < NB) {
+    const int bb = warp;                   // block column; this warp fills T_{bb+D, bb}
+    const int rA = (bb + D) * 16;
+    // Y = sum_{m=bb}^{bb+D-1} A_{bb+D,m} T_{m,bb}   (16 x 16, K = 16 D)
+    float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int k = 0; k < 16 * D; k += 2) {
-      const float av = arow[k], aw = arow[k + 1];
-      const int r0 = bb * 16 + k, c0 = bb * 16 + c;
-      y0 = fmaf(av, s_T[tix(r0, c0)], y0);
-      y1 = fmaf(av, s_T[tix(r0, c0 + 8)], y1);
-      z0 = fmaf(aw, s_T[tix(r0 + 1, c0)], z0);
-      z1 = fmaf(aw, s_T[tix(r0 + 1, c0 + 8)], z1);
-    }
-    s_Y[(bb * 16 + r) * 17 + c] = y0 + z0;
-    s_Y[(bb * 16 + r) * 17 + c + 8] = y1 + z1;
-  }
-  wg_sync<BAR_PREP>();
-  for (int it = t; it < ITEMS; it += WG) {
-    const int bb = it >> 7, r = (it >> 3) & 15, c = it & 7;
-    const int rowT = (bb + D) * 16 + r;
-    const float* ycol = s_Y + (bb * 16) * 17 + c;
-    float t0 = 0.f, t1 = 0.f, u0 = 0.f, u1 = 0.f;
+    for (int k0 = 0; k0 < 16 * D; k0 += 8) {
+      const int ca = bb * 16 + k0;
+      const float a[4] = {s_A[(rA + g) * A_LD + ca + q], s_A[(rA + g + 8) * A_LD + ca + q],
+                          s_A[(rA + g) * A_LD + ca + q + 4], s_A[(rA + g + 8) * A_LD + ca + q + 4]};
 #pragma unroll
-    for (int k = 0; k < 16; k += 2) {
-      const float tv = s_T[tix(rowT, (bb + D) * 16 + k)], tw = s_T[tix(rowT, (bb + D) * 16 + k + 1)];
-      t0 = fmaf(tv, ycol[k * 17], t0);
-      t1 = fmaf(tv, ycol[k * 17 + 8], t1);
-      u0 = fmaf(tw, ycol[(k + 1) * 17], u0);
-      u1 = fmaf(tw, ycol[(k + 1) * 17 + 8], u1);
+      for (int nt = 0; nt < 2; ++nt) {
+        const int cb = bb * 16 + nt * 8 + g;
+        const float b[2] = {s_T[tix(ca + q, cb)], s_T[tix(ca + q + 4, cb)]};
+        mma_3xtf32(y[nt], a, b);
+      }
     }
-    s_T[tix(rowT, bb * 16 + c)] = -(t0 + u0);
-    s_T[tix(rowT, bb * 16 + c + 8)] = -(t1 + u1);
+    float* Yb = s_Y + bb * 16 * 17;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      Yb[g * 17 + nt * 8 + 2 * q] = y[nt][0];
+      Yb[g * 17 + nt * 8 + 2 * q + 1] = y[nt][1];
+      Yb[(g + 8) * 17 + nt * 8 + 2 * q] = y[nt][2];
+      Yb[(g + 8) * 17 + nt * 8 + 2 * q + 1] = y[nt][3];
+    }
+    __syncwarp();
+    // T_{bb+D, bb} = -T_{bb+D, bb+D} Y   (16 x 16, K = 16)
+    float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int k0 = 0; k0 < 16; k0 += 8) {
+      const float a[4] = {s_T[tix(rA + g, rA + k0 + q)], s_T[tix(rA + g + 8, rA + k0 + q)],
+                          s_T[tix(rA + g, rA + k0 + q + 4)], s_T[tix(rA + g + 8, rA + k0 + q + 4)]};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const float b[2] = {Yb[(k0 + q) * 17 + nt * 8 + g], Yb[(k0 + q + 4) * 17 + nt * 8 + g]};
+        mma_3xtf32(z[nt], a, b);
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int cc = bb * 16 + nt * 8 + 2 * q;
+      s_T[tix(rA + g, cc)] = -z[nt][0];
+      s_T[tix(rA + g, cc + 1)] = -z[nt][1];
+      s_T[tix(rA + g + 8, cc)] = -z[nt][2];
+      s_T[tix(rA + g + 8, cc + 1)] = -z[nt][3];
+    }
   }
   wg_sync<BAR_PREP>();
 }
@@ -462,6 +535,7 @@ __global__ void __maxnreg__(224)
     float* s_A = reinterpret_cast<float*>(sm + OFF_A);
     float* s_T = reinterpret_cast<float*>(sm + OFF_T1);
     float* s_Y = reinterpret_cast<float*>(sm + OFF_Y);
+    float* s_dec = reinterpret_cast<float*>(sm + OFF_DEC);
     uint32_t pphase = 0;
     float a_in = 1.f, b_in = 0.f;
     if (n_chunks > 0) load_gate_inputs(p, seq_start, min(C, len), h, t, a_in, b_in);
@@ -476,7 +550,7 @@ __global__ void __maxnreg__(224)
 
       // ---- gates of chunk c (the buffer's previous user, chunk c-3, is finished);
       // the next chunk's inputs are fetched now and used one iteration later
-      compute_gates(G, s_carry, valid, t, a_in, b_in);
+      compute_gates(G, s_carry, s_dec, valid, t, a_in, b_in);
       if (c + 1 < n_chunks) load_gate_inputs(p, tok0 + C, min(C, seq_end - tok0 - C), h, t, a_in, b_in);
       wg_sync<BAR_PREP>();
       if (t == 0) mbar_arrive(&bars[B_GATES + c % 3]);
@@ -511,18 +585,29 @@ __global__ void __maxnreg__(224)
       {
         // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32) and
         // P = tril(D o Q K^T) (rows 64-127, bf16 operand), 32 columns of G at a time
+        // D_ij = e_i F[I-1][j] below the diagonal block (I = i / 16), Dd[I][i-16I][j-16I]
+        // inside it, 0 above; all factors were tabulated with the gates.
         const int i = t & 63;
-        const float gi = G.g[i], bi = G.b[i];
+        const int I = i >> 4;
+        const float ei = s_dec[i];
+        const float* Frow = s_dec + 64 + (I > 0 ? I - 1 : 0) * 64;
+        const float* Ddr = s_dec + 256 + I * 256 + (i & 15) * 16;
         uint8_t* pt = sm + OFF_P + s * 8192;
         float gr[64];
         tmem_ld64(tmem + lane_off + COL_GW, gr);
+#pragma unroll
+        for (int jj = 0; jj < C; ++jj) {
+          const int bj = jj >> 4;
+          float dv_ = 0.f;
+          if (bj < I) dv_ = ei * Frow[jj];
+          else if (bj == I) dv_ = Ddr[jj & 15];
+          gr[jj] *= dv_;
+        }
         if (t < C) {
+          const float bi = G.b[i];
 #pragma unroll
-          for (int jj = 0; jj < C; ++jj)
-            s_A[i * A_LD + jj] = (jj < i) ? bi * __expf(gi - G.g[jj]) * gr[jj] : 0.f;
+          for (int jj = 0; jj < C; ++jj) s_A[i * A_LD + jj] = (jj < i) ? bi * gr[jj] : 0.f;
         } else {
-#pragma unroll
-          for (int jj = 0; jj < C; ++jj) gr[jj] = (jj <= i) ? __expf(gi - G.g[jj]) * gr[jj] : 0.f;
           store_row64_bf16(pt, i, gr);
         }
       }

@@ -78,27 +78,26 @@ constexpr uint32_t OFF_WT = 114688;       // W^T bf16 [128 dk][64 tok] (MN-major
 constexpr uint32_t OFF_UT = 131072;       // U^T bf16 [128 dv][64 tok]
 constexpr uint32_t OFF_UTP = 147456;      // U^T diag(gamma_C/gamma) bf16; output staging
 constexpr uint32_t OFF_P = 163840;        // P bf16 [64][64], two buffers (chunk parity)
-constexpr uint32_t OFF_T1 = 180224;       // T diag(b gamma) bf16 [64][64] (T fp32 scratch overlays T1|T2)
+constexpr uint32_t OFF_T1 = 180224;       // T diag(b gamma) bf16 [64][64]
 constexpr uint32_t OFF_T2 = 188416;       // T diag(b) bf16 [64][64]
-constexpr uint32_t OFF_A = 196608;        // A fp32 [64][65] (padded rows)
-constexpr int A_LD = 65;
-// T scratch: 64 x 64 fp32 with the column XOR-swizzled by (row mod 4) * 8, so
-// that column reads across four consecutive rows hit distinct banks.
-__device__ __forceinline__ int tix(int row, int col) { return row * 64 + (col ^ ((row & 3) << 3)); }
-constexpr uint32_t OFF_Y = OFF_A + 64 * A_LD * 4;     // solve scratch 48 x 17 fp32
-constexpr uint32_t OFF_GATE = OFF_Y + 48 * 17 * 4;    // 3 buffers x {g, gamma, b, b*gamma, gamma_C/gamma}
+// A and T (fp32) in compact lower-block-triangular form: the ten 16 x 16 blocks
+// (a, b), a >= b, each stored row-major with row stride 20 (the tf32 mma
+// fragment loads of a warp then hit 32 distinct banks); blocks 324 floats apart
+// so that the four diagonal blocks start in different banks.
+constexpr int BLK_LD = 20;
+constexpr int BLK_FLOATS = 16 * BLK_LD + 4;
+__device__ __forceinline__ int blk(int a, int b) { return (a * (a + 1) / 2 + b) * BLK_FLOATS; }
+constexpr uint32_t LT_BYTES = 10 * BLK_FLOATS * 4;
+constexpr uint32_t OFF_A = 196608;                    // A, compact blocks
+constexpr uint32_t OFF_TS = OFF_A + LT_BYTES;         // T, compact blocks (also the solve's scratch)
+constexpr uint32_t OFF_GATE = OFF_TS + LT_BYTES;      // 3 buffers x {g2, gamma, b, b*gamma, gamma_C/gamma}
 constexpr uint32_t GATE_BYTES = 5 * 64 * 4;
-// prep-only decay tables of the current chunk: row factors e_i = exp(g_i - g_16I),
-// column factors F[I-1][j] = exp(g_16I - g_j) (j < 16I, I = 1..3), and the
-// in-block decays Dd[I][r][c] = exp(g_{16I+r} - g_{16I+c}) (c <= r, else 0)
-constexpr uint32_t OFF_DEC = OFF_GATE + 3 * GATE_BYTES;
-constexpr uint32_t DEC_BYTES = (64 + 3 * 64 + 4 * 256) * 4;
-constexpr uint32_t OFF_BAR = OFF_DEC + DEC_BYTES;
+constexpr uint32_t OFF_BAR = OFF_GATE + 3 * GATE_BYTES;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;          // tmem base, abort flag, scan carry
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
-static_assert(OFF_T1 + 64 * 64 * 4 <= OFF_A, "T scratch must fit over T1|T2");
+static_assert(OFF_GATE % 16 == 0 && (BLK_FLOATS * 4) % 16 == 0, "vector access alignment");
 
 // mbarriers (index into the barrier array)
 enum : int {
@@ -128,7 +127,7 @@ struct Params {
 
 // Per-chunk gate vectors (one buffer).
 struct Gates {
-  float* g;      // prefix sum of log a
+  float* g2;     // prefix sum of log2 a (log2 gamma)
   float* gamma;  // exp(g)
   float* b;      // write strength (0 past the sequence end)
   float* bg;     // b * gamma
@@ -222,18 +221,19 @@ __device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int row, const f
   }
 }
 
-// exp(x) for x <= 0 as 2^(x log2 e) with the hardware base-2 exponential
-// (relative error about 2^-22; results below 2^-126 flush to zero).
-constexpr float kLog2e = 1.4426950408889634f;
-__device__ __forceinline__ float exp_nonpos(float x) {
+// 2^x with the hardware base-2 exponential (relative error about 2^-22;
+// results below 2^-126 flush to zero).  Every decay factor of the chunk is
+// 2^(g2_i - g2_j) with g2 = log2 gamma.
+__device__ __forceinline__ float ex2_approx(float x) {
   float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * kLog2e));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
 // Warp-level m16n8k8 tf32 MMA (fp32 accumulate) for the 16 x 16 blocks of the
 // solve, with each operand split into a tf32 high part and a tf32 remainder:
-// a b ~= ah bh + ah bl + al bh, which keeps the products close to fp32.
+// a b ~= ah bh + ah bl + al bh, which keeps the products close to fp32.  The
+// three partial products go to separate accumulators (independent chains).
 __device__ __forceinline__ uint32_t to_tf32(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -250,39 +250,111 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-__device__ __forceinline__ void mma_3xtf32(float (&d)[4], const float (&a)[4], const float (&b)[2]) {
-  uint32_t ah[4], al[4], bh[2], bl[2];
+
+// Fragments of one compact 16 x 16 block (g = lane / 4, q = lane % 4):
+// as the A operand (two k-steps of 16 x 8) or as the B operand (two k-steps
+// x two n-tiles of 8 x 8).
+__device__ __forceinline__ void frag_a(float (&a)[2][4], const float* blkp, int g, int q) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) split_tf32(a[i], ah[i], al[i]);
+  for (int ks = 0; ks < 2; ++ks) {
+    a[ks][0] = blkp[g * BLK_LD + ks * 8 + q];
+    a[ks][1] = blkp[(g + 8) * BLK_LD + ks * 8 + q];
+    a[ks][2] = blkp[g * BLK_LD + ks * 8 + q + 4];
+    a[ks][3] = blkp[(g + 8) * BLK_LD + ks * 8 + q + 4];
+  }
+}
+__device__ __forceinline__ void frag_b(float (&b)[2][2][2], const float* blkp, int g, int q) {
 #pragma unroll
-  for (int i = 0; i < 2; ++i) split_tf32(b[i], bh[i], bl[i]);
-  mma_tf32(d, al, bh);
-  mma_tf32(d, ah, bl);
-  mma_tf32(d, ah, bh);
+  for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      b[ks][nt][0] = blkp[(ks * 8 + q) * BLK_LD + nt * 8 + g];
+      b[ks][nt][1] = blkp[(ks * 8 + q + 4) * BLK_LD + nt * 8 + g];
+    }
+}
+// acc[nt][term] += A B for one block pair (K = 16)
+__device__ __forceinline__ void mma_blk(float (&acc)[2][3][4], const float (&a)[2][4],
+                                        const float (&b)[2][2][2]) {
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    uint32_t ah[4], al[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) split_tf32(a[ks][e], ah[e], al[e]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      uint32_t bh[2], bl[2];
+      split_tf32(b[ks][nt][0], bh[0], bl[0]);
+      split_tf32(b[ks][nt][1], bh[1], bl[1]);
+      mma_tf32(acc[nt][0], ah, bh);
+      mma_tf32(acc[nt][1], ah, bl);
+      mma_tf32(acc[nt][2], al, bh);
+    }
+  }
+}
+__device__ __forceinline__ void acc_zero(float (&acc)[2][3][4]) {
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][k][e] = 0.f;
+}
+// Sums the three partial products, times `sign`, into the accumulator layout
+// (res[nt] = rows g, g, g+8, g+8 x columns nt*8 + 2q, +1, 2q, +1).
+__device__ __forceinline__ void acc_sum(float (&res)[2][4], const float (&acc)[2][3][4], float sign) {
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) res[nt][e] = sign * (acc[nt][0][e] + (acc[nt][1][e] + acc[nt][2][e]));
+}
+__device__ __forceinline__ void store_res(float* blkp, const float (&res)[2][4], int g, int q) {
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    *reinterpret_cast<float2*>(blkp + g * BLK_LD + nt * 8 + 2 * q) = make_float2(res[nt][0], res[nt][1]);
+    *reinterpret_cast<float2*>(blkp + (g + 8) * BLK_LD + nt * 8 + 2 * q) = make_float2(res[nt][2], res[nt][3]);
+  }
+}
+// T block (a, b) from the accumulator layout into the bf16 operands
+// T1 = T diag(b gamma) and T2 = T diag(b).
+__device__ __forceinline__ void store_res_t12(uint8_t* sm, const Gates& G, int a, int b,
+                                              const float (&res)[2][4], int g, int q) {
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const int col = b * 16 + nt * 8 + 2 * q;
+    const float2 bg = *reinterpret_cast<const float2*>(G.bg + col);
+    const float2 bb = *reinterpret_cast<const float2*>(G.b + col);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = a * 16 + g + 8 * h;
+      const float x0 = res[nt][2 * h], x1 = res[nt][2 * h + 1];
+      *reinterpret_cast<uint32_t*>(sm + OFF_T1 + sw128_offset(row, col)) = pack_bf16x2(x0 * bg.x, x1 * bg.y);
+      *reinterpret_cast<uint32_t*>(sm + OFF_T2 + sw128_offset(row, col)) = pack_bf16x2(x0 * bb.x, x1 * bb.y);
+    }
+  }
 }
 
-// Gate inputs of one token (threads 0-63 of the prep warpgroup): log a and b,
-// or 0 past the sequence end.  Issued one chunk ahead so the global-memory
-// latency is hidden behind the current chunk.
+// Gate inputs of one token (threads 0-63 of the prep warpgroup): a and b, or
+// a = 1, b = 0 past the sequence end.  Issued one chunk ahead so the
+// global-memory latency is hidden behind the current chunk.
 __device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int valid, int h, int t,
-                                                 float& la, float& bb) {
-  la = 0.f;
+                                                 float& a_in, float& bb) {
+  a_in = 1.f;
   bb = 0.f;
   if (t < valid) {
     const size_t ti = (size_t)(tok0 + t) * p.H + h;
-    la = __ldg(p.a + ti);
+    a_in = __ldg(p.a + ti);
     bb = __ldg(p.b + ti);
   }
 }
 
 // Gate vectors of one chunk (all 128 prep threads call this; threads 0-63 own
-// one token each).  Rows past the sequence end get log a = 0 and b = 0.
-__device__ __forceinline__ void compute_gates(Gates G, float* s_carry, float* s_dec, int valid,
-                                              int t, float a_in, float bb) {
+// one token each).  Rows past the sequence end get a = 1 and b = 0.
+__device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid, int t, float a_in,
+                                              float bb) {
   const int lane = t & 31;
   float la = 0.f;
   if (t < C) {
-    la = (t < valid) ? logf(a_in) : 0.f;
+    la = (t < valid) ? log2f(a_in) : 0.f;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const float y = __shfl_up_sync(0xffffffffu, la, off);
@@ -294,115 +366,131 @@ __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, float* s_
   wg_sync<BAR_PREP>();
   if (t < C) {
     if (t >= 32) la += *s_carry;
-    G.g[t] = la;
+    G.g2[t] = la;
   }
   wg_sync<BAR_PREP>();
   if (t < C) {
-    const float gC = G.g[C - 1];
-    const float gam = exp_nonpos(la);
+    const float gam = ex2_approx(la);
     G.gamma[t] = gam;
-    G.bg[t] = G.b[t] * gam;
-    G.r[t] = exp_nonpos(gC - la);
-    s_dec[t] = exp_nonpos(la - G.g[t & ~15]);                         // e_i
-  }
-  // F[I-1][j] = exp(g_16I - g_j) for j < 16I: 96 entries
-  for (int u = t; u < 96; u += WG) {
-    const int I = (u < 16) ? 1 : (u < 48 ? 2 : 3);
-    const int jj = u - (I == 1 ? 0 : (I == 2 ? 16 : 48));
-    s_dec[64 + (I - 1) * 64 + jj] = exp_nonpos(G.g[16 * I] - G.g[jj]);
-  }
-  // Dd[I][r][c] = exp(g_{16I+r} - g_{16I+c}) for c <= r
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int u = t + k * WG;
-    const int I = u >> 8, r = (u >> 4) & 15, cc = u & 15;
-    s_dec[256 + u] = (cc <= r) ? exp_nonpos(G.g[16 * I + r] - G.g[16 * I + cc]) : 0.f;
+    G.bg[t] = bb * gam;
+    G.r[t] = ex2_approx(G.g2[C - 1] - la);
   }
 }
 
-// T = (I + A)^{-1} for the strictly lower 64 x 64 matrix A (fp32, row stride
-// A_LD), blocked by 16.  The diagonal blocks are inverted by forward
-// substitution (one column per thread); the off-diagonal blocks follow by
-// block distance D: T_{b+D,b} = -T_{b+D,b+D} sum_{m=b}^{b+D-1} A_{b+D,m} T_{m,b}.
-// s_T receives T (swizzled by tix(); its upper block triangle is left unset);
-// s_Y is 3 x 16 x 17 fp32 scratch.  All prep threads take part.
-template <int D>
-__device__ __forceinline__ void offdiag_level(const float* s_A, float* s_T, float* s_Y, int t) {
-  constexpr int NB = 4 - D;
+// T = (I + A)^{-1} for the strictly lower 64 x 64 matrix A, both in compact
+// block form.  The diagonal blocks are inverted by forward substitution (one
+// column per thread); the rest follows by recursive doubling of the 2 x 2
+// block inverse [[L1, 0], [M, L2]]^{-1} = [[L1^-1, 0], [-L2^-1 M L1^-1, L2^-1]]:
+// first the 16-blocks (1,0) and (3,2), then the 32 x 32 block below the
+// diagonal as Y = A_21 T_top, T_21 = -T_bot Y.  Every T block is also written,
+// rounded to bf16 and column-scaled, into the T1 and T2 operand tiles (their
+// upper block triangle is zero from the start).  All prep threads take part.
+__device__ __forceinline__ void solve_t(uint8_t* sm, const Gates& G, const float* s_A, float* s_T,
+                                        int t) {
   const int warp = t >> 5, lane = t & 31;
-  const int g = lane >> 2, q = lane & 3;   // mma fragment coordinates
-  if (warp < NB) {
-    const int bb = warp;                   // block column; this warp fills T_{bb+D, bb}
-    const int rA = (bb + D) * 16;
-    // Y = sum_{m=bb}^{bb+D-1} A_{bb+D,m} T_{m,bb}   (16 x 16, K = 16 D)
-    float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int k0 = 0; k0 < 16 * D; k0 += 8) {
-      const int ca = bb * 16 + k0;
-      const float a[4] = {s_A[(rA + g) * A_LD + ca + q], s_A[(rA + g + 8) * A_LD + ca + q],
-                          s_A[(rA + g) * A_LD + ca + q + 4], s_A[(rA + g + 8) * A_LD + ca + q + 4]};
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int cb = bb * 16 + nt * 8 + g;
-        const float b[2] = {s_T[tix(ca + q, cb)], s_T[tix(ca + q + 4, cb)]};
-        mma_3xtf32(y[nt], a, b);
-      }
-    }
-    float* Yb = s_Y + bb * 16 * 17;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      Yb[g * 17 + nt * 8 + 2 * q] = y[nt][0];
-      Yb[g * 17 + nt * 8 + 2 * q + 1] = y[nt][1];
-      Yb[(g + 8) * 17 + nt * 8 + 2 * q] = y[nt][2];
-      Yb[(g + 8) * 17 + nt * 8 + 2 * q + 1] = y[nt][3];
-    }
-    __syncwarp();
-    // T_{bb+D, bb} = -T_{bb+D, bb+D} Y   (16 x 16, K = 16)
-    float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int k0 = 0; k0 < 16; k0 += 8) {
-      const float a[4] = {s_T[tix(rA + g, rA + k0 + q)], s_T[tix(rA + g + 8, rA + k0 + q)],
-                          s_T[tix(rA + g, rA + k0 + q + 4)], s_T[tix(rA + g + 8, rA + k0 + q + 4)]};
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const float b[2] = {Yb[(k0 + q) * 17 + nt * 8 + g], Yb[(k0 + q + 4) * 17 + nt * 8 + g]};
-        mma_3xtf32(z[nt], a, b);
-      }
-    }
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int cc = bb * 16 + nt * 8 + 2 * q;
-      s_T[tix(rA + g, cc)] = -z[nt][0];
-      s_T[tix(rA + g, cc + 1)] = -z[nt][1];
-      s_T[tix(rA + g + 8, cc)] = -z[nt][2];
-      s_T[tix(rA + g + 8, cc + 1)] = -z[nt][3];
-    }
-  }
-  wg_sync<BAR_PREP>();
-}
-
-__device__ __forceinline__ void invert_unit_lower_64(const float* s_A, float* s_T, float* s_Y, int t) {
+  const int g = lane >> 2, q = lane & 3;
   if (t < 64) {
-    const int r0 = (t >> 4) * 16, c = t & 15;
+    const int a = t >> 4, c = t & 15;
+    const float* Ad = s_A + blk(a, a);
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       float acc0 = (i == c) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
       for (int m = 0; m + 1 < i; m += 2) {
-        acc0 = fmaf(-s_A[(r0 + i) * A_LD + r0 + m], x[m], acc0);
-        acc1 = fmaf(-s_A[(r0 + i) * A_LD + r0 + m + 1], x[m + 1], acc1);
+        acc0 = fmaf(-Ad[i * BLK_LD + m], x[m], acc0);
+        acc1 = fmaf(-Ad[i * BLK_LD + m + 1], x[m + 1], acc1);
       }
-      if (i & 1) acc0 = fmaf(-s_A[(r0 + i) * A_LD + r0 + i - 1], x[i - 1], acc0);
+      if (i & 1) acc0 = fmaf(-Ad[i * BLK_LD + i - 1], x[i - 1], acc0);
       x[i] = acc0 + acc1;
     }
+    float* Td = s_T + blk(a, a);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s_T[tix(r0 + i, r0 + c)] = x[i];
+    for (int i = 0; i < 16; ++i) Td[i * BLK_LD + c] = x[i];
   }
   wg_sync<BAR_PREP>();
-  offdiag_level<1>(s_A, s_T, s_Y, t);
-  offdiag_level<2>(s_A, s_T, s_Y, t);
-  offdiag_level<3>(s_A, s_T, s_Y, t);
+  if (warp < 2) {
+    // T_{a+1,a} = -T_{a+1,a+1} (A_{a+1,a} T_{a,a}),  a = 0, 2
+    const int a = warp * 2;
+    float* out = s_T + blk(a + 1, a);
+    float fa[2][4], fb[2][2][2], acc[2][3][4], res[2][4];
+    frag_a(fa, s_A + blk(a + 1, a), g, q);
+    frag_b(fb, s_T + blk(a, a), g, q);
+    acc_zero(acc);
+    mma_blk(acc, fa, fb);
+    acc_sum(res, acc, 1.f);
+    store_res(out, res, g, q);        // Y, kept in the output block until it is replaced
+    __syncwarp();
+    frag_a(fa, s_T + blk(a + 1, a + 1), g, q);
+    frag_b(fb, out, g, q);
+    __syncwarp();
+    acc_zero(acc);
+    mma_blk(acc, fa, fb);
+    acc_sum(res, acc, -1.f);
+    store_res(out, res, g, q);
+    store_res_t12(sm, G, a + 1, a, res, g, q);
+  } else {
+    // meanwhile: the diagonal blocks into T1 and T2 (one row half per item)
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int u = (t - 64) + k * 64;         // 0..127
+      const int a = u >> 5, r = (u >> 1) & 15, half = u & 1;
+      const float* src = s_T + blk(a, a) + r * BLK_LD + half * 8;
+      const float4 x0 = *reinterpret_cast<const float4*>(src);
+      const float4 x1 = *reinterpret_cast<const float4*>(src + 4);
+      const int col = a * 16 + half * 8, row = a * 16 + r;
+      const float4 bg0 = *reinterpret_cast<const float4*>(G.bg + col);
+      const float4 bg1 = *reinterpret_cast<const float4*>(G.bg + col + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(G.b + col);
+      const float4 b1 = *reinterpret_cast<const float4*>(G.b + col + 4);
+      uint4 o1, o2;
+      o1.x = pack_bf16x2(x0.x * bg0.x, x0.y * bg0.y);
+      o1.y = pack_bf16x2(x0.z * bg0.z, x0.w * bg0.w);
+      o1.z = pack_bf16x2(x1.x * bg1.x, x1.y * bg1.y);
+      o1.w = pack_bf16x2(x1.z * bg1.z, x1.w * bg1.w);
+      o2.x = pack_bf16x2(x0.x * b0.x, x0.y * b0.y);
+      o2.y = pack_bf16x2(x0.z * b0.z, x0.w * b0.w);
+      o2.z = pack_bf16x2(x1.x * b1.x, x1.y * b1.y);
+      o2.w = pack_bf16x2(x1.z * b1.z, x1.w * b1.w);
+      *reinterpret_cast<uint4*>(sm + OFF_T1 + sw128_offset(row, col)) = o1;
+      *reinterpret_cast<uint4*>(sm + OFF_T2 + sw128_offset(row, col)) = o2;
+    }
+  }
+  wg_sync<BAR_PREP>();
+  // Y_{a,b} = sum_{k=b}^{1} A_{a,k} T_{k,b}  (a = 2, 3; b = 0, 1), into block (a, b)
+  const int a2 = 2 + (warp >> 1), b2 = warp & 1;
+  {
+    float fa[2][4], fb[2][2][2], acc[2][3][4], res[2][4];
+    acc_zero(acc);
+    frag_a(fa, s_A + blk(a2, 1), g, q);
+    frag_b(fb, s_T + blk(1, b2), g, q);
+    mma_blk(acc, fa, fb);
+    if (b2 == 0) {
+      frag_a(fa, s_A + blk(a2, 0), g, q);
+      frag_b(fb, s_T + blk(0, 0), g, q);
+      mma_blk(acc, fa, fb);
+    }
+    acc_sum(res, acc, 1.f);
+    store_res(s_T + blk(a2, b2), res, g, q);
+  }
+  wg_sync<BAR_PREP>();
+  // T_{a,b} = -sum_{m=2}^{a} T_{a,m} Y_{m,b}
+  {
+    float fa0[2][4], fb0[2][2][2], fa1[2][4], fb1[2][2][2], acc[2][3][4], res[2][4];
+    frag_a(fa0, s_T + blk(a2, a2), g, q);
+    frag_b(fb0, s_T + blk(a2, b2), g, q);
+    if (a2 == 3) {
+      frag_a(fa1, s_T + blk(3, 2), g, q);
+      frag_b(fb1, s_T + blk(2, b2), g, q);
+    }
+    wg_sync<BAR_PREP>();                   // every Y is read before any is replaced
+    acc_zero(acc);
+    mma_blk(acc, fa0, fb0);
+    if (a2 == 3) mma_blk(acc, fa1, fb1);
+    acc_sum(res, acc, -1.f);
+    store_res(s_T + blk(a2, b2), res, g, q);
+    store_res_t12(sm, G, a2, b2, res, g, q);
+  }
 }
 
 // Sigma^T row j (fp32, in tensor memory) -> bf16 operand tile for the next
@@ -533,9 +621,12 @@ __global__ void __maxnreg__(224)
     const int t = tid;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float* s_A = reinterpret_cast<float*>(sm + OFF_A);
-    float* s_T = reinterpret_cast<float*>(sm + OFF_T1);
-    float* s_Y = reinterpret_cast<float*>(sm + OFF_Y);
-    float* s_dec = reinterpret_cast<float*>(sm + OFF_DEC);
+    float* s_T = reinterpret_cast<float*>(sm + OFF_TS);
+    {
+      // the upper block triangle of T1 and T2 stays zero for the whole sequence
+      uint4* z = reinterpret_cast<uint4*>(sm + OFF_T1);
+      for (int u = t; u < 2 * 8192 / 16; u += WG) z[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
     uint32_t pphase = 0;
     float a_in = 1.f, b_in = 0.f;
     if (n_chunks > 0) load_gate_inputs(p, seq_start, min(C, len), h, t, a_in, b_in);
@@ -550,7 +641,7 @@ __global__ void __maxnreg__(224)
 
       // ---- gates of chunk c (the buffer's previous user, chunk c-3, is finished);
       // the next chunk's inputs are fetched now and used one iteration later
-      compute_gates(G, s_carry, s_dec, valid, t, a_in, b_in);
+      compute_gates(G, s_carry, valid, t, a_in, b_in);
       if (c + 1 < n_chunks) load_gate_inputs(p, tok0 + C, min(C, seq_end - tok0 - C), h, t, a_in, b_in);
       wg_sync<BAR_PREP>();
       if (t == 0) mbar_arrive(&bars[B_GATES + c % 3]);
@@ -583,67 +674,55 @@ __global__ void __maxnreg__(224)
           !wg_wait<BAR_PREP>(&bars[B_CHUNK_DONE + s], ((c >> 1) - 1) & 1, s_abort, p.status))
         break;
       {
-        // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32) and
-        // P = tril(D o Q K^T) (rows 64-127, bf16 operand), 32 columns of G at a time
-        // D_ij = e_i F[I-1][j] below the diagonal block (I = i / 16), Dd[I][i-16I][j-16I]
-        // inside it, 0 above; all factors were tabulated with the gates.
+        // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32, compact blocks) and
+        // P = tril(D o Q K^T) (rows 64-127, bf16 operand), D_ij = 2^(g2_i - g2_j).
+        // Thread t owns row i of its half; warps 0 and 2 hold rows 0-31, whose
+        // columns 32-63 are all zero.
         const int i = t & 63;
-        const int I = i >> 4;
-        const float ei = s_dec[i];
-        const float* Frow = s_dec + 64 + (I > 0 ? I - 1 : 0) * 64;
-        const float* Ddr = s_dec + 256 + I * 256 + (i & 15) * 16;
-        uint8_t* pt = sm + OFF_P + s * 8192;
+        const bool hi = (warp & 1) != 0;
+        const float gi = G.g2[i];
+        const float sc = (t < C) ? G.b[i] : 1.f;
+        const int lim = (t < C) ? i : i + 1;          // columns j < lim are kept
         float gr[64];
         tmem_ld64(tmem + lane_off + COL_GW, gr);
 #pragma unroll
-        for (int jj = 0; jj < C; ++jj) {
-          const int bj = jj >> 4;
-          float dv_ = 0.f;
-          if (bj < I) dv_ = ei * Frow[jj];
-          else if (bj == I) dv_ = Ddr[jj & 15];
-          gr[jj] *= dv_;
+        for (int j4 = 0; j4 < 16; ++j4) {
+          if (j4 < 8 || hi) {
+            const float4 gj = *reinterpret_cast<const float4*>(G.g2 + 4 * j4);
+            const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int jj = 4 * j4 + e;
+              const float d = ex2_approx(gi - gjv[e]);
+              gr[jj] = (jj < lim) ? (sc * gr[jj]) * d : 0.f;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) gr[4 * j4 + e] = 0.f;
+          }
         }
         if (t < C) {
-          const float bi = G.b[i];
+          const int I = i >> 4;
+          float* arow = s_A + (i & 15) * BLK_LD;
 #pragma unroll
-          for (int jj = 0; jj < C; ++jj) s_A[i * A_LD + jj] = (jj < i) ? bi * gr[jj] : 0.f;
+          for (int bj = 0; bj < 4; ++bj) {
+            if (bj <= I) {
+              float4* dst = reinterpret_cast<float4*>(arow + blk(I, bj));
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                dst[k] = make_float4(gr[16 * bj + 4 * k], gr[16 * bj + 4 * k + 1], gr[16 * bj + 4 * k + 2],
+                                     gr[16 * bj + 4 * k + 3]);
+            }
+          }
         } else {
-          store_row64_bf16(pt, i, gr);
+          store_row64_bf16(sm + OFF_P + s * 8192, i, gr);
         }
       }
       tc_fence_before();
       wg_sync<BAR_PREP>();
 
-      // ---- T = (I + A)^{-1}, then T1 = T diag(b gamma), T2 = T diag(b) (bf16, over the T scratch)
-      invert_unit_lower_64(s_A, s_T, s_Y, t);
-      {
-        float tv[4][8];
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int it = t + k4 * WG;
-          const int i = it >> 3, q8 = (it & 7) * 8;
-          const bool zero = ((q8 >> 4) > (i >> 4));
-#pragma unroll
-          for (int e = 0; e < 8; ++e) tv[k4][e] = zero ? 0.f : s_T[tix(i, q8 + e)];
-        }
-        wg_sync<BAR_PREP>();
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int it = t + k4 * WG;
-          const int i = it >> 3, q8 = (it & 7) * 8;
-          uint4 o1, o2;
-          o1.x = pack_bf16x2(tv[k4][0] * G.bg[q8 + 0], tv[k4][1] * G.bg[q8 + 1]);
-          o1.y = pack_bf16x2(tv[k4][2] * G.bg[q8 + 2], tv[k4][3] * G.bg[q8 + 3]);
-          o1.z = pack_bf16x2(tv[k4][4] * G.bg[q8 + 4], tv[k4][5] * G.bg[q8 + 5]);
-          o1.w = pack_bf16x2(tv[k4][6] * G.bg[q8 + 6], tv[k4][7] * G.bg[q8 + 7]);
-          o2.x = pack_bf16x2(tv[k4][0] * G.b[q8 + 0], tv[k4][1] * G.b[q8 + 1]);
-          o2.y = pack_bf16x2(tv[k4][2] * G.b[q8 + 2], tv[k4][3] * G.b[q8 + 3]);
-          o2.z = pack_bf16x2(tv[k4][4] * G.b[q8 + 4], tv[k4][5] * G.b[q8 + 5]);
-          o2.w = pack_bf16x2(tv[k4][6] * G.b[q8 + 6], tv[k4][7] * G.b[q8 + 7]);
-          *reinterpret_cast<uint4*>(sm + OFF_T1 + sw128_offset(i, q8)) = o1;
-          *reinterpret_cast<uint4*>(sm + OFF_T2 + sw128_offset(i, q8)) = o2;
-        }
-      }
+      // ---- T = (I + A)^{-1}, written as T1 = T diag(b gamma), T2 = T diag(b) (bf16)
+      solve_t(sm, G, s_A, s_T, t);
       fence_proxy_async_smem();
       wg_sync<BAR_PREP>();
 

@@ -76,28 +76,78 @@ def profiled_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during a timed region."""
+    """SM clock and clock-event reasons sampled during a timed region.
 
+    NVML is polled every `period_s` from a background thread (the timed regions
+    here last milliseconds, too short for nvidia-smi's start-up); the device is
+    matched to the CUDA device by PCI location.  nvidia-smi -lms is the fallback
+    when NVML is unavailable."""
+
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    _NVML_NAMES = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+                   "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+                   "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+                   "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, cuda_index: int, period_s: float = 0.002):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.samples = []      # (sm_mhz, reason bitmask or set of names)
+        self.max_mhz = None
         self.proc = None
+        self.thread = None
+
+    def _nvml_handle(self, nv):
+        import torch
+        props = torch.cuda.get_device_properties(self.cuda_index)
+        want = (getattr(props, "pci_domain_id", None), getattr(props, "pci_bus_id", None),
+                getattr(props, "pci_device_id", None))
+        for i in range(nv.nvmlDeviceGetCount()):
+            h = nv.nvmlDeviceGetHandleByIndex(i)
+            pci = nv.nvmlDeviceGetPciInfo(h)
+            if (pci.domain, pci.bus, pci.device) == want:
+                return h
+        return None
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._nvml_handle(nv)
+            if h is None:
+                raise RuntimeError("no NVML device matches the CUDA device")
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            masks = {n: getattr(nv, a) for n, a in self._NVML_NAMES.items()}
+            self.stop = threading.Event()
+
+            def poll():
+                while not self.stop.is_set():
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((float(sm), {n for n, m in masks.items() if r & m}))
+                    self.stop.wait(self.period)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
         except Exception:
-            self.proc = None
+            self.thread = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.cuda_index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                self.proc = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -105,27 +155,26 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            for line in out.splitlines():
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, self.max_mhz = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                self.samples.append((sm, {n for n, v in zip(self.REASONS, parts[5:9])
+                                          if v.lower() == "active"}))
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 def dist_setup(n_gpus: int):
@@ -357,11 +406,12 @@ def bench_prefill_workload(wl, dev, args, peaks, world):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     n = max(1, args.steps)
-    e0.record(stream)
-    for _ in range(n):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        e0.record(stream)
+        for _ in range(n):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
     t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n
     tokens = inp["total_tokens"]
     bytes_launch = (prefill_bytes_per_token_head(wl.dk, wl.dv) * tokens * wl.H
@@ -371,7 +421,7 @@ def bench_prefill_workload(wl, dev, args, peaks, world):
     res = {"tokens_per_s": world * tokens / t, "ms_per_step": t * 1e3, "loops": wl.loops,
            "tokens": tokens, "heads": wl.H, "dk": wl.dk, "dv": wl.dv,
            "achieved_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
-           "algorithmic_bytes_per_launch": bytes_launch}
+           "algorithmic_bytes_per_launch": bytes_launch, "clocks": clocks.summary()}
     del inp, o, ST
     return res
 
@@ -395,17 +445,18 @@ def bench_decode(wl, dev, args, peaks, world):
     n = max(1, args.steps)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        e0.record(stream)
+        for _ in range(n):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
     t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n
     nbytes = decode_bytes_per_head_state(wl.dk, wl.dv) * wl.n_seq * wl.H
     gbs = nbytes / t / 1e9
     res = {"state_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"], "ms_per_step": t * 1e3,
            "seq_tokens_per_s": world * 256 / t * 1.0, "slots": wl.n_seq, "heads": wl.H,
-           "bytes_per_step": nbytes,
+           "bytes_per_step": nbytes, "clocks": clocks.summary(),
            "note": "one step = one token for 256 sequences x 24 layers x 4 loops (all slots)"}
     del inp, o
     return res

@@ -61,12 +61,17 @@ constexpr int BAR_PREP = 1;      // named barriers of the two warpgroups
 constexpr int BAR_STATE = 2;
 
 // tensor-memory columns (fp32 accumulators, lane = row)
-constexpr uint32_t COL_GW = 0;    // [K;Q] K^T, then W^T, of the prep chunk    128 x 64
+constexpr uint32_t COL_GW = 0;    // [K;Q] K^T, then W^T, of a prep chunk      2 x 128 x 64 (0, 320)
 constexpr uint32_t COL_U = 64;    // U^T, two buffers (chunk parity)           2 x 128 x 64
 constexpr uint32_t COL_OA = 192;  // Sigma^T Q^T                                128 x 64
 constexpr uint32_t COL_OB = 256;  // U^T P^T                                    128 x 64
+constexpr uint32_t COL_GW1 = 320; // second G / W^T buffer                      128 x 64
 constexpr uint32_t COL_S = 384;   // Sigma^T fp32 (kept pre-decayed by gamma_C) 128 x 128
 constexpr uint32_t TMEM_COLS = 512;
+static_assert(COL_GW + 64 <= COL_U && COL_U + 128 <= COL_OA && COL_OA + 64 <= COL_OB &&
+                  COL_OB + 64 <= COL_GW1 && COL_GW1 + 64 <= COL_S && COL_S + 128 <= TMEM_COLS,
+              "tensor-memory regions overlap");
+__device__ __forceinline__ uint32_t col_gw(int c) { return (c & 1) ? COL_GW1 : COL_GW; }
 
 // Shared-memory plan (offsets from a 1024-byte aligned base).
 constexpr uint32_t OFF_KQ = 0;            // 2 stages x 32 KB: [K0|Q0|K1|Q1] 8 KB slabs
@@ -103,13 +108,14 @@ static_assert(OFF_GATE % 16 == 0 && (BLK_FLOATS * 4) % 16 == 0, "vector access a
 enum : int {
   B_KQ_FULL = 0,      // [2] TMA K, Q landed
   B_V_FULL = 2,       //     TMA V landed
-  B_GATES = 3,        // [3] prep: gate vectors of a chunk written
+  B_GATES = 3,        // [3] state: gate vectors of a chunk written
   B_W_READY = 6,      //     prep: W^T tile written, U~ in tensor memory
   B_W_CONSUMED = 7,   //     state: U MMA done, W^T tile free
   B_CHUNK_DONE = 8,   // [2] state: chunk finished (U and P buffers free)
-  B_PREP_MMA = 10,    //     commits of the prep warpgroup
+  B_PREP_MMA = 10,    //     prep: U~ and W^T products done
   B_STATE_MMA = 11,   //     commits of the state warpgroup
-  NBAR = 12
+  B_G_MMA = 12,       // [2] prep: G of a chunk done (by tensor-memory buffer)
+  NBAR = 14
 };
 
 struct Params {
@@ -333,9 +339,9 @@ __device__ __forceinline__ void store_res_t12(uint8_t* sm, const Gates& G, int a
   }
 }
 
-// Gate inputs of one token (threads 0-63 of the prep warpgroup): a and b, or
-// a = 1, b = 0 past the sequence end.  Issued one chunk ahead so the
-// global-memory latency is hidden behind the current chunk.
+// Gate inputs of one token (threads 0-63 of the state warpgroup): a and b, or
+// a = 1, b = 0 past the sequence end.  Issued well before they are used so the
+// global-memory latency is hidden behind a chunk.
 __device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int valid, int h, int t,
                                                  float& a_in, float& bb) {
   a_in = 1.f;
@@ -347,8 +353,9 @@ __device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int 
   }
 }
 
-// Gate vectors of one chunk (all 128 prep threads call this; threads 0-63 own
-// one token each).  Rows past the sequence end get a = 1 and b = 0.
+// Gate vectors of one chunk (all 128 threads of a warpgroup call this; threads
+// 0-63 own one token each).  Rows past the sequence end get a = 1 and b = 0.
+template <int BAR>
 __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid, int t, float a_in,
                                               float bb) {
   const int lane = t & 31;
@@ -363,12 +370,12 @@ __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid
     if (t == 31) *s_carry = la;
     G.b[t] = bb;
   }
-  wg_sync<BAR_PREP>();
+  wg_sync<BAR>();
   if (t < C) {
     if (t >= 32) la += *s_carry;
     G.g2[t] = la;
   }
-  wg_sync<BAR_PREP>();
+  wg_sync<BAR>();
   if (t < C) {
     const float gam = ex2_approx(la);
     G.gamma[t] = gam;
@@ -551,13 +558,11 @@ __global__ void __maxnreg__(224)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
-  float* s_carry = reinterpret_cast<float*>(sm + OFF_MISC + 8);
   // loads issued so far: K/Q per stage, V (read back to drain in-flight copies on exit)
   volatile int* s_issued = reinterpret_cast<volatile int*>(sm + OFF_MISC + 16);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
-  const int lane = tid & 31;
 
   // work unit
   const int slice = blockIdx.x % p.n_slices;
@@ -628,48 +633,43 @@ __global__ void __maxnreg__(224)
       for (int u = t; u < 2 * 8192 / 16; u += WG) z[u] = make_uint4(0u, 0u, 0u, 0u);
     }
     uint32_t pphase = 0;
-    float a_in = 1.f, b_in = 0.f;
-    if (n_chunks > 0) load_gate_inputs(p, seq_start, min(C, len), h, t, a_in, b_in);
-#pragma unroll 1
-    for (int c = 0; c < n_chunks; ++c) {
+    // K, Q of chunk c (optional in-place L2 norm), then G = [K; Q] K^T into
+    // tensor-memory buffer c % 2 (M = 128, N = 64, K = dk).  Issued one chunk
+    // ahead so the product runs while the previous chunk's W^T is converted.
+    auto issue_g = [&](int c) -> bool {
       const int s = c & 1;
-      const int tok0 = seq_start + c * C;
-      const int valid = min(C, seq_end - tok0);
-      const Gates G = gates_at(sm, c % 3);
-      uint8_t* kq = sm + OFF_KQ + s * KQ_BYTES;
-      const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
-
-      // ---- gates of chunk c (the buffer's previous user, chunk c-3, is finished);
-      // the next chunk's inputs are fetched now and used one iteration later
-      compute_gates(G, s_carry, valid, t, a_in, b_in);
-      if (c + 1 < n_chunks) load_gate_inputs(p, tok0 + C, min(C, seq_end - tok0 - C), h, t, a_in, b_in);
-      wg_sync<BAR_PREP>();
-      if (t == 0) mbar_arrive(&bars[B_GATES + c % 3]);
-
-      // ---- K, Q of chunk c; optional in-place L2 norm
-      if (!wg_wait<BAR_PREP>(&bars[B_KQ_FULL + s], (c >> 1) & 1, s_abort, p.status)) break;
+      if (!wg_wait<BAR_PREP>(&bars[B_KQ_FULL + s], (c >> 1) & 1, s_abort, p.status)) return false;
       if (p.flags & GDN_QK_L2NORM) {
-        l2norm_row(kq, t & 63, t < 64 ? 0u : 8192u);   // rows 0-63: K, rows 64-127: Q
+        l2norm_row(sm + OFF_KQ + s * KQ_BYTES, t & 63, t < 64 ? 0u : 8192u);   // rows 0-63: K, 64-127: Q
         fence_proxy_async_smem();
         wg_sync<BAR_PREP>();
       }
-
-      // ---- G = [K; Q] K^T   (M = 128, N = 64, K = dk)
       if (t == 0) {
         tc_fence_after();
+        const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + COL_GW, kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
+          mma_bf16(tmem + col_gw(c), kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
                    kk > 0);
         }
-        mma_commit(&bars[B_PREP_MMA]);
+        mma_commit(&bars[B_G_MMA + s]);
       }
-      if (!wg_wait<BAR_PREP>(&bars[B_PREP_MMA], pphase, s_abort, p.status)) break;
-      pphase ^= 1;
-      tc_fence_after();
+      return true;
+    };
+    bool ok = (n_chunks == 0) || issue_g(0);
+#pragma unroll 1
+    for (int c = 0; c < n_chunks && ok; ++c) {
+      const int s = c & 1;
+      const int tok0 = seq_start + c * C;
+      const Gates G = gates_at(sm, c % 3);
+      const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
 
-      // ---- P buffer s and U buffer s are free once chunk c-2 is finished
+      // ---- G of chunk c, its gates (from the state warpgroup), and the P and U
+      // buffers s (free once chunk c-2 is finished)
+      if (!wg_wait<BAR_PREP>(&bars[B_G_MMA + s], (c >> 1) & 1, s_abort, p.status)) break;
+      tc_fence_after();
+      if (!wg_wait<BAR_PREP>(&bars[B_GATES + c % 3], (c / 3) & 1, s_abort, p.status)) break;
       if (c >= 2 &&
           !wg_wait<BAR_PREP>(&bars[B_CHUNK_DONE + s], ((c >> 1) - 1) & 1, s_abort, p.status))
         break;
@@ -684,7 +684,7 @@ __global__ void __maxnreg__(224)
         const float sc = (t < C) ? G.b[i] : 1.f;
         const int lim = (t < C) ? i : i + 1;          // columns j < lim are kept
         float gr[64];
-        tmem_ld64(tmem + lane_off + COL_GW, gr);
+        tmem_ld64(tmem + lane_off + col_gw(c), gr);
 #pragma unroll
         for (int j4 = 0; j4 < 16; ++j4) {
           if (j4 < 8 || hi) {
@@ -735,11 +735,13 @@ __global__ void __maxnreg__(224)
         for (int kk = 0; kk < C / 16; ++kk) {
           mma_bf16(tmem + COL_U + s * 64, mndesc(v_a + kk * 2048, 8192),
                    kdesc(sbase + OFF_T2 + kk * 32), idesc_bf16(128, 64, 1, 0), kk > 0);
-          mma_bf16(tmem + COL_GW, mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
+          mma_bf16(tmem + col_gw(c), mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
                    idesc_bf16(128, 64, 1, 0), kk > 0);
         }
         mma_commit(&bars[B_PREP_MMA]);
       }
+      // ---- next chunk's G, queued behind these products
+      if (c + 1 < n_chunks && !issue_g(c + 1)) break;
       if (!wg_wait<BAR_PREP>(&bars[B_PREP_MMA], pphase, s_abort, p.status)) break;
       pphase ^= 1;
       tc_fence_after();
@@ -752,7 +754,7 @@ __global__ void __maxnreg__(224)
       if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
       {
         float wr[64];
-        tmem_ld64(tmem + lane_off + COL_GW, wr);
+        tmem_ld64(tmem + lane_off + col_gw(c), wr);
         store_row64_bf16(sm + OFF_WT, t, wr);
       }
       tc_fence_before();
@@ -768,13 +770,29 @@ __global__ void __maxnreg__(224)
     uint32_t sphase = 0;
     bool ok = true;
 
-    // initial state: tensor memory holds gamma_C(0) * S0, the bf16 operand holds S0
-    float decay0 = 1.f;
+    float* s_carry = reinterpret_cast<float*>(sm + OFF_MISC + 8);
+    // gate vectors of chunks 0 and 1 (later ones are built two chunks ahead,
+    // at the end of each chunk); a_in, b_in hold the inputs of the next chunk
+    // to build
+    float a_in, b_in;
+    auto gates_of = [&](int c) {
+      compute_gates<BAR_STATE>(gates_at(sm, c % 3), s_carry, min(C, seq_end - (seq_start + c * C)), j,
+                               a_in, b_in);
+      if (c + 1 < n_chunks)
+        load_gate_inputs(p, seq_start + (c + 1) * C, min(C, seq_end - (seq_start + (c + 1) * C)), h, j,
+                         a_in, b_in);
+      wg_sync<BAR_STATE>();
+      if (j == 0) mbar_arrive(&bars[B_GATES + c % 3]);
+    };
     if (n_chunks > 0) {
-      ok = wg_wait<BAR_STATE>(&bars[B_GATES + 0], 0, s_abort, p.status);
-      decay0 = gates_at(sm, 0).gamma[C - 1];
+      load_gate_inputs(p, seq_start, min(C, len), h, j, a_in, b_in);
+      gates_of(0);
+      if (n_chunks > 1) gates_of(1);
     }
-    if (ok) {
+
+    // initial state: tensor memory holds gamma_C(0) * S0, the bf16 operand holds S0
+    const float decay0 = (n_chunks > 0) ? gates_at(sm, 0).gamma[C - 1] : 1.f;
+    {
 #pragma unroll 1
       for (int piece = 0; piece < 4; ++piece) {
         float x[32];
@@ -867,11 +885,7 @@ __global__ void __maxnreg__(224)
       }
 
       // ---- next chunk's Sigma^T operand (bf16) and pre-decayed fp32 state; S_T at the end
-      float decay = 1.f;
-      if (!last) {
-        if (!wg_wait<BAR_STATE>(&bars[B_GATES + (c + 1) % 3], ((c + 1) / 3) & 1, s_abort, p.status)) break;
-        decay = gates_at(sm, (c + 1) % 3).gamma[C - 1];
-      }
+      const float decay = last ? 1.f : gates_at(sm, (c + 1) % 3).gamma[C - 1];   // built by this warpgroup
       refresh_state(tmem + lane_off + COL_S, sm + OFF_SIG, j, decay, !last,
                     (last && p.S_T) ? p.S_T + state_base : nullptr, dv);
 
@@ -912,6 +926,9 @@ __global__ void __maxnreg__(224)
       fence_proxy_async_smem();
       wg_sync<BAR_STATE>();
       if (j == 0) mbar_arrive(&bars[B_CHUNK_DONE + s]);
+
+      // ---- gate vectors of chunk c+2 (their buffer's previous user, chunk c-1, is finished)
+      if (c + 2 < n_chunks) gates_of(c + 2);
     }
   }
 

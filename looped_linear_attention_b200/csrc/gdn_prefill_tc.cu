@@ -95,8 +95,8 @@ __device__ __forceinline__ int blk(int a, int b) { return (a * (a + 1) / 2 + b) 
 constexpr uint32_t LT_BYTES = 10 * BLK_FLOATS * 4;
 constexpr uint32_t OFF_A = 196608;                    // A, compact blocks
 constexpr uint32_t OFF_TS = OFF_A + LT_BYTES;         // T, compact blocks (also the solve's scratch)
-constexpr uint32_t OFF_GATE = OFF_TS + LT_BYTES;      // 3 buffers x {g2, gamma, b, b*gamma, gamma_C/gamma}
-constexpr uint32_t GATE_BYTES = 5 * 64 * 4;
+constexpr uint32_t OFF_GATE = OFF_TS + LT_BYTES;      // 3 buffers of gate vectors (struct Gates)
+constexpr uint32_t GATE_BYTES = 8 * 64 * 4;
 constexpr uint32_t OFF_BAR = OFF_GATE + 3 * GATE_BYTES;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;          // tmem base, abort flag, scan carry
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
@@ -109,13 +109,14 @@ enum : int {
   B_KQ_FULL = 0,      // [2] TMA K, Q landed
   B_V_FULL = 2,       //     TMA V landed
   B_GATES = 3,        // [3] state: gate vectors of a chunk written
-  B_W_READY = 6,      //     prep: W^T tile written, U~ in tensor memory
-  B_W_CONSUMED = 7,   //     state: U MMA done, W^T tile free
+  B_W_READY = 6,      //     prep: U~^T and W^T of a chunk in tensor memory
+  B_W_CONSUMED = 7,   //     state: W^T read out of tensor memory (its buffer is free)
   B_CHUNK_DONE = 8,   // [2] state: chunk finished (U and P buffers free)
   B_PREP_MMA = 10,    //     prep: U~ and W^T products done
   B_STATE_MMA = 11,   //     commits of the state warpgroup
   B_G_MMA = 12,       // [2] prep: G of a chunk done (by tensor-memory buffer)
-  NBAR = 14
+  B_OA_MMA = 14,      //     state: O_A of a chunk done
+  NBAR = 15
 };
 
 struct Params {
@@ -138,11 +139,14 @@ struct Gates {
   float* b;      // write strength (0 past the sequence end)
   float* bg;     // b * gamma
   float* r;      // gamma_C / gamma = exp(g_C - g)
+  float* e;      // 2^(g2_i - m), m = (g2_0 + g2_{C-1}) / 2 (row factor of D)
+  float* f;      // 2^(m - g2_j) (column factor of D)
+  float* flag;   // [0]: 1 when |g2_0 - g2_{C-1}| < 64, so that e_i f_j = D_ij in range
 };
 
 __device__ __forceinline__ Gates gates_at(uint8_t* sm, int buf) {
   float* base = reinterpret_cast<float*>(sm + OFF_GATE + buf * GATE_BYTES);
-  return Gates{base, base + 64, base + 128, base + 192, base + 256};
+  return Gates{base, base + 64, base + 128, base + 192, base + 256, base + 320, base + 384, base + 448};
 }
 
 // Named barrier of one warpgroup (the warp is reconverged first: the barrier is
@@ -377,59 +381,74 @@ __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid
   }
   wg_sync<BAR>();
   if (t < C) {
+    const float g0 = G.g2[0], gl = G.g2[C - 1];
+    const float mid = 0.5f * (g0 + gl);
     const float gam = ex2_approx(la);
     G.gamma[t] = gam;
     G.bg[t] = bb * gam;
-    G.r[t] = ex2_approx(G.g2[C - 1] - la);
+    G.r[t] = ex2_approx(gl - la);
+    G.e[t] = ex2_approx(la - mid);
+    G.f[t] = ex2_approx(mid - la);
+    if (t == 0) G.flag[0] = (fabsf(g0 - gl) < 64.f) ? 1.f : 0.f;
+  }
+}
+
+// x <- L^{-1} x for the unit lower 16 x 16 diagonal block L = I + A_LL of A
+// (compact block `ad`), one right-hand side per thread.  Rows of A are read 4
+// entries at a time; A's entries on and above its diagonal are stored as zeros,
+// so whole 4-vectors can be used.
+__device__ __forceinline__ void fwd_subst16(const float* ad, float (&x)[16]) {
+#pragma unroll
+  for (int i = 1; i < 16; ++i) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < i; m += 4) {
+      const float4 a4 = *reinterpret_cast<const float4*>(ad + i * BLK_LD + m);
+      acc[0] = fmaf(a4.x, x[m], acc[0]);
+      acc[1] = fmaf(a4.y, x[m + 1], acc[1]);
+      acc[2] = fmaf(a4.z, x[m + 2], acc[2]);
+      acc[3] = fmaf(a4.w, x[m + 3], acc[3]);
+    }
+    x[i] -= (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
 }
 
 // T = (I + A)^{-1} for the strictly lower 64 x 64 matrix A, both in compact
-// block form.  The diagonal blocks are inverted by forward substitution (one
-// column per thread); the rest follows by recursive doubling of the 2 x 2
-// block inverse [[L1, 0], [M, L2]]^{-1} = [[L1^-1, 0], [-L2^-1 M L1^-1, L2^-1]]:
-// first the 16-blocks (1,0) and (3,2), then the 32 x 32 block below the
-// diagonal as Y = A_21 T_top, T_21 = -T_bot Y.  Every T block is also written,
-// rounded to bf16 and column-scaled, into the T1 and T2 operand tiles (their
-// upper block triangle is zero from the start).  All prep threads take part.
+// block form, by recursive doubling of the 2 x 2 block inverse
+//     [[L1, 0], [M, L2]]^{-1} = [[L1^-1, 0], [-(L2^-1 M) L1^-1, L2^-1]].
+// Forward substitution inside the 16 x 16 diagonal blocks gives, in one pass,
+// the four T_aa = L_a^-1 and Z_{a+1,a} = L_{a+1}^-1 A_{a+1,a} for a = 0, 2;
+// then T_{a+1,a} = -Z_{a+1,a} T_aa, and the 32 x 32 block below the diagonal
+// as Y = A_21 T_top, T_21 = -T_bot Y (warp-level tf32 MMAs, 3xTF32).  Every T
+// block is also written, rounded to bf16 and column-scaled, into the T1 and T2
+// operand tiles (their upper block triangle is zero from the start).  All prep
+// threads take part.
 __device__ __forceinline__ void solve_t(uint8_t* sm, const Gates& G, const float* s_A, float* s_T,
                                         int t) {
   const int warp = t >> 5, lane = t & 31;
   const int g = lane >> 2, q = lane & 3;
-  if (t < 64) {
-    const int a = t >> 4, c = t & 15;
-    const float* Ad = s_A + blk(a, a);
+  if (t < 96) {
+    // threads 0-63: T_aa column c (a = t / 16); 64-79: Z_10 column c; 80-95: Z_32 column c
+    const int c = t & 15;
+    const int L = (t < 64) ? (t >> 4) : ((t < 80) ? 1 : 3);
+    const bool rhs_a = (t >= 64);
     float x[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float acc0 = (i == c) ? 1.f : 0.f, acc1 = 0.f;
+    for (int i = 0; i < 16; ++i)
+      x[i] = rhs_a ? s_A[blk(L, L - 1) + i * BLK_LD + c] : ((i == c) ? 1.f : 0.f);
+    fwd_subst16(s_A + blk(L, L), x);
+    float* out = s_T + (rhs_a ? blk(L, L - 1) : blk(L, L));
 #pragma unroll
-      for (int m = 0; m + 1 < i; m += 2) {
-        acc0 = fmaf(-Ad[i * BLK_LD + m], x[m], acc0);
-        acc1 = fmaf(-Ad[i * BLK_LD + m + 1], x[m + 1], acc1);
-      }
-      if (i & 1) acc0 = fmaf(-Ad[i * BLK_LD + i - 1], x[i - 1], acc0);
-      x[i] = acc0 + acc1;
-    }
-    float* Td = s_T + blk(a, a);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) Td[i * BLK_LD + c] = x[i];
+    for (int i = 0; i < 16; ++i) out[i * BLK_LD + c] = x[i];
   }
   wg_sync<BAR_PREP>();
   if (warp < 2) {
-    // T_{a+1,a} = -T_{a+1,a+1} (A_{a+1,a} T_{a,a}),  a = 0, 2
+    // T_{a+1,a} = -Z_{a+1,a} T_aa  (a = 0, 2), over Z in place
     const int a = warp * 2;
     float* out = s_T + blk(a + 1, a);
     float fa[2][4], fb[2][2][2], acc[2][3][4], res[2][4];
-    frag_a(fa, s_A + blk(a + 1, a), g, q);
+    frag_a(fa, out, g, q);
     frag_b(fb, s_T + blk(a, a), g, q);
-    acc_zero(acc);
-    mma_blk(acc, fa, fb);
-    acc_sum(res, acc, 1.f);
-    store_res(out, res, g, q);        // Y, kept in the output block until it is replaced
-    __syncwarp();
-    frag_a(fa, s_T + blk(a + 1, a + 1), g, q);
-    frag_b(fb, out, g, q);
     __syncwarp();
     acc_zero(acc);
     mma_blk(acc, fa, fb);
@@ -562,7 +581,7 @@ __global__ void __maxnreg__(224)
   volatile int* s_issued = reinterpret_cast<volatile int*>(sm + OFF_MISC + 16);
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5;
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);   // warp-uniform by construction
 
   // work unit
   const int slice = blockIdx.x % p.n_slices;
@@ -644,16 +663,19 @@ __global__ void __maxnreg__(224)
         fence_proxy_async_smem();
         wg_sync<BAR_PREP>();
       }
-      if (t == 0) {
+      if (warp == 0) {
         tc_fence_after();
         const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + col_gw(c), kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
-                   kk > 0);
+          for (int kk = 0; kk < DK / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16(tmem + col_gw(c), kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
+                     kk > 0);
+          }
+          mma_commit(&bars[B_G_MMA + s]);
         }
-        mma_commit(&bars[B_G_MMA + s]);
+        __syncwarp();
       }
       return true;
     };
@@ -675,30 +697,50 @@ __global__ void __maxnreg__(224)
         break;
       {
         // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32, compact blocks) and
-        // P = tril(D o Q K^T) (rows 64-127, bf16 operand), D_ij = 2^(g2_i - g2_j).
-        // Thread t owns row i of its half; warps 0 and 2 hold rows 0-31, whose
-        // columns 32-63 are all zero.
+        // P = tril(D o Q K^T) (rows 64-127, bf16 operand), D_ij = 2^(g2_i - g2_j),
+        // taken as e_i f_j when the chunk's decay range allows (no exponential per
+        // entry), else one exponential per entry.  Thread t owns row i of its half;
+        // warps 0 and 2 hold rows 0-31, whose columns 32-63 are all zero.
         const int i = t & 63;
         const bool hi = (warp & 1) != 0;
-        const float gi = G.g2[i];
         const float sc = (t < C) ? G.b[i] : 1.f;
         const int lim = (t < C) ? i : i + 1;          // columns j < lim are kept
         float gr[64];
         tmem_ld64(tmem + lane_off + col_gw(c), gr);
+        if (G.flag[0] != 0.f) {
+          const float sce = sc * G.e[i];
 #pragma unroll
-        for (int j4 = 0; j4 < 16; ++j4) {
-          if (j4 < 8 || hi) {
-            const float4 gj = *reinterpret_cast<const float4*>(G.g2 + 4 * j4);
-            const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+          for (int j4 = 0; j4 < 16; ++j4) {
+            if (j4 < 8 || hi) {
+              const float4 f4 = *reinterpret_cast<const float4*>(G.f + 4 * j4);
+              const float fv[4] = {f4.x, f4.y, f4.z, f4.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int jj = 4 * j4 + e;
-              const float d = ex2_approx(gi - gjv[e]);
-              gr[jj] = (jj < lim) ? (sc * gr[jj]) * d : 0.f;
+              for (int e = 0; e < 4; ++e) {
+                const int jj = 4 * j4 + e;
+                gr[jj] = (jj < lim) ? (gr[jj] * fv[e]) * sce : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) gr[4 * j4 + e] = 0.f;
             }
-          } else {
+          }
+        } else {
+          const float gi = G.g2[i];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) gr[4 * j4 + e] = 0.f;
+          for (int j4 = 0; j4 < 16; ++j4) {
+            if (j4 < 8 || hi) {
+              const float4 gj = *reinterpret_cast<const float4*>(G.g2 + 4 * j4);
+              const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int jj = 4 * j4 + e;
+                const float d = ex2_approx(gi - gjv[e]);
+                gr[jj] = (jj < lim) ? (sc * gr[jj]) * d : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) gr[4 * j4 + e] = 0.f;
+            }
           }
         }
         if (t < C) {
@@ -728,39 +770,37 @@ __global__ void __maxnreg__(224)
 
       // ---- U~^T = V^T T2^T (into U buffer s) and W^T = K^T T1^T (M = 128, N = 64, K = 64 tokens)
       if (!wg_wait<BAR_PREP>(&bars[B_V_FULL], c & 1, s_abort, p.status)) break;
-      if (t == 0) {
+      if (warp == 0) {
         tc_fence_after();
         const uint32_t v_a = sbase + OFF_V;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          mma_bf16(tmem + COL_U + s * 64, mndesc(v_a + kk * 2048, 8192),
-                   kdesc(sbase + OFF_T2 + kk * 32), idesc_bf16(128, 64, 1, 0), kk > 0);
-          mma_bf16(tmem + col_gw(c), mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
-                   idesc_bf16(128, 64, 1, 0), kk > 0);
+          for (int kk = 0; kk < C / 16; ++kk) {
+            mma_bf16(tmem + COL_U + s * 64, mndesc(v_a + kk * 2048, 8192),
+                     kdesc(sbase + OFF_T2 + kk * 32), idesc_bf16(128, 64, 1, 0), kk > 0);
+            mma_bf16(tmem + col_gw(c), mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
+                     idesc_bf16(128, 64, 1, 0), kk > 0);
+          }
+          mma_commit(&bars[B_PREP_MMA]);
         }
-        mma_commit(&bars[B_PREP_MMA]);
+        __syncwarp();
       }
-      // ---- next chunk's G, queued behind these products
-      if (c + 1 < n_chunks && !issue_g(c + 1)) break;
+      // ---- next chunk's G, queued behind these products, into the buffer that
+      // held W^T of chunk c-1 (free once the state warpgroup has read it)
+      if (c + 1 < n_chunks) {
+        if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
+        if (!issue_g(c + 1)) break;
+      }
       if (!wg_wait<BAR_PREP>(&bars[B_PREP_MMA], pphase, s_abort, p.status)) break;
       pphase ^= 1;
-      tc_fence_after();
-      if (t == 0 && c + 1 < n_chunks) {   // the V stage is free: load V of chunk c+1
-        load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, tok0 + C);
-        s_issued[2] = c + 2;
+      if (t == 0) {
+        tc_fence_before();
+        mbar_arrive(&bars[B_W_READY]);     // U~^T and W^T of chunk c are in tensor memory
+        if (c + 1 < n_chunks) {            // the V stage is free: load V of chunk c+1
+          load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, tok0 + C);
+          s_issued[2] = c + 2;
+        }
       }
-
-      // ---- W^T tile (row d = t): free once the state warpgroup's U MMA of chunk c-1 is done
-      if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
-      {
-        float wr[64];
-        tmem_ld64(tmem + lane_off + col_gw(c), wr);
-        store_row64_bf16(sm + OFF_WT, t, wr);
-      }
-      tc_fence_before();
-      fence_proxy_async_smem();
-      wg_sync<BAR_PREP>();
-      if (t == 0) mbar_arrive(&bars[B_W_READY]);
     }
   } else {
     // ================================================================ state warpgroup
@@ -832,24 +872,45 @@ __global__ void __maxnreg__(224)
       const Gates G = gates_at(sm, c % 3);
       const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
 
-      // ---- U^T -= Sigma^T W^T (onto U~^T in buffer s)  and  O_A^T = Sigma^T Q^T
+      // ---- O_A^T = Sigma^T Q^T (needs no W: it runs while W^T is converted)
       if (!wg_wait<BAR_STATE>(&bars[B_W_READY], c & 1, s_abort, p.status)) break;
-      if (j == 0) {
-        tc_fence_after();
+      tc_fence_after();
+      if (warp == 4) {
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint64_t a_sig = kdesc(sbase + OFF_SIG + (kk >> 2) * 16384 + (kk & 3) * 32);
-          mma_bf16(tmem + COL_U + s * 64, a_sig, mndesc(sbase + OFF_WT + kk * 2048, 8192),
-                   idesc_bf16(128, 64, 0, 1, /*neg_b=*/1), 1);
-          mma_bf16(tmem + COL_OA, a_sig, kdesc(kq_a + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32),
-                   idesc_bf16(128, 64, 0, 0), kk > 0);
+          for (int kk = 0; kk < DK / 16; ++kk)
+            mma_bf16(tmem + COL_OA, kdesc(sbase + OFF_SIG + (kk >> 2) * 16384 + (kk & 3) * 32),
+                     kdesc(kq_a + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32), idesc_bf16(128, 64, 0, 0),
+                     kk > 0);
+          mma_commit(&bars[B_OA_MMA]);
         }
-        mma_commit(&bars[B_STATE_MMA]);
+        __syncwarp();
+      }
+      // ---- W^T tile (row d = j) out of tensor memory; its buffer is then free for G of chunk c+2
+      {
+        float wr[64];
+        tmem_ld64(tmem + lane_off + col_gw(c), wr);
+        store_row64_bf16(sm + OFF_WT, j, wr);
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      wg_sync<BAR_STATE>();
+      if (j == 0) mbar_arrive(&bars[B_W_CONSUMED]);
+      // ---- U^T -= Sigma^T W^T (onto U~^T in buffer s)
+      if (warp == 4) {
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk)
+            mma_bf16(tmem + COL_U + s * 64, kdesc(sbase + OFF_SIG + (kk >> 2) * 16384 + (kk & 3) * 32),
+                     mndesc(sbase + OFF_WT + kk * 2048, 8192), idesc_bf16(128, 64, 0, 1, /*neg_b=*/1), 1);
+          mma_commit(&bars[B_STATE_MMA]);
+        }
+        __syncwarp();
       }
       if (!wg_wait<BAR_STATE>(&bars[B_STATE_MMA], sphase, s_abort, p.status)) break;
       sphase ^= 1;
       tc_fence_after();
-      if (j == 0) mbar_arrive(&bars[B_W_CONSUMED]);
 
       // ---- U^T row j -> operand tiles U^T and U^T diag(gamma_C / gamma)
       {
@@ -865,16 +926,19 @@ __global__ void __maxnreg__(224)
       wg_sync<BAR_STATE>();
 
       // ---- O_B^T = U^T P^T (N = 64)  and  Sigma^T += U'^T K (N = dk), K = 64 tokens
-      if (j == 0) {
+      if (warp == 4) {
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          mma_bf16(tmem + COL_OB, kdesc(sbase + OFF_UT + kk * 32),
-                   kdesc(sbase + OFF_P + s * 8192 + kk * 32), idesc_bf16(128, 64, 0, 0), kk > 0);
-          mma_bf16(tmem + COL_S, kdesc(sbase + OFF_UTP + kk * 32), mndesc(kq_a + kk * 2048, 16384),
-                   idesc_bf16(128, 128, 0, 1), 1);
+          for (int kk = 0; kk < C / 16; ++kk) {
+            mma_bf16(tmem + COL_OB, kdesc(sbase + OFF_UT + kk * 32),
+                     kdesc(sbase + OFF_P + s * 8192 + kk * 32), idesc_bf16(128, 64, 0, 0), kk > 0);
+            mma_bf16(tmem + COL_S, kdesc(sbase + OFF_UTP + kk * 32), mndesc(kq_a + kk * 2048, 16384),
+                     idesc_bf16(128, 128, 0, 1), 1);
+          }
+          mma_commit(&bars[B_STATE_MMA]);
         }
-        mma_commit(&bars[B_STATE_MMA]);
+        __syncwarp();
       }
       if (!wg_wait<BAR_STATE>(&bars[B_STATE_MMA], sphase, s_abort, p.status)) break;
       sphase ^= 1;
@@ -891,6 +955,8 @@ __global__ void __maxnreg__(224)
 
       // ---- outputs: o[tok0 + i][h][col0 + j] = scale (gamma_i O_A + O_B), staged
       // through shared memory ([64 tok][128 dv] bf16) for 16-byte coalesced stores
+      if (!wg_wait<BAR_STATE>(&bars[B_OA_MMA], c & 1, s_abort, p.status)) break;
+      tc_fence_after();
       {
         uint8_t* stage = sm + OFF_UTP;
         float oo[64];

@@ -162,6 +162,28 @@ def test_prefill_tc_fixed_length_ragged():
     _status_ok()
 
 
+def test_prefill_tc_strong_and_mixed_decay():
+    """Chunks whose decay spans more than 2^64 inside 64 tokens take the
+    per-entry exponential path of the decay matrix; the others use its
+    row x column factorisation.  Head 0 decays hard everywhere (a = 0.05), head 1
+    alternates hard and mild chunks, head 2 mixes the workload's gates with
+    near-resets (a = 1e-20) and exact a = 1."""
+    wl = _wl("long_prefill", n_seq=2, H=3, seq_len=333, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu")
+    a = inp["a"].clone()
+    tok = torch.arange(a.shape[0])
+    pos = tok % 333
+    a[:, 0] = 0.05
+    a[:, 1] = torch.where((pos // 64) % 2 == 0, torch.tensor(0.3), torch.tensor(0.98))
+    a[pos % 37 == 5, 2] = 1e-20
+    a[pos % 11 == 3, 2] = 1.0
+    inp["a"] = a
+    o, ST = _gpu_prefill(inp)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+    _status_ok()
+
+
 def test_prefill_tc_zero_initial_state():
     wl = _wl("long_prefill", n_seq=1, H=2, seq_len=192)
     inp = W.prefill_inputs(wl, "cpu")

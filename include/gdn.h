@@ -58,6 +58,9 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
                               x / sqrt(sum x^2 + 1e-6), then round to io dtype */
 #define GDN_PRECISE   0x2u /* prefill: use the fp32 CUDA-core chunk kernel even
                               for bf16 inputs (slower, fp32 operands)          */
+#define GDN_SINGLE_PASS 0x4u /* prefill: run every (sequence, head) chain in one
+                              pass even when a segmented schedule would be
+                              chosen (see gdn_chunk_fwd)                       */
 
 /*
  * Prefill over packed or variable-length sequences.
@@ -99,11 +102,27 @@ typedef struct {
 } gdn_fwd_params;
 
 /* Bytes of device workspace gdn_chunk_fwd needs for these parameters (may be 0).
- * Returns (size_t)-1 if the parameters are invalid. */
+ * Returns (size_t)-1 if the parameters are invalid.  The need is non-zero only
+ * when the segmented schedule is chosen (see below); it is a function of the
+ * shapes, flags and the current device's SM count. */
 size_t gdn_chunk_fwd_workspace(const gdn_fwd_params *p);
 
-/* Chunkwise prefill (chunks of 64 tokens).  ws/ws_bytes: device workspace of at
- * least gdn_chunk_fwd_workspace(p) bytes (NULL/0 allowed when that is 0). */
+/* Chunkwise prefill (chunks of 64 tokens).
+ *
+ * Schedule.  Each (sequence, head, 128-wide dv slice) chain normally runs in
+ * one pass.  When fixed-length sequences (cu_seqlens == NULL) give too few
+ * chains to fill the GPU, every sequence is instead cut into segments whose
+ * state update is affine in the start state, S_end = M S_start + B: a first
+ * launch computes each segment's B (from a zero state) and dk x dk transition
+ * M, a second kernel chains the segment start states in fp32, and a third
+ * launch runs every segment from its start state and writes the outputs
+ * (three launches, all on `stream`).  The outputs equal the one-pass outputs up
+ * to rounding.  GDN_SINGLE_PASS disables it.
+ *
+ * ws/ws_bytes: device workspace of at least gdn_chunk_fwd_workspace(p) bytes,
+ * 256-byte aligned, owned by the caller and not read back afterwards.
+ * ws == NULL with ws_bytes == 0 is always accepted and selects the one-pass
+ * schedule; a non-NULL ws smaller than the need returns GDN_ERR_WORKSPACE. */
 gdn_status gdn_chunk_fwd(const gdn_fwd_params *p, void *ws, size_t ws_bytes,
                          cudaStream_t stream);
 

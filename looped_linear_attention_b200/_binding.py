@@ -29,6 +29,7 @@ GDN_BF16 = 1
 
 GDN_QK_L2NORM = 0x1
 GDN_PRECISE = 0x2
+GDN_SINGLE_PASS = 0x4
 
 _DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
 
@@ -154,10 +155,29 @@ def gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     if ws == ctypes.c_size_t(-1).value:
         raise GdnError(GDN_ERR_INVALID, "gdn_chunk_fwd")
     work = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
+    if work is not None and stream is not None:
+        work.record_stream(stream)
     st = lib.gdn_chunk_fwd(ctypes.byref(p), _ptr(work), ctypes.c_size_t(ws), _stream_ptr(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd")
     return o, S_T
+
+
+def prefill_workspace_bytes(n_seq: int, seq_len: int, H: int, dk: int, dv: int,
+                            dtype: torch.dtype = torch.bfloat16, flags: int = 0,
+                            varlen: bool = False) -> int:
+    """gdn_chunk_fwd_workspace for a call of this shape (no device memory is
+    touched).  Non-zero means the segmented schedule: three launches per call."""
+    T = n_seq * seq_len
+    fake = 1 << 40          # aligned placeholders: the query only reads shapes and flags
+    p = gdn_fwd_params(fake, fake + (1 << 36), fake + (2 << 36), fake + (3 << 36),
+                       fake + (4 << 36), None, fake + (5 << 36), None,
+                       fake + (6 << 36) if varlen else None, n_seq, 0 if varlen else seq_len, T,
+                       H, dk, dv, _DTYPES[dtype], 1.0, int(flags))
+    ws = library().gdn_chunk_fwd_workspace(ctypes.byref(p))
+    if ws == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_INVALID, "gdn_chunk_fwd_workspace")
+    return int(ws)
 
 
 def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,

@@ -18,6 +18,14 @@
 
 namespace gdn {
 
+// Schedule of one tensor-core prefill call: n_segs = 1 runs each chain in one
+// pass, else fixed-length sequences are cut into n_segs segments of seg_tok
+// tokens (state passing between segments).
+struct SegPlan {
+  int n_segs;
+  int seg_tok;
+};
+
 // Upper bound for any device-side wait: about 2 s of SM clock.  A wait that
 // runs this long records GDN_ERR_TIMEOUT and gives up instead of hanging.
 constexpr long long kWaitLimitCycles = 4000000000LL;

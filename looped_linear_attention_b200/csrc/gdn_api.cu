@@ -7,7 +7,10 @@
 
 namespace gdn {
 bool prefill_tc_supported(const gdn_fwd_params* p);
-gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
+SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms);
+size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan);
+gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const SegPlan& plan, void* ws,
+                             cudaStream_t stream);
 gdn_status launch_prefill_simt(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
                           const float* b, float* S, void* o, int N, int H, int dk, int dv,
@@ -68,7 +71,7 @@ gdn_status validate_fwd(const gdn_fwd_params* p) {
   if (!dtype_ok(p->io_dtype)) return GDN_ERR_INVALID;
   if (p->n_seq < 0 || p->H <= 0 || p->dk <= 0 || p->dv <= 0 || p->total_tokens < 0)
     return GDN_ERR_INVALID;
-  if (p->flags & ~(GDN_QK_L2NORM | GDN_PRECISE)) return GDN_ERR_INVALID;
+  if (p->flags & ~(GDN_QK_L2NORM | GDN_PRECISE | GDN_SINGLE_PASS)) return GDN_ERR_INVALID;
   if (!p->cu_seqlens) {
     if (p->seq_len < 0) return GDN_ERR_INVALID;
     if ((long long)p->n_seq * p->seq_len != (long long)p->total_tokens) return GDN_ERR_INVALID;
@@ -126,15 +129,15 @@ const char* gdn_status_string(gdn_status s) {
 
 size_t gdn_chunk_fwd_workspace(const gdn_fwd_params* p) {
   if (validate_fwd(p) != GDN_OK) return (size_t)-1;
-  return 0;
+  if (p->total_tokens == 0) return 0;
+  return gdn::prefill_segment_workspace(p, gdn::plan_prefill_segments(p, sm_count()));
 }
 
 gdn_status gdn_chunk_fwd(const gdn_fwd_params* p, void* ws, size_t ws_bytes,
                          cudaStream_t stream) {
   const gdn_status v = validate_fwd(p);
   if (v != GDN_OK) return v;
-  (void)ws;
-  (void)ws_bytes;
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)) return GDN_ERR_INVALID;
   if (p->n_seq == 0) return GDN_OK;
   if (p->total_tokens == 0) {
     // every sequence is empty: S_T = S0 (or zero)
@@ -146,9 +149,16 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_params* p, void* ws, size_t ws_bytes,
                           : cudaMemsetAsync(p->S_T, 0, bytes, stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
   }
+  const bool tc = gdn::prefill_tc_supported(p);
+  gdn::SegPlan plan = tc ? gdn::plan_prefill_segments(p, sm_count()) : gdn::SegPlan{1, 0};
+  if (plan.n_segs > 1) {
+    const size_t need = gdn::prefill_segment_workspace(p, plan);
+    if (!ws && ws_bytes == 0) plan = gdn::SegPlan{1, 0};   // no workspace: one pass
+    else if (!ws || ws_bytes < need) return GDN_ERR_WORKSPACE;
+  }
   unsigned* st = status_ptr();
   if (!st) return GDN_ERR_CUDA;
-  if (gdn::prefill_tc_supported(p)) return gdn::launch_prefill_tc(p, st, stream);
+  if (tc) return gdn::launch_prefill_tc(p, st, plan, ws, stream);
   return gdn::launch_prefill_simt(p, st, stream);
 }
 

@@ -130,6 +130,18 @@ struct Params {
   int n_seq, seq_len, total_tokens, H, dv, n_slices;
   float scale;
   unsigned flags;
+  // Segment schedule (fixed-length sequences cut into n_segs segments of
+  // seg_tok tokens; mode 0 runs whole sequences in one pass):
+  //   mode 1: segments 0 .. n_segs-2 from a zero state, no outputs.  Slices
+  //           0 .. n_slices-1 write the segment's state contribution to Bws;
+  //           one extra slice runs V = 0 from the identity and writes the
+  //           segment's dk x dk transition to Mws.
+  //   mode 2: every segment from its start state in Sst, with outputs; the last
+  //           segment writes S_T.
+  int mode, n_segs, seg_tok;
+  float* Bws;          // [n_seq][n_segs-1][H][dk][dv]
+  float* Mws;          // [n_seq][n_segs-1][H][dk][dk]
+  const float* Sst;    // [n_seq][n_segs][H][dk][dv]
 };
 
 // Per-chunk gate vectors (one buffer).
@@ -583,11 +595,17 @@ __global__ void __maxnreg__(224)
   const int tid = threadIdx.x;
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);   // warp-uniform by construction
 
-  // work unit
-  const int slice = blockIdx.x % p.n_slices;
-  const int chain = blockIdx.x / p.n_slices;
+  // work unit: (sequence or segment, head, dv slice)
+  const int slices_here = p.n_slices + (p.mode == 1 ? 1 : 0);
+  const int slice = blockIdx.x % slices_here;
+  const int chain = blockIdx.x / slices_here;
   const int h = chain % p.H;
-  const int seq = chain / p.H;
+  const int unit = chain / p.H;
+  const int units_per_seq = (p.mode == 0) ? 1 : (p.mode == 1 ? p.n_segs - 1 : p.n_segs);
+  const int seq = unit / units_per_seq;
+  const int part = unit % units_per_seq;
+  const bool ident = (p.mode == 1 && slice == p.n_slices);   // transition slice: V = 0, S0 = I
+  const bool outputs = (p.mode != 1);
   int seq_start, seq_end;
   if (p.cu_seqlens) {
     seq_start = p.cu_seqlens[seq];
@@ -595,6 +613,10 @@ __global__ void __maxnreg__(224)
   } else {
     seq_start = seq * p.seq_len;
     seq_end = seq_start + p.seq_len;
+    if (p.mode != 0) {
+      seq_start += part * p.seg_tok;
+      seq_end = min(seq_end, seq_start + p.seg_tok);
+    }
   }
   {
     // offsets outside [0, total_tokens] or decreasing: clamp, and report
@@ -607,7 +629,7 @@ __global__ void __maxnreg__(224)
   const int len = seq_end - seq_start;
   const int n_chunks = (len + C - 1) / C;
   const int H = p.H, dv = p.dv;
-  const int col0 = slice * DVS;
+  const int col0 = ident ? 0 : slice * DVS;
 
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], 1);
@@ -636,8 +658,10 @@ __global__ void __maxnreg__(224)
       load_kq(sm, &bars[B_KQ_FULL + 1], &tm_q, &tm_k, 1, h, seq_start + C);
       s_issued[1] = 1;
     }
-    load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, seq_start);
-    s_issued[2] = 1;
+    if (!ident) {
+      load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, seq_start);
+      s_issued[2] = 1;
+    }
   }
 
   if (warp < 4) {
@@ -768,16 +792,18 @@ __global__ void __maxnreg__(224)
       fence_proxy_async_smem();
       wg_sync<BAR_PREP>();
 
-      // ---- U~^T = V^T T2^T (into U buffer s) and W^T = K^T T1^T (M = 128, N = 64, K = 64 tokens)
-      if (!wg_wait<BAR_PREP>(&bars[B_V_FULL], c & 1, s_abort, p.status)) break;
+      // ---- U~^T = V^T T2^T (into U buffer s) and W^T = K^T T1^T (M = 128, N = 64, K = 64 tokens);
+      // the transition slice has V = 0 and so no U~
+      if (!ident && !wg_wait<BAR_PREP>(&bars[B_V_FULL], c & 1, s_abort, p.status)) break;
       if (warp == 0) {
         tc_fence_after();
         const uint32_t v_a = sbase + OFF_V;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
-            mma_bf16(tmem + COL_U + s * 64, mndesc(v_a + kk * 2048, 8192),
-                     kdesc(sbase + OFF_T2 + kk * 32), idesc_bf16(128, 64, 1, 0), kk > 0);
+            if (!ident)
+              mma_bf16(tmem + COL_U + s * 64, mndesc(v_a + kk * 2048, 8192),
+                       kdesc(sbase + OFF_T2 + kk * 32), idesc_bf16(128, 64, 1, 0), kk > 0);
             mma_bf16(tmem + col_gw(c), mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
                      idesc_bf16(128, 64, 1, 0), kk > 0);
           }
@@ -786,17 +812,18 @@ __global__ void __maxnreg__(224)
         __syncwarp();
       }
       // ---- next chunk's G, queued behind these products, into the buffer that
-      // held W^T of chunk c-1 (free once the state warpgroup has read it)
-      if (c + 1 < n_chunks) {
-        if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
-        if (!issue_g(c + 1)) break;
-      }
+      // held W^T of chunk c-1 (free once the state warpgroup has read it).  The
+      // wait is taken in every chunk, the last included: W_READY of chunk c is
+      // only arrived after the state warpgroup has seen W_READY of chunk c-1,
+      // so that barrier never runs two phases ahead of its waiter.
+      if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
+      if (c + 1 < n_chunks && !issue_g(c + 1)) break;
       if (!wg_wait<BAR_PREP>(&bars[B_PREP_MMA], pphase, s_abort, p.status)) break;
       pphase ^= 1;
       if (t == 0) {
         tc_fence_before();
         mbar_arrive(&bars[B_W_READY]);     // U~^T and W^T of chunk c are in tensor memory
-        if (c + 1 < n_chunks) {            // the V stage is free: load V of chunk c+1
+        if (!ident && c + 1 < n_chunks) {  // the V stage is free: load V of chunk c+1
           load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, tok0 + C);
           s_issued[2] = c + 2;
         }
@@ -806,7 +833,27 @@ __global__ void __maxnreg__(224)
     // ================================================================ state warpgroup
     const int j = tid - WG;                                   // dv row owned
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    // initial state: s0 (rows dk, row stride ld0), the identity (transition
+    // slice) or zero; final state to st (row stride ldT) or nowhere
     const size_t state_base = ((size_t)seq * H + h) * DK * (size_t)dv + col0 + j;
+    const float* s0 = nullptr;
+    float* st = nullptr;
+    size_t ldT = dv;
+    if (p.mode == 0) {
+      s0 = p.S0 ? p.S0 + state_base : nullptr;
+      st = p.S_T ? p.S_T + state_base : nullptr;
+    } else if (p.mode == 1) {
+      const size_t u = (size_t)seq * (p.n_segs - 1) + part;
+      if (ident) {
+        st = p.Mws + (u * H + h) * DK * DK + j;
+        ldT = DK;
+      } else {
+        st = p.Bws + (u * H + h) * DK * (size_t)dv + col0 + j;
+      }
+    } else {
+      s0 = p.Sst + (((size_t)seq * p.n_segs + part) * H + h) * DK * (size_t)dv + col0 + j;
+      if (part == p.n_segs - 1 && p.S_T) st = p.S_T + state_base;
+    }
     uint32_t sphase = 0;
     bool ok = true;
 
@@ -838,7 +885,8 @@ __global__ void __maxnreg__(224)
         float x[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          x[e] = p.S0 ? __ldg(p.S0 + state_base + (size_t)(piece * 32 + e) * dv) : 0.f;
+          x[e] = ident ? ((piece * 32 + e == j) ? 1.f : 0.f)
+                       : (s0 ? __ldg(s0 + (size_t)(piece * 32 + e) * dv) : 0.f);
         uint8_t* slab = sm + OFF_SIG + (piece >> 1) * 16384;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -849,9 +897,9 @@ __global__ void __maxnreg__(224)
           o.w = pack_bf16x2(x[cc * 8 + 6], x[cc * 8 + 7]);
           *reinterpret_cast<uint4*>(slab + sw128_offset(j, (piece & 1) * 32 + cc * 8)) = o;
         }
-        if (n_chunks == 0 && p.S_T) {
+        if (n_chunks == 0 && st) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) p.S_T[state_base + (size_t)(piece * 32 + e) * dv] = x[e];
+          for (int e = 0; e < 32; ++e) st[(size_t)(piece * 32 + e) * ldT] = x[e];
         }
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[e] *= decay0;
@@ -875,7 +923,7 @@ __global__ void __maxnreg__(224)
       // ---- O_A^T = Sigma^T Q^T (needs no W: it runs while W^T is converted)
       if (!wg_wait<BAR_STATE>(&bars[B_W_READY], c & 1, s_abort, p.status)) break;
       tc_fence_after();
-      if (warp == 4) {
+      if (outputs && warp == 4) {
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk)
@@ -903,7 +951,8 @@ __global__ void __maxnreg__(224)
 #pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk)
             mma_bf16(tmem + COL_U + s * 64, kdesc(sbase + OFF_SIG + (kk >> 2) * 16384 + (kk & 3) * 32),
-                     mndesc(sbase + OFF_WT + kk * 2048, 8192), idesc_bf16(128, 64, 0, 1, /*neg_b=*/1), 1);
+                     mndesc(sbase + OFF_WT + kk * 2048, 8192), idesc_bf16(128, 64, 0, 1, /*neg_b=*/1),
+                     ident ? (kk > 0) : 1);
           mma_commit(&bars[B_STATE_MMA]);
         }
         __syncwarp();
@@ -931,8 +980,9 @@ __global__ void __maxnreg__(224)
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
-            mma_bf16(tmem + COL_OB, kdesc(sbase + OFF_UT + kk * 32),
-                     kdesc(sbase + OFF_P + s * 8192 + kk * 32), idesc_bf16(128, 64, 0, 0), kk > 0);
+            if (outputs)
+              mma_bf16(tmem + COL_OB, kdesc(sbase + OFF_UT + kk * 32),
+                       kdesc(sbase + OFF_P + s * 8192 + kk * 32), idesc_bf16(128, 64, 0, 0), kk > 0);
             mma_bf16(tmem + COL_S, kdesc(sbase + OFF_UTP + kk * 32), mndesc(kq_a + kk * 2048, 16384),
                      idesc_bf16(128, 128, 0, 1), 1);
           }
@@ -950,42 +1000,44 @@ __global__ void __maxnreg__(224)
 
       // ---- next chunk's Sigma^T operand (bf16) and pre-decayed fp32 state; S_T at the end
       const float decay = last ? 1.f : gates_at(sm, (c + 1) % 3).gamma[C - 1];   // built by this warpgroup
-      refresh_state(tmem + lane_off + COL_S, sm + OFF_SIG, j, decay, !last,
-                    (last && p.S_T) ? p.S_T + state_base : nullptr, dv);
+      refresh_state(tmem + lane_off + COL_S, sm + OFF_SIG, j, decay, !last, last ? st : nullptr,
+                    (int)ldT);
 
       // ---- outputs: o[tok0 + i][h][col0 + j] = scale (gamma_i O_A + O_B), staged
       // through shared memory ([64 tok][128 dv] bf16) for 16-byte coalesced stores
-      if (!wg_wait<BAR_STATE>(&bars[B_OA_MMA], c & 1, s_abort, p.status)) break;
-      tc_fence_after();
-      {
-        uint8_t* stage = sm + OFF_UTP;
-        float oo[64];
-        tmem_ld64(tmem + lane_off + COL_OA, oo);
+      if (outputs) {
+        if (!wg_wait<BAR_STATE>(&bars[B_OA_MMA], c & 1, s_abort, p.status)) break;
+        tc_fence_after();
+        {
+          uint8_t* stage = sm + OFF_UTP;
+          float oo[64];
+          tmem_ld64(tmem + lane_off + COL_OA, oo);
 #pragma unroll
-        for (int i = 0; i < C; ++i) oo[i] *= G.gamma[i];
+          for (int i = 0; i < C; ++i) oo[i] *= G.gamma[i];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float ob[32];
-          tmem_ld32(tmem + lane_off + COL_OB + half * 32, ob);
+          for (int half = 0; half < 2; ++half) {
+            float ob[32];
+            tmem_ld32(tmem + lane_off + COL_OB + half * 32, ob);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) oo[half * 32 + e] = p.scale * (oo[half * 32 + e] + ob[e]);
+            for (int e = 0; e < 32; ++e) oo[half * 32 + e] = p.scale * (oo[half * 32 + e] + ob[e]);
+          }
+#pragma unroll
+          for (int i = 0; i < C; ++i)
+            *reinterpret_cast<__nv_bfloat16*>(stage + i * 256 + j * 2) = __float2bfloat16_rn(oo[i]);
         }
+        tc_fence_before();
+        wg_sync<BAR_STATE>();
+        {
+          const uint8_t* stage = sm + OFF_UTP;
 #pragma unroll
-        for (int i = 0; i < C; ++i)
-          *reinterpret_cast<__nv_bfloat16*>(stage + i * 256 + j * 2) = __float2bfloat16_rn(oo[i]);
-      }
-      tc_fence_before();
-      wg_sync<BAR_STATE>();
-      {
-        const uint8_t* stage = sm + OFF_UTP;
-#pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8) {
-          const int it = j + k8 * WG;
-          const int i = it >> 4, q = it & 15;
-          if (i < valid) {
-            const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
-            __nv_bfloat16* dst = p.o + ((size_t)(tok0 + i) * H + h) * dv + col0 + q * 8;
-            __stcs(reinterpret_cast<uint4*>(dst), v);
+          for (int k8 = 0; k8 < 8; ++k8) {
+            const int it = j + k8 * WG;
+            const int i = it >> 4, q = it & 15;
+            if (i < valid) {
+              const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
+              __nv_bfloat16* dst = p.o + ((size_t)(tok0 + i) * H + h) * dv + col0 + q * 8;
+              __stcs(reinterpret_cast<uint4*>(dst), v);
+            }
           }
         }
       }
@@ -1053,7 +1105,119 @@ bool prefill_tc_supported(const gdn_fwd_params* p) {
          !(p->flags & GDN_PRECISE);
 }
 
-gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream) {
+// ------------------------------------------------------------------ segments
+// Combine step of the segmented schedule: for one (sequence, head) and 16
+// columns of dv, S_0 = S0 (or 0) and S_{p+1} = M_p S_p + B_p for p = 0 .. n_segs-2,
+// in fp32 on the CUDA cores; every S_p is written to Sst.
+namespace tc {
+constexpr int CMB_COLS = 16;
+__global__ void __launch_bounds__(256)
+    gdn_segment_combine_kernel(const float* __restrict__ S0, const float* __restrict__ Bws,
+                               const float* __restrict__ Mws, float* __restrict__ Sst, int H, int dv,
+                               int n_segs) {
+  __shared__ __align__(16) float sS[DK][CMB_COLS];
+  const int ncb = dv / CMB_COLS;
+  const int cb = blockIdx.x % ncb;
+  const int hh = (blockIdx.x / ncb) % H;
+  const int seq = blockIdx.x / (ncb * H);
+  const int t = threadIdx.x;
+  const int r = t >> 1, c0 = (t & 1) * 8;          // row r, columns c0 .. c0+7 of the block
+  const size_t sd = (size_t)DK * dv;                 // one state [dk][dv]
+  const size_t col = (size_t)r * dv + cb * CMB_COLS + c0;
+  float x[8];
+  {
+    const float* s0 = S0 ? S0 + ((size_t)seq * H + hh) * sd + col : nullptr;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = s0 ? s0[e] : 0.f;
+  }
+  for (int pp = 0;; ++pp) {
+    float* dst = Sst + (((size_t)seq * n_segs + pp) * H + hh) * sd + col;
+    *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
+    if (pp + 1 >= n_segs) break;
+    __syncthreads();                                   // previous step's reads of sS are done
+    *reinterpret_cast<float4*>(&sS[r][c0]) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4*>(&sS[r][c0 + 4]) = make_float4(x[4], x[5], x[6], x[7]);
+    __syncthreads();
+    const size_t u = ((size_t)seq * (n_segs - 1) + pp) * H + hh;
+    const float* M = Mws + u * DK * DK + (size_t)r * DK;
+    const float* B = Bws + u * sd + col;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = B[e];
+#pragma unroll 4
+    for (int k = 0; k < DK; k += 4) {
+      const float4 m4 = *reinterpret_cast<const float4*>(M + k);
+      const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const float4 s_lo = *reinterpret_cast<const float4*>(&sS[k + kk][c0]);
+        const float4 s_hi = *reinterpret_cast<const float4*>(&sS[k + kk][c0 + 4]);
+        x[0] = fmaf(mv[kk], s_lo.x, x[0]);
+        x[1] = fmaf(mv[kk], s_lo.y, x[1]);
+        x[2] = fmaf(mv[kk], s_lo.z, x[2]);
+        x[3] = fmaf(mv[kk], s_lo.w, x[3]);
+        x[4] = fmaf(mv[kk], s_hi.x, x[4]);
+        x[5] = fmaf(mv[kk], s_hi.y, x[5]);
+        x[6] = fmaf(mv[kk], s_hi.z, x[6]);
+        x[7] = fmaf(mv[kk], s_hi.w, x[7]);
+      }
+    }
+  }
+}
+}  // namespace tc
+
+// Chooses the schedule of a tensor-core prefill: n_segs = 1 is one pass per
+// chain; otherwise fixed-length sequences are cut into n_segs segments of
+// seg_tok tokens.  The cost model counts chunk steps on the critical path:
+// waves of CTAs (one CTA per SM) times chunks per CTA, for the one-pass launch
+// against the two segmented launches plus the combine.
+SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
+  SegPlan plan{1, 0};
+  if (!prefill_tc_supported(p) || p->cu_seqlens || (p->flags & GDN_SINGLE_PASS) || p->n_seq <= 0 ||
+      p->seq_len <= tc::C || sms <= 0)
+    return plan;
+  const long long chains = (long long)p->n_seq * p->H;
+  const long long slices = p->dv / tc::DVS;
+  const int n_chunks = (p->seq_len + tc::C - 1) / tc::C;
+  auto waves = [&](long long ctas) { return (double)((ctas + sms - 1) / sms); };
+  const double one_pass = waves(chains * slices) * n_chunks;
+  double best = 0.0;
+  SegPlan cand{1, 0};
+  for (int seg = 1; seg < n_chunks; ++seg) {
+    const int P = (n_chunks + seg - 1) / seg;
+    if (P < 2) break;
+    const double cost = waves(chains * (P - 1) * (slices + 1)) * seg + waves(chains * P * slices) * seg +
+                        0.25 * (P - 1) + 1.0;
+    if (cand.n_segs == 1 || cost < best) {
+      best = cost;
+      cand = SegPlan{P, seg * tc::C};
+    }
+  }
+  // segmented only when clearly cheaper than one pass
+  return (cand.n_segs > 1 && best < 0.85 * one_pass) ? cand : plan;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan) {
+  if (plan.n_segs <= 1) return 0;
+  const size_t sd = (size_t)p->H * tc::DK * p->dv * sizeof(float);
+  const size_t md = (size_t)p->H * tc::DK * tc::DK * sizeof(float);
+  const size_t n = (size_t)p->n_seq;
+  return align256(n * (plan.n_segs - 1) * sd) + align256(n * (plan.n_segs - 1) * md) +
+         align256(n * plan.n_segs * sd);
+}
+
+static gdn_status tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const tc::Params& kp, long long blocks, cudaStream_t stream) {
+  if (blocks <= 0) return GDN_OK;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  tc::gdn_prefill_tc_kernel<<<(unsigned)blocks, tc::THREADS, tc::SMEM_BYTES, stream>>>(mq, mk, mv, kp);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const SegPlan& plan, void* ws,
+                             cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(tc::gdn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1082,12 +1246,37 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, cudaStre
   kp.n_slices = p->dv / tc::DVS;
   kp.scale = p->scale;
   kp.flags = p->flags;
-  const long long blocks = (long long)p->n_seq * p->H * kp.n_slices;
-  if (blocks <= 0) return GDN_OK;
-  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
-  tc::gdn_prefill_tc_kernel<<<(unsigned)blocks, tc::THREADS, tc::SMEM_BYTES, stream>>>(mq, mk, mv,
-                                                                                      kp);
-  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  kp.mode = 0;
+  kp.n_segs = 1;
+  kp.seg_tok = 0;
+  kp.Bws = kp.Mws = nullptr;
+  kp.Sst = nullptr;
+  const long long chains = (long long)p->n_seq * p->H;
+  if (plan.n_segs <= 1) return tc_launch(mq, mk, mv, kp, chains * kp.n_slices, stream);
+
+  // segmented: workspace = [B | M | start states]
+  const int P = plan.n_segs;
+  const size_t sd = (size_t)p->H * tc::DK * p->dv * sizeof(float);
+  const size_t md = (size_t)p->H * tc::DK * tc::DK * sizeof(float);
+  char* w = static_cast<char*>(ws);
+  kp.Bws = reinterpret_cast<float*>(w);
+  w += align256((size_t)p->n_seq * (P - 1) * sd);
+  kp.Mws = reinterpret_cast<float*>(w);
+  w += align256((size_t)p->n_seq * (P - 1) * md);
+  float* sst = reinterpret_cast<float*>(w);
+  kp.Sst = sst;
+  kp.n_segs = P;
+  kp.seg_tok = plan.seg_tok;
+  kp.mode = 1;
+  gdn_status st = tc_launch(mq, mk, mv, kp, chains * (P - 1) * (kp.n_slices + 1), stream);
+  if (st != GDN_OK) return st;
+  const long long cblocks = chains * (p->dv / tc::CMB_COLS);
+  if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  tc::gdn_segment_combine_kernel<<<(unsigned)cblocks, 256, 0, stream>>>(p->S0, kp.Bws, kp.Mws, sst, p->H,
+                                                                         p->dv, P);
+  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  kp.mode = 2;
+  return tc_launch(mq, mk, mv, kp, chains * P * kp.n_slices, stream);
 }
 
 }  // namespace gdn

@@ -10,6 +10,8 @@ TOL_BF16_S = 5e-3              # bf16 inputs: final fp32 state
 
 def rel_l2(x, ref) -> float:
     x = np.asarray(x.detach().cpu().double().numpy() if hasattr(x, "detach") else x, dtype=np.float64)
+    if hasattr(ref, "detach"):
+        ref = ref.detach().cpu().double().numpy()
     ref = np.asarray(ref, dtype=np.float64)
     den = np.linalg.norm(ref)
     num = np.linalg.norm(x - ref)

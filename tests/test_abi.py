@@ -91,6 +91,57 @@ def test_workspace_query_is_zero_for_valid_shapes(lib):
     assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
 
 
+def _state_set(H, dk, dv):
+    return H * dk * dv * 4
+
+
+def test_workspace_segmented_schedule_for_few_long_chains(lib):
+    """One 4096-token sequence x 16 heads fills 16 of 148 SMs in one pass: the
+    query asks for the segmented schedule's buffers (8 segments of 512 tokens:
+    B and M for 7 segments, start states for 8)."""
+    p = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16)
+    sd = _state_set(16, 128, 128)
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 7 * sd + 7 * sd + 8 * sd
+
+
+@pytest.mark.parametrize("kw", [
+    dict(flags=B.GDN_SINGLE_PASS),                                     # forced one pass
+    dict(n_seq=8, seq_len=16384, total_tokens=8 * 16384, H=16, o=1 << 40),   # enough chains
+    dict(n_seq=1, seq_len=4096, total_tokens=4096, H=16, io_dtype=B.GDN_F32),   # fp32 kernel
+    dict(n_seq=1, seq_len=4096, total_tokens=4096, H=16, flags=B.GDN_PRECISE),
+    dict(n_seq=1, seq_len=64, total_tokens=64, H=16),                  # a single chunk
+])
+def test_workspace_zero_for_one_pass_schedules(lib, kw):
+    kw.setdefault("n_seq", 1)
+    kw.setdefault("seq_len", 4096)
+    kw.setdefault("total_tokens", kw["n_seq"] * kw["seq_len"])
+    p = _params(**kw)
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
+
+
+def test_workspace_zero_for_varlen(lib):
+    p = _params(n_seq=1, seq_len=0, total_tokens=4096, H=16, cu_seqlens=1 << 32)
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
+
+
+def test_prefill_rejects_short_or_misaligned_workspace_on_host(lib):
+    p = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16)
+    need = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
+    assert need > 0
+    assert lib.gdn_chunk_fwd(ctypes.byref(p), ctypes.c_void_p(1 << 34), need - 256,
+                             None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_chunk_fwd(ctypes.byref(p), None, need, None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_chunk_fwd(ctypes.byref(p), ctypes.c_void_p((1 << 34) + 16), need,
+                             None) == B.GDN_ERR_INVALID
+
+
+def test_python_workspace_query_matches_c(lib):
+    import looped_linear_attention_b200 as lla
+    assert lla.prefill_workspace_bytes(1, 4096, 16, 128, 128) == 22 * _state_set(16, 128, 128)
+    assert lla.prefill_workspace_bytes(1, 4096, 16, 128, 128, flags=B.GDN_SINGLE_PASS) == 0
+    assert lla.prefill_workspace_bytes(64, 1000, 16, 128, 256, varlen=True) == 0
+
+
 @pytest.mark.parametrize("args,expect", [
     (dict(dk=96), B.GDN_ERR_UNSUPPORTED),
     (dict(dv=40), B.GDN_ERR_UNSUPPORTED),

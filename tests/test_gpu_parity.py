@@ -184,6 +184,50 @@ def test_prefill_tc_strong_and_mixed_decay():
     _status_ok()
 
 
+def test_prefill_tc_segmented_equals_single_pass_and_oracle():
+    """Few long chains take the segmented schedule (segment contributions from a
+    zero state and dk x dk transitions, chained in fp32, then every segment from
+    its start state); GDN_SINGLE_PASS runs the same inputs as one pass per chain."""
+    wl = _wl("long_prefill", n_seq=2, H=2, seq_len=1000, random_s0=True)
+    assert lla.prefill_workspace_bytes(2, 1000, 2, 128, 128) > 0
+    inp = W.prefill_inputs(wl, "cpu")
+    o_s, S_s = _gpu_prefill(inp)
+    o_1, S_1 = _gpu_prefill(inp, flags=lla.GDN_SINGLE_PASS)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o_s, S_s, o_ref, S_ref, fp32=False)
+    _check(o_1, S_1, o_ref, S_ref, fp32=False)
+    assert rel_l2(o_s, o_1) < TOL_BF16_O and rel_l2(S_s, S_1) < TOL_BF16_S
+    _status_ok()
+
+
+def test_prefill_tc_segmented_dv256_l2norm_scale():
+    """Segmented schedule with two dv slices per head (plus the transition
+    slice), in-kernel L2 norm and an output scale."""
+    wl = dataclasses.replace(W.WORKLOADS["varlen"], name="seg256", varlen=False, n_seq=1, H=2,
+                             seq_len=777, normalize_qk=False)
+    assert lla.prefill_workspace_bytes(1, 777, 2, 128, 256) > 0
+    inp = W.prefill_inputs(wl, "cpu")
+    o, ST = _gpu_prefill(inp, scale=0.125, flags=lla.GDN_QK_L2NORM)
+    o_ref, S_ref = _oracle_prefill(inp, scale=0.125, normalize=True)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+    _status_ok()
+
+
+def test_prefill_tc_segmented_strong_decay_in_place():
+    """Segment transitions under hard decay (a = 0.05: the transition is nearly
+    zero) and mild decay (a = 0.999), with S_T written over S0."""
+    wl = _wl("long_prefill", n_seq=1, H=2, seq_len=2000, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu")
+    a = inp["a"].clone()
+    a[:, 0] = 0.05
+    a[:, 1] = 0.999
+    inp["a"] = a
+    o, ST = _gpu_prefill(inp, alias=True)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+    _status_ok()
+
+
 def test_prefill_tc_zero_initial_state():
     wl = _wl("long_prefill", n_seq=1, H=2, seq_len=192)
     inp = W.prefill_inputs(wl, "cpu")
@@ -285,6 +329,20 @@ def test_full_long_prefill_sampled():
     torch.cuda.synchronize()
     _status_ok()
     _sample_chain_check(inp, o, ST, [(0, 0), (7, 15), (3, 9)])
+
+
+def test_full_looped_shape_segmented_sampled():
+    """The looped workload's mixer shape (one 4096-token sequence x 16 heads)
+    runs the segmented schedule, as in the benchmark; sampled heads against the
+    oracle, outputs and final states."""
+    wl = W.WORKLOADS["looped_prefill"]
+    assert lla.prefill_workspace_bytes(1, wl.seq_len, wl.H, wl.dk, wl.dv) > 0
+    inp = W.prefill_inputs(wl, "cuda")
+    o, ST = lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], None, None,
+                              n_seq=1)
+    torch.cuda.synchronize()
+    _status_ok()
+    _sample_chain_check(inp, o, ST, [(0, 0), (0, 7), (0, 15)])
 
 
 def test_full_varlen_sampled():

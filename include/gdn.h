@@ -127,6 +127,31 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_params *p, void *ws, size_t ws_bytes,
                          cudaStream_t stream);
 
 /*
+ * gdn_chunk_fwd without a workspace argument, for callers that cannot allocate
+ * device memory for it: a plugin inside an engine or framework that owns all
+ * device memory through its own pool and forbids direct cudaMalloc (it would
+ * bypass the pool's accounting and limits), or code on a latency-critical path
+ * that must not call cudaMalloc because that call can synchronise the device.
+ * The paper has no counterpart to this entry point; it is this library's own
+ * addition.
+ *
+ * The segmented schedule's scratch is one array compiled into the library:
+ * 32 MiB (33554432 bytes) of device memory that every GPU which loads the
+ * library holds until the process exits.  A call whose
+ * gdn_chunk_fwd_workspace(p) exceeds that returns GDN_ERR_WORKSPACE without
+ * launching anything; a call that needs no workspace runs as gdn_chunk_fwd.
+ * Nothing is allocated or freed.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array, which keeps the last call's
+ * contents (nothing in it needs clearing between calls): calls whose kernels
+ * overlap on the GPU, on different streams, race on it.  Otherwise the same
+ * contract, results and errors as gdn_chunk_fwd.
+ */
+gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_params *p, cudaStream_t stream);
+
+/*
  * One decode step: one new token for each of N independent state slots (a slot
  * is one sequence x layer x loop state), H heads each.
  *   q, k [N][H][dk], v [N][H][dv], o [N][H][dv]  io_dtype

@@ -1,0 +1,90 @@
+"""gdn_chunk_fwd_noalloc: prefill for callers that cannot allocate device memory
+(a plugin whose host engine owns every device allocation through its own pool,
+or a path that must not call cudaMalloc because it can synchronise the device).
+Its segmented schedule runs out of a 32 MiB scratch array compiled into the
+library instead of a caller-provided workspace.
+
+Called through the C ABI twice in a row, on different inputs (stale scratch
+contents from the first call would show in the second), and compared with
+gdn_chunk_fwd, the allocating entry point, on the same inputs.  This file is
+collected last so that a failure here does not hide the other tests.
+"""
+import ctypes
+import dataclasses
+
+import pytest
+import torch
+
+import looped_linear_attention_b200 as lla
+from looped_linear_attention_b200 import _binding as B
+from looped_linear_attention_b200 import workloads as W
+from gpu_util import TOL_BF16_O, TOL_BF16_S, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_BYTES = 32 << 20        # the compiled-in scratch, as stated in include/gdn.h
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from looped_linear_attention_b200 import build
+    build.build()
+    handle = lla.library()
+    handle.gdn_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(B.gdn_fwd_params), ctypes.c_void_p]
+    handle.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
+    torch.cuda.init()
+    yield handle
+    assert lla.gdn_get_device_status() == lla.GDN_OK
+
+
+def _inputs(label, n_seq, H, L):
+    wl = dataclasses.replace(W.WORKLOADS["long_prefill"], name=label, n_seq=n_seq, H=H,
+                             seq_len=L, random_s0=True)
+    return W.prefill_inputs(wl, "cuda")
+
+
+def _params(inp, o, S_T):
+    T, H, dk = inp["q"].shape
+    return B.gdn_fwd_params(inp["q"].data_ptr(), inp["k"].data_ptr(), inp["v"].data_ptr(),
+                            inp["a"].data_ptr(), inp["b"].data_ptr(), inp["S0"].data_ptr(),
+                            o.data_ptr(), S_T.data_ptr(), None, inp["n_seq"], inp["seq_len"], T,
+                            H, dk, inp["v"].shape[2], B.GDN_BF16, 1.0, 0)
+
+
+def test_noalloc_matches_gdn_chunk_fwd_on_two_calls(lib):
+    """One 4096-token sequence x 16 heads: the segmented schedule (22 MB of
+    scratch, within the 32 MiB array)."""
+    n_seq, H, L = 1, 16, 4096
+    need = lla.prefill_workspace_bytes(n_seq, L, H, 128, 128)
+    assert 0 < need <= SCRATCH_BYTES
+    cases = []
+    for call in range(2):
+        inp = _inputs(f"noalloc-{call}", n_seq, H, L)
+        o_ref, S_ref = lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"],
+                                         inp["S0"], n_seq=n_seq)
+        o = torch.full_like(o_ref, float("nan"))
+        S_T = torch.full_like(S_ref, float("nan"))
+        cases.append((inp, o_ref, S_ref, o, S_T))
+    torch.cuda.synchronize()
+    for inp, _, _, o, S_T in cases:            # the two calls, back to back
+        p = _params(inp, o, S_T)
+        assert lib.gdn_chunk_fwd_noalloc(ctypes.byref(p), None) == B.GDN_OK
+    torch.cuda.synchronize()
+    assert lla.gdn_get_device_status() == lla.GDN_OK
+    for _, o_ref, S_ref, o, S_T in cases:
+        assert rel_l2(o, o_ref) < TOL_BF16_O
+        assert rel_l2(S_T, S_ref) < TOL_BF16_S
+
+
+def test_noalloc_rejects_shapes_beyond_the_scratch(lib):
+    """A call whose segmented schedule would need more than the 32 MiB array
+    (here 24 chains of 65536 tokens) returns GDN_ERR_WORKSPACE before it
+    launches anything, so placeholder pointers suffice."""
+    n_seq, H, L = 1, 24, 65536
+    need = lla.prefill_workspace_bytes(n_seq, L, H, 128, 128)
+    assert need > SCRATCH_BYTES
+    base = 1 << 40
+    p = B.gdn_fwd_params(base, base + (1 << 36), base + (2 << 36), base + (3 << 36),
+                         base + (4 << 36), None, base + (5 << 36), None, None, n_seq, L,
+                         n_seq * L, H, 128, 128, B.GDN_BF16, 1.0, 0)
+    assert lib.gdn_chunk_fwd_noalloc(ctypes.byref(p), None) == B.GDN_ERR_WORKSPACE

@@ -1108,60 +1108,99 @@ bool prefill_tc_supported(const gdn_fwd_params* p) {
 // ------------------------------------------------------------------ segments
 // Combine step of the segmented schedule: for one (sequence, head) and 16
 // columns of dv, S_0 = S0 (or 0) and S_{p+1} = M_p S_p + B_p for p = 0 .. n_segs-2,
-// in fp32 on the CUDA cores; every S_p is written to Sst.
+// in fp32 on the CUDA cores; every S_p is written to Sst.  M_p (dk x dk) is
+// staged in shared memory by cp.async, one step ahead (double buffer); each
+// thread owns 2 rows x 4 columns of the 128 x 16 block.
 namespace tc {
 constexpr int CMB_COLS = 16;
+constexpr int CMB_MLD = 132;                       // padded row stride of a staged M (floats)
+constexpr uint32_t CMB_SMEM = (2 * DK * CMB_MLD + DK * CMB_COLS) * 4;
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __global__ void __launch_bounds__(256)
     gdn_segment_combine_kernel(const float* __restrict__ S0, const float* __restrict__ Bws,
                                const float* __restrict__ Mws, float* __restrict__ Sst, int H, int dv,
                                int n_segs) {
-  __shared__ __align__(16) float sS[DK][CMB_COLS];
+  extern __shared__ __align__(16) float cmb_smem[];
+  float* sM0 = cmb_smem;
+  float* sM1 = cmb_smem + DK * CMB_MLD;
+  float* sS = cmb_smem + 2 * DK * CMB_MLD;         // [128][16]
   const int ncb = dv / CMB_COLS;
   const int cb = blockIdx.x % ncb;
   const int hh = (blockIdx.x / ncb) % H;
   const int seq = blockIdx.x / (ncb * H);
   const int t = threadIdx.x;
-  const int r = t >> 1, c0 = (t & 1) * 8;          // row r, columns c0 .. c0+7 of the block
-  const size_t sd = (size_t)DK * dv;                 // one state [dk][dv]
-  const size_t col = (size_t)r * dv + cb * CMB_COLS + c0;
-  float x[8];
+  const int r0 = (t >> 2) * 2, c0 = (t & 3) * 4;  // rows r0, r0+1; columns c0 .. c0+3
+  const size_t sd = (size_t)DK * dv;               // one state [dk][dv]
+  const size_t col = (size_t)cb * CMB_COLS + c0;
+  auto mptr = [&](int pp) { return Mws + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * DK * DK; };
+  auto stage = [&](int pp, float* dst) {
+    const float* M = mptr(pp);
+#pragma unroll 4
+    for (int idx = t; idx < DK * (DK / 4); idx += 256) {
+      const int r = idx >> 5, e4 = (idx & 31) * 4;
+      cp_async16(dst + r * CMB_MLD + e4, M + (size_t)r * DK + e4);
+    }
+    cp_async_commit();
+  };
+  if (n_segs > 1) stage(0, sM0);
+  float x[2][4];
   {
-    const float* s0 = S0 ? S0 + ((size_t)seq * H + hh) * sd + col : nullptr;
+    const float* s0 = S0 ? S0 + ((size_t)seq * H + hh) * sd : nullptr;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = s0 ? s0[e] : 0.f;
+    for (int i = 0; i < 2; ++i) {
+      const float4 v = s0 ? *reinterpret_cast<const float4*>(s0 + (size_t)(r0 + i) * dv + col)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[i][0] = v.x, x[i][1] = v.y, x[i][2] = v.z, x[i][3] = v.w;
+    }
   }
   for (int pp = 0;; ++pp) {
     float* dst = Sst + (((size_t)seq * n_segs + pp) * H + hh) * sd + col;
-    *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
-    *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float4 v = make_float4(x[i][0], x[i][1], x[i][2], x[i][3]);
+      *reinterpret_cast<float4*>(dst + (size_t)(r0 + i) * dv) = v;
+      *reinterpret_cast<float4*>(sS + (r0 + i) * CMB_COLS + c0) = v;
+    }
     if (pp + 1 >= n_segs) break;
-    __syncthreads();                                   // previous step's reads of sS are done
-    *reinterpret_cast<float4*>(&sS[r][c0]) = make_float4(x[0], x[1], x[2], x[3]);
-    *reinterpret_cast<float4*>(&sS[r][c0 + 4]) = make_float4(x[4], x[5], x[6], x[7]);
-    __syncthreads();
-    const size_t u = ((size_t)seq * (n_segs - 1) + pp) * H + hh;
-    const float* M = Mws + u * DK * DK + (size_t)r * DK;
-    const float* B = Bws + u * sd + col;
+    const bool prefetch = (pp + 2 < n_segs);
+    if (prefetch) stage(pp + 1, ((pp + 1) & 1) ? sM1 : sM0);
+    const float* B = Bws + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + col;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = B[e];
-#pragma unroll 4
-    for (int k = 0; k < DK; k += 4) {
-      const float4 m4 = *reinterpret_cast<const float4*>(M + k);
-      const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+    for (int i = 0; i < 2; ++i) {
+      const float4 v = *reinterpret_cast<const float4*>(B + (size_t)(r0 + i) * dv);
+      x[i][0] = v.x, x[i][1] = v.y, x[i][2] = v.z, x[i][3] = v.w;
+    }
+    if (prefetch) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncthreads();                                // M_pp and S_pp are in shared memory
+    const float* M = (pp & 1) ? sM1 : sM0;
+#pragma unroll 2
+    for (int e = 0; e < DK; e += 4) {
+      const float4 m0 = *reinterpret_cast<const float4*>(M + r0 * CMB_MLD + e);
+      const float4 m1 = *reinterpret_cast<const float4*>(M + (r0 + 1) * CMB_MLD + e);
+      const float mv[2][4] = {{m0.x, m0.y, m0.z, m0.w}, {m1.x, m1.y, m1.z, m1.w}};
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const float4 s_lo = *reinterpret_cast<const float4*>(&sS[k + kk][c0]);
-        const float4 s_hi = *reinterpret_cast<const float4*>(&sS[k + kk][c0 + 4]);
-        x[0] = fmaf(mv[kk], s_lo.x, x[0]);
-        x[1] = fmaf(mv[kk], s_lo.y, x[1]);
-        x[2] = fmaf(mv[kk], s_lo.z, x[2]);
-        x[3] = fmaf(mv[kk], s_lo.w, x[3]);
-        x[4] = fmaf(mv[kk], s_hi.x, x[4]);
-        x[5] = fmaf(mv[kk], s_hi.y, x[5]);
-        x[6] = fmaf(mv[kk], s_hi.z, x[6]);
-        x[7] = fmaf(mv[kk], s_hi.w, x[7]);
+      for (int k = 0; k < 4; ++k) {
+        const float4 sv = *reinterpret_cast<const float4*>(sS + (e + k) * CMB_COLS + c0);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          x[i][0] = fmaf(mv[i][k], sv.x, x[i][0]);
+          x[i][1] = fmaf(mv[i][k], sv.y, x[i][1]);
+          x[i][2] = fmaf(mv[i][k], sv.z, x[i][2]);
+          x[i][3] = fmaf(mv[i][k], sv.w, x[i][3]);
+        }
       }
     }
+    __syncthreads();                                // every read of S_pp and M_pp is done
   }
 }
 }  // namespace tc
@@ -1272,8 +1311,15 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   if (st != GDN_OK) return st;
   const long long cblocks = chains * (p->dv / tc::CMB_COLS);
   if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
-  tc::gdn_segment_combine_kernel<<<(unsigned)cblocks, 256, 0, stream>>>(p->S0, kp.Bws, kp.Mws, sst, p->H,
-                                                                         p->dv, P);
+  static bool cmb_attr_set = false;
+  if (!cmb_attr_set) {
+    if (cudaFuncSetAttribute(tc::gdn_segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc::CMB_SMEM) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    cmb_attr_set = true;
+  }
+  tc::gdn_segment_combine_kernel<<<(unsigned)cblocks, 256, tc::CMB_SMEM, stream>>>(p->S0, kp.Bws, kp.Mws, sst,
+                                                                                 p->H, p->dv, P);
   if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   kp.mode = 2;
   return tc_launch(mq, mk, mv, kp, chains * P * kp.n_slices, stream);

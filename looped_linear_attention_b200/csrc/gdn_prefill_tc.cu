@@ -1174,16 +1174,19 @@ __global__ void __launch_bounds__(256)
     if (pp + 1 >= n_segs) break;
     const bool prefetch = (pp + 2 < n_segs);
     if (prefetch) stage(pp + 1, ((pp + 1) & 1) ? sM1 : sM0);
+    // B_pp is loaded now and added after the product, so its latency is hidden
     const float* B = Bws + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + col;
+    float4 bv[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const float4 v = *reinterpret_cast<const float4*>(B + (size_t)(r0 + i) * dv);
-      x[i][0] = v.x, x[i][1] = v.y, x[i][2] = v.z, x[i][3] = v.w;
+      bv[i] = *reinterpret_cast<const float4*>(B + (size_t)(r0 + i) * dv);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[i][j] = 0.f;
     }
     if (prefetch) cp_async_wait<1>(); else cp_async_wait<0>();
     __syncthreads();                                // M_pp and S_pp are in shared memory
     const float* M = (pp & 1) ? sM1 : sM0;
-#pragma unroll 2
+#pragma unroll
     for (int e = 0; e < DK; e += 4) {
       const float4 m0 = *reinterpret_cast<const float4*>(M + r0 * CMB_MLD + e);
       const float4 m1 = *reinterpret_cast<const float4*>(M + (r0 + 1) * CMB_MLD + e);
@@ -1199,6 +1202,13 @@ __global__ void __launch_bounds__(256)
           x[i][3] = fmaf(mv[i][k], sv.w, x[i][3]);
         }
       }
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      x[i][0] += bv[i].x;
+      x[i][1] += bv[i].y;
+      x[i][2] += bv[i].z;
+      x[i][3] += bv[i].w;
     }
     __syncthreads();                                // every read of S_pp and M_pp is done
   }
@@ -1219,14 +1229,16 @@ SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
   const long long slices = p->dv / tc::DVS;
   const int n_chunks = (p->seq_len + tc::C - 1) / tc::C;
   auto waves = [&](long long ctas) { return (double)((ctas + sms - 1) / sms); };
-  const double one_pass = waves(chains * slices) * n_chunks;
+  const double one_pass = waves(chains * slices) * (n_chunks + 1.5);
   double best = 0.0;
   SegPlan cand{1, 0};
   for (int seg = 1; seg < n_chunks; ++seg) {
     const int P = (n_chunks + seg - 1) / seg;
     if (P < 2) break;
-    const double cost = waves(chains * (P - 1) * (slices + 1)) * seg + waves(chains * P * slices) * seg +
-                        0.25 * (P - 1) + 1.0;
+    // a launch wave costs its chunks plus about 1.5 chunk steps of pipeline
+    // fill and drain; a combine step about 0.8 of a chunk step
+    const double cost = waves(chains * (P - 1) * (slices + 1)) * (seg + 1.5) +
+                        waves(chains * P * slices) * (seg + 1.5) + 0.8 * (P - 1) + 0.5;
     if (cand.n_segs == 1 || cost < best) {
       best = cost;
       cand = SegPlan{P, seg * tc::C};

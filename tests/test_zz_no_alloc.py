@@ -78,13 +78,14 @@ def test_noalloc_matches_gdn_chunk_fwd_on_two_calls(lib):
 
 def test_noalloc_rejects_shapes_beyond_the_scratch(lib):
     """A call whose segmented schedule would need more than the 32 MiB array
-    (here 24 chains of 65536 tokens) returns GDN_ERR_WORKSPACE before it
-    launches anything, so placeholder pointers suffice."""
-    n_seq, H, L = 1, 24, 65536
-    need = lla.prefill_workspace_bytes(n_seq, L, H, 128, 128)
+    (here 3 heads of one 131072-token sequence with dv = 256) returns
+    GDN_ERR_WORKSPACE before it launches anything, so placeholder pointers
+    suffice."""
+    n_seq, H, L, dv = 1, 3, 131072, 256
+    need = lla.prefill_workspace_bytes(n_seq, L, H, 128, dv)
     assert need > SCRATCH_BYTES
     base = 1 << 40
     p = B.gdn_fwd_params(base, base + (1 << 36), base + (2 << 36), base + (3 << 36),
                          base + (4 << 36), None, base + (5 << 36), None, None, n_seq, L,
-                         n_seq * L, H, 128, 128, B.GDN_BF16, 1.0, 0)
+                         n_seq * L, H, 128, dv, B.GDN_BF16, 1.0, 0)
     assert lib.gdn_chunk_fwd_noalloc(ctypes.byref(p), None) == B.GDN_ERR_WORKSPACE

@@ -169,14 +169,29 @@ __device__ __forceinline__ void wg_sync() {
   asm volatile("bar.sync %0, 128;" ::"n"(ID) : "memory");
 }
 
-// All threads of a warpgroup wait on `bar`; the outcome is made uniform through
-// the abort flag so that no thread leaves the schedule alone.
+// Warpgroup barrier that also ORs a predicate over its 128 threads
+// (bar.red.or): every thread gets the same answer, even when the abort flag is
+// set by the other warpgroup while the threads are reading it.
+template <int ID>
+__device__ __forceinline__ bool wg_sync_or(bool pred) {
+  __syncwarp();
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "n"(ID)
+      : "memory");
+  return r != 0;
+}
+
+// All threads of a warpgroup wait on `bar`; the outcome (abort flag seen by any
+// thread) is made uniform so that no thread leaves the schedule alone.
 template <int ID>
 __device__ __forceinline__ bool wg_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                         unsigned* status) {
   mbar_wait_bounded(bar, parity, abort, status);
-  wg_sync<ID>();
-  return *abort == 0;
+  return !wg_sync_or<ID>(*abort != 0);
 }
 
 // K-major, 128-byte swizzled operand: rows of 128 bytes, 8-row groups 1024 B apart.
@@ -667,6 +682,7 @@ __global__ void __maxnreg__(224)
   if (warp < 4) {
     // ================================================================ prep warpgroup
     const int t = tid;
+    const int lane = t & 31;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float* s_A = reinterpret_cast<float*>(sm + OFF_A);
     float* s_T = reinterpret_cast<float*>(sm + OFF_TS);
@@ -676,19 +692,26 @@ __global__ void __maxnreg__(224)
       for (int u = t; u < 2 * 8192 / 16; u += WG) z[u] = make_uint4(0u, 0u, 0u, 0u);
     }
     uint32_t pphase = 0;
-    // K, Q of chunk c (optional in-place L2 norm), then G = [K; Q] K^T into
-    // tensor-memory buffer c % 2 (M = 128, N = 64, K = dk).  Issued one chunk
-    // ahead so the product runs while the previous chunk's W^T is converted.
-    auto issue_g = [&](int c) -> bool {
+    const bool l2n = (p.flags & GDN_QK_L2NORM) != 0;
+    // K, Q of chunk c with the optional in-place L2 norm: every thread waits for
+    // the tiles and normalises its row (K rows 0-63, Q rows 64-127)
+    auto kq_normalise = [&](int c) -> bool {
       const int s = c & 1;
       if (!wg_wait<BAR_PREP>(&bars[B_KQ_FULL + s], (c >> 1) & 1, s_abort, p.status)) return false;
-      if (p.flags & GDN_QK_L2NORM) {
-        l2norm_row(sm + OFF_KQ + s * KQ_BYTES, t & 63, t < 64 ? 0u : 8192u);   // rows 0-63: K, 64-127: Q
-        fence_proxy_async_smem();
-        wg_sync<BAR_PREP>();
-      }
-      if (warp == 0) {
-        tc_fence_after();
+      l2norm_row(sm + OFF_KQ + s * KQ_BYTES, t & 63, t < 64 ? 0u : 8192u);
+      fence_proxy_async_smem();
+      wg_sync<BAR_PREP>();
+      return true;
+    };
+    // G = [K; Q] K^T of chunk c into tensor-memory buffer c % 2 (M = 128, N = 64,
+    // K = dk), issued by warp 0 (which alone waits for the tiles when no norm is
+    // applied).  Returns false if a wait gave up.
+    auto issue_g = [&](int c) -> bool {
+      const int s = c & 1;
+      bool okw = true;
+      if (!l2n) okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_KQ_FULL + s], (c >> 1) & 1, s_abort, p.status));
+      tc_fence_after();
+      if (okw) {
         const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
         if (elect_one()) {
 #pragma unroll
@@ -699,11 +722,15 @@ __global__ void __maxnreg__(224)
           }
           mma_commit(&bars[B_G_MMA + s]);
         }
-        __syncwarp();
       }
-      return true;
+      __syncwarp();
+      return okw;
     };
-    bool ok = (n_chunks == 0) || issue_g(0);
+    bool ok = true;
+    if (n_chunks > 0) {
+      if (l2n) ok = kq_normalise(0);
+      if (ok && warp == 0) issue_g(0);   // a failed wait sets the abort flag, seen below
+    }
 #pragma unroll 1
     for (int c = 0; c < n_chunks && ok; ++c) {
       const int s = c & 1;
@@ -712,13 +739,16 @@ __global__ void __maxnreg__(224)
       const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
 
       // ---- G of chunk c, its gates (from the state warpgroup), and the P and U
-      // buffers s (free once chunk c-2 is finished)
-      if (!wg_wait<BAR_PREP>(&bars[B_G_MMA + s], (c >> 1) & 1, s_abort, p.status)) break;
+      // buffers s (free once chunk c-2 is finished): each thread waits on the
+      // three barriers, then one warpgroup barrier makes the outcome uniform
+      {
+        bool okw = mbar_wait_bounded(&bars[B_G_MMA + s], (c >> 1) & 1, s_abort, p.status);
+        okw = okw && mbar_wait_bounded(&bars[B_GATES + c % 3], (c / 3) & 1, s_abort, p.status);
+        if (c >= 2)
+          okw = okw && mbar_wait_bounded(&bars[B_CHUNK_DONE + s], ((c >> 1) - 1) & 1, s_abort, p.status);
+        if (wg_sync_or<BAR_PREP>(!okw || *s_abort != 0)) break;   // a failed wait set the abort flag
+      }
       tc_fence_after();
-      if (!wg_wait<BAR_PREP>(&bars[B_GATES + c % 3], (c / 3) & 1, s_abort, p.status)) break;
-      if (c >= 2 &&
-          !wg_wait<BAR_PREP>(&bars[B_CHUNK_DONE + s], ((c >> 1) - 1) & 1, s_abort, p.status))
-        break;
       {
         // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32, compact blocks) and
         // P = tril(D o Q K^T) (rows 64-127, bf16 operand), D_ij = 2^(g2_i - g2_j),
@@ -792,41 +822,56 @@ __global__ void __maxnreg__(224)
       fence_proxy_async_smem();
       wg_sync<BAR_PREP>();
 
-      // ---- U~^T = V^T T2^T (into U buffer s) and W^T = K^T T1^T (M = 128, N = 64, K = 64 tokens);
-      // the transition slice has V = 0 and so no U~
-      if (!ident && !wg_wait<BAR_PREP>(&bars[B_V_FULL], c & 1, s_abort, p.status)) break;
+      // ---- U~^T = V^T T2^T (into U buffer s) and W^T = K^T T1^T (M = 128, N = 64, K = 64 tokens),
+      // then G of chunk c+1, queued behind them.  Warp 0 issues both and alone
+      // takes the waits they need (V; the buffer of W^T(c-1), free once the state
+      // warpgroup has read it; the K/Q tiles), then waits for the products and
+      // arrives W_READY.  The other warps go straight on to chunk c+1 and wait
+      // there for G(c+1), whose completion implies these products' (same issuing
+      // lane, in order), so the T1/T2 and P tiles they overwrite are free.  No
+      // warp leaves the loop alone: after a failed wait warp 0 only skips work,
+      // and the next warpgroup barrier sees the abort flag.  Waiting for
+      // W_CONSUMED(c-1) in every chunk also keeps W_READY from running two
+      // phases ahead of the state warpgroup.
       if (warp == 0) {
+        // (every wait's outcome is made warp-uniform before the elected lane acts on it)
+        bool okw = ident || __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_V_FULL], c & 1, s_abort, p.status));
         tc_fence_after();
-        const uint32_t v_a = sbase + OFF_V;
-        if (elect_one()) {
+        if (okw) {
+          const uint32_t v_a = sbase + OFF_V;
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < C / 16; ++kk) {
-            if (!ident)
-              mma_bf16(tmem + COL_U + s * 64, mndesc(v_a + kk * 2048, 8192),
-                       kdesc(sbase + OFF_T2 + kk * 32), idesc_bf16(128, 64, 1, 0), kk > 0);
-            mma_bf16(tmem + col_gw(c), mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
-                     idesc_bf16(128, 64, 1, 0), kk > 0);
+            for (int kk = 0; kk < C / 16; ++kk) {
+              if (!ident)
+                mma_bf16(tmem + COL_U + s * 64, mndesc(v_a + kk * 2048, 8192),
+                         kdesc(sbase + OFF_T2 + kk * 32), idesc_bf16(128, 64, 1, 0), kk > 0);
+              mma_bf16(tmem + col_gw(c), mndesc(kq_a + kk * 2048, 16384), kdesc(sbase + OFF_T1 + kk * 32),
+                       idesc_bf16(128, 64, 1, 0), kk > 0);
+            }
+            mma_commit(&bars[B_PREP_MMA]);
           }
-          mma_commit(&bars[B_PREP_MMA]);
+        }
+        __syncwarp();
+        if (okw && c >= 1)
+          okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status));
+        if (!l2n && okw && c + 1 < n_chunks) okw = issue_g(c + 1);
+        if (okw) okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_PREP_MMA], pphase, s_abort, p.status));
+        pphase ^= 1;
+        if (okw && lane == 0) {
+          tc_fence_before();
+          mbar_arrive(&bars[B_W_READY]);     // U~^T and W^T of chunk c are in tensor memory
+          if (!ident && c + 1 < n_chunks) {  // the V stage is free: load V of chunk c+1
+            load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, tok0 + C);
+            s_issued[2] = c + 2;
+          }
         }
         __syncwarp();
       }
-      // ---- next chunk's G, queued behind these products, into the buffer that
-      // held W^T of chunk c-1 (free once the state warpgroup has read it).  The
-      // wait is taken in every chunk, the last included: W_READY of chunk c is
-      // only arrived after the state warpgroup has seen W_READY of chunk c-1,
-      // so that barrier never runs two phases ahead of its waiter.
-      if (c >= 1 && !wg_wait<BAR_PREP>(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status)) break;
-      if (c + 1 < n_chunks && !issue_g(c + 1)) break;
-      if (!wg_wait<BAR_PREP>(&bars[B_PREP_MMA], pphase, s_abort, p.status)) break;
-      pphase ^= 1;
-      if (t == 0) {
-        tc_fence_before();
-        mbar_arrive(&bars[B_W_READY]);     // U~^T and W^T of chunk c are in tensor memory
-        if (!ident && c + 1 < n_chunks) {  // the V stage is free: load V of chunk c+1
-          load_v(sm, &bars[B_V_FULL], &tm_v, col0, h, tok0 + C);
-          s_issued[2] = c + 2;
-        }
+      if (l2n && c + 1 < n_chunks) {
+        // normalise K, Q of chunk c+1 (all threads), then warp 0 issues its G
+        // (its buffer was released above, before W_READY of chunk c)
+        if (!kq_normalise(c + 1)) break;
+        if (warp == 0 && !__any_sync(0xffffffffu, *s_abort != 0)) issue_g(c + 1);
       }
     }
   } else {

@@ -469,9 +469,11 @@ def bench_decode(wl, dev, args, peaks, world):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def cpu_baseline(seconds_target: float = 15.0, sample_tokens: int = 1024):
+def cpu_baseline(seconds_target: float = 15.0, sample_tokens: int = 4096):
     """The oracle as it stands, on the first `sample_tokens` tokens of the
-    looped-prefill workload (all 4 loops, full width), on this host's cores."""
+    looped-prefill workload (all 4 loops, full width; by default the whole
+    4096-token sequence), repeated until about `seconds_target` seconds of CPU
+    work have run, on this host's cores."""
     import torch
     import oracle
     from looped_linear_attention_b200 import workloads as W
@@ -485,7 +487,7 @@ def cpu_baseline(seconds_target: float = 15.0, sample_tokens: int = 1024):
                               inp["a"][:, :Ls], inp["b"][:, :Ls], inp["rho"], wl.H, wl.dk, wl.dv)
         runs += 1
         el = time.perf_counter() - t0
-        if el > seconds_target or runs >= 3:
+        if el > seconds_target or runs >= 50:
             break
     value = Ls * runs / el
     try:
@@ -549,8 +551,9 @@ def run_profile_case(args):
     else:
         inp = W.prefill_inputs(wl, dev)
         cu = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).to(dev)
+        fl = lla.GDN_SINGLE_PASS if args.single_pass else 0
         run = lambda: lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S0"], cu,
-                                        n_seq=inp["n_seq"])
+                                        n_seq=inp["n_seq"], flags=fl)
     for _ in range(args.warmup + args.steps):
         run()
     torch.cuda.synchronize()
@@ -573,6 +576,8 @@ def main():
     ap.add_argument("--profile", choices=["tiny", "long_prefill", "varlen", "decode"], default=None,
                     help="run only this workload's kernel (for profiler captures)")
     ap.add_argument("--n-seq", type=int, default=0, help="sequences (or decode slots) for --profile")
+    ap.add_argument("--single-pass", action="store_true",
+                    help="--profile: force the one-pass prefill schedule (GDN_SINGLE_PASS)")
     args = ap.parse_args()
     if args.profile:
         run_profile_case(args)

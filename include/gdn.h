@@ -61,6 +61,13 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 #define GDN_SINGLE_PASS 0x4u /* prefill: run every (sequence, head) chain in one
                               pass even when a segmented schedule would be
                               chosen (see gdn_chunk_fwd)                       */
+#define GDN_TEST_WAIT_TIMEOUT 0x40000000u
+                           /* test hook of the tensor-core prefill: one thread
+                              waits on a barrier that nothing arrives, so the
+                              bounded wait runs out (about 2 s); the call then
+                              ends with GDN_ERR_TIMEOUT in the device status
+                              word and no outputs, and the context stays
+                              usable.  Other paths ignore it.                  */
 
 /*
  * Prefill over packed or variable-length sequences.

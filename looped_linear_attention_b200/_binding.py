@@ -30,6 +30,7 @@ GDN_BF16 = 1
 GDN_QK_L2NORM = 0x1
 GDN_PRECISE = 0x2
 GDN_SINGLE_PASS = 0x4
+GDN_TEST_WAIT_TIMEOUT = 0x40000000
 
 _DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
 

@@ -71,7 +71,8 @@ gdn_status validate_fwd(const gdn_fwd_params* p) {
   if (!dtype_ok(p->io_dtype)) return GDN_ERR_INVALID;
   if (p->n_seq < 0 || p->H <= 0 || p->dk <= 0 || p->dv <= 0 || p->total_tokens < 0)
     return GDN_ERR_INVALID;
-  if (p->flags & ~(GDN_QK_L2NORM | GDN_PRECISE | GDN_SINGLE_PASS)) return GDN_ERR_INVALID;
+  if (p->flags & ~(GDN_QK_L2NORM | GDN_PRECISE | GDN_SINGLE_PASS | GDN_TEST_WAIT_TIMEOUT))
+    return GDN_ERR_INVALID;
   if (!p->cu_seqlens) {
     if (p->seq_len < 0) return GDN_ERR_INVALID;
     if ((long long)p->n_seq * p->seq_len != (long long)p->total_tokens) return GDN_ERR_INVALID;

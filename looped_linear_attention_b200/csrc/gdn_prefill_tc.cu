@@ -116,7 +116,8 @@ enum : int {
   B_STATE_MMA = 11,   //     commits of the state warpgroup
   B_G_MMA = 12,       // [2] prep: G of a chunk done (by tensor-memory buffer)
   B_OA_MMA = 14,      //     state: O_A of a chunk done
-  NBAR = 15
+  B_NEVER = 15,       //     arrived by nobody (GDN_TEST_WAIT_TIMEOUT)
+  NBAR = 16
 };
 
 struct Params {
@@ -902,6 +903,12 @@ __global__ void __maxnreg__(224)
     uint32_t sphase = 0;
     bool ok = true;
 
+    if (p.flags & GDN_TEST_WAIT_TIMEOUT) {
+      // test hook: a wait that nothing ends runs out, records GDN_ERR_TIMEOUT
+      // and sets the abort flag, which ends every other wait of the block
+      if (j == 0) mbar_wait_bounded(&bars[B_NEVER], 0, s_abort, p.status);
+      ok = !wg_sync_or<BAR_STATE>(*s_abort != 0);
+    }
     float* s_carry = reinterpret_cast<float*>(sm + OFF_MISC + 8);
     // gate vectors of chunks 0 and 1 (later ones are built two chunks ahead,
     // at the end of each chunk); a_in, b_in hold the inputs of the next chunk
@@ -916,7 +923,7 @@ __global__ void __maxnreg__(224)
       wg_sync<BAR_STATE>();
       if (j == 0) mbar_arrive(&bars[B_GATES + c % 3]);
     };
-    if (n_chunks > 0) {
+    if (ok && n_chunks > 0) {
       load_gate_inputs(p, seq_start, min(C, len), h, j, a_in, b_in);
       gates_of(0);
       if (n_chunks > 1) gates_of(1);

@@ -228,6 +228,25 @@ def test_prefill_tc_segmented_strong_decay_in_place():
     _status_ok()
 
 
+def test_bounded_wait_runs_out_and_context_stays_usable():
+    """Failure detection on the device: GDN_TEST_WAIT_TIMEOUT makes one wait of
+    the tensor-core prefill wait on a barrier that nothing arrives.  The wait
+    gives up after about 2 s, the block aborts every other wait, drains its
+    copies and frees tensor memory; the host reads GDN_ERR_TIMEOUT, and the next
+    call on the same context runs and matches the oracle."""
+    wl = _wl("long_prefill", n_seq=1, H=1, seq_len=200, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu")
+    q, k, v, a, b = (inp[n].cuda() for n in ("q", "k", "v", "a", "b"))
+    lla.gdn_chunk_fwd(q, k, v, a, b, inp["S0"].cuda(), n_seq=1, flags=lla.GDN_TEST_WAIT_TIMEOUT)
+    torch.cuda.synchronize()
+    assert lla.gdn_get_device_status() == lla.GDN_ERR_TIMEOUT
+    assert lla.gdn_get_device_status() == lla.GDN_OK          # reading clears the word
+    o, ST = _gpu_prefill(inp)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+    _status_ok()
+
+
 def test_prefill_tc_zero_initial_state():
     wl = _wl("long_prefill", n_seq=1, H=2, seq_len=192)
     inp = W.prefill_inputs(wl, "cpu")

@@ -14,7 +14,8 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
 gdn_status launch_prefill_simt(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
                           const float* b, float* S, void* o, int N, int H, int dk, int dv,
-                          gdn_dtype dt, float scale, unsigned flags, cudaStream_t stream);
+                          gdn_dtype dt, float scale, unsigned flags, int num_sms, unsigned* status,
+                          cudaStream_t stream);
 cudaError_t launch_loop_residual(const void* h_tilde, const void* h_prev, const float* rho,
                                  void* h_out, int64_t rows, int d, gdn_dtype dt, int num_sms,
                                  cudaStream_t stream);
@@ -183,8 +184,8 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
     const char* s0 = reinterpret_cast<const char*>(S);
     if (o0 < s0 + sb && s0 < o0 + ob) return GDN_ERR_INVALID;
   }
-  const cudaError_t e =
-      gdn::launch_decode(q, k, v, a, b, S, o, N, H, dk, dv, io_dtype, scale, flags, stream);
+  const cudaError_t e = gdn::launch_decode(q, k, v, a, b, S, o, N, H, dk, dv, io_dtype, scale, flags,
+                                           sm_count(), status_ptr(), stream);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -10,11 +10,15 @@
 //     Sigma <- a Sigma + k u^T                     (in place)
 // which is Sigma_t = a (I - b k k^T) Sigma_{t-1} + b k v^T, o = scale Sigma_t^T q.
 //
-// HBM-bound: each head-state is read once and written once, 128-bit accesses
-// coalesced along dv, the state held in registers between the read and the
-// write.  One CTA of 8 warps handles one (slot, head, dv block of 32*VEC
-// columns); lane l owns VEC consecutive columns and warp w owns DK/8 rows, the
-// dk reductions go through shared memory.
+// HBM-bound: each head-state is read once and written once.  Two kernels:
+//   * gdn_decode_stream_kernel (dk = dv = 128, bf16 tokens): persistent, one
+//     CTA per SM; states move by bulk asynchronous copies through a 3-stage
+//     shared-memory ring, so copies of neighbouring items overlap the math.
+//   * gdn_decode_kernel (every other shape): one CTA of 8 warps per (slot,
+//     head, dv block of 32*VEC columns), 128-bit accesses coalesced along dv,
+//     the state held in registers between the read and the write; lane l owns
+//     VEC consecutive columns and warp w owns DK/8 rows.
+// In both, the dk reductions go through shared memory.
 #include "common.cuh"
 
 namespace gdn {
@@ -148,6 +152,188 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
+// Streaming variant for dk = dv = 128 with bf16 tokens: one persistent CTA per
+// SM walks (slot, head) items; each item's 64 KB state and its q, k, v arrive
+// by bulk asynchronous copies into a 3-stage shared-memory ring (two items
+// ahead), the CTA computes from shared memory and writes the updated state
+// back with a bulk store, so loads and stores of neighbouring items overlap
+// the arithmetic and every SM keeps about 130 KB in flight.
+namespace dec {
+constexpr int DK = 128, DV = 128, THREADS = 256, STAGES = 3;
+constexpr uint32_t STATE_BYTES = DK * DV * 4;                 // 65536
+constexpr uint32_t VEC_BYTES = 128 * 2;                       // one bf16 vector
+constexpr uint32_t STAGE_BYTES = STATE_BYTES + 3 * VEC_BYTES; // state | q | k | v
+constexpr uint32_t OFF_RED = STAGES * STAGE_BYTES;            // [8 warps][2][128] fp32 partial sums
+constexpr uint32_t OFF_BAR = OFF_RED + 8 * 2 * DV * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
+static_assert(SMEM_BYTES <= 232448, "decode ring exceeds shared memory");
+static_assert(STAGE_BYTES % 128 == 0, "stage alignment");
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gdn_decode_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                             const __nv_bfloat16* __restrict__ v, const float* __restrict__ a,
+                             const float* __restrict__ b, float* S, __nv_bfloat16* o, long long NH,
+                             float scale, unsigned flags, unsigned* status) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + OFF_BAR);
+  float* red = reinterpret_cast<float*>(dsm + OFF_RED);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + OFF_BAR + 8 * STAGES);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long first = blockIdx.x, step = gridDim.x;
+  const int n_items = (first < NH) ? (int)((NH - first + step - 1) / step) : 0;
+  if (tid == 0) {
+    for (int i = 0; i < STAGES; ++i) mbar_init(&full[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // thread 0: item n of this CTA into stage n % STAGES
+  auto issue = [&](int n) {
+    const long long sh = first + (long long)n * step;
+    uint8_t* st = dsm + (n % STAGES) * STAGE_BYTES;
+    uint64_t* bar = &full[n % STAGES];
+    mbar_arrive_expect_tx(bar, STAGE_BYTES);
+    bulk_load(st, S + sh * (DK * DV), STATE_BYTES, bar);
+    bulk_load(st + STATE_BYTES, q + sh * DK, VEC_BYTES, bar);
+    bulk_load(st + STATE_BYTES + VEC_BYTES, k + sh * DK, VEC_BYTES, bar);
+    bulk_load(st + STATE_BYTES + 2 * VEC_BYTES, v + sh * DV, VEC_BYTES, bar);
+  };
+  int issued = 0;
+  if (tid == 0) {
+    for (; issued < min(2, n_items); ++issued) issue(issued);
+  }
+  float a_next = 0.f, b_next = 0.f;
+  if (n_items > 0) {
+    a_next = __ldg(a + first);
+    b_next = __ldg(b + first);
+  }
+  const int r0 = warp * (DK / 8);                 // this thread: rows r0 .. r0+15, columns 4 lane .. +3
+  for (int n = 0; n < n_items; ++n) {
+    const long long sh = first + (long long)n * step;
+    const float aa = a_next, bb = b_next;
+    if (n + 1 < n_items) {                        // gates of the next item, a whole item ahead
+      a_next = __ldg(a + sh + step);
+      b_next = __ldg(b + sh + step);
+    }
+    uint8_t* st = dsm + (n % STAGES) * STAGE_BYTES;
+    const bool okw = mbar_wait_bounded(&full[n % STAGES], (n / STAGES) & 1, abort_flag, status);
+    if (__syncthreads_or(!okw || *abort_flag != 0)) break;
+    float* sS = reinterpret_cast<float*>(st);
+    const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(st + STATE_BYTES);
+    const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(st + STATE_BYTES + VEC_BYTES);
+    const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(st + STATE_BYTES + 2 * VEC_BYTES);
+    // norms and k.q over the whole vectors (every warp, no block sync needed)
+    float qq = 0.f, kk = 0.f, kq = 0.f;
+#pragma unroll
+    for (int e = 0; e < DK / 32; ++e) {
+      const float qe = __bfloat162float(sq[lane + 32 * e]);
+      const float ke = __bfloat162float(sk[lane + 32 * e]);
+      qq = fmaf(qe, qe, qq);
+      kk = fmaf(ke, ke, kk);
+      kq = fmaf(ke, qe, kq);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      kk += __shfl_xor_sync(0xffffffffu, kk, off);
+      kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    }
+    float nq = 1.f, nk = 1.f;
+    if (flags & GDN_QK_L2NORM) {
+      nq = 1.0f / sqrtf(qq + kQkNormEps);
+      nk = 1.0f / sqrtf(kk + kQkNormEps);
+    }
+    // this thread's 16 x 4 block of the state, and its partial x_k, x_q
+    float s[DK / 8][4], kr[DK / 8];
+    float xk[4] = {0.f, 0.f, 0.f, 0.f}, xq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < DK / 8; ++i) {
+      const float4 t = *reinterpret_cast<const float4*>(sS + (r0 + i) * DV + 4 * lane);
+      s[i][0] = t.x, s[i][1] = t.y, s[i][2] = t.z, s[i][3] = t.w;
+      kr[i] = __bfloat162float(sk[r0 + i]) * nk;
+      const float qr = __bfloat162float(sq[r0 + i]) * nq;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        xk[c] = fmaf(s[i][c], kr[i], xk[c]);
+        xq[c] = fmaf(s[i][c], qr, xq[c]);
+      }
+    }
+    *reinterpret_cast<float4*>(red + (warp * 2 + 0) * DV + 4 * lane) = make_float4(xk[0], xk[1], xk[2], xk[3]);
+    *reinterpret_cast<float4*>(red + (warp * 2 + 1) * DV + 4 * lane) = make_float4(xq[0], xq[1], xq[2], xq[3]);
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) xk[c] = xq[c] = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const float4 pk = *reinterpret_cast<const float4*>(red + (w * 2 + 0) * DV + 4 * lane);
+      const float4 pq = *reinterpret_cast<const float4*>(red + (w * 2 + 1) * DV + 4 * lane);
+      xk[0] += pk.x, xk[1] += pk.y, xk[2] += pk.z, xk[3] += pk.w;
+      xq[0] += pq.x, xq[1] += pq.y, xq[2] += pq.z, xq[3] += pq.w;
+    }
+    const float kqn = kq * nk * nq;
+    float u[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) u[c] = bb * (__bfloat162float(sv[4 * lane + c]) - aa * xk[c]);
+    if (warp == 0) {
+      uint2 ov;
+      ov.x = pack_bf16x2(scale * fmaf(aa, xq[0], kqn * u[0]), scale * fmaf(aa, xq[1], kqn * u[1]));
+      ov.y = pack_bf16x2(scale * fmaf(aa, xq[2], kqn * u[2]), scale * fmaf(aa, xq[3], kqn * u[3]));
+      *reinterpret_cast<uint2*>(o + sh * DV + 4 * lane) = ov;
+    }
+#pragma unroll
+    for (int i = 0; i < DK / 8; ++i) {
+      float4 t;
+      t.x = fmaf(aa, s[i][0], kr[i] * u[0]);
+      t.y = fmaf(aa, s[i][1], kr[i] * u[1]);
+      t.z = fmaf(aa, s[i][2], kr[i] * u[2]);
+      t.w = fmaf(aa, s[i][3], kr[i] * u[3]);
+      *reinterpret_cast<float4*>(sS + (r0 + i) * DV + 4 * lane) = t;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();        // the new state is in the stage; every read of red is done
+    if (tid == 0) {
+      bulk_store(S + sh * (DK * DV), sS, STATE_BYTES);
+      if (issued < n_items) {
+        // item n+2 goes into the stage of item n-1, whose store has read it by now
+        bulk_wait_read<1>();
+        issue(issued);
+        ++issued;
+      }
+    }
+  }
+  if (tid == 0) {
+    // leave no bulk copy in flight: loads issued but not consumed, and stores
+    for (int n = 0; n < issued; ++n) {
+      if (n >= issued - STAGES)
+        mbar_wait_bounded(&full[n % STAGES], (n / STAGES) & 1, nullptr, status);
+    }
+    bulk_wait_all();
+  }
+  __syncthreads();
+}
+}  // namespace dec
+
 template <int DK, typename T>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* a,
                                    const float* b, float* S, void* o, long long NH, int dv,
@@ -168,8 +354,25 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, 
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
                           const float* b, float* S, void* o, int N, int H, int dk, int dv,
-                          gdn_dtype dt, float scale, unsigned flags, cudaStream_t stream) {
+                          gdn_dtype dt, float scale, unsigned flags, int num_sms, unsigned* status,
+                          cudaStream_t stream) {
   const long long NH = (long long)N * H;
+  if (NH == 0) return cudaSuccess;
+  if (dt == GDN_BF16 && dk == dec::DK && dv == dec::DV && status) {
+    static bool attr_set = false;
+    if (!attr_set) {
+      const cudaError_t e = cudaFuncSetAttribute(dec::gdn_decode_stream_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)dec::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    const long long blocks = NH < num_sms ? NH : num_sms;
+    dec::gdn_decode_stream_kernel<<<(unsigned)blocks, dec::THREADS, dec::SMEM_BYTES, stream>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a, b, S,
+        (__nv_bfloat16*)o, NH, scale, flags, status);
+    return cudaGetLastError();
+  }
   if (dt == GDN_BF16) {
     return dk == 128 ? launch_decode_t<128, __nv_bfloat16>(q, k, v, a, b, S, o, NH, dv, scale, flags, stream)
                      : launch_decode_t<64, __nv_bfloat16>(q, k, v, a, b, S, o, NH, dv, scale, flags, stream);

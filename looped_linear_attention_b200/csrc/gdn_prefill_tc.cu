@@ -51,13 +51,16 @@ constexpr int C = 64;            // chunk length
 constexpr int DK = 128;          // key/query width (this kernel)
 constexpr int DVS = 128;         // dv slice per CTA
 constexpr int WG = 128;          // one warpgroup (tensor-memory lanes 0-127)
-// warps 0-3: prep warpgroup (state-independent part of chunk c+1); its thread 0
-//            also issues the TMA loads of V (one stage)
-// warps 4-7: state warpgroup (state-dependent part of chunk c); its thread 0
-//            also issues the TMA loads of K and Q (two stages)
-// Two warps per SM sub-partition leave room for 224 registers per thread.
-constexpr int THREADS = 2 * WG;
-constexpr int BAR_PREP = 1;      // named barriers of the two warpgroups
+// warps 0-7:  prep team (state-independent part of chunk c+1); its thread 0
+//             also issues the TMA loads of V (one stage)
+// warps 8-15: state team (state-dependent part of chunk c); its thread 0 also
+//             issues the TMA loads of K and Q (two stages)
+// Warps w and w+4 of a team reach the same 32 tensor-memory lanes (w mod 4) and
+// split the columns of each row between them; 4 warps per SM sub-partition
+// with up to 128 registers per thread.
+constexpr int TEAM = 2 * WG;
+constexpr int THREADS = 2 * TEAM;
+constexpr int BAR_PREP = 1;      // named barriers of the two teams
 constexpr int BAR_STATE = 2;
 
 // tensor-memory columns (fp32 accumulators, lane = row)
@@ -167,10 +170,10 @@ __device__ __forceinline__ Gates gates_at(uint8_t* sm, int buf) {
 template <int ID>
 __device__ __forceinline__ void wg_sync() {
   __syncwarp();
-  asm volatile("bar.sync %0, 128;" ::"n"(ID) : "memory");
+  asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(TEAM) : "memory");
 }
 
-// Warpgroup barrier that also ORs a predicate over its 128 threads
+// Team barrier that also ORs a predicate over its 256 threads
 // (bar.red.or): every thread gets the same answer, even when the abort flag is
 // set by the other warpgroup while the threads are reading it.
 template <int ID>
@@ -178,10 +181,10 @@ __device__ __forceinline__ bool wg_sync_or(bool pred) {
   __syncwarp();
   uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 128, p;\n\t"
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)pred), "n"(ID)
+      : "r"((uint32_t)pred), "n"(ID), "n"(TEAM)
       : "memory");
   return r != 0;
 }
@@ -206,13 +209,14 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t saddr, uint32_t lbo) {
 // Normalise one 128-element bf16 row of a [K0|Q0|K1|Q1] stage tile in place:
 // x / sqrt(sum x^2 + eps) in fp32, rounded to bf16.
 __device__ __forceinline__ void l2norm_row(uint8_t* kq, int row_in_tile, uint32_t tile_off) {
+  // two passes over the row in shared memory (sum of squares, then scale), so
+  // that the row is never held in registers whole
   float ss = 0.f;
-  uint4 v[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
     const uint32_t off = tile_off + (c >> 3) * 16384 + sw128_offset(row_in_tile, (c & 7) * 8);
-    v[c] = *reinterpret_cast<const uint4*>(kq + off);
-    const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+    const uint4 v = *reinterpret_cast<const uint4*>(kq + off);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float lo = bf16_lo(w[e]), hi = bf16_hi(w[e]);
@@ -224,11 +228,12 @@ __device__ __forceinline__ void l2norm_row(uint8_t* kq, int row_in_tile, uint32_
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
     const uint32_t off = tile_off + (c >> 3) * 16384 + sw128_offset(row_in_tile, (c & 7) * 8);
+    const uint4 v = *reinterpret_cast<const uint4*>(kq + off);
     uint4 o;
-    o.x = pack_bf16x2(bf16_lo(v[c].x) * inv, bf16_hi(v[c].x) * inv);
-    o.y = pack_bf16x2(bf16_lo(v[c].y) * inv, bf16_hi(v[c].y) * inv);
-    o.z = pack_bf16x2(bf16_lo(v[c].z) * inv, bf16_hi(v[c].z) * inv);
-    o.w = pack_bf16x2(bf16_lo(v[c].w) * inv, bf16_hi(v[c].w) * inv);
+    o.x = pack_bf16x2(bf16_lo(v.x) * inv, bf16_hi(v.x) * inv);
+    o.y = pack_bf16x2(bf16_lo(v.y) * inv, bf16_hi(v.y) * inv);
+    o.z = pack_bf16x2(bf16_lo(v.z) * inv, bf16_hi(v.z) * inv);
+    o.w = pack_bf16x2(bf16_lo(v.w) * inv, bf16_hi(v.w) * inv);
     *reinterpret_cast<uint4*>(kq + off) = o;
   }
 }
@@ -301,73 +306,58 @@ __device__ __forceinline__ void frag_a(float (&a)[2][4], const float* blkp, int 
     a[ks][3] = blkp[(g + 8) * BLK_LD + ks * 8 + q + 4];
   }
 }
-__device__ __forceinline__ void frag_b(float (&b)[2][2][2], const float* blkp, int g, int q) {
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      b[ks][nt][0] = blkp[(ks * 8 + q) * BLK_LD + nt * 8 + g];
-      b[ks][nt][1] = blkp[(ks * 8 + q + 4) * BLK_LD + nt * 8 + g];
-    }
-}
-// acc[nt][term] += A B for one block pair (K = 16)
-__device__ __forceinline__ void mma_blk(float (&acc)[2][3][4], const float (&a)[2][4],
-                                        const float (&b)[2][2][2]) {
+// B-operand fragments of one 8-column n-tile `nt` of a compact block (two
+// k-steps of 8 x 8).
+__device__ __forceinline__ void frag_b(float (&b)[2][2], const float* blkp, int nt, int g, int q) {
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
-    uint32_t ah[4], al[4];
+    b[ks][0] = blkp[(ks * 8 + q) * BLK_LD + nt * 8 + g];
+    b[ks][1] = blkp[(ks * 8 + q + 4) * BLK_LD + nt * 8 + g];
+  }
+}
+// acc[term] += A B for one block pair (K = 16), one n-tile
+__device__ __forceinline__ void mma_blk(float (&acc)[3][4], const float (&a)[2][4], const float (&b)[2][2]) {
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    uint32_t ah[4], al[4], bh[2], bl[2];
 #pragma unroll
     for (int e = 0; e < 4; ++e) split_tf32(a[ks][e], ah[e], al[e]);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      uint32_t bh[2], bl[2];
-      split_tf32(b[ks][nt][0], bh[0], bl[0]);
-      split_tf32(b[ks][nt][1], bh[1], bl[1]);
-      mma_tf32(acc[nt][0], ah, bh);
-      mma_tf32(acc[nt][1], ah, bl);
-      mma_tf32(acc[nt][2], al, bh);
-    }
+    split_tf32(b[ks][0], bh[0], bl[0]);
+    split_tf32(b[ks][1], bh[1], bl[1]);
+    mma_tf32(acc[0], ah, bh);
+    mma_tf32(acc[1], ah, bl);
+    mma_tf32(acc[2], al, bh);
   }
 }
-__device__ __forceinline__ void acc_zero(float (&acc)[2][3][4]) {
+__device__ __forceinline__ void acc_zero(float (&acc)[3][4]) {
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
+  for (int k = 0; k < 3; ++k)
 #pragma unroll
-    for (int k = 0; k < 3; ++k)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][k][e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
 }
 // Sums the three partial products, times `sign`, into the accumulator layout
-// (res[nt] = rows g, g, g+8, g+8 x columns nt*8 + 2q, +1, 2q, +1).
-__device__ __forceinline__ void acc_sum(float (&res)[2][4], const float (&acc)[2][3][4], float sign) {
+// (res = rows g, g, g+8, g+8 x columns nt*8 + 2q, +1, 2q, +1).
+__device__ __forceinline__ void acc_sum(float (&res)[4], const float (&acc)[3][4], float sign) {
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) res[nt][e] = sign * (acc[nt][0][e] + (acc[nt][1][e] + acc[nt][2][e]));
+  for (int e = 0; e < 4; ++e) res[e] = sign * (acc[0][e] + (acc[1][e] + acc[2][e]));
 }
-__device__ __forceinline__ void store_res(float* blkp, const float (&res)[2][4], int g, int q) {
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    *reinterpret_cast<float2*>(blkp + g * BLK_LD + nt * 8 + 2 * q) = make_float2(res[nt][0], res[nt][1]);
-    *reinterpret_cast<float2*>(blkp + (g + 8) * BLK_LD + nt * 8 + 2 * q) = make_float2(res[nt][2], res[nt][3]);
-  }
+__device__ __forceinline__ void store_res(float* blkp, const float (&res)[4], int nt, int g, int q) {
+  *reinterpret_cast<float2*>(blkp + g * BLK_LD + nt * 8 + 2 * q) = make_float2(res[0], res[1]);
+  *reinterpret_cast<float2*>(blkp + (g + 8) * BLK_LD + nt * 8 + 2 * q) = make_float2(res[2], res[3]);
 }
-// T block (a, b) from the accumulator layout into the bf16 operands
-// T1 = T diag(b gamma) and T2 = T diag(b).
+// n-tile nt of T block (a, b) from the accumulator layout into the bf16
+// operands T1 = T diag(b gamma) and T2 = T diag(b).
 __device__ __forceinline__ void store_res_t12(uint8_t* sm, const Gates& G, int a, int b,
-                                              const float (&res)[2][4], int g, int q) {
+                                              const float (&res)[4], int nt, int g, int q) {
+  const int col = b * 16 + nt * 8 + 2 * q;
+  const float2 bg = *reinterpret_cast<const float2*>(G.bg + col);
+  const float2 bb = *reinterpret_cast<const float2*>(G.b + col);
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    const int col = b * 16 + nt * 8 + 2 * q;
-    const float2 bg = *reinterpret_cast<const float2*>(G.bg + col);
-    const float2 bb = *reinterpret_cast<const float2*>(G.b + col);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row = a * 16 + g + 8 * h;
-      const float x0 = res[nt][2 * h], x1 = res[nt][2 * h + 1];
-      *reinterpret_cast<uint32_t*>(sm + OFF_T1 + sw128_offset(row, col)) = pack_bf16x2(x0 * bg.x, x1 * bg.y);
-      *reinterpret_cast<uint32_t*>(sm + OFF_T2 + sw128_offset(row, col)) = pack_bf16x2(x0 * bb.x, x1 * bb.y);
-    }
+  for (int h = 0; h < 2; ++h) {
+    const int row = a * 16 + g + 8 * h;
+    const float x0 = res[2 * h], x1 = res[2 * h + 1];
+    *reinterpret_cast<uint32_t*>(sm + OFF_T1 + sw128_offset(row, col)) = pack_bf16x2(x0 * bg.x, x1 * bg.y);
+    *reinterpret_cast<uint32_t*>(sm + OFF_T2 + sw128_offset(row, col)) = pack_bf16x2(x0 * bb.x, x1 * bb.y);
   }
 }
 
@@ -447,10 +437,10 @@ __device__ __forceinline__ void fwd_subst16(const float* ad, float (&x)[16]) {
 // Forward substitution inside the 16 x 16 diagonal blocks gives, in one pass,
 // the four T_aa = L_a^-1 and Z_{a+1,a} = L_{a+1}^-1 A_{a+1,a} for a = 0, 2;
 // then T_{a+1,a} = -Z_{a+1,a} T_aa, and the 32 x 32 block below the diagonal
-// as Y = A_21 T_top, T_21 = -T_bot Y (warp-level tf32 MMAs, 3xTF32).  Every T
-// block is also written, rounded to bf16 and column-scaled, into the T1 and T2
-// operand tiles (their upper block triangle is zero from the start).  All prep
-// threads take part.
+// as Y = A_21 T_top, T_21 = -T_bot Y (warp-level tf32 MMAs, 3xTF32, one
+// 8-column n-tile per warp).  Every T block is also written, rounded to bf16
+// and column-scaled, into the T1 and T2 operand tiles (their upper block
+// triangle is zero from the start).  All 256 threads of the prep team call it.
 __device__ __forceinline__ void solve_t(uint8_t* sm, const Gates& G, const float* s_A, float* s_T,
                                         int t) {
   const int warp = t >> 5, lane = t & 31;
@@ -470,29 +460,21 @@ __device__ __forceinline__ void solve_t(uint8_t* sm, const Gates& G, const float
     for (int i = 0; i < 16; ++i) out[i * BLK_LD + c] = x[i];
   }
   wg_sync<BAR_PREP>();
-  if (warp < 2) {
-    // T_{a+1,a} = -Z_{a+1,a} T_aa  (a = 0, 2), over Z in place
-    const int a = warp * 2;
-    float* out = s_T + blk(a + 1, a);
-    float fa[2][4], fb[2][2][2], acc[2][3][4], res[2][4];
-    frag_a(fa, out, g, q);
-    frag_b(fb, s_T + blk(a, a), g, q);
-    __syncwarp();
-    acc_zero(acc);
-    mma_blk(acc, fa, fb);
-    acc_sum(res, acc, -1.f);
-    store_res(out, res, g, q);
-    store_res_t12(sm, G, a + 1, a, res, g, q);
-  } else {
-    // meanwhile: the diagonal blocks into T1 and T2 (one row half per item)
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int u = (t - 64) + k * 64;         // 0..127
-      const int a = u >> 5, r = (u >> 1) & 15, half = u & 1;
-      const float* src = s_T + blk(a, a) + r * BLK_LD + half * 8;
+  {
+    // warps 0-3: T_{a+1,a} = -Z_{a+1,a} T_aa (a = 0, 2), n-tile warp % 2, over Z in place;
+    // warps 4-7 meanwhile: the diagonal blocks into T1 and T2 (one row half per thread)
+    const int a = (warp >> 1) * 2, nt = warp & 1;
+    float fa[2][4], fb[2][2], acc[3][4], res[4];
+    if (warp < 4) {
+      frag_a(fa, s_T + blk(a + 1, a), g, q);
+      frag_b(fb, s_T + blk(a, a), nt, g, q);
+    } else {
+      const int u = t - 128;                 // 0..127
+      const int ad = u >> 5, r = (u >> 1) & 15, half = u & 1;
+      const float* src = s_T + blk(ad, ad) + r * BLK_LD + half * 8;
       const float4 x0 = *reinterpret_cast<const float4*>(src);
       const float4 x1 = *reinterpret_cast<const float4*>(src + 4);
-      const int col = a * 16 + half * 8, row = a * 16 + r;
+      const int col = ad * 16 + half * 8, row = ad * 16 + r;
       const float4 bg0 = *reinterpret_cast<const float4*>(G.bg + col);
       const float4 bg1 = *reinterpret_cast<const float4*>(G.bg + col + 4);
       const float4 b0 = *reinterpret_cast<const float4*>(G.b + col);
@@ -509,67 +491,74 @@ __device__ __forceinline__ void solve_t(uint8_t* sm, const Gates& G, const float
       *reinterpret_cast<uint4*>(sm + OFF_T1 + sw128_offset(row, col)) = o1;
       *reinterpret_cast<uint4*>(sm + OFF_T2 + sw128_offset(row, col)) = o2;
     }
+    wg_sync<BAR_PREP>();                     // both n-tile warps have read Z before it is replaced
+    if (warp < 4) {
+      acc_zero(acc);
+      mma_blk(acc, fa, fb);
+      acc_sum(res, acc, -1.f);
+      store_res(s_T + blk(a + 1, a), res, nt, g, q);
+      store_res_t12(sm, G, a + 1, a, res, nt, g, q);
+    }
   }
   wg_sync<BAR_PREP>();
-  // Y_{a,b} = sum_{k=b}^{1} A_{a,k} T_{k,b}  (a = 2, 3; b = 0, 1), into block (a, b)
-  const int a2 = 2 + (warp >> 1), b2 = warp & 1;
+  // Y_{a,b} = sum_{k=b}^{1} A_{a,k} T_{k,b}  (a = 2, 3; b = 0, 1), n-tile warp % 2, into block (a, b)
+  const int bk = warp >> 1, nt = warp & 1;
+  const int a2 = 2 + (bk >> 1), b2 = bk & 1;
   {
-    float fa[2][4], fb[2][2][2], acc[2][3][4], res[2][4];
+    float fa[2][4], fb[2][2], acc[3][4], res[4];
     acc_zero(acc);
     frag_a(fa, s_A + blk(a2, 1), g, q);
-    frag_b(fb, s_T + blk(1, b2), g, q);
+    frag_b(fb, s_T + blk(1, b2), nt, g, q);
     mma_blk(acc, fa, fb);
     if (b2 == 0) {
       frag_a(fa, s_A + blk(a2, 0), g, q);
-      frag_b(fb, s_T + blk(0, 0), g, q);
+      frag_b(fb, s_T + blk(0, 0), nt, g, q);
       mma_blk(acc, fa, fb);
     }
     acc_sum(res, acc, 1.f);
-    store_res(s_T + blk(a2, b2), res, g, q);
+    store_res(s_T + blk(a2, b2), res, nt, g, q);
   }
   wg_sync<BAR_PREP>();
   // T_{a,b} = -sum_{m=2}^{a} T_{a,m} Y_{m,b}
   {
-    float fa0[2][4], fb0[2][2][2], fa1[2][4], fb1[2][2][2], acc[2][3][4], res[2][4];
+    float fa0[2][4], fb0[2][2], fa1[2][4], fb1[2][2], acc[3][4], res[4];
     frag_a(fa0, s_T + blk(a2, a2), g, q);
-    frag_b(fb0, s_T + blk(a2, b2), g, q);
+    frag_b(fb0, s_T + blk(a2, b2), nt, g, q);
     if (a2 == 3) {
       frag_a(fa1, s_T + blk(3, 2), g, q);
-      frag_b(fb1, s_T + blk(2, b2), g, q);
+      frag_b(fb1, s_T + blk(2, b2), nt, g, q);
     }
     wg_sync<BAR_PREP>();                   // every Y is read before any is replaced
     acc_zero(acc);
     mma_blk(acc, fa0, fb0);
     if (a2 == 3) mma_blk(acc, fa1, fb1);
     acc_sum(res, acc, -1.f);
-    store_res(s_T + blk(a2, b2), res, g, q);
-    store_res_t12(sm, G, a2, b2, res, g, q);
+    store_res(s_T + blk(a2, b2), res, nt, g, q);
+    store_res_t12(sm, G, a2, b2, res, nt, g, q);
   }
 }
 
-// Sigma^T row j (fp32, in tensor memory) -> bf16 operand tile for the next
-// chunk; the tensor-memory copy is scaled by `decay` (gamma_C of the next
-// chunk) so that the next carry MMA accumulates onto gamma_C Sigma.  With
-// `st_out`, the unscaled fp32 row is also written as column j of S_T.
-__device__ __forceinline__ void refresh_state(uint32_t taddr, uint8_t* sig, int j, float decay,
-                                              bool scale_tmem, float* st_out, int dv) {
+// Half hf (dk columns 64 hf .. 64 hf + 63) of Sigma^T row j (fp32, in tensor
+// memory) -> bf16 operand tile (slab hf) for the next chunk; the tensor-memory
+// copy is scaled by `decay` (gamma_C of the next chunk) so that the next carry
+// MMA accumulates onto gamma_C Sigma.  With `st_out`, the unscaled fp32 row is
+// also written to S_T (rows dk, row stride `ld`).
+__device__ __forceinline__ void refresh_state(uint32_t taddr, uint8_t* sig, int j, int hf, float decay,
+                                              bool scale_tmem, float* st_out, int ld) {
 #pragma unroll 1
   for (int piece = 0; piece < 2; ++piece) {
-    float x[64];
-    tmem_ld64(taddr + piece * 64, x);
-    store_row64_bf16(sig + piece * 16384, j, x);
+    float x[32];
+    const uint32_t col = hf * 64 + piece * 32;
+    tmem_ld32(taddr + col, x);
+    store_row32_bf16(sig + hf * 16384, j, piece * 32, x);
     if (st_out) {
 #pragma unroll
-      for (int e = 0; e < 64; ++e) st_out[(size_t)(piece * 64 + e) * dv] = x[e];
+      for (int e = 0; e < 32; ++e) st_out[(size_t)(col + e) * ld] = x[e];
     }
     if (scale_tmem) {
-      float y[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) y[e] = x[e] * decay;
-      tmem_st32(taddr + piece * 64, y);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) y[e] = x[32 + e] * decay;
-      tmem_st32(taddr + piece * 64 + 32, y);
+      for (int e = 0; e < 32; ++e) x[e] *= decay;
+      tmem_st32(taddr + col, x);
     }
   }
   tmem_wait_st();
@@ -592,7 +581,7 @@ __device__ __forceinline__ void load_v(uint8_t* sm, uint64_t* bar, const CUtenso
   tma_load_3d(sm + OFF_V + 8192, tv, bar, col0 + 64, h, tok0);
 }
 
-__global__ void __maxnreg__(224)
+__global__ void __launch_bounds__(THREADS, 1)
     gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -680,26 +669,27 @@ __global__ void __maxnreg__(224)
     }
   }
 
-  if (warp < 4) {
-    // ================================================================ prep warpgroup
-    const int t = tid;
+  if (warp < 8) {
+    // ================================================================ prep team
+    const int t = tid;                       // 0..255
     const int lane = t & 31;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int hf = t >> 7;                   // column half of a tensor-memory row
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     float* s_A = reinterpret_cast<float*>(sm + OFF_A);
     float* s_T = reinterpret_cast<float*>(sm + OFF_TS);
     {
       // the upper block triangle of T1 and T2 stays zero for the whole sequence
       uint4* z = reinterpret_cast<uint4*>(sm + OFF_T1);
-      for (int u = t; u < 2 * 8192 / 16; u += WG) z[u] = make_uint4(0u, 0u, 0u, 0u);
+      for (int u = t; u < 2 * 8192 / 16; u += TEAM) z[u] = make_uint4(0u, 0u, 0u, 0u);
     }
     uint32_t pphase = 0;
     const bool l2n = (p.flags & GDN_QK_L2NORM) != 0;
-    // K, Q of chunk c with the optional in-place L2 norm: every thread waits for
-    // the tiles and normalises its row (K rows 0-63, Q rows 64-127)
+    // K, Q of chunk c with the optional in-place L2 norm: the team waits for the
+    // tiles and threads 0-127 normalise one row each (K rows 0-63, Q rows 64-127)
     auto kq_normalise = [&](int c) -> bool {
       const int s = c & 1;
       if (!wg_wait<BAR_PREP>(&bars[B_KQ_FULL + s], (c >> 1) & 1, s_abort, p.status)) return false;
-      l2norm_row(sm + OFF_KQ + s * KQ_BYTES, t & 63, t < 64 ? 0u : 8192u);
+      if (t < WG) l2norm_row(sm + OFF_KQ + s * KQ_BYTES, t & 63, t < 64 ? 0u : 8192u);
       fence_proxy_async_smem();
       wg_sync<BAR_PREP>();
       return true;
@@ -754,65 +744,64 @@ __global__ void __maxnreg__(224)
         // A = strict_lower(diag(b) (D o K K^T)) (rows 0-63, fp32, compact blocks) and
         // P = tril(D o Q K^T) (rows 64-127, bf16 operand), D_ij = 2^(g2_i - g2_j),
         // taken as e_i f_j when the chunk's decay range allows (no exponential per
-        // entry), else one exponential per entry.  Thread t owns row i of its half;
-        // warps 0 and 2 hold rows 0-31, whose columns 32-63 are all zero.
-        const int i = t & 63;
-        const bool hi = (warp & 1) != 0;
-        const float sc = (t < C) ? G.b[i] : 1.f;
-        const int lim = (t < C) ? i : i + 1;          // columns j < lim are kept
-        float gr[64];
-        tmem_ld64(tmem + lane_off + col_gw(c), gr);
-        if (G.flag[0] != 0.f) {
-          const float sce = sc * G.e[i];
+        // entry), else one exponential per entry.  Thread t owns columns
+        // 32 hf .. 32 hf + 31 of row i of its half; rows 0-31 (warps 0, 2, 4, 6)
+        // have only zeros in columns 32-63.
+        const int tq = t & 127;
+        const int i = tq & 63;
+        const int cb = hf * 32;                         // first column of this thread
+        const bool zero_half = (hf == 1) && ((warp & 1) == 0);
+        const float sc = (tq < C) ? G.b[i] : 1.f;
+        const int lim = (tq < C) ? i : i + 1;           // columns j < lim are kept
+        float gr[32];
+        if (zero_half) {
 #pragma unroll
-          for (int j4 = 0; j4 < 16; ++j4) {
-            if (j4 < 8 || hi) {
-              const float4 f4 = *reinterpret_cast<const float4*>(G.f + 4 * j4);
+          for (int e = 0; e < 32; ++e) gr[e] = 0.f;
+        } else {
+          tmem_ld32(tmem + lane_off + col_gw(c) + cb, gr);
+          if (G.flag[0] != 0.f) {
+            const float sce = sc * G.e[i];
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 f4 = *reinterpret_cast<const float4*>(G.f + cb + 4 * j4);
               const float fv[4] = {f4.x, f4.y, f4.z, f4.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int jj = 4 * j4 + e;
-                gr[jj] = (jj < lim) ? (gr[jj] * fv[e]) * sce : 0.f;
+                const int jj = cb + 4 * j4 + e;
+                gr[4 * j4 + e] = (jj < lim) ? (gr[4 * j4 + e] * fv[e]) * sce : 0.f;
               }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) gr[4 * j4 + e] = 0.f;
             }
-          }
-        } else {
-          const float gi = G.g2[i];
+          } else {
+            const float gi = G.g2[i];
 #pragma unroll
-          for (int j4 = 0; j4 < 16; ++j4) {
-            if (j4 < 8 || hi) {
-              const float4 gj = *reinterpret_cast<const float4*>(G.g2 + 4 * j4);
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 gj = *reinterpret_cast<const float4*>(G.g2 + cb + 4 * j4);
               const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int jj = 4 * j4 + e;
+                const int jj = cb + 4 * j4 + e;
                 const float d = ex2_approx(gi - gjv[e]);
-                gr[jj] = (jj < lim) ? (sc * gr[jj]) * d : 0.f;
+                gr[4 * j4 + e] = (jj < lim) ? (sc * gr[4 * j4 + e]) * d : 0.f;
               }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) gr[4 * j4 + e] = 0.f;
             }
           }
         }
-        if (t < C) {
+        if (tq < C) {
           const int I = i >> 4;
           float* arow = s_A + (i & 15) * BLK_LD;
 #pragma unroll
-          for (int bj = 0; bj < 4; ++bj) {
+          for (int bl = 0; bl < 2; ++bl) {
+            const int bj = 2 * hf + bl;
             if (bj <= I) {
               float4* dst = reinterpret_cast<float4*>(arow + blk(I, bj));
 #pragma unroll
               for (int k = 0; k < 4; ++k)
-                dst[k] = make_float4(gr[16 * bj + 4 * k], gr[16 * bj + 4 * k + 1], gr[16 * bj + 4 * k + 2],
-                                     gr[16 * bj + 4 * k + 3]);
+                dst[k] = make_float4(gr[16 * bl + 4 * k], gr[16 * bl + 4 * k + 1], gr[16 * bl + 4 * k + 2],
+                                     gr[16 * bl + 4 * k + 3]);
             }
           }
         } else {
-          store_row64_bf16(sm + OFF_P + s * 8192, i, gr);
+          store_row32_bf16(sm + OFF_P + s * 8192, i, cb, gr);
         }
       }
       tc_fence_before();
@@ -876,8 +865,10 @@ __global__ void __maxnreg__(224)
       }
     }
   } else {
-    // ================================================================ state warpgroup
-    const int j = tid - WG;                                   // dv row owned
+    // ================================================================ state team
+    const int jt = tid - TEAM;                                // 0..255
+    const int j = jt & 127;                                   // dv row owned (tensor-memory lane)
+    const int hf = jt >> 7;                                   // column half of the row
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     // initial state: s0 (rows dk, row stride ld0), the identity (transition
     // slice) or zero; final state to st (row stride ldT) or nowhere
@@ -906,7 +897,7 @@ __global__ void __maxnreg__(224)
     if (p.flags & GDN_TEST_WAIT_TIMEOUT) {
       // test hook: a wait that nothing ends runs out, records GDN_ERR_TIMEOUT
       // and sets the abort flag, which ends every other wait of the block
-      if (j == 0) mbar_wait_bounded(&bars[B_NEVER], 0, s_abort, p.status);
+      if (jt == 0) mbar_wait_bounded(&bars[B_NEVER], 0, s_abort, p.status);
       ok = !wg_sync_or<BAR_STATE>(*s_abort != 0);
     }
     float* s_carry = reinterpret_cast<float*>(sm + OFF_MISC + 8);
@@ -915,25 +906,26 @@ __global__ void __maxnreg__(224)
     // to build
     float a_in, b_in;
     auto gates_of = [&](int c) {
-      compute_gates<BAR_STATE>(gates_at(sm, c % 3), s_carry, min(C, seq_end - (seq_start + c * C)), j,
+      compute_gates<BAR_STATE>(gates_at(sm, c % 3), s_carry, min(C, seq_end - (seq_start + c * C)), jt,
                                a_in, b_in);
       if (c + 1 < n_chunks)
-        load_gate_inputs(p, seq_start + (c + 1) * C, min(C, seq_end - (seq_start + (c + 1) * C)), h, j,
+        load_gate_inputs(p, seq_start + (c + 1) * C, min(C, seq_end - (seq_start + (c + 1) * C)), h, jt,
                          a_in, b_in);
       wg_sync<BAR_STATE>();
-      if (j == 0) mbar_arrive(&bars[B_GATES + c % 3]);
+      if (jt == 0) mbar_arrive(&bars[B_GATES + c % 3]);
     };
     if (ok && n_chunks > 0) {
-      load_gate_inputs(p, seq_start, min(C, len), h, j, a_in, b_in);
+      load_gate_inputs(p, seq_start, min(C, len), h, jt, a_in, b_in);
       gates_of(0);
       if (n_chunks > 1) gates_of(1);
     }
 
     // initial state: tensor memory holds gamma_C(0) * S0, the bf16 operand holds S0
+    // (this thread: dk columns 64 hf .. 64 hf + 63 of row j)
     const float decay0 = (n_chunks > 0) ? gates_at(sm, 0).gamma[C - 1] : 1.f;
     {
 #pragma unroll 1
-      for (int piece = 0; piece < 4; ++piece) {
+      for (int piece = 2 * hf; piece < 2 * hf + 2; ++piece) {
         float x[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e)
@@ -975,7 +967,7 @@ __global__ void __maxnreg__(224)
       // ---- O_A^T = Sigma^T Q^T (needs no W: it runs while W^T is converted)
       if (!wg_wait<BAR_STATE>(&bars[B_W_READY], c & 1, s_abort, p.status)) break;
       tc_fence_after();
-      if (outputs && warp == 4) {
+      if (outputs && warp == 8) {
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk)
@@ -986,18 +978,19 @@ __global__ void __maxnreg__(224)
         }
         __syncwarp();
       }
-      // ---- W^T tile (row d = j) out of tensor memory; its buffer is then free for G of chunk c+2
+      // ---- W^T tile (row d = j, tokens 32 hf ..) out of tensor memory; its buffer
+      // is then free for G of chunk c+2
       {
-        float wr[64];
-        tmem_ld64(tmem + lane_off + col_gw(c), wr);
-        store_row64_bf16(sm + OFF_WT, j, wr);
+        float wr[32];
+        tmem_ld32(tmem + lane_off + col_gw(c) + 32 * hf, wr);
+        store_row32_bf16(sm + OFF_WT, j, 32 * hf, wr);
       }
       tc_fence_before();
       fence_proxy_async_smem();
       wg_sync<BAR_STATE>();
-      if (j == 0) mbar_arrive(&bars[B_W_CONSUMED]);
+      if (jt == 0) mbar_arrive(&bars[B_W_CONSUMED]);
       // ---- U^T -= Sigma^T W^T (onto U~^T in buffer s)
-      if (warp == 4) {
+      if (warp == 8) {
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
@@ -1013,21 +1006,27 @@ __global__ void __maxnreg__(224)
       sphase ^= 1;
       tc_fence_after();
 
-      // ---- U^T row j -> operand tiles U^T and U^T diag(gamma_C / gamma)
+      // ---- U^T row j (tokens 32 hf ..) -> operand tiles U^T and U^T diag(gamma_C / gamma)
       {
-        float ur[64];
-        tmem_ld64(tmem + lane_off + COL_U + s * 64, ur);
-        store_row64_bf16(sm + OFF_UT, j, ur);
+        float ur[32];
+        tmem_ld32(tmem + lane_off + COL_U + s * 64 + 32 * hf, ur);
+        store_row32_bf16(sm + OFF_UT, j, 32 * hf, ur);
 #pragma unroll
-        for (int e = 0; e < C; ++e) ur[e] *= G.r[e];
-        store_row64_bf16(sm + OFF_UTP, j, ur);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 r4 = *reinterpret_cast<const float4*>(G.r + 32 * hf + 4 * e4);
+          ur[4 * e4] *= r4.x;
+          ur[4 * e4 + 1] *= r4.y;
+          ur[4 * e4 + 2] *= r4.z;
+          ur[4 * e4 + 3] *= r4.w;
+        }
+        store_row32_bf16(sm + OFF_UTP, j, 32 * hf, ur);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       wg_sync<BAR_STATE>();
 
       // ---- O_B^T = U^T P^T (N = 64)  and  Sigma^T += U'^T K (N = dk), K = 64 tokens
-      if (warp == 4) {
+      if (warp == 8) {
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
@@ -1045,14 +1044,14 @@ __global__ void __maxnreg__(224)
       if (!wg_wait<BAR_STATE>(&bars[B_STATE_MMA], sphase, s_abort, p.status)) break;
       sphase ^= 1;
       tc_fence_after();
-      if (j == 0 && c + 2 < n_chunks) {   // last read of the K, Q stage is done: load chunk c+2
+      if (jt == 0 && c + 2 < n_chunks) {  // last read of the K, Q stage is done: load chunk c+2
         load_kq(sm, &bars[B_KQ_FULL + s], &tm_q, &tm_k, s, h, tok0 + 2 * C);
         s_issued[s] = (c >> 1) + 2;
       }
 
       // ---- next chunk's Sigma^T operand (bf16) and pre-decayed fp32 state; S_T at the end
-      const float decay = last ? 1.f : gates_at(sm, (c + 1) % 3).gamma[C - 1];   // built by this warpgroup
-      refresh_state(tmem + lane_off + COL_S, sm + OFF_SIG, j, decay, !last, last ? st : nullptr,
+      const float decay = last ? 1.f : gates_at(sm, (c + 1) % 3).gamma[C - 1];   // built by this team
+      refresh_state(tmem + lane_off + COL_S, sm + OFF_SIG, j, hf, decay, !last, last ? st : nullptr,
                     (int)ldT);
 
       // ---- outputs: o[tok0 + i][h][col0 + j] = scale (gamma_i O_A + O_B), staged
@@ -1061,29 +1060,30 @@ __global__ void __maxnreg__(224)
         if (!wg_wait<BAR_STATE>(&bars[B_OA_MMA], c & 1, s_abort, p.status)) break;
         tc_fence_after();
         {
+          // this thread: dv row j, tokens 32 hf .. 32 hf + 31
           uint8_t* stage = sm + OFF_UTP;
-          float oo[64];
-          tmem_ld64(tmem + lane_off + COL_OA, oo);
+          float oo[32], ob[32];
+          tmem_ld32(tmem + lane_off + COL_OA + 32 * hf, oo);
+          tmem_ld32(tmem + lane_off + COL_OB + 32 * hf, ob);
 #pragma unroll
-          for (int i = 0; i < C; ++i) oo[i] *= G.gamma[i];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 g4 = *reinterpret_cast<const float4*>(G.gamma + 32 * hf + 4 * e4);
+            const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float ob[32];
-            tmem_ld32(tmem + lane_off + COL_OB + half * 32, ob);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) oo[half * 32 + e] = p.scale * (oo[half * 32 + e] + ob[e]);
+            for (int e = 0; e < 4; ++e)
+              oo[4 * e4 + e] = p.scale * fmaf(oo[4 * e4 + e], gv[e], ob[4 * e4 + e]);
           }
 #pragma unroll
-          for (int i = 0; i < C; ++i)
-            *reinterpret_cast<__nv_bfloat16*>(stage + i * 256 + j * 2) = __float2bfloat16_rn(oo[i]);
+          for (int e = 0; e < 32; ++e)
+            *reinterpret_cast<__nv_bfloat16*>(stage + (32 * hf + e) * 256 + j * 2) = __float2bfloat16_rn(oo[e]);
         }
         tc_fence_before();
         wg_sync<BAR_STATE>();
         {
           const uint8_t* stage = sm + OFF_UTP;
 #pragma unroll
-          for (int k8 = 0; k8 < 8; ++k8) {
-            const int it = j + k8 * WG;
+          for (int k8 = 0; k8 < 4; ++k8) {
+            const int it = jt + k8 * TEAM;
             const int i = it >> 4, q = it & 15;
             if (i < valid) {
               const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
@@ -1095,7 +1095,7 @@ __global__ void __maxnreg__(224)
       }
       fence_proxy_async_smem();
       wg_sync<BAR_STATE>();
-      if (j == 0) mbar_arrive(&bars[B_CHUNK_DONE + s]);
+      if (jt == 0) mbar_arrive(&bars[B_CHUNK_DONE + s]);
 
       // ---- gate vectors of chunk c+2 (their buffer's previous user, chunk c-1, is finished)
       if (c + 2 < n_chunks) gates_of(c + 2);

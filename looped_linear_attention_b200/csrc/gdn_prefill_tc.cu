@@ -844,7 +844,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (okw && c >= 1)
           okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status));
-        if (!l2n && okw && c + 1 < n_chunks) okw = issue_g(c + 1);
+        // G(1) only: later chunks' G products are issued by the state team (two chunks ahead)
+        if (!l2n && okw && c == 0 && n_chunks > 1) okw = issue_g(1);
         if (okw) okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_PREP_MMA], pphase, s_abort, p.status));
         pphase ^= 1;
         if (okw && lane == 0) {
@@ -857,11 +858,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         __syncwarp();
       }
-      if (l2n && c + 1 < n_chunks) {
-        // normalise K, Q of chunk c+1 (all threads), then warp 0 issues its G
-        // (its buffer was released above, before W_READY of chunk c)
-        if (!kq_normalise(c + 1)) break;
-        if (warp == 0 && !__any_sync(0xffffffffu, *s_abort != 0)) issue_g(c + 1);
+      if (l2n && c == 0 && n_chunks > 1) {
+        // normalise K, Q of chunk 1 (all threads), then warp 0 issues its G
+        if (!kq_normalise(1)) break;
+        if (warp == 0 && !__any_sync(0xffffffffu, *s_abort != 0)) issue_g(1);
       }
     }
   } else {
@@ -1041,6 +1041,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         __syncwarp();
       }
+      // ---- gate vectors of chunk c+2 while the products run (their buffer's
+      // previous user, chunk c-1, is finished)
+      if (c + 2 < n_chunks) gates_of(c + 2);
       if (!wg_wait<BAR_STATE>(&bars[B_STATE_MMA], sphase, s_abort, p.status)) break;
       sphase ^= 1;
       tc_fence_after();
@@ -1097,8 +1100,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       wg_sync<BAR_STATE>();
       if (jt == 0) mbar_arrive(&bars[B_CHUNK_DONE + s]);
 
-      // ---- gate vectors of chunk c+2 (their buffer's previous user, chunk c-1, is finished)
-      if (c + 2 < n_chunks) gates_of(c + 2);
+      // ---- G = [K; Q] K^T of chunk c+2 into tensor-memory buffer c % 2 (it held
+      // W^T of chunk c, read at the start of this chunk), after its K, Q tiles
+      // have landed in stage s (loaded above) and, with the flag, been normalised
+      if (c + 2 < n_chunks) {
+        const int c2 = c + 2;
+        if (!wg_wait<BAR_STATE>(&bars[B_KQ_FULL + s], (c2 >> 1) & 1, s_abort, p.status)) break;
+        if (p.flags & GDN_QK_L2NORM) {
+          if (jt < WG) l2norm_row(sm + OFF_KQ + s * KQ_BYTES, jt & 63, jt < 64 ? 0u : 8192u);
+          fence_proxy_async_smem();
+          wg_sync<BAR_STATE>();
+        }
+        if (warp == 8) {
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16(tmem + col_gw(c2), kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
+                       kk > 0);
+            }
+            mma_commit(&bars[B_G_MMA + s]);
+          }
+          __syncwarp();
+        }
+      }
     }
   }
 

@@ -59,3 +59,68 @@ class LoopedPrefill:
             B.loop_residual(self.o.view(L, H * dv), h_prev, rho[tau], out=h_next)
             h_prev = h_next
         return h_prev
+
+
+class HostPipeline:
+    """Looped-prefill steps whose inputs and results live in pinned host memory.
+
+    Each `submit` copies one step's h0, a, b to the device, runs the step on the
+    caller's current stream and copies h^(T) back, all asynchronously.  Two
+    device buffer sets and two copy streams (host-to-device, device-to-host)
+    let the copies of one step overlap the compute of its neighbours; events
+    keep a buffer set from being refilled before the step that used it is done.
+    The host buffers of a step must stay untouched until the event that
+    `submit` returns has completed (its copy-out is then finished)."""
+
+    def __init__(self, runner: LoopedPrefill, device):
+        L, d, T = runner.L, runner.H * runner.dv, runner.loops
+        self.runner = runner
+        self.dev = torch.device(device)
+        self.h = [torch.empty(L, d, dtype=torch.bfloat16, device=self.dev) for _ in range(2)]
+        self.a = [torch.empty(T, L, runner.H, dtype=torch.float32, device=self.dev) for _ in range(2)]
+        self.b = [torch.empty(T, L, runner.H, dtype=torch.float32, device=self.dev) for _ in range(2)]
+        self.out = [torch.empty(L, d, dtype=torch.bfloat16, device=self.dev) for _ in range(2)]
+        self.s_in = torch.cuda.Stream(self.dev)
+        self.s_out = torch.cuda.Stream(self.dev)
+        self.inputs_free = [None, None]     # compute of the last step that read buffer set k
+        self.output_free = [None, None]     # copy-out of the last step that wrote out[k]
+        self.n = 0
+
+    def submit(self, h_host, a_host, b_host, out_host, Wq, Wk, Wv, rho, scale: float = 1.0):
+        compute = torch.cuda.current_stream(self.dev)
+        k = self.n % 2
+        self.n += 1
+        with torch.cuda.stream(self.s_in):
+            if self.inputs_free[k] is not None:
+                self.s_in.wait_event(self.inputs_free[k])
+            self.h[k].copy_(h_host, non_blocking=True)
+            self.a[k].copy_(a_host, non_blocking=True)
+            self.b[k].copy_(b_host, non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(self.s_in)
+        compute.wait_event(loaded)
+        if self.output_free[k] is not None:
+            compute.wait_event(self.output_free[k])
+        self.runner.run(self.h[k], Wq, Wk, Wv, self.a[k], self.b[k], rho, scale=scale, out=self.out[k])
+        done = torch.cuda.Event()
+        done.record(compute)
+        self.inputs_free[k] = done
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(done)
+            out_host.copy_(self.out[k], non_blocking=True)
+            copied = torch.cuda.Event()
+            copied.record(self.s_out)
+        self.output_free[k] = copied
+        return copied
+
+    def join(self, stream=None):
+        """Makes `stream` (default: the current one) wait for every copy submitted so far."""
+        stream = torch.cuda.current_stream(self.dev) if stream is None else stream
+        stream.wait_stream(self.s_in)
+        stream.wait_stream(self.s_out)
+
+    def start_after(self, stream=None):
+        """Makes the copy streams wait for work already queued on `stream`."""
+        stream = torch.cuda.current_stream(self.dev) if stream is None else stream
+        self.s_in.wait_stream(stream)
+        self.s_out.wait_stream(stream)

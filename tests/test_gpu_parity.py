@@ -421,3 +421,32 @@ def test_looped_prefill_end_to_end():
     o_ref, _ = oracle.gdn_fwd(oracle.qk_l2norm(host(q)), oracle.qk_l2norm(host(k)), host(v),
                               inp["a"][0], inp["b"][0])
     assert rel_l2(host(o), o_ref) < TOL_BF16_O
+
+
+def test_host_pipeline_matches_device_steps():
+    """HostPipeline (pinned host inputs and results, copies overlapped with the
+    neighbouring steps' compute) gives the same h^(T) as LoopedPrefill.run on
+    device inputs, step by step, for three different inputs in a row."""
+    wl = dataclasses.replace(W.WORKLOADS["looped_prefill"], seq_len=512)
+    base = W.looped_inputs(wl, "cpu")
+    L, d = base["L"], base["d"]
+    runner = lla.LoopedPrefill(L, wl.H, wl.dk, wl.dv, wl.loops, "cuda")
+    pipe = lla.HostPipeline(runner, "cuda")
+    W_dev = [base[n].cuda() for n in ("Wq", "Wk", "Wv")]
+    rho = base["rho"].cuda()
+    g = torch.Generator().manual_seed(W.seed_for("test", "host-pipeline"))
+    steps = []
+    for i in range(3):
+        h0 = torch.randn(L, d, generator=g).bfloat16().pin_memory()
+        a = (base["a"] ** (1.0 + 0.1 * i)).contiguous().pin_memory()
+        b = base["b"].clone().pin_memory()
+        out = torch.empty(L, d, dtype=torch.bfloat16).pin_memory()
+        steps.append((h0, a, b, out))
+        pipe.submit(h0, a, b, out, *W_dev, rho)
+    pipe.join()
+    torch.cuda.synchronize()
+    _status_ok()
+    for h0, a, b, out in steps:
+        ref = runner.run(h0.cuda(), *W_dev, a.cuda(), b.cuda(), rho)
+        torch.cuda.synchronize()
+        assert torch.equal(out, host(ref))

@@ -1186,13 +1186,15 @@ bool prefill_tc_supported(const gdn_fwd_params* p) {
 // ------------------------------------------------------------------ segments
 // Combine step of the segmented schedule: for one (sequence, head) and 16
 // columns of dv, S_0 = S0 (or 0) and S_{p+1} = M_p S_p + B_p for p = 0 .. n_segs-2,
-// in fp32 on the CUDA cores; every S_p is written to Sst.  M_p (dk x dk) is
-// staged in shared memory by cp.async, one step ahead (double buffer); each
-// thread owns 2 rows x 4 columns of the 128 x 16 block.
+// with every S_p written to Sst.  The products run on the warp-level tensor
+// cores with the 3xTF32 split (fp32-level accuracy): warp w owns rows
+// 16w .. 16w+15 of the 128 x 16 block.  M_p (dk x dk) is staged in shared
+// memory by cp.async one step ahead (double buffer).
 namespace tc {
 constexpr int CMB_COLS = 16;
 constexpr int CMB_MLD = 132;                       // padded row stride of a staged M (floats)
-constexpr uint32_t CMB_SMEM = (2 * DK * CMB_MLD + DK * CMB_COLS) * 4;
+constexpr int CMB_SLD = 24;                        // padded row stride of the S block (floats)
+constexpr uint32_t CMB_SMEM = (2 * DK * CMB_MLD + DK * CMB_SLD) * 4;
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
@@ -1211,15 +1213,16 @@ __global__ void __launch_bounds__(256)
   extern __shared__ __align__(16) float cmb_smem[];
   float* sM0 = cmb_smem;
   float* sM1 = cmb_smem + DK * CMB_MLD;
-  float* sS = cmb_smem + 2 * DK * CMB_MLD;         // [128][16]
+  float* sS = cmb_smem + 2 * DK * CMB_MLD;         // [128][CMB_SLD], 16 columns used
   const int ncb = dv / CMB_COLS;
   const int cb = blockIdx.x % ncb;
   const int hh = (blockIdx.x / ncb) % H;
   const int seq = blockIdx.x / (ncb * H);
-  const int t = threadIdx.x;
-  const int r0 = (t >> 2) * 2, c0 = (t & 3) * 4;  // rows r0, r0+1; columns c0 .. c0+3
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int r0 = warp * 16;                        // this warp's rows r0 .. r0+15
   const size_t sd = (size_t)DK * dv;               // one state [dk][dv]
-  const size_t col = (size_t)cb * CMB_COLS + c0;
+  const size_t colb = (size_t)cb * CMB_COLS;
   auto mptr = [&](int pp) { return Mws + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * DK * DK; };
   auto stage = [&](int pp, float* dst) {
     const float* M = mptr(pp);
@@ -1231,62 +1234,77 @@ __global__ void __launch_bounds__(256)
     cp_async_commit();
   };
   if (n_segs > 1) stage(0, sM0);
+  // x[nt][e]: rows r0+g (e = 0, 1) and r0+g+8 (e = 2, 3), columns nt*8 + 2q (+1)
   float x[2][4];
   {
-    const float* s0 = S0 ? S0 + ((size_t)seq * H + hh) * sd : nullptr;
+    const float* s0 = S0 ? S0 + ((size_t)seq * H + hh) * sd + colb : nullptr;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float4 v = s0 ? *reinterpret_cast<const float4*>(s0 + (size_t)(r0 + i) * dv + col)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-      x[i][0] = v.x, x[i][1] = v.y, x[i][2] = v.z, x[i][3] = v.w;
-    }
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const float2 v = s0 ? *reinterpret_cast<const float2*>(s0 + (size_t)(r0 + g + 8 * hr) * dv + nt * 8 + 2 * q)
+                            : make_float2(0.f, 0.f);
+        x[nt][2 * hr] = v.x;
+        x[nt][2 * hr + 1] = v.y;
+      }
   }
   for (int pp = 0;; ++pp) {
-    float* dst = Sst + (((size_t)seq * n_segs + pp) * H + hh) * sd + col;
+    float* dst = Sst + (((size_t)seq * n_segs + pp) * H + hh) * sd + colb;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float4 v = make_float4(x[i][0], x[i][1], x[i][2], x[i][3]);
-      *reinterpret_cast<float4*>(dst + (size_t)(r0 + i) * dv) = v;
-      *reinterpret_cast<float4*>(sS + (r0 + i) * CMB_COLS + c0) = v;
-    }
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const float2 v = make_float2(x[nt][2 * hr], x[nt][2 * hr + 1]);
+        const int r = r0 + g + 8 * hr, c = nt * 8 + 2 * q;
+        *reinterpret_cast<float2*>(dst + (size_t)r * dv + c) = v;
+        *reinterpret_cast<float2*>(sS + r * CMB_SLD + c) = v;
+      }
     if (pp + 1 >= n_segs) break;
     const bool prefetch = (pp + 2 < n_segs);
     if (prefetch) stage(pp + 1, ((pp + 1) & 1) ? sM1 : sM0);
     // B_pp is loaded now and added after the product, so its latency is hidden
-    const float* B = Bws + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + col;
-    float4 bv[2];
+    const float* B = Bws + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb;
+    float2 bv[2][2];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      bv[i] = *reinterpret_cast<const float4*>(B + (size_t)(r0 + i) * dv);
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) x[i][j] = 0.f;
-    }
+      for (int hr = 0; hr < 2; ++hr)
+        bv[nt][hr] = *reinterpret_cast<const float2*>(B + (size_t)(r0 + g + 8 * hr) * dv + nt * 8 + 2 * q);
     if (prefetch) cp_async_wait<1>(); else cp_async_wait<0>();
     __syncthreads();                                // M_pp and S_pp are in shared memory
     const float* M = (pp & 1) ? sM1 : sM0;
+    float acc[2][3][4];
 #pragma unroll
-    for (int e = 0; e < DK; e += 4) {
-      const float4 m0 = *reinterpret_cast<const float4*>(M + r0 * CMB_MLD + e);
-      const float4 m1 = *reinterpret_cast<const float4*>(M + (r0 + 1) * CMB_MLD + e);
-      const float mv[2][4] = {{m0.x, m0.y, m0.z, m0.w}, {m1.x, m1.y, m1.z, m1.w}};
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 sv = *reinterpret_cast<const float4*>(sS + (e + k) * CMB_COLS + c0);
+      for (int k = 0; k < 3; ++k)
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          x[i][0] = fmaf(mv[i][k], sv.x, x[i][0]);
-          x[i][1] = fmaf(mv[i][k], sv.y, x[i][1]);
-          x[i][2] = fmaf(mv[i][k], sv.z, x[i][2]);
-          x[i][3] = fmaf(mv[i][k], sv.w, x[i][3]);
-        }
+        for (int e = 0; e < 4; ++e) acc[nt][k][e] = 0.f;
+#pragma unroll 4
+    for (int k0 = 0; k0 < DK; k0 += 8) {
+      uint32_t ah[4], al[4];
+      split_tf32(M[(r0 + g) * CMB_MLD + k0 + q], ah[0], al[0]);
+      split_tf32(M[(r0 + g + 8) * CMB_MLD + k0 + q], ah[1], al[1]);
+      split_tf32(M[(r0 + g) * CMB_MLD + k0 + q + 4], ah[2], al[2]);
+      split_tf32(M[(r0 + g + 8) * CMB_MLD + k0 + q + 4], ah[3], al[3]);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t bh[2], bl[2];
+        split_tf32(sS[(k0 + q) * CMB_SLD + nt * 8 + g], bh[0], bl[0]);
+        split_tf32(sS[(k0 + q + 4) * CMB_SLD + nt * 8 + g], bh[1], bl[1]);
+        mma_tf32(acc[nt][0], ah, bh);
+        mma_tf32(acc[nt][1], ah, bl);
+        mma_tf32(acc[nt][2], al, bh);
       }
     }
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      x[i][0] += bv[i].x;
-      x[i][1] += bv[i].y;
-      x[i][2] += bv[i].z;
-      x[i][3] += bv[i].w;
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[nt][e] = acc[nt][0][e] + (acc[nt][1][e] + acc[nt][2][e]);
+      x[nt][0] += bv[nt][0].x;
+      x[nt][1] += bv[nt][0].y;
+      x[nt][2] += bv[nt][1].x;
+      x[nt][3] += bv[nt][1].y;
     }
     __syncthreads();                                // every read of S_pp and M_pp is done
   }

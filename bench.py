@@ -285,9 +285,10 @@ def run_ours(args, rank, world, local):
     gdn_bytes = prefill_bytes_per_token_head(wl.dk, wl.dv) * L * wl.H
     achieved = gdn_bytes / gdn_avg_s / 1e9
     hbm_peak = peaks["hbm_gbs"]
-    # this library's kernels per loop: the mixer (three launches on the segmented
-    # schedule, one otherwise) and the loop residual
-    mixer_launches = 3 if lla.prefill_workspace_bytes(1, L, wl.H, wl.dk, wl.dv) > 0 else 1
+    # this library's kernels per loop: the mixer (one launch per pass, plus the
+    # combine on the segmented schedule) and the loop residual
+    sched = lla.prefill_schedule(1, L, wl.H, wl.dk, wl.dv)
+    mixer_launches = sched["launches"]
     launches = args.steps * wl.loops * (mixer_launches + 1)
 
     # ---- end to end through host buffers (pinned), same step
@@ -335,8 +336,10 @@ def run_ours(args, rank, world, local):
                      "peak_source": peak_kind, "traffic": profiled_traffic(),
                      "algorithmic_bytes_per_launch": gdn_bytes,
                      "avg_launch_ms": gdn_avg_s * 1e3,
-                     "schedule": ("segmented: state pass, combine, output pass (3 launches per "
-                                  "mixer call, timed together)" if mixer_launches == 3
+                     "schedule": (f"segmented: {sched['n_segs']} segments of {sched['seg_tok']} "
+                                  "tokens; segment 0 in full beside the later segments' state "
+                                  f"pass, combine, output pass ({mixer_launches} launches per "
+                                  "mixer call, timed together)" if sched["n_segs"] > 1
                                   else "one pass per chain (1 launch per mixer call)")},
         "gpu_launches": launches,
         "e2e": e2e,

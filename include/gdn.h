@@ -114,17 +114,30 @@ typedef struct {
  * shapes, flags and the current device's SM count. */
 size_t gdn_chunk_fwd_workspace(const gdn_fwd_params *p);
 
+/* The schedule gdn_chunk_fwd takes for these parameters when it is given a
+ * workspace of gdn_chunk_fwd_workspace(p) bytes (host only, no device memory
+ * touched).  Any output pointer may be NULL.
+ *   n_segs:   1 = one pass per chain; >= 2 = segments of seg_tok tokens.
+ *   seg_tok:  0 for one pass.
+ *   launches: stream operations the call enqueues: 0 (nothing to do), 1 (one
+ *             pass, or the copy or clear of S_T when every sequence is empty),
+ *             2 (two segments: no combine step) or 3.
+ * Parameters gdn_chunk_fwd would reject return the same error status. */
+gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg_tok,
+                                  int *launches);
+
 /* Chunkwise prefill (chunks of 64 tokens).
  *
  * Schedule.  Each (sequence, head, 128-wide dv slice) chain normally runs in
  * one pass.  When fixed-length sequences (cu_seqlens == NULL) give too few
  * chains to fill the GPU, every sequence is instead cut into segments whose
- * state update is affine in the start state, S_end = M S_start + B: a first
- * launch computes each segment's B (from a zero state) and dk x dk transition
- * M, a second kernel chains the segment start states in fp32, and a third
- * launch runs every segment from its start state and writes the outputs
- * (three launches, all on `stream`).  The outputs equal the one-pass outputs up
- * to rounding.  GDN_SINGLE_PASS disables it.
+ * state update is affine in the start state, S_end = M S_start + B.  A first
+ * launch runs segment 0 in full from S0 and, beside it, computes every later
+ * segment's B (from a zero state) and dk x dk transition M, except the last
+ * segment's; a second kernel chains the segment start states in fp32 (skipped
+ * with two segments), and a third launch runs segments 1 .. P-1 from their
+ * start states and writes their outputs (all on `stream`).  The outputs equal
+ * the one-pass outputs up to rounding.  GDN_SINGLE_PASS disables it.
  *
  * ws/ws_bytes: device workspace of at least gdn_chunk_fwd_workspace(p) bytes,
  * 256-byte aligned, owned by the caller and not read back afterwards.

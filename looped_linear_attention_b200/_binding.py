@@ -67,6 +67,9 @@ def library() -> ctypes.CDLL:
         vp, i32, u32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_float
         lib.gdn_chunk_fwd_workspace.argtypes = [ctypes.POINTER(gdn_fwd_params)]
         lib.gdn_chunk_fwd_workspace.restype = ctypes.c_size_t
+        lib.gdn_chunk_fwd_schedule.argtypes = [ctypes.POINTER(gdn_fwd_params)] + [
+            ctypes.POINTER(ctypes.c_int)] * 3
+        lib.gdn_chunk_fwd_schedule.restype = i32
         lib.gdn_chunk_fwd.argtypes = [ctypes.POINTER(gdn_fwd_params), vp, ctypes.c_size_t, vp]
         lib.gdn_chunk_fwd.restype = i32
         lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
@@ -164,21 +167,39 @@ def gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     return o, S_T
 
 
+def _shape_params(n_seq, seq_len, H, dk, dv, dtype, flags, varlen):
+    T = n_seq * seq_len
+    fake = 1 << 40          # aligned placeholders: the queries only read shapes and flags
+    return gdn_fwd_params(fake, fake + (1 << 36), fake + (2 << 36), fake + (3 << 36),
+                          fake + (4 << 36), None, fake + (5 << 36), None,
+                          fake + (6 << 36) if varlen else None, n_seq, 0 if varlen else seq_len, T,
+                          H, dk, dv, _DTYPES[dtype], 1.0, int(flags))
+
+
 def prefill_workspace_bytes(n_seq: int, seq_len: int, H: int, dk: int, dv: int,
                             dtype: torch.dtype = torch.bfloat16, flags: int = 0,
                             varlen: bool = False) -> int:
     """gdn_chunk_fwd_workspace for a call of this shape (no device memory is
-    touched).  Non-zero means the segmented schedule: three launches per call."""
-    T = n_seq * seq_len
-    fake = 1 << 40          # aligned placeholders: the query only reads shapes and flags
-    p = gdn_fwd_params(fake, fake + (1 << 36), fake + (2 << 36), fake + (3 << 36),
-                       fake + (4 << 36), None, fake + (5 << 36), None,
-                       fake + (6 << 36) if varlen else None, n_seq, 0 if varlen else seq_len, T,
-                       H, dk, dv, _DTYPES[dtype], 1.0, int(flags))
+    touched).  Non-zero means the segmented schedule."""
+    p = _shape_params(n_seq, seq_len, H, dk, dv, dtype, flags, varlen)
     ws = library().gdn_chunk_fwd_workspace(ctypes.byref(p))
     if ws == ctypes.c_size_t(-1).value:
         raise GdnError(GDN_ERR_INVALID, "gdn_chunk_fwd_workspace")
     return int(ws)
+
+
+def prefill_schedule(n_seq: int, seq_len: int, H: int, dk: int, dv: int,
+                     dtype: torch.dtype = torch.bfloat16, flags: int = 0,
+                     varlen: bool = False) -> dict:
+    """gdn_chunk_fwd_schedule for a call of this shape, given its workspace:
+    {"n_segs", "seg_tok", "launches"} (n_segs = 1: one pass per chain)."""
+    p = _shape_params(n_seq, seq_len, H, dk, dv, dtype, flags, varlen)
+    n, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    st = library().gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok),
+                                          ctypes.byref(launches))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd_schedule")
+    return {"n_segs": n.value, "seg_tok": tok.value, "launches": launches.value}
 
 
 def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,

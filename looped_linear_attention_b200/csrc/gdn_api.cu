@@ -135,6 +135,22 @@ size_t gdn_chunk_fwd_workspace(const gdn_fwd_params* p) {
   return gdn::prefill_segment_workspace(p, gdn::plan_prefill_segments(p, sm_count()));
 }
 
+gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params* p, int* n_segs, int* seg_tok, int* launches) {
+  const gdn_status v = validate_fwd(p);
+  if (v != GDN_OK) return v;
+  gdn::SegPlan plan{1, 0};
+  if (p->total_tokens > 0 && gdn::prefill_tc_supported(p)) plan = gdn::plan_prefill_segments(p, sm_count());
+  int n = 1;                                           // one pass
+  if (p->n_seq == 0) n = 0;
+  else if (p->total_tokens == 0) n = (p->S_T && p->S0 != p->S_T) ? 1 : 0;   // a copy or a clear of S_T
+  else if (plan.n_segs > 2) n = 3;
+  else if (plan.n_segs == 2) n = 2;
+  if (n_segs) *n_segs = plan.n_segs;
+  if (seg_tok) *seg_tok = plan.seg_tok;
+  if (launches) *launches = n;
+  return GDN_OK;
+}
+
 gdn_status gdn_chunk_fwd(const gdn_fwd_params* p, void* ws, size_t ws_bytes,
                          cudaStream_t stream) {
   const gdn_status v = validate_fwd(p);

@@ -134,18 +134,20 @@ struct Params {
   int n_seq, seq_len, total_tokens, H, dv, n_slices;
   float scale;
   unsigned flags;
-  // Segment schedule (fixed-length sequences cut into n_segs segments of
+  // Segment schedule (fixed-length sequences cut into n_segs >= 2 segments of
   // seg_tok tokens; mode 0 runs whole sequences in one pass):
-  //   mode 1: segments 0 .. n_segs-2 from a zero state, no outputs.  Slices
-  //           0 .. n_slices-1 write the segment's state contribution to Bws;
-  //           one extra slice runs V = 0 from the identity and writes the
-  //           segment's dk x dk transition to Mws.
-  //   mode 2: every segment from its start state in Sst, with outputs; the last
-  //           segment writes S_T.
+  //   mode 1: segment 0 runs in full from S0 (outputs, and its end state S_1
+  //           to Sst slot 0); the CTAs after those run segments 1 .. n_segs-2
+  //           from a zero state without outputs.  Their slices 0 .. n_slices-1
+  //           write the segment's state contribution B_p to Bws slot p-1; one
+  //           extra slice runs V = 0 from the identity and writes the
+  //           segment's dk x dk transition M_p to Mws slot p-1.
+  //   mode 2: segments 1 .. n_segs-1 from their start states S_p in Sst slot
+  //           p-1, with outputs; the last segment writes S_T.
   int mode, n_segs, seg_tok;
-  float* Bws;          // [n_seq][n_segs-1][H][dk][dv]
-  float* Mws;          // [n_seq][n_segs-1][H][dk][dk]
-  const float* Sst;    // [n_seq][n_segs][H][dk][dv]
+  float* Bws;          // [n_seq][n_segs-2][H][dk][dv]
+  float* Mws;          // [n_seq][n_segs-2][H][dk][dk]
+  float* Sst;          // [n_seq][n_segs-1][H][dk][dv]
 };
 
 // Per-chunk gate vectors (one buffer).
@@ -601,16 +603,34 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);   // warp-uniform by construction
 
   // work unit: (sequence or segment, head, dv slice)
-  const int slices_here = p.n_slices + (p.mode == 1 ? 1 : 0);
-  const int slice = blockIdx.x % slices_here;
-  const int chain = blockIdx.x / slices_here;
-  const int h = chain % p.H;
-  const int unit = chain / p.H;
-  const int units_per_seq = (p.mode == 0) ? 1 : (p.mode == 1 ? p.n_segs - 1 : p.n_segs);
-  const int seq = unit / units_per_seq;
-  const int part = unit % units_per_seq;
-  const bool ident = (p.mode == 1 && slice == p.n_slices);   // transition slice: V = 0, S0 = I
-  const bool outputs = (p.mode != 1);
+  int slice, h, seq, part;
+  bool partial = false;   // a segment run from a zero state or the identity, without outputs
+  {
+    int bid = (int)blockIdx.x;
+    int slices_here = p.n_slices;
+    int units_per_seq = 1, first_part = 0;
+    if (p.mode == 1) {
+      const int n_first = p.n_seq * p.H * p.n_slices;   // segment 0 of every chain, run in full
+      if (bid >= n_first) {
+        bid -= n_first;
+        partial = true;
+        slices_here = p.n_slices + 1;
+        units_per_seq = p.n_segs - 2;
+        first_part = 1;
+      }
+    } else if (p.mode == 2) {
+      units_per_seq = p.n_segs - 1;
+      first_part = 1;
+    }
+    slice = bid % slices_here;
+    const int chain = bid / slices_here;
+    h = chain % p.H;
+    const int unit = chain / p.H;
+    seq = unit / units_per_seq;
+    part = first_part + unit % units_per_seq;
+  }
+  const bool ident = partial && slice == p.n_slices;   // transition slice: V = 0, S0 = I
+  const bool outputs = !partial;
   int seq_start, seq_end;
   if (p.cu_seqlens) {
     seq_start = p.cu_seqlens[seq];
@@ -879,8 +899,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (p.mode == 0) {
       s0 = p.S0 ? p.S0 + state_base : nullptr;
       st = p.S_T ? p.S_T + state_base : nullptr;
+    } else if (p.mode == 1 && !partial) {   // segment 0: S_1 to start-state slot 0
+      s0 = p.S0 ? p.S0 + state_base : nullptr;
+      st = p.Sst + ((size_t)seq * (p.n_segs - 1) * H + h) * DK * (size_t)dv + col0 + j;
     } else if (p.mode == 1) {
-      const size_t u = (size_t)seq * (p.n_segs - 1) + part;
+      const size_t u = (size_t)seq * (p.n_segs - 2) + (part - 1);
       if (ident) {
         st = p.Mws + (u * H + h) * DK * DK + j;
         ldT = DK;
@@ -888,7 +911,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         st = p.Bws + (u * H + h) * DK * (size_t)dv + col0 + j;
       }
     } else {
-      s0 = p.Sst + (((size_t)seq * p.n_segs + part) * H + h) * DK * (size_t)dv + col0 + j;
+      s0 = p.Sst + (((size_t)seq * (p.n_segs - 1) + (part - 1)) * H + h) * DK * (size_t)dv + col0 + j;
       if (part == p.n_segs - 1 && p.S_T) st = p.S_T + state_base;
     }
     uint32_t sphase = 0;
@@ -1185,8 +1208,9 @@ bool prefill_tc_supported(const gdn_fwd_params* p) {
 
 // ------------------------------------------------------------------ segments
 // Combine step of the segmented schedule: for one (sequence, head) and 16
-// columns of dv, S_0 = S0 (or 0) and S_{p+1} = M_p S_p + B_p for p = 0 .. n_segs-2,
-// with every S_p written to Sst.  The products run on the warp-level tensor
+// columns of dv, S_{p+1} = M_p S_p + B_p for p = 1 .. n_segs-2, starting from
+// S_1 (written by the segment-0 CTAs) and writing every S_p, p >= 2, to Sst
+// (slot p-1; M_p and B_p sit in slot p-1 of theirs).  The products run on the warp-level tensor
 // cores with the 3xTF32 split (fp32-level accuracy): warp w owns rows
 // 16w .. 16w+15 of the 128 x 16 block.  M_p (dk x dk) is staged in shared
 // memory by cp.async one step ahead (double buffer).
@@ -1207,9 +1231,8 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 __global__ void __launch_bounds__(256)
-    gdn_segment_combine_kernel(const float* __restrict__ S0, const float* __restrict__ Bws,
-                               const float* __restrict__ Mws, float* __restrict__ Sst, int H, int dv,
-                               int n_segs) {
+    gdn_segment_combine_kernel(const float* __restrict__ Bws, const float* __restrict__ Mws,
+                               float* __restrict__ Sst, int H, int dv, int n_segs) {
   extern __shared__ __align__(16) float cmb_smem[];
   float* sM0 = cmb_smem;
   float* sM1 = cmb_smem + DK * CMB_MLD;
@@ -1223,7 +1246,10 @@ __global__ void __launch_bounds__(256)
   const int r0 = warp * 16;                        // this warp's rows r0 .. r0+15
   const size_t sd = (size_t)DK * dv;               // one state [dk][dv]
   const size_t colb = (size_t)cb * CMB_COLS;
-  auto mptr = [&](int pp) { return Mws + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * DK * DK; };
+  // slot i holds M_{i+1}, B_{i+1} and S_{i+1}; n_steps products chain S_1 .. S_{n_segs-1}
+  const int n_steps = n_segs - 2;
+  auto mptr = [&](int pp) { return Mws + (((size_t)seq * n_steps + pp) * H + hh) * DK * DK; };
+  auto sptr = [&](int pp) { return Sst + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb; };
   auto stage = [&](int pp, float* dst) {
     const float* M = mptr(pp);
 #pragma unroll 4
@@ -1233,37 +1259,34 @@ __global__ void __launch_bounds__(256)
     }
     cp_async_commit();
   };
-  if (n_segs > 1) stage(0, sM0);
+  if (n_steps <= 0) return;
+  stage(0, sM0);
   // x[nt][e]: rows r0+g (e = 0, 1) and r0+g+8 (e = 2, 3), columns nt*8 + 2q (+1)
   float x[2][4];
-  {
-    const float* s0 = S0 ? S0 + ((size_t)seq * H + hh) * sd + colb : nullptr;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+  for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const float2 v = s0 ? *reinterpret_cast<const float2*>(s0 + (size_t)(r0 + g + 8 * hr) * dv + nt * 8 + 2 * q)
-                            : make_float2(0.f, 0.f);
-        x[nt][2 * hr] = v.x;
-        x[nt][2 * hr + 1] = v.y;
-      }
-  }
+    for (int hr = 0; hr < 2; ++hr) {
+      const float2 v = *reinterpret_cast<const float2*>(sptr(0) + (size_t)(r0 + g + 8 * hr) * dv + nt * 8 + 2 * q);
+      x[nt][2 * hr] = v.x;
+      x[nt][2 * hr + 1] = v.y;
+    }
   for (int pp = 0;; ++pp) {
-    float* dst = Sst + (((size_t)seq * n_segs + pp) * H + hh) * sd + colb;
+    // S_{pp+1} (x) to the operand block, and to Sst unless it came from there
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const float2 v = make_float2(x[nt][2 * hr], x[nt][2 * hr + 1]);
         const int r = r0 + g + 8 * hr, c = nt * 8 + 2 * q;
-        *reinterpret_cast<float2*>(dst + (size_t)r * dv + c) = v;
+        if (pp > 0) *reinterpret_cast<float2*>(sptr(pp) + (size_t)r * dv + c) = v;
         *reinterpret_cast<float2*>(sS + r * CMB_SLD + c) = v;
       }
-    if (pp + 1 >= n_segs) break;
-    const bool prefetch = (pp + 2 < n_segs);
+    if (pp >= n_steps) break;
+    const bool prefetch = (pp + 1 < n_steps);
     if (prefetch) stage(pp + 1, ((pp + 1) & 1) ? sM1 : sM0);
-    // B_pp is loaded now and added after the product, so its latency is hidden
-    const float* B = Bws + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb;
+    // B is loaded now and added after the product, so its latency is hidden
+    const float* B = Bws + (((size_t)seq * n_steps + pp) * H + hh) * sd + colb;
     float2 bv[2][2];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -1315,7 +1338,10 @@ __global__ void __launch_bounds__(256)
 // chain; otherwise fixed-length sequences are cut into n_segs segments of
 // seg_tok tokens.  The cost model counts chunk steps on the critical path:
 // waves of CTAs (one CTA per SM) times chunks per CTA, for the one-pass launch
-// against the two segmented launches plus the combine.
+// against the two segmented launches plus the combine.  The first segmented
+// launch holds segment 0 of every chain (run in full) and segments
+// 1 .. n_segs-2 with one transition slice each; the second holds segments
+// 1 .. n_segs-1.
 SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
   SegPlan plan{1, 0};
   if (!prefill_tc_supported(p) || p->cu_seqlens || (p->flags & GDN_SINGLE_PASS) || p->n_seq <= 0 ||
@@ -1333,8 +1359,9 @@ SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
     if (P < 2) break;
     // a launch wave costs its chunks plus about 1.5 chunk steps of pipeline
     // fill and drain; a combine step about 0.8 of a chunk step
-    const double cost = waves(chains * (P - 1) * (slices + 1)) * (seg + 1.5) +
-                        waves(chains * P * slices) * (seg + 1.5) + 0.8 * (P - 1) + 0.5;
+    const double cost = waves(chains * (slices + (long long)(P - 2) * (slices + 1))) * (seg + 1.5) +
+                        waves(chains * (P - 1) * slices) * (seg + 1.5) +
+                        (P > 2 ? 0.8 * (P - 2) + 0.5 : 0.0);
     if (cand.n_segs == 1 || cost < best) {
       best = cost;
       cand = SegPlan{P, seg * tc::C};
@@ -1351,8 +1378,8 @@ size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan) {
   const size_t sd = (size_t)p->H * tc::DK * p->dv * sizeof(float);
   const size_t md = (size_t)p->H * tc::DK * tc::DK * sizeof(float);
   const size_t n = (size_t)p->n_seq;
-  return align256(n * (plan.n_segs - 1) * sd) + align256(n * (plan.n_segs - 1) * md) +
-         align256(n * plan.n_segs * sd);
+  return align256(n * (plan.n_segs - 2) * sd) + align256(n * (plan.n_segs - 2) * md) +
+         align256(n * (plan.n_segs - 1) * sd);
 }
 
 static gdn_status tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -1401,36 +1428,38 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   const long long chains = (long long)p->n_seq * p->H;
   if (plan.n_segs <= 1) return tc_launch(mq, mk, mv, kp, chains * kp.n_slices, stream);
 
-  // segmented: workspace = [B | M | start states]
+  // segmented: workspace = [B_1 .. B_{P-2} | M_1 .. M_{P-2} | S_1 .. S_{P-1}]
   const int P = plan.n_segs;
   const size_t sd = (size_t)p->H * tc::DK * p->dv * sizeof(float);
   const size_t md = (size_t)p->H * tc::DK * tc::DK * sizeof(float);
   char* w = static_cast<char*>(ws);
   kp.Bws = reinterpret_cast<float*>(w);
-  w += align256((size_t)p->n_seq * (P - 1) * sd);
+  w += align256((size_t)p->n_seq * (P - 2) * sd);
   kp.Mws = reinterpret_cast<float*>(w);
-  w += align256((size_t)p->n_seq * (P - 1) * md);
-  float* sst = reinterpret_cast<float*>(w);
-  kp.Sst = sst;
+  w += align256((size_t)p->n_seq * (P - 2) * md);
+  kp.Sst = reinterpret_cast<float*>(w);
   kp.n_segs = P;
   kp.seg_tok = plan.seg_tok;
   kp.mode = 1;
-  gdn_status st = tc_launch(mq, mk, mv, kp, chains * (P - 1) * (kp.n_slices + 1), stream);
+  gdn_status st =
+      tc_launch(mq, mk, mv, kp, chains * (kp.n_slices + (long long)(P - 2) * (kp.n_slices + 1)), stream);
   if (st != GDN_OK) return st;
-  const long long cblocks = chains * (p->dv / tc::CMB_COLS);
-  if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
-  static bool cmb_attr_set = false;
-  if (!cmb_attr_set) {
-    if (cudaFuncSetAttribute(tc::gdn_segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::CMB_SMEM) != cudaSuccess)
-      return GDN_ERR_CUDA;
-    cmb_attr_set = true;
+  if (P > 2) {
+    const long long cblocks = chains * (p->dv / tc::CMB_COLS);
+    if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    static bool cmb_attr_set = false;
+    if (!cmb_attr_set) {
+      if (cudaFuncSetAttribute(tc::gdn_segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc::CMB_SMEM) != cudaSuccess)
+        return GDN_ERR_CUDA;
+      cmb_attr_set = true;
+    }
+    tc::gdn_segment_combine_kernel<<<(unsigned)cblocks, 256, tc::CMB_SMEM, stream>>>(kp.Bws, kp.Mws, kp.Sst,
+                                                                                   p->H, p->dv, P);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   }
-  tc::gdn_segment_combine_kernel<<<(unsigned)cblocks, 256, tc::CMB_SMEM, stream>>>(p->S0, kp.Bws, kp.Mws, sst,
-                                                                                 p->H, p->dv, P);
-  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   kp.mode = 2;
-  return tc_launch(mq, mk, mv, kp, chains * P * kp.n_slices, stream);
+  return tc_launch(mq, mk, mv, kp, chains * (P - 1) * kp.n_slices, stream);
 }
 
 }  // namespace gdn

@@ -97,14 +97,22 @@ def _state_set(H, dk, dv):
 
 def test_workspace_segmented_schedule_for_few_long_chains(lib):
     """One 4096-token sequence x 16 heads fills 16 of 148 SMs in one pass: the
-    query asks for the segmented schedule's buffers, B and M (dk = dv here) for
-    P-1 segments and start states for P, i.e. (3P - 2) state sets, P >= 2."""
+    query asks for the segmented schedule's buffers.  Segment 0 runs in full
+    from S0, so B and M (dk = dv here) are kept for segments 1 .. P-2 and start
+    states for segments 1 .. P-1, i.e. (3P - 5) state sets, P >= 2; the
+    schedule query reports the same P."""
     p = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16)
     sd = _state_set(16, 128, 128)
     need = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
     assert need > 0 and need % sd == 0
     sets = need // sd
-    assert (sets + 2) % 3 == 0 and 2 <= (sets + 2) // 3 <= 64
+    assert (sets + 5) % 3 == 0 and 2 <= (sets + 5) // 3 <= 64
+    n, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok),
+                                      ctypes.byref(launches)) == B.GDN_OK
+    P = (sets + 5) // 3
+    assert n.value == P and (P - 1) * tok.value < 4096 <= P * tok.value and tok.value % 64 == 0
+    assert launches.value == (3 if P > 2 else 2)
 
 
 @pytest.mark.parametrize("kw", [
@@ -120,6 +128,21 @@ def test_workspace_zero_for_one_pass_schedules(lib, kw):
     kw.setdefault("total_tokens", kw["n_seq"] * kw["seq_len"])
     p = _params(**kw)
     assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
+    n, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok),
+                                      ctypes.byref(launches)) == B.GDN_OK
+    assert (n.value, tok.value, launches.value) == (1, 0, 1)
+
+
+def test_schedule_query_rejects_what_the_call_rejects(lib):
+    p = _params(dk=96)                                    # dk outside {64, 128}
+    bad = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
+    assert bad == ctypes.c_size_t(-1).value
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), None, None, None) != B.GDN_OK
+    empty = _params(n_seq=0, seq_len=64, total_tokens=0)
+    launches = ctypes.c_int(-1)
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(empty), None, None, ctypes.byref(launches)) == B.GDN_OK
+    assert launches.value == 0
 
 
 def test_workspace_zero_for_varlen(lib):

@@ -185,9 +185,11 @@ def test_prefill_tc_strong_and_mixed_decay():
 
 
 def test_prefill_tc_segmented_equals_single_pass_and_oracle():
-    """Few long chains take the segmented schedule (segment contributions from a
-    zero state and dk x dk transitions, chained in fp32, then every segment from
-    its start state); GDN_SINGLE_PASS runs the same inputs as one pass per chain."""
+    """Few long chains take the segmented schedule (segment 0 in full from S0;
+    later segments' contributions from a zero state and dk x dk transitions,
+    chained in fp32, then segments 1 .. P-1 from their start states); two
+    sequences, so every per-sequence slot of the workspace is used.
+    GDN_SINGLE_PASS runs the same inputs as one pass per chain."""
     wl = _wl("long_prefill", n_seq=2, H=2, seq_len=1000, random_s0=True)
     assert lla.prefill_workspace_bytes(2, 1000, 2, 128, 128) > 0
     inp = W.prefill_inputs(wl, "cpu")

@@ -52,8 +52,8 @@ def _params(inp, o, S_T):
 
 
 def test_noalloc_matches_gdn_chunk_fwd_on_two_calls(lib):
-    """One 4096-token sequence x 16 heads: the segmented schedule (22 MB of
-    scratch, within the 32 MiB array)."""
+    """One 4096-token sequence x 16 heads: the segmented schedule, whose
+    scratch fits the 32 MiB array."""
     n_seq, H, L = 1, 16, 4096
     need = lla.prefill_workspace_bytes(n_seq, L, H, 128, 128)
     assert 0 < need <= SCRATCH_BYTES

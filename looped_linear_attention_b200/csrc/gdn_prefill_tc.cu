@@ -16,24 +16,27 @@
 // Sigma_t = a_t Sigma_{t-1} + k_t u_t^T, and the three lines above follow by
 // unrolling that inside the chunk.
 //
-// Data path (one CTA per (sequence, head, 128-wide slice of dv); three roles:
-// a prep warpgroup builds the state-independent operands of chunk c+1 -- gates,
-// G, A, P, T, T1, T2, U~, W^T -- while a state warpgroup runs chunk c -- the
+// Data path (one CTA per (sequence, head, 128-wide slice of dv); two teams of
+// eight warps: a prep team builds the state-independent operands of chunk c+1
+// -- A, P, T, T1, T2, U~, W^T -- while a state team runs chunk c -- the
 // Sigma-dependent MMAs, the U^T operands, the state refresh and the outputs --
-// and a producer warp streams K, Q (2 stages) and V (1 stage) in by TMA.  Each
-// warpgroup issues its own MMAs; the hand-offs are mbarriers indexed by buffer
+// and, two chunks ahead, the gate vectors, the K/Q loads and the G product.
+// Each team issues its own MMAs; the hand-offs are mbarriers indexed by buffer
 // slot, so no waiter can fall two phases behind):
 //   * every product is issued TRANSPOSED so its M dimension is 128 (dv rows of
 //     Sigma^T, dk rows of W^T, or the stacked [K; Q] rows) and lands in tensor
 //     memory with lane = row: G = [K;Q] K^T, U^T = V^T T2^T - Sigma^T W^T,
 //     W^T = K^T T1^T, O_A^T = Sigma^T Q^T, O_B^T = U^T P^T,
 //     Sigma^T += (U^T diag(gamma_C/gamma)) K.
-//   * q, k, v tiles arrive by TMA (128-byte swizzle) into a 2-stage ring filled
-//     by a producer warp; K and V are read straight from their tiles as
-//     MN-major operands.  Operands computed in the CTA (T1, T2, P, W^T, U^T,
-//     Sigma^T) are rounded to bf16 and written as whole 16-byte chunks in the
-//     same swizzled layout (W^T is an MN-major B operand, so every thread
-//     writes one contiguous row).
+//   * q, k, v tiles arrive by TMA (128-byte swizzle; K and Q in a 2-stage
+//     ring, V in one stage); K and V are read straight from their tiles as
+//     MN-major operands.  With the q/k L2 norm the tiles stay as loaded: the
+//     inverse row norms are folded into the fp32 factors that meet q and k
+//     (the row and column factors of A and P, T1's column scale, the carry's
+//     gamma_C / gamma and the output's gamma).  Operands computed in the CTA
+//     (T1, T2, P, W^T, U^T, Sigma^T) are rounded to bf16 and written as whole
+//     16-byte chunks in the same swizzled layout (W^T is an MN-major B
+//     operand, so every thread writes one contiguous row).
 //   * the fp32 master state stays in tensor memory for the whole sequence,
 //     kept pre-multiplied by the next chunk's gamma_C so that the carry MMA
 //     accumulates straight onto it; its bf16 copy in shared memory feeds the
@@ -51,10 +54,11 @@ constexpr int C = 64;            // chunk length
 constexpr int DK = 128;          // key/query width (this kernel)
 constexpr int DVS = 128;         // dv slice per CTA
 constexpr int WG = 128;          // one warpgroup (tensor-memory lanes 0-127)
-// warps 0-7:  prep team (state-independent part of chunk c+1); its thread 0
+// warps 0-7:  prep team (state-independent part of chunk c+1); its warp 0
 //             also issues the TMA loads of V (one stage)
-// warps 8-15: state team (state-dependent part of chunk c); its thread 0 also
-//             issues the TMA loads of K and Q (two stages)
+// warps 8-15: state team (state-dependent part of chunk c); it also issues
+//             the TMA loads of K and Q (two stages), folds their norms and
+//             issues their G product
 // Warps w and w+4 of a team reach the same 32 tensor-memory lanes (w mod 4) and
 // split the columns of each row between them; 4 warps per SM sub-partition
 // with up to 128 registers per thread.
@@ -99,7 +103,7 @@ constexpr uint32_t LT_BYTES = 10 * BLK_FLOATS * 4;
 constexpr uint32_t OFF_A = 196608;                    // A, compact blocks
 constexpr uint32_t OFF_TS = OFF_A + LT_BYTES;         // T, compact blocks (also the solve's scratch)
 constexpr uint32_t OFF_GATE = OFF_TS + LT_BYTES;      // 3 buffers of gate vectors (struct Gates)
-constexpr uint32_t GATE_BYTES = 8 * 64 * 4;
+constexpr uint32_t GATE_BYTES = 11 * 64 * 4;
 constexpr uint32_t OFF_BAR = OFF_GATE + 3 * GATE_BYTES;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;          // tmem base, abort flag, scan carry
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
@@ -160,11 +164,18 @@ struct Gates {
   float* e;      // 2^(g2_i - m), m = (g2_0 + g2_{C-1}) / 2 (row factor of D)
   float* f;      // 2^(m - g2_j) (column factor of D)
   float* flag;   // [0]: 1 when |g2_0 - g2_{C-1}| < 64, so that e_i f_j = D_ij in range
+  // With the q/k L2 norm the tiles stay as loaded and the prep team folds the
+  // inverse row norms into the factors that meet them (at the top of the chunk):
+  // r, bg and f take 1/|k_j| (f becomes 1/|k_j| alone when flag is 0), and
+  float* gq;     // gamma_i / |q_i| (output factor of Sigma^T Q^T)
+  float* kn;     // 1 / |k_i|
+  float* qn;     // 1 / |q_i|
 };
 
 __device__ __forceinline__ Gates gates_at(uint8_t* sm, int buf) {
   float* base = reinterpret_cast<float*>(sm + OFF_GATE + buf * GATE_BYTES);
-  return Gates{base, base + 64, base + 128, base + 192, base + 256, base + 320, base + 384, base + 448};
+  return Gates{base,       base + 64,  base + 128, base + 192, base + 256, base + 320,
+               base + 384, base + 448, base + 512, base + 576, base + 640};
 }
 
 // Named barrier of one warpgroup (the warp is reconverged first: the barrier is
@@ -210,33 +221,43 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t saddr, uint32_t lbo) {
 
 // Normalise one 128-element bf16 row of a [K0|Q0|K1|Q1] stage tile in place:
 // x / sqrt(sum x^2 + eps) in fp32, rounded to bf16.
-__device__ __forceinline__ void l2norm_row(uint8_t* kq, int row_in_tile, uint32_t tile_off) {
-  // two passes over the row in shared memory (sum of squares, then scale), so
-  // that the row is never held in registers whole
-  float ss = 0.f;
+// Inverse L2 norms of the chunk's 64 K rows and 64 Q rows (one stage of K/Q
+// tiles, as loaded) for the 256 threads of a team, two threads per row, each
+// summing the squares of one 64-column slab; the factors are folded into the
+// chunk's gate vectors (see struct Gates).  Every thread of the team calls it
+// (warp shuffles); it reads shared memory only, so after a failed wait it just
+// produces values that the abort discards.
+__device__ __forceinline__ void fold_qk_norms(const uint8_t* kq, const Gates& G, int t) {
+  const int row = t >> 1, slab = t & 1;            // rows 0-63: K, 64-127: Q
+  const int r = row & 63;
+  const uint32_t base = (row < C ? 0u : 8192u) + slab * 16384u;
+  uint4 v[8];                                      // all loads first, then the sums
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint32_t off = tile_off + (c >> 3) * 16384 + sw128_offset(row_in_tile, (c & 7) * 8);
-    const uint4 v = *reinterpret_cast<const uint4*>(kq + off);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(kq + base + sw128_offset(r, c * 8));
+  float ss[4] = {0.f, 0.f, 0.f, 0.f};              // four independent partial sums
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float lo = bf16_lo(w[e]), hi = bf16_hi(w[e]);
-      ss = fmaf(lo, lo, ss);
-      ss = fmaf(hi, hi, ss);
+      ss[e] = fmaf(lo, lo, ss[e]);
+      ss[e] = fmaf(hi, hi, ss[e]);
     }
   }
-  const float inv = 1.0f / sqrtf(ss + kQkNormEps);
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint32_t off = tile_off + (c >> 3) * 16384 + sw128_offset(row_in_tile, (c & 7) * 8);
-    const uint4 v = *reinterpret_cast<const uint4*>(kq + off);
-    uint4 o;
-    o.x = pack_bf16x2(bf16_lo(v.x) * inv, bf16_hi(v.x) * inv);
-    o.y = pack_bf16x2(bf16_lo(v.y) * inv, bf16_hi(v.y) * inv);
-    o.z = pack_bf16x2(bf16_lo(v.z) * inv, bf16_hi(v.z) * inv);
-    o.w = pack_bf16x2(bf16_lo(v.w) * inv, bf16_hi(v.w) * inv);
-    *reinterpret_cast<uint4*>(kq + off) = o;
+  float sum = (ss[0] + ss[1]) + (ss[2] + ss[3]);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  const float inv = rsqrtf(sum + kQkNormEps);
+  if (slab == 0) {
+    if (row < C) {
+      G.kn[r] = inv;
+      G.r[r] *= inv;
+      G.bg[r] *= inv;
+      G.f[r] = (G.flag[0] != 0.f ? G.f[r] : 1.f) * inv;
+    } else {
+      G.qn[r] = inv;
+      G.gq[r] = G.gamma[r] * inv;
+    }
   }
 }
 
@@ -582,7 +603,6 @@ __device__ __forceinline__ void load_v(uint8_t* sm, uint64_t* bar, const CUtenso
   tma_load_3d(sm + OFF_V, tv, bar, col0, h, tok0);
   tma_load_3d(sm + OFF_V + 8192, tv, bar, col0 + 64, h, tok0);
 }
-
 __global__ void __launch_bounds__(THREADS, 1)
     gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -704,44 +724,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     uint32_t pphase = 0;
     const bool l2n = (p.flags & GDN_QK_L2NORM) != 0;
-    // K, Q of chunk c with the optional in-place L2 norm: the team waits for the
-    // tiles and threads 0-127 normalise one row each (K rows 0-63, Q rows 64-127)
-    auto kq_normalise = [&](int c) -> bool {
-      const int s = c & 1;
-      if (!wg_wait<BAR_PREP>(&bars[B_KQ_FULL + s], (c >> 1) & 1, s_abort, p.status)) return false;
-      if (t < WG) l2norm_row(sm + OFF_KQ + s * KQ_BYTES, t & 63, t < 64 ? 0u : 8192u);
-      fence_proxy_async_smem();
-      wg_sync<BAR_PREP>();
-      return true;
-    };
-    // G = [K; Q] K^T of chunk c into tensor-memory buffer c % 2 (M = 128, N = 64,
-    // K = dk), issued by warp 0 (which alone waits for the tiles when no norm is
-    // applied).  Returns false if a wait gave up.
-    auto issue_g = [&](int c) -> bool {
-      const int s = c & 1;
-      bool okw = true;
-      if (!l2n) okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_KQ_FULL + s], (c >> 1) & 1, s_abort, p.status));
-      tc_fence_after();
-      if (okw) {
-        const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < DK / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16(tmem + col_gw(c), kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
-                     kk > 0);
-          }
-          mma_commit(&bars[B_G_MMA + s]);
-        }
-      }
-      __syncwarp();
-      return okw;
-    };
     bool ok = true;
-    if (n_chunks > 0) {
-      if (l2n) ok = kq_normalise(0);
-      if (ok && warp == 0) issue_g(0);   // a failed wait sets the abort flag, seen below
-    }
 #pragma unroll 1
     for (int c = 0; c < n_chunks && ok; ++c) {
       const int s = c & 1;
@@ -749,9 +732,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const Gates G = gates_at(sm, c % 3);
       const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
 
-      // ---- G of chunk c, its gates (from the state warpgroup), and the P and U
-      // buffers s (free once chunk c-2 is finished): each thread waits on the
-      // three barriers, then one warpgroup barrier makes the outcome uniform
+      // ---- G of chunk c and its gate vectors (both from the state team, the
+      // gates with the q/k norms folded in), and the P and U buffers s (free
+      // once chunk c-2 is finished): each thread waits on the three barriers,
+      // then one team barrier makes the outcome uniform
       {
         bool okw = mbar_wait_bounded(&bars[B_G_MMA + s], (c >> 1) & 1, s_abort, p.status);
         okw = okw && mbar_wait_bounded(&bars[B_GATES + c % 3], (c / 3) & 1, s_abort, p.status);
@@ -771,7 +755,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int i = tq & 63;
         const int cb = hf * 32;                         // first column of this thread
         const bool zero_half = (hf == 1) && ((warp & 1) == 0);
-        const float sc = (tq < C) ? G.b[i] : 1.f;
+        // row factor: b_i (A rows) or 1 (P rows), times the row's inverse norm;
+        // the column factor f_j carries 1/|k_j| (and is 1/|k_j| alone on the
+        // exponential path)
+        const float sc = (tq < C) ? (l2n ? G.b[i] * G.kn[i] : G.b[i]) : (l2n ? G.qn[i] : 1.f);
         const int lim = (tq < C) ? i : i + 1;           // columns j < lim are kept
         float gr[32];
         if (zero_half) {
@@ -797,11 +784,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j4 = 0; j4 < 8; ++j4) {
               const float4 gj = *reinterpret_cast<const float4*>(G.g2 + cb + 4 * j4);
               const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+              const float4 f4 = l2n ? *reinterpret_cast<const float4*>(G.f + cb + 4 * j4)
+                                    : make_float4(1.f, 1.f, 1.f, 1.f);
+              const float fv[4] = {f4.x, f4.y, f4.z, f4.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int jj = cb + 4 * j4 + e;
                 const float d = ex2_approx(gi - gjv[e]);
-                gr[4 * j4 + e] = (jj < lim) ? (sc * gr[4 * j4 + e]) * d : 0.f;
+                gr[4 * j4 + e] = (jj < lim) ? (sc * gr[4 * j4 + e]) * (d * fv[e]) : 0.f;
               }
             }
           }
@@ -832,17 +822,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_proxy_async_smem();
       wg_sync<BAR_PREP>();
 
-      // ---- U~^T = V^T T2^T (into U buffer s) and W^T = K^T T1^T (M = 128, N = 64, K = 64 tokens),
-      // then G of chunk c+1, queued behind them.  Warp 0 issues both and alone
-      // takes the waits they need (V; the buffer of W^T(c-1), free once the state
-      // warpgroup has read it; the K/Q tiles), then waits for the products and
-      // arrives W_READY.  The other warps go straight on to chunk c+1 and wait
-      // there for G(c+1), whose completion implies these products' (same issuing
-      // lane, in order), so the T1/T2 and P tiles they overwrite are free.  No
+      // ---- U~^T = V^T T2^T (into U buffer s) and W^T = K^T T1^T (M = 128, N = 64, K = 64 tokens).
+      // Warp 0 issues them and alone takes the waits they need (V; then the
+      // buffer of W^T(c-1), free once the state team has read it), waits for the
+      // products and arrives W_READY.  The other warps go straight on to chunk
+      // c+1 and wait there for G(c+1); its products are issued behind these
+      // (one tensor pipe, in order) and complete after them, so the T1/T2 and P
+      // tiles they overwrite are free.  No
       // warp leaves the loop alone: after a failed wait warp 0 only skips work,
-      // and the next warpgroup barrier sees the abort flag.  Waiting for
+      // and the next team barrier sees the abort flag.  Waiting for
       // W_CONSUMED(c-1) in every chunk also keeps W_READY from running two
-      // phases ahead of the state warpgroup.
+      // phases ahead of the state team.
       if (warp == 0) {
         // (every wait's outcome is made warp-uniform before the elected lane acts on it)
         bool okw = ident || __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_V_FULL], c & 1, s_abort, p.status));
@@ -864,8 +854,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (okw && c >= 1)
           okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_W_CONSUMED], (c - 1) & 1, s_abort, p.status));
-        // G(1) only: later chunks' G products are issued by the state team (two chunks ahead)
-        if (!l2n && okw && c == 0 && n_chunks > 1) okw = issue_g(1);
         if (okw) okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_PREP_MMA], pphase, s_abort, p.status));
         pphase ^= 1;
         if (okw && lane == 0) {
@@ -878,11 +866,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         __syncwarp();
       }
-      if (l2n && c == 0 && n_chunks > 1) {
-        // normalise K, Q of chunk 1 (all threads), then warp 0 issues its G
-        if (!kq_normalise(1)) break;
-        if (warp == 0 && !__any_sync(0xffffffffu, *s_abort != 0)) issue_g(1);
-      }
     }
   } else {
     // ================================================================ state team
@@ -890,6 +873,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int j = jt & 127;                                   // dv row owned (tensor-memory lane)
     const int hf = jt >> 7;                                   // column half of the row
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const bool l2n = (p.flags & GDN_QK_L2NORM) != 0;
     // initial state: s0 (rows dk, row stride ld0), the identity (transition
     // slice) or zero; final state to st (row stride ldT) or nowhere
     const size_t state_base = ((size_t)seq * H + h) * DK * (size_t)dv + col0 + j;
@@ -925,8 +909,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     float* s_carry = reinterpret_cast<float*>(sm + OFF_MISC + 8);
     // gate vectors of chunks 0 and 1 (later ones are built two chunks ahead,
-    // at the end of each chunk); a_in, b_in hold the inputs of the next chunk
-    // to build
+    // while the products of each chunk run); a_in, b_in hold the inputs of the
+    // next chunk to build
     float a_in, b_in;
     auto gates_of = [&](int c) {
       compute_gates<BAR_STATE>(gates_at(sm, c % 3), s_carry, min(C, seq_end - (seq_start + c * C)), jt,
@@ -935,12 +919,43 @@ __global__ void __launch_bounds__(THREADS, 1)
         load_gate_inputs(p, seq_start + (c + 1) * C, min(C, seq_end - (seq_start + (c + 1) * C)), h, jt,
                          a_in, b_in);
       wg_sync<BAR_STATE>();
-      if (jt == 0) mbar_arrive(&bars[B_GATES + c % 3]);
+    };
+    // Hands chunk c2 to the prep team once its K, Q tiles have landed: with the
+    // norm flag the inverse row norms are folded into its gate vectors (the
+    // tiles stay as loaded), the gates are released, and warp 8 issues
+    // G = [K; Q] K^T (M = 128, N = 64, K = dk) into tensor-memory buffer
+    // c2 % 2, whose last content, W^T of chunk c2-2, this team has read.
+    // Returns false (uniformly) if the wait gave up.
+    auto release_chunk = [&](int c2) -> bool {
+      const int s2 = c2 & 1;
+      if (!wg_wait<BAR_STATE>(&bars[B_KQ_FULL + s2], (c2 >> 1) & 1, s_abort, p.status)) return false;
+      if (l2n) {
+        fold_qk_norms(sm + OFF_KQ + s2 * KQ_BYTES, gates_at(sm, c2 % 3), jt);
+        wg_sync<BAR_STATE>();
+      }
+      if (jt == 0) mbar_arrive(&bars[B_GATES + c2 % 3]);
+      if (warp == 8) {
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t kq2 = sbase + OFF_KQ + s2 * KQ_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16(tmem + col_gw(c2), kdesc(kq2 + off), kdesc(kq2 + off), idesc_bf16(128, 64, 0, 0),
+                     kk > 0);
+          }
+          mma_commit(&bars[B_G_MMA + s2]);
+        }
+        __syncwarp();
+      }
+      return true;
     };
     if (ok && n_chunks > 0) {
       load_gate_inputs(p, seq_start, min(C, len), h, jt, a_in, b_in);
       gates_of(0);
       if (n_chunks > 1) gates_of(1);
+#pragma unroll 1
+      for (int c2 = 0; c2 < min(2, n_chunks) && ok; ++c2) ok = release_chunk(c2);
     }
 
     // initial state: tensor memory holds gamma_C(0) * S0, the bf16 operand holds S0
@@ -1065,7 +1080,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
       }
       // ---- gate vectors of chunk c+2 while the products run (their buffer's
-      // previous user, chunk c-1, is finished)
+      // previous user, chunk c-1, is finished; they are released with its G)
       if (c + 2 < n_chunks) gates_of(c + 2);
       if (!wg_wait<BAR_STATE>(&bars[B_STATE_MMA], sphase, s_abort, p.status)) break;
       sphase ^= 1;
@@ -1093,7 +1108,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(tmem + lane_off + COL_OB + 32 * hf, ob);
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 g4 = *reinterpret_cast<const float4*>(G.gamma + 32 * hf + 4 * e4);
+            const float4 g4 = *reinterpret_cast<const float4*>((l2n ? G.gq : G.gamma) + 32 * hf + 4 * e4);
             const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -1123,31 +1138,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       wg_sync<BAR_STATE>();
       if (jt == 0) mbar_arrive(&bars[B_CHUNK_DONE + s]);
 
-      // ---- G = [K; Q] K^T of chunk c+2 into tensor-memory buffer c % 2 (it held
-      // W^T of chunk c, read at the start of this chunk), after its K, Q tiles
-      // have landed in stage s (loaded above) and, with the flag, been normalised
-      if (c + 2 < n_chunks) {
-        const int c2 = c + 2;
-        if (!wg_wait<BAR_STATE>(&bars[B_KQ_FULL + s], (c2 >> 1) & 1, s_abort, p.status)) break;
-        if (p.flags & GDN_QK_L2NORM) {
-          if (jt < WG) l2norm_row(sm + OFF_KQ + s * KQ_BYTES, jt & 63, jt < 64 ? 0u : 8192u);
-          fence_proxy_async_smem();
-          wg_sync<BAR_STATE>();
-        }
-        if (warp == 8) {
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16(tmem + col_gw(c2), kdesc(kq_a + off), kdesc(kq_a + off), idesc_bf16(128, 64, 0, 0),
-                       kk > 0);
-            }
-            mma_commit(&bars[B_G_MMA + s]);
-          }
-          __syncwarp();
-        }
-      }
+      // ---- chunk c+2 to the prep team (its K, Q tiles were loaded above)
+      if (c + 2 < n_chunks && !release_chunk(c + 2)) break;
     }
   }
 

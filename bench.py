@@ -336,10 +336,11 @@ def run_ours(args, rank, world, local):
                      "peak_source": peak_kind, "traffic": profiled_traffic(),
                      "algorithmic_bytes_per_launch": gdn_bytes,
                      "avg_launch_ms": gdn_avg_s * 1e3,
-                     "schedule": (f"segmented: {sched['n_segs']} segments of {sched['seg_tok']} "
-                                  "tokens; segment 0 in full beside the later segments' state "
-                                  f"pass, combine, output pass ({mixer_launches} launches per "
-                                  "mixer call, timed together)" if sched["n_segs"] > 1
+                     "schedule": (f"segmented: segment 0 of {sched['seg0_tok']} tokens in full "
+                                  f"beside the state pass of {sched['n_segs'] - 1} segments of "
+                                  f"{sched['seg_tok']} tokens, combine, output pass "
+                                  f"({mixer_launches} launches per mixer call, timed together)"
+                                  if sched["n_segs"] > 1
                                   else "one pass per chain (1 launch per mixer call)")},
         "gpu_launches": launches,
         "e2e": e2e,

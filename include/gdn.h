@@ -117,14 +117,15 @@ size_t gdn_chunk_fwd_workspace(const gdn_fwd_params *p);
 /* The schedule gdn_chunk_fwd takes for these parameters when it is given a
  * workspace of gdn_chunk_fwd_workspace(p) bytes (host only, no device memory
  * touched).  Any output pointer may be NULL.
- *   n_segs:   1 = one pass per chain; >= 2 = segments of seg_tok tokens.
- *   seg_tok:  0 for one pass.
+ *   n_segs:   1 = one pass per chain; >= 2 = segment 0 of seg0_tok tokens,
+ *             then segments of seg_tok tokens (the last one may be shorter).
+ *   seg0_tok, seg_tok: 0 for one pass.
  *   launches: stream operations the call enqueues: 0 (nothing to do), 1 (one
  *             pass, or the copy or clear of S_T when every sequence is empty),
  *             2 (two segments: no combine step) or 3.
  * Parameters gdn_chunk_fwd would reject return the same error status. */
-gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg_tok,
-                                  int *launches);
+gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg0_tok,
+                                  int *seg_tok, int *launches);
 
 /* Chunkwise prefill (chunks of 64 tokens).
  *

@@ -68,7 +68,7 @@ def library() -> ctypes.CDLL:
         lib.gdn_chunk_fwd_workspace.argtypes = [ctypes.POINTER(gdn_fwd_params)]
         lib.gdn_chunk_fwd_workspace.restype = ctypes.c_size_t
         lib.gdn_chunk_fwd_schedule.argtypes = [ctypes.POINTER(gdn_fwd_params)] + [
-            ctypes.POINTER(ctypes.c_int)] * 3
+            ctypes.POINTER(ctypes.c_int)] * 4
         lib.gdn_chunk_fwd_schedule.restype = i32
         lib.gdn_chunk_fwd.argtypes = [ctypes.POINTER(gdn_fwd_params), vp, ctypes.c_size_t, vp]
         lib.gdn_chunk_fwd.restype = i32
@@ -192,14 +192,15 @@ def prefill_schedule(n_seq: int, seq_len: int, H: int, dk: int, dv: int,
                      dtype: torch.dtype = torch.bfloat16, flags: int = 0,
                      varlen: bool = False) -> dict:
     """gdn_chunk_fwd_schedule for a call of this shape, given its workspace:
-    {"n_segs", "seg_tok", "launches"} (n_segs = 1: one pass per chain)."""
+    {"n_segs", "seg0_tok", "seg_tok", "launches"} (n_segs = 1: one pass per chain)."""
     p = _shape_params(n_seq, seq_len, H, dk, dv, dtype, flags, varlen)
-    n, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    st = library().gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok),
-                                          ctypes.byref(launches))
+    n, tok0, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    st = library().gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
+                                          ctypes.byref(tok), ctypes.byref(launches))
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd_schedule")
-    return {"n_segs": n.value, "seg_tok": tok.value, "launches": launches.value}
+    return {"n_segs": n.value, "seg0_tok": tok0.value, "seg_tok": tok.value,
+            "launches": launches.value}
 
 
 def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,

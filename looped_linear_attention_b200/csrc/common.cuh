@@ -23,7 +23,8 @@ namespace gdn {
 // tokens (state passing between segments).
 struct SegPlan {
   int n_segs;
-  int seg_tok;
+  int seg_tok;     // tokens of segments 1 .. n_segs-1 (the last one may be shorter)
+  int seg0_tok;    // tokens of segment 0
 };
 
 // Upper bound for any device-side wait: about 2 s of SM clock.  A wait that
@@ -94,6 +95,16 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
+// Programmatic dependent launch.  A grid launched with programmatic stream
+// serialization may start before the previous grid in its stream has
+// finished: griddep_wait() blocks until that grid has completed and its memory
+// writes are visible; griddep_launch_dependents() lets the next such grid
+// start once every CTA of this grid has signalled it (or exited).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

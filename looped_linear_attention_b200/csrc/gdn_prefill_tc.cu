@@ -138,8 +138,9 @@ struct Params {
   int n_seq, seq_len, total_tokens, H, dv, n_slices;
   float scale;
   unsigned flags;
-  // Segment schedule (fixed-length sequences cut into n_segs >= 2 segments of
-  // seg_tok tokens; mode 0 runs whole sequences in one pass):
+  // Segment schedule (fixed-length sequences cut into n_segs >= 2 segments:
+  // segment 0 of seg0_tok tokens, the others of seg_tok, the last one possibly
+  // shorter; mode 0 runs whole sequences in one pass):
   //   mode 1: segment 0 runs in full from S0 (outputs, and its end state S_1
   //           to Sst slot 0); the CTAs after those run segments 1 .. n_segs-2
   //           from a zero state without outputs.  Their slices 0 .. n_slices-1
@@ -148,7 +149,7 @@ struct Params {
   //           segment's dk x dk transition M_p to Mws slot p-1.
   //   mode 2: segments 1 .. n_segs-1 from their start states S_p in Sst slot
   //           p-1, with outputs; the last segment writes S_T.
-  int mode, n_segs, seg_tok;
+  int mode, n_segs, seg_tok, seg0_tok;
   float* Bws;          // [n_seq][n_segs-2][H][dk][dv]
   float* Mws;          // [n_seq][n_segs-2][H][dk][dk]
   float* Sst;          // [n_seq][n_segs-1][H][dk][dv]
@@ -621,6 +622,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int tid = threadIdx.x;
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);   // warp-uniform by construction
+  // segmented schedule: the combine kernel may be launched now (it waits for
+  // this grid before it reads anything)
+  if (p.mode == 1) griddep_launch_dependents();
 
   // work unit: (sequence or segment, head, dv slice)
   int slice, h, seq, part;
@@ -659,8 +663,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     seq_start = seq * p.seq_len;
     seq_end = seq_start + p.seq_len;
     if (p.mode != 0) {
-      seq_start += part * p.seg_tok;
-      seq_end = min(seq_end, seq_start + p.seg_tok);
+      seq_start += (part == 0) ? 0 : p.seg0_tok + (part - 1) * p.seg_tok;
+      seq_end = min(seq_end, seq_start + (part == 0 ? p.seg0_tok : p.seg_tok));
     }
   }
   {
@@ -959,7 +963,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     // initial state: tensor memory holds gamma_C(0) * S0, the bf16 operand holds S0
-    // (this thread: dk columns 64 hf .. 64 hf + 63 of row j)
+    // (this thread: dk columns 64 hf .. 64 hf + 63 of row j).  The output pass
+    // may have started before the kernels that write its start states have
+    // finished: everything above ran meanwhile, the start state waits for them.
+    if (p.mode == 2) griddep_wait();
     const float decay0 = (n_chunks > 0) ? gates_at(sm, 0).gamma[C - 1] : 1.f;
     {
 #pragma unroll 1
@@ -1226,6 +1233,10 @@ __global__ void __launch_bounds__(256)
     gdn_segment_combine_kernel(const float* __restrict__ Bws, const float* __restrict__ Mws,
                                float* __restrict__ Sst, int H, int dv, int n_segs) {
   extern __shared__ __align__(16) float cmb_smem[];
+  // launched as a programmatic dependent of the state pass: let the output
+  // pass launch, then wait for the state pass before reading its results
+  griddep_launch_dependents();
+  griddep_wait();
   float* sM0 = cmb_smem;
   float* sM1 = cmb_smem + DK * CMB_MLD;
   float* sS = cmb_smem + 2 * DK * CMB_MLD;         // [128][CMB_SLD], 16 columns used
@@ -1327,36 +1338,42 @@ __global__ void __launch_bounds__(256)
 }  // namespace tc
 
 // Chooses the schedule of a tensor-core prefill: n_segs = 1 is one pass per
-// chain; otherwise fixed-length sequences are cut into n_segs segments of
-// seg_tok tokens.  The cost model counts chunk steps on the critical path:
-// waves of CTAs (one CTA per SM) times chunks per CTA, for the one-pass launch
-// against the two segmented launches plus the combine.  The first segmented
-// launch holds segment 0 of every chain (run in full) and segments
-// 1 .. n_segs-2 with one transition slice each; the second holds segments
-// 1 .. n_segs-1.
+// chain; otherwise fixed-length sequences are cut into a segment 0 of seg0_tok
+// tokens and n_segs-1 segments of seg_tok.  The cost model counts chunk steps
+// on the critical path: waves of CTAs (one CTA per SM) times chunks per CTA,
+// for the one-pass launch against the two segmented launches plus the
+// combine.  The first segmented launch holds segment 0 of every chain (run in
+// full, with outputs) and segments 1 .. n_segs-2 with one transition slice
+// each (no outputs); the second holds segments 1 .. n_segs-1.  A chunk with
+// outputs costs kOutputChunk chunk steps (it adds the output products and
+// their epilogue), so segment 0 is made shorter than the others.
 SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
-  SegPlan plan{1, 0};
+  SegPlan plan{1, 0, 0};
   if (!prefill_tc_supported(p) || p->cu_seqlens || (p->flags & GDN_SINGLE_PASS) || p->n_seq <= 0 ||
       p->seq_len <= tc::C || sms <= 0)
     return plan;
+  constexpr double kOutputChunk = 1.15;   // chunk step of a CTA with outputs / without
   const long long chains = (long long)p->n_seq * p->H;
   const long long slices = p->dv / tc::DVS;
   const int n_chunks = (p->seq_len + tc::C - 1) / tc::C;
   auto waves = [&](long long ctas) { return (double)((ctas + sms - 1) / sms); };
-  const double one_pass = waves(chains * slices) * (n_chunks + 1.5);
+  const double one_pass = waves(chains * slices) * (n_chunks * kOutputChunk + 1.5);
   double best = 0.0;
-  SegPlan cand{1, 0};
+  SegPlan cand{1, 0, 0};
   for (int seg = 1; seg < n_chunks; ++seg) {
-    const int P = (n_chunks + seg - 1) / seg;
-    if (P < 2) break;
-    // a launch wave costs its chunks plus about 1.5 chunk steps of pipeline
-    // fill and drain; a combine step about 0.8 of a chunk step
-    const double cost = waves(chains * (slices + (long long)(P - 2) * (slices + 1))) * (seg + 1.5) +
-                        waves(chains * (P - 1) * slices) * (seg + 1.5) +
-                        (P > 2 ? 0.8 * (P - 2) + 0.5 : 0.0);
-    if (cand.n_segs == 1 || cost < best) {
-      best = cost;
-      cand = SegPlan{P, seg * tc::C};
+    for (int seg0 = seg; seg0 >= 1 && seg0 >= seg - 4; --seg0) {
+      if (seg0 >= n_chunks) continue;
+      const int P = 1 + (n_chunks - seg0 + seg - 1) / seg;
+      // a launch wave costs its longest CTA's chunks plus about 1.5 chunk steps
+      // of pipeline fill and drain; a combine step about 0.8 of a chunk step
+      const double cost =
+          waves(chains * (slices + (long long)(P - 2) * (slices + 1))) *
+              (fmax(seg0 * kOutputChunk, (double)seg) + 1.5) +
+          waves(chains * (P - 1) * slices) * (seg * kOutputChunk + 1.5) + (P > 2 ? 0.8 * (P - 2) + 0.5 : 0.0);
+      if (cand.n_segs == 1 || cost < best) {
+        best = cost;
+        cand = SegPlan{P, seg * tc::C, seg0 * tc::C};
+      }
     }
   }
   // segmented only when clearly cheaper than one pass
@@ -1374,12 +1391,32 @@ size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan) {
          align256(n * (plan.n_segs - 1) * sd);
 }
 
+// Launch configuration; `dependent` launches with programmatic stream
+// serialization (the grid may start while the previous one in the stream is
+// finishing and orders its reads of that grid's results by griddep_wait()).
+struct LaunchCfg {
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  LaunchCfg(unsigned blocks, unsigned threads, size_t smem, cudaStream_t stream, bool dependent) {
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+  }
+};
+
 static gdn_status tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const tc::Params& kp, long long blocks, cudaStream_t stream) {
+                            const tc::Params& kp, long long blocks, cudaStream_t stream,
+                            bool dependent = false) {
   if (blocks <= 0) return GDN_OK;
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
-  tc::gdn_prefill_tc_kernel<<<(unsigned)blocks, tc::THREADS, tc::SMEM_BYTES, stream>>>(mq, mk, mv, kp);
-  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  LaunchCfg lc((unsigned)blocks, tc::THREADS, tc::SMEM_BYTES, stream, dependent);
+  const cudaError_t e = cudaLaunchKernelEx(&lc.cfg, tc::gdn_prefill_tc_kernel, mq, mk, mv, kp);
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const SegPlan& plan, void* ws,
@@ -1415,6 +1452,7 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   kp.mode = 0;
   kp.n_segs = 1;
   kp.seg_tok = 0;
+  kp.seg0_tok = 0;
   kp.Bws = kp.Mws = nullptr;
   kp.Sst = nullptr;
   const long long chains = (long long)p->n_seq * p->H;
@@ -1432,6 +1470,7 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   kp.Sst = reinterpret_cast<float*>(w);
   kp.n_segs = P;
   kp.seg_tok = plan.seg_tok;
+  kp.seg0_tok = plan.seg0_tok;
   kp.mode = 1;
   gdn_status st =
       tc_launch(mq, mk, mv, kp, chains * (kp.n_slices + (long long)(P - 2) * (kp.n_slices + 1)), stream);
@@ -1446,12 +1485,13 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
         return GDN_ERR_CUDA;
       cmb_attr_set = true;
     }
-    tc::gdn_segment_combine_kernel<<<(unsigned)cblocks, 256, tc::CMB_SMEM, stream>>>(kp.Bws, kp.Mws, kp.Sst,
-                                                                                   p->H, p->dv, P);
-    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    LaunchCfg lc((unsigned)cblocks, 256, tc::CMB_SMEM, stream, /*dependent=*/true);
+    if (cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_combine_kernel, (const float*)kp.Bws,
+                           (const float*)kp.Mws, kp.Sst, p->H, p->dv, P) != cudaSuccess)
+      return GDN_ERR_CUDA;
   }
   kp.mode = 2;
-  return tc_launch(mq, mk, mv, kp, chains * (P - 1) * kp.n_slices, stream);
+  return tc_launch(mq, mk, mv, kp, chains * (P - 1) * kp.n_slices, stream, /*dependent=*/true);
 }
 
 }  // namespace gdn

@@ -6,8 +6,9 @@ stack is applied T times, and the loop state is
 h^(tau) = h~^(tau) + rho_tau (.) h^(tau-1).  In this workload the block output
 h~^(tau) is the GDN output itself, reshaped [L, H*dv] = [L, d] (d = H*dv), from
 a zero initial state each loop; q and k are L2-normalised per head inside the
-mixer kernel.  The projections are plain torch GEMMs (outside the mixer's hot
-path); the mixer and the residual run in this library's kernels.
+mixer kernel.  The three projections are one batched torch GEMM over the
+stacked weights [W_q; W_k; W_v] (outside the mixer's hot path); the mixer and
+the residual run in this library's kernels.
 """
 from __future__ import annotations
 
@@ -28,23 +29,30 @@ class LoopedPrefill:
         self.time_mixer = time_mixer
         self.mixer_events = []
         self.L, self.H, self.dk, self.dv, self.loops = L, H, dk, dv, loops
-        self.q = torch.empty(L, H, dk, dtype=dtype, device=device)
-        self.k = torch.empty(L, H, dk, dtype=dtype, device=device)
-        self.v = torch.empty(L, H, dv, dtype=dtype, device=device)
+        assert d_in == H * dv, "the loop state feeds the next projection: H*dk must equal H*dv"
+        # q, k, v as the three planes of one [3, L, d] buffer (one batched GEMM)
+        self.qkv = torch.empty(3, L, d_in, dtype=dtype, device=device)
+        self.q = self.qkv[0].view(L, H, dk)
+        self.k = self.qkv[1].view(L, H, dk)
+        self.v = self.qkv[2].view(L, H, dv)
         self.o = torch.empty(L, H, dv, dtype=dtype, device=device)
         self.h = [torch.empty(L, H * dv, dtype=dtype, device=device) for _ in range(2)]
-        assert d_in == H * dv, "the loop state feeds the next projection: H*dk must equal H*dv"
 
     def run(self, h0: torch.Tensor, Wq: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor,
             a: torch.Tensor, b: torch.Tensor, rho: torch.Tensor, scale: float = 1.0,
             out: Optional[torch.Tensor] = None) -> torch.Tensor:
-        """h0 [L, d]; W* [d, d]; a, b [T, L, H] fp32; rho [T, d] fp32. Returns h^(T)."""
-        L, H, dk, dv = self.L, self.H, self.dk, self.dv
+        """h0 [L, d]; W* [d, d]; a, b [T, L, H] fp32; rho [T, d] fp32. Returns h^(T).
+
+        Wq, Wk, Wv given as the three planes of one [3, d, d] tensor (see
+        `stack_weights`) are used in place; otherwise they are stacked into a
+        new tensor on every call."""
+        L, H, dv = self.L, self.H, self.dv
+        W3 = stacked_view(Wq, Wk, Wv)
+        if W3 is None:
+            W3 = torch.stack((Wq, Wk, Wv))
         h_prev = h0
         for tau in range(self.loops):
-            torch.matmul(h_prev, Wq, out=self.q.view(L, H * dk))
-            torch.matmul(h_prev, Wk, out=self.k.view(L, H * dk))
-            torch.matmul(h_prev, Wv, out=self.v.view(L, H * dv))
+            torch.matmul(h_prev.unsqueeze(0), W3, out=self.qkv)
             if self.time_mixer:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
@@ -59,6 +67,29 @@ class LoopedPrefill:
             B.loop_residual(self.o.view(L, H * dv), h_prev, rho[tau], out=h_next)
             h_prev = h_next
         return h_prev
+
+
+def stack_weights(Wq: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor):
+    """One [3, d, d] tensor holding W_q, W_k, W_v, and its three planes (pass
+    those to `LoopedPrefill.run` to avoid a copy per call)."""
+    W3 = torch.stack((Wq, Wk, Wv)).contiguous()
+    return W3, W3[0], W3[1], W3[2]
+
+
+def stacked_view(Wq: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor) -> Optional[torch.Tensor]:
+    """[3, d, d] view of W_q, W_k, W_v when they are consecutive planes of one
+    contiguous allocation, else None."""
+    ws = (Wq, Wk, Wv)
+    if Wq.dim() != 2 or any(w.shape != Wq.shape or w.dtype != Wq.dtype or w.device != Wq.device
+                            or not w.is_contiguous() for w in ws):
+        return None
+    n = Wq.numel()
+    base = Wq.untyped_storage().data_ptr()
+    if any(w.untyped_storage().data_ptr() != base for w in ws):
+        return None
+    if Wk.storage_offset() != Wq.storage_offset() + n or Wv.storage_offset() != Wq.storage_offset() + 2 * n:
+        return None
+    return Wq.as_strided((3,) + tuple(Wq.shape), (n,) + tuple(Wq.stride()))
 
 
 class HostPipeline:

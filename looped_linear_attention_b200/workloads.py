@@ -180,17 +180,17 @@ def decode_inputs(wl: Workload, device="cpu", n_slots=None, step: int = 0):
 
 def looped_inputs(wl: Workload, device="cpu", seq_len=None, d_model=None):
     """Looped-prefill workload: h0 [L, d] bf16, W_q/W_k/W_v [d, d] bf16 with
-    N(0, variance 1/d) entries, and per loop tau: a, b [T, L, H] fp32 and
-    rho [T, d] ~ U(0, 0.5) fp32."""
+    N(0, variance 1/d) entries (the three planes of one [3, d, d] tensor), and
+    per loop tau: a, b [T, L, H] fp32 and rho [T, d] ~ U(0, 0.5) fp32."""
     L = wl.seq_len if seq_len is None else seq_len
     d = (wl.H * wl.dk) if d_model is None else d_model
     g = _gen(device, wl.name, "h0")
     h0 = torch.randn(L, d, generator=g, device=device, dtype=torch.float32).to(wl.dtype)
-    Ws = []
-    for name in ("Wq", "Wk", "Wv"):
+    Ws = torch.empty(3, d, d, device=device, dtype=wl.dtype)   # W_q, W_k, W_v as planes
+    for i, name in enumerate(("Wq", "Wk", "Wv")):
         gw = _gen(device, wl.name, name)
-        Ws.append((torch.randn(d, d, generator=gw, device=device, dtype=torch.float32)
-                   / float(np.sqrt(d))).to(wl.dtype))
+        Ws[i] = (torch.randn(d, d, generator=gw, device=device, dtype=torch.float32)
+                 / float(np.sqrt(d))).to(wl.dtype)
     a = torch.empty(wl.loops, L, wl.H, device=device)
     b = torch.empty(wl.loops, L, wl.H, device=device)
     rho = torch.empty(wl.loops, d, device=device)

@@ -107,11 +107,13 @@ def test_workspace_segmented_schedule_for_few_long_chains(lib):
     assert need > 0 and need % sd == 0
     sets = need // sd
     assert (sets + 5) % 3 == 0 and 2 <= (sets + 5) // 3 <= 64
-    n, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok),
-                                      ctypes.byref(launches)) == B.GDN_OK
+    n, tok0, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
+                                      ctypes.byref(tok), ctypes.byref(launches)) == B.GDN_OK
     P = (sets + 5) // 3
-    assert n.value == P and (P - 1) * tok.value < 4096 <= P * tok.value and tok.value % 64 == 0
+    assert n.value == P and tok.value % 64 == 0 and tok0.value % 64 == 0
+    assert 0 < tok0.value <= tok.value
+    assert tok0.value + (P - 2) * tok.value < 4096 <= tok0.value + (P - 1) * tok.value
     assert launches.value == (3 if P > 2 else 2)
 
 
@@ -128,20 +130,21 @@ def test_workspace_zero_for_one_pass_schedules(lib, kw):
     kw.setdefault("total_tokens", kw["n_seq"] * kw["seq_len"])
     p = _params(**kw)
     assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
-    n, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok),
-                                      ctypes.byref(launches)) == B.GDN_OK
-    assert (n.value, tok.value, launches.value) == (1, 0, 1)
+    n, tok0, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
+                                      ctypes.byref(tok), ctypes.byref(launches)) == B.GDN_OK
+    assert (n.value, tok0.value, tok.value, launches.value) == (1, 0, 0, 1)
 
 
 def test_schedule_query_rejects_what_the_call_rejects(lib):
     p = _params(dk=96)                                    # dk outside {64, 128}
     bad = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
     assert bad == ctypes.c_size_t(-1).value
-    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), None, None, None) != B.GDN_OK
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), None, None, None, None) != B.GDN_OK
     empty = _params(n_seq=0, seq_len=64, total_tokens=0)
     launches = ctypes.c_int(-1)
-    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(empty), None, None, ctypes.byref(launches)) == B.GDN_OK
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(empty), None, None, None,
+                                      ctypes.byref(launches)) == B.GDN_OK
     assert launches.value == 0
 
 
@@ -209,3 +212,24 @@ def test_empty_work_is_a_no_op(lib):
                                B.GDN_BF16, 1.0, 0, None) == B.GDN_OK
     p = _params(n_seq=0, seq_len=0, total_tokens=0)
     assert lib.gdn_chunk_fwd(ctypes.byref(p), None, 0, None) == B.GDN_OK
+
+
+def test_stacked_projection_weights_are_used_in_place():
+    """The looped step runs q, k, v as one batched GEMM over [W_q; W_k; W_v]:
+    weights that are consecutive planes of one allocation (as the workload
+    generator and stack_weights give them) are viewed, not copied; any other
+    arrangement is recognised as such (and stacked by the runner)."""
+    import dataclasses
+    import torch
+    from looped_linear_attention_b200 import workloads as W
+    from looped_linear_attention_b200.looped import stack_weights, stacked_view
+    inp = W.looped_inputs(dataclasses.replace(W.WORKLOADS["looped_prefill"], seq_len=64), "cpu")
+    Wq, Wk, Wv = inp["Wq"], inp["Wk"], inp["Wv"]
+    v = stacked_view(Wq, Wk, Wv)
+    assert v is not None and v.data_ptr() == Wq.data_ptr()
+    assert all(torch.equal(v[i], w) for i, w in enumerate((Wq, Wk, Wv)))
+    assert stacked_view(Wq.clone(), Wk.clone(), Wv.clone()) is None
+    assert stacked_view(Wk, Wq, Wv) is None
+    assert stacked_view(Wq, Wk, Wv[:, :-1]) is None
+    W3, q, k, w = stack_weights(Wq.clone(), Wk.clone(), Wv.clone())
+    assert stacked_view(q, k, w).data_ptr() == W3.data_ptr()

@@ -425,6 +425,21 @@ def test_looped_prefill_end_to_end():
     assert rel_l2(host(o), o_ref) < TOL_BF16_O
 
 
+def test_looped_step_same_with_stacked_or_separate_weights():
+    """The batched q/k/v projection gives the same h^(T) whether the weights
+    come as planes of one [3, d, d] tensor (used in place) or as three separate
+    tensors (stacked by the runner)."""
+    wl = dataclasses.replace(W.WORKLOADS["looped_prefill"], seq_len=256)
+    inp = W.looped_inputs(wl, "cuda")
+    runner = lla.LoopedPrefill(inp["L"], wl.H, wl.dk, wl.dv, wl.loops, "cuda")
+    args = (inp["a"], inp["b"], inp["rho"])
+    h_view = runner.run(inp["h0"], inp["Wq"], inp["Wk"], inp["Wv"], *args).clone()
+    h_sep = runner.run(inp["h0"], inp["Wq"].clone(), inp["Wk"].clone(), inp["Wv"].clone(), *args)
+    torch.cuda.synchronize()
+    _status_ok()
+    assert torch.equal(h_view, h_sep)
+
+
 def test_host_pipeline_matches_device_steps():
     """HostPipeline (pinned host inputs and results, copies overlapped with the
     neighbouring steps' compute) gives the same h^(T) as LoopedPrefill.run on

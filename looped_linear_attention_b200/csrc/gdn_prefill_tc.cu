@@ -1206,17 +1206,21 @@ bool prefill_tc_supported(const gdn_fwd_params* p) {
 }
 
 // ------------------------------------------------------------------ segments
-// Combine step of the segmented schedule: for one (sequence, head) and 16
-// columns of dv, S_{p+1} = M_p S_p + B_p for p = 1 .. n_segs-2, starting from
-// S_1 (written by the segment-0 CTAs) and writing every S_p, p >= 2, to Sst
-// (slot p-1; M_p and B_p sit in slot p-1 of theirs).  The products run on the warp-level tensor
-// cores with the 3xTF32 split (fp32-level accuracy): warp w owns rows
-// 16w .. 16w+15 of the 128 x 16 block.  M_p (dk x dk) is staged in shared
-// memory by cp.async one step ahead (double buffer).
+// Combine step of the segmented schedule: for one (sequence, head) and
+// CMB_COLS columns of dv, S_{p+1} = M_p S_p + B_p for p = 1 .. n_segs-2,
+// starting from S_1 (written by the segment-0 CTAs) and writing every S_p,
+// p >= 2, to Sst (slot p-1; M_p and B_p sit in slot p-1 of theirs).  The
+// products run on the warp-level tensor cores with the 3xTF32 split
+// (fp32-level accuracy): warp w owns rows 16w .. 16w+15 of the 128 x CMB_COLS
+// block.  M_p (dk x dk) is staged in shared memory by cp.async one step ahead
+// (double buffer).
 namespace tc {
-constexpr int CMB_COLS = 16;
+constexpr int CMB_COLS = 16;                       // columns of dv per CTA
+constexpr int CMB_NT = CMB_COLS / 8;               // 8-column mma tiles per warp
 constexpr int CMB_MLD = 132;                       // padded row stride of a staged M (floats)
-constexpr int CMB_SLD = 24;                        // padded row stride of the S block (floats)
+constexpr int CMB_SLD = CMB_COLS + 8;              // padded row stride of the S block (floats)
+static_assert(CMB_COLS % 8 == 0 && CMB_SLD % 32 != 0 && (CMB_SLD % 32) % 8 == 0,
+              "S-block fragment reads are conflict-free with a row stride of 8 or 24 mod 32");
 constexpr uint32_t CMB_SMEM = (2 * DK * CMB_MLD + DK * CMB_SLD) * 4;
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
@@ -1239,7 +1243,7 @@ __global__ void __launch_bounds__(256)
   griddep_wait();
   float* sM0 = cmb_smem;
   float* sM1 = cmb_smem + DK * CMB_MLD;
-  float* sS = cmb_smem + 2 * DK * CMB_MLD;         // [128][CMB_SLD], 16 columns used
+  float* sS = cmb_smem + 2 * DK * CMB_MLD;         // [128][CMB_SLD], CMB_COLS columns used
   const int ncb = dv / CMB_COLS;
   const int cb = blockIdx.x % ncb;
   const int hh = (blockIdx.x / ncb) % H;
@@ -1265,9 +1269,9 @@ __global__ void __launch_bounds__(256)
   if (n_steps <= 0) return;
   stage(0, sM0);
   // x[nt][e]: rows r0+g (e = 0, 1) and r0+g+8 (e = 2, 3), columns nt*8 + 2q (+1)
-  float x[2][4];
+  float x[CMB_NT][4];
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
+  for (int nt = 0; nt < CMB_NT; ++nt)
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
       const float2 v = *reinterpret_cast<const float2*>(sptr(0) + (size_t)(r0 + g + 8 * hr) * dv + nt * 8 + 2 * q);
@@ -1277,7 +1281,7 @@ __global__ void __launch_bounds__(256)
   for (int pp = 0;; ++pp) {
     // S_{pp+1} (x) to the operand block, and to Sst unless it came from there
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < CMB_NT; ++nt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const float2 v = make_float2(x[nt][2 * hr], x[nt][2 * hr + 1]);
@@ -1290,18 +1294,18 @@ __global__ void __launch_bounds__(256)
     if (prefetch) stage(pp + 1, ((pp + 1) & 1) ? sM1 : sM0);
     // B is loaded now and added after the product, so its latency is hidden
     const float* B = Bws + (((size_t)seq * n_steps + pp) * H + hh) * sd + colb;
-    float2 bv[2][2];
+    float2 bv[CMB_NT][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < CMB_NT; ++nt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr)
         bv[nt][hr] = *reinterpret_cast<const float2*>(B + (size_t)(r0 + g + 8 * hr) * dv + nt * 8 + 2 * q);
     if (prefetch) cp_async_wait<1>(); else cp_async_wait<0>();
     __syncthreads();                                // M_pp and S_pp are in shared memory
     const float* M = (pp & 1) ? sM1 : sM0;
-    float acc[2][3][4];
+    float acc[CMB_NT][3][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < CMB_NT; ++nt)
 #pragma unroll
       for (int k = 0; k < 3; ++k)
 #pragma unroll
@@ -1314,7 +1318,7 @@ __global__ void __launch_bounds__(256)
       split_tf32(M[(r0 + g) * CMB_MLD + k0 + q + 4], ah[2], al[2]);
       split_tf32(M[(r0 + g + 8) * CMB_MLD + k0 + q + 4], ah[3], al[3]);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
+      for (int nt = 0; nt < CMB_NT; ++nt) {
         uint32_t bh[2], bl[2];
         split_tf32(sS[(k0 + q) * CMB_SLD + nt * 8 + g], bh[0], bl[0]);
         split_tf32(sS[(k0 + q + 4) * CMB_SLD + nt * 8 + g], bh[1], bl[1]);
@@ -1324,7 +1328,7 @@ __global__ void __launch_bounds__(256)
       }
     }
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nt = 0; nt < CMB_NT; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) x[nt][e] = acc[nt][0][e] + (acc[nt][1][e] + acc[nt][2][e]);
       x[nt][0] += bv[nt][0].x;

@@ -122,7 +122,8 @@ size_t gdn_chunk_fwd_workspace(const gdn_fwd_params *p);
  *   seg0_tok, seg_tok: 0 for one pass.
  *   launches: stream operations the call enqueues: 0 (nothing to do), 1 (one
  *             pass, or the copy or clear of S_T when every sequence is empty),
- *             2 (two segments: no combine step) or 3.
+ *             2 (two segments: no combine step; or a varlen call with its
+ *             length sort) or 3.
  * Parameters gdn_chunk_fwd would reject return the same error status. */
 gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg0_tok,
                                   int *seg_tok, int *launches);
@@ -139,6 +140,11 @@ gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg
  * with two segments), and a third launch runs segments 1 .. P-1 from their
  * start states and writes their outputs (all on `stream`).  The outputs equal
  * the one-pass outputs up to rounding.  GDN_SINGLE_PASS disables it.
+ * Varlen calls (cu_seqlens != NULL) always run one pass; when they take more
+ * blocks than the GPU runs at once and have at most 4096 sequences, a first
+ * launch sorts the sequences by length on the device (longest first, into the
+ * workspace) and the blocks take them in that order, so that the longest
+ * chains do not start last.  The outputs do not depend on the order.
  *
  * ws/ws_bytes: device workspace of at least gdn_chunk_fwd_workspace(p) bytes,
  * 256-byte aligned, owned by the caller and not read back afterwards.

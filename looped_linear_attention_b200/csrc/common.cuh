@@ -25,6 +25,7 @@ struct SegPlan {
   int n_segs;
   int seg_tok;     // tokens of segments 1 .. n_segs-1 (the last one may be shorter)
   int seg0_tok;    // tokens of segment 0
+  int lpt;         // varlen, one pass: sequences launched longest first (order in the workspace)
 };
 
 // Upper bound for any device-side wait: about 2 s of SM clock.  A wait that

@@ -139,13 +139,13 @@ gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params* p, int* n_segs, int* seg
                                   int* launches) {
   const gdn_status v = validate_fwd(p);
   if (v != GDN_OK) return v;
-  gdn::SegPlan plan{1, 0, 0};
+  gdn::SegPlan plan{1, 0, 0, 0};
   if (p->total_tokens > 0 && gdn::prefill_tc_supported(p)) plan = gdn::plan_prefill_segments(p, sm_count());
   int n = 1;                                           // one pass
   if (p->n_seq == 0) n = 0;
   else if (p->total_tokens == 0) n = (p->S_T && p->S0 != p->S_T) ? 1 : 0;   // a copy or a clear of S_T
   else if (plan.n_segs > 2) n = 3;
-  else if (plan.n_segs == 2) n = 2;
+  else if (plan.n_segs == 2 || plan.lpt) n = 2;
   if (n_segs) *n_segs = plan.n_segs;
   if (seg0_tok) *seg0_tok = plan.seg0_tok;
   if (seg_tok) *seg_tok = plan.seg_tok;
@@ -170,10 +170,10 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_params* p, void* ws, size_t ws_bytes,
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
   }
   const bool tc = gdn::prefill_tc_supported(p);
-  gdn::SegPlan plan = tc ? gdn::plan_prefill_segments(p, sm_count()) : gdn::SegPlan{1, 0, 0};
-  if (plan.n_segs > 1) {
+  gdn::SegPlan plan = tc ? gdn::plan_prefill_segments(p, sm_count()) : gdn::SegPlan{1, 0, 0, 0};
+  if (plan.n_segs > 1 || plan.lpt) {
     const size_t need = gdn::prefill_segment_workspace(p, plan);
-    if (!ws && ws_bytes == 0) plan = gdn::SegPlan{1, 0, 0};   // no workspace: one pass
+    if (!ws && ws_bytes == 0) plan = gdn::SegPlan{1, 0, 0, 0};   // no workspace: one pass, natural order
     else if (!ws || ws_bytes < need) return GDN_ERR_WORKSPACE;
   }
   unsigned* st = status_ptr();

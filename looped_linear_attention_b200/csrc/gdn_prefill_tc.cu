@@ -150,6 +150,7 @@ struct Params {
   //   mode 2: segments 1 .. n_segs-1 from their start states S_p in Sst slot
   //           p-1, with outputs; the last segment writes S_T.
   int mode, n_segs, seg_tok, seg0_tok;
+  const int32_t* order;  // mode 0, varlen: sequences longest first (block order), or null
   float* Bws;          // [n_seq][n_segs-2][H][dk][dv]
   float* Mws;          // [n_seq][n_segs-2][H][dk][dk]
   float* Sst;          // [n_seq][n_segs-1][H][dk][dv]
@@ -652,6 +653,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int unit = chain / p.H;
     seq = unit / units_per_seq;
     part = first_part + unit % units_per_seq;
+    if (p.order) seq = __ldg(p.order + seq);   // longest sequences in the first blocks
   }
   const bool ident = partial && slice == p.n_slices;   // transition slice: V = 0, S0 = I
   const bool outputs = !partial;
@@ -1339,6 +1341,46 @@ __global__ void __launch_bounds__(256)
     __syncthreads();                                // every read of S_pp and M_pp is done
   }
 }
+// Longest-processing-time order of varlen sequences: order[r] is the sequence
+// with the r-th largest length (ties by index), so that block r of a one-pass
+// launch (blocks are dispatched roughly in index order) takes the longest
+// remaining chain.  One CTA sorts (length, index) keys with a bitonic network
+// in shared memory; lengths come from cu_seqlens, clamped to [0, 2^31).
+constexpr int kLptMaxSeqs = 4096;
+constexpr int kLptThreads = 1024;
+__global__ void __launch_bounds__(kLptThreads)
+    gdn_lpt_order_kernel(const int32_t* __restrict__ cu, int n_seq, int32_t* __restrict__ order) {
+  __shared__ unsigned long long key[kLptMaxSeqs];
+  int n2 = 1;
+  while (n2 < n_seq) n2 <<= 1;
+  for (int i = threadIdx.x; i < n2; i += kLptThreads) {
+    unsigned long long k = ~0ull;                  // padding sorts last
+    if (i < n_seq) {
+      long long len = (long long)__ldg(cu + i + 1) - (long long)__ldg(cu + i);
+      len = len < 0 ? 0 : (len > 0x7fffffffLL ? 0x7fffffffLL : len);
+      k = ((unsigned long long)(0x7fffffffu - (unsigned)len) << 32) | (unsigned)i;
+    }
+    key[i] = k;
+  }
+  __syncthreads();
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += kLptThreads) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const unsigned long long a = key[i], b = key[j];
+          const bool ascending = (i & size) == 0;
+          if ((a > b) == ascending) {
+            key[i] = b;
+            key[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n_seq; i += kLptThreads) order[i] = (int32_t)(key[i] & 0xffffffffu);
+}
 }  // namespace tc
 
 // Chooses the schedule of a tensor-core prefill: n_segs = 1 is one pass per
@@ -1352,10 +1394,17 @@ __global__ void __launch_bounds__(256)
 // outputs costs kOutputChunk chunk steps (it adds the output products and
 // their epilogue), so segment 0 is made shorter than the others.
 SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
-  SegPlan plan{1, 0, 0};
-  if (!prefill_tc_supported(p) || p->cu_seqlens || (p->flags & GDN_SINGLE_PASS) || p->n_seq <= 0 ||
-      p->seq_len <= tc::C || sms <= 0)
+  SegPlan plan{1, 0, 0, 0};
+  if (!prefill_tc_supported(p) || p->n_seq <= 0 || sms <= 0) return plan;
+  if (p->cu_seqlens) {
+    // varlen: one pass; with more blocks than one wave, the sequences are
+    // launched longest first (an LPT order sorted on the device), so that the
+    // longest chains do not start in the last wave
+    const long long blocks = (long long)p->n_seq * p->H * (p->dv / tc::DVS);
+    plan.lpt = (p->n_seq >= 2 && p->n_seq <= tc::kLptMaxSeqs && blocks > sms) ? 1 : 0;
     return plan;
+  }
+  if ((p->flags & GDN_SINGLE_PASS) || p->seq_len <= tc::C) return plan;
   constexpr double kOutputChunk = 1.15;   // chunk step of a CTA with outputs / without
   const long long chains = (long long)p->n_seq * p->H;
   const long long slices = p->dv / tc::DVS;
@@ -1363,7 +1412,7 @@ SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
   auto waves = [&](long long ctas) { return (double)((ctas + sms - 1) / sms); };
   const double one_pass = waves(chains * slices) * (n_chunks * kOutputChunk + 1.5);
   double best = 0.0;
-  SegPlan cand{1, 0, 0};
+  SegPlan cand{1, 0, 0, 0};
   for (int seg = 1; seg < n_chunks; ++seg) {
     for (int seg0 = seg; seg0 >= 1 && seg0 >= seg - 4; --seg0) {
       if (seg0 >= n_chunks) continue;
@@ -1376,7 +1425,7 @@ SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
           waves(chains * (P - 1) * slices) * (seg * kOutputChunk + 1.5) + (P > 2 ? 0.8 * (P - 2) + 0.5 : 0.0);
       if (cand.n_segs == 1 || cost < best) {
         best = cost;
-        cand = SegPlan{P, seg * tc::C, seg0 * tc::C};
+        cand = SegPlan{P, seg * tc::C, seg0 * tc::C, 0};
       }
     }
   }
@@ -1387,6 +1436,7 @@ SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan) {
+  if (plan.lpt) return align256((size_t)p->n_seq * sizeof(int32_t));
   if (plan.n_segs <= 1) return 0;
   const size_t sd = (size_t)p->H * tc::DK * p->dv * sizeof(float);
   const size_t md = (size_t)p->H * tc::DK * tc::DK * sizeof(float);
@@ -1459,7 +1509,14 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   kp.seg0_tok = 0;
   kp.Bws = kp.Mws = nullptr;
   kp.Sst = nullptr;
+  kp.order = nullptr;
   const long long chains = (long long)p->n_seq * p->H;
+  if (plan.lpt) {
+    int32_t* order = static_cast<int32_t*>(ws);
+    tc::gdn_lpt_order_kernel<<<1, tc::kLptThreads, 0, stream>>>(p->cu_seqlens, p->n_seq, order);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    kp.order = order;
+  }
   if (plan.n_segs <= 1) return tc_launch(mq, mk, mv, kp, chains * kp.n_slices, stream);
 
   // segmented: workspace = [B_1 .. B_{P-2} | M_1 .. M_{P-2} | S_1 .. S_{P-1}]

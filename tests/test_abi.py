@@ -148,9 +148,23 @@ def test_schedule_query_rejects_what_the_call_rejects(lib):
     assert launches.value == 0
 
 
-def test_workspace_zero_for_varlen(lib):
-    p = _params(n_seq=1, seq_len=0, total_tokens=4096, H=16, cu_seqlens=1 << 32)
-    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
+def test_varlen_workspace_holds_the_longest_first_order(lib):
+    """Varlen calls run one pass.  With more blocks than one wave they ask for
+    one int32 per sequence (the device-sorted longest-first order of the
+    sequences) and take two launches; one wave, a single sequence, the precise
+    path and more sequences than the sort handles need none."""
+    def query(**kw):
+        p = _params(seq_len=0, cu_seqlens=1 << 32, o=1 << 40, **kw)
+        n, launches = ctypes.c_int(), ctypes.c_int()
+        assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), None, None,
+                                          ctypes.byref(launches)) == B.GDN_OK
+        return lib.gdn_chunk_fwd_workspace(ctypes.byref(p)), n.value, launches.value
+    assert query(n_seq=64, total_tokens=64 * 1000, H=16, dv=256) == (256, 1, 2)
+    assert query(n_seq=1000, total_tokens=1000 * 100, H=16) == (4096, 1, 2)
+    assert query(n_seq=1, total_tokens=4096, H=16) == (0, 1, 1)
+    assert query(n_seq=4, total_tokens=4000, H=2) == (0, 1, 1)
+    assert query(n_seq=64, total_tokens=64 * 1000, H=16, dv=256, flags=B.GDN_PRECISE) == (0, 1, 1)
+    assert query(n_seq=5000, total_tokens=5000 * 10, H=16) == (0, 1, 1)
 
 
 def test_prefill_rejects_short_or_misaligned_workspace_on_host(lib):
@@ -170,7 +184,8 @@ def test_python_workspace_query_matches_c(lib):
     assert lla.prefill_workspace_bytes(1, 4096, 16, 128, 128) == lib.gdn_chunk_fwd_workspace(
         ctypes.byref(p))
     assert lla.prefill_workspace_bytes(1, 4096, 16, 128, 128, flags=B.GDN_SINGLE_PASS) == 0
-    assert lla.prefill_workspace_bytes(64, 1000, 16, 128, 256, varlen=True) == 0
+    assert lla.prefill_workspace_bytes(64, 1000, 16, 128, 256, varlen=True) == 256   # the order
+    assert lla.prefill_workspace_bytes(4, 1000, 2, 128, 128, varlen=True) == 0       # one wave
 
 
 @pytest.mark.parametrize("args,expect", [

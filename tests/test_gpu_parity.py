@@ -267,6 +267,34 @@ def test_prefill_tc_varlen_dv256_l2norm():
     _status_ok()
 
 
+def test_varlen_longest_first_order_matches_natural_order():
+    """With more blocks than one wave a varlen call launches its sequences
+    longest first (an order sorted on the device into the workspace).  Each
+    chain's arithmetic does not depend on where it runs, so the outputs equal
+    those of the natural order (no workspace) bit for bit; lengths include 0,
+    1, a full chunk and ties; both agree with the oracle."""
+    import ctypes
+    from looped_linear_attention_b200 import _binding as B
+    lengths = [0, 1, 64, 65, 700, 300, 300, 129, 5, 640] * 4       # 40 sequences
+    wl = _wl("varlen", H=4, dv=128, random_s0=True)                 # 40 x 4 = 160 blocks
+    inp = W.prefill_inputs(wl, "cpu", lengths=lengths)
+    assert lla.prefill_schedule(len(lengths), 100, 4, 128, 128, varlen=True)["launches"] == 2
+    o_lpt, S_lpt = _gpu_prefill(inp)                                 # the binding passes the workspace
+    q, k, v, a, b, s0 = (inp[n].cuda() for n in ("q", "k", "v", "a", "b", "S0"))
+    cu = torch.from_numpy(inp["cu_seqlens"]).cuda()
+    o = torch.full_like(q[:, :, :128], float("nan"))
+    S_T = torch.full_like(s0, float("nan"))
+    p = B.gdn_fwd_params(q.data_ptr(), k.data_ptr(), v.data_ptr(), a.data_ptr(), b.data_ptr(),
+                         s0.data_ptr(), o.data_ptr(), S_T.data_ptr(), cu.data_ptr(), len(lengths), 0,
+                         inp["total_tokens"], 4, 128, 128, B.GDN_BF16, 1.0, 0)
+    assert lla.library().gdn_chunk_fwd(ctypes.byref(p), None, 0, None) == lla.GDN_OK
+    torch.cuda.synchronize()
+    _status_ok()
+    assert torch.equal(host(o), o_lpt) and torch.equal(host(S_T), S_lpt)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o_lpt, S_lpt, o_ref, S_ref, fp32=False)
+
+
 def test_prefill_tc_in_place_state():
     wl = _wl("long_prefill", n_seq=2, H=2, seq_len=130, random_s0=True)
     inp = W.prefill_inputs(wl, "cpu")

@@ -23,6 +23,7 @@ the same workload.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
 import os
@@ -255,28 +256,41 @@ def run_ours(args, rank, world, local):
         runner.run(inp["h0"], inp["Wq"], inp["Wk"], inp["Wv"], inp["a"], inp["b"], inp["rho"],
                    out=out)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    runner.mixer_events.clear()
-    step_events = []
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        for _ in range(args.steps):
+    def timed(one_step, sampler=None):
+        """W warm-up steps, then K steps between CUDA events on the launching
+        stream (L2 flushed before each); returns the per-step milliseconds."""
+        for _ in range(args.warmup):
             flush.zero_()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            step()
-            e1.record(stream)
-            step_events.append((e0, e1))
+            one_step()
         torch.cuda.synchronize()
-    barrier(world)
-    gdn_events = list(runner.mixer_events)
+        events = []
+        barrier(world)
+        torch.cuda.synchronize()
+        with (sampler if sampler is not None else contextlib.nullcontext()):
+            for _ in range(args.steps):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                one_step()
+                e1.record(stream)
+                events.append((e0, e1))
+            torch.cuda.synchronize()
+        barrier(world)
+        return [a.elapsed_time(b) for a, b in events]
+
+    # stream-launched steps: per-mixer-call CUDA events for the roofline
+    step_ms_stream = timed(step)
+    gdn_events = list(runner.mixer_events)[-args.steps * wl.loops:]
     runner.time_mixer = False
-    step_ms = [a.elapsed_time(b) for a, b in step_events]
+    # the step as one CUDA-graph replay (every launch of the T loops, no host
+    # work between them): the headline value
+    runner_g = lla.LoopedPrefill(L, wl.H, wl.dk, wl.dv, wl.loops, dev)
+    out_g = torch.empty(L, d, dtype=torch.bfloat16, device=dev)
+    graph, _ = runner_g.capture(inp["h0"], inp["Wq"], inp["Wk"], inp["Wv"], inp["a"], inp["b"],
+                                inp["rho"], out=out_g)
+    clocks = ClockSampler(local)
+    step_ms = timed(graph.replay, clocks)
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
     tokens_per_step = L
     value = world * tokens_per_step * args.steps / total_s
@@ -328,6 +342,8 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; random-init projection weights)",
+        "step_launch": "one CUDA-graph replay per step (all T loops; LoopedPrefill.capture)",
+        "ms_per_step_stream": max_over_ranks(sum(step_ms_stream) / 1e3, world) * 1e3 / args.steps,
         "config": {"workload": "looped_prefill", "batch": 1, "seq_len": L, "d_model": d,
                    "heads": wl.H, "dk": wl.dk, "dv": wl.dv, "loops": wl.loops, "chunk": 64,
                    "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)"},

@@ -68,6 +68,32 @@ class LoopedPrefill:
             h_prev = h_next
         return h_prev
 
+    def capture(self, h0: torch.Tensor, Wq: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor,
+                a: torch.Tensor, b: torch.Tensor, rho: torch.Tensor, scale: float = 1.0,
+                out: Optional[torch.Tensor] = None):
+        """Records one `run` on these tensors into a CUDA graph.
+
+        Returns (graph, h): each graph.replay() repeats the whole T-loop step
+        (projections, mixer launches, residuals; no host work) on the same
+        buffers and leaves h^(T) in h.  The tensors' contents may change between
+        replays, their storage may not.  One eager run on a side stream first
+        sets up the library's lazy state (launch attributes, the status word)
+        outside the capture."""
+        dev = self.qkv.device
+        timing, self.time_mixer = self.time_mixer, False
+        try:
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(side):
+                self.run(h0, Wq, Wk, Wv, a, b, rho, scale=scale, out=out)
+            torch.cuda.current_stream(dev).wait_stream(side)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                h = self.run(h0, Wq, Wk, Wv, a, b, rho, scale=scale, out=out)
+        finally:
+            self.time_mixer = timing
+        return graph, h
+
 
 def stack_weights(Wq: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor):
     """One [3, d, d] tensor holding W_q, W_k, W_v, and its three planes (pass
@@ -100,10 +126,13 @@ class HostPipeline:
     device buffer sets and two copy streams (host-to-device, device-to-host)
     let the copies of one step overlap the compute of its neighbours; events
     keep a buffer set from being refilled before the step that used it is done.
-    The host buffers of a step must stay untouched until the event that
-    `submit` returns has completed (its copy-out is then finished)."""
+    With `graphs` (the default) the compute of a step is a CUDA-graph replay:
+    one graph per buffer set, captured on first use (and again when the
+    weights, rho or scale change).  The host buffers of a step must stay
+    untouched until the event that `submit` returns has completed (its
+    copy-out is then finished)."""
 
-    def __init__(self, runner: LoopedPrefill, device):
+    def __init__(self, runner: LoopedPrefill, device, graphs: bool = True):
         L, d, T = runner.L, runner.H * runner.dv, runner.loops
         self.runner = runner
         self.dev = torch.device(device)
@@ -116,6 +145,8 @@ class HostPipeline:
         self.inputs_free = [None, None]     # compute of the last step that read buffer set k
         self.output_free = [None, None]     # copy-out of the last step that wrote out[k]
         self.n = 0
+        self.graphs = graphs
+        self.graph = [None, None]           # (key, CUDA graph) per buffer set
 
     def submit(self, h_host, a_host, b_host, out_host, Wq, Wk, Wv, rho, scale: float = 1.0):
         compute = torch.cuda.current_stream(self.dev)
@@ -132,7 +163,7 @@ class HostPipeline:
         compute.wait_event(loaded)
         if self.output_free[k] is not None:
             compute.wait_event(self.output_free[k])
-        self.runner.run(self.h[k], Wq, Wk, Wv, self.a[k], self.b[k], rho, scale=scale, out=self.out[k])
+        self._compute(k, Wq, Wk, Wv, rho, scale)
         done = torch.cuda.Event()
         done.record(compute)
         self.inputs_free[k] = done
@@ -143,6 +174,19 @@ class HostPipeline:
             copied.record(self.s_out)
         self.output_free[k] = copied
         return copied
+
+    def _compute(self, k, Wq, Wk, Wv, rho, scale):
+        args = (self.h[k], Wq, Wk, Wv, self.a[k], self.b[k], rho)
+        if not self.graphs:
+            self.runner.run(*args, scale=scale, out=self.out[k])
+            return
+        # a replay reads whatever the captured addresses hold, so the key is
+        # the operands' storage, not their values
+        key = (Wq.data_ptr(), Wk.data_ptr(), Wv.data_ptr(), rho.data_ptr(), float(scale))
+        if self.graph[k] is None or self.graph[k][0] != key:
+            graph, _ = self.runner.capture(*args, scale=scale, out=self.out[k])
+            self.graph[k] = (key, graph)
+        self.graph[k][1].replay()
 
     def join(self, stream=None):
         """Makes `stream` (default: the current one) wait for every copy submitted so far."""

@@ -468,6 +468,32 @@ def test_looped_step_same_with_stacked_or_separate_weights():
     assert torch.equal(h_view, h_sep)
 
 
+def test_looped_step_graph_replay_equals_stream_run():
+    """The looped step captured in a CUDA graph (the segmented mixer's
+    dependent launches included) gives the stream-launched step's h^(T) bit for
+    bit, and again after its inputs are overwritten in place."""
+    wl = dataclasses.replace(W.WORKLOADS["looped_prefill"], seq_len=1024)
+    inp = W.looped_inputs(wl, "cuda")
+    assert lla.prefill_schedule(1, 1024, wl.H, wl.dk, wl.dv)["n_segs"] > 1
+    runner = lla.LoopedPrefill(inp["L"], wl.H, wl.dk, wl.dv, wl.loops, "cuda")
+    W3 = (inp["Wq"], inp["Wk"], inp["Wv"])
+    out = torch.empty(inp["L"], inp["d"], dtype=torch.bfloat16, device="cuda")
+    graph, h = runner.capture(inp["h0"], *W3, inp["a"], inp["b"], inp["rho"], out=out)
+    assert h.data_ptr() == out.data_ptr()
+    for i in range(2):
+        if i:
+            g = torch.Generator(device="cuda").manual_seed(W.seed_for("test", "graph", i))
+            inp["h0"].copy_(torch.randn(inp["h0"].shape, generator=g, device="cuda"))
+            inp["a"].pow_(1.05)
+        graph.replay()
+        torch.cuda.synchronize()
+        got = out.clone()
+        ref = runner.run(inp["h0"], *W3, inp["a"], inp["b"], inp["rho"]).clone()
+        torch.cuda.synchronize()
+        _status_ok()
+        assert torch.equal(got, ref)
+
+
 def test_host_pipeline_matches_device_steps():
     """HostPipeline (pinned host inputs and results, copies overlapped with the
     neighbouring steps' compute) gives the same h^(T) as LoopedPrefill.run on

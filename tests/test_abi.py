@@ -248,3 +248,31 @@ def test_stacked_projection_weights_are_used_in_place():
     assert stacked_view(Wq, Wk, Wv[:, :-1]) is None
     W3, q, k, w = stack_weights(Wq.clone(), Wk.clone(), Wv.clone())
     assert stacked_view(q, k, w).data_ptr() == W3.data_ptr()
+
+
+@pytest.mark.parametrize("n_seq,L,H,dv", [(1, 4096, 16, 128), (1, 8192, 16, 128), (2, 4096, 16, 128),
+                                         (1, 16384, 16, 128), (1, 4096, 8, 128), (1, 2048, 16, 128),
+                                         (1, 1024, 16, 128), (2, 1000, 2, 128), (1, 777, 2, 256),
+                                         (1, 2000, 2, 128), (3, 3000, 4, 256), (1, 130, 1, 128)])
+def test_segment_plan_covers_the_sequence(lib, n_seq, L, H, dv):
+    """The planner's segments tile each sequence exactly: segment 0 of seg0_tok
+    tokens, then segments of seg_tok (whole chunks of 64, segment 0 no longer
+    than the others), the last one ragged but not empty; and the workspace the
+    query asks for is exactly B and M for segments 1 .. P-2 plus start states
+    for segments 1 .. P-1, each buffer 256-byte aligned."""
+    p = _params(n_seq=n_seq, seq_len=L, total_tokens=n_seq * L, H=H, dv=dv, o=1 << 40)
+    n, tok0, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
+                                      ctypes.byref(tok), ctypes.byref(launches)) == B.GDN_OK
+    need = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
+    P = n.value
+    if P == 1:
+        assert (tok0.value, tok.value, launches.value, need) == (0, 0, 1, 0)
+        return
+    assert tok.value % 64 == 0 and tok0.value % 64 == 0 and 0 < tok0.value <= tok.value
+    assert tok0.value + (P - 2) * tok.value < L <= tok0.value + (P - 1) * tok.value
+    assert launches.value == (3 if P > 2 else 2)
+    align = lambda x: (x + 255) // 256 * 256
+    sd, md = H * 128 * dv * 4, H * 128 * 128 * 4
+    assert need == (align(n_seq * (P - 2) * sd) + align(n_seq * (P - 2) * md)
+                    + align(n_seq * (P - 1) * sd))

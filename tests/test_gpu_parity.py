@@ -295,6 +295,32 @@ def test_varlen_longest_first_order_matches_natural_order():
     _check(o_lpt, S_lpt, o_ref, S_ref, fp32=False)
 
 
+def test_varlen_longest_first_in_place_state_and_graph_capture():
+    """A multi-wave varlen call (length sort, then the prefill in that order)
+    with S_T written over S0, against the oracle; the same call captured in a
+    CUDA graph and replayed gives the eager call's outputs bit for bit."""
+    lengths = [700, 0, 64, 1, 300, 129, 65, 640, 300, 5] * 4
+    wl = _wl("varlen", H=4, dv=128, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu", lengths=lengths)
+    o, ST = _gpu_prefill(inp, alias=True)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(o, ST, o_ref, S_ref, fp32=False)
+    q, k, v, a, b = (inp[n].cuda() for n in ("q", "k", "v", "a", "b"))
+    s0 = inp["S0"].cuda()
+    cu = torch.from_numpy(inp["cu_seqlens"]).cuda()
+    o_e, S_e = lla.gdn_chunk_fwd(q, k, v, a, b, s0, cu)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        o_g, S_g = lla.gdn_chunk_fwd(q, k, v, a, b, s0, cu)
+    o_g.zero_()
+    S_g.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    _status_ok()
+    assert torch.equal(o_g, o_e) and torch.equal(S_g, S_e)
+
+
 def test_prefill_tc_in_place_state():
     wl = _wl("long_prefill", n_seq=2, H=2, seq_len=130, random_s0=True)
     inp = W.prefill_inputs(wl, "cpu")

@@ -76,6 +76,28 @@ def test_noalloc_matches_gdn_chunk_fwd_on_two_calls(lib):
         assert rel_l2(S_T, S_ref) < TOL_BF16_S
 
 
+def test_noalloc_varlen_longest_first(lib):
+    """A multi-wave varlen call keeps its length-sorted order in the scratch
+    array; outputs equal those of gdn_chunk_fwd."""
+    lengths = [640, 3, 64, 300, 0, 129] * 8                  # 48 sequences x 4 heads
+    wl = dataclasses.replace(W.WORKLOADS["varlen"], name="noalloc-varlen", H=4, dv=128,
+                             random_s0=True)
+    inp = W.prefill_inputs(wl, "cuda", lengths=lengths)
+    cu = torch.from_numpy(inp["cu_seqlens"]).cuda()
+    assert lla.prefill_workspace_bytes(len(lengths), 200, 4, 128, 128, varlen=True) > 0
+    o_ref, S_ref = lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S0"], cu)
+    o = torch.full_like(o_ref, float("nan"))
+    S_T = torch.full_like(S_ref, float("nan"))
+    p = B.gdn_fwd_params(inp["q"].data_ptr(), inp["k"].data_ptr(), inp["v"].data_ptr(),
+                         inp["a"].data_ptr(), inp["b"].data_ptr(), inp["S0"].data_ptr(),
+                         o.data_ptr(), S_T.data_ptr(), cu.data_ptr(), len(lengths), 0,
+                         inp["total_tokens"], 4, 128, 128, B.GDN_BF16, 1.0, 0)
+    assert lib.gdn_chunk_fwd_noalloc(ctypes.byref(p), None) == B.GDN_OK
+    torch.cuda.synchronize()
+    assert lla.gdn_get_device_status() == lla.GDN_OK
+    assert torch.equal(o, o_ref) and torch.equal(S_T, S_ref)
+
+
 def test_noalloc_rejects_shapes_beyond_the_scratch(lib):
     """A call whose segmented schedule would need more than the 32 MiB array
     (here 3 heads of one 131072-token sequence with dv = 256) returns

@@ -832,11 +832,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       // Warp 0 issues them and alone takes the waits they need (V; then the
       // buffer of W^T(c-1), free once the state team has read it), waits for the
       // products and arrives W_READY.  The other warps go straight on to chunk
-      // c+1 and wait there for G(c+1); its products are issued behind these
-      // (one tensor pipe, in order) and complete after them, so the T1/T2 and P
-      // tiles they overwrite are free.  No
-      // warp leaves the loop alone: after a failed wait warp 0 only skips work,
-      // and the next team barrier sees the abort flag.  Waiting for
+      // c+1; the team barrier at its top also waits for warp 0, which has seen
+      // these products complete by then, so the T1/T2 tiles they overwrite in
+      // the next solve are free.  No warp leaves the loop alone: after a failed
+      // wait warp 0 only skips work, and the next team barrier sees the abort
+      // flag.  Waiting for
       // W_CONSUMED(c-1) in every chunk also keeps W_READY from running two
       // phases ahead of the state team.
       if (warp == 0) {

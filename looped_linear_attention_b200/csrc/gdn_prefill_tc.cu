@@ -277,18 +277,6 @@ __device__ __forceinline__ void store_row32_bf16(uint8_t* tile, int row, int col
   }
 }
 
-__device__ __forceinline__ void store_row64_bf16(uint8_t* tile, int row, const float (&x)[64]) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 o;
-    o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
-    o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
-    o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
-    o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
-    *reinterpret_cast<uint4*>(tile + sw128_offset(row, c * 8)) = o;
-  }
-}
-
 // 2^x with the hardware base-2 exponential (relative error about 2^-22;
 // results below 2^-126 flush to zero).  Every decay factor of the chunk is
 // 2^(g2_i - g2_j) with g2 = log2 gamma.

@@ -332,3 +332,31 @@ def test_looped_forward_single_token_reads_back_value():
     n2 = (hh * hh).sum(-1, keepdims=True)
     expect = oracle.round_bf16((n2 / (n2 + 1e-6) * hh).reshape(1, d))
     np.testing.assert_array_equal(out, expect)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_segment_state_update_is_affine_in_its_start_state(seed):
+    """The state a segment ends in is M S_start + B: B is the end state from a
+    zero start, and M (dk x dk) is the end state of a run with v = 0 from the
+    identity (columns of the identity as dv = dk values).  The segmented
+    schedule relies on exactly this; the oracle must satisfy it for any start
+    state, and chaining the segments' (M, B) must give the one-pass end state."""
+    rng = np.random.default_rng(300 + seed)
+    L, H, dk, dv = 37, 2, 5, 3
+    q, k, v, a, b = _rand_case(rng, L, H, dk, dv, b_range=(0.0, 2.0))
+    S_start = rng.standard_normal((1, H, dk, dv))
+    _, S_direct = oracle.gdn_fwd(q, k, v, a, b, S_start)
+    _, B = oracle.gdn_fwd(q, k, v, a, b, None)
+    eye = np.broadcast_to(np.eye(dk), (1, H, dk, dk)).copy()
+    _, M = oracle.gdn_fwd(q[:, :, :], k, np.zeros((L, H, dk)), a, b, eye)
+    np.testing.assert_allclose(S_direct[0], np.einsum("hij,hjk->hik", M[0], S_start[0]) + B[0],
+                               rtol=1e-12, atol=1e-12)
+    # three segments chained through their (M, B) pairs equal one pass
+    cuts = [0, 11, 24, L]
+    S = S_start[0]
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        sl = slice(lo, hi)
+        _, Bp = oracle.gdn_fwd(q[sl], k[sl], v[sl], a[sl], b[sl], None)
+        _, Mp = oracle.gdn_fwd(q[sl], k[sl], np.zeros((hi - lo, H, dk)), a[sl], b[sl], eye)
+        S = np.einsum("hij,hjk->hik", Mp[0], S) + Bp[0]
+    np.testing.assert_allclose(S, S_direct[0], rtol=1e-11, atol=1e-11)

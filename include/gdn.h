@@ -55,7 +55,12 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 /* Flags for gdn_fwd_params.flags and gdn_decode_step(). */
 #define GDN_QK_L2NORM 0x1u /* normalise q and k per head in fp32 before use:
-                              x / sqrt(sum x^2 + 1e-6), then round to io dtype */
+                              x / sqrt(sum x^2 + 1e-6).  The precise prefill
+                              rounds the normalised vectors to io dtype; the
+                              tensor-core prefill and decode apply the inverse
+                              norms as fp32 factors to the products of the
+                              inputs as given (the same map, one rounding
+                              fewer)                                           */
 #define GDN_PRECISE   0x2u /* prefill: use the fp32 CUDA-core chunk kernel even
                               for bf16 inputs (slower, fp32 operands)          */
 #define GDN_SINGLE_PASS 0x4u /* prefill: run every (sequence, head) chain in one

@@ -88,7 +88,9 @@ class LoopedPrefill:
                 self.run(h0, Wq, Wk, Wv, a, b, rho, scale=scale, out=out)
             torch.cuda.current_stream(dev).wait_stream(side)
             graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
+            # thread-local capture: CUDA calls of other threads (a process
+            # group's watchdog, for one) do not invalidate it
+            with torch.cuda.graph(graph, capture_error_mode="thread_local"):
                 h = self.run(h0, Wq, Wk, Wv, a, b, rho, scale=scale, out=out)
         finally:
             self.time_mixer = timing

@@ -8,6 +8,8 @@ share no code.
 Every function works in float64 on host arrays and follows the definition on
 the page, not any kernel's blocking:
 
+* ``gdn_bwd`` -- reverse mode of ``gdn_fwd`` (gradients through the outputs
+  and the final states), token by token backwards over stored forward states.
 * ``gdn_fwd`` / ``gdn_decode`` -- the gated delta rule, token by token
   ("LT2: Linear-Time Looped Transformers", §2, "LT2." paragraph: state
   S_t in R^{dk x dv}; the mixer is Gated DeltaNet, Appendix C).  The per-token
@@ -59,6 +61,11 @@ def _load():
                                        ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_double]
         lib.oracle_gdn_fwd.restype = ctypes.c_int
+        lib.oracle_gdn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ip,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_double,
+                                       dp, dp, dp, dp, dp, dp]
+        lib.oracle_gdn_bwd.restype = ctypes.c_int
         lib.oracle_gdn_decode.argtypes = [dp, dp, dp, dp, dp, dp, dp,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_double]
@@ -116,6 +123,38 @@ def gdn_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, scale: float = 1.0):
     if rc != 0:
         raise ValueError("oracle_gdn_fwd rejected its arguments")
     return o, ST
+
+
+def gdn_bwd(q, k, v, a, b, dO, S0=None, dST=None, cu_seqlens=None, scale: float = 1.0):
+    """Reverse mode of ``gdn_fwd``: gradients of a loss through its outputs
+    (dO [n_tok, H, dv]) and final states (dST [n_seq, H, dk, dv] or None).
+    Returns a dict of float64 arrays dq, dk, dv, da, db, dS0 (the gradient
+    with respect to the start states, zeros-start included)."""
+    q, k, v, a, b, dO = (_f64(t) for t in (q, k, v, a, b, dO))
+    n_tok, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is None:
+        cu = np.array([0, n_tok], dtype=np.int32)
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int32))
+    n_seq = cu.shape[0] - 1
+    if int(cu[-1]) > n_tok or int(cu[0]) < 0:
+        raise ValueError("cu_seqlens out of range")
+    s0 = None if S0 is None else _f64(S0)
+    dst = None if dST is None else _f64(dST)
+    out = dict(dq=np.zeros((n_tok, H, dk)), dk=np.zeros((n_tok, H, dk)), dv=np.zeros((n_tok, H, dv)),
+               da=np.zeros((n_tok, H)), db=np.zeros((n_tok, H)), dS0=np.zeros((n_seq, H, dk, dv)))
+    rc = _load().oracle_gdn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), None if s0 is None else _ptr(s0),
+        _ptr(dO), None if dst is None else _ptr(dst), _ptr(cu, ctypes.c_int32),
+        n_seq, H, dk, dv, float(scale),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["da"]), _ptr(out["db"]),
+        _ptr(out["dS0"]))
+    if rc != 0:
+        raise ValueError("oracle_gdn_bwd rejected its arguments")
+    return out
 
 
 def gdn_decode(q, k, v, a, b, S, scale: float = 1.0):

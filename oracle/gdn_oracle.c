@@ -109,6 +109,137 @@ int oracle_gdn_fwd(const double *q, const double *k, const double *v,
     return bad ? -1 : 0;
 }
 
+/* Reverse mode of the prefill: gradients of a scalar loss that depends on the
+ * outputs o (through dO = dloss/do) and on the final states (through
+ * dST = dloss/dS_T, or NULL for none).  Per chain, token by token backwards,
+ * with G_t the gradient with respect to Sigma_t (the part flowing back from
+ * the later tokens and the final state, plus the readout of token t itself):
+ *
+ *     G_t          = dSigma_t + scale q_t dO_t^T
+ *     x_t          = Sigma_{t-1}^T k_t,      y_t = G_t^T k_t          (dv)
+ *     dq_t         = scale Sigma_t dO_t
+ *     dv_t         = b_t y_t
+ *     dk_t         = -a_t b_t (G_t x_t + Sigma_{t-1} y_t) + b_t G_t v_t
+ *     da_t         = <G_t, Sigma_{t-1}> - b_t y_t . x_t
+ *     db_t         = y_t . (v_t - a_t x_t)
+ *     dSigma_{t-1} = a_t (G_t - b_t k_t y_t^T)
+ *
+ * and dS0 = dSigma_0.  Each term is the derivative of one factor of the
+ * update Sigma_t = a_t (Sigma_{t-1} - b_t k_t x_t^T) + b_t k_t v_t^T or of the
+ * readout.  The forward states Sigma_0 .. Sigma_L of a chain are recomputed
+ * with the same token step and kept in memory ((L + 1) dk dv doubles per
+ * chain in flight).  Output layouts as the inputs; dS0 may be NULL.
+ * Returns 0, or -1 on bad arguments or memory exhaustion. */
+int oracle_gdn_bwd(const double *q, const double *k, const double *v,
+                   const double *a, const double *b, const double *S0,
+                   const double *dO, const double *dST, const int32_t *cu_seqlens,
+                   int n_seq, int H, int dk, int dv, double scale,
+                   double *dq, double *dk_out, double *dv_out, double *da, double *db,
+                   double *dS0)
+{
+    if (!q || !k || !v || !a || !b || !dO || !cu_seqlens) return -1;
+    if (!dq || !dk_out || !dv_out || !da || !db) return -1;
+    if (n_seq < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    for (int s = 0; s < n_seq; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
+    const long n_chain = (long)n_seq * H;
+    const size_t sz = (size_t)dk * dv;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *G = (double *)malloc(sizeof(double) * sz);
+        double *x = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *y = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *scratch = (double *)malloc(sizeof(double) * (size_t)dv);
+        if (!G || !x || !y || !scratch) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long c = 0; c < n_chain; ++c) {
+                const int s = (int)(c / H), h = (int)(c % H);
+                const int t0 = cu_seqlens[s], t1 = cu_seqlens[s + 1];
+                const int L = t1 - t0;
+                const size_t sidx = ((size_t)s * H + h) * sz;
+                /* forward states Sigma_0 .. Sigma_L of this chain */
+                double *states = (double *)malloc(sizeof(double) * sz * (size_t)(L + 1));
+                if (!states) {
+#pragma omp atomic write
+                    bad = 1;
+                    continue;
+                }
+                if (S0) memcpy(states, S0 + sidx, sizeof(double) * sz);
+                else memset(states, 0, sizeof(double) * sz);
+                for (int i = 0; i < L; ++i) {
+                    const size_t th = (size_t)(t0 + i) * H + h;
+                    memcpy(states + sz * (size_t)(i + 1), states + sz * (size_t)i, sizeof(double) * sz);
+                    gdn_token_step(states + sz * (size_t)(i + 1), dk, dv, q + th * dk, k + th * dk,
+                                   v + th * dv, a[th], b[th], scale, NULL, scratch);
+                }
+                /* backwards: G starts as the final-state gradient */
+                if (dST) memcpy(G, dST + sidx, sizeof(double) * sz);
+                else memset(G, 0, sizeof(double) * sz);
+                for (int i = L - 1; i >= 0; --i) {
+                    const size_t th = (size_t)(t0 + i) * H + h;
+                    const double *qt = q + th * dk, *kt = k + th * dk, *vt = v + th * dv;
+                    const double *dOt = dO + th * dv;
+                    const double at = a[th], bt = b[th];
+                    const double *Sig = states + sz * (size_t)(i + 1);    /* Sigma_t     */
+                    const double *Sp = states + sz * (size_t)i;           /* Sigma_{t-1} */
+                    /* G_t += scale q_t dO_t^T */
+                    for (int r = 0; r < dk; ++r)
+                        for (int j = 0; j < dv; ++j) G[(size_t)r * dv + j] += scale * qt[r] * dOt[j];
+                    /* dq_t = scale Sigma_t dO_t */
+                    for (int r = 0; r < dk; ++r) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dv; ++j) acc += Sig[(size_t)r * dv + j] * dOt[j];
+                        dq[th * dk + r] = scale * acc;
+                    }
+                    /* x = Sigma_{t-1}^T k,  y = G^T k */
+                    for (int j = 0; j < dv; ++j) x[j] = y[j] = 0.0;
+                    for (int r = 0; r < dk; ++r)
+                        for (int j = 0; j < dv; ++j) {
+                            x[j] += kt[r] * Sp[(size_t)r * dv + j];
+                            y[j] += kt[r] * G[(size_t)r * dv + j];
+                        }
+                    /* dv_t = b y */
+                    for (int j = 0; j < dv; ++j) dv_out[th * dv + j] = bt * y[j];
+                    /* dk_t = -a b (G x + Sigma_{t-1} y) + b G v */
+                    for (int r = 0; r < dk; ++r) {
+                        double gx = 0.0, sy = 0.0, gv = 0.0;
+                        for (int j = 0; j < dv; ++j) {
+                            gx += G[(size_t)r * dv + j] * x[j];
+                            sy += Sp[(size_t)r * dv + j] * y[j];
+                            gv += G[(size_t)r * dv + j] * vt[j];
+                        }
+                        dk_out[th * dk + r] = -at * bt * (gx + sy) + bt * gv;
+                    }
+                    /* da_t = <G, Sigma_{t-1}> - b y.x ;  db_t = y.(v - a x) */
+                    double gs = 0.0, yx = 0.0, yv = 0.0;
+                    for (size_t e = 0; e < sz; ++e) gs += G[e] * Sp[e];
+                    for (int j = 0; j < dv; ++j) {
+                        yx += y[j] * x[j];
+                        yv += y[j] * vt[j];
+                    }
+                    da[th] = gs - bt * yx;
+                    db[th] = yv - at * yx;
+                    /* dSigma_{t-1} = a (G - b k y^T) */
+                    for (int r = 0; r < dk; ++r)
+                        for (int j = 0; j < dv; ++j)
+                            G[(size_t)r * dv + j] = at * (G[(size_t)r * dv + j] - bt * kt[r] * y[j]);
+                }
+                if (dS0) memcpy(dS0 + sidx, G, sizeof(double) * sz);
+                free(states);
+            }
+        }
+        free(G);
+        free(x);
+        free(y);
+        free(scratch);
+    }
+    return bad ? -1 : 0;
+}
+
 /* Decode: one token for each of N independent slots (a slot is one
  * sequence x layer x loop state), H heads each; S [N][H][dk][dv] updated in
  * place, o [N][H][dv]. */

@@ -27,10 +27,22 @@ MUTATIONS = {
                                   "const double ki = q[i];\n        double *row"),
 }
 
+# mistakes in the reverse mode, caught by its own pins
+BWD_MUTATIONS = {
+    "bwd_key_cross_term_dropped": ("dk_out[th * dk + r] = -at * bt * (gx + sy) + bt * gv;",
+                                   "dk_out[th * dk + r] = -at * bt * gx + bt * gv;"),
+    "bwd_adjoint_decay_dropped": ("G[(size_t)r * dv + j] = at * (G[(size_t)r * dv + j] - bt * kt[r] * y[j]);",
+                                  "G[(size_t)r * dv + j] = (G[(size_t)r * dv + j] - bt * kt[r] * y[j]);"),
+    "bwd_query_grad_uses_previous_state": ("acc += Sig[(size_t)r * dv + j] * dOt[j];",
+                                           "acc += Sp[(size_t)r * dv + j] * dOt[j];"),
+    "bwd_write_strength_sign": ("db[th] = yv - at * yx;", "db[th] = yv + at * yx;"),
+}
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS))
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(BWD_MUTATIONS))
 def test_pins_catch_planted_mistake(tmp_path, name):
-    src, dst = MUTATIONS[name]
+    src, dst = MUTATIONS[name] if name in MUTATIONS else BWD_MUTATIONS[name]
+    pins = "test_oracle_pins.py" if name in MUTATIONS else "test_oracle_bwd_pins.py"
     shutil.copytree(os.path.join(ROOT, "oracle"), tmp_path / "oracle",
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
     shutil.copytree(os.path.join(ROOT, "tests"), tmp_path / "tests",
@@ -41,7 +53,7 @@ def test_pins_catch_planted_mistake(tmp_path, name):
     cfile.write_text(text.replace(src, dst))
     env = dict(os.environ, PYTHONPATH=str(tmp_path))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        str(tmp_path / "tests" / "test_oracle_pins.py")],
+                        str(tmp_path / "tests" / pins)],
                        cwd=tmp_path, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
     assert "failed" in r.stdout

@@ -320,6 +320,8 @@ def run_ours(args, rank, world, local):
         torch.cuda.empty_cache()
         extras["varlen"] = bench_prefill_workload(W.WORKLOADS["varlen"], dev, args, peaks, world)
         torch.cuda.empty_cache()
+        extras["backward"] = bench_backward(dev, args, peaks, world)
+        torch.cuda.empty_cache()
 
     st = lla.gdn_get_device_status()
     if st != lla.GDN_OK:
@@ -486,6 +488,51 @@ def bench_decode(wl, dev, args, peaks, world):
            "note": "one step = one token for 256 sequences x 24 layers x 4 loops (all slots)"}
     del inp, o
     return res
+
+
+def bench_backward(dev, args, peaks, world):
+    """One reverse-mode call (gdn_chunk_bwd) on 8 sequences x 1024 tokens x 16
+    heads, dk = dv = 128, bf16 inputs, with a final-state gradient.  Algorithmic
+    bytes per (token, head): q, k, v and grad_o in bf16 (8 dk), a and b, and the
+    fp32 gradients of q, k, v, a and b (12 dk + 8); plus S0, grad_S_T, grad_S0
+    per chain."""
+    import dataclasses
+    import torch
+    import looped_linear_attention_b200 as lla
+    from looped_linear_attention_b200 import workloads as W
+    wl = dataclasses.replace(W.WORKLOADS["long_prefill"], name="backward", n_seq=8, seq_len=1024,
+                             random_s0=True)
+    inp = W.prefill_inputs(wl, dev)
+    g = torch.Generator(device=dev).manual_seed(W.seed_for("bench", "backward"))
+    go = torch.randn(inp["v"].shape, generator=g, device=dev).to(wl.dtype)
+    gST = torch.randn(wl.n_seq, wl.H, wl.dk, wl.dv, generator=g, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return lla.gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], go, inp["S0"], gST,
+                                 n_seq=wl.n_seq)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    n = 2
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        e0.record(stream)
+        for _ in range(n):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n
+    tokens = wl.n_seq * wl.seq_len
+    nbytes = tokens * wl.H * (8 * wl.dk + 12 * wl.dk + 8 + 8) + 3 * wl.n_seq * wl.H * wl.dk * wl.dv * 4
+    gbs = nbytes / t / 1e9
+    return {"tokens_per_s": world * tokens / t, "ms_per_call": t * 1e3, "achieved_gbs": gbs,
+            "frac_of_hbm": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
+            "tokens": tokens, "heads": wl.H, "dk": wl.dk, "dv": wl.dv, "clocks": clocks.summary(),
+            "kernel": "gdn_bwd_kernel (first path: fp32 CUDA cores, one CTA per chain)"}
 
 
 # ------------------------------------------------------------------ CPU oracle

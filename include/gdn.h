@@ -184,6 +184,59 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_params *p, void *ws, size_t ws_bytes,
 gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_params *p, cudaStream_t stream);
 
 /*
+ * Reverse mode of gdn_chunk_fwd: gradients of a loss that depends on the
+ * outputs o (through grad_o = dloss/do) and on the final states S_T (through
+ * grad_S_T) with respect to q, k, v, a, b and S0.  Per token, with G_t the
+ * gradient with respect to S_t (the part flowing back from the later tokens and
+ * the final state, plus the readout of token t), x_t = S_{t-1}^T k_t and
+ * y_t = G_t^T k_t:
+ *     G_t      = dS_t + scale q_t grad_o_t^T
+ *     grad_q_t = scale S_t grad_o_t          grad_v_t = b_t y_t
+ *     grad_k_t = -a_t b_t (G_t x_t + S_{t-1} y_t) + b_t G_t v_t
+ *     grad_a_t = <G_t, S_{t-1}> - b_t y_t . x_t
+ *     grad_b_t = y_t . (v_t - a_t x_t)
+ *     dS_{t-1} = a_t (G_t - b_t k_t y_t^T)
+ * and grad_S0 = dS_0: the derivatives of the factors of the update as written
+ * above gdn_fwd_params ("LT2: Linear-Time Looped Transformers", §2).
+ *
+ * Inputs as in gdn_fwd_params (q, k, v, a, b, S0, cu_seqlens, n_seq, seq_len,
+ * total_tokens, H, dk, dv, io_dtype, scale), plus
+ *   grad_o      [total_tokens][H][dv]   io_dtype
+ *   grad_S_T    [n_seq][H][dk][dv]      fp32, or NULL (no loss term on S_T)
+ * Outputs, fp32, overwritten, none overlapping an input:
+ *   grad_q, grad_k [total_tokens][H][dk]; grad_v [total_tokens][H][dv];
+ *   grad_a, grad_b [total_tokens][H];     grad_S0 [n_seq][H][dk][dv] or NULL.
+ * Supported: dk in {64, 128}; dv a multiple of 32, at most 256; flags 0 (the
+ * in-kernel q/k norm has no reverse mode here: differentiate it outside).
+ * This first implementation runs on the CUDA cores in fp32: one CTA per
+ * (sequence, head) chain, which recomputes the forward states from checkpoints
+ * it takes every 64 tokens and walks each chunk backwards.
+ * ws/ws_bytes: device workspace of at least gdn_chunk_bwd_workspace(p) bytes,
+ * 256-byte aligned (the checkpoints, one chunk of states and the running G of
+ * every chain); a missing or short workspace returns GDN_ERR_WORKSPACE.
+ */
+typedef struct {
+    const void *q, *k, *v;
+    const float *a, *b;
+    const float *S0;
+    const void *grad_o;
+    const float *grad_S_T;
+    float *grad_q, *grad_k, *grad_v, *grad_a, *grad_b, *grad_S0;
+    const int32_t *cu_seqlens;
+    int n_seq, seq_len, total_tokens, H, dk, dv;
+    gdn_dtype io_dtype;
+    float scale;
+    unsigned flags;
+} gdn_bwd_params;
+
+/* Bytes of device workspace gdn_chunk_bwd needs (host only); (size_t)-1 if the
+ * parameters are invalid. */
+size_t gdn_chunk_bwd_workspace(const gdn_bwd_params *p);
+
+gdn_status gdn_chunk_bwd(const gdn_bwd_params *p, void *ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/*
  * One decode step: one new token for each of N independent state slots (a slot
  * is one sequence x layer x loop state), H heads each.
  *   q, k [N][H][dk], v [N][H][dv], o [N][H][dv]  io_dtype

@@ -14,13 +14,14 @@ No compute runs in Python: if the library is missing, every entry point raises.
 """
 from ._binding import (GDN_BF16, GDN_ERR_CUDA, GDN_ERR_INVALID, GDN_ERR_TIMEOUT,
                        GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_F32, GDN_OK, GDN_PRECISE,
-                       GDN_QK_L2NORM, GDN_SINGLE_PASS, GDN_TEST_WAIT_TIMEOUT, GdnError, gdn_chunk_fwd, gdn_decode_step,
+                       GDN_QK_L2NORM, GDN_SINGLE_PASS, GDN_TEST_WAIT_TIMEOUT, GdnError, gdn_chunk_bwd,
+                       gdn_chunk_fwd, gdn_decode_step,
                        gdn_get_device_status, library, loop_residual, prefill_schedule, prefill_workspace_bytes,
                        status_string, version)
 from .looped import HostPipeline, LoopedPrefill, stack_weights
 
 __all__ = [
-    "gdn_chunk_fwd", "gdn_decode_step", "loop_residual", "gdn_get_device_status",
+    "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "loop_residual", "gdn_get_device_status",
     "prefill_schedule", "prefill_workspace_bytes",
     "LoopedPrefill", "HostPipeline", "stack_weights", "GdnError", "library", "status_string", "version",
     "GDN_OK", "GDN_ERR_INVALID", "GDN_ERR_UNSUPPORTED", "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT",

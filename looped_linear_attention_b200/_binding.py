@@ -52,6 +52,20 @@ class gdn_fwd_params(ctypes.Structure):
     ]
 
 
+class gdn_bwd_params(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("a", ctypes.c_void_p), ("b", ctypes.c_void_p), ("S0", ctypes.c_void_p),
+        ("grad_o", ctypes.c_void_p), ("grad_S_T", ctypes.c_void_p),
+        ("grad_q", ctypes.c_void_p), ("grad_k", ctypes.c_void_p), ("grad_v", ctypes.c_void_p),
+        ("grad_a", ctypes.c_void_p), ("grad_b", ctypes.c_void_p), ("grad_S0", ctypes.c_void_p),
+        ("cu_seqlens", ctypes.c_void_p),
+        ("n_seq", ctypes.c_int), ("seq_len", ctypes.c_int), ("total_tokens", ctypes.c_int),
+        ("H", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
+        ("io_dtype", ctypes.c_int), ("scale", ctypes.c_float), ("flags", ctypes.c_uint),
+    ]
+
+
 _lib = None
 
 
@@ -70,6 +84,10 @@ def library() -> ctypes.CDLL:
         lib.gdn_chunk_fwd_schedule.argtypes = [ctypes.POINTER(gdn_fwd_params)] + [
             ctypes.POINTER(ctypes.c_int)] * 4
         lib.gdn_chunk_fwd_schedule.restype = i32
+        lib.gdn_chunk_bwd_workspace.argtypes = [ctypes.POINTER(gdn_bwd_params)]
+        lib.gdn_chunk_bwd_workspace.restype = ctypes.c_size_t
+        lib.gdn_chunk_bwd.argtypes = [ctypes.POINTER(gdn_bwd_params), vp, ctypes.c_size_t, vp]
+        lib.gdn_chunk_bwd.restype = i32
         lib.gdn_chunk_fwd.argtypes = [ctypes.POINTER(gdn_fwd_params), vp, ctypes.c_size_t, vp]
         lib.gdn_chunk_fwd.restype = i32
         lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
@@ -165,6 +183,59 @@ def gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd")
     return o, S_T
+
+
+def gdn_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,
+                  b: torch.Tensor, grad_o: torch.Tensor, S0: Optional[torch.Tensor] = None,
+                  grad_S_T: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
+                  *, n_seq: Optional[int] = None, scale: float = 1.0, want_grad_S0: bool = True,
+                  stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Reverse mode of gdn_chunk_fwd (see gdn_chunk_bwd in include/gdn.h).
+
+    Inputs as gdn_chunk_fwd plus grad_o [T, H, dv] (io dtype) and grad_S_T
+    [n_seq, H, dk, dv] fp32 (or None).  Returns fp32 gradients
+    {"q", "k", "v", "a", "b", "S0"} ("S0" None unless want_grad_S0)."""
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    _check(q, "q", q.dtype)
+    _check(k, "k", q.dtype, (T, H, dk))
+    _check(v, "v", q.dtype, (T, H, dv))
+    _check(grad_o, "grad_o", q.dtype, (T, H, dv))
+    _check(a, "a", torch.float32, (T, H))
+    _check(b, "b", torch.float32, (T, H))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        ns, seq_len = cu_seqlens.numel() - 1, 0
+    else:
+        ns = 1 if n_seq is None else int(n_seq)
+        if ns <= 0 or T % ns != 0:
+            raise ValueError("without cu_seqlens, the token count must be n_seq * seq_len")
+        seq_len = T // ns
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (ns, H, dk, dv))
+    if grad_S_T is not None:
+        _check(grad_S_T, "grad_S_T", torch.float32, (ns, H, dk, dv))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"q": torch.empty(T, H, dk, **f32), "k": torch.empty(T, H, dk, **f32),
+         "v": torch.empty(T, H, dv, **f32), "a": torch.empty(T, H, **f32), "b": torch.empty(T, H, **f32),
+         "S0": torch.empty(ns, H, dk, dv, **f32) if want_grad_S0 else None}
+    p = gdn_bwd_params(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0), _ptr(grad_o),
+                       _ptr(grad_S_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["a"]),
+                       _ptr(g["b"]), _ptr(g["S0"]), _ptr(cu_seqlens), ns, seq_len, T, H, dk, dv,
+                       _DTYPES[q.dtype], float(scale), 0)
+    lib = library()
+    ws = lib.gdn_chunk_bwd_workspace(ctypes.byref(p))
+    if ws == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_INVALID, "gdn_chunk_bwd")
+    work = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
+    if work is not None and stream is not None:
+        work.record_stream(stream)
+    st = lib.gdn_chunk_bwd(ctypes.byref(p), _ptr(work), ctypes.c_size_t(ws), _stream_ptr(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_bwd")
+    return g
 
 
 def _shape_params(n_seq, seq_len, H, dk, dv, dtype, flags, varlen):

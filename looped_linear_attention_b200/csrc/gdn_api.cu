@@ -19,6 +19,8 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
 cudaError_t launch_loop_residual(const void* h_tilde, const void* h_prev, const float* rho,
                                  void* h_out, int64_t rows, int d, gdn_dtype dt, int num_sms,
                                  cudaStream_t stream);
+size_t bwd_workspace(const gdn_bwd_params* p);
+gdn_status launch_bwd(const gdn_bwd_params* p, unsigned* status, void* ws, cudaStream_t stream);
 }  // namespace gdn
 
 // Device status word: kernels record the first error they hit (atomicCAS from 0).
@@ -111,9 +113,50 @@ gdn_status validate_fwd(const gdn_fwd_params* p) {
   return GDN_OK;
 }
 
+gdn_status validate_bwd(const gdn_bwd_params* p) {
+  if (!p) return GDN_ERR_INVALID;
+  if (!dtype_ok(p->io_dtype)) return GDN_ERR_INVALID;
+  if (p->n_seq < 0 || p->H <= 0 || p->total_tokens < 0 || p->dk <= 0 || p->dv <= 0) return GDN_ERR_INVALID;
+  if (p->flags != 0) return GDN_ERR_UNSUPPORTED;
+  if (p->dk != 64 && p->dk != 128) return GDN_ERR_UNSUPPORTED;
+  if (p->dv % 32 != 0 || p->dv > 256) return GDN_ERR_UNSUPPORTED;
+  if (!p->cu_seqlens) {
+    if (p->seq_len < 0 || (long long)p->n_seq * p->seq_len != p->total_tokens) return GDN_ERR_INVALID;
+  }
+  if (p->n_seq == 0) return GDN_OK;
+  if (p->total_tokens > 0) {
+    const void* need[] = {p->q, p->k, p->v, p->a, p->b, p->grad_o,
+                          p->grad_q, p->grad_k, p->grad_v, p->grad_a, p->grad_b};
+    for (const void* x : need)
+      if (!x || !aligned16(x)) return GDN_ERR_INVALID;
+  }
+  const void* opt[] = {p->S0, p->grad_S_T, p->grad_S0, p->cu_seqlens};
+  for (const void* x : opt)
+    if (x && !aligned16(x)) return GDN_ERR_INVALID;
+  return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t gdn_chunk_bwd_workspace(const gdn_bwd_params* p) {
+  if (validate_bwd(p) != GDN_OK) return (size_t)-1;
+  if (p->n_seq == 0) return 0;
+  return gdn::bwd_workspace(p);
+}
+
+gdn_status gdn_chunk_bwd(const gdn_bwd_params* p, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const gdn_status v = validate_bwd(p);
+  if (v != GDN_OK) return v;
+  if (p->n_seq == 0) return GDN_OK;
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)) return GDN_ERR_INVALID;
+  const size_t need = gdn::bwd_workspace(p);
+  if (!ws || ws_bytes < need) return GDN_ERR_WORKSPACE;
+  unsigned* st = status_ptr();
+  if (!st) return GDN_ERR_CUDA;
+  return gdn::launch_bwd(p, st, ws, stream);
+}
 
 int gdn_version(void) { return 100; }
 

@@ -276,3 +276,41 @@ def test_segment_plan_covers_the_sequence(lib, n_seq, L, H, dv):
     sd, md = H * 128 * dv * 4, H * 128 * 128 * 4
     assert need == (align(n_seq * (P - 2) * sd) + align(n_seq * (P - 2) * md)
                     + align(n_seq * (P - 1) * sd))
+
+
+def _bwd_params(**kw):
+    p = B.gdn_bwd_params()
+    base = dict(q=1 << 32, k=2 << 32, v=3 << 32, a=4 << 32, b=5 << 32, grad_o=6 << 32,
+                grad_q=7 << 32, grad_k=8 << 32, grad_v=9 << 32, grad_a=10 << 32, grad_b=11 << 32,
+                n_seq=2, seq_len=100, total_tokens=200, H=2, dk=128, dv=128,
+                io_dtype=B.GDN_BF16, scale=1.0, flags=0)
+    base.update(kw)
+    for name, val in base.items():
+        setattr(p, name, val)
+    return p
+
+
+def test_backward_validation_and_workspace(lib):
+    """gdn_chunk_bwd: host-side rejections before any launch, and a workspace of
+    one checkpoint slot per 64 tokens (plus two per sequence and one) per head,
+    one chunk of 65 states and the running gradient per chain."""
+    p = _bwd_params()
+    need = lib.gdn_chunk_bwd_workspace(ctypes.byref(p))
+    sd = 128 * 128 * 4
+    align = lambda x: (x + 255) // 256 * 256
+    slots = 200 // 64 + 2 * 2 + 1
+    assert need == align(2 * slots * sd) + align(4 * 65 * sd) + align(4 * sd)
+    bad = ctypes.c_size_t(-1).value
+    for kw, status in [(dict(dk=96), B.GDN_ERR_UNSUPPORTED), (dict(dv=300), B.GDN_ERR_UNSUPPORTED),
+                       (dict(dv=48), B.GDN_ERR_UNSUPPORTED), (dict(flags=B.GDN_QK_L2NORM), B.GDN_ERR_UNSUPPORTED),
+                       (dict(H=0), B.GDN_ERR_INVALID), (dict(total_tokens=199), B.GDN_ERR_INVALID),
+                       (dict(grad_o=None), B.GDN_ERR_INVALID), (dict(q=(1 << 32) + 8), B.GDN_ERR_INVALID)]:
+        q = _bwd_params(**kw)
+        assert lib.gdn_chunk_bwd_workspace(ctypes.byref(q)) == bad, kw
+        assert lib.gdn_chunk_bwd(ctypes.byref(q), ctypes.c_void_p(1 << 40), 1 << 40, None) == status, kw
+    assert lib.gdn_chunk_bwd(ctypes.byref(p), None, 0, None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_chunk_bwd(ctypes.byref(p), ctypes.c_void_p(1 << 40), need - 256, None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_chunk_bwd(ctypes.byref(p), ctypes.c_void_p((1 << 40) + 16), need, None) == B.GDN_ERR_INVALID
+    empty = _bwd_params(n_seq=0, seq_len=0, total_tokens=0)
+    assert lib.gdn_chunk_bwd_workspace(ctypes.byref(empty)) == 0
+    assert lib.gdn_chunk_bwd(ctypes.byref(empty), None, 0, None) == B.GDN_OK

@@ -314,3 +314,26 @@ def test_backward_validation_and_workspace(lib):
     empty = _bwd_params(n_seq=0, seq_len=0, total_tokens=0)
     assert lib.gdn_chunk_bwd_workspace(ctypes.byref(empty)) == 0
     assert lib.gdn_chunk_bwd(ctypes.byref(empty), None, 0, None) == B.GDN_OK
+
+
+def test_backward_checkpoint_slots_never_overlap():
+    """The reverse-mode kernel keeps chain (s, h)'s checkpoints in slots
+    t0 / 64 + 2 s .. + ceil(len / 64) - 1 of head h, with total / 64 + 2 n + 1
+    slots per head in the workspace: over random length mixes (zeros, single
+    tokens, exact multiples of 64) no two sequences share a slot and every slot
+    is inside the allocation."""
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for trial in range(300):
+        n = int(rng.integers(1, 40))
+        lens = rng.choice([0, 1, 63, 64, 65, 128, 129, int(rng.integers(0, 700))], size=n)
+        cu = np.concatenate([[0], np.cumsum(lens)])
+        total = int(cu[-1])
+        slots = total // 64 + 2 * n + 1
+        used = set()
+        for s in range(n):
+            base = int(cu[s]) // 64 + 2 * s
+            for c in range((int(lens[s]) + 63) // 64):
+                slot = base + c
+                assert 0 <= slot < slots and slot not in used, (trial, s, c)
+                used.add(slot)

@@ -30,6 +30,10 @@
  *     gdn_get_device_status().
  *   - Thread safety: calls on different streams may run concurrently; they share
  *     only read-only launch constants and the device status word.
+ *   - Devices: the kernels' shared-memory launch attributes are set on the
+ *     first call of the process, on the device current then; run one process
+ *     per GPU (as the benchmark and the tests do).  A process that drives
+ *     several GPUs gets GDN_ERR_CUDA on launches for the others.
  */
 #ifndef LOOPED_GDN_H
 #define LOOPED_GDN_H

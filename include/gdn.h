@@ -32,8 +32,9 @@
  *     only read-only launch constants and the device status word.
  *   - Devices: the kernels' shared-memory launch attributes are set on the
  *     first call of the process, on the device current then; run one process
- *     per GPU (as the benchmark and the tests do).  A process that drives
- *     several GPUs gets GDN_ERR_CUDA on launches for the others.
+ *     per GPU (as the benchmark and the tests do).  Driving several GPUs from
+ *     one process is not tested; a launch that the attributes do not cover
+ *     fails with GDN_ERR_CUDA (no fault).
  */
 #ifndef LOOPED_GDN_H
 #define LOOPED_GDN_H

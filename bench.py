@@ -330,6 +330,8 @@ def run_ours(args, rank, world, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)
+        if "backward" in extras:   # the reverse mode's oracle, beside its GPU figure
+            extras["backward"]["cpu_baseline"] = cpu_baseline_backward()
 
     line = {
         "metric": METRIC,
@@ -565,6 +567,34 @@ def cpu_baseline(seconds_target: float = 15.0, sample_tokens: int = 4096):
             "sample": f"first {Ls} of {wl.seq_len} tokens, all {wl.loops} loops, d={wl.H * wl.dk}, "
                       f"{runs} run(s), {el:.1f} s; fp64 C oracle (OpenMP) + numpy projections",
             "cpu": model}
+
+
+def cpu_baseline_backward(seconds_target: float = 3.0, sample_tokens: int = 256):
+    """The oracle's reverse mode beside the GPU one: the first `sample_tokens`
+    tokens of each of the 16 heads of one sequence of the backward workload
+    (dk = dv = 128, with a final-state gradient), repeated for about
+    `seconds_target` seconds on this host's cores."""
+    import dataclasses
+    import torch
+    import oracle
+    from looped_linear_attention_b200 import workloads as W
+    wl = dataclasses.replace(W.WORKLOADS["long_prefill"], name="backward", n_seq=1,
+                             seq_len=sample_tokens, random_s0=True)
+    inp = W.prefill_inputs(wl, "cpu")
+    g = torch.Generator().manual_seed(W.seed_for("bench", "backward", "cpu"))
+    go = torch.randn(inp["v"].shape, generator=g).to(wl.dtype)
+    gST = torch.randn(1, wl.H, wl.dk, wl.dv, generator=g)
+    t0 = time.perf_counter()
+    runs = 0
+    while True:
+        oracle.gdn_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], go, inp["S0"], gST)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el > seconds_target or runs >= 20:
+            break
+    return {"value": sample_tokens * runs / el, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{sample_tokens} tokens x {wl.H} heads, dk = dv = {wl.dk}, "
+                                        f"{runs} run(s), {el:.1f} s; fp64 C oracle (OpenMP)"}
 
 
 def run_reference(args, rank, world):

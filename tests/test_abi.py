@@ -337,3 +337,15 @@ def test_backward_checkpoint_slots_never_overlap():
                 slot = base + c
                 assert 0 <= slot < slots and slot not in used, (trial, s, c)
                 used.add(slot)
+
+
+def test_backward_binding_refuses_host_tensors():
+    """The Python entry point of the reverse mode takes device tensors only and
+    refuses host ones before any library call (no CPU fallback)."""
+    import torch
+    T, H, dk, dv = 8, 2, 64, 64
+    q = torch.zeros(T, H, dk, dtype=torch.bfloat16)
+    a = torch.zeros(T, H)
+    v = torch.zeros(T, H, dv, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        lla.gdn_chunk_bwd(q, q, v, a, a, v)

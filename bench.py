@@ -17,8 +17,8 @@ Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
 the workload (weak scaling, no collective on the data path); the timed region
 is bracketed by a barrier + synchronize and the time is the max over ranks.
 
---impl reference times the CPU oracle (rank 0 only) on a bounded sample of
-the same workload.
+--impl reference times the CPU oracle (rank 0 only) on the same workload:
+every step is the whole 4096-token sequence through all 4 loops.
 """
 from __future__ import annotations
 
@@ -330,7 +330,13 @@ def run_ours(args, rank, world, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)
-        if "backward" in extras:   # the reverse mode's oracle, beside its GPU figure
+        # each workload's oracle beside its GPU figure
+        for name in ("long_prefill", "varlen"):
+            if name in extras:
+                extras[name]["cpu_baseline"] = cpu_baseline_prefill(name)
+        if "decode" in extras:
+            extras["decode"]["cpu_baseline"] = cpu_baseline_decode()
+        if "backward" in extras:
             extras["backward"]["cpu_baseline"] = cpu_baseline_backward()
 
     line = {
@@ -597,16 +603,78 @@ def cpu_baseline_backward(seconds_target: float = 3.0, sample_tokens: int = 256)
                                         f"{runs} run(s), {el:.1f} s; fp64 C oracle (OpenMP)"}
 
 
+def cpu_baseline_prefill(name: str, seconds_target: float = 4.0):
+    """The oracle on a sample of a prefill workload: one whole sequence (every
+    head) of the long-prefill workload, or the varlen sequence of median
+    length, one loop, repeated for about `seconds_target` seconds on this
+    host's cores; scaled to the workload's T loops (T calls over the same
+    inputs), so the figure reads like the GPU's tokens/s."""
+    import dataclasses
+    import numpy as np
+    import oracle
+    from looped_linear_attention_b200 import workloads as W
+    wl = W.WORKLOADS[name]
+    if wl.varlen:
+        lens = W.varlen_lengths(wl)
+        s = int(np.argsort(lens)[len(lens) // 2])
+        L = int(lens[s])
+        inp = W.prefill_inputs(dataclasses.replace(wl, name=wl.name), "cpu", lengths=[L])
+        what = f"sequence {s} of {wl.n_seq} (median length {L}), all {wl.H} heads, dv = {wl.dv}"
+    else:
+        L = wl.seq_len
+        inp = W.prefill_inputs(wl, "cpu", n_seq=1)
+        what = f"sequence 0 of {wl.n_seq} ({L} tokens), all {wl.H} heads"
+    cu = np.array([0, L], dtype=np.int32)
+    t0 = time.perf_counter()
+    runs = 0
+    while True:
+        oracle.gdn_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S0"], cu)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el > seconds_target or runs >= 20:
+            break
+    per_loop = el / runs
+    return {"value": L / (wl.loops * per_loop), "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{what}, one loop, {runs} run(s), {el:.1f} s; scaled to {wl.loops} loops "
+                      f"(tokens / (loops x time per loop)); fp64 C oracle (OpenMP over heads)"}
+
+
+def cpu_baseline_decode(seconds_target: float = 4.0, n_slots: int = 256):
+    """The oracle's decode step on `n_slots` of the decode workload's 24576
+    slots (all 16 heads), repeated for about `seconds_target` seconds; scaled to
+    the whole step (all slots) as sequence-tokens/s and state GB/s."""
+    import oracle
+    from looped_linear_attention_b200 import workloads as W
+    wl = W.WORKLOADS["decode"]
+    inp = W.decode_inputs(wl, "cpu", n_slots=n_slots)
+    t0 = time.perf_counter()
+    runs = 0
+    while True:
+        oracle.gdn_decode(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S"])
+        runs += 1
+        el = time.perf_counter() - t0
+        if el > seconds_target or runs >= 50:
+            break
+    step_s = el / runs * wl.n_seq / n_slots
+    nbytes = decode_bytes_per_head_state(wl.dk, wl.dv) * wl.n_seq * wl.H
+    return {"value": 256 / step_s, "unit": "seq-tokens/s", "state_gbs": nbytes / step_s / 1e9,
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n_slots} of {wl.n_seq} slots x {wl.H} heads, {runs} run(s), {el:.1f} s; "
+                      f"scaled to the whole step (x {wl.n_seq // n_slots}); fp64 C oracle (OpenMP)"}
+
+
 def run_reference(args, rank, world):
-    """CPU oracle arm: rank 0 only, bounded samples of the looped-prefill workload."""
+    """CPU oracle arm: rank 0 only; every step is the whole looped-prefill
+    configuration (the 4096-token sequence, all 4 loops), as in cpu_baseline."""
     if rank != 0:
         return
     import oracle
     oracle.build()
     for _ in range(max(0, min(args.warmup, 1))):
-        cpu_baseline(0.0, sample_tokens=256)
+        cpu_baseline(0.0)
     times = []
-    Ls = 512
+    Ls = 4096
     for _ in range(args.steps):
         r = cpu_baseline(0.0, sample_tokens=Ls)
         times.append(Ls / r["value"])
@@ -624,7 +692,8 @@ def run_reference(args, rank, world):
                    "loops": wl.loops, "parallelism": "cpu oracle, rank 0"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
                          "kind": "oracle",
-                         "sample": f"each step: first {Ls} of {wl.seq_len} tokens, all {wl.loops} loops"},
+                         "sample": f"each step: all {Ls} of {wl.seq_len} tokens, all {wl.loops} loops "
+                                   f"(the whole configuration)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -5,6 +5,8 @@
 // commit, loads/stores and the proxy fences that order them, plus bf16 packing.
 #pragma once
 
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -263,5 +265,24 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 }
 
 constexpr float kQkNormEps = 1e-6f;
+
+// ------------------------------------------------------------------ host
+constexpr int kMaxDevices = 64;
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per device (the attribute belongs to the device's context).
+// `done` is the kernel's own per-device flag array; concurrent first calls
+// from several host threads may both set the attribute, which is harmless.
+template <typename Kernel>
+inline cudaError_t smem_attr_once(std::atomic<bool> (&done)[kMaxDevices], Kernel* kernel, size_t bytes) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+  return e;
+}
 
 }  // namespace gdn

@@ -28,7 +28,7 @@ __device__ unsigned g_gdn_device_status = 0;
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+using gdn::kMaxDevices;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -68,6 +68,23 @@ bool dtype_ok(gdn_dtype t) { return t == GDN_F32 || t == GDN_BF16; }
 
 size_t elem_bytes(gdn_dtype t) { return t == GDN_BF16 ? 2 : 4; }
 
+// A device buffer as a byte range; a null pointer overlaps nothing.
+struct Range {
+  const void* ptr;
+  size_t bytes;
+};
+
+template <size_t N>
+bool overlaps_any(const Range& x, const Range (&others)[N]) {
+  const char* x0 = static_cast<const char*>(x.ptr);
+  if (!x0 || x.bytes == 0) return false;
+  for (const Range& r : others) {
+    const char* r0 = static_cast<const char*>(r.ptr);
+    if (r0 && r.bytes && r0 < x0 + x.bytes && x0 < r0 + r.bytes) return true;
+  }
+  return false;
+}
+
 // Shape/pointer checks shared by the workspace query and the launch.
 gdn_status validate_fwd(const gdn_fwd_params* p) {
   if (!p) return GDN_ERR_INVALID;
@@ -95,20 +112,13 @@ gdn_status validate_fwd(const gdn_fwd_params* p) {
     if (a0 < b0 + bytes && b0 < a0 + bytes) return GDN_ERR_INVALID;
   }
   if (any_tokens && p->o) {
-    // the output may not overlap any input
-    const size_t ob = (size_t)p->total_tokens * p->H * p->dv * elem_bytes(p->io_dtype);
-    const char* o0 = reinterpret_cast<const char*>(p->o);
-    struct R { const void* ptr; size_t bytes; } ins[] = {
-        {p->q, (size_t)p->total_tokens * p->H * p->dk * elem_bytes(p->io_dtype)},
-        {p->k, (size_t)p->total_tokens * p->H * p->dk * elem_bytes(p->io_dtype)},
-        {p->v, (size_t)p->total_tokens * p->H * p->dv * elem_bytes(p->io_dtype)},
-        {p->a, (size_t)p->total_tokens * p->H * sizeof(float)},
-        {p->b, (size_t)p->total_tokens * p->H * sizeof(float)},
-    };
-    for (const R& r : ins) {
-      const char* s = reinterpret_cast<const char*>(r.ptr);
-      if (s && s < o0 + ob && o0 < s + r.bytes) return GDN_ERR_INVALID;
-    }
+    // the output may not overlap any input or either state
+    const size_t tok = (size_t)p->total_tokens * p->H, eb = elem_bytes(p->io_dtype);
+    const size_t sb = (size_t)p->n_seq * p->H * p->dk * p->dv * sizeof(float);
+    const Range others[] = {{p->q, tok * p->dk * eb}, {p->k, tok * p->dk * eb},
+                            {p->v, tok * p->dv * eb}, {p->a, tok * sizeof(float)},
+                            {p->b, tok * sizeof(float)}, {p->S0, sb}, {p->S_T, sb}};
+    if (overlaps_any({p->o, tok * p->dv * eb}, others)) return GDN_ERR_INVALID;
   }
   return GDN_OK;
 }
@@ -239,11 +249,11 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
   for (const void* x : ptrs)
     if (!aligned16(x)) return GDN_ERR_INVALID;
   {
-    const size_t ob = (size_t)N * H * dv * elem_bytes(io_dtype);
-    const size_t sb = (size_t)N * H * dk * dv * sizeof(float);
-    const char* o0 = reinterpret_cast<const char*>(o);
-    const char* s0 = reinterpret_cast<const char*>(S);
-    if (o0 < s0 + sb && s0 < o0 + ob) return GDN_ERR_INVALID;
+    // o may not overlap the state or any input (other CTAs still read them)
+    const size_t nh = (size_t)N * H, eb = elem_bytes(io_dtype);
+    const Range others[] = {{S, nh * dk * dv * sizeof(float)}, {q, nh * dk * eb}, {k, nh * dk * eb},
+                            {v, nh * dv * eb}, {a, nh * sizeof(float)}, {b, nh * sizeof(float)}};
+    if (overlaps_any({o, nh * dv * eb}, others)) return GDN_ERR_INVALID;
   }
   const cudaError_t e = gdn::launch_decode(q, k, v, a, b, S, o, N, H, dk, dv, io_dtype, scale, flags,
                                            sm_count(), status_ptr(), stream);

@@ -359,14 +359,9 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
   const long long NH = (long long)N * H;
   if (NH == 0) return cudaSuccess;
   if (dt == GDN_BF16 && dk == dec::DK && dv == dec::DV && status) {
-    static bool attr_set = false;
-    if (!attr_set) {
-      const cudaError_t e = cudaFuncSetAttribute(dec::gdn_decode_stream_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)dec::SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const cudaError_t e = smem_attr_once(attr_set, dec::gdn_decode_stream_kernel, dec::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     const long long blocks = NH < num_sms ? NH : num_sms;
     dec::gdn_decode_stream_kernel<<<(unsigned)blocks, dec::THREADS, dec::SMEM_BYTES, stream>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a, b, S,

@@ -15,7 +15,7 @@ namespace {
 constexpr size_t kNoallocScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
+using gdn::kMaxDevices;
 
 // Device address of g_noalloc_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once

@@ -228,14 +228,10 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_simt_kernel(const Para
 
 template <int DK, typename T>
 static cudaError_t launch_t(const Params& kp, long long blocks, cudaStream_t stream) {
-  static bool attr_set = false;
+  static std::atomic<bool> attr_set[kMaxDevices];
   const size_t bytes = Plan<DK>::BYTES;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gdn_prefill_simt_kernel<DK, T>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = smem_attr_once(attr_set, gdn_prefill_simt_kernel<DK, T>, bytes);
+  if (e != cudaSuccess) return e;
   gdn_prefill_simt_kernel<DK, T><<<(unsigned)blocks, THREADS, bytes, stream>>>(kp);
   return cudaGetLastError();
 }

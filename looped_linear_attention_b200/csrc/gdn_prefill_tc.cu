@@ -1463,13 +1463,9 @@ static gdn_status tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const 
 
 gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const SegPlan& plan, void* ws,
                              cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(tc::gdn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::SMEM_BYTES) != cudaSuccess)
-      return GDN_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_set[kMaxDevices];
+  if (smem_attr_once(attr_set, tc::gdn_prefill_tc_kernel, tc::SMEM_BYTES) != cudaSuccess)
+    return GDN_ERR_CUDA;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, p->q, p->dk, p->H, p->total_tokens) ||
       !make_map(&mk, p->k, p->dk, p->H, p->total_tokens) ||
@@ -1527,13 +1523,9 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   if (P > 2) {
     const long long cblocks = chains * (p->dv / tc::CMB_COLS);
     if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
-    static bool cmb_attr_set = false;
-    if (!cmb_attr_set) {
-      if (cudaFuncSetAttribute(tc::gdn_segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)tc::CMB_SMEM) != cudaSuccess)
-        return GDN_ERR_CUDA;
-      cmb_attr_set = true;
-    }
+    static std::atomic<bool> cmb_attr_set[kMaxDevices];
+    if (smem_attr_once(cmb_attr_set, tc::gdn_segment_combine_kernel, tc::CMB_SMEM) != cudaSuccess)
+      return GDN_ERR_CUDA;
     LaunchCfg lc((unsigned)cblocks, 256, tc::CMB_SMEM, stream, /*dependent=*/true);
     if (cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_combine_kernel, (const float*)kp.Bws,
                            (const float*)kp.Mws, kp.Sst, p->H, p->dv, P) != cudaSuccess)

@@ -75,6 +75,8 @@ def _params(**kw):
     (dict(q=0), B.GDN_ERR_INVALID),                      # null input with tokens
     (dict(S0=1 << 20, S_T=(1 << 20) + 64), B.GDN_ERR_INVALID),   # partial state overlap
     (dict(o=16), B.GDN_ERR_INVALID),                     # output overlaps q
+    (dict(S0=(1 << 28) + 4096), B.GDN_ERR_INVALID),      # output overlaps S0
+    (dict(S_T=(1 << 28) - 4096), B.GDN_ERR_INVALID),     # output overlaps S_T
 ])
 def test_prefill_rejects_bad_arguments_on_host(lib, bad, expect):
     p = _params(**bad)
@@ -195,6 +197,9 @@ def test_python_workspace_query_matches_c(lib):
     (dict(flags=B.GDN_PRECISE), B.GDN_ERR_INVALID),
     (dict(q=8), B.GDN_ERR_INVALID),
     (dict(o=1 << 20), B.GDN_ERR_INVALID),                # output inside the state
+    (dict(o=16), B.GDN_ERR_INVALID),                     # output over q
+    (dict(o=1 << 24, v=(1 << 24) + 512), B.GDN_ERR_INVALID),   # output over v
+    (dict(o=1 << 24, a=(1 << 24) + 16), B.GDN_ERR_INVALID),    # output over a
 ])
 def test_decode_rejects_bad_arguments_on_host(lib, args, expect):
     base = dict(q=16, k=32, v=48, a=64, b=80, S=1 << 20, o=1 << 30, N=4, H=2, dk=128, dv=128,

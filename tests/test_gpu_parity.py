@@ -16,7 +16,8 @@ import torch
 import oracle
 import looped_linear_attention_b200 as lla
 from looped_linear_attention_b200 import workloads as W
-from gpu_util import TOL_BF16_O, TOL_BF16_S, TOL_F32, bf16_ulp, host, rel_l2
+from gpu_util import (TOL_BF16_O, TOL_BF16_S, TOL_F32, bf16_ulp, check_prefill, host, rel_l2,
+                      seq_bounds)
 
 pytestmark = pytest.mark.gpu
 
@@ -67,13 +68,11 @@ def _oracle_prefill(inp, scale=1.0, normalize=False, S0="inp"):
     return oracle.gdn_fwd(q, k, inp["v"], inp["a"], inp["b"], s0, cu, scale)
 
 
-def _check(o, ST, o_ref, S_ref, fp32):
-    eo, es = rel_l2(o, o_ref), rel_l2(ST, S_ref)
-    if fp32:
-        assert eo < TOL_F32 and es < TOL_F32, (eo, es)
-    else:
-        assert eo < TOL_BF16_O and es < TOL_BF16_S, (eo, es)
-    return eo, es
+def _check(o, ST, o_ref, S_ref, fp32, inp=None, bounds=None):
+    """Whole-tensor, per-sequence and worst-chunk bars (gpu_util.check_prefill)."""
+    if bounds is None:
+        bounds = seq_bounds(inp)
+    return check_prefill(o, ST, o_ref, S_ref, bounds, fp32)
 
 
 # ------------------------------------------------------------------ residual
@@ -135,7 +134,7 @@ def test_prefill_tiny_workload_fp32():
     inp = W.prefill_inputs(W.WORKLOADS["tiny"], "cpu")
     o, ST = _gpu_prefill(inp)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o, ST, o_ref, S_ref, fp32=True)
+    _check(o, ST, o_ref, S_ref, fp32=True, inp=inp)
     _status_ok()
 
 
@@ -147,7 +146,7 @@ def test_prefill_precise_varlen_edges(dk, dv):
     inp = W.prefill_inputs(wl, "cpu", lengths=[0, 1, 63, 64, 65, 200])
     o, ST = _gpu_prefill(inp, scale=0.5, flags=lla.GDN_QK_L2NORM)
     o_ref, S_ref = _oracle_prefill(inp, scale=0.5, normalize=True)
-    _check(o, ST, o_ref, S_ref, fp32=True)
+    _check(o, ST, o_ref, S_ref, fp32=True, inp=inp)
     np.testing.assert_allclose(ST[0].numpy(), inp["S0"][0].numpy(), rtol=0, atol=0)
     _status_ok()
 
@@ -158,7 +157,7 @@ def test_prefill_tc_fixed_length_ragged():
     inp = W.prefill_inputs(wl, "cpu")
     o, ST = _gpu_prefill(inp)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
     _status_ok()
 
 
@@ -180,7 +179,7 @@ def test_prefill_tc_strong_and_mixed_decay():
     inp["a"] = a
     o, ST = _gpu_prefill(inp)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
     _status_ok()
 
 
@@ -196,8 +195,8 @@ def test_prefill_tc_segmented_equals_single_pass_and_oracle():
     o_s, S_s = _gpu_prefill(inp)
     o_1, S_1 = _gpu_prefill(inp, flags=lla.GDN_SINGLE_PASS)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o_s, S_s, o_ref, S_ref, fp32=False)
-    _check(o_1, S_1, o_ref, S_ref, fp32=False)
+    _check(o_s, S_s, o_ref, S_ref, fp32=False, inp=inp)
+    _check(o_1, S_1, o_ref, S_ref, fp32=False, inp=inp)
     assert rel_l2(o_s, o_1) < TOL_BF16_O and rel_l2(S_s, S_1) < TOL_BF16_S
     _status_ok()
 
@@ -211,7 +210,7 @@ def test_prefill_tc_segmented_dv256_l2norm_scale():
     inp = W.prefill_inputs(wl, "cpu")
     o, ST = _gpu_prefill(inp, scale=0.125, flags=lla.GDN_QK_L2NORM)
     o_ref, S_ref = _oracle_prefill(inp, scale=0.125, normalize=True)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
     _status_ok()
 
 
@@ -226,7 +225,7 @@ def test_prefill_tc_segmented_strong_decay_in_place():
     inp["a"] = a
     o, ST = _gpu_prefill(inp, alias=True)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
     _status_ok()
 
 
@@ -245,7 +244,7 @@ def test_bounded_wait_runs_out_and_context_stays_usable():
     assert lla.gdn_get_device_status() == lla.GDN_OK          # reading clears the word
     o, ST = _gpu_prefill(inp)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
     _status_ok()
 
 
@@ -254,7 +253,7 @@ def test_prefill_tc_zero_initial_state():
     inp = W.prefill_inputs(wl, "cpu")
     o, ST = _gpu_prefill(inp)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
 
 
 def test_prefill_tc_varlen_dv256_l2norm():
@@ -262,7 +261,7 @@ def test_prefill_tc_varlen_dv256_l2norm():
     inp = W.prefill_inputs(wl, "cpu", lengths=[0, 1, 63, 64, 65, 129, 700])
     o, ST = _gpu_prefill(inp, scale=0.125, flags=lla.GDN_QK_L2NORM)
     o_ref, S_ref = _oracle_prefill(inp, scale=0.125, normalize=True)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
     np.testing.assert_array_equal(ST[0].numpy(), inp["S0"][0].numpy())
     _status_ok()
 
@@ -292,7 +291,7 @@ def test_varlen_longest_first_order_matches_natural_order():
     _status_ok()
     assert torch.equal(host(o), o_lpt) and torch.equal(host(S_T), S_lpt)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o_lpt, S_lpt, o_ref, S_ref, fp32=False)
+    _check(o_lpt, S_lpt, o_ref, S_ref, fp32=False, inp=inp)
 
 
 def test_varlen_longest_first_in_place_state_and_graph_capture():
@@ -304,7 +303,7 @@ def test_varlen_longest_first_in_place_state_and_graph_capture():
     inp = W.prefill_inputs(wl, "cpu", lengths=lengths)
     o, ST = _gpu_prefill(inp, alias=True)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
     q, k, v, a, b = (inp[n].cuda() for n in ("q", "k", "v", "a", "b"))
     s0 = inp["S0"].cuda()
     cu = torch.from_numpy(inp["cu_seqlens"]).cuda()
@@ -373,7 +372,7 @@ def test_prefill_tc_in_place_state():
     inp = W.prefill_inputs(wl, "cpu")
     o, ST = _gpu_prefill(inp, alias=True)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o, ST, o_ref, S_ref, fp32=False)
+    _check(o, ST, o_ref, S_ref, fp32=False, inp=inp)
 
 
 def test_prefill_tc_matches_precise_path_and_oracle():
@@ -382,7 +381,7 @@ def test_prefill_tc_matches_precise_path_and_oracle():
     o_tc, S_tc = _gpu_prefill(inp)
     o_pr, S_pr = _gpu_prefill(inp, flags=lla.GDN_PRECISE)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(o_tc, S_tc, o_ref, S_ref, fp32=False)
+    _check(o_tc, S_tc, o_ref, S_ref, fp32=False, inp=inp)
     # the fp32 path only sees bf16 rounding of its outputs
     assert rel_l2(o_pr, o_ref) < 4e-3 and rel_l2(S_pr, S_ref) < TOL_F32
 
@@ -408,7 +407,7 @@ def test_prefill_split_and_resume():
     o1, S1 = _gpu_prefill(first)
     o2, S2 = _gpu_prefill(second, S0=S1)
     o_ref, S_ref = _oracle_prefill(inp)
-    _check(torch.cat([o1, o2]), S2, o_ref, S_ref, fp32=False)
+    _check(torch.cat([o1, o2]), S2, o_ref, S_ref, fp32=False, inp=inp)
 
 
 def test_decode_continues_prefill():
@@ -439,7 +438,8 @@ def _sample_chain_check(inp, o, ST, chains):
         o_ref, S_ref = oracle.gdn_fwd(host(inp["q"][sl, h:h + 1]), host(inp["k"][sl, h:h + 1]),
                                       host(inp["v"][sl, h:h + 1]), host(inp["a"][sl, h:h + 1]),
                                       host(inp["b"][sl, h:h + 1]), s0)
-        _check(host(o[sl, h:h + 1]), host(ST[s:s + 1, h:h + 1]), o_ref, S_ref, fp32=False)
+        _check(host(o[sl, h:h + 1]), host(ST[s:s + 1, h:h + 1]), o_ref, S_ref, fp32=False,
+               bounds=[(0, t1 - t0)])
 
 
 def test_full_long_prefill_sampled():

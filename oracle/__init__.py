@@ -94,12 +94,28 @@ def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
 
-def gdn_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, scale: float = 1.0):
+def sigmoid(z):
+    """1 / (1 + e^-z) in float64, computed from e^-|z| so that no step overflows."""
+    z = _f64(z)
+    e = np.exp(-np.abs(z))
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def output_gate(o, gate):
+    """Head-wise sigmoid output gate ("LT2: Linear-Time Looped Transformers",
+    §3, the gated-attention paragraph: a head-specific sigmoid gate after the
+    mixer).  o [n_tok, H, dv] times sigmoid(gate) [n_tok, H], one factor per
+    token and head; the recurrence's state is not touched."""
+    return _f64(o) * sigmoid(gate)[..., None]
+
+
+def gdn_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, scale: float = 1.0, gate=None):
     """Gated delta rule over packed sequences.
 
     q, k: [n_tok, H, dk]; v: [n_tok, H, dv]; a, b: [n_tok, H];
     S0: [n_seq, H, dk, dv] or None (zeros); cu_seqlens: int [n_seq+1] or None
-    (one sequence of n_tok tokens).  Returns (o [n_tok, H, dv], S_T [n_seq, H, dk, dv]).
+    (one sequence of n_tok tokens); gate: [n_tok, H] logits of the head-wise
+    output gate, or None.  Returns (o [n_tok, H, dv], S_T [n_seq, H, dk, dv]).
     """
     q, k, v, a, b = (_f64(t) for t in (q, k, v, a, b))
     n_tok, H, dk = q.shape
@@ -122,6 +138,8 @@ def gdn_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, scale: float = 1.0):
         _ptr(cu, ctypes.c_int32), n_seq, H, dk, dv, float(scale))
     if rc != 0:
         raise ValueError("oracle_gdn_fwd rejected its arguments")
+    if gate is not None:
+        o = output_gate(o, gate)
     return o, ST
 
 
@@ -157,9 +175,10 @@ def gdn_bwd(q, k, v, a, b, dO, S0=None, dST=None, cu_seqlens=None, scale: float 
     return out
 
 
-def gdn_decode(q, k, v, a, b, S, scale: float = 1.0):
+def gdn_decode(q, k, v, a, b, S, scale: float = 1.0, gate=None):
     """One token per slot.  q, k: [N, H, dk]; v: [N, H, dv]; a, b: [N, H];
-    S: [N, H, dk, dv].  Returns (o [N, H, dv], S_new); the input is not modified."""
+    S: [N, H, dk, dv]; gate: [N, H] output-gate logits or None.
+    Returns (o [N, H, dv], S_new); the input is not modified."""
     q, k, v, a, b = (_f64(t) for t in (q, k, v, a, b))
     S = _f64(S).copy()
     N, H, dk = q.shape
@@ -169,6 +188,8 @@ def gdn_decode(q, k, v, a, b, S, scale: float = 1.0):
                                    _ptr(S), _ptr(o), N, H, dk, dv, float(scale))
     if rc != 0:
         raise ValueError("oracle_gdn_decode rejected its arguments")
+    if gate is not None:
+        o = output_gate(o, gate)
     return o, S
 
 
@@ -197,13 +218,15 @@ def round_bf16(x) -> np.ndarray:
 
 
 def looped_forward(h0, Wq, Wk, Wv, a, b, rho, H: int, dk: int, dv: int,
-                   scale: float = 1.0, return_all: bool = False):
+                   scale: float = 1.0, return_all: bool = False, Wg=None):
     """T loops of the looped-prefill workload on one sequence.
 
     Per loop tau ("LT2: Linear-Time Looped Transformers", §2, "LT2." paragraph):
     q, k, v = h^(tau-1) W_{q,k,v} (rounded to bf16, the workload's tensor type);
     q, k L2-normalised per head; o = GDN(q, k, v, a_tau, b_tau) from a zero
-    state; h~^(tau) = o as [L, H*dv] (rounded to bf16);
+    state; with the gated variant (§3, gated-attention paragraph) o is scaled
+    per head by sigmoid(h^(tau-1) W_g), W_g [d, H], the logits taken in fp32
+    from the bf16 state; h~^(tau) = o as [L, H*dv] (rounded to bf16);
     h^(tau) = h~^(tau) + rho_tau (.) h^(tau-1) (rounded to bf16).
     a, b: [T, L, H]; rho: [T, H*dv].  Returns h^(T) (and every h^(tau) if asked).
     """
@@ -217,7 +240,8 @@ def looped_forward(h0, Wq, Wk, Wv, a, b, rho, H: int, dk: int, dv: int,
         k = round_bf16(h @ Wk).reshape(L, H, dk)
         v = round_bf16(h @ Wv).reshape(L, H, dv)
         q, k = qk_l2norm(q), qk_l2norm(k)
-        o, _ = gdn_fwd(q, k, v, a[tau], b[tau], None, None, scale)
+        z = None if Wg is None else (h @ _f64(Wg)).astype(np.float32).astype(np.float64)
+        o, _ = gdn_fwd(q, k, v, a[tau], b[tau], None, None, scale, gate=z)
         h_tilde = round_bf16(o.reshape(L, H * dv))
         h = round_bf16(loop_residual(h_tilde, h, rho[tau]))
         outs.append(h)

@@ -360,3 +360,52 @@ def test_segment_state_update_is_affine_in_its_start_state(seed):
         _, Mp = oracle.gdn_fwd(q[sl], k[sl], np.zeros((hi - lo, H, dk)), a[sl], b[sl], eye)
         S = np.einsum("hij,hjk->hik", Mp[0], S) + Bp[0]
     np.testing.assert_allclose(S, S_direct[0], rtol=1e-11, atol=1e-11)
+
+
+# ------------------------------------------------------------ output gate
+def test_output_gate_closed_forms():
+    """Head-wise sigmoid output gate (§3, gated-attention paragraph): sigmoid of
+    ln 3 is exactly 3/4 and of -ln 3 exactly 1/4 (a sign slip swaps them), a
+    logit of 0 halves the output, a large logit leaves it as it is, and the
+    factor belongs to its own (token, head) (a transposed index moves the
+    3/4 to another head).  The state is never gated."""
+    rng = np.random.default_rng(15)
+    L, H, dk, dv = 9, 3, 4, 5
+    q, k, v, a, b = _rand_case(rng, L, H, dk, dv)
+    S0 = rng.standard_normal((1, H, dk, dv))
+    o, S = oracle.gdn_fwd(q, k, v, a, b, S0)
+    z = np.zeros((L, H))
+    z[:, 0] = np.log(3.0)
+    z[:, 1] = -np.log(3.0)
+    z[::2, 2] = 60.0
+    og, Sg = oracle.gdn_fwd(q, k, v, a, b, S0, gate=z)
+    np.testing.assert_array_equal(Sg, S)
+    np.testing.assert_allclose(og[:, 0], 0.75 * o[:, 0], rtol=1e-15)
+    np.testing.assert_allclose(og[:, 1], 0.25 * o[:, 1], rtol=1e-15)
+    np.testing.assert_allclose(og[::2, 2], o[::2, 2], rtol=1e-15)
+    np.testing.assert_array_equal(og[1::2, 2], 0.5 * o[1::2, 2])
+    np.testing.assert_allclose(oracle.sigmoid(np.array([-800.0, 800.0])), [0.0, 1.0], atol=0)
+    # the same factor in decode
+    od, _ = oracle.gdn_decode(q[:1], k[:1], v[:1], a[:1], b[:1], S0, gate=z[:1])
+    o1, _ = oracle.gdn_decode(q[:1], k[:1], v[:1], a[:1], b[:1], S0)
+    np.testing.assert_allclose(od[0, 0], 0.75 * o1[0, 0], rtol=1e-15)
+
+
+def test_looped_forward_gate_single_token():
+    """One token, W = I, a = b = 1, rho = 0 and the gate weights W_g chosen so
+    that head h's logit is ln 3 (head 0) or 0 (head 1): the read-back value
+    (||h||^2 / (||h||^2 + eps)) h of each head is scaled by 3/4 and by 1/2."""
+    H, dk = 2, 4
+    d = H * dk
+    h0 = oracle.round_bf16(np.array([[1.0, -2.0, 0.5, 3.0, 0.25, 1.5, -1.0, 2.0]]))
+    Wg = np.zeros((d, H))
+    Wg[0, 0] = np.log(3.0) / h0[0, 0]        # logit of head 0: h0[0] * Wg[0, 0]
+    a = np.ones((1, 1, H))
+    b = np.ones((1, 1, H))
+    out = oracle.looped_forward(h0, np.eye(d), np.eye(d), np.eye(d), a, b, np.zeros((1, d)),
+                                H, dk, dk, Wg=Wg)
+    hh = h0.reshape(H, dk)
+    n2 = (hh * hh).sum(-1, keepdims=True)
+    z = np.array([[float(np.float32(np.log(3.0)))], [0.0]])
+    expect = oracle.round_bf16((oracle.sigmoid(z) * n2 / (n2 + 1e-6) * hh).reshape(1, d))
+    np.testing.assert_array_equal(out, expect)

@@ -16,6 +16,13 @@ oracle at the usual bars (relative L2 1e-2 on bf16 outputs, 5e-3 on states,
     I - k k^T with b = 1 on raw keys);
   * a chain of 128 Householder reflections (random unit keys, b = 2) that
     realises a random orthogonal map of a 128 x 128 state.
+The exact-reflection chains (a = 1 throughout, every chunk a full rotation of
+the state) are the one regime where the bf16 operands of the tensor-core path
+(the state, W, U and T, each rounded once per chunk) add up past the 5e-3
+state bar: about 6.3e-3 after one to five chunks, reproduced by a CPU
+emulation of those roundings.  There the fp32 chunk kernel (GDN_PRECISE) is
+the path that meets the bars; the tensor-core error is still checked, against
+1e-2, as a regression guard and not as a parity claim.
 """
 import dataclasses
 
@@ -193,12 +200,21 @@ def test_transposition_chain_permutes_state_rows(normalised):
                a=torch.ones(L, H), b=torch.full((L, H), 2.0 if normalised else 1.0), S0=S0,
                cu_seqlens=None, n_seq=1, seq_len=L, total_tokens=L)
     flags = lla.GDN_QK_L2NORM if normalised else 0
-    o, ST = _run(inp, flags=flags)
     o_ref, S_ref = _ref(inp, normalize=normalised)
     perm = _permuted(S0[0].numpy().astype(np.float64), pairs)
     # the oracle realises the permutation (up to the norm's eps with the flag)
     assert rel_l2(S_ref[0], perm) < (1e-4 if normalised else 1e-12)
-    check_prefill(o, ST, o_ref, S_ref, [(0, L)], fp32=False)
+    _exact_reflection_checks(inp, flags, o_ref, S_ref, L)
+
+
+def _exact_reflection_checks(inp, flags, o_ref, S_ref, L):
+    """GDN_PRECISE meets the bars (fp32 state error, bf16 output rounding);
+    the tensor-core path stays within its measured envelope."""
+    o, ST = _run(inp, flags=flags | lla.GDN_PRECISE)
+    err = check_prefill(o, ST, o_ref, S_ref, [(0, L)], fp32=False)
+    assert err["S"] < TOL_F32, err
+    o, ST = _run(inp, flags=flags)
+    assert rel_l2(o, o_ref) < TOL_BF16_O and rel_l2(ST, S_ref) < 2 * TOL_BF16_S
 
 
 def test_householder_chain_realises_orthogonal_map():
@@ -214,7 +230,6 @@ def test_householder_chain_realises_orthogonal_map():
     S0 = torch.randn(1, H, n, n, generator=g)
     inp = dict(q=q, k=k, v=torch.zeros(L, H, n, dtype=torch.bfloat16), a=torch.ones(L, H),
                b=torch.full((L, H), 2.0), S0=S0, cu_seqlens=None, n_seq=1, seq_len=L, total_tokens=L)
-    o, ST = _run(inp)
     o_ref, S_ref = _ref(inp)
     kd = k.double().numpy()
     for h in range(H):
@@ -222,4 +237,4 @@ def test_householder_chain_realises_orthogonal_map():
         for t in range(L):
             P = (np.eye(n) - 2.0 * np.outer(kd[t, h], kd[t, h])) @ P
         np.testing.assert_allclose(S_ref[0, h], P @ S0[0, h].double().numpy(), atol=1e-10)
-    check_prefill(o, ST, o_ref, S_ref, [(0, L)], fp32=False)
+    _exact_reflection_checks(inp, 0, o_ref, S_ref, L)

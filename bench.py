@@ -213,10 +213,11 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 # ------------------------------------------------------------------ byte / flop accounting
-def prefill_bytes_per_token_head(dk, dv, io_bytes=2):
+def prefill_bytes_per_token_head(dk, dv, io_bytes=2, residual=False):
     """Algorithmic HBM bytes of one token of one head in one prefill launch:
-    q, k (dk each), v and o (dv each) in the io dtype, a and b in fp32."""
-    return io_bytes * (2 * dk + 2 * dv) + 8
+    q, k (dk each), v and o (dv each) in the io dtype, a and b in fp32; with the
+    loop residual fused into the output, also h_prev (dv, io dtype)."""
+    return io_bytes * (2 * dk + 2 * dv + (dv if residual else 0)) + 8
 
 
 def prefill_state_bytes(n_seq, H, dk, dv, s0, st):
@@ -296,14 +297,14 @@ def run_ours(args, rank, world, local):
     value = world * tokens_per_step * args.steps / total_s
     gdn_ms = [a.elapsed_time(b) for a, b in gdn_events]
     gdn_avg_s = statistics.mean(gdn_ms) / 1e3
-    gdn_bytes = prefill_bytes_per_token_head(wl.dk, wl.dv) * L * wl.H
+    gdn_bytes = prefill_bytes_per_token_head(wl.dk, wl.dv, residual=runner.fused_residual) * L * wl.H
     achieved = gdn_bytes / gdn_avg_s / 1e9
     hbm_peak = peaks["hbm_gbs"]
     # this library's kernels per loop: the mixer (one launch per pass, plus the
     # combine on the segmented schedule) and the loop residual
     sched = lla.prefill_schedule(1, L, wl.H, wl.dk, wl.dv)
     mixer_launches = sched["launches"]
-    launches = args.steps * wl.loops * (mixer_launches + 1)
+    launches = args.steps * wl.loops * runner_g.launches_per_loop()
 
     # ---- end to end through host buffers (pinned), same step
     e2e = run_e2e(args, runner, inp, wl, dev, stream, world)

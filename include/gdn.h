@@ -96,9 +96,23 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
  *              = total_tokens), or NULL: n_seq sequences of seq_len tokens each
  *              (total_tokens = n_seq * seq_len).
  *   scale      multiplies every output (1.0 reproduces the recurrence as written).
+ * Optional epilogue of the looped block, applied to each output in this order
+ * (every pointer NULL = that step off):
+ *   gate       [total_tokens][H] fp32 logits of the head-wise sigmoid output
+ *              gate: o_t,h <- sigmoid(gate_t,h) o_t,h (one factor per token and
+ *              head; "LT2: Linear-Time Looped Transformers", §3, the
+ *              gated-attention paragraph: a head-specific sigmoid gate after the
+ *              mixer).  The state is not gated.
+ *   h_prev, rho  the loop residual of §2 ("LT2." paragraph) fused into the
+ *              output: o <- round(o) + rho (.) h_prev, computed in fp32 and
+ *              rounded to io_dtype (round(o) is the output as it would be
+ *              stored, so the result equals gdn_chunk_fwd followed by
+ *              loop_residual).  h_prev [total_tokens][H*dv] io_dtype (o's
+ *              layout), rho [H*dv] fp32; both or neither.  o may be h_prev
+ *              itself (exact aliasing, for an in-place loop state).
  * Each (sequence, head) chain starts from its S0 and runs the recurrence over its
  * own tokens; a sequence of length 0 writes no output and S_T = S0.
- * o must not overlap q, k, v, a, b, S0 or S_T.
+ * o must not overlap q, k, v, a, b, S0, S_T or gate, nor h_prev other than exactly.
  *
  * Supported: dk in {64, 128}; dv a multiple of 64, at most 512; H >= 1.
  * bf16 with dk = 128 and dv a multiple of 128 runs on the tensor-core (tcgen05)
@@ -116,6 +130,9 @@ typedef struct {
     gdn_dtype io_dtype;
     float scale;
     unsigned flags;
+    const float *gate;       /* optional epilogue, see above */
+    const void *h_prev;
+    const float *rho;
 } gdn_fwd_params;
 
 /* Bytes of device workspace gdn_chunk_fwd needs for these parameters (may be 0).
@@ -254,6 +271,19 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            const float *a, const float *b, float *S, void *o,
                            int N, int H, int dk, int dv, gdn_dtype io_dtype,
                            float scale, unsigned flags, cudaStream_t stream);
+
+/*
+ * gdn_decode_step with the looped block's output epilogue, as in
+ * gdn_fwd_params: gate [N][H] fp32 logits of the head-wise sigmoid output gate
+ * (or NULL), and the loop residual o <- round(o) + rho (.) h_prev with
+ * h_prev [N][H*dv] io_dtype and rho [H*dv] fp32 (both or neither; o may be
+ * h_prev exactly).  With every epilogue pointer NULL it is gdn_decode_step.
+ */
+gdn_status gdn_decode_step_looped(const void *q, const void *k, const void *v,
+                                  const float *a, const float *b, float *S, void *o,
+                                  const float *gate, const void *h_prev, const float *rho,
+                                  int N, int H, int dk, int dv, gdn_dtype io_dtype,
+                                  float scale, unsigned flags, cudaStream_t stream);
 
 /*
  * Loop residual h_out = h_tilde + rho (.) h_prev, computed in fp32 and rounded

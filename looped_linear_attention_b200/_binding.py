@@ -49,6 +49,7 @@ class gdn_fwd_params(ctypes.Structure):
         ("n_seq", ctypes.c_int), ("seq_len", ctypes.c_int), ("total_tokens", ctypes.c_int),
         ("H", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
         ("io_dtype", ctypes.c_int), ("scale", ctypes.c_float), ("flags", ctypes.c_uint),
+        ("gate", ctypes.c_void_p), ("h_prev", ctypes.c_void_p), ("rho", ctypes.c_void_p),
     ]
 
 
@@ -93,6 +94,9 @@ def library() -> ctypes.CDLL:
         lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                         f32, u32, vp]
         lib.gdn_decode_step.restype = i32
+        lib.gdn_decode_step_looped.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                               i32, i32, f32, u32, vp]
+        lib.gdn_decode_step_looped.restype = i32
         lib.loop_residual.argtypes = [vp, vp, vp, vp, ctypes.c_int64, i32, i32, vp]
         lib.loop_residual.restype = i32
         lib.gdn_status_string.argtypes = [i32]
@@ -129,17 +133,33 @@ def _check(t: torch.Tensor, name: str, dtype=None, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _check_epilogue(gate, h_prev, rho, T, H, dv, dtype):
+    if gate is not None:
+        _check(gate, "gate", torch.float32, (T, H))
+    if (h_prev is None) != (rho is None):
+        raise ValueError("h_prev and rho come together (the loop residual)")
+    if h_prev is not None:
+        _check(h_prev, "h_prev", dtype)
+        if h_prev.numel() != T * H * dv:
+            raise ValueError(f"h_prev must hold {T} x {H * dv} elements")
+        _check(rho, "rho", torch.float32, (H * dv,))
+
+
 def gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,
                   b: torch.Tensor, S0: Optional[torch.Tensor] = None,
                   cu_seqlens: Optional[torch.Tensor] = None, *, n_seq: Optional[int] = None,
                   scale: float = 1.0, flags: int = 0, o: Optional[torch.Tensor] = None,
                   S_T: Optional[torch.Tensor] = None, return_state: bool = True,
+                  gate: Optional[torch.Tensor] = None, h_prev: Optional[torch.Tensor] = None,
+                  rho: Optional[torch.Tensor] = None,
                   stream: Optional[torch.cuda.Stream] = None):
     """Chunkwise prefill (see gdn_chunk_fwd in include/gdn.h).
 
     q, k: [T, H, dk]; v: [T, H, dv] (fp32 or bf16); a, b: [T, H] fp32;
     S0: [n_seq, H, dk, dv] fp32 or None; cu_seqlens: int32 [n_seq+1] on the device,
     or None with n_seq sequences of T // n_seq tokens (n_seq defaults to 1).
+    Looped-block epilogue: gate [T, H] fp32 output-gate logits; h_prev (T x H*dv,
+    io dtype) with rho [H*dv] fp32 adds the loop residual (o may be h_prev's storage).
     Returns (o, S_T) (S_T is None when return_state is False)."""
     if q.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {q.dtype}")
@@ -161,17 +181,21 @@ def gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
         seq_len = T // ns
     if S0 is not None:
         _check(S0, "S0", torch.float32, (ns, H, dk, dv))
+    _check_epilogue(gate, h_prev, rho, T, H, dv, q.dtype)
     if o is None:
         o = torch.empty(T, H, dv, dtype=q.dtype, device=q.device)
     else:
-        _check(o, "o", q.dtype, (T, H, dv))
+        _check(o, "o", q.dtype)
+        if o.numel() != T * H * dv:
+            raise ValueError(f"o must hold {T} x {H} x {dv} elements")
     if S_T is None and return_state:
         S_T = torch.empty(ns, H, dk, dv, dtype=torch.float32, device=q.device)
     elif S_T is not None:
         _check(S_T, "S_T", torch.float32, (ns, H, dk, dv))
     p = gdn_fwd_params(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0), _ptr(o),
                        _ptr(S_T), _ptr(cu_seqlens), ns, seq_len, T, H, dk, dv,
-                       _DTYPES[q.dtype], float(scale), int(flags))
+                       _DTYPES[q.dtype], float(scale), int(flags), _ptr(gate), _ptr(h_prev),
+                       _ptr(rho))
     lib = library()
     ws = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
     if ws == ctypes.c_size_t(-1).value:
@@ -276,9 +300,11 @@ def prefill_schedule(n_seq: int, seq_len: int, H: int, dk: int, dv: int,
 
 def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,
                     b: torch.Tensor, S: torch.Tensor, *, scale: float = 1.0, flags: int = 0,
-                    o: Optional[torch.Tensor] = None,
+                    o: Optional[torch.Tensor] = None, gate: Optional[torch.Tensor] = None,
+                    h_prev: Optional[torch.Tensor] = None, rho: Optional[torch.Tensor] = None,
                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """One token per slot; S [N, H, dk, dv] fp32 is updated in place. Returns o [N, H, dv]."""
+    """One token per slot; S [N, H, dk, dv] fp32 is updated in place. Returns o [N, H, dv].
+    gate / h_prev / rho: the looped-block epilogue (gdn_decode_step_looped)."""
     if q.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {q.dtype}")
     N, H, dk = q.shape
@@ -289,13 +315,22 @@ def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.
     _check(a, "a", torch.float32, (N, H))
     _check(b, "b", torch.float32, (N, H))
     _check(S, "S", torch.float32, (N, H, dk, dv))
+    _check_epilogue(gate, h_prev, rho, N, H, dv, q.dtype)
     if o is None:
         o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
     else:
-        _check(o, "o", q.dtype, (N, H, dv))
-    st = library().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S), _ptr(o),
-                                   N, H, dk, dv, _DTYPES[q.dtype], float(scale), int(flags),
-                                   _stream_ptr(stream))
+        _check(o, "o", q.dtype)
+        if o.numel() != N * H * dv:
+            raise ValueError(f"o must hold {N} x {H} x {dv} elements")
+    if gate is None and h_prev is None:
+        st = library().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S), _ptr(o),
+                                       N, H, dk, dv, _DTYPES[q.dtype], float(scale), int(flags),
+                                       _stream_ptr(stream))
+    else:
+        st = library().gdn_decode_step_looped(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S),
+                                              _ptr(o), _ptr(gate), _ptr(h_prev), _ptr(rho), N, H, dk,
+                                              dv, _DTYPES[q.dtype], float(scale), int(flags),
+                                              _stream_ptr(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_decode_step")
     return o

@@ -13,9 +13,9 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
                              cudaStream_t stream);
 gdn_status launch_prefill_simt(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
-                          const float* b, float* S, void* o, int N, int H, int dk, int dv,
-                          gdn_dtype dt, float scale, unsigned flags, int num_sms, unsigned* status,
-                          cudaStream_t stream);
+                          const float* b, float* S, void* o, const float* gate, const void* h_prev,
+                          const float* rho, int N, int H, int dk, int dv, gdn_dtype dt, float scale,
+                          unsigned flags, int num_sms, unsigned* status, cudaStream_t stream);
 cudaError_t launch_loop_residual(const void* h_tilde, const void* h_prev, const float* rho,
                                  void* h_out, int64_t rows, int d, gdn_dtype dt, int num_sms,
                                  cudaStream_t stream);
@@ -101,9 +101,11 @@ gdn_status validate_fwd(const gdn_fwd_params* p) {
   if (p->dv % 64 != 0 || p->dv > 512) return GDN_ERR_UNSUPPORTED;
   const bool any_tokens = p->total_tokens > 0;
   if (any_tokens && (!p->q || !p->k || !p->v || !p->a || !p->b || !p->o)) return GDN_ERR_INVALID;
-  const void* ptrs[] = {p->q, p->k, p->v, p->a, p->b, p->S0, p->o, p->S_T, p->cu_seqlens};
+  const void* ptrs[] = {p->q, p->k, p->v, p->a, p->b, p->S0, p->o, p->S_T, p->cu_seqlens,
+                        p->gate, p->h_prev, p->rho};
   for (const void* q : ptrs)
     if (q && !aligned16(q)) return GDN_ERR_INVALID;
+  if ((p->h_prev == nullptr) != (p->rho == nullptr)) return GDN_ERR_INVALID;
   if (p->S_T && p->S0 && p->S_T != p->S0) {
     // partial overlap of S0 and S_T is not allowed (exact aliasing is)
     const size_t bytes = (size_t)p->n_seq * p->H * p->dk * p->dv * sizeof(float);
@@ -117,7 +119,9 @@ gdn_status validate_fwd(const gdn_fwd_params* p) {
     const size_t sb = (size_t)p->n_seq * p->H * p->dk * p->dv * sizeof(float);
     const Range others[] = {{p->q, tok * p->dk * eb}, {p->k, tok * p->dk * eb},
                             {p->v, tok * p->dv * eb}, {p->a, tok * sizeof(float)},
-                            {p->b, tok * sizeof(float)}, {p->S0, sb}, {p->S_T, sb}};
+                            {p->b, tok * sizeof(float)}, {p->S0, sb}, {p->S_T, sb},
+                            {p->gate, tok * sizeof(float)}, {p->rho, (size_t)p->H * p->dv * sizeof(float)},
+                            {p->h_prev == p->o ? nullptr : p->h_prev, tok * p->dv * eb}};
     if (overlaps_any({p->o, tok * p->dv * eb}, others)) return GDN_ERR_INVALID;
   }
   return GDN_OK;
@@ -239,24 +243,39 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
                            const float* b, float* S, void* o, int N, int H, int dk, int dv,
                            gdn_dtype io_dtype, float scale, unsigned flags,
                            cudaStream_t stream) {
+  return gdn_decode_step_looped(q, k, v, a, b, S, o, nullptr, nullptr, nullptr, N, H, dk, dv, io_dtype,
+                                scale, flags, stream);
+}
+
+gdn_status gdn_decode_step_looped(const void* q, const void* k, const void* v, const float* a,
+                                  const float* b, float* S, void* o, const float* gate,
+                                  const void* h_prev, const float* rho, int N, int H, int dk, int dv,
+                                  gdn_dtype io_dtype, float scale, unsigned flags, cudaStream_t stream) {
   if (!dtype_ok(io_dtype) || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return GDN_ERR_INVALID;
   if (flags & ~GDN_QK_L2NORM) return GDN_ERR_INVALID;
   if (dk != 64 && dk != 128) return GDN_ERR_UNSUPPORTED;
   if (dv % 64 != 0 || dv > 512) return GDN_ERR_UNSUPPORTED;
   if (N == 0) return GDN_OK;
   if (!q || !k || !v || !a || !b || !S || !o) return GDN_ERR_INVALID;
+  if ((h_prev == nullptr) != (rho == nullptr)) return GDN_ERR_INVALID;
   const void* ptrs[] = {q, k, v, a, b, S, o};
   for (const void* x : ptrs)
     if (!aligned16(x)) return GDN_ERR_INVALID;
+  const void* opt[] = {gate, h_prev, rho};
+  for (const void* x : opt)
+    if (x && !aligned16(x)) return GDN_ERR_INVALID;
   {
-    // o may not overlap the state or any input (other CTAs still read them)
+    // o may not overlap the state or any input (other CTAs still read them);
+    // h_prev may be o itself (each element is read and then written by one thread)
     const size_t nh = (size_t)N * H, eb = elem_bytes(io_dtype);
     const Range others[] = {{S, nh * dk * dv * sizeof(float)}, {q, nh * dk * eb}, {k, nh * dk * eb},
-                            {v, nh * dv * eb}, {a, nh * sizeof(float)}, {b, nh * sizeof(float)}};
+                            {v, nh * dv * eb}, {a, nh * sizeof(float)}, {b, nh * sizeof(float)},
+                            {gate, nh * sizeof(float)}, {rho, (size_t)H * dv * sizeof(float)},
+                            {h_prev == o ? nullptr : h_prev, nh * dv * eb}};
     if (overlaps_any({o, nh * dv * eb}, others)) return GDN_ERR_INVALID;
   }
-  const cudaError_t e = gdn::launch_decode(q, k, v, a, b, S, o, N, H, dk, dv, io_dtype, scale, flags,
-                                           sm_count(), status_ptr(), stream);
+  const cudaError_t e = gdn::launch_decode(q, k, v, a, b, S, o, gate, h_prev, rho, N, H, dk, dv, io_dtype,
+                                           scale, flags, sm_count(), status_ptr(), stream);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -18,7 +18,9 @@
 //     head, dv block of 32*VEC columns), 128-bit accesses coalesced along dv,
 //     the state held in registers between the read and the write; lane l owns
 //     VEC consecutive columns and warp w owns DK/8 rows.
-// In both, the dk reductions go through shared memory.
+// In both, the dk reductions go through shared memory.  Optionally the output
+// takes the looped block's epilogue (include/gdn.h, gdn_decode_step_looped):
+// the head-wise sigmoid gate, then the loop residual o <- round(o) + rho (.) h_prev.
 #include "common.cuh"
 
 namespace gdn {
@@ -36,11 +38,31 @@ __device__ __forceinline__ float2 ld_f2_stream(const float* p) {
   return r;
 }
 
+// Output epilogue of the looped block for one output element: the gate factor
+// og (1 without a gate), then, with the residual, round to the io dtype and add
+// rho (.) h_prev in fp32.
+struct Epilogue {
+  const float* gate;    // [slots][H] logits, or null
+  const void* h_prev;   // [slots][H*dv] io dtype, or null
+  const float* rho;     // [H*dv]
+  int H;
+};
+__device__ __forceinline__ float gate_factor(const Epilogue& ep, long long sh) {
+  return ep.gate ? 1.f / (1.f + __expf(-__ldg(ep.gate + sh))) : 1.f;
+}
+template <typename T>
+__device__ __forceinline__ T epilogue_out(const Epilogue& ep, float y, long long sh, int dv, int col) {
+  if (!ep.h_prev) return from_f32<T>(y);
+  const long long h = sh % ep.H;
+  const float hp = to_f32(static_cast<const T*>(ep.h_prev)[sh * dv + col]);
+  return from_f32<T>(fmaf(__ldg(ep.rho + h * dv + col), hp, to_f32(from_f32<T>(y))));
+}
+
 template <int DK, int VEC, typename T>
 __global__ void __launch_bounds__(256, 2)
     gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       const float* __restrict__ a, const float* __restrict__ b, float* S, T* o,
-                      int dv, float scale, unsigned flags) {
+                      int dv, float scale, unsigned flags, const Epilogue ep) {
   constexpr int RPW = DK / 8;          // rows per warp
   constexpr int COLS = 32 * VEC;       // columns per CTA
   constexpr int KPL = DK / 32;         // q/k elements per lane for the norms
@@ -130,8 +152,10 @@ __global__ void __launch_bounds__(256, 2)
   for (int c = 0; c < VEC; ++c) u[c] = bb * (to_f32(vp[c]) - aa * xk[c]);
   if (warp == 0) {
     T* op = o + sh * (long long)dv + c0;
+    const float og = gate_factor(ep, sh);
 #pragma unroll
-    for (int c = 0; c < VEC; ++c) op[c] = from_f32<T>(scale * fmaf(aa, xq[c], kqn * u[c]));
+    for (int c = 0; c < VEC; ++c)
+      op[c] = epilogue_out<T>(ep, og * (scale * fmaf(aa, xq[c], kqn * u[c])), sh, dv, c0 + c);
   }
 #pragma unroll
   for (int i = 0; i < RPW; ++i) {
@@ -194,7 +218,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     gdn_decode_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                              const __nv_bfloat16* __restrict__ v, const float* __restrict__ a,
                              const float* __restrict__ b, float* S, __nv_bfloat16* o, long long NH,
-                             float scale, unsigned flags, unsigned* status) {
+                             float scale, unsigned flags, unsigned* status, const Epilogue ep) {
   extern __shared__ __align__(128) uint8_t dsm[];
   uint64_t* full = reinterpret_cast<uint64_t*>(dsm + OFF_BAR);
   float* red = reinterpret_cast<float*>(dsm + OFF_RED);
@@ -296,9 +320,24 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int c = 0; c < 4; ++c) u[c] = bb * (__bfloat162float(sv[4 * lane + c]) - aa * xk[c]);
     if (warp == 0) {
+      float y[4];
+      const float og = gate_factor(ep, sh);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) y[c] = og * (scale * fmaf(aa, xq[c], kqn * u[c]));
       uint2 ov;
-      ov.x = pack_bf16x2(scale * fmaf(aa, xq[0], kqn * u[0]), scale * fmaf(aa, xq[1], kqn * u[1]));
-      ov.y = pack_bf16x2(scale * fmaf(aa, xq[2], kqn * u[2]), scale * fmaf(aa, xq[3], kqn * u[3]));
+      if (ep.h_prev) {
+        const uint2 hp = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(ep.h_prev) +
+                                                         sh * DV + 4 * lane);
+        const float4 r = __ldg(reinterpret_cast<const float4*>(ep.rho + (sh % ep.H) * DV + 4 * lane));
+        // o rounded to bf16 first, as loop_residual would see it
+        ov.x = pack_bf16x2(fmaf(r.x, bf16_lo(hp.x), to_f32(from_f32<__nv_bfloat16>(y[0]))),
+                           fmaf(r.y, bf16_hi(hp.x), to_f32(from_f32<__nv_bfloat16>(y[1]))));
+        ov.y = pack_bf16x2(fmaf(r.z, bf16_lo(hp.y), to_f32(from_f32<__nv_bfloat16>(y[2]))),
+                           fmaf(r.w, bf16_hi(hp.y), to_f32(from_f32<__nv_bfloat16>(y[3]))));
+      } else {
+        ov.x = pack_bf16x2(y[0], y[1]);
+        ov.y = pack_bf16x2(y[2], y[3]);
+      }
       *reinterpret_cast<uint2*>(o + sh * DV + 4 * lane) = ov;
     }
 #pragma unroll
@@ -337,7 +376,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 template <int DK, typename T>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* a,
                                    const float* b, float* S, void* o, long long NH, int dv,
-                                   float scale, unsigned flags, cudaStream_t stream) {
+                                   float scale, unsigned flags, const Epilogue& ep, cudaStream_t stream) {
   const bool wide = (dv % 128) == 0;
   const int cols = wide ? 128 : 64;
   const long long blocks = NH * (dv / cols);
@@ -345,18 +384,19 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, 
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   if (wide)
     gdn_decode_kernel<DK, 4, T><<<(unsigned)blocks, 256, 0, stream>>>(
-        (const T*)q, (const T*)k, (const T*)v, a, b, S, (T*)o, dv, scale, flags);
+        (const T*)q, (const T*)k, (const T*)v, a, b, S, (T*)o, dv, scale, flags, ep);
   else
     gdn_decode_kernel<DK, 2, T><<<(unsigned)blocks, 256, 0, stream>>>(
-        (const T*)q, (const T*)k, (const T*)v, a, b, S, (T*)o, dv, scale, flags);
+        (const T*)q, (const T*)k, (const T*)v, a, b, S, (T*)o, dv, scale, flags, ep);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
-                          const float* b, float* S, void* o, int N, int H, int dk, int dv,
-                          gdn_dtype dt, float scale, unsigned flags, int num_sms, unsigned* status,
-                          cudaStream_t stream) {
+                          const float* b, float* S, void* o, const float* gate, const void* h_prev,
+                          const float* rho, int N, int H, int dk, int dv, gdn_dtype dt, float scale,
+                          unsigned flags, int num_sms, unsigned* status, cudaStream_t stream) {
   const long long NH = (long long)N * H;
+  const Epilogue ep{gate, h_prev, rho, H};
   if (NH == 0) return cudaSuccess;
   if (dt == GDN_BF16 && dk == dec::DK && dv == dec::DV && status) {
     static std::atomic<bool> attr_set[kMaxDevices];
@@ -365,15 +405,15 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
     const long long blocks = NH < num_sms ? NH : num_sms;
     dec::gdn_decode_stream_kernel<<<(unsigned)blocks, dec::THREADS, dec::SMEM_BYTES, stream>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a, b, S,
-        (__nv_bfloat16*)o, NH, scale, flags, status);
+        (__nv_bfloat16*)o, NH, scale, flags, status, ep);
     return cudaGetLastError();
   }
   if (dt == GDN_BF16) {
-    return dk == 128 ? launch_decode_t<128, __nv_bfloat16>(q, k, v, a, b, S, o, NH, dv, scale, flags, stream)
-                     : launch_decode_t<64, __nv_bfloat16>(q, k, v, a, b, S, o, NH, dv, scale, flags, stream);
+    return dk == 128 ? launch_decode_t<128, __nv_bfloat16>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream)
+                     : launch_decode_t<64, __nv_bfloat16>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream);
   }
-  return dk == 128 ? launch_decode_t<128, float>(q, k, v, a, b, S, o, NH, dv, scale, flags, stream)
-                   : launch_decode_t<64, float>(q, k, v, a, b, S, o, NH, dv, scale, flags, stream);
+  return dk == 128 ? launch_decode_t<128, float>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream)
+                   : launch_decode_t<64, float>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream);
 }
 
 }  // namespace gdn

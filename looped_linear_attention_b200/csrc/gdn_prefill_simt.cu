@@ -32,8 +32,8 @@ struct Plan {
   static constexpr int T = A + C * LDC;            // [C][LDC]
   static constexpr int P = T + C * LDC;            // [C][LDC]
   static constexpr int U = P + C * LDC;            // [C][LDC]
-  static constexpr int G = U + C * LDC;            // g, gamma, b: 3 x C
-  static constexpr int FLOATS = G + 3 * C + 4;
+  static constexpr int G = U + C * LDC;            // g, gamma, b, gamma_C / gamma: 4 x C
+  static constexpr int FLOATS = G + 4 * C + 4;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 
@@ -44,6 +44,9 @@ struct Params {
   void* o;
   const int32_t* cu_seqlens;
   unsigned* status;
+  const float* gate;     // [tokens][H] output-gate logits, or null
+  const void* h_prev;    // [tokens][H*dv] loop residual input (io dtype), or null
+  const float* rho;      // [H*dv]
   int n_seq, seq_len, total_tokens, H, dv, n_slices;
   float scale;
   unsigned flags;
@@ -66,6 +69,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_simt_kernel(const Para
   float* sg = sm + PL::G;
   float* sgam = sg + C;
   float* sb = sg + 2 * C;
+  float* sr = sg + 3 * C;
 
   const int tid = threadIdx.x;
   const int slice = blockIdx.x % p.n_slices;
@@ -150,7 +154,10 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_simt_kernel(const Para
       }
     }
     __syncthreads();
-    if (tid < C) sgam[tid] = expf(sg[tid]);
+    if (tid < C) {
+      sgam[tid] = expf(sg[tid]);
+      sr[tid] = expf(sg[C - 1] - sg[tid]);   // gamma_C / gamma_i (never 0 / 0)
+    }
     // ---- A and P
     for (int e = tid; e < C * C; e += THREADS) {
       const int i = e / C, j = e % C;
@@ -198,14 +205,23 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_simt_kernel(const Para
       sU[i * LDC + c] = acc;
     }
     __syncthreads();
-    // ---- O = scale (diag(gamma) Q Sigma_0 + P U)
+    // ---- O = scale (diag(gamma) Q Sigma_0 + P U), then the output gate and
+    // the loop residual (o rounded to the io dtype first, as loop_residual sees
+    // it; h_prev is read by the thread that then writes the same element)
     for (int e = tid; e < C * DVS; e += THREADS) {
       const int i = e / DVS, c = e % DVS;
       if (i >= valid) continue;
       float qs = 0.f, pu = 0.f;
       for (int d = 0; d < DK; ++d) qs = fmaf(sQ[i * LDK + d], sSig[d * LDC + c], qs);
       for (int j = 0; j <= i; ++j) pu = fmaf(sP[i * LDC + j], sU[j * LDC + c], pu);
-      o[((size_t)(tok0 + i) * H + h) * dv + col0 + c] = from_f32<T>(p.scale * fmaf(sgam[i], qs, pu));
+      float y = p.scale * fmaf(sgam[i], qs, pu);
+      const size_t off = ((size_t)(tok0 + i) * H + h) * dv + col0 + c;
+      if (p.gate) y *= 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + i) * H + h]));
+      if (p.h_prev) {
+        const float hp = to_f32(static_cast<const T*>(p.h_prev)[off]);
+        y = fmaf(p.rho[(size_t)h * dv + col0 + c], hp, to_f32(from_f32<T>(y)));
+      }
+      o[off] = from_f32<T>(y);
     }
     __syncthreads();
     // ---- Sigma_C = gamma_C Sigma_0 + K^T diag(gamma_C / gamma) U
@@ -213,7 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_simt_kernel(const Para
     for (int e = tid; e < DK * DVS; e += THREADS) {
       const int d = e / DVS, c = e % DVS;
       float acc = 0.f;
-      for (int i = 0; i < C; ++i) acc = fmaf(sK[i * LDK + d] * (gC / sgam[i]), sU[i * LDC + c], acc);
+      for (int i = 0; i < C; ++i) acc = fmaf(sK[i * LDK + d] * sr[i], sU[i * LDC + c], acc);
       sSig[d * LDC + c] = fmaf(gC, sSig[d * LDC + c], acc);
     }
   }
@@ -250,6 +266,9 @@ gdn_status launch_prefill_simt(const gdn_fwd_params* p, unsigned* status, cudaSt
   kp.o = p->o;
   kp.cu_seqlens = p->cu_seqlens;
   kp.status = status;
+  kp.gate = p->gate;
+  kp.h_prev = p->h_prev;
+  kp.rho = p->rho;
   kp.n_seq = p->n_seq;
   kp.seq_len = p->seq_len;
   kp.total_tokens = p->total_tokens;

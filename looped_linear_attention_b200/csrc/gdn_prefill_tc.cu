@@ -135,6 +135,11 @@ struct Params {
   __nv_bfloat16* o;
   const int32_t* cu_seqlens;
   unsigned* status;
+  // epilogue of the looped block (null = off): head-wise output gate logits
+  // [tokens][H] and the loop residual o += rho (.) h_prev ([tokens][H*dv], [H*dv])
+  const float* gate;
+  const __nv_bfloat16* h_prev;
+  const float* rho;
   int n_seq, seq_len, total_tokens, H, dv, n_slices;
   float scale;
   unsigned flags;
@@ -166,12 +171,12 @@ struct Gates {
   float* e;      // 2^(g2_i - m), m = (g2_0 + g2_{C-1}) / 2 (row factor of D)
   float* f;      // 2^(m - g2_j) (column factor of D)
   float* flag;   // [0]: 1 when |g2_0 - g2_{C-1}| < 64, so that e_i f_j = D_ij in range
-  // With the q/k L2 norm the tiles stay as loaded and the prep team folds the
-  // inverse row norms into the factors that meet them (at the top of the chunk):
-  // r, bg and f take 1/|k_j| (f becomes 1/|k_j| alone when flag is 0), and
-  float* gq;     // gamma_i / |q_i| (output factor of Sigma^T Q^T)
+  // With the q/k L2 norm the tiles stay as loaded and the state team folds the
+  // inverse row norms into the factors that meet them: r, bg and f take
+  // 1/|k_j| (f becomes 1/|k_j| alone when flag is 0), and qn, gq take 1/|q_i|.
+  float* gq;     // gamma_i qn_i (output factor of Sigma^T Q^T)
   float* kn;     // 1 / |k_i|
-  float* qn;     // 1 / |q_i|
+  float* qn;     // output row factor: sigmoid(gate_i) (1 without the gate), times 1/|q_i|
 };
 
 __device__ __forceinline__ Gates gates_at(uint8_t* sm, int buf) {
@@ -257,8 +262,9 @@ __device__ __forceinline__ void fold_qk_norms(const uint8_t* kq, const Gates& G,
       G.bg[r] *= inv;
       G.f[r] = (G.flag[0] != 0.f ? G.f[r] : 1.f) * inv;
     } else {
-      G.qn[r] = inv;
-      G.gq[r] = G.gamma[r] * inv;
+      const float qs = G.qn[r] * inv;
+      G.qn[r] = qs;
+      G.gq[r] = G.gamma[r] * qs;
     }
   }
 }
@@ -374,17 +380,20 @@ __device__ __forceinline__ void store_res_t12(uint8_t* sm, const Gates& G, int a
   }
 }
 
-// Gate inputs of one token (threads 0-63 of the state warpgroup): a and b, or
-// a = 1, b = 0 past the sequence end.  Issued well before they are used so the
-// global-memory latency is hidden behind a chunk.
+// Gate inputs of one token (threads 0-63 of the state warpgroup): a, b and the
+// output gate sigmoid(gate) (1 without one), or a = 1, b = 0 past the sequence
+// end.  Issued well before they are used so the global-memory latency is
+// hidden behind a chunk.
 __device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int valid, int h, int t,
-                                                 float& a_in, float& bb) {
+                                                 float& a_in, float& bb, float& og) {
   a_in = 1.f;
   bb = 0.f;
+  og = 1.f;
   if (t < valid) {
     const size_t ti = (size_t)(tok0 + t) * p.H + h;
     a_in = __ldg(p.a + ti);
     bb = __ldg(p.b + ti);
+    if (p.gate) og = 1.f / (1.f + __expf(-__ldg(p.gate + ti)));
   }
 }
 
@@ -392,7 +401,7 @@ __device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int 
 // 0-63 own one token each).  Rows past the sequence end get a = 1 and b = 0.
 template <int BAR>
 __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid, int t, float a_in,
-                                              float bb) {
+                                              float bb, float og) {
   const int lane = t & 31;
   float la = 0.f;
   if (t < C) {
@@ -416,6 +425,8 @@ __device__ __forceinline__ void compute_gates(Gates G, float* s_carry, int valid
     const float mid = 0.5f * (g0 + gl);
     const float gam = ex2_approx(la);
     G.gamma[t] = gam;
+    G.qn[t] = og;
+    G.gq[t] = gam * og;
     G.bg[t] = bb * gam;
     G.r[t] = ex2_approx(gl - la);
     G.e[t] = ex2_approx(la - mid);
@@ -749,10 +760,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int i = tq & 63;
         const int cb = hf * 32;                         // first column of this thread
         const bool zero_half = (hf == 1) && ((warp & 1) == 0);
-        // row factor: b_i (A rows) or 1 (P rows), times the row's inverse norm;
-        // the column factor f_j carries 1/|k_j| (and is 1/|k_j| alone on the
+        // row factor: b_i (A rows) or the output row factor qn_i (P rows: the
+        // output gate and 1/|q_i|), times 1/|k_i| on A rows with the norm; the
+        // column factor f_j carries 1/|k_j| (and is 1/|k_j| alone on the
         // exponential path)
-        const float sc = (tq < C) ? (l2n ? G.b[i] * G.kn[i] : G.b[i]) : (l2n ? G.qn[i] : 1.f);
+        const float sc = (tq < C) ? (l2n ? G.b[i] * G.kn[i] : G.b[i]) : G.qn[i];
         const int lim = (tq < C) ? i : i + 1;           // columns j < lim are kept
         float gr[32];
         if (zero_half) {
@@ -905,13 +917,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     // gate vectors of chunks 0 and 1 (later ones are built two chunks ahead,
     // while the products of each chunk run); a_in, b_in hold the inputs of the
     // next chunk to build
-    float a_in, b_in;
+    float a_in, b_in, og_in;
     auto gates_of = [&](int c) {
       compute_gates<BAR_STATE>(gates_at(sm, c % 3), s_carry, min(C, seq_end - (seq_start + c * C)), jt,
-                               a_in, b_in);
+                               a_in, b_in, og_in);
       if (c + 1 < n_chunks)
         load_gate_inputs(p, seq_start + (c + 1) * C, min(C, seq_end - (seq_start + (c + 1) * C)), h, jt,
-                         a_in, b_in);
+                         a_in, b_in, og_in);
       wg_sync<BAR_STATE>();
     };
     // Hands chunk c2 to the prep team once its K, Q tiles have landed: with the
@@ -945,7 +957,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       return true;
     };
     if (ok && n_chunks > 0) {
-      load_gate_inputs(p, seq_start, min(C, len), h, jt, a_in, b_in);
+      load_gate_inputs(p, seq_start, min(C, len), h, jt, a_in, b_in, og_in);
       gates_of(0);
       if (n_chunks > 1) gates_of(1);
 #pragma unroll 1
@@ -1105,7 +1117,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(tmem + lane_off + COL_OB + 32 * hf, ob);
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 g4 = *reinterpret_cast<const float4*>((l2n ? G.gq : G.gamma) + 32 * hf + 4 * e4);
+            const float4 g4 = *reinterpret_cast<const float4*>(G.gq + 32 * hf + 4 * e4);
             const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -1118,15 +1130,45 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_before();
         wg_sync<BAR_STATE>();
         {
+          // 16-byte vectors: this thread stores columns col0 + 8 q .. + 7 of rows
+          // jt / 16 + 16 k8; with the loop residual it adds rho (.) h_prev of the
+          // same elements (read by this thread just before it writes them, so o
+          // may be h_prev itself), after the rounding of o, as loop_residual does
           const uint8_t* stage = sm + OFF_UTP;
+          const int q = jt & 15;
+          const size_t row0 = ((size_t)tok0 * H + h) * dv + col0 + q * 8;
+          const size_t row_stride = (size_t)H * dv;
+          if (p.h_prev) {
+            uint4 hp[4];
 #pragma unroll
-          for (int k8 = 0; k8 < 4; ++k8) {
-            const int it = jt + k8 * TEAM;
-            const int i = it >> 4, q = it & 15;
-            if (i < valid) {
-              const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
-              __nv_bfloat16* dst = p.o + ((size_t)(tok0 + i) * H + h) * dv + col0 + q * 8;
-              __stcs(reinterpret_cast<uint4*>(dst), v);
+            for (int k8 = 0; k8 < 4; ++k8) {
+              const int i = (jt >> 4) + 16 * k8;
+              if (i < valid) hp[k8] = *reinterpret_cast<const uint4*>(p.h_prev + row0 + i * row_stride);
+            }
+            const float4 r0 = __ldg(reinterpret_cast<const float4*>(p.rho + (size_t)h * dv + col0 + q * 8));
+            const float4 r1 = __ldg(reinterpret_cast<const float4*>(p.rho + (size_t)h * dv + col0 + q * 8 + 4));
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+              const int i = (jt >> 4) + 16 * k8;
+              if (i < valid) {
+                const uint4 x = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
+                const uint4 y = hp[k8];
+                uint4 v;
+                v.x = pack_bf16x2(fmaf(r0.x, bf16_lo(y.x), bf16_lo(x.x)), fmaf(r0.y, bf16_hi(y.x), bf16_hi(x.x)));
+                v.y = pack_bf16x2(fmaf(r0.z, bf16_lo(y.y), bf16_lo(x.y)), fmaf(r0.w, bf16_hi(y.y), bf16_hi(x.y)));
+                v.z = pack_bf16x2(fmaf(r1.x, bf16_lo(y.z), bf16_lo(x.z)), fmaf(r1.y, bf16_hi(y.z), bf16_hi(x.z)));
+                v.w = pack_bf16x2(fmaf(r1.z, bf16_lo(y.w), bf16_lo(x.w)), fmaf(r1.w, bf16_hi(y.w), bf16_hi(x.w)));
+                __stcs(reinterpret_cast<uint4*>(p.o + row0 + i * row_stride), v);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+              const int i = (jt >> 4) + 16 * k8;
+              if (i < valid) {
+                const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
+                __stcs(reinterpret_cast<uint4*>(p.o + row0 + i * row_stride), v);
+              }
             }
           }
         }
@@ -1479,6 +1521,9 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   kp.o = static_cast<__nv_bfloat16*>(p->o);
   kp.cu_seqlens = p->cu_seqlens;
   kp.status = status;
+  kp.gate = p->gate;
+  kp.h_prev = static_cast<const __nv_bfloat16*>(p->h_prev);
+  kp.rho = p->rho;
   kp.n_seq = p->n_seq;
   kp.seq_len = p->seq_len;
   kp.total_tokens = p->total_tokens;

@@ -8,7 +8,12 @@ h~^(tau) is the GDN output itself, reshaped [L, H*dv] = [L, d] (d = H*dv), from
 a zero initial state each loop; q and k are L2-normalised per head inside the
 mixer kernel.  The three projections are one batched torch GEMM over the
 stacked weights [W_q; W_k; W_v] (outside the mixer's hot path); the mixer and
-the residual run in this library's kernels.
+the residual run in this library's kernels: by default the residual is fused
+into the mixer's output epilogue (one launch fewer per loop, and the mixer
+output never makes a round trip through HBM), or it runs as loop_residual.
+The gated variant (§3, gated-attention paragraph) adds a head-wise sigmoid
+output gate whose logits h^(tau-1) W_g (W_g [d, H] fp32) are one more torch
+GEMM per loop; the gate itself is applied in the mixer's epilogue.
 """
 from __future__ import annotations
 
@@ -23,8 +28,9 @@ class LoopedPrefill:
     """Pre-allocated buffers for repeated looped-prefill steps (graph-capturable)."""
 
     def __init__(self, L: int, H: int, dk: int, dv: int, loops: int, device,
-                 dtype=torch.bfloat16, time_mixer: bool = False):
+                 dtype=torch.bfloat16, time_mixer: bool = False, fused_residual: bool = True):
         d_in = H * dk
+        self.fused_residual = fused_residual
         # optional CUDA-event pairs around every mixer launch (for per-kernel timing)
         self.time_mixer = time_mixer
         self.mixer_events = []
@@ -36,12 +42,20 @@ class LoopedPrefill:
         self.k = self.qkv[1].view(L, H, dk)
         self.v = self.qkv[2].view(L, H, dv)
         self.o = torch.empty(L, H, dv, dtype=dtype, device=device)
+        self.z = torch.empty(L, H, dtype=torch.float32, device=device)     # output-gate logits
         self.h = [torch.empty(L, H * dv, dtype=dtype, device=device) for _ in range(2)]
+
+    def launches_per_loop(self) -> int:
+        """This library's kernel launches per loop: the mixer's (its schedule)
+        plus the loop residual when it is not fused."""
+        sched = B.prefill_schedule(1, self.L, self.H, self.dk, self.dv, flags=B.GDN_QK_L2NORM)
+        return sched["launches"] + (0 if self.fused_residual else 1)
 
     def run(self, h0: torch.Tensor, Wq: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor,
             a: torch.Tensor, b: torch.Tensor, rho: torch.Tensor, scale: float = 1.0,
-            out: Optional[torch.Tensor] = None) -> torch.Tensor:
-        """h0 [L, d]; W* [d, d]; a, b [T, L, H] fp32; rho [T, d] fp32. Returns h^(T).
+            out: Optional[torch.Tensor] = None, Wg: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """h0 [L, d]; W* [d, d]; a, b [T, L, H] fp32; rho [T, d] fp32; Wg [d, H]
+        fp32 output-gate weights or None. Returns h^(T).
 
         Wq, Wk, Wv given as the three planes of one [3, d, d] tensor (see
         `stack_weights`) are used in place; otherwise they are stacked into a
@@ -53,24 +67,34 @@ class LoopedPrefill:
         h_prev = h0
         for tau in range(self.loops):
             torch.matmul(h_prev.unsqueeze(0), W3, out=self.qkv)
+            z = None
+            if Wg is not None:
+                torch.matmul(h_prev.float(), Wg, out=self.z)
+                z = self.z
+            last = tau == self.loops - 1
+            h_next = out if (last and out is not None) else self.h[tau % 2]
             if self.time_mixer:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record()
-            B.gdn_chunk_fwd(self.q, self.k, self.v, a[tau], b[tau], None, scale=scale,
-                            flags=B.GDN_QK_L2NORM, o=self.o, return_state=False)
+            if self.fused_residual:
+                B.gdn_chunk_fwd(self.q, self.k, self.v, a[tau], b[tau], None, scale=scale,
+                                flags=B.GDN_QK_L2NORM, o=h_next, return_state=False, gate=z,
+                                h_prev=h_prev, rho=rho[tau])
+            else:
+                B.gdn_chunk_fwd(self.q, self.k, self.v, a[tau], b[tau], None, scale=scale,
+                                flags=B.GDN_QK_L2NORM, o=self.o, return_state=False, gate=z)
             if self.time_mixer:
                 e1.record()
                 self.mixer_events.append((e0, e1))
-            last = tau == self.loops - 1
-            h_next = out if (last and out is not None) else self.h[tau % 2]
-            B.loop_residual(self.o.view(L, H * dv), h_prev, rho[tau], out=h_next)
+            if not self.fused_residual:
+                B.loop_residual(self.o.view(L, H * dv), h_prev, rho[tau], out=h_next)
             h_prev = h_next
         return h_prev
 
     def capture(self, h0: torch.Tensor, Wq: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor,
                 a: torch.Tensor, b: torch.Tensor, rho: torch.Tensor, scale: float = 1.0,
-                out: Optional[torch.Tensor] = None):
+                out: Optional[torch.Tensor] = None, Wg: Optional[torch.Tensor] = None):
         """Records one `run` on these tensors into a CUDA graph.
 
         Returns (graph, h): each graph.replay() repeats the whole T-loop step
@@ -85,13 +109,13 @@ class LoopedPrefill:
             side = torch.cuda.Stream(dev)
             side.wait_stream(torch.cuda.current_stream(dev))
             with torch.cuda.stream(side):
-                self.run(h0, Wq, Wk, Wv, a, b, rho, scale=scale, out=out)
+                self.run(h0, Wq, Wk, Wv, a, b, rho, scale=scale, out=out, Wg=Wg)
             torch.cuda.current_stream(dev).wait_stream(side)
             graph = torch.cuda.CUDAGraph()
             # thread-local capture: CUDA calls of other threads (a process
             # group's watchdog, for one) do not invalidate it
             with torch.cuda.graph(graph, capture_error_mode="thread_local"):
-                h = self.run(h0, Wq, Wk, Wv, a, b, rho, scale=scale, out=out)
+                h = self.run(h0, Wq, Wk, Wv, a, b, rho, scale=scale, out=out, Wg=Wg)
         finally:
             self.time_mixer = timing
         return graph, h

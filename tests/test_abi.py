@@ -354,3 +354,36 @@ def test_backward_binding_refuses_host_tensors():
     v = torch.zeros(T, H, dv, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA tensor"):
         lla.gdn_chunk_bwd(q, q, v, a, a, v)
+
+
+def test_prefill_epilogue_validation(lib):
+    """The looped-block epilogue: h_prev and rho come together, o may be
+    h_prev exactly but overlap it no other way, and may not overlap the gate."""
+    ok = _params(h_prev=1 << 28, rho=1 << 24, gate=1 << 26)          # o == h_prev
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(ok)) != ctypes.c_size_t(-1).value
+    for bad in (dict(h_prev=1 << 30),                                # no rho
+                dict(rho=1 << 24),                                   # no h_prev
+                dict(h_prev=(1 << 28) + 256, rho=1 << 24),           # partial overlap with o
+                dict(gate=(1 << 28) + 64),                           # gate inside o
+                dict(gate=(1 << 26) + 8)):                           # misaligned
+        p = _params(**bad)
+        assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == ctypes.c_size_t(-1).value, bad
+        assert lib.gdn_chunk_fwd(ctypes.byref(p), None, 0, None) == B.GDN_ERR_INVALID, bad
+
+
+@pytest.mark.parametrize("args", [
+    dict(h_prev=1 << 24),                                            # no rho
+    dict(rho=1 << 24),                                               # no h_prev
+    dict(gate=(1 << 26) + 4),                                        # misaligned gate
+    dict(h_prev=(1 << 30) + 512, rho=1 << 24),                       # partial overlap with o
+    dict(gate=1 << 30),                                              # gate inside o
+])
+def test_decode_looped_rejects_bad_epilogue_on_host(lib, args):
+    base = dict(q=16, k=32, v=48, a=64, b=80, S=1 << 20, o=1 << 30, gate=None, h_prev=None,
+                rho=None, N=4, H=2, dk=128, dv=128, dt=B.GDN_BF16, scale=1.0, flags=0)
+    base.update(args)
+    st = lib.gdn_decode_step_looped(base["q"], base["k"], base["v"], base["a"], base["b"], base["S"],
+                                    base["o"], base["gate"], base["h_prev"], base["rho"], base["N"],
+                                    base["H"], base["dk"], base["dv"], base["dt"], base["scale"],
+                                    base["flags"], None)
+    assert st == B.GDN_ERR_INVALID

@@ -149,24 +149,34 @@ size_t gdn_chunk_fwd_workspace(const gdn_fwd_params *p);
  *   seg0_tok, seg_tok: 0 for one pass.
  *   launches: stream operations the call enqueues: 0 (nothing to do), 1 (one
  *             pass, or the copy or clear of S_T when every sequence is empty),
- *             2 (two segments: no combine step; or a varlen call with its
- *             length sort) or 3.
+ *             2 or 3 (see the schedules below; a varlen call with its length
+ *             sort takes 2).
+ *   corrected: 1 for the corrected segmented schedule, else 0.
  * Parameters gdn_chunk_fwd would reject return the same error status. */
 gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg0_tok,
-                                  int *seg_tok, int *launches);
+                                  int *seg_tok, int *launches, int *corrected);
 
 /* Chunkwise prefill (chunks of 64 tokens).
  *
  * Schedule.  Each (sequence, head, 128-wide dv slice) chain normally runs in
  * one pass.  When fixed-length sequences (cu_seqlens == NULL) give too few
  * chains to fill the GPU, every sequence is instead cut into segments whose
- * state update is affine in the start state, S_end = M S_start + B.  A first
- * launch runs segment 0 in full from S0 and, beside it, computes every later
- * segment's B (from a zero state) and dk x dk transition M, except the last
- * segment's; a second kernel chains the segment start states in fp32 (skipped
- * with two segments), and a third launch runs segments 1 .. P-1 from their
- * start states and writes their outputs (all on `stream`).  The outputs equal
- * the one-pass outputs up to rounding.  GDN_SINGLE_PASS disables it.
+ * state update is affine in the start state, S_end = M S_start + B, with one
+ * of two schedules (all launches on `stream`):
+ *   corrected (the default): a first launch runs segment 0 in full from S0
+ *     and, beside it, every later segment from a zero state, writing its
+ *     zero-start outputs into o, its B, its dk x dk transition M, and the
+ *     per-token rows qhat_i = M_i^T q_i (scaled like o_i) that carry the
+ *     start state's share of each output; a second kernel chains the start
+ *     states (and S_T) in fp32 (skipped when there is nothing to chain); a
+ *     third adds qhat_i^T S_p to the outputs (tensor cores) and applies the
+ *     loop residual.
+ *   output pass (when o is h_prev itself, which the first launch would
+ *     overwrite): the first launch computes B and M of segments 1 .. P-2
+ *     without outputs, the combine chains the start states, and a third
+ *     launch runs segments 1 .. P-1 again from their start states.
+ * The outputs equal the one-pass outputs up to rounding.  GDN_SINGLE_PASS
+ * disables segmenting.
  * Varlen calls (cu_seqlens != NULL) always run one pass; when they take more
  * blocks than the GPU runs at once and have at most 4096 sequences, a first
  * launch sorts the sequences by length on the device (longest first, into the

@@ -83,7 +83,7 @@ def library() -> ctypes.CDLL:
         lib.gdn_chunk_fwd_workspace.argtypes = [ctypes.POINTER(gdn_fwd_params)]
         lib.gdn_chunk_fwd_workspace.restype = ctypes.c_size_t
         lib.gdn_chunk_fwd_schedule.argtypes = [ctypes.POINTER(gdn_fwd_params)] + [
-            ctypes.POINTER(ctypes.c_int)] * 4
+            ctypes.POINTER(ctypes.c_int)] * 5
         lib.gdn_chunk_fwd_schedule.restype = i32
         lib.gdn_chunk_bwd_workspace.argtypes = [ctypes.POINTER(gdn_bwd_params)]
         lib.gdn_chunk_bwd_workspace.restype = ctypes.c_size_t
@@ -285,17 +285,24 @@ def prefill_workspace_bytes(n_seq: int, seq_len: int, H: int, dk: int, dv: int,
 
 def prefill_schedule(n_seq: int, seq_len: int, H: int, dk: int, dv: int,
                      dtype: torch.dtype = torch.bfloat16, flags: int = 0,
-                     varlen: bool = False) -> dict:
+                     varlen: bool = False, with_state: bool = True,
+                     residual_in_place: bool = False) -> dict:
     """gdn_chunk_fwd_schedule for a call of this shape, given its workspace:
-    {"n_segs", "seg0_tok", "seg_tok", "launches"} (n_segs = 1: one pass per chain)."""
+    {"n_segs", "seg0_tok", "seg_tok", "launches", "corrected"} (n_segs = 1: one
+    pass per chain).  with_state: the call writes S_T; residual_in_place: o is
+    the loop residual's h_prev itself."""
     p = _shape_params(n_seq, seq_len, H, dk, dv, dtype, flags, varlen)
-    n, tok0, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    if with_state:
+        p.S_T = (1 << 40) + (8 << 36)
+    if residual_in_place:
+        p.h_prev, p.rho = p.o, (1 << 40) + (9 << 36)
+    n, tok0, tok, launches, corr = (ctypes.c_int() for _ in range(5))
     st = library().gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
-                                          ctypes.byref(tok), ctypes.byref(launches))
+                                          ctypes.byref(tok), ctypes.byref(launches), ctypes.byref(corr))
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd_schedule")
     return {"n_segs": n.value, "seg0_tok": tok0.value, "seg_tok": tok.value,
-            "launches": launches.value}
+            "launches": launches.value, "corrected": corr.value}
 
 
 def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,

@@ -28,6 +28,8 @@ struct SegPlan {
   int seg_tok;     // tokens of segments 1 .. n_segs-1 (the last one may be shorter)
   int seg0_tok;    // tokens of segment 0
   int lpt;         // varlen, one pass: sequences launched longest first (order in the workspace)
+  int corrected;   // segmented: outputs of segments 1 .. n_segs-1 from a zero state, then
+                   // corrected by their start states (else a second pass recomputes them)
 };
 
 // Upper bound for any device-side wait: about 2 s of SM clock.  A wait that

@@ -193,20 +193,22 @@ size_t gdn_chunk_fwd_workspace(const gdn_fwd_params* p) {
 }
 
 gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params* p, int* n_segs, int* seg0_tok, int* seg_tok,
-                                  int* launches) {
+                                  int* launches, int* corrected) {
   const gdn_status v = validate_fwd(p);
   if (v != GDN_OK) return v;
-  gdn::SegPlan plan{1, 0, 0, 0};
+  gdn::SegPlan plan{1, 0, 0, 0, 0};
   if (p->total_tokens > 0 && gdn::prefill_tc_supported(p)) plan = gdn::plan_prefill_segments(p, sm_count());
   int n = 1;                                           // one pass
   if (p->n_seq == 0) n = 0;
   else if (p->total_tokens == 0) n = (p->S_T && p->S0 != p->S_T) ? 1 : 0;   // a copy or a clear of S_T
-  else if (plan.n_segs > 2) n = 3;
+  else if (plan.corrected) n = (plan.n_segs > 2 || p->S_T) ? 3 : 2;          // state pass, combine, correction
+  else if (plan.n_segs > 2) n = 3;                                          // state pass, combine, output pass
   else if (plan.n_segs == 2 || plan.lpt) n = 2;
   if (n_segs) *n_segs = plan.n_segs;
   if (seg0_tok) *seg0_tok = plan.seg0_tok;
   if (seg_tok) *seg_tok = plan.seg_tok;
   if (launches) *launches = n;
+  if (corrected) *corrected = plan.corrected;
   return GDN_OK;
 }
 
@@ -227,10 +229,10 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_params* p, void* ws, size_t ws_bytes,
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
   }
   const bool tc = gdn::prefill_tc_supported(p);
-  gdn::SegPlan plan = tc ? gdn::plan_prefill_segments(p, sm_count()) : gdn::SegPlan{1, 0, 0, 0};
+  gdn::SegPlan plan = tc ? gdn::plan_prefill_segments(p, sm_count()) : gdn::SegPlan{1, 0, 0, 0, 0};
   if (plan.n_segs > 1 || plan.lpt) {
     const size_t need = gdn::prefill_segment_workspace(p, plan);
-    if (!ws && ws_bytes == 0) plan = gdn::SegPlan{1, 0, 0, 0};   // no workspace: one pass, natural order
+    if (!ws && ws_bytes == 0) plan = gdn::SegPlan{1, 0, 0, 0, 0};   // no workspace: one pass, natural order
     else if (!ws || ws_bytes < need) return GDN_ERR_WORKSPACE;
   }
   unsigned* st = status_ptr();

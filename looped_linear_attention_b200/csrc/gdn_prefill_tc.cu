@@ -154,11 +154,19 @@ struct Params {
   //           segment's dk x dk transition M_p to Mws slot p-1.
   //   mode 2: segments 1 .. n_segs-1 from their start states S_p in Sst slot
   //           p-1, with outputs; the last segment writes S_T.
+  //   mode 3: the state pass of the corrected schedule: as mode 1, but for
+  //           segments 1 .. n_segs-1 (B_p, M_p in slot p-1), and with
+  //           outputs: the slices write each segment's zero-start output o^0
+  //           into o (gated, no residual), the transition slice its outputs
+  //           qhat_i = scale og_i M_{p,i}^T q_i (the start state's share of
+  //           o_i is then qhat_i^T S_p, added by gdn_segment_correct_kernel)
+  //           into qhat [tokens][H][dk].
   int mode, n_segs, seg_tok, seg0_tok;
   const int32_t* order;  // mode 0, varlen: sequences longest first (block order), or null
-  float* Bws;          // [n_seq][n_segs-2][H][dk][dv]
-  float* Mws;          // [n_seq][n_segs-2][H][dk][dk]
+  float* Bws;          // [n_seq][n_part][H][dk][dv], n_part = n_segs-2 (mode 1) or n_segs-1 (mode 3)
+  float* Mws;          // [n_seq][n_part][H][dk][dk]
   float* Sst;          // [n_seq][n_segs-1][H][dk][dv]
+  __nv_bfloat16* qhat; // mode 3: [total_tokens][H][dk]
 };
 
 // Per-chunk gate vectors (one buffer).
@@ -624,22 +632,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);   // warp-uniform by construction
   // segmented schedule: the combine kernel may be launched now (it waits for
   // this grid before it reads anything)
-  if (p.mode == 1) griddep_launch_dependents();
+  if (p.mode == 1 || p.mode == 3) griddep_launch_dependents();
 
   // work unit: (sequence or segment, head, dv slice)
   int slice, h, seq, part;
-  bool partial = false;   // a segment run from a zero state or the identity, without outputs
+  bool partial = false;   // a segment run from a zero state or the identity
+  const bool state_pass = (p.mode == 1 || p.mode == 3);
+  const int n_part = (p.mode == 3) ? p.n_segs - 1 : p.n_segs - 2;   // segments with B, M
   {
     int bid = (int)blockIdx.x;
     int slices_here = p.n_slices;
     int units_per_seq = 1, first_part = 0;
-    if (p.mode == 1) {
+    if (state_pass) {
       const int n_first = p.n_seq * p.H * p.n_slices;   // segment 0 of every chain, run in full
       if (bid >= n_first) {
         bid -= n_first;
         partial = true;
         slices_here = p.n_slices + 1;
-        units_per_seq = p.n_segs - 2;
+        units_per_seq = n_part;
         first_part = 1;
       }
     } else if (p.mode == 2) {
@@ -655,7 +665,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (p.order) seq = __ldg(p.order + seq);   // longest sequences in the first blocks
   }
   const bool ident = partial && slice == p.n_slices;   // transition slice: V = 0, S0 = I
-  const bool outputs = !partial;
+  // outputs: whole segments, and every segment of the corrected state pass
+  // (zero-start outputs, or qhat from the transition slice); the loop residual
+  // only where the output is final
+  const bool outputs = !partial || p.mode == 3;
+  const bool residual = (p.h_prev != nullptr) && !partial;
   int seq_start, seq_end;
   if (p.cu_seqlens) {
     seq_start = p.cu_seqlens[seq];
@@ -889,11 +903,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (p.mode == 0) {
       s0 = p.S0 ? p.S0 + state_base : nullptr;
       st = p.S_T ? p.S_T + state_base : nullptr;
-    } else if (p.mode == 1 && !partial) {   // segment 0: S_1 to start-state slot 0
+    } else if (state_pass && !partial) {   // segment 0: S_1 to start-state slot 0
       s0 = p.S0 ? p.S0 + state_base : nullptr;
       st = p.Sst + ((size_t)seq * (p.n_segs - 1) * H + h) * DK * (size_t)dv + col0 + j;
-    } else if (p.mode == 1) {
-      const size_t u = (size_t)seq * (p.n_segs - 2) + (part - 1);
+    } else if (state_pass) {
+      const size_t u = (size_t)seq * n_part + (part - 1);
       if (ident) {
         st = p.Mws + (u * H + h) * DK * DK + j;
         ldT = DK;
@@ -1011,6 +1025,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       const Gates G = gates_at(sm, c % 3);
       const uint32_t kq_a = sbase + OFF_KQ + s * KQ_BYTES;
 
+      // ---- the rows of h_prev this chunk's epilogue adds (loop residual) into
+      // L2, one 128-byte line per thread, so the epilogue's loads do not wait
+      // on HBM
+      if (outputs && residual && jt < 2 * C) {
+        const int i = jt >> 1;
+        if (i < valid) {
+          const __nv_bfloat16* line = p.h_prev + ((size_t)(tok0 + i) * H + h) * dv + col0 + (jt & 1) * 64;
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(line));
+        }
+      }
       // ---- O_A^T = Sigma^T Q^T (needs no W: it runs while W^T is converted)
       if (!wg_wait<BAR_STATE>(&bars[B_W_READY], c & 1, s_abort, p.status)) break;
       tc_fence_after();
@@ -1136,9 +1160,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           // may be h_prev itself), after the rounding of o, as loop_residual does
           const uint8_t* stage = sm + OFF_UTP;
           const int q = jt & 15;
-          const size_t row0 = ((size_t)tok0 * H + h) * dv + col0 + q * 8;
-          const size_t row_stride = (size_t)H * dv;
-          if (p.h_prev) {
+          // the transition slice of the corrected state pass writes qhat (rows of dk)
+          __nv_bfloat16* out = ident ? p.qhat : p.o;
+          const int ow = ident ? DK : dv;
+          const size_t row0 = ((size_t)tok0 * H + h) * ow + col0 + q * 8;
+          const size_t row_stride = (size_t)H * ow;
+          if (residual) {
             uint4 hp[4];
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8) {
@@ -1158,7 +1185,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 v.y = pack_bf16x2(fmaf(r0.z, bf16_lo(y.y), bf16_lo(x.y)), fmaf(r0.w, bf16_hi(y.y), bf16_hi(x.y)));
                 v.z = pack_bf16x2(fmaf(r1.x, bf16_lo(y.z), bf16_lo(x.z)), fmaf(r1.y, bf16_hi(y.z), bf16_hi(x.z)));
                 v.w = pack_bf16x2(fmaf(r1.z, bf16_lo(y.w), bf16_lo(x.w)), fmaf(r1.w, bf16_hi(y.w), bf16_hi(x.w)));
-                __stcs(reinterpret_cast<uint4*>(p.o + row0 + i * row_stride), v);
+                __stcs(reinterpret_cast<uint4*>(out + row0 + i * row_stride), v);
               }
             }
           } else {
@@ -1167,7 +1194,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               const int i = (jt >> 4) + 16 * k8;
               if (i < valid) {
                 const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + q * 16);
-                __stcs(reinterpret_cast<uint4*>(p.o + row0 + i * row_stride), v);
+                __stcs(reinterpret_cast<uint4*>(out + row0 + i * row_stride), v);
               }
             }
           }
@@ -1239,9 +1266,12 @@ bool prefill_tc_supported(const gdn_fwd_params* p) {
 
 // ------------------------------------------------------------------ segments
 // Combine step of the segmented schedule: for one (sequence, head) and
-// CMB_COLS columns of dv, S_{p+1} = M_p S_p + B_p for p = 1 .. n_segs-2,
+// CMB_COLS columns of dv, S_{p+1} = M_p S_p + B_p for p = 1 .. n_steps,
 // starting from S_1 (written by the segment-0 CTAs) and writing every S_p,
-// p >= 2, to Sst (slot p-1; M_p and B_p sit in slot p-1 of theirs).  The
+// p >= 2, to Sst (slot p-1; M_p and B_p sit in slot p-1 of theirs).  With
+// n_steps = n_segs - 2 (output-pass schedule) the last one is S_{n_segs-1};
+// with n_steps = n_segs - 1 (corrected schedule) the last one, S_{n_segs}, is
+// the final state and goes to S_T (or nowhere when S_T is null).  The
 // products run on the warp-level tensor cores with the 3xTF32 split
 // (fp32-level accuracy): warp w owns rows 16w .. 16w+15 of the 128 x CMB_COLS
 // block.  M_p (dk x dk) is staged in shared memory by cp.async one step ahead
@@ -1267,7 +1297,8 @@ __device__ __forceinline__ void cp_async_wait() {
 
 __global__ void __launch_bounds__(256)
     gdn_segment_combine_kernel(const float* __restrict__ Bws, const float* __restrict__ Mws,
-                               float* __restrict__ Sst, int H, int dv, int n_segs) {
+                               float* __restrict__ Sst, float* __restrict__ S_T, int H, int dv,
+                               int n_segs, int n_part, int n_steps) {
   extern __shared__ __align__(16) float cmb_smem[];
   // launched as a programmatic dependent of the state pass: let the output
   // pass launch, then wait for the state pass before reading its results
@@ -1285,10 +1316,13 @@ __global__ void __launch_bounds__(256)
   const int r0 = warp * 16;                        // this warp's rows r0 .. r0+15
   const size_t sd = (size_t)DK * dv;               // one state [dk][dv]
   const size_t colb = (size_t)cb * CMB_COLS;
-  // slot i holds M_{i+1}, B_{i+1} and S_{i+1}; n_steps products chain S_1 .. S_{n_segs-1}
-  const int n_steps = n_segs - 2;
-  auto mptr = [&](int pp) { return Mws + (((size_t)seq * n_steps + pp) * H + hh) * DK * DK; };
-  auto sptr = [&](int pp) { return Sst + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb; };
+  // slot i holds M_{i+1}, B_{i+1} and S_{i+1}; n_steps products chain S_1 .. S_{n_steps+1}
+  // n_part (M, B) slots per sequence
+  auto mptr = [&](int pp) { return Mws + (((size_t)seq * n_part + pp) * H + hh) * DK * DK; };
+  auto sptr = [&](int pp) -> float* {      // S_{pp+1}
+    if (pp <= n_segs - 2) return Sst + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb;
+    return S_T ? S_T + ((size_t)seq * H + hh) * sd + colb : nullptr;
+  };
   auto stage = [&](int pp, float* dst) {
     const float* M = mptr(pp);
 #pragma unroll 4
@@ -1311,21 +1345,22 @@ __global__ void __launch_bounds__(256)
       x[nt][2 * hr + 1] = v.y;
     }
   for (int pp = 0;; ++pp) {
-    // S_{pp+1} (x) to the operand block, and to Sst unless it came from there
+    // S_{pp+1} (x) to the operand block, and to Sst (or S_T) unless it came from there
+    float* dst = (pp > 0) ? sptr(pp) : nullptr;
 #pragma unroll
     for (int nt = 0; nt < CMB_NT; ++nt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const float2 v = make_float2(x[nt][2 * hr], x[nt][2 * hr + 1]);
         const int r = r0 + g + 8 * hr, c = nt * 8 + 2 * q;
-        if (pp > 0) *reinterpret_cast<float2*>(sptr(pp) + (size_t)r * dv + c) = v;
+        if (dst) *reinterpret_cast<float2*>(dst + (size_t)r * dv + c) = v;
         *reinterpret_cast<float2*>(sS + r * CMB_SLD + c) = v;
       }
     if (pp >= n_steps) break;
     const bool prefetch = (pp + 1 < n_steps);
     if (prefetch) stage(pp + 1, ((pp + 1) & 1) ? sM1 : sM0);
     // B is loaded now and added after the product, so its latency is hidden
-    const float* B = Bws + (((size_t)seq * n_steps + pp) * H + hh) * sd + colb;
+    const float* B = Bws + (((size_t)seq * n_part + pp) * H + hh) * sd + colb;
     float2 bv[CMB_NT][2];
 #pragma unroll
     for (int nt = 0; nt < CMB_NT; ++nt)
@@ -1371,6 +1406,181 @@ __global__ void __launch_bounds__(256)
     __syncthreads();                                // every read of S_pp and M_pp is done
   }
 }
+// Output correction of the corrected segmented schedule.  Segment p >= 1 of a
+// chain ran from a zero state in the state pass and wrote its zero-start
+// outputs o^0 into o; its transition slice wrote qhat_i = scale og_i
+// M_{p,i}^T q_i (og_i: the output gate and 1/|q_i|).  The state is affine in
+// the start state, so the outputs from the true start state S_p are
+//     o_i = o^0_i + S_p^T qhat_i,
+// which this kernel adds for one (sequence, head, 128-wide dv slice) and a
+// tile of up to 128 tokens of one segment, then applies the loop residual.
+// The product is one tcgen05 MMA chain (M = 128 tokens, N = 128 columns of
+// dv, K = dk = 128) into tensor memory: qhat arrives by TMA (K-major, 128-byte
+// swizzle), S_p (fp32, from the combine or segment 0) is rounded to bf16 into
+// an MN-major operand tile.  Launched as a programmatic dependent: it waits
+// for the previous grid before reading anything the state pass wrote.
+constexpr int COR_THREADS = 128;
+constexpr int COR_ROWS = 128;                      // tokens per tile
+constexpr uint32_t COR_OFF_A = 0;                  // qhat: 2 slabs [128 tok][64 dk] bf16
+constexpr uint32_t COR_OFF_B = 32768;              // S_p: 2 blocks [128 dk][64 dv] bf16, MN-major
+constexpr uint32_t COR_OFF_BAR = 65536;            // 2 mbarriers, tmem base, abort flag
+constexpr uint32_t COR_SMEM = COR_OFF_BAR + 64 + 1024;
+
+struct CorParams {
+  __nv_bfloat16* o;
+  const __nv_bfloat16* h_prev;   // loop residual (or null) and its rho
+  const float* rho;
+  const float* Sst;              // [n_seq][n_segs-1][H][dk][dv], S_p in slot p-1
+  unsigned* status;
+  int H, dv, n_slices, seq_len, seg0_tok, seg_tok, n_segs, tiles_mid, tiles_per_seq;
+};
+
+__global__ void __launch_bounds__(COR_THREADS, 1)
+    gdn_segment_correct_kernel(const __grid_constant__ CUtensorMap tm_qh, const CorParams p) {
+  extern __shared__ __align__(1024) uint8_t csm_raw[];
+  uint8_t* sm = csm_raw;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(sm) & 1023u) {
+    if (tid == 0) record_status(p.status, GDN_ERR_CUDA);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + COR_OFF_BAR);   // [0] qhat landed, [1] MMA done
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + COR_OFF_BAR + 16);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + COR_OFF_BAR + 20);
+  // block -> (sequence, head, slice, tile); tiles enumerate segments 1 .. n_segs-1
+  int bid = (int)blockIdx.x;
+  const int tile = bid % p.tiles_per_seq;
+  bid /= p.tiles_per_seq;
+  const int slice = bid % p.n_slices;
+  bid /= p.n_slices;
+  const int h = bid % p.H;
+  const int seq = bid / p.H;
+  const int tps = (p.seg_tok + COR_ROWS - 1) / COR_ROWS;
+  int part, i0;
+  if (tile < p.tiles_mid) {
+    part = 1 + tile / tps;
+    i0 = (tile % tps) * COR_ROWS;
+  } else {
+    part = p.n_segs - 1;
+    i0 = (tile - p.tiles_mid) * COR_ROWS;
+  }
+  const int seg_start = p.seg0_tok + (part - 1) * p.seg_tok;
+  const int seg_len = min(p.seg_tok, p.seq_len - seg_start);
+  const int rows = min(COR_ROWS, seg_len - i0);
+  const int tok0 = seq * p.seq_len + seg_start + i0;
+  const int col0 = slice * DVS;
+
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qh);
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, 128);
+    tmem_relinquish();
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t sbase = smem_u32(sm);
+
+  griddep_wait();                                  // qhat, o^0 and S_p are written
+  const bool have_rows = rows > 0;
+  if (tid == 0 && have_rows) {
+    mbar_arrive_expect_tx(&bars[0], 32768);
+    tma_load_3d(sm + COR_OFF_A, &tm_qh, &bars[0], 0, h, tok0);
+    tma_load_3d(sm + COR_OFF_A + 8192, &tm_qh, &bars[0], 0, h, tok0 + 64);
+    tma_load_3d(sm + COR_OFF_A + 16384, &tm_qh, &bars[0], 64, h, tok0);
+    tma_load_3d(sm + COR_OFF_A + 24576, &tm_qh, &bars[0], 64, h, tok0 + 64);
+  }
+  // S_p (fp32 [dk][dv]) -> bf16 MN-major tile: block nb holds columns
+  // 64 nb .. 64 nb + 63, row k (dk) 128 bytes, swizzled like a TMA tile
+  const float* Sp = p.Sst + (((size_t)seq * (p.n_segs - 1) + (part - 1)) * p.H + h) * DK * (size_t)p.dv + col0;
+#pragma unroll 4
+  for (int it = 0; it < 16 && have_rows; ++it) {
+    const int u = tid + it * COR_THREADS;          // 2048 chunks of 8 columns
+    const int k = u >> 4, cc = u & 15;
+    const float4 x0 = __ldg(reinterpret_cast<const float4*>(Sp + (size_t)k * p.dv + cc * 8));
+    const float4 x1 = __ldg(reinterpret_cast<const float4*>(Sp + (size_t)k * p.dv + cc * 8 + 4));
+    uint4 v;
+    v.x = pack_bf16x2(x0.x, x0.y);
+    v.y = pack_bf16x2(x0.z, x0.w);
+    v.z = pack_bf16x2(x1.x, x1.y);
+    v.w = pack_bf16x2(x1.z, x1.w);
+    *reinterpret_cast<uint4*>(sm + COR_OFF_B + (cc >> 3) * 16384 + sw128_offset(k, (cc & 7) * 8)) = v;
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  bool ok = have_rows;
+  if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[0], 0, s_abort, p.status));
+  if (ok && warp == 0) {
+    tc_fence_after();
+    if (elect_one()) {
+#pragma unroll
+      for (int kk = 0; kk < DK / 16; ++kk)
+        mma_bf16(tmem, kdesc(sbase + COR_OFF_A + (kk >> 2) * 16384 + (kk & 3) * 32),
+                 mndesc(sbase + COR_OFF_B + kk * 2048, 16384), idesc_bf16(128, 128, 0, 1), kk > 0);
+      mma_commit(&bars[1]);
+    }
+    __syncwarp();
+  }
+  if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[1], 0, s_abort, p.status));
+  tc_fence_after();
+  if (ok) {
+    // thread: token row 32 warp + lane of the tile, 32 columns at a time
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const size_t off = ((size_t)(tok0 + r) * p.H + h) * p.dv + col0;
+#pragma unroll 1
+    for (int piece = 0; piece < DVS / 32; ++piece) {
+      float acc[32];
+      tmem_ld32(tmem + lane_off + piece * 32, acc);
+      if (r < rows) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + off + piece * 32);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 x = dst[c];
+          float y[8] = {bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y),
+                        bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w)};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] += acc[c * 8 + e];
+          if (p.h_prev) {
+            // the loop residual on the output rounded to bf16, as loop_residual sees it
+            const uint4 hp = *reinterpret_cast<const uint4*>(p.h_prev + off + piece * 32 + c * 8);
+            const float hv[8] = {bf16_lo(hp.x), bf16_hi(hp.x), bf16_lo(hp.y), bf16_hi(hp.y),
+                                 bf16_lo(hp.z), bf16_hi(hp.z), bf16_lo(hp.w), bf16_hi(hp.w)};
+            const float* rr = p.rho + (size_t)h * p.dv + col0 + piece * 32 + c * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              y[e] = fmaf(__ldg(rr + e), hv[e], __bfloat162float(__float2bfloat16_rn(y[e])));
+          }
+          uint4 v;
+          v.x = pack_bf16x2(y[0], y[1]);
+          v.y = pack_bf16x2(y[2], y[3]);
+          v.z = pack_bf16x2(y[4], y[5]);
+          v.w = pack_bf16x2(y[6], y[7]);
+          dst[c] = v;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && have_rows && !ok) {
+    // never leave the block with a bulk copy still landing in its shared memory
+    mbar_wait_bounded(&bars[0], 0, nullptr, p.status);
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // Longest-processing-time order of varlen sequences: order[r] is the sequence
 // with the r-th largest length (ties by index), so that block r of a one-pass
 // launch (blocks are dispatched roughly in index order) takes the longest
@@ -1416,15 +1626,23 @@ __global__ void __launch_bounds__(kLptThreads)
 // Chooses the schedule of a tensor-core prefill: n_segs = 1 is one pass per
 // chain; otherwise fixed-length sequences are cut into a segment 0 of seg0_tok
 // tokens and n_segs-1 segments of seg_tok.  The cost model counts chunk steps
-// on the critical path: waves of CTAs (one CTA per SM) times chunks per CTA,
-// for the one-pass launch against the two segmented launches plus the
-// combine.  The first segmented launch holds segment 0 of every chain (run in
-// full, with outputs) and segments 1 .. n_segs-2 with one transition slice
-// each (no outputs); the second holds segments 1 .. n_segs-1.  A chunk with
-// outputs costs kOutputChunk chunk steps (it adds the output products and
-// their epilogue), so segment 0 is made shorter than the others.
+// on the critical path: waves of CTAs (one CTA per SM) times chunks per CTA.
+//   one pass: every chain in one launch.
+//   output-pass schedule: the state pass holds segment 0 of every chain (run
+//     in full, with outputs) and segments 1 .. n_segs-2 with one transition
+//     slice each (no outputs); a combine chains the start states; an output
+//     pass recomputes segments 1 .. n_segs-1 from them.
+//   corrected schedule: the state pass holds segment 0 and segments
+//     1 .. n_segs-1 with their transition slices, all with outputs (the
+//     zero-start outputs and the transition's qhat); the combine chains the
+//     start states (and the final one); a correction adds S_p^T qhat to the
+//     outputs.  Not used when o is h_prev itself: the zero-start outputs are
+//     kept in o until the correction, which must still read h_prev.
+// A chunk with outputs costs kOutputChunk chunk steps (it adds the output
+// products and their epilogue), so segment 0 is made shorter than the others
+// in the output-pass schedule.
 SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
-  SegPlan plan{1, 0, 0, 0};
+  SegPlan plan{1, 0, 0, 0, 0};
   if (!prefill_tc_supported(p) || p->n_seq <= 0 || sms <= 0) return plan;
   if (p->cu_seqlens) {
     // varlen: one pass; with more blocks than one wave, the sequences are
@@ -1436,26 +1654,37 @@ SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
   }
   if ((p->flags & GDN_SINGLE_PASS) || p->seq_len <= tc::C) return plan;
   constexpr double kOutputChunk = 1.15;   // chunk step of a CTA with outputs / without
+  constexpr double kFill = 1.5;           // pipeline fill and drain of a launch wave
+  const bool can_correct = !(p->h_prev && p->h_prev == p->o);
   const long long chains = (long long)p->n_seq * p->H;
   const long long slices = p->dv / tc::DVS;
   const int n_chunks = (p->seq_len + tc::C - 1) / tc::C;
   auto waves = [&](long long ctas) { return (double)((ctas + sms - 1) / sms); };
-  const double one_pass = waves(chains * slices) * (n_chunks * kOutputChunk + 1.5);
+  const double one_pass = waves(chains * slices) * (n_chunks * kOutputChunk + kFill);
   double best = 0.0;
-  SegPlan cand{1, 0, 0, 0};
+  SegPlan cand{1, 0, 0, 0, 0};
+  auto consider = [&](double cost, const SegPlan& c) {
+    if (cand.n_segs == 1 || cost < best) {
+      best = cost;
+      cand = c;
+    }
+  };
   for (int seg = 1; seg < n_chunks; ++seg) {
     for (int seg0 = seg; seg0 >= 1 && seg0 >= seg - 4; --seg0) {
       if (seg0 >= n_chunks) continue;
       const int P = 1 + (n_chunks - seg0 + seg - 1) / seg;
-      // a launch wave costs its longest CTA's chunks plus about 1.5 chunk steps
-      // of pipeline fill and drain; a combine step about 0.8 of a chunk step
+      // output-pass schedule; a combine step costs about 0.8 of a chunk step
       const double cost =
           waves(chains * (slices + (long long)(P - 2) * (slices + 1))) *
-              (fmax(seg0 * kOutputChunk, (double)seg) + 1.5) +
-          waves(chains * (P - 1) * slices) * (seg * kOutputChunk + 1.5) + (P > 2 ? 0.8 * (P - 2) + 0.5 : 0.0);
-      if (cand.n_segs == 1 || cost < best) {
-        best = cost;
-        cand = SegPlan{P, seg * tc::C, seg0 * tc::C, 0};
+              (fmax(seg0 * kOutputChunk, (double)seg) + kFill) +
+          waves(chains * (P - 1) * slices) * (seg * kOutputChunk + kFill) + (P > 2 ? 0.8 * (P - 2) + 0.5 : 0.0);
+      consider(cost, SegPlan{P, seg * tc::C, seg0 * tc::C, 0, 0});
+      if (can_correct && seg0 == seg) {
+        // corrected schedule: every state-pass CTA has outputs; the correction
+        // costs about 1.5 chunk steps
+        const double cc = waves(chains * (slices + (long long)(P - 1) * (slices + 1))) *
+                              (seg * kOutputChunk + kFill) + 0.8 * (P - 1) + 0.5 + 1.5;
+        consider(cc, SegPlan{P, seg * tc::C, seg0 * tc::C, 0, 1});
       }
     }
   }
@@ -1465,14 +1694,20 @@ SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Workspace of a segmented schedule: [B | M | S | qhat] with B and M for
+// n_part segments (n_segs-2 in the output-pass schedule, n_segs-1 in the
+// corrected one), start states S_1 .. S_{n_segs-1}, and for the corrected
+// schedule qhat [total_tokens][H][dk] bf16; each buffer 256-byte aligned.
 size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan) {
   if (plan.lpt) return align256((size_t)p->n_seq * sizeof(int32_t));
   if (plan.n_segs <= 1) return 0;
   const size_t sd = (size_t)p->H * tc::DK * p->dv * sizeof(float);
   const size_t md = (size_t)p->H * tc::DK * tc::DK * sizeof(float);
   const size_t n = (size_t)p->n_seq;
-  return align256(n * (plan.n_segs - 2) * sd) + align256(n * (plan.n_segs - 2) * md) +
-         align256(n * (plan.n_segs - 1) * sd);
+  const size_t n_part = plan.corrected ? plan.n_segs - 1 : plan.n_segs - 2;
+  const size_t qh = plan.corrected ? (size_t)p->total_tokens * p->H * tc::DK * 2 : 0;
+  return align256(n * n_part * sd) + align256(n * n_part * md) + align256(n * (plan.n_segs - 1) * sd) +
+         align256(qh);
 }
 
 // Launch configuration; `dependent` launches with programmatic stream
@@ -1538,6 +1773,7 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   kp.seg0_tok = 0;
   kp.Bws = kp.Mws = nullptr;
   kp.Sst = nullptr;
+  kp.qhat = nullptr;
   kp.order = nullptr;
   const long long chains = (long long)p->n_seq * p->H;
   if (plan.lpt) {
@@ -1548,24 +1784,29 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   }
   if (plan.n_segs <= 1) return tc_launch(mq, mk, mv, kp, chains * kp.n_slices, stream);
 
-  // segmented: workspace = [B_1 .. B_{P-2} | M_1 .. M_{P-2} | S_1 .. S_{P-1}]
+  // segmented: workspace = [B | M | S_1 .. S_{P-1} | qhat] (prefill_segment_workspace)
   const int P = plan.n_segs;
+  const int n_part = plan.corrected ? P - 1 : P - 2;
   const size_t sd = (size_t)p->H * tc::DK * p->dv * sizeof(float);
   const size_t md = (size_t)p->H * tc::DK * tc::DK * sizeof(float);
   char* w = static_cast<char*>(ws);
   kp.Bws = reinterpret_cast<float*>(w);
-  w += align256((size_t)p->n_seq * (P - 2) * sd);
+  w += align256((size_t)p->n_seq * n_part * sd);
   kp.Mws = reinterpret_cast<float*>(w);
-  w += align256((size_t)p->n_seq * (P - 2) * md);
+  w += align256((size_t)p->n_seq * n_part * md);
   kp.Sst = reinterpret_cast<float*>(w);
+  w += align256((size_t)p->n_seq * (P - 1) * sd);
+  kp.qhat = plan.corrected ? reinterpret_cast<__nv_bfloat16*>(w) : nullptr;
   kp.n_segs = P;
   kp.seg_tok = plan.seg_tok;
   kp.seg0_tok = plan.seg0_tok;
-  kp.mode = 1;
+  kp.mode = plan.corrected ? 3 : 1;
   gdn_status st =
-      tc_launch(mq, mk, mv, kp, chains * (kp.n_slices + (long long)(P - 2) * (kp.n_slices + 1)), stream);
+      tc_launch(mq, mk, mv, kp, chains * (kp.n_slices + (long long)n_part * (kp.n_slices + 1)), stream);
   if (st != GDN_OK) return st;
-  if (P > 2) {
+  // combine: start states S_2 .. S_{P-1} (and S_T in the corrected schedule)
+  const int n_steps = plan.corrected ? (p->S_T ? P - 1 : P - 2) : P - 2;
+  if (n_steps > 0) {
     const long long cblocks = chains * (p->dv / tc::CMB_COLS);
     if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     static std::atomic<bool> cmb_attr_set[kMaxDevices];
@@ -1573,11 +1814,42 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
       return GDN_ERR_CUDA;
     LaunchCfg lc((unsigned)cblocks, 256, tc::CMB_SMEM, stream, /*dependent=*/true);
     if (cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_combine_kernel, (const float*)kp.Bws,
-                           (const float*)kp.Mws, kp.Sst, p->H, p->dv, P) != cudaSuccess)
+                           (const float*)kp.Mws, kp.Sst, plan.corrected ? p->S_T : nullptr, p->H, p->dv,
+                           P, n_part, n_steps) != cudaSuccess)
       return GDN_ERR_CUDA;
   }
-  kp.mode = 2;
-  return tc_launch(mq, mk, mv, kp, chains * (P - 1) * kp.n_slices, stream, /*dependent=*/true);
+  if (!plan.corrected) {
+    kp.mode = 2;
+    return tc_launch(mq, mk, mv, kp, chains * (P - 1) * kp.n_slices, stream, /*dependent=*/true);
+  }
+  // correction of the outputs of segments 1 .. P-1
+  CUtensorMap mqh;
+  if (!make_map(&mqh, kp.qhat, tc::DK, p->H, p->total_tokens)) return GDN_ERR_CUDA;
+  tc::CorParams cp;
+  cp.o = kp.o;
+  cp.h_prev = kp.h_prev;
+  cp.rho = kp.rho;
+  cp.Sst = kp.Sst;
+  cp.status = status;
+  cp.H = p->H;
+  cp.dv = p->dv;
+  cp.n_slices = kp.n_slices;
+  cp.seq_len = p->seq_len;
+  cp.seg0_tok = plan.seg0_tok;
+  cp.seg_tok = plan.seg_tok;
+  cp.n_segs = P;
+  const int tps = (plan.seg_tok + tc::COR_ROWS - 1) / tc::COR_ROWS;
+  const int last_len = p->seq_len - plan.seg0_tok - (P - 2) * plan.seg_tok;
+  cp.tiles_mid = (P - 2) * tps;
+  cp.tiles_per_seq = cp.tiles_mid + (last_len + tc::COR_ROWS - 1) / tc::COR_ROWS;
+  const long long cor_blocks = chains * kp.n_slices * cp.tiles_per_seq;
+  if (cor_blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  static std::atomic<bool> cor_attr_set[kMaxDevices];
+  if (smem_attr_once(cor_attr_set, tc::gdn_segment_correct_kernel, tc::COR_SMEM) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  LaunchCfg lc((unsigned)cor_blocks, tc::COR_THREADS, tc::COR_SMEM, stream, /*dependent=*/true);
+  return cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_correct_kernel, mqh, cp) == cudaSuccess ? GDN_OK
+                                                                                              : GDN_ERR_CUDA;
 }
 
 }  // namespace gdn

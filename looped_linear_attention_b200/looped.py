@@ -48,7 +48,8 @@ class LoopedPrefill:
     def launches_per_loop(self) -> int:
         """This library's kernel launches per loop: the mixer's (its schedule)
         plus the loop residual when it is not fused."""
-        sched = B.prefill_schedule(1, self.L, self.H, self.dk, self.dv, flags=B.GDN_QK_L2NORM)
+        sched = B.prefill_schedule(1, self.L, self.H, self.dk, self.dv, flags=B.GDN_QK_L2NORM,
+                                   with_state=False)
         return sched["launches"] + (0 if self.fused_residual else 1)
 
     def run(self, h0: torch.Tensor, Wq: torch.Tensor, Wk: torch.Tensor, Wv: torch.Tensor,

@@ -97,26 +97,42 @@ def _state_set(H, dk, dv):
     return H * dk * dv * 4
 
 
+def _schedule(lib, p):
+    n, tok0, tok, launches, corr = (ctypes.c_int() for _ in range(5))
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
+                                      ctypes.byref(tok), ctypes.byref(launches),
+                                      ctypes.byref(corr)) == B.GDN_OK
+    return n.value, tok0.value, tok.value, launches.value, corr.value
+
+
+def _segmented_need(n_seq, L, H, dv, P, corrected):
+    """Workspace of a segmented schedule: B and M for segments 1 .. P-2 (output
+    pass) or 1 .. P-1 (corrected), start states for segments 1 .. P-1, and in
+    the corrected schedule qhat [tokens][H][dk] bf16; each 256-byte aligned."""
+    align = lambda x: (x + 255) // 256 * 256
+    sd, md = H * 128 * dv * 4, H * 128 * 128 * 4
+    n_part = P - 1 if corrected else P - 2
+    return (align(n_seq * n_part * sd) + align(n_seq * n_part * md) + align(n_seq * (P - 1) * sd)
+            + (align(n_seq * L * H * 128 * 2) if corrected else 0))
+
+
 def test_workspace_segmented_schedule_for_few_long_chains(lib):
     """One 4096-token sequence x 16 heads fills 16 of 148 SMs in one pass: the
-    query asks for the segmented schedule's buffers.  Segment 0 runs in full
-    from S0, so B and M (dk = dv here) are kept for segments 1 .. P-2 and start
-    states for segments 1 .. P-1, i.e. (3P - 5) state sets, P >= 2; the
-    schedule query reports the same P."""
-    p = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16)
-    sd = _state_set(16, 128, 128)
+    query asks for the corrected segmented schedule's buffers, and the schedule
+    query reports its segments and launches (state pass, combine, correction).
+    With o = h_prev (the loop residual in place) the output-pass schedule is
+    taken instead."""
+    p = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16, S_T=1 << 36)
     need = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
-    assert need > 0 and need % sd == 0
-    sets = need // sd
-    assert (sets + 5) % 3 == 0 and 2 <= (sets + 5) // 3 <= 64
-    n, tok0, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
-                                      ctypes.byref(tok), ctypes.byref(launches)) == B.GDN_OK
-    P = (sets + 5) // 3
-    assert n.value == P and tok.value % 64 == 0 and tok0.value % 64 == 0
-    assert 0 < tok0.value <= tok.value
-    assert tok0.value + (P - 2) * tok.value < 4096 <= tok0.value + (P - 1) * tok.value
-    assert launches.value == (3 if P > 2 else 2)
+    P, tok0, tok, launches, corr = _schedule(lib, p)
+    assert corr == 1 and P >= 2 and launches == 3
+    assert need == _segmented_need(1, 4096, 16, 128, P, True)
+    assert tok % 64 == 0 and tok0 % 64 == 0 and 0 < tok0 <= tok
+    assert tok0 + (P - 2) * tok < 4096 <= tok0 + (P - 1) * tok
+    p_in_place = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16, h_prev=1 << 28, rho=1 << 24)
+    P2, _, _, launches2, corr2 = _schedule(lib, p_in_place)
+    assert corr2 == 0 and P2 >= 2 and launches2 == (3 if P2 > 2 else 2)
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p_in_place)) == _segmented_need(1, 4096, 16, 128, P2, False)
 
 
 @pytest.mark.parametrize("kw", [
@@ -132,21 +148,18 @@ def test_workspace_zero_for_one_pass_schedules(lib, kw):
     kw.setdefault("total_tokens", kw["n_seq"] * kw["seq_len"])
     p = _params(**kw)
     assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
-    n, tok0, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
-                                      ctypes.byref(tok), ctypes.byref(launches)) == B.GDN_OK
-    assert (n.value, tok0.value, tok.value, launches.value) == (1, 0, 0, 1)
+    assert _schedule(lib, p) == (1, 0, 0, 1, 0)
 
 
 def test_schedule_query_rejects_what_the_call_rejects(lib):
     p = _params(dk=96)                                    # dk outside {64, 128}
     bad = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
     assert bad == ctypes.c_size_t(-1).value
-    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), None, None, None, None) != B.GDN_OK
+    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), None, None, None, None, None) != B.GDN_OK
     empty = _params(n_seq=0, seq_len=64, total_tokens=0)
     launches = ctypes.c_int(-1)
     assert lib.gdn_chunk_fwd_schedule(ctypes.byref(empty), None, None, None,
-                                      ctypes.byref(launches)) == B.GDN_OK
+                                      ctypes.byref(launches), None) == B.GDN_OK
     assert launches.value == 0
 
 
@@ -159,7 +172,7 @@ def test_varlen_workspace_holds_the_longest_first_order(lib):
         p = _params(seq_len=0, cu_seqlens=1 << 32, o=1 << 40, **kw)
         n, launches = ctypes.c_int(), ctypes.c_int()
         assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), None, None,
-                                          ctypes.byref(launches)) == B.GDN_OK
+                                          ctypes.byref(launches), None) == B.GDN_OK
         return lib.gdn_chunk_fwd_workspace(ctypes.byref(p)), n.value, launches.value
     assert query(n_seq=64, total_tokens=64 * 1000, H=16, dv=256) == (256, 1, 2)
     assert query(n_seq=1000, total_tokens=1000 * 100, H=16) == (4096, 1, 2)
@@ -262,25 +275,24 @@ def test_stacked_projection_weights_are_used_in_place():
 def test_segment_plan_covers_the_sequence(lib, n_seq, L, H, dv):
     """The planner's segments tile each sequence exactly: segment 0 of seg0_tok
     tokens, then segments of seg_tok (whole chunks of 64, segment 0 no longer
-    than the others), the last one ragged but not empty; and the workspace the
-    query asks for is exactly B and M for segments 1 .. P-2 plus start states
-    for segments 1 .. P-1, each buffer 256-byte aligned."""
-    p = _params(n_seq=n_seq, seq_len=L, total_tokens=n_seq * L, H=H, dv=dv, o=1 << 40)
-    n, tok0, tok, launches = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    assert lib.gdn_chunk_fwd_schedule(ctypes.byref(p), ctypes.byref(n), ctypes.byref(tok0),
-                                      ctypes.byref(tok), ctypes.byref(launches)) == B.GDN_OK
-    need = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
-    P = n.value
-    if P == 1:
-        assert (tok0.value, tok.value, launches.value, need) == (0, 0, 1, 0)
-        return
-    assert tok.value % 64 == 0 and tok0.value % 64 == 0 and 0 < tok0.value <= tok.value
-    assert tok0.value + (P - 2) * tok.value < L <= tok0.value + (P - 1) * tok.value
-    assert launches.value == (3 if P > 2 else 2)
-    align = lambda x: (x + 255) // 256 * 256
-    sd, md = H * 128 * dv * 4, H * 128 * 128 * 4
-    assert need == (align(n_seq * (P - 2) * sd) + align(n_seq * (P - 2) * md)
-                    + align(n_seq * (P - 1) * sd))
+    than the others), the last one ragged but not empty; the workspace the
+    query asks for is exactly that schedule's buffers; and the launch count
+    matches it (with and without a final state)."""
+    for st in (None, 1 << 36):
+        p = _params(n_seq=n_seq, seq_len=L, total_tokens=n_seq * L, H=H, dv=dv, o=1 << 40, S_T=st)
+        P, tok0, tok, launches, corr = _schedule(lib, p)
+        need = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
+        if P == 1:
+            assert (tok0, tok, launches, need, corr) == (0, 0, 1, 0, 0)
+            continue
+        assert tok % 64 == 0 and tok0 % 64 == 0 and 0 < tok0 <= tok
+        assert tok0 + (P - 2) * tok < L <= tok0 + (P - 1) * tok
+        if corr:
+            assert tok0 == tok
+            assert launches == (3 if (P > 2 or st) else 2)
+        else:
+            assert launches == (3 if P > 2 else 2)
+        assert need == _segmented_need(n_seq, L, H, dv, P, corr)
 
 
 def _bwd_params(**kw):

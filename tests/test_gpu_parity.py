@@ -201,6 +201,27 @@ def test_prefill_tc_segmented_equals_single_pass_and_oracle():
     _status_ok()
 
 
+def test_prefill_tc_corrected_schedule_with_and_without_final_state():
+    """The corrected segmented schedule (zero-start outputs of segments 1 .. P-1
+    plus qhat^T S_p from their chained start states): with a final state the
+    combine also chains S_T; without one it stops at S_{P-1}.  Both give the
+    oracle's outputs, and the same outputs bit for bit (the correction does
+    not depend on the last combine step)."""
+    wl = _wl("long_prefill", n_seq=2, H=2, seq_len=1000, random_s0=True)
+    sched = lla.prefill_schedule(2, 1000, 2, 128, 128)
+    assert sched["corrected"] == 1 and sched["n_segs"] > 2
+    assert lla.prefill_schedule(2, 1000, 2, 128, 128, with_state=False)["launches"] == 3
+    inp = W.prefill_inputs(wl, "cpu")
+    q, k, v, a, b, s0 = (inp[n].cuda() for n in ("q", "k", "v", "a", "b", "S0"))
+    o1, ST = lla.gdn_chunk_fwd(q, k, v, a, b, s0, n_seq=2)
+    o2, none = lla.gdn_chunk_fwd(q, k, v, a, b, s0, n_seq=2, return_state=False)
+    torch.cuda.synchronize()
+    _status_ok()
+    assert none is None and torch.equal(o1, o2)
+    o_ref, S_ref = _oracle_prefill(inp)
+    _check(host(o1), host(ST), o_ref, S_ref, fp32=False, inp=inp)
+
+
 def test_prefill_tc_segmented_dv256_l2norm_scale():
     """Segmented schedule with two dv slices per head (plus the transition
     slice), in-kernel L2 norm and an output scale."""

@@ -14,6 +14,10 @@ the page, not any kernel's blocking:
   ("LT2: Linear-Time Looped Transformers", §2, "LT2." paragraph: state
   S_t in R^{dk x dv}; the mixer is Gated DeltaNet, Appendix C).  The per-token
   loop is the C routine in ``gdn_oracle.c``.
+* ``kda_fwd`` / ``kda_decode`` -- the per-channel (diagonal) gate variant, the
+  KDA mixer of the LT2 mixer list (Appendix C), token by token.
+* ``output_gate`` -- the head-wise sigmoid output gate (§3, gated-attention
+  paragraph).
 * ``loop_residual`` -- h = h_tilde + rho (.) h_prev (same paragraph).
 * ``qk_l2norm`` -- per-head L2 normalisation of q and k, x / sqrt(sum x^2 + eps),
   the input recipe of the looped workloads (the pages do not print it; eps is
@@ -70,6 +74,10 @@ def _load():
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_double]
         lib.oracle_gdn_decode.restype = ctypes.c_int
+        lib.oracle_kda_fwd.argtypes = lib.oracle_gdn_fwd.argtypes
+        lib.oracle_kda_fwd.restype = ctypes.c_int
+        lib.oracle_kda_decode.argtypes = lib.oracle_gdn_decode.argtypes
+        lib.oracle_kda_decode.restype = ctypes.c_int
         lib.oracle_loop_residual.argtypes = [dp, dp, dp, dp, ctypes.c_long, ctypes.c_int]
         lib.oracle_loop_residual.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
@@ -188,6 +196,59 @@ def gdn_decode(q, k, v, a, b, S, scale: float = 1.0, gate=None):
                                    _ptr(S), _ptr(o), N, H, dk, dv, float(scale))
     if rc != 0:
         raise ValueError("oracle_gdn_decode rejected its arguments")
+    if gate is not None:
+        o = output_gate(o, gate)
+    return o, S
+
+
+def kda_fwd(q, k, v, a, b, S0=None, cu_seqlens=None, scale: float = 1.0, gate=None):
+    """Per-channel (diagonal) gate variant, the KDA mixer of the LT2 mixer list
+    ("LT2: Linear-Time Looped Transformers", Appendix C; the pages print no
+    update rule, the reading is written out in ``gdn_oracle.c``):
+    Sigma_t = (I - b_t k_t k_t^T) Diag(a_t) Sigma_{t-1} + b_t k_t v_t^T,
+    o_t = scale Sigma_t^T q_t.  As ``gdn_fwd``, with a [n_tok, H, dk]."""
+    q, k, v, a, b = (_f64(t) for t in (q, k, v, a, b))
+    n_tok, H, dk = q.shape
+    dv = v.shape[2]
+    if a.shape != (n_tok, H, dk):
+        raise ValueError("a must be [n_tok, H, dk]")
+    if cu_seqlens is None:
+        cu = np.array([0, n_tok], dtype=np.int32)
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int32))
+    n_seq = cu.shape[0] - 1
+    if int(cu[-1]) > n_tok or int(cu[0]) < 0:
+        raise ValueError("cu_seqlens out of range")
+    s0 = None if S0 is None else _f64(S0)
+    o = np.zeros((n_tok, H, dv))
+    ST = np.zeros((n_seq, H, dk, dv))
+    rc = _load().oracle_kda_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+        None if s0 is None else _ptr(s0), _ptr(o), _ptr(ST),
+        _ptr(cu, ctypes.c_int32), n_seq, H, dk, dv, float(scale))
+    if rc != 0:
+        raise ValueError("oracle_kda_fwd rejected its arguments")
+    if gate is not None:
+        o = output_gate(o, gate)
+    return o, ST
+
+
+def kda_decode(q, k, v, a, b, S, scale: float = 1.0, gate=None):
+    """One token per slot of the per-channel gate variant (a [N, H, dk]).
+    Returns (o [N, H, dv], S_new); the input is not modified."""
+    q, k, v, a, b = (_f64(t) for t in (q, k, v, a, b))
+    S = _f64(S).copy()
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    if a.shape != (N, H, dk):
+        raise ValueError("a must be [N, H, dk]")
+    o = np.zeros((N, H, dv))
+    rc = _load().oracle_kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                   _ptr(S), _ptr(o), N, H, dk, dv, float(scale))
+    if rc != 0:
+        raise ValueError("oracle_kda_decode rejected its arguments")
     if gate is not None:
         o = output_gate(o, gate)
     return o, S

@@ -270,6 +270,125 @@ int oracle_gdn_decode(const double *q, const double *k, const double *v,
     return bad ? -1 : 0;
 }
 
+/* ------------------------------------------------------------------------
+ * Per-channel (diagonal) gate variant, the KDA mixer named among the LT2
+ * mixers ("LT2: Linear-Time Looped Transformers", Appendix C; the DPLR block
+ * of §2 and Appendix B.1 in its general diagonal form).  The pages print no
+ * update rule for it; the reading taken here replaces the scalar decay a_t of
+ * the gated delta rule by a diagonal Diag(a_t), a_t in (0, 1]^{dk}, acting on
+ * the key side of the state before the delta step:
+ *
+ *     Sigma_t = (I - b_t k_t k_t^T) Diag(a_t) Sigma_{t-1} + b_t k_t v_t^T
+ *     o_t     = scale * Sigma_t^T q_t
+ *
+ * which is the gated delta rule when every entry of a_t is the same.  It is
+ * evaluated as written: Z = Diag(a) Sigma (row i scaled by a_i), y = k^T Z,
+ * Sigma_t = Z - b k y + b k v^T.  Layout of a: [n_tok][H][dk].
+ * ------------------------------------------------------------------------ */
+static void kda_token_step(double *sig, int dk, int dv,
+                           const double *q, const double *k, const double *v,
+                           const double *a, double b, double scale,
+                           double *o, double *y)
+{
+    /* Z = Diag(a) Sigma_{t-1}, in place */
+    for (int i = 0; i < dk; ++i) {
+        double *row = sig + (size_t)i * dv;
+        for (int j = 0; j < dv; ++j) row[j] *= a[i];
+    }
+    /* y = k^T Z */
+    for (int j = 0; j < dv; ++j) y[j] = 0.0;
+    for (int i = 0; i < dk; ++i) {
+        const double kc = k[i];
+        const double *row = sig + (size_t)i * dv;
+        for (int j = 0; j < dv; ++j) y[j] += kc * row[j];
+    }
+    /* Sigma_t = Z - b k y + b k v^T */
+    for (int i = 0; i < dk; ++i) {
+        const double kc = k[i];
+        double *row = sig + (size_t)i * dv;
+        for (int j = 0; j < dv; ++j) row[j] = row[j] - b * kc * y[j] + b * kc * v[j];
+    }
+    if (o) {
+        for (int j = 0; j < dv; ++j) o[j] = 0.0;
+        for (int i = 0; i < dk; ++i) {
+            const double qi = q[i];
+            const double *row = sig + (size_t)i * dv;
+            for (int j = 0; j < dv; ++j) o[j] += qi * row[j];
+        }
+        for (int j = 0; j < dv; ++j) o[j] *= scale;
+    }
+}
+
+/* Prefill of the per-channel gate variant over packed sequences (as
+ * oracle_gdn_fwd, with a [n_tok][H][dk]). */
+int oracle_kda_fwd(const double *q, const double *k, const double *v,
+                   const double *a, const double *b, const double *S0,
+                   double *o, double *ST, const int32_t *cu_seqlens,
+                   int n_seq, int H, int dk, int dv, double scale)
+{
+    if (!q || !k || !v || !a || !b || !o || !cu_seqlens) return -1;
+    if (n_seq < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    for (int s = 0; s < n_seq; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
+    const long n_chain = (long)n_seq * H;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *sig = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+        double *y = (double *)malloc(sizeof(double) * (size_t)dv);
+        if (!sig || !y) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long c = 0; c < n_chain; ++c) {
+                const int s = (int)(c / H), h = (int)(c % H);
+                const size_t sidx = ((size_t)s * H + h) * (size_t)dk * dv;
+                if (S0) memcpy(sig, S0 + sidx, sizeof(double) * (size_t)dk * dv);
+                else memset(sig, 0, sizeof(double) * (size_t)dk * dv);
+                for (int t = cu_seqlens[s]; t < cu_seqlens[s + 1]; ++t) {
+                    const size_t th = (size_t)t * H + h;
+                    kda_token_step(sig, dk, dv, q + th * dk, k + th * dk, v + th * dv,
+                                   a + th * dk, b[th], scale, o + th * dv, y);
+                }
+                if (ST) memcpy(ST + sidx, sig, sizeof(double) * (size_t)dk * dv);
+            }
+        }
+        free(sig);
+        free(y);
+    }
+    return bad ? -1 : 0;
+}
+
+/* One decode step of the per-channel gate variant for N slots x H heads
+ * (a [N][H][dk]); S is updated in place. */
+int oracle_kda_decode(const double *q, const double *k, const double *v,
+                      const double *a, const double *b, double *S, double *o,
+                      int N, int H, int dk, int dv, double scale)
+{
+    if (!q || !k || !v || !a || !b || !S || !o) return -1;
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    const long n_chain = (long)N * H;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *y = (double *)malloc(sizeof(double) * (size_t)dv);
+        if (!y) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (long c = 0; c < n_chain; ++c) {
+                kda_token_step(S + (size_t)c * dk * dv, dk, dv, q + (size_t)c * dk,
+                               k + (size_t)c * dk, v + (size_t)c * dv, a + (size_t)c * dk, b[c],
+                               scale, o + (size_t)c * dv, y);
+            }
+        }
+        free(y);
+    }
+    return bad ? -1 : 0;
+}
+
 /* Per-loop learned residual ("LT2: Linear-Time Looped Transformers", §2,
  * "LT2." paragraph): h = h_tilde + rho (.) h_prev, rho per channel.
  * h_tilde, h_prev, h_out [rows][d]; rho [d]. */

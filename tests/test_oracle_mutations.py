@@ -39,18 +39,40 @@ BWD_MUTATIONS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(BWD_MUTATIONS))
+# mistakes in the per-channel gate variant, caught by its own pins; a list of
+# (anchor, replacement) pairs is applied in order
+KDA_MUTATIONS = {
+    "kda_decay_dropped": ("row[j] *= a[i];", "row[j] *= 1.0;"),
+    "kda_decay_channel_reversed": ("row[j] *= a[i];", "row[j] *= a[dk - 1 - i];"),
+    "kda_decay_after_delta": [("row[j] *= a[i];", "row[j] *= 1.0;"),
+                              ("row[j] = row[j] - b * kc * y[j] + b * kc * v[j];",
+                               "row[j] = a[i] * (row[j] - b * kc * y[j]) + b * kc * v[j];")],
+    "kda_gate_of_first_channel": ("row[j] *= a[i];", "row[j] *= a[0];"),
+}
+
+
+def _pairs(name):
+    for table in (MUTATIONS, BWD_MUTATIONS, KDA_MUTATIONS):
+        if name in table:
+            m = table[name]
+            return m if isinstance(m, list) else [m]
+    raise KeyError(name)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(BWD_MUTATIONS) + sorted(KDA_MUTATIONS))
 def test_pins_catch_planted_mistake(tmp_path, name):
-    src, dst = MUTATIONS[name] if name in MUTATIONS else BWD_MUTATIONS[name]
-    pins = "test_oracle_pins.py" if name in MUTATIONS else "test_oracle_bwd_pins.py"
+    pins = ("test_oracle_pins.py" if name in MUTATIONS else
+            "test_oracle_bwd_pins.py" if name in BWD_MUTATIONS else "test_oracle_kda_pins.py")
     shutil.copytree(os.path.join(ROOT, "oracle"), tmp_path / "oracle",
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
     shutil.copytree(os.path.join(ROOT, "tests"), tmp_path / "tests",
                     ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutations.py"))
     cfile = tmp_path / "oracle" / "gdn_oracle.c"
     text = cfile.read_text()
-    assert text.count(src) == 1, f"mutation anchor not found once: {src!r}"
-    cfile.write_text(text.replace(src, dst))
+    for src, dst in _pairs(name):
+        assert text.count(src) == 1, f"mutation anchor not found once: {src!r}"
+        text = text.replace(src, dst)
+    cfile.write_text(text)
     env = dict(os.environ, PYTHONPATH=str(tmp_path))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         str(tmp_path / "tests" / pins)],

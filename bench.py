@@ -715,6 +715,19 @@ def run_profile_case(args):
     if args.profile == "decode":
         inp = W.decode_inputs(wl, dev)
         run = lambda: lla.gdn_decode_step(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S"])
+    elif args.profile == "looped_prefill":
+        # the looped step's mixer call: in-kernel q/k norm, the loop residual
+        # fused into the output, no final state
+        inp = W.prefill_inputs(wl, dev)
+        g = torch.Generator(device=dev).manual_seed(W.seed_for("profile", "h_prev"))
+        d = wl.H * wl.dv
+        hp = torch.randn(inp["total_tokens"], d, generator=g, device=dev).to(wl.dtype)
+        rho = 0.5 * torch.rand(d, generator=g, device=dev)
+        out = torch.empty_like(hp)
+        fl = lla.GDN_QK_L2NORM | (lla.GDN_SINGLE_PASS if args.single_pass else 0)
+        run = lambda: lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], None, None,
+                                        n_seq=inp["n_seq"], flags=fl, o=out, return_state=False,
+                                        h_prev=hp, rho=rho)
     else:
         inp = W.prefill_inputs(wl, dev)
         cu = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).to(dev)
@@ -740,7 +753,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile", choices=["tiny", "long_prefill", "varlen", "decode"], default=None,
+    ap.add_argument("--profile", choices=["tiny", "looped_prefill", "long_prefill", "varlen", "decode"],
+                    default=None,
                     help="run only this workload's kernel (for profiler captures)")
     ap.add_argument("--n-seq", type=int, default=0, help="sequences (or decode slots) for --profile")
     ap.add_argument("--single-pass", action="store_true",

@@ -71,6 +71,16 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 #define GDN_SINGLE_PASS 0x4u /* prefill: run every (sequence, head) chain in one
                               pass even when a segmented schedule would be
                               chosen (see gdn_chunk_fwd)                       */
+#define GDN_CHANNEL_GATE 0x8u /* per-channel (diagonal) decay, the KDA mixer of
+                              the LT2 mixer list ("LT2: Linear-Time Looped
+                              Transformers", Appendix C; the DPLR block of §2
+                              with a diagonal decay).  a is [tokens][H][dk]
+                              fp32, a_t in (0, 1]^{dk}, and the update reads
+                                Sigma_t = (I - b_t k_t k_t^T) Diag(a_t)
+                                          Sigma_{t-1} + b_t k_t v_t^T
+                              (the gated delta rule when a_t's entries are
+                              equal).  Prefill runs the fp32 CUDA-core KDA
+                              chunk kernel; decode both decode kernels       */
 #define GDN_TEST_WAIT_TIMEOUT 0x40000000u
                            /* test hook of the tensor-core prefill: one thread
                               waits on a barrier that nothing arrives, so the
@@ -84,7 +94,8 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
  *
  *   q, k       [total_tokens][H][dk]   io_dtype
  *   v          [total_tokens][H][dv]   io_dtype
- *   a, b       [total_tokens][H]       fp32.  a_t in (0, 1] is the decay gate,
+ *   a, b       [total_tokens][H]       fp32.  a_t in (0, 1] is the decay gate
+ *                                      ([total_tokens][H][dk] with GDN_CHANNEL_GATE),
  *                                      b_t the write strength (any finite value;
  *                                      b in [0, 2] keeps ||I - b k k^T|| <= 1 for
  *                                      unit keys, Appendix B.1).
@@ -272,9 +283,9 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_params *p, void *ws, size_t ws_bytes,
  * One decode step: one new token for each of N independent state slots (a slot
  * is one sequence x layer x loop state), H heads each.
  *   q, k [N][H][dk], v [N][H][dv], o [N][H][dv]  io_dtype
- *   a, b [N][H] fp32
+ *   a, b [N][H] fp32 (a [N][H][dk] with GDN_CHANNEL_GATE)
  *   S    [N][H][dk][dv] fp32, read and overwritten in place with S_t.
- * flags: GDN_QK_L2NORM as above.  Supported: dk in {64, 128}, dv a multiple of
+ * flags: GDN_QK_L2NORM, GDN_CHANNEL_GATE as above.  Supported: dk in {64, 128}, dv a multiple of
  * 64 up to 512.  o must not overlap S or the inputs.
  */
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v,

@@ -30,6 +30,7 @@ GDN_BF16 = 1
 GDN_QK_L2NORM = 0x1
 GDN_PRECISE = 0x2
 GDN_SINGLE_PASS = 0x4
+GDN_CHANNEL_GATE = 0x8
 GDN_TEST_WAIT_TIMEOUT = 0x40000000
 
 _DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
@@ -168,7 +169,7 @@ def gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     _check(q, "q", q.dtype)
     _check(k, "k", q.dtype, (T, H, dk))
     _check(v, "v", q.dtype, (T, H, dv))
-    _check(a, "a", torch.float32, (T, H))
+    _check(a, "a", torch.float32, (T, H, dk) if flags & GDN_CHANNEL_GATE else (T, H))
     _check(b, "b", torch.float32, (T, H))
     if cu_seqlens is not None:
         _check(cu_seqlens, "cu_seqlens", torch.int32)
@@ -319,7 +320,7 @@ def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.
     _check(q, "q", q.dtype)
     _check(k, "k", q.dtype, (N, H, dk))
     _check(v, "v", q.dtype, (N, H, dv))
-    _check(a, "a", torch.float32, (N, H))
+    _check(a, "a", torch.float32, (N, H, dk) if flags & GDN_CHANNEL_GATE else (N, H))
     _check(b, "b", torch.float32, (N, H))
     _check(S, "S", torch.float32, (N, H, dk, dv))
     _check_epilogue(gate, h_prev, rho, N, H, dv, q.dtype)

@@ -12,6 +12,7 @@ size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan);
 gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const SegPlan& plan, void* ws,
                              cudaStream_t stream);
 gdn_status launch_prefill_simt(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
+gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
                           const float* b, float* S, void* o, const float* gate, const void* h_prev,
                           const float* rho, int N, int H, int dk, int dv, gdn_dtype dt, float scale,
@@ -91,7 +92,7 @@ gdn_status validate_fwd(const gdn_fwd_params* p) {
   if (!dtype_ok(p->io_dtype)) return GDN_ERR_INVALID;
   if (p->n_seq < 0 || p->H <= 0 || p->dk <= 0 || p->dv <= 0 || p->total_tokens < 0)
     return GDN_ERR_INVALID;
-  if (p->flags & ~(GDN_QK_L2NORM | GDN_PRECISE | GDN_SINGLE_PASS | GDN_TEST_WAIT_TIMEOUT))
+  if (p->flags & ~(GDN_QK_L2NORM | GDN_PRECISE | GDN_SINGLE_PASS | GDN_CHANNEL_GATE | GDN_TEST_WAIT_TIMEOUT))
     return GDN_ERR_INVALID;
   if (!p->cu_seqlens) {
     if (p->seq_len < 0) return GDN_ERR_INVALID;
@@ -117,8 +118,9 @@ gdn_status validate_fwd(const gdn_fwd_params* p) {
     // the output may not overlap any input or either state
     const size_t tok = (size_t)p->total_tokens * p->H, eb = elem_bytes(p->io_dtype);
     const size_t sb = (size_t)p->n_seq * p->H * p->dk * p->dv * sizeof(float);
+    const size_t ab = tok * sizeof(float) * ((p->flags & GDN_CHANNEL_GATE) ? p->dk : 1);
     const Range others[] = {{p->q, tok * p->dk * eb}, {p->k, tok * p->dk * eb},
-                            {p->v, tok * p->dv * eb}, {p->a, tok * sizeof(float)},
+                            {p->v, tok * p->dv * eb}, {p->a, ab},
                             {p->b, tok * sizeof(float)}, {p->S0, sb}, {p->S_T, sb},
                             {p->gate, tok * sizeof(float)}, {p->rho, (size_t)p->H * p->dv * sizeof(float)},
                             {p->h_prev == p->o ? nullptr : p->h_prev, tok * p->dv * eb}};
@@ -238,6 +240,7 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_params* p, void* ws, size_t ws_bytes,
   unsigned* st = status_ptr();
   if (!st) return GDN_ERR_CUDA;
   if (tc) return gdn::launch_prefill_tc(p, st, plan, ws, stream);
+  if (p->flags & GDN_CHANNEL_GATE) return gdn::launch_prefill_kda(p, st, stream);
   return gdn::launch_prefill_simt(p, st, stream);
 }
 
@@ -254,7 +257,7 @@ gdn_status gdn_decode_step_looped(const void* q, const void* k, const void* v, c
                                   const void* h_prev, const float* rho, int N, int H, int dk, int dv,
                                   gdn_dtype io_dtype, float scale, unsigned flags, cudaStream_t stream) {
   if (!dtype_ok(io_dtype) || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return GDN_ERR_INVALID;
-  if (flags & ~GDN_QK_L2NORM) return GDN_ERR_INVALID;
+  if (flags & ~(GDN_QK_L2NORM | GDN_CHANNEL_GATE)) return GDN_ERR_INVALID;
   if (dk != 64 && dk != 128) return GDN_ERR_UNSUPPORTED;
   if (dv % 64 != 0 || dv > 512) return GDN_ERR_UNSUPPORTED;
   if (N == 0) return GDN_OK;
@@ -271,8 +274,9 @@ gdn_status gdn_decode_step_looped(const void* q, const void* k, const void* v, c
     // h_prev may be o itself (each element is read and then written by one thread)
     const size_t nh = (size_t)N * H, eb = elem_bytes(io_dtype);
     const Range others[] = {{S, nh * dk * dv * sizeof(float)}, {q, nh * dk * eb}, {k, nh * dk * eb},
-                            {v, nh * dv * eb}, {a, nh * sizeof(float)}, {b, nh * sizeof(float)},
-                            {gate, nh * sizeof(float)}, {rho, (size_t)H * dv * sizeof(float)},
+                            {v, nh * dv * eb},
+                            {a, nh * sizeof(float) * ((flags & GDN_CHANNEL_GATE) ? dk : 1)},
+                            {b, nh * sizeof(float)}, {gate, nh * sizeof(float)}, {rho, (size_t)H * dv * sizeof(float)},
                             {h_prev == o ? nullptr : h_prev, nh * dv * eb}};
     if (overlaps_any({o, nh * dv * eb}, others)) return GDN_ERR_INVALID;
   }

@@ -18,7 +18,13 @@
 //     head, dv block of 32*VEC columns), 128-bit accesses coalesced along dv,
 //     the state held in registers between the read and the write; lane l owns
 //     VEC consecutive columns and warp w owns DK/8 rows.
-// In both, the dk reductions go through shared memory.  Optionally the output
+// In both, the dk reductions go through shared memory.
+//
+// With GDN_CHANNEL_GATE the decay is per channel (the KDA variant:
+// Sigma_t = (I - b k k^T) Diag(a) Sigma_{t-1} + b k v^T, a in (0, 1]^{dk}, read
+// from a [slots][H][dk]): then x_k = (Diag(a) Sigma)^T k and x_q likewise,
+// u = b (v - x_k), o = scale (x_q + (k . q) u), and row r of the state becomes
+// a_r Sigma_r + k_r u^T; with a scalar gate these are the lines above.  Optionally the output
 // takes the looped block's epilogue (include/gdn.h, gdn_decode_step_looped):
 // the head-wise sigmoid gate, then the loop residual o <- round(o) + rho (.) h_prev.
 #include "common.cuh"
@@ -58,7 +64,7 @@ __device__ __forceinline__ T epilogue_out(const Epilogue& ep, float y, long long
   return from_f32<T>(fmaf(__ldg(ep.rho + h * dv + col), hp, to_f32(from_f32<T>(y))));
 }
 
-template <int DK, int VEC, typename T>
+template <int DK, int VEC, typename T, bool CG>
 __global__ void __launch_bounds__(256, 2)
     gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       const float* __restrict__ a, const float* __restrict__ b, float* S, T* o,
@@ -98,7 +104,7 @@ __global__ void __launch_bounds__(256, 2)
     nq = 1.0f / sqrtf(qq + kQkNormEps);
     nk = 1.0f / sqrtf(kk + kQkNormEps);
   }
-  const float aa = a[sh], bb = b[sh];
+  const float aa = CG ? 1.f : a[sh], bb = b[sh];
 
   // load this thread's RPW x VEC block of the state
   float s[RPW][VEC];
@@ -113,7 +119,7 @@ __global__ void __launch_bounds__(256, 2)
       s[i][0] = t.x; s[i][1] = t.y;
     }
   }
-  float kr[RPW];
+  float kr[RPW], ar[RPW];              // key entries and the decay of each row
   float xk[VEC], xq[VEC];
 #pragma unroll
   for (int c = 0; c < VEC; ++c) xk[c] = xq[c] = 0.f;
@@ -121,11 +127,14 @@ __global__ void __launch_bounds__(256, 2)
   for (int i = 0; i < RPW; ++i) {
     const int r = warp * RPW + i;
     kr[i] = to_f32(kp[r]) * nk;
+    ar[i] = CG ? __ldg(a + sh * DK + r) : aa;
     const float qr = to_f32(qp[r]) * nq;
+    const float kw = CG ? kr[i] * ar[i] : kr[i];
+    const float qw = CG ? qr * ar[i] : qr;
 #pragma unroll
     for (int c = 0; c < VEC; ++c) {
-      xk[c] = fmaf(s[i][c], kr[i], xk[c]);
-      xq[c] = fmaf(s[i][c], qr, xq[c]);
+      xk[c] = fmaf(s[i][c], kw, xk[c]);
+      xq[c] = fmaf(s[i][c], qw, xq[c]);
     }
   }
 #pragma unroll
@@ -162,15 +171,15 @@ __global__ void __launch_bounds__(256, 2)
     float* dst = Sp + (long long)i * dv;
     if constexpr (VEC == 4) {
       float4 t;
-      t.x = fmaf(aa, s[i][0], kr[i] * u[0]);
-      t.y = fmaf(aa, s[i][1], kr[i] * u[1]);
-      t.z = fmaf(aa, s[i][2], kr[i] * u[2]);
-      t.w = fmaf(aa, s[i][3], kr[i] * u[3]);
+      t.x = fmaf(ar[i], s[i][0], kr[i] * u[0]);
+      t.y = fmaf(ar[i], s[i][1], kr[i] * u[1]);
+      t.z = fmaf(ar[i], s[i][2], kr[i] * u[2]);
+      t.w = fmaf(ar[i], s[i][3], kr[i] * u[3]);
       __stcs(reinterpret_cast<float4*>(dst), t);
     } else {
       float2 t;
-      t.x = fmaf(aa, s[i][0], kr[i] * u[0]);
-      t.y = fmaf(aa, s[i][1], kr[i] * u[1]);
+      t.x = fmaf(ar[i], s[i][0], kr[i] * u[0]);
+      t.y = fmaf(ar[i], s[i][1], kr[i] * u[1]);
       __stcs(reinterpret_cast<float2*>(dst), t);
     }
   }
@@ -186,12 +195,17 @@ namespace dec {
 constexpr int DK = 128, DV = 128, THREADS = 256, STAGES = 3;
 constexpr uint32_t STATE_BYTES = DK * DV * 4;                 // 65536
 constexpr uint32_t VEC_BYTES = 128 * 2;                       // one bf16 vector
-constexpr uint32_t STAGE_BYTES = STATE_BYTES + 3 * VEC_BYTES; // state | q | k | v
-constexpr uint32_t OFF_RED = STAGES * STAGE_BYTES;            // [8 warps][2][128] fp32 partial sums
-constexpr uint32_t OFF_BAR = OFF_RED + 8 * 2 * DV * 4;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
-static_assert(SMEM_BYTES <= 232448, "decode ring exceeds shared memory");
-static_assert(STAGE_BYTES % 128 == 0, "stage alignment");
+constexpr uint32_t GATE_VEC_BYTES = DK * 4;                  // per-channel decay (fp32)
+// stage: state | q | k | v [| a, with the per-channel gate]
+template <bool CG>
+struct Ring {
+  static constexpr uint32_t STAGE_BYTES = STATE_BYTES + 3 * VEC_BYTES + (CG ? GATE_VEC_BYTES : 0);
+  static constexpr uint32_t OFF_RED = STAGES * STAGE_BYTES;   // [8 warps][2][128] fp32 partial sums
+  static constexpr uint32_t OFF_BAR = OFF_RED + 8 * 2 * DV * 4;
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
+  static_assert(SMEM_BYTES <= 232448, "decode ring exceeds shared memory");
+  static_assert(STAGE_BYTES % 128 == 0, "stage alignment");
+};
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -214,15 +228,18 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+template <bool CG>
 __global__ void __launch_bounds__(THREADS, 1)
     gdn_decode_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                              const __nv_bfloat16* __restrict__ v, const float* __restrict__ a,
                              const float* __restrict__ b, float* S, __nv_bfloat16* o, long long NH,
                              float scale, unsigned flags, unsigned* status, const Epilogue ep) {
+  using R = Ring<CG>;
+  constexpr uint32_t STAGE_BYTES = R::STAGE_BYTES;
   extern __shared__ __align__(128) uint8_t dsm[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + OFF_BAR);
-  float* red = reinterpret_cast<float*>(dsm + OFF_RED);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + OFF_BAR + 8 * STAGES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + R::OFF_BAR);
+  float* red = reinterpret_cast<float*>(dsm + R::OFF_RED);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + R::OFF_BAR + 8 * STAGES);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long first = blockIdx.x, step = gridDim.x;
   const int n_items = (first < NH) ? (int)((NH - first + step - 1) / step) : 0;
@@ -242,6 +259,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     bulk_load(st + STATE_BYTES, q + sh * DK, VEC_BYTES, bar);
     bulk_load(st + STATE_BYTES + VEC_BYTES, k + sh * DK, VEC_BYTES, bar);
     bulk_load(st + STATE_BYTES + 2 * VEC_BYTES, v + sh * DV, VEC_BYTES, bar);
+    if (CG) bulk_load(st + STATE_BYTES + 3 * VEC_BYTES, a + sh * DK, GATE_VEC_BYTES, bar);
   };
   int issued = 0;
   if (tid == 0) {
@@ -249,7 +267,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   float a_next = 0.f, b_next = 0.f;
   if (n_items > 0) {
-    a_next = __ldg(a + first);
+    a_next = CG ? 1.f : __ldg(a + first);
     b_next = __ldg(b + first);
   }
   const int r0 = warp * (DK / 8);                 // this thread: rows r0 .. r0+15, columns 4 lane .. +3
@@ -257,7 +275,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long sh = first + (long long)n * step;
     const float aa = a_next, bb = b_next;
     if (n + 1 < n_items) {                        // gates of the next item, a whole item ahead
-      a_next = __ldg(a + sh + step);
+      if (!CG) a_next = __ldg(a + sh + step);
       b_next = __ldg(b + sh + step);
     }
     uint8_t* st = dsm + (n % STAGES) * STAGE_BYTES;
@@ -267,6 +285,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(st + STATE_BYTES);
     const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(st + STATE_BYTES + VEC_BYTES);
     const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(st + STATE_BYTES + 2 * VEC_BYTES);
+    const float* sa = reinterpret_cast<const float*>(st + STATE_BYTES + 3 * VEC_BYTES);   // CG only
     // norms and k.q over the whole vectors (every warp, no block sync needed)
     float qq = 0.f, kk = 0.f, kq = 0.f;
 #pragma unroll
@@ -289,18 +308,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       nk = 1.0f / sqrtf(kk + kQkNormEps);
     }
     // this thread's 16 x 4 block of the state, and its partial x_k, x_q
-    float s[DK / 8][4], kr[DK / 8];
+    float s[DK / 8][4], kr[DK / 8], ar[DK / 8];
     float xk[4] = {0.f, 0.f, 0.f, 0.f}, xq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < DK / 8; ++i) {
       const float4 t = *reinterpret_cast<const float4*>(sS + (r0 + i) * DV + 4 * lane);
       s[i][0] = t.x, s[i][1] = t.y, s[i][2] = t.z, s[i][3] = t.w;
       kr[i] = __bfloat162float(sk[r0 + i]) * nk;
+      ar[i] = CG ? sa[r0 + i] : aa;
       const float qr = __bfloat162float(sq[r0 + i]) * nq;
+      const float kw = CG ? kr[i] * ar[i] : kr[i];
+      const float qw = CG ? qr * ar[i] : qr;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        xk[c] = fmaf(s[i][c], kr[i], xk[c]);
-        xq[c] = fmaf(s[i][c], qr, xq[c]);
+        xk[c] = fmaf(s[i][c], kw, xk[c]);
+        xq[c] = fmaf(s[i][c], qw, xq[c]);
       }
     }
     *reinterpret_cast<float4*>(red + (warp * 2 + 0) * DV + 4 * lane) = make_float4(xk[0], xk[1], xk[2], xk[3]);
@@ -343,10 +365,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int i = 0; i < DK / 8; ++i) {
       float4 t;
-      t.x = fmaf(aa, s[i][0], kr[i] * u[0]);
-      t.y = fmaf(aa, s[i][1], kr[i] * u[1]);
-      t.z = fmaf(aa, s[i][2], kr[i] * u[2]);
-      t.w = fmaf(aa, s[i][3], kr[i] * u[3]);
+      t.x = fmaf(ar[i], s[i][0], kr[i] * u[0]);
+      t.y = fmaf(ar[i], s[i][1], kr[i] * u[1]);
+      t.z = fmaf(ar[i], s[i][2], kr[i] * u[2]);
+      t.w = fmaf(ar[i], s[i][3], kr[i] * u[3]);
       *reinterpret_cast<float4*>(sS + (r0 + i) * DV + 4 * lane) = t;
     }
     fence_proxy_async_smem();
@@ -373,7 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 }  // namespace dec
 
-template <int DK, typename T>
+template <int DK, typename T, bool CG>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* a,
                                    const float* b, float* S, void* o, long long NH, int dv,
                                    float scale, unsigned flags, const Epilogue& ep, cudaStream_t stream) {
@@ -383,12 +405,42 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, 
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   if (wide)
-    gdn_decode_kernel<DK, 4, T><<<(unsigned)blocks, 256, 0, stream>>>(
+    gdn_decode_kernel<DK, 4, T, CG><<<(unsigned)blocks, 256, 0, stream>>>(
         (const T*)q, (const T*)k, (const T*)v, a, b, S, (T*)o, dv, scale, flags, ep);
   else
-    gdn_decode_kernel<DK, 2, T><<<(unsigned)blocks, 256, 0, stream>>>(
+    gdn_decode_kernel<DK, 2, T, CG><<<(unsigned)blocks, 256, 0, stream>>>(
         (const T*)q, (const T*)k, (const T*)v, a, b, S, (T*)o, dv, scale, flags, ep);
   return cudaGetLastError();
+}
+
+template <bool CG>
+static cudaError_t launch_stream(const void* q, const void* k, const void* v, const float* a,
+                                 const float* b, float* S, void* o, long long NH, float scale,
+                                 unsigned flags, int num_sms, unsigned* status, const Epilogue& ep,
+                                 cudaStream_t stream) {
+  static std::atomic<bool> attr_set[kMaxDevices];
+  const cudaError_t e = smem_attr_once(attr_set, dec::gdn_decode_stream_kernel<CG>, dec::Ring<CG>::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const long long blocks = NH < num_sms ? NH : num_sms;
+  dec::gdn_decode_stream_kernel<CG><<<(unsigned)blocks, dec::THREADS, dec::Ring<CG>::SMEM_BYTES, stream>>>(
+      (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a, b, S,
+      (__nv_bfloat16*)o, NH, scale, flags, status, ep);
+  return cudaGetLastError();
+}
+
+template <bool CG>
+static cudaError_t launch_decode_cg(const void* q, const void* k, const void* v, const float* a,
+                                    const float* b, float* S, void* o, long long NH, int dk, int dv,
+                                    gdn_dtype dt, float scale, unsigned flags, int num_sms,
+                                    unsigned* status, const Epilogue& ep, cudaStream_t stream) {
+  if (dt == GDN_BF16 && dk == dec::DK && dv == dec::DV && status)
+    return launch_stream<CG>(q, k, v, a, b, S, o, NH, scale, flags, num_sms, status, ep, stream);
+  if (dt == GDN_BF16) {
+    return dk == 128 ? launch_decode_t<128, __nv_bfloat16, CG>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream)
+                     : launch_decode_t<64, __nv_bfloat16, CG>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream);
+  }
+  return dk == 128 ? launch_decode_t<128, float, CG>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream)
+                   : launch_decode_t<64, float, CG>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream);
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
@@ -398,22 +450,9 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
   const long long NH = (long long)N * H;
   const Epilogue ep{gate, h_prev, rho, H};
   if (NH == 0) return cudaSuccess;
-  if (dt == GDN_BF16 && dk == dec::DK && dv == dec::DV && status) {
-    static std::atomic<bool> attr_set[kMaxDevices];
-    const cudaError_t e = smem_attr_once(attr_set, dec::gdn_decode_stream_kernel, dec::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    const long long blocks = NH < num_sms ? NH : num_sms;
-    dec::gdn_decode_stream_kernel<<<(unsigned)blocks, dec::THREADS, dec::SMEM_BYTES, stream>>>(
-        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a, b, S,
-        (__nv_bfloat16*)o, NH, scale, flags, status, ep);
-    return cudaGetLastError();
-  }
-  if (dt == GDN_BF16) {
-    return dk == 128 ? launch_decode_t<128, __nv_bfloat16>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream)
-                     : launch_decode_t<64, __nv_bfloat16>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream);
-  }
-  return dk == 128 ? launch_decode_t<128, float>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream)
-                   : launch_decode_t<64, float>(q, k, v, a, b, S, o, NH, dv, scale, flags, ep, stream);
+  if (flags & GDN_CHANNEL_GATE)
+    return launch_decode_cg<true>(q, k, v, a, b, S, o, NH, dk, dv, dt, scale, flags, num_sms, status, ep, stream);
+  return launch_decode_cg<false>(q, k, v, a, b, S, o, NH, dk, dv, dt, scale, flags, num_sms, status, ep, stream);
 }
 
 }  // namespace gdn

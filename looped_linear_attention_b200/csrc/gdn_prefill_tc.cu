@@ -1261,7 +1261,7 @@ static bool make_map(CUtensorMap* m, const void* base, int width, int H, int tot
 
 bool prefill_tc_supported(const gdn_fwd_params* p) {
   return p->io_dtype == GDN_BF16 && p->dk == tc::DK && p->dv % tc::DVS == 0 &&
-         !(p->flags & GDN_PRECISE);
+         !(p->flags & (GDN_PRECISE | GDN_CHANNEL_GATE));
 }
 
 // ------------------------------------------------------------------ segments

@@ -109,6 +109,18 @@ def gates(n_tok: int, H: int, device, *parts, dtype=torch.float32):
     return a.to(dtype), b.to(dtype)
 
 
+def channel_gates(n_tok: int, H: int, dk: int, device, *parts):
+    """Per-channel decay a [n_tok, H, dk] = exp(-softplus(N(-3, 1))) drawn for
+    every channel (the scalar gate's distribution, one draw per channel) and
+    b = sigmoid(N(0, 1)) [n_tok, H], for the per-channel (KDA) variant."""
+    g = _gen(device, *parts, "channel-gates")
+    x = torch.randn(n_tok, H, dk, generator=g, device=device, dtype=torch.float32) - 3.0
+    sp = torch.clamp(x, min=0) + torch.log1p(torch.exp(-x.abs()))
+    a = torch.exp(-sp)
+    b = torch.sigmoid(torch.randn(n_tok, H, generator=g, device=device, dtype=torch.float32))
+    return a, b
+
+
 def qkv(n_tok: int, H: int, dk: int, dv: int, dtype, normalize: bool, device,
         *parts, chunk_tokens: int = 1 << 16):
     """q, k [n_tok, H, dk] and v [n_tok, H, dv] in `dtype` (drawn in fp32,

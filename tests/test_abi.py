@@ -399,3 +399,20 @@ def test_decode_looped_rejects_bad_epilogue_on_host(lib, args):
                                     base["H"], base["dk"], base["dv"], base["dt"], base["scale"],
                                     base["flags"], None)
     assert st == B.GDN_ERR_INVALID
+
+
+def test_channel_gate_flag_validation(lib):
+    """GDN_CHANNEL_GATE (per-channel decay, a [tokens][H][dk]) is accepted by
+    prefill and decode; the output may not overlap any of a's dk-wide rows,
+    and the prefill takes no segmented schedule (no workspace)."""
+    p = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16, flags=B.GDN_CHANNEL_GATE)
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
+    assert _schedule(lib, p) == (1, 0, 0, 1, 0)
+    # a of 64 tokens x 2 heads x 128 channels x 4 B = 64 KiB: an output 32 KiB past it overlaps
+    bad = _params(a=1 << 20, o=(1 << 20) + (32 << 10), flags=B.GDN_CHANNEL_GATE)
+    assert lib.gdn_chunk_fwd(ctypes.byref(bad), None, 0, None) == B.GDN_ERR_INVALID
+    ok = _params(a=1 << 20, o=(1 << 20) + (32 << 10))               # scalar a: 512 B, no overlap
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(ok)) != ctypes.c_size_t(-1).value
+    st = lib.gdn_decode_step(16, 32, 48, 1 << 20, 80, 1 << 24, (1 << 20) + 2048, 4, 2, 128, 128,
+                             B.GDN_BF16, 1.0, B.GDN_CHANNEL_GATE, None)
+    assert st == B.GDN_ERR_INVALID                                 # o inside a's 4 KiB

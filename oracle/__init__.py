@@ -16,6 +16,8 @@ the page, not any kernel's blocking:
   loop is the C routine in ``gdn_oracle.c``.
 * ``kda_fwd`` / ``kda_decode`` -- the per-channel (diagonal) gate variant, the
   KDA mixer of the LT2 mixer list (Appendix C), token by token.
+* ``swa_fwd`` -- sliding-window causal softmax attention, the window mixer
+  of the hybrid loops (§2, Appendix C), one query at a time.
 * ``output_gate`` -- the head-wise sigmoid output gate (§3, gated-attention
   paragraph).
 * ``loop_residual`` -- h = h_tilde + rho (.) h_prev (same paragraph).
@@ -48,7 +50,7 @@ def build(force: bool = False) -> str:
             os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
-               "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC]
+               "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -78,6 +80,9 @@ def _load():
         lib.oracle_kda_fwd.restype = ctypes.c_int
         lib.oracle_kda_decode.argtypes = lib.oracle_gdn_decode.argtypes
         lib.oracle_kda_decode.restype = ctypes.c_int
+        lib.oracle_swa_fwd.argtypes = [dp, dp, dp, dp, ip, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double]
+        lib.oracle_swa_fwd.restype = ctypes.c_int
         lib.oracle_loop_residual.argtypes = [dp, dp, dp, dp, ctypes.c_long, ctypes.c_int]
         lib.oracle_loop_residual.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
@@ -252,6 +257,31 @@ def kda_decode(q, k, v, a, b, S, scale: float = 1.0, gate=None):
     if gate is not None:
         o = output_gate(o, gate)
     return o, S
+
+
+def swa_fwd(q, k, v, window: int, cu_seqlens=None, scale=None):
+    """Sliding-window causal softmax attention ("LT2: Linear-Time Looped
+    Transformers", §2 and Appendix C): query t attends to the keys
+    [t - window + 1, t] of its own sequence.  q, k [n_tok, H, d], v [n_tok, H, dv];
+    scale defaults to 1 / sqrt(d).  Returns o [n_tok, H, dv]."""
+    q, k, v = (_f64(t) for t in (q, k, v))
+    n_tok, H, d = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is None:
+        cu = np.array([0, n_tok], dtype=np.int32)
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int32))
+    if int(cu[-1]) > n_tok or int(cu[0]) < 0:
+        raise ValueError("cu_seqlens out of range")
+    sc = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    o = np.zeros((n_tok, H, dv))
+    rc = _load().oracle_swa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu, ctypes.c_int32),
+                                cu.shape[0] - 1, H, d, dv, int(window), sc)
+    if rc != 0:
+        raise ValueError("oracle_swa_fwd rejected its arguments")
+    return o
 
 
 def loop_residual(h_tilde, h_prev, rho):

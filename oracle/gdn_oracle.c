@@ -28,6 +28,7 @@
  *   S0, ST [n_seq][H][dk][dv] (S0 may be NULL = zeros; ST may be NULL)
  *   cu_seqlens int32 [n_seq+1], token offsets of each packed sequence.
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -266,6 +267,69 @@ int oracle_gdn_decode(const double *q, const double *k, const double *v,
             }
         }
         free(y);
+    }
+    return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Sliding-window softmax attention, the window mixer of the hybrid LT2 loops
+ * ("LT2: Linear-Time Looped Transformers", §2: a sliding-window block of
+ * window w; Appendix C: windowed variants attend to the w - 1 previous
+ * tokens and the token itself, no future tokens).  For query t of a sequence
+ * starting at t0, over the keys j in [max(t0, t - w + 1), t]:
+ *
+ *     s_j = scale q_t . k_j,   p_j = exp(s_j - max_j s_j),
+ *     o_t = sum_j p_j v_j / sum_j p_j
+ *
+ * evaluated as written, one query at a time, in double precision.
+ * Layouts: q, k [n_tok][H][d], v, o [n_tok][H][dv].
+ * ------------------------------------------------------------------------ */
+int oracle_swa_fwd(const double *q, const double *k, const double *v, double *o,
+                   const int32_t *cu_seqlens, int n_seq, int H, int d, int dv,
+                   int window, double scale)
+{
+    if (!q || !k || !v || !o || !cu_seqlens) return -1;
+    if (n_seq < 0 || H <= 0 || d <= 0 || dv <= 0 || window < 1) return -1;
+    for (int s = 0; s < n_seq; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
+    const long n_tok = cu_seqlens[n_seq] - cu_seqlens[0];
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *sc = (double *)malloc(sizeof(double) * (size_t)window);
+        if (!sc) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long u = 0; u < n_tok * H; ++u) {
+                const long t = cu_seqlens[0] + u / H;
+                const int h = (int)(u % H);
+                int s = 0;
+                while (cu_seqlens[s + 1] <= t) ++s;
+                const long lo = (t - window + 1 > cu_seqlens[s]) ? t - window + 1 : cu_seqlens[s];
+                const double *qt = q + ((size_t)t * H + h) * d;
+                double m = -1.0 / 0.0;
+                for (long j = lo; j <= t; ++j) {
+                    const double *kj = k + ((size_t)j * H + h) * d;
+                    double acc = 0.0;
+                    for (int c = 0; c < d; ++c) acc += qt[c] * kj[c];
+                    sc[j - lo] = scale * acc;
+                    if (sc[j - lo] > m) m = sc[j - lo];
+                }
+                double l = 0.0;
+                double *ot = o + ((size_t)t * H + h) * dv;
+                for (int c = 0; c < dv; ++c) ot[c] = 0.0;
+                for (long j = lo; j <= t; ++j) {
+                    const double p = exp(sc[j - lo] - m);
+                    l += p;
+                    const double *vj = v + ((size_t)j * H + h) * dv;
+                    for (int c = 0; c < dv; ++c) ot[c] += p * vj[c];
+                }
+                for (int c = 0; c < dv; ++c) ot[c] /= l;
+            }
+        }
+        free(sc);
     }
     return bad ? -1 : 0;
 }

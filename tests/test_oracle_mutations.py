@@ -51,18 +51,29 @@ KDA_MUTATIONS = {
 }
 
 
+# mistakes in the sliding-window attention, caught by its own pins
+SWA_MUTATIONS = {
+    "swa_window_one_wider": ("(t - window + 1 > cu_seqlens[s]) ? t - window + 1",
+                             "(t - window > cu_seqlens[s]) ? t - window"),
+    "swa_scale_dropped": ("sc[j - lo] = scale * acc;", "sc[j - lo] = acc;"),
+    "swa_not_normalised": ("for (int c = 0; c < dv; ++c) ot[c] /= l;", "(void)l;"),
+}
+
+
 def _pairs(name):
-    for table in (MUTATIONS, BWD_MUTATIONS, KDA_MUTATIONS):
+    for table in (MUTATIONS, BWD_MUTATIONS, KDA_MUTATIONS, SWA_MUTATIONS):
         if name in table:
             m = table[name]
             return m if isinstance(m, list) else [m]
     raise KeyError(name)
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(BWD_MUTATIONS) + sorted(KDA_MUTATIONS))
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(BWD_MUTATIONS) + sorted(KDA_MUTATIONS)
+                         + sorted(SWA_MUTATIONS))
 def test_pins_catch_planted_mistake(tmp_path, name):
     pins = ("test_oracle_pins.py" if name in MUTATIONS else
-            "test_oracle_bwd_pins.py" if name in BWD_MUTATIONS else "test_oracle_kda_pins.py")
+            "test_oracle_bwd_pins.py" if name in BWD_MUTATIONS else
+            "test_oracle_kda_pins.py" if name in KDA_MUTATIONS else "test_oracle_swa_pins.py")
     shutil.copytree(os.path.join(ROOT, "oracle"), tmp_path / "oracle",
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
     shutil.copytree(os.path.join(ROOT, "tests"), tmp_path / "tests",

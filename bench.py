@@ -323,6 +323,10 @@ def run_ours(args, rank, world, local):
         torch.cuda.empty_cache()
         extras["backward"] = bench_backward(dev, args, peaks, world)
         torch.cuda.empty_cache()
+        extras["swa"] = bench_swa(dev, args, peaks, world)
+        torch.cuda.empty_cache()
+        extras["kda"] = bench_kda(dev, args, peaks, world)
+        torch.cuda.empty_cache()
 
     st = lla.gdn_get_device_status()
     if st != lla.GDN_OK:
@@ -339,6 +343,10 @@ def run_ours(args, rank, world, local):
             extras["decode"]["cpu_baseline"] = cpu_baseline_decode()
         if "backward" in extras:
             extras["backward"]["cpu_baseline"] = cpu_baseline_backward()
+        if "swa" in extras:
+            extras["swa"]["cpu_baseline"] = cpu_baseline_swa()
+        if "kda" in extras:
+            extras["kda"]["cpu_baseline"] = cpu_baseline_kda()
 
     line = {
         "metric": METRIC,
@@ -497,6 +505,98 @@ def bench_decode(wl, dev, args, peaks, world):
            "note": "one step = one token for 256 sequences x 24 layers x 4 loops (all slots)"}
     del inp, o
     return res
+
+
+def swa_flops(lengths, window, H, d=128, dv=128):
+    """Algorithmic FLOPs of sliding-window attention: for every query, 2 d
+    (q . k) and 2 dv (p v) per key in its window."""
+    import numpy as np
+    keys = 0
+    for L in lengths:
+        t = np.arange(L)
+        keys += int(np.minimum(t + 1, window).sum())
+    return keys * H * (2 * d + 2 * dv)
+
+
+def bench_swa(dev, args, peaks, world, window=2048, L=4096, H=16):
+    """Sliding-window attention of the hybrid loops at the 1.3B setting
+    (w = 2048) on the looped workload's shape (L = 4096, 16 heads of 128),
+    T = 4 loops per step; tensor-bound: achieved algorithmic TFLOP/s against
+    the measured bf16 peak."""
+    import torch
+    import looped_linear_attention_b200 as lla
+    from looped_linear_attention_b200 import workloads as W
+    q, k, v = W.qkv(L, H, 128, 128, torch.bfloat16, False, dev, "bench", "swa")
+    o = torch.empty_like(v)
+    loops = 4
+
+    def step():
+        for _ in range(loops):
+            lla.swa_fwd(q, k, v, window, o=o)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    n = max(1, args.steps)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        e0.record()
+        for _ in range(n):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n
+    flops = swa_flops([L], window, H)
+    tflops = flops * loops / t / 1e12
+    return {"tokens_per_s": world * L / t, "ms_per_step": t * 1e3, "loops": loops, "window": window,
+            "tokens": L, "heads": H, "d": 128, "achieved_tflops": tflops,
+            "frac_of_bf16_peak": tflops / peaks["bf16_tflops"], "peak_kind": "burst (kernel timed alone)",
+            "algorithmic_flops_per_launch": flops, "clocks": clocks.summary(),
+            "kernel": "swa_fwd_kernel (tcgen05 S = Q K^T and O += P V, windowed online softmax)"}
+
+
+def bench_kda(dev, args, peaks, world, L=4096, H=16):
+    """The per-channel (diagonal) gate variant, KDA, on the looped workload's
+    mixer shape (L = 4096, 16 heads, dk = dv = 128, bf16, in-kernel q/k norm),
+    T = 4 loops per step; HBM roofline as the scalar-gate prefill, with a at
+    dk floats per token and head."""
+    import dataclasses
+    import torch
+    import looped_linear_attention_b200 as lla
+    from looped_linear_attention_b200 import workloads as W
+    wl = dataclasses.replace(W.WORKLOADS["looped_prefill"], name="kda")
+    inp = W.prefill_inputs(wl, dev)
+    a, b = W.channel_gates(L, H, 128, dev, "bench", "kda")
+    o = torch.empty(L, H, 128, dtype=torch.bfloat16, device=dev)
+    loops = 4
+    fl = lla.GDN_QK_L2NORM | lla.GDN_CHANNEL_GATE
+
+    def step():
+        for _ in range(loops):
+            lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], a, b, None, flags=fl, o=o, return_state=False)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    n = max(1, min(args.steps, 5))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        e0.record()
+        for _ in range(n):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n
+    nbytes = (prefill_bytes_per_token_head(128, 128) + 4 * 127) * L * H   # a: dk floats, not one
+    gbs = nbytes / (t / loops) / 1e9
+    return {"tokens_per_s": world * L / t, "ms_per_step": t * 1e3, "loops": loops, "tokens": L, "heads": H,
+            "achieved_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
+            "clocks": clocks.summary(),
+            "kernel": "gdn_prefill_kda_kernel (first path: fp32 CUDA cores, one CTA per (sequence, head, 64 columns))"}
 
 
 def bench_backward(dev, args, peaks, world):
@@ -665,6 +765,51 @@ def cpu_baseline_decode(seconds_target: float = 4.0, n_slots: int = 256):
                       f"scaled to the whole step (x {wl.n_seq // n_slots}); fp64 C oracle (OpenMP)"}
 
 
+def cpu_baseline_swa(seconds_target: float = 3.0, window: int = 2048, L: int = 4096, heads: int = 2):
+    """The oracle's sliding-window attention on `heads` of the 16 heads of the
+    swa workload (L = 4096, w = 2048), scaled to all heads and T = 4 loops."""
+    import torch
+    import oracle
+    from looped_linear_attention_b200 import workloads as W
+    q, k, v = W.qkv(L, heads, 128, 128, torch.bfloat16, False, "cpu", "bench", "swa", "cpu")
+    t0 = time.perf_counter()
+    runs = 0
+    while True:
+        oracle.swa_fwd(q, k, v, window)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el > seconds_target or runs >= 20:
+            break
+    step_s = el / runs * (16 / heads) * 4
+    return {"value": L / step_s, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{heads} of 16 heads, L = {L}, w = {window}, {runs} run(s), {el:.1f} s; scaled to "
+                      f"16 heads and 4 loops; fp64 C oracle (OpenMP)"}
+
+
+def cpu_baseline_kda(seconds_target: float = 3.0, L: int = 4096):
+    """The oracle's per-channel gate variant on the kda workload (all 16
+    heads, L = 4096), one loop, scaled to T = 4 loops."""
+    import dataclasses
+    import numpy as np
+    import oracle
+    from looped_linear_attention_b200 import workloads as W
+    wl = dataclasses.replace(W.WORKLOADS["looped_prefill"], name="kda")
+    inp = W.prefill_inputs(wl, "cpu")
+    a, b = W.channel_gates(L, 16, 128, "cpu", "bench", "kda")
+    q, k = oracle.qk_l2norm(inp["q"]), oracle.qk_l2norm(inp["k"])
+    t0 = time.perf_counter()
+    runs = 0
+    while True:
+        oracle.kda_fwd(q, k, inp["v"], a, b)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el > seconds_target or runs >= 20:
+            break
+    return {"value": L / (4 * el / runs), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{L} tokens x 16 heads, one loop, {runs} run(s), {el:.1f} s; scaled to 4 loops; "
+                      f"fp64 C oracle (OpenMP)"}
+
+
 def run_reference(args, rank, world):
     """CPU oracle arm: rank 0 only; every step is the whole looped-prefill
     configuration (the 4096-token sequence, all 4 loops), as in cpu_baseline."""
@@ -708,11 +853,17 @@ def run_profile_case(args):
     from looped_linear_attention_b200 import workloads as W
     import dataclasses
     torch.cuda.set_device(0)
-    wl = W.WORKLOADS[args.profile]
+    wl = W.WORKLOADS.get(args.profile, W.WORKLOADS["looped_prefill"])
     if args.n_seq:
         wl = dataclasses.replace(wl, n_seq=args.n_seq)
     dev = torch.device("cuda", 0)
-    if args.profile == "decode":
+    if args.profile == "swa":
+        # sliding-window attention, w = 2048, on the looped workload's shape
+        q, k, v = W.qkv(4096, 16, 128, 128, torch.bfloat16, False, dev, "bench", "swa")
+        o = torch.empty_like(v)
+        run = lambda: lla.swa_fwd(q, k, v, 2048, o=o)
+        wl = W.WORKLOADS["looped_prefill"]
+    elif args.profile == "decode":
         inp = W.decode_inputs(wl, dev)
         run = lambda: lla.gdn_decode_step(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["S"])
     elif args.profile == "looped_prefill":
@@ -753,7 +904,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile", choices=["tiny", "looped_prefill", "long_prefill", "varlen", "decode"],
+    ap.add_argument("--profile", choices=["tiny", "looped_prefill", "long_prefill", "varlen", "decode", "swa"],
                     default=None,
                     help="run only this workload's kernel (for profiler captures)")
     ap.add_argument("--n-seq", type=int, default=0, help="sequences (or decode slots) for --profile")

@@ -316,6 +316,38 @@ gdn_status loop_residual(const void *h_tilde, const void *h_prev, const float *r
                          void *h_out, int64_t rows, int d, gdn_dtype io_dtype,
                          cudaStream_t stream);
 
+/*
+ * Sliding-window causal softmax attention, the window mixer of the hybrid LT2
+ * loops ("LT2: Linear-Time Looped Transformers", §2: a sliding-window block of
+ * window w, whose receptive field grows to T w over T loops; Appendix C: the
+ * windowed variants attend to the w - 1 previous tokens and the token itself,
+ * none after it).  For query t of a sequence starting at t0, over the keys
+ * j in [max(t0, t - w + 1), t]:
+ *     o_t = sum_j softmax_j(scale q_t . k_j) v_j
+ *
+ *   q, k       [total_tokens][H][d]   bf16
+ *   v, o       [total_tokens][H][dv]  bf16 (o written; must not overlap q, k, v)
+ *   cu_seqlens device int32 [n_seq+1] token offsets, or NULL: n_seq sequences of
+ *              seq_len tokens each (total_tokens = n_seq * seq_len).
+ *   max_seq_len  with cu_seqlens: no sequence is longer (the grid is sized by
+ *              it; a longer sequence records GDN_ERR_INVALID in the device
+ *              status word and loses its last queries).  Ignored without.
+ *   window     w >= 1 (w >= a sequence's length gives full causal attention).
+ *   scale      score scale (1/sqrt(d) is the usual one).
+ * Supported: bf16, d = dv = 128, H >= 1.  One launch; tensor cores (tcgen05)
+ * for Q K^T and P V.  Async on `stream`; nothing allocated.
+ */
+typedef struct {
+    const void *q, *k, *v;
+    void *o;
+    const int32_t *cu_seqlens;
+    int n_seq, seq_len, max_seq_len, total_tokens, H, d, dv, window;
+    gdn_dtype io_dtype;
+    float scale;
+} swa_params;
+
+gdn_status swa_fwd(const swa_params *p, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char *gdn_status_string(gdn_status s);
 

@@ -8,6 +8,7 @@ This package is its thin Python binding plus the seeded workload generators:
     gdn_decode_step  one token per state slot, in-place state update
     GDN_CHANNEL_GATE flag: the per-channel (diagonal) gate variant, KDA
     loop_residual    h = h_tilde + rho (.) h_prev
+    swa_fwd          sliding-window causal softmax attention (the hybrid loops' window mixer)
     LoopedPrefill    T loops of projection -> GDN -> loop residual
     HostPipeline     looped-prefill steps on pinned host buffers, copies overlapped
 
@@ -18,11 +19,12 @@ from ._binding import (GDN_BF16, GDN_ERR_CUDA, GDN_ERR_INVALID, GDN_ERR_TIMEOUT,
                        GDN_QK_L2NORM, GDN_SINGLE_PASS, GDN_CHANNEL_GATE, GDN_TEST_WAIT_TIMEOUT, GdnError, gdn_chunk_bwd,
                        gdn_chunk_fwd, gdn_decode_step,
                        gdn_get_device_status, library, loop_residual, prefill_schedule, prefill_workspace_bytes,
-                       status_string, version)
+                       status_string, swa_fwd, version)
 from .looped import HostPipeline, LoopedPrefill, stack_weights
 
 __all__ = [
-    "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "loop_residual", "gdn_get_device_status",
+    "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "loop_residual", "swa_fwd",
+    "gdn_get_device_status",
     "prefill_schedule", "prefill_workspace_bytes",
     "LoopedPrefill", "HostPipeline", "stack_weights", "GdnError", "library", "status_string", "version",
     "GDN_OK", "GDN_ERR_INVALID", "GDN_ERR_UNSUPPORTED", "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT",

@@ -68,6 +68,16 @@ class gdn_bwd_params(ctypes.Structure):
     ]
 
 
+class swa_params(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("o", ctypes.c_void_p),
+        ("cu_seqlens", ctypes.c_void_p),
+        ("n_seq", ctypes.c_int), ("seq_len", ctypes.c_int), ("max_seq_len", ctypes.c_int),
+        ("total_tokens", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("dv", ctypes.c_int),
+        ("window", ctypes.c_int), ("io_dtype", ctypes.c_int), ("scale", ctypes.c_float),
+    ]
+
+
 _lib = None
 
 
@@ -100,6 +110,8 @@ def library() -> ctypes.CDLL:
         lib.gdn_decode_step_looped.restype = i32
         lib.loop_residual.argtypes = [vp, vp, vp, vp, ctypes.c_int64, i32, i32, vp]
         lib.loop_residual.restype = i32
+        lib.swa_fwd.argtypes = [ctypes.POINTER(swa_params), vp]
+        lib.swa_fwd.restype = i32
         lib.gdn_status_string.argtypes = [i32]
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_get_device_status.argtypes = [vp]
@@ -364,6 +376,42 @@ def loop_residual(h_tilde: torch.Tensor, h_prev: torch.Tensor, rho: torch.Tensor
     if st != GDN_OK:
         raise GdnError(st, "loop_residual")
     return out
+
+
+def swa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int,
+            cu_seqlens: Optional[torch.Tensor] = None, *, n_seq: Optional[int] = None,
+            max_seq_len: Optional[int] = None, scale: Optional[float] = None,
+            o: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Sliding-window causal softmax attention (see swa_fwd in include/gdn.h).
+
+    q, k: [T, H, d]; v: [T, H, dv] bf16; cu_seqlens int32 [n_seq+1] on the
+    device with max_seq_len (defaults to T), or None with n_seq sequences of
+    T // n_seq tokens; scale defaults to 1/sqrt(d). Returns o [T, H, dv]."""
+    T, H, d = q.shape
+    dv = v.shape[2]
+    _check(q, "q", torch.bfloat16)
+    _check(k, "k", torch.bfloat16, (T, H, d))
+    _check(v, "v", torch.bfloat16, (T, H, dv))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        ns, seq_len = cu_seqlens.numel() - 1, 0
+        msl = T if max_seq_len is None else int(max_seq_len)
+    else:
+        ns = 1 if n_seq is None else int(n_seq)
+        if ns <= 0 or T % ns != 0:
+            raise ValueError("without cu_seqlens, the token count must be n_seq * seq_len")
+        seq_len, msl = T // ns, T // ns
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=q.dtype, device=q.device)
+    else:
+        _check(o, "o", q.dtype, (T, H, dv))
+    sc = float(d) ** -0.5 if scale is None else float(scale)
+    p = swa_params(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), ns, seq_len, msl, T, H, d, dv,
+                   int(window), GDN_BF16, sc)
+    st = library().swa_fwd(ctypes.byref(p), _stream_ptr(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "swa_fwd")
+    return o
 
 
 def gdn_get_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:

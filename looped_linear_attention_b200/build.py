@@ -43,7 +43,8 @@ def _stale(out: str, deps) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "gdn.h")]
+    deps = (sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
+            + glob.glob(os.path.join(INCLUDE, "*.h")))
     if not force and not _stale(LIB_PATH, deps):
         return LIB_PATH
     tmp = LIB_PATH + f".tmp{os.getpid()}"
@@ -69,7 +70,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
 # Kernels that drive tcgen05 / tensor memory must not spill registers: spills
 # around asynchronously written tensor-memory load registers were the one
 # difference between faulting and clean builds of the prefill kernel.
-SPILL_FREE_KERNELS = ("gdn_prefill_tc_kernel",)
+SPILL_FREE_KERNELS = ("gdn_prefill_tc_kernel", "gdn_segment_correct_kernel", "swa_fwd_kernel")
 
 
 def check_no_spills(ptxas_log: str):

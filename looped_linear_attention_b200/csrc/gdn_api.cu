@@ -20,6 +20,7 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
 cudaError_t launch_loop_residual(const void* h_tilde, const void* h_prev, const float* rho,
                                  void* h_out, int64_t rows, int d, gdn_dtype dt, int num_sms,
                                  cudaStream_t stream);
+gdn_status launch_swa(const swa_params* p, unsigned* status, cudaStream_t stream);
 size_t bwd_workspace(const gdn_bwd_params* p);
 gdn_status launch_bwd(const gdn_bwd_params* p, unsigned* status, void* ws, cudaStream_t stream);
 }  // namespace gdn
@@ -295,6 +296,29 @@ gdn_status loop_residual(const void* h_tilde, const void* h_prev, const float* r
   const cudaError_t e = gdn::launch_loop_residual(h_tilde, h_prev, rho, h_out, rows, d, io_dtype,
                                                   sm_count(), stream);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status swa_fwd(const swa_params* p, cudaStream_t stream) {
+  if (!p || !dtype_ok(p->io_dtype)) return GDN_ERR_INVALID;
+  if (p->n_seq < 0 || p->H <= 0 || p->total_tokens < 0 || p->window < 1 || p->d <= 0 || p->dv <= 0)
+    return GDN_ERR_INVALID;
+  if (p->io_dtype != GDN_BF16 || p->d != 128 || p->dv != 128) return GDN_ERR_UNSUPPORTED;
+  if (p->cu_seqlens) {
+    if (p->max_seq_len < 0) return GDN_ERR_INVALID;
+  } else if (p->seq_len < 0 || (long long)p->n_seq * p->seq_len != p->total_tokens) {
+    return GDN_ERR_INVALID;
+  }
+  if (p->n_seq == 0 || p->total_tokens == 0) return GDN_OK;
+  const void* need[] = {p->q, p->k, p->v, p->o};
+  for (const void* x : need)
+    if (!x || !aligned16(x)) return GDN_ERR_INVALID;
+  if (p->cu_seqlens && !aligned16(p->cu_seqlens)) return GDN_ERR_INVALID;
+  const size_t tok = (size_t)p->total_tokens * p->H * 2;
+  const Range others[] = {{p->q, tok * p->d}, {p->k, tok * p->d}, {p->v, tok * p->dv}};
+  if (overlaps_any({p->o, tok * p->dv}, others)) return GDN_ERR_INVALID;
+  unsigned* st = status_ptr();
+  if (!st) return GDN_ERR_CUDA;
+  return gdn::launch_swa(p, st, stream);
 }
 
 gdn_status gdn_get_device_status(cudaStream_t stream) {

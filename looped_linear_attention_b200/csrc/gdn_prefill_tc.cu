@@ -46,6 +46,7 @@
 //   * every wait is bounded (GDN_ERR_TIMEOUT) so a fault in the schedule cannot
 //     hang the GPU.
 #include "common.cuh"
+#include "tma_host.h"
 
 namespace gdn {
 namespace tc {
@@ -1227,38 +1228,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 }  // namespace tc
 
 // Host launcher: builds the TMA descriptors (3-D views [tokens][H][width] of
-// q, k, v with 64 x 1 x 64 boxes) and launches one CTA per (sequence, head,
-// 128-wide dv slice).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult qres;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
-            cudaSuccess &&
-        qres == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-static bool make_map(CUtensorMap* m, const void* base, int width, int H, int total_tokens) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)total_tokens};
-  cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)width * 2 * H};
-  cuuint32_t box[3] = {64, 1, 64};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
+// q, k, v with 64 x 1 x 64 boxes, tma_host.h) and launches one CTA per
+// (sequence, head, 128-wide dv slice).
 bool prefill_tc_supported(const gdn_fwd_params* p) {
   return p->io_dtype == GDN_BF16 && p->dk == tc::DK && p->dv % tc::DVS == 0 &&
          !(p->flags & (GDN_PRECISE | GDN_CHANNEL_GATE));

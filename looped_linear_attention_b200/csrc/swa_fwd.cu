@@ -1,0 +1,363 @@
+// Sliding-window causal softmax attention on the 5th-generation tensor cores
+// (tcgen05 MMA with tensor-memory accumulators, TMA-fed shared memory), sm_100a.
+//
+// The window mixer of the hybrid LT2 loops ("LT2: Linear-Time Looped
+// Transformers", §2: a sliding-window block of window w, whose receptive
+// field grows to T w over T loops; Appendix C: the windowed variants attend to
+// the w - 1 previous tokens and the token itself, none after it).  For query
+// t of a sequence starting at t0, over the keys j in [max(t0, t - w + 1), t]:
+//     o_t = sum_j softmax_j(scale q_t . k_j) v_j.
+//
+// One CTA of 128 threads per (sequence, head, tile of 128 queries) walks the
+// 128-key tiles that the tile's windows touch, flash-attention style:
+//   * Q (once), K and V tiles (double-buffered) arrive by TMA in the 128-byte
+//     swizzle; S = Q K^T and O += P V are tcgen05 MMAs (M = 128 queries,
+//     N = 128, K = 128) issued by one thread, accumulating in tensor memory
+//     (two S buffers, so S of the next tile runs while this one's softmax is
+//     computed, and O);
+//   * thread r owns query row r (tensor-memory lane r): it masks the row to
+//     its window, keeps the running maximum m and sum l in base 2, writes
+//     P = 2^(s - m) as the bf16 A operand of the next MMA, and rescales its O
+//     row in tensor memory only when the maximum grew by more than 2^8
+//     (otherwise the stale maximum keeps every P <= 2^8; the result is the
+//     same after the final division by l);
+//   * K of tile t+2 is loaded once S_t is done, V of tile t+1 once O of tile
+//     t-1 is done; every wait is bounded (GDN_ERR_TIMEOUT).
+// The epilogue divides by l and stores bf16 rows, staged through shared
+// memory for 16-byte coalesced stores.
+#include "common.cuh"
+#include "tma_host.h"
+
+namespace gdn {
+namespace swa {
+
+constexpr int D = 128;        // head width of q, k and v
+constexpr int BM = 128;       // queries per CTA
+constexpr int BN = 128;       // keys per tile
+constexpr int THREADS = 128;
+constexpr uint32_t TILE_BYTES = 32768;           // 128 rows x 128 bf16, two 64-column slabs
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + TILE_BYTES;    // 2 buffers
+constexpr uint32_t OFF_V = OFF_K + 2 * TILE_BYTES;  // 2 buffers
+constexpr uint32_t OFF_P = OFF_V + 2 * TILE_BYTES;  // P (bf16 A operand); output staging
+constexpr uint32_t OFF_BAR = OFF_P + TILE_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
+// tensor-memory columns: S (two buffers) and O
+constexpr uint32_t COL_S = 0;
+constexpr uint32_t COL_O = 256;
+constexpr uint32_t TMEM_COLS = 512;
+
+enum : int { B_Q = 0, B_K = 1, B_V = 3, B_S = 5, B_O = 7, NBAR = 8 };   // [2] for K, V, S
+
+struct Params {
+  __nv_bfloat16* o;
+  const int32_t* cu_seqlens;
+  unsigned* status;
+  int n_seq, seq_len, max_seq_len, total_tokens, H, window;
+  float scale_log2;   // scale * log2(e)
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return smem_desc(saddr, 16, 1024); }
+__device__ __forceinline__ uint64_t mndesc(uint32_t saddr, uint32_t lbo) { return smem_desc(saddr, lbo, 1024); }
+
+// One 128 x 128 tile (tokens tok0 .. tok0 + 127 of head h) in two 64-column slabs.
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int h,
+                                          int tok0) {
+  mbar_arrive_expect_tx(bar, TILE_BYTES);
+  tma_load_3d(dst, map, bar, 0, h, tok0);
+  tma_load_3d(dst + 8192, map, bar, 0, h, tok0 + 64);
+  tma_load_3d(dst + 16384, map, bar, 64, h, tok0);
+  tma_load_3d(dst + 24576, map, bar, 64, h, tok0 + 64);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(sm) & 1023u) {
+    if (tid == 0) record_status(p.status, GDN_ERR_CUDA);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 8 * NBAR);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_BAR + 8 * NBAR + 4);
+
+  // block -> (sequence, head, query tile); query tiles fastest so that
+  // neighbouring CTAs share K and V tiles in L2
+  const int n_qt = (p.max_seq_len + BM - 1) / BM;
+  const int qt = blockIdx.x % n_qt;
+  const int h = (blockIdx.x / n_qt) % p.H;
+  const int seq = blockIdx.x / (n_qt * p.H);
+  int seq_start, seq_end;
+  if (p.cu_seqlens) {
+    seq_start = p.cu_seqlens[seq];
+    seq_end = p.cu_seqlens[seq + 1];
+  } else {
+    seq_start = seq * p.seq_len;
+    seq_end = seq_start + p.seq_len;
+  }
+  {
+    const int s0 = min(max(seq_start, 0), p.total_tokens);
+    const int s1 = min(max(seq_end, s0), p.total_tokens);
+    bool bad = (s0 != seq_start || s1 != seq_end);
+    // a sequence longer than max_seq_len would lose its last queries
+    bad = bad || (qt == n_qt - 1 && s1 - s0 > p.max_seq_len);
+    if (bad && tid == 0) record_status(p.status, GDN_ERR_INVALID);
+    seq_start = s0;
+    seq_end = s1;
+  }
+  const int q0 = seq_start + qt * BM;
+  if (q0 >= seq_end) return;                       // past this sequence (uniform per CTA)
+  // key tiles (128 keys from the sequence start) touched by the windows of this tile
+  const int key_lo = max(seq_start, q0 - p.window + 1);
+  const int key_hi = min(q0 + BM - 1, seq_end - 1);
+  const int t_first = (key_lo - seq_start) / BN;
+  const int n_tiles = (key_hi - seq_start) / BN - t_first + 1;
+  auto key_tok = [&](int t) { return seq_start + (t_first + t) * BN; };
+
+  if (tid == 0) {
+    for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t sbase = smem_u32(sm);
+  int k_issued = 0, v_issued = 0;                 // tiles whose K / V loads thread 0 issued
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    load_tile(sm + OFF_Q, &tm_q, &bars[B_Q], h, q0);
+    for (; k_issued < min(2, n_tiles); ++k_issued)
+      load_tile(sm + OFF_K + k_issued * TILE_BYTES, &tm_k, &bars[B_K + k_issued], h, key_tok(k_issued));
+    for (; v_issued < min(2, n_tiles); ++v_issued)
+      load_tile(sm + OFF_V + v_issued * TILE_BYTES, &tm_v, &bars[B_V + v_issued], h, key_tok(v_issued));
+  }
+  // S = Q K_t^T into S buffer t % 2 (thread 0 of a converged warp 0)
+  auto issue_s = [&](int t) {
+    const uint32_t kt = sbase + OFF_K + (t & 1) * TILE_BYTES;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+      mma_bf16(tmem + COL_S + (t & 1) * BN, kdesc(sbase + OFF_Q + off), kdesc(kt + off),
+               idesc_bf16(128, 128, 0, 0), kk > 0);
+    }
+    mma_commit(&bars[B_S + (t & 1)]);
+  };
+  bool ok = true;
+  if (warp == 0) {
+    bool okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_Q], 0, s_abort, p.status));
+    okw = okw && __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_K], 0, s_abort, p.status));
+    tc_fence_after();
+    if (okw && elect_one()) issue_s(0);
+    __syncwarp();
+  }
+  ok = !__syncthreads_or(*s_abort != 0);
+
+  const int r = tid;                               // query row of this thread
+  const int q_tok = q0 + r;
+  const bool row_valid = q_tok < seq_end;
+  const int win_lo = q_tok - p.window + 1;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  float m_run = -1e30f, l_run = 0.f;               // running maximum (base 2) and sum
+  for (int t = 0; t < n_tiles && ok; ++t) {
+    const int kt0 = key_tok(t);
+    // ---- S_t is in tensor memory
+    if (__syncthreads_or(!mbar_wait_bounded(&bars[B_S + (t & 1)], (t >> 1) & 1, s_abort, p.status))) break;
+    tc_fence_after();
+    if (warp == 0) {
+      // K of tile t+2 into the buffer S_t has finished reading; S_{t+1} into the other S buffer
+      if (lane == 0 && k_issued < n_tiles && k_issued == t + 2) {
+        load_tile(sm + OFF_K + (t & 1) * TILE_BYTES, &tm_k, &bars[B_K + (t & 1)], h, key_tok(t + 2));
+        ++k_issued;
+      }
+      if (t + 1 < n_tiles) {
+        const bool okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_K + ((t + 1) & 1)],
+                                                                    ((t + 1) >> 1) & 1, s_abort, p.status));
+        tc_fence_after();
+        if (okw && elect_one()) issue_s(t + 1);
+      }
+      __syncwarp();
+    }
+    // ---- pass 1: the row maximum of this tile over the row's window (base 2)
+    const uint32_t s_col = tmem + lane_off + COL_S + (t & 1) * BN;
+    float tmax = -INFINITY;
+#pragma unroll 1
+    for (int piece = 0; piece < BN / 32; ++piece) {
+      float x[32];
+      tmem_ld32(s_col + piece * 32, x);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int j = kt0 + piece * 32 + e;
+        const bool in = row_valid && j <= q_tok && j >= win_lo;
+        tmax = fmaxf(tmax, in ? x[e] * p.scale_log2 : -INFINITY);
+      }
+    }
+    const float m_new = fmaxf(m_run, tmax);
+    // lazy rescale: only when the maximum grew by more than 8 (in base 2)
+    const bool grow = (t > 0) && (m_new > m_run + 8.f);
+    const float alpha = grow ? ex2(m_run - m_new) : 1.f;
+    if (t == 0 || grow) m_run = m_new;
+    // ---- O of tile t-1 is done: P and V_{t-1} are free, O may be rescaled
+    if (t > 0) {
+      if (__syncthreads_or(!mbar_wait_bounded(&bars[B_O], (t - 1) & 1, s_abort, p.status))) break;
+      tc_fence_after();
+      if (tid == 0 && v_issued < n_tiles && v_issued == t + 1) {
+        load_tile(sm + OFF_V + ((t + 1) & 1) * TILE_BYTES, &tm_v, &bars[B_V + ((t + 1) & 1)], h,
+                  key_tok(t + 1));
+        ++v_issued;
+      }
+      if (__any_sync(0xffffffffu, grow)) {
+        l_run *= alpha;
+#pragma unroll 1
+        for (int piece = 0; piece < D / 32; ++piece) {
+          float y[32];
+          tmem_ld32(tmem + lane_off + COL_O + piece * 32, y);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) y[e] *= alpha;
+          tmem_st32(tmem + lane_off + COL_O + piece * 32, y);
+        }
+        tmem_wait_st();
+      }
+    }
+    // ---- pass 2: P = 2^(s - m) (bf16, swizzled A operand), l += sum P
+    float lsum = 0.f;
+#pragma unroll 1
+    for (int piece = 0; piece < BN / 32; ++piece) {
+      float x[32];
+      tmem_ld32(s_col + piece * 32, x);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int j = kt0 + piece * 32 + e;
+        const bool in = row_valid && j <= q_tok && j >= win_lo;
+        x[e] = in ? ex2(x[e] * p.scale_log2 - m_run) : 0.f;
+        lsum += x[e];
+      }
+      const int c0 = piece * 32;
+      uint8_t* slab = sm + OFF_P + (c0 >> 6) * 16384;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint4 o;
+        o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
+        o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
+        o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
+        o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
+        *reinterpret_cast<uint4*>(slab + sw128_offset(r, (c0 & 63) + c * 8)) = o;
+      }
+    }
+    l_run += lsum;
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- O += P V_t
+    if (warp == 0) {
+      const bool okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_V + (t & 1)], (t >> 1) & 1,
+                                                                  s_abort, p.status));
+      tc_fence_after();
+      if (okw && elect_one()) {
+        const uint32_t vt = sbase + OFF_V + (t & 1) * TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_bf16(tmem + COL_O, kdesc(sbase + OFF_P + (kk >> 2) * 16384 + (kk & 3) * 32),
+                   mndesc(vt + kk * 2048, 16384), idesc_bf16(128, 128, 0, 1), (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[B_O]);
+      }
+      __syncwarp();
+    }
+    ok = !__syncthreads_or(*s_abort != 0);
+  }
+  // ---- epilogue: O / l, staged through shared memory for coalesced stores
+  if (ok && n_tiles > 0)
+    ok = !__syncthreads_or(!mbar_wait_bounded(&bars[B_O], (n_tiles - 1) & 1, s_abort, p.status));
+  tc_fence_after();
+  if (ok) {
+    const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    uint8_t* stage = sm + OFF_P;                   // [128 rows][256 B], 16-byte chunks XOR-swizzled
+#pragma unroll 1
+    for (int piece = 0; piece < D / 32; ++piece) {
+      float y[32];
+      tmem_ld32(tmem + lane_off + COL_O + piece * 32, y);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint4 o;
+        o.x = pack_bf16x2(y[c * 8 + 0] * inv, y[c * 8 + 1] * inv);
+        o.y = pack_bf16x2(y[c * 8 + 2] * inv, y[c * 8 + 3] * inv);
+        o.z = pack_bf16x2(y[c * 8 + 4] * inv, y[c * 8 + 5] * inv);
+        o.w = pack_bf16x2(y[c * 8 + 6] * inv, y[c * 8 + 7] * inv);
+        const int chunk = piece * 4 + c;
+        *reinterpret_cast<uint4*>(stage + r * 256 + ((chunk ^ (r & 15)) * 16)) = o;
+      }
+    }
+    __syncthreads();
+    const int rows = min(BM, seq_end - q0);
+#pragma unroll 4
+    for (int it = tid; it < BM * 16; it += THREADS) {
+      const int i = it >> 4, chunk = it & 15;
+      if (i < rows) {
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + i * 256 + ((chunk ^ (i & 15)) * 16));
+        __stcs(reinterpret_cast<uint4*>(p.o + ((size_t)(q0 + i) * p.H + h) * D + chunk * 8), v);
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {
+    // never leave with a bulk copy still landing in shared memory: every load
+    // issued is waited for (the waits above may have been skipped on abort)
+    mbar_wait_bounded(&bars[B_Q], 0, nullptr, p.status);
+    for (int t = max(0, k_issued - 2); t < k_issued; ++t)
+      mbar_wait_bounded(&bars[B_K + (t & 1)], (t >> 1) & 1, nullptr, p.status);
+    for (int t = max(0, v_issued - 2); t < v_issued; ++t)
+      mbar_wait_bounded(&bars[B_V + (t & 1)], (t >> 1) & 1, nullptr, p.status);
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace swa
+
+gdn_status launch_swa(const swa_params* p, unsigned* status, cudaStream_t stream) {
+  static std::atomic<bool> attr_set[kMaxDevices];
+  if (smem_attr_once(attr_set, swa::swa_fwd_kernel, swa::SMEM_BYTES) != cudaSuccess) return GDN_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, p->q, swa::D, p->H, p->total_tokens) || !make_map(&mk, p->k, swa::D, p->H, p->total_tokens) ||
+      !make_map(&mv, p->v, swa::D, p->H, p->total_tokens))
+    return GDN_ERR_CUDA;
+  swa::Params kp;
+  kp.o = static_cast<__nv_bfloat16*>(p->o);
+  kp.cu_seqlens = p->cu_seqlens;
+  kp.status = status;
+  kp.n_seq = p->n_seq;
+  kp.seq_len = p->seq_len;
+  kp.max_seq_len = p->cu_seqlens ? p->max_seq_len : p->seq_len;
+  kp.total_tokens = p->total_tokens;
+  kp.H = p->H;
+  kp.window = p->window;
+  kp.scale_log2 = p->scale * 1.4426950408889634f;
+  const long long blocks = (long long)p->n_seq * p->H * ((kp.max_seq_len + swa::BM - 1) / swa::BM);
+  if (blocks <= 0) return GDN_OK;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  swa::swa_fwd_kernel<<<(unsigned)blocks, swa::THREADS, swa::SMEM_BYTES, stream>>>(mq, mk, mv, kp);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace gdn

@@ -1242,7 +1242,9 @@ bool prefill_tc_supported(const gdn_fwd_params* p) {
 // p >= 2, to Sst (slot p-1; M_p and B_p sit in slot p-1 of theirs).  With
 // n_steps = n_segs - 2 (output-pass schedule) the last one is S_{n_segs-1};
 // with n_steps = n_segs - 1 (corrected schedule) the last one, S_{n_segs}, is
-// the final state and goes to S_T (or nowhere when S_T is null).  The
+// the final state and goes to S_T (or nowhere when S_T is null).  With Sb
+// (corrected schedule) every start state S_1 .. S_{n_segs-1} is also written
+// rounded to bf16 into Sb (same layout as Sst), the correction's operand.  The
 // products run on the warp-level tensor cores with the 3xTF32 split
 // (fp32-level accuracy): warp w owns rows 16w .. 16w+15 of the 128 x CMB_COLS
 // block.  M_p (dk x dk) is staged in shared memory by cp.async one step ahead
@@ -1268,8 +1270,9 @@ __device__ __forceinline__ void cp_async_wait() {
 
 __global__ void __launch_bounds__(256)
     gdn_segment_combine_kernel(const float* __restrict__ Bws, const float* __restrict__ Mws,
-                               float* __restrict__ Sst, float* __restrict__ S_T, int H, int dv,
-                               int n_segs, int n_part, int n_steps) {
+                               float* __restrict__ Sst, float* __restrict__ S_T,
+                               __nv_bfloat16* __restrict__ Sb, int H, int dv, int n_segs, int n_part,
+                               int n_steps) {
   extern __shared__ __align__(16) float cmb_smem[];
   // launched as a programmatic dependent of the state pass: let the output
   // pass launch, then wait for the state pass before reading its results
@@ -1303,8 +1306,8 @@ __global__ void __launch_bounds__(256)
     }
     cp_async_commit();
   };
-  if (n_steps <= 0) return;
-  stage(0, sM0);
+  if (n_steps <= 0 && !Sb) return;
+  if (n_steps > 0) stage(0, sM0);
   // x[nt][e]: rows r0+g (e = 0, 1) and r0+g+8 (e = 2, 3), columns nt*8 + 2q (+1)
   float x[CMB_NT][4];
 #pragma unroll
@@ -1316,8 +1319,12 @@ __global__ void __launch_bounds__(256)
       x[nt][2 * hr + 1] = v.y;
     }
   for (int pp = 0;; ++pp) {
-    // S_{pp+1} (x) to the operand block, and to Sst (or S_T) unless it came from there
+    // S_{pp+1} (x) to the operand block, and to Sst (or S_T) unless it came from
+    // there; its bf16 copy for the correction (start states only)
     float* dst = (pp > 0) ? sptr(pp) : nullptr;
+    __nv_bfloat16* dstb = (Sb && pp <= n_segs - 2)
+                              ? Sb + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb
+                              : nullptr;
 #pragma unroll
     for (int nt = 0; nt < CMB_NT; ++nt)
 #pragma unroll
@@ -1325,6 +1332,7 @@ __global__ void __launch_bounds__(256)
         const float2 v = make_float2(x[nt][2 * hr], x[nt][2 * hr + 1]);
         const int r = r0 + g + 8 * hr, c = nt * 8 + 2 * q;
         if (dst) *reinterpret_cast<float2*>(dst + (size_t)r * dv + c) = v;
+        if (dstb) *reinterpret_cast<uint32_t*>(dstb + (size_t)r * dv + c) = pack_bf16x2(v.x, v.y);
         *reinterpret_cast<float2*>(sS + r * CMB_SLD + c) = v;
       }
     if (pp >= n_steps) break;
@@ -1385,29 +1393,54 @@ __global__ void __launch_bounds__(256)
 //     o_i = o^0_i + S_p^T qhat_i,
 // which this kernel adds for one (sequence, head, 128-wide dv slice) and a
 // tile of up to 128 tokens of one segment, then applies the loop residual.
-// The product is one tcgen05 MMA chain (M = 128 tokens, N = 128 columns of
-// dv, K = dk = 128) into tensor memory: qhat arrives by TMA (K-major, 128-byte
-// swizzle), S_p (fp32, from the combine or segment 0) is rounded to bf16 into
-// an MN-major operand tile.  Launched as a programmatic dependent: it waits
-// for the previous grid before reading anything the state pass wrote.
+// Every operand arrives by TMA in the 128-byte swizzle: qhat (K-major A),
+// S_p rounded to bf16 by the combine (MN-major B: rows of dk, 64 columns of
+// dv per 128-byte row), o^0 and h_prev (token rows); the product is one
+// tcgen05 MMA chain (M = 128 tokens, N = 128 columns of dv, K = dk = 128) into
+// tensor memory.  The result is written over the o^0 tile in shared memory
+// and stored as 16-byte coalesced rows.  Launched as a programmatic
+// dependent: h_prev (an input) is requested first, everything the state pass
+// and the combine wrote only after griddepcontrol.wait.
 constexpr int COR_THREADS = 128;
 constexpr int COR_ROWS = 128;                      // tokens per tile
-constexpr uint32_t COR_OFF_A = 0;                  // qhat: 2 slabs [128 tok][64 dk] bf16
-constexpr uint32_t COR_OFF_B = 32768;              // S_p: 2 blocks [128 dk][64 dv] bf16, MN-major
-constexpr uint32_t COR_OFF_BAR = 65536;            // 2 mbarriers, tmem base, abort flag
+constexpr uint32_t COR_TILE = 32768;               // 128 rows x 128 bf16 in two 64-column slabs
+constexpr uint32_t COR_OFF_A = 0;                  // qhat
+constexpr uint32_t COR_OFF_B = COR_OFF_A + COR_TILE;   // S_p (bf16, MN-major)
+constexpr uint32_t COR_OFF_O = COR_OFF_B + COR_TILE;   // o^0, then the result
+constexpr uint32_t COR_OFF_H = COR_OFF_O + COR_TILE;   // h_prev
+constexpr uint32_t COR_OFF_BAR = COR_OFF_H + COR_TILE; // 3 mbarriers, tmem base, abort flag
 constexpr uint32_t COR_SMEM = COR_OFF_BAR + 64 + 1024;
 
 struct CorParams {
   __nv_bfloat16* o;
-  const __nv_bfloat16* h_prev;   // loop residual (or null) and its rho
-  const float* rho;
-  const float* Sst;              // [n_seq][n_segs-1][H][dk][dv], S_p in slot p-1
+  const float* rho;              // loop residual's rho (with h_prev), or null
   unsigned* status;
   int H, dv, n_slices, seq_len, seg0_tok, seg_tok, n_segs, tiles_mid, tiles_per_seq;
+  int residual;
 };
 
+// One 128-token tile of a [tokens][H][width] map (two 64-column slabs, two
+// 64-row boxes each).
+__device__ __forceinline__ void cor_load_rows(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                              int h, int tok0) {
+  tma_load_3d(dst, map, bar, c0, h, tok0);
+  tma_load_3d(dst + 8192, map, bar, c0, h, tok0 + 64);
+  tma_load_3d(dst + 16384, map, bar, c0 + 64, h, tok0);
+  tma_load_3d(dst + 24576, map, bar, c0 + 64, h, tok0 + 64);
+}
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                            int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __global__ void __launch_bounds__(COR_THREADS, 1)
-    gdn_segment_correct_kernel(const __grid_constant__ CUtensorMap tm_qh, const CorParams p) {
+    gdn_segment_correct_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_sb,
+                               const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_h,
+                               const CorParams p) {
   extern __shared__ __align__(1024) uint8_t csm_raw[];
   uint8_t* sm = csm_raw;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1415,9 +1448,10 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
     if (tid == 0) record_status(p.status, GDN_ERR_CUDA);
     return;
   }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + COR_OFF_BAR);   // [0] qhat landed, [1] MMA done
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + COR_OFF_BAR + 16);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + COR_OFF_BAR + 20);
+  // [0] qhat and S_p landed, [1] o^0 (and h_prev) landed, [2] MMA done
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + COR_OFF_BAR);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + COR_OFF_BAR + 24);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + COR_OFF_BAR + 28);
   // block -> (sequence, head, slice, tile); tiles enumerate segments 1 .. n_segs-1
   int bid = (int)blockIdx.x;
   const int tile = bid % p.tiles_per_seq;
@@ -1440,13 +1474,13 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
   const int rows = min(COR_ROWS, seg_len - i0);
   const int tok0 = seq * p.seq_len + seg_start + i0;
   const int col0 = slice * DVS;
+  // row of S_p in the [n_seq * (n_segs-1) * H * dk][dv] view of the bf16 start states
+  const int sb_row = ((seq * (p.n_segs - 1) + (part - 1)) * p.H + h) * DK;
 
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
     *s_abort = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_qh);
   }
   if (warp == 0) {
     tmem_alloc(s_tmem, 128);
@@ -1458,84 +1492,86 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = smem_u32(sm);
-
-  griddep_wait();                                  // qhat, o^0 and S_p are written
   const bool have_rows = rows > 0;
   if (tid == 0 && have_rows) {
-    mbar_arrive_expect_tx(&bars[0], 32768);
-    tma_load_3d(sm + COR_OFF_A, &tm_qh, &bars[0], 0, h, tok0);
-    tma_load_3d(sm + COR_OFF_A + 8192, &tm_qh, &bars[0], 0, h, tok0 + 64);
-    tma_load_3d(sm + COR_OFF_A + 16384, &tm_qh, &bars[0], 64, h, tok0);
-    tma_load_3d(sm + COR_OFF_A + 24576, &tm_qh, &bars[0], 64, h, tok0 + 64);
+    tma_prefetch_desc(&tm_qh);
+    tma_prefetch_desc(&tm_sb);
+    tma_prefetch_desc(&tm_o);
+    mbar_arrive_expect_tx(&bars[1], p.residual ? 2 * COR_TILE : COR_TILE);
+    if (p.residual) cor_load_rows(sm + COR_OFF_H, &tm_h, &bars[1], col0, h, tok0);   // an input
   }
-  // S_p (fp32 [dk][dv]) -> bf16 MN-major tile: block nb holds columns
-  // 64 nb .. 64 nb + 63, row k (dk) 128 bytes, swizzled like a TMA tile
-  const float* Sp = p.Sst + (((size_t)seq * (p.n_segs - 1) + (part - 1)) * p.H + h) * DK * (size_t)p.dv + col0;
-#pragma unroll 4
-  for (int it = 0; it < 16 && have_rows; ++it) {
-    const int u = tid + it * COR_THREADS;          // 2048 chunks of 8 columns
-    const int k = u >> 4, cc = u & 15;
-    const float4 x0 = __ldg(reinterpret_cast<const float4*>(Sp + (size_t)k * p.dv + cc * 8));
-    const float4 x1 = __ldg(reinterpret_cast<const float4*>(Sp + (size_t)k * p.dv + cc * 8 + 4));
-    uint4 v;
-    v.x = pack_bf16x2(x0.x, x0.y);
-    v.y = pack_bf16x2(x0.z, x0.w);
-    v.z = pack_bf16x2(x1.x, x1.y);
-    v.w = pack_bf16x2(x1.z, x1.w);
-    *reinterpret_cast<uint4*>(sm + COR_OFF_B + (cc >> 3) * 16384 + sw128_offset(k, (cc & 7) * 8)) = v;
+  griddep_wait();                                  // qhat, o^0 and S_p are written
+  if (tid == 0 && have_rows) {
+    mbar_arrive_expect_tx(&bars[0], 2 * COR_TILE);
+    cor_load_rows(sm + COR_OFF_A, &tm_qh, &bars[0], 0, h, tok0);
+    tma_load_2d(sm + COR_OFF_B, &tm_sb, &bars[0], col0, sb_row);
+    tma_load_2d(sm + COR_OFF_B + 16384, &tm_sb, &bars[0], col0 + 64, sb_row);
+    cor_load_rows(sm + COR_OFF_O, &tm_o, &bars[1], col0, h, tok0);
   }
-  fence_proxy_async_smem();
-  __syncthreads();
   bool ok = have_rows;
-  if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[0], 0, s_abort, p.status));
   if (ok && warp == 0) {
+    const bool okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[0], 0, s_abort, p.status));
     tc_fence_after();
-    if (elect_one()) {
+    if (okw && elect_one()) {
 #pragma unroll
       for (int kk = 0; kk < DK / 16; ++kk)
         mma_bf16(tmem, kdesc(sbase + COR_OFF_A + (kk >> 2) * 16384 + (kk & 3) * 32),
                  mndesc(sbase + COR_OFF_B + kk * 2048, 16384), idesc_bf16(128, 128, 0, 1), kk > 0);
-      mma_commit(&bars[1]);
+      mma_commit(&bars[2]);
     }
     __syncwarp();
   }
-  if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[1], 0, s_abort, p.status));
+  if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[1], 0, s_abort, p.status) || *s_abort != 0);
+  if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[2], 0, s_abort, p.status));
   tc_fence_after();
   if (ok) {
-    // thread: token row 32 warp + lane of the tile, 32 columns at a time
+    // thread: token row r of the tile; the result replaces o^0 in shared memory
     const int r = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const size_t off = ((size_t)(tok0 + r) * p.H + h) * p.dv + col0;
 #pragma unroll 1
     for (int piece = 0; piece < DVS / 32; ++piece) {
       float acc[32];
       tmem_ld32(tmem + lane_off + piece * 32, acc);
-      if (r < rows) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o + off + piece * 32);
+      const int cbase = piece * 32;
+      const uint32_t slab = (uint32_t)(cbase >> 6) * 16384;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 x = dst[c];
-          float y[8] = {bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y),
-                        bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w)};
+      for (int c = 0; c < 4; ++c) {
+        const int col = (cbase & 63) + c * 8;
+        uint4* ov = reinterpret_cast<uint4*>(sm + COR_OFF_O + slab + sw128_offset(r, col));
+        const uint4 x = *ov;
+        float y[8] = {bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y),
+                      bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w)};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] += acc[c * 8 + e];
-          if (p.h_prev) {
-            // the loop residual on the output rounded to bf16, as loop_residual sees it
-            const uint4 hp = *reinterpret_cast<const uint4*>(p.h_prev + off + piece * 32 + c * 8);
-            const float hv[8] = {bf16_lo(hp.x), bf16_hi(hp.x), bf16_lo(hp.y), bf16_hi(hp.y),
-                                 bf16_lo(hp.z), bf16_hi(hp.z), bf16_lo(hp.w), bf16_hi(hp.w)};
-            const float* rr = p.rho + (size_t)h * p.dv + col0 + piece * 32 + c * 8;
+        for (int e = 0; e < 8; ++e) y[e] += acc[c * 8 + e];
+        if (p.residual) {
+          // the loop residual on the output rounded to bf16, as loop_residual sees it
+          const uint4 hp = *reinterpret_cast<const uint4*>(sm + COR_OFF_H + slab + sw128_offset(r, col));
+          const float hv[8] = {bf16_lo(hp.x), bf16_hi(hp.x), bf16_lo(hp.y), bf16_hi(hp.y),
+                               bf16_lo(hp.z), bf16_hi(hp.z), bf16_lo(hp.w), bf16_hi(hp.w)};
+          const float4 r0 = __ldg(reinterpret_cast<const float4*>(p.rho + (size_t)h * p.dv + col0 + cbase + c * 8));
+          const float4 r1 = __ldg(reinterpret_cast<const float4*>(p.rho + (size_t)h * p.dv + col0 + cbase + c * 8 + 4));
+          const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              y[e] = fmaf(__ldg(rr + e), hv[e], __bfloat162float(__float2bfloat16_rn(y[e])));
-          }
-          uint4 v;
-          v.x = pack_bf16x2(y[0], y[1]);
-          v.y = pack_bf16x2(y[2], y[3]);
-          v.z = pack_bf16x2(y[4], y[5]);
-          v.w = pack_bf16x2(y[6], y[7]);
-          dst[c] = v;
+          for (int e = 0; e < 8; ++e) y[e] = fmaf(rr[e], hv[e], __bfloat162float(__float2bfloat16_rn(y[e])));
         }
+        uint4 v;
+        v.x = pack_bf16x2(y[0], y[1]);
+        v.y = pack_bf16x2(y[2], y[3]);
+        v.z = pack_bf16x2(y[4], y[5]);
+        v.w = pack_bf16x2(y[6], y[7]);
+        *ov = v;
+      }
+    }
+    __syncthreads();
+    // coalesced 16-byte stores of the valid rows (a row past the segment
+    // belongs to another segment or sequence and is not touched)
+#pragma unroll 4
+    for (int it = tid; it < COR_ROWS * 16; it += COR_THREADS) {
+      const int i = it >> 4, chunk = it & 15;
+      if (i < rows) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sm + COR_OFF_O + (chunk >> 3) * 16384 +
+                                                        sw128_offset(i, (chunk & 7) * 8));
+        __stcs(reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + i) * p.H + h) * p.dv + col0 + chunk * 8), v);
       }
     }
   }
@@ -1545,6 +1581,7 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
   if (tid == 0 && have_rows && !ok) {
     // never leave the block with a bulk copy still landing in its shared memory
     mbar_wait_bounded(&bars[0], 0, nullptr, p.status);
+    mbar_wait_bounded(&bars[1], 0, nullptr, p.status);
   }
   if (warp == 0) {
     tc_fence_after();
@@ -1665,10 +1702,11 @@ SegPlan plan_prefill_segments(const gdn_fwd_params* p, int sms) {
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Workspace of a segmented schedule: [B | M | S | qhat] with B and M for
+// Workspace of a segmented schedule: [B | M | S | qhat | Sb] with B and M for
 // n_part segments (n_segs-2 in the output-pass schedule, n_segs-1 in the
 // corrected one), start states S_1 .. S_{n_segs-1}, and for the corrected
-// schedule qhat [total_tokens][H][dk] bf16; each buffer 256-byte aligned.
+// schedule qhat [total_tokens][H][dk] bf16 and the start states in bf16;
+// each buffer 256-byte aligned.
 size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan) {
   if (plan.lpt) return align256((size_t)p->n_seq * sizeof(int32_t));
   if (plan.n_segs <= 1) return 0;
@@ -1677,8 +1715,9 @@ size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan) {
   const size_t n = (size_t)p->n_seq;
   const size_t n_part = plan.corrected ? plan.n_segs - 1 : plan.n_segs - 2;
   const size_t qh = plan.corrected ? (size_t)p->total_tokens * p->H * tc::DK * 2 : 0;
+  const size_t sb = plan.corrected ? n * (plan.n_segs - 1) * sd / 2 : 0;
   return align256(n * n_part * sd) + align256(n * n_part * md) + align256(n * (plan.n_segs - 1) * sd) +
-         align256(qh);
+         align256(qh) + align256(sb);
 }
 
 // Launch configuration; `dependent` launches with programmatic stream
@@ -1768,6 +1807,8 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   kp.Sst = reinterpret_cast<float*>(w);
   w += align256((size_t)p->n_seq * (P - 1) * sd);
   kp.qhat = plan.corrected ? reinterpret_cast<__nv_bfloat16*>(w) : nullptr;
+  w += plan.corrected ? align256((size_t)p->total_tokens * p->H * tc::DK * 2) : 0;
+  __nv_bfloat16* Sb = plan.corrected ? reinterpret_cast<__nv_bfloat16*>(w) : nullptr;
   kp.n_segs = P;
   kp.seg_tok = plan.seg_tok;
   kp.seg0_tok = plan.seg0_tok;
@@ -1775,9 +1816,10 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   gdn_status st =
       tc_launch(mq, mk, mv, kp, chains * (kp.n_slices + (long long)n_part * (kp.n_slices + 1)), stream);
   if (st != GDN_OK) return st;
-  // combine: start states S_2 .. S_{P-1} (and S_T in the corrected schedule)
+  // combine: start states S_2 .. S_{P-1} (and S_T in the corrected schedule,
+  // with every start state also in bf16 for the correction)
   const int n_steps = plan.corrected ? (p->S_T ? P - 1 : P - 2) : P - 2;
-  if (n_steps > 0) {
+  if (n_steps > 0 || plan.corrected) {
     const long long cblocks = chains * (p->dv / tc::CMB_COLS);
     if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     static std::atomic<bool> cmb_attr_set[kMaxDevices];
@@ -1785,8 +1827,8 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
       return GDN_ERR_CUDA;
     LaunchCfg lc((unsigned)cblocks, 256, tc::CMB_SMEM, stream, /*dependent=*/true);
     if (cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_combine_kernel, (const float*)kp.Bws,
-                           (const float*)kp.Mws, kp.Sst, plan.corrected ? p->S_T : nullptr, p->H, p->dv,
-                           P, n_part, n_steps) != cudaSuccess)
+                           (const float*)kp.Mws, kp.Sst, plan.corrected ? p->S_T : nullptr, Sb, p->H,
+                           p->dv, P, n_part, n_steps) != cudaSuccess)
       return GDN_ERR_CUDA;
   }
   if (!plan.corrected) {
@@ -1794,13 +1836,16 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
     return tc_launch(mq, mk, mv, kp, chains * (P - 1) * kp.n_slices, stream, /*dependent=*/true);
   }
   // correction of the outputs of segments 1 .. P-1
-  CUtensorMap mqh;
-  if (!make_map(&mqh, kp.qhat, tc::DK, p->H, p->total_tokens)) return GDN_ERR_CUDA;
+  CUtensorMap mqh, msb, mo, mh;
+  if (!make_map(&mqh, kp.qhat, tc::DK, p->H, p->total_tokens) ||
+      !make_map_2d(&msb, Sb, p->dv, (long long)p->n_seq * (P - 1) * p->H * tc::DK, 64, 128) ||
+      !make_map(&mo, p->o, p->dv, p->H, p->total_tokens) ||
+      !make_map(&mh, p->h_prev ? p->h_prev : p->o, p->dv, p->H, p->total_tokens))
+    return GDN_ERR_CUDA;
   tc::CorParams cp;
   cp.o = kp.o;
-  cp.h_prev = kp.h_prev;
   cp.rho = kp.rho;
-  cp.Sst = kp.Sst;
+  cp.residual = p->h_prev != nullptr;
   cp.status = status;
   cp.H = p->H;
   cp.dv = p->dv;
@@ -1819,8 +1864,9 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   if (smem_attr_once(cor_attr_set, tc::gdn_segment_correct_kernel, tc::COR_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
   LaunchCfg lc((unsigned)cor_blocks, tc::COR_THREADS, tc::COR_SMEM, stream, /*dependent=*/true);
-  return cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_correct_kernel, mqh, cp) == cudaSuccess ? GDN_OK
-                                                                                              : GDN_ERR_CUDA;
+  return cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_correct_kernel, mqh, msb, mo, mh, cp) == cudaSuccess
+             ? GDN_OK
+             : GDN_ERR_CUDA;
 }
 
 }  // namespace gdn

@@ -108,12 +108,13 @@ def _schedule(lib, p):
 def _segmented_need(n_seq, L, H, dv, P, corrected):
     """Workspace of a segmented schedule: B and M for segments 1 .. P-2 (output
     pass) or 1 .. P-1 (corrected), start states for segments 1 .. P-1, and in
-    the corrected schedule qhat [tokens][H][dk] bf16; each 256-byte aligned."""
+    the corrected schedule qhat [tokens][H][dk] bf16 and the start states in
+    bf16; each 256-byte aligned."""
     align = lambda x: (x + 255) // 256 * 256
     sd, md = H * 128 * dv * 4, H * 128 * 128 * 4
     n_part = P - 1 if corrected else P - 2
     return (align(n_seq * n_part * sd) + align(n_seq * n_part * md) + align(n_seq * (P - 1) * sd)
-            + (align(n_seq * L * H * 128 * 2) if corrected else 0))
+            + (align(n_seq * L * H * 128 * 2) + align(n_seq * (P - 1) * sd // 2) if corrected else 0))
 
 
 def test_workspace_segmented_schedule_for_few_long_chains(lib):

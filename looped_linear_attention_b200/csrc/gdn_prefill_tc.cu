@@ -1385,6 +1385,242 @@ __global__ void __launch_bounds__(256)
     __syncthreads();                                // every read of S_pp and M_pp is done
   }
 }
+// The combine on the 5th-generation tensor cores (corrected schedule).  For
+// one (sequence, head, 64 columns of dv), S_{p+1} = M_p S_p + B_p for
+// p = 1 .. n_steps, with the product as tcgen05 MMAs of kind::tf32 in three
+// terms, M_hi S_hi + M_hi S_lo + M_lo S_hi (x = hi + lo, hi = tf32(x),
+// lo = tf32(x - hi)): fp32-level accuracy, M = 128 rows of M_p, N = 64,
+// K = 128, accumulated in tensor memory.  M_p (fp32, written by the
+// transition slice) arrives by TMA into the hi tile in the 128-byte swizzle
+// (K-major, 32 K-elements per 128-byte row) and is split in place; S_p lives
+// in shared memory as the MN-major B operand (32 columns per 128-byte row).
+// M_{p+1} is requested as soon as the product of step p has read M_p.  Every
+// start state is written in fp32 (Sst, or S_T for the last) and rounded to
+// bf16 (Sb) for the correction.
+constexpr int CTC_THREADS = 128;
+constexpr int CTC_COLS = 64;                          // columns of dv per CTA
+constexpr uint32_t CTC_A_BYTES = 65536;               // 128 x 128 fp32
+constexpr uint32_t CTC_B_BYTES = 32768;               // 128 x 64 fp32
+constexpr uint32_t CTC_OFF_AH = 0;
+constexpr uint32_t CTC_OFF_AL = CTC_OFF_AH + CTC_A_BYTES;
+constexpr uint32_t CTC_OFF_BH = CTC_OFF_AL + CTC_A_BYTES;
+constexpr uint32_t CTC_OFF_BL = CTC_OFF_BH + CTC_B_BYTES;
+constexpr uint32_t CTC_OFF_BAR = CTC_OFF_BL + CTC_B_BYTES;
+constexpr uint32_t CTC_SMEM = CTC_OFF_BAR + 64 + 1024;
+static_assert(CTC_SMEM <= 232448, "tensor-core combine exceeds shared memory");
+
+// kind::tf32 instruction descriptor: fp32 D, tf32 A (K-major) and B (MN-major).
+__host__ __device__ constexpr uint32_t idesc_tf32_kmn(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (1u << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_tf32_tc(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+// Byte offset of fp32 element (k, n) of the MN-major B tile: 32-column blocks
+// 16 KB apart, row k 128 bytes, 16-byte chunks XOR (k mod 8).
+__device__ __forceinline__ uint32_t ctc_b_offset(int k, int n) {
+  const int chunk = ((n & 31) >> 2) ^ (k & 7);
+  return (uint32_t)((n >> 5) * 16384 + k * 128 + chunk * 16 + (n & 3) * 4);
+}
+
+__global__ void __launch_bounds__(CTC_THREADS, 1)
+    gdn_segment_combine_tc_kernel(const __grid_constant__ CUtensorMap tm_m, const float* __restrict__ Bws,
+                                  float* __restrict__ Sst, float* __restrict__ S_T,
+                                  __nv_bfloat16* __restrict__ Sb, unsigned* status, int H, int dv,
+                                  int n_segs, int n_part, int n_steps) {
+  extern __shared__ __align__(1024) uint8_t ctc_raw[];
+  uint8_t* sm = ctc_raw;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  // launched as a programmatic dependent of the state pass: let the
+  // correction launch, then wait for the state pass before reading its results
+  griddep_launch_dependents();
+  if (smem_u32(sm) & 1023u) {
+    if (tid == 0) record_status(status, GDN_ERR_CUDA);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CTC_OFF_BAR);    // [0] M landed, [1] MMA done
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CTC_OFF_BAR + 16);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + CTC_OFF_BAR + 20);
+  const int ncb = dv / CTC_COLS;
+  const int cb = blockIdx.x % ncb;
+  const int hh = (blockIdx.x / ncb) % H;
+  const int seq = blockIdx.x / (ncb * H);
+  const size_t sd = (size_t)DK * dv;
+  const size_t colb = (size_t)cb * CTC_COLS;
+  const int r = tid;                                   // row of the state / of M_p
+  auto sptr = [&](int pp) -> float* {                  // S_{pp+1}
+    if (pp <= n_segs - 2) return Sst + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb;
+    return S_T ? S_T + ((size_t)seq * H + hh) * sd + colb : nullptr;
+  };
+  // row of M_p (slot pp) in the [n_seq * n_part * H * dk][dk] view of the transitions
+  auto m_row = [&](int pp) { return ((seq * n_part + pp) * H + hh) * DK; };
+  auto load_m = [&](int pp) {
+    mbar_arrive_expect_tx(&bars[0], CTC_A_BYTES);
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+          " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(sm + CTC_OFF_AH + sl * 16384)),
+          "l"(reinterpret_cast<uint64_t>(&tm_m)), "r"(sl * 32), "r"(m_row(pp)), "r"(smem_u32(&bars[0]))
+          : "memory");
+    }
+  };
+
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, CTC_COLS);
+    tmem_relinquish();
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t sbase = smem_u32(sm);
+  griddep_wait();                                      // S_1, B and M are written
+  if (tid == 0 && n_steps > 0) {
+    tma_prefetch_desc(&tm_m);
+    load_m(0);
+  }
+  // x: this thread's row of S_{pp+1} (64 columns), starting from S_1
+  float x[CTC_COLS];
+  {
+    const float4* src = reinterpret_cast<const float4*>(sptr(0) + (size_t)r * dv);
+#pragma unroll
+    for (int c = 0; c < CTC_COLS / 4; ++c) {
+      const float4 v = __ldg(src + c);
+      x[4 * c] = v.x, x[4 * c + 1] = v.y, x[4 * c + 2] = v.z, x[4 * c + 3] = v.w;
+    }
+  }
+  bool ok = true;
+  for (int pp = 0;; ++pp) {
+    // S_{pp+1}: to Sst / S_T (unless it came from there), to Sb in bf16, and
+    // as the hi/lo B operand of the next product
+    float* dst = (pp > 0) ? sptr(pp) : nullptr;
+    if (dst) {
+      float4* d4 = reinterpret_cast<float4*>(dst + (size_t)r * dv);
+#pragma unroll
+      for (int c = 0; c < CTC_COLS / 4; ++c) d4[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+    }
+    if (Sb && pp <= n_segs - 2) {
+      uint4* b4 = reinterpret_cast<uint4*>(Sb + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb +
+                                           (size_t)r * dv);
+#pragma unroll
+      for (int c = 0; c < CTC_COLS / 8; ++c) {
+        uint4 u;
+        u.x = pack_bf16x2(x[8 * c], x[8 * c + 1]);
+        u.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
+        u.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
+        u.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
+        b4[c] = u;
+      }
+    }
+    if (pp >= n_steps || !ok) break;
+#pragma unroll
+    for (int c = 0; c < CTC_COLS / 4; ++c) {
+      float4 hi, lo;
+      hi.x = tf32_round(x[4 * c]);
+      hi.y = tf32_round(x[4 * c + 1]);
+      hi.z = tf32_round(x[4 * c + 2]);
+      hi.w = tf32_round(x[4 * c + 3]);
+      lo.x = tf32_round(x[4 * c] - hi.x);
+      lo.y = tf32_round(x[4 * c + 1] - hi.y);
+      lo.z = tf32_round(x[4 * c + 2] - hi.z);
+      lo.w = tf32_round(x[4 * c + 3] - hi.w);
+      *reinterpret_cast<float4*>(sm + CTC_OFF_BH + ctc_b_offset(r, 4 * c)) = hi;
+      *reinterpret_cast<float4*>(sm + CTC_OFF_BL + ctc_b_offset(r, 4 * c)) = lo;
+    }
+    // B_pp of this row, needed after the product
+    const float4* bsrc = reinterpret_cast<const float4*>(
+        Bws + (((size_t)seq * n_part + pp) * H + hh) * sd + colb + (size_t)r * dv);
+#pragma unroll
+    for (int c = 0; c < CTC_COLS / 4; ++c) {
+      const float4 v = __ldg(bsrc + c);
+      x[4 * c] = v.x, x[4 * c + 1] = v.y, x[4 * c + 2] = v.z, x[4 * c + 3] = v.w;
+    }
+    // M_pp landed: split it in place into its hi (A_hi) and lo (A_lo) halves;
+    // thread r owns the 512 bytes of row r in every slab
+    if (__syncthreads_or(!mbar_wait_bounded(&bars[0], pp & 1, s_abort, status))) {
+      ok = false;
+      break;
+    }
+#pragma unroll 4
+    for (int u = 0; u < 32; ++u) {
+      const uint32_t off = (uint32_t)(u >> 3) * 16384 + (uint32_t)r * 128 + (uint32_t)(u & 7) * 16;
+      float4* ph = reinterpret_cast<float4*>(sm + CTC_OFF_AH + off);
+      const float4 v = *ph;
+      float4 hi, lo;
+      hi.x = tf32_round(v.x), hi.y = tf32_round(v.y), hi.z = tf32_round(v.z), hi.w = tf32_round(v.w);
+      lo.x = tf32_round(v.x - hi.x), lo.y = tf32_round(v.y - hi.y);
+      lo.z = tf32_round(v.z - hi.z), lo.w = tf32_round(v.w - hi.w);
+      *ph = hi;
+      *reinterpret_cast<float4*>(sm + CTC_OFF_AL + off) = lo;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t idesc = idesc_tf32_kmn(128, CTC_COLS);
+#pragma unroll
+        for (int term = 0; term < 3; ++term) {
+          const uint32_t a = sbase + (term == 2 ? CTC_OFF_AL : CTC_OFF_AH);
+          const uint32_t b = sbase + (term == 1 ? CTC_OFF_BL : CTC_OFF_BH);
+#pragma unroll
+          for (int kk = 0; kk < DK / 8; ++kk)
+            mma_tf32_tc(tmem, kdesc(a + (kk >> 2) * 16384 + (kk & 3) * 32), mndesc(b + kk * 1024, 16384), idesc,
+                        (term > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars[1]);
+      }
+      __syncwarp();
+    }
+    if (__syncthreads_or(!mbar_wait_bounded(&bars[1], pp & 1, s_abort, status))) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    if (tid == 0 && pp + 1 < n_steps) load_m(pp + 1);  // A tiles are free again
+    {
+      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+      float acc[32];
+#pragma unroll
+      for (int half = 0; half < CTC_COLS / 32; ++half) {
+        tmem_ld32(tmem + lane_off + half * 32, acc);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[half * 32 + e] += acc[e];
+      }
+    }
+    tc_fence_before();
+    __syncthreads();                                   // every B read done before it is rewritten
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, CTC_COLS);
+  }
+}
+
 // Output correction of the corrected segmented schedule.  Segment p >= 1 of a
 // chain ran from a zero state in the state pass and wrote its zero-start
 // outputs o^0 into o; its transition slice wrote qhat_i = scale og_i
@@ -1393,30 +1629,33 @@ __global__ void __launch_bounds__(256)
 //     o_i = o^0_i + S_p^T qhat_i,
 // which this kernel adds for one (sequence, head, 128-wide dv slice) and a
 // tile of up to 128 tokens of one segment, then applies the loop residual.
-// Every operand arrives by TMA in the 128-byte swizzle: qhat (K-major A),
-// S_p rounded to bf16 by the combine (MN-major B: rows of dk, 64 columns of
-// dv per 128-byte row), o^0 and h_prev (token rows); the product is one
-// tcgen05 MMA chain (M = 128 tokens, N = 128 columns of dv, K = dk = 128) into
-// tensor memory.  The result is written over the o^0 tile in shared memory
-// and stored as 16-byte coalesced rows.  Launched as a programmatic
-// dependent: h_prev (an input) is requested first, everything the state pass
-// and the combine wrote only after griddepcontrol.wait.
+// qhat (K-major A), S_p rounded to bf16 by the combine (MN-major B: rows of
+// dk, 64 columns of dv per 128-byte row) and o^0 arrive by TMA in the 128-byte
+// swizzle; the product is one tcgen05 MMA chain (M = 128 tokens, N = 128
+// columns of dv, K = dk = 128) into tensor memory.  Thread r adds row r of
+// the product to o^0 and writes the sum, rounded to bf16, over the o^0 tile;
+// the tile then leaves as coalesced 16-byte rows, each with the loop residual
+// rho (.) h_prev added (h_prev read where it is stored, after an L2 prefetch
+// issued at entry; rho staged in shared memory).  96 KB of shared memory: two
+// CTAs per SM.  Launched as a programmatic dependent: inputs are touched
+// before griddepcontrol.wait, anything the state pass or the combine wrote
+// only after it.
 constexpr int COR_THREADS = 128;
 constexpr int COR_ROWS = 128;                      // tokens per tile
 constexpr uint32_t COR_TILE = 32768;               // 128 rows x 128 bf16 in two 64-column slabs
 constexpr uint32_t COR_OFF_A = 0;                  // qhat
 constexpr uint32_t COR_OFF_B = COR_OFF_A + COR_TILE;   // S_p (bf16, MN-major)
-constexpr uint32_t COR_OFF_O = COR_OFF_B + COR_TILE;   // o^0, then the result
-constexpr uint32_t COR_OFF_H = COR_OFF_O + COR_TILE;   // h_prev
-constexpr uint32_t COR_OFF_BAR = COR_OFF_H + COR_TILE; // 3 mbarriers, tmem base, abort flag
+constexpr uint32_t COR_OFF_O = COR_OFF_B + COR_TILE;   // o^0, then o^0 + S_p^T qhat
+constexpr uint32_t COR_OFF_RHO = COR_OFF_O + COR_TILE; // rho of the slice (128 fp32)
+constexpr uint32_t COR_OFF_BAR = COR_OFF_RHO + 512;    // 3 mbarriers, tmem base, abort flag
 constexpr uint32_t COR_SMEM = COR_OFF_BAR + 64 + 1024;
 
 struct CorParams {
   __nv_bfloat16* o;
-  const float* rho;              // loop residual's rho (with h_prev), or null
+  const __nv_bfloat16* h_prev;   // loop residual input (or null) and its rho
+  const float* rho;
   unsigned* status;
   int H, dv, n_slices, seq_len, seg0_tok, seg_tok, n_segs, tiles_mid, tiles_per_seq;
-  int residual;
 };
 
 // One 128-token tile of a [tokens][H][width] map (two 64-column slabs, two
@@ -1437,10 +1676,9 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-__global__ void __launch_bounds__(COR_THREADS, 1)
+__global__ void __launch_bounds__(COR_THREADS, 2)
     gdn_segment_correct_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_sb,
-                               const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_h,
-                               const CorParams p) {
+                               const __grid_constant__ CUtensorMap tm_o, const CorParams p) {
   extern __shared__ __align__(1024) uint8_t csm_raw[];
   uint8_t* sm = csm_raw;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1448,10 +1686,11 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
     if (tid == 0) record_status(p.status, GDN_ERR_CUDA);
     return;
   }
-  // [0] qhat and S_p landed, [1] o^0 (and h_prev) landed, [2] MMA done
+  // [0] qhat and S_p landed, [1] o^0 landed, [2] MMA done
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + COR_OFF_BAR);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + COR_OFF_BAR + 24);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + COR_OFF_BAR + 28);
+  float* s_rho = reinterpret_cast<float*>(sm + COR_OFF_RHO);
   // block -> (sequence, head, slice, tile); tiles enumerate segments 1 .. n_segs-1
   int bid = (int)blockIdx.x;
   const int tile = bid % p.tiles_per_seq;
@@ -1476,6 +1715,7 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
   const int col0 = slice * DVS;
   // row of S_p in the [n_seq * (n_segs-1) * H * dk][dv] view of the bf16 start states
   const int sb_row = ((seq * (p.n_segs - 1) + (part - 1)) * p.H + h) * DK;
+  const size_t row_elems = (size_t)p.H * p.dv;
 
   if (tid == 0) {
     for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
@@ -1486,6 +1726,17 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
     tmem_alloc(s_tmem, 128);
     tmem_relinquish();
   }
+  // inputs first: rho into shared memory, this tile's h_prev rows into L2
+  if (p.h_prev) {
+    s_rho[tid] = __ldg(p.rho + (size_t)h * p.dv + col0 + tid);
+    for (int u = tid; u < 2 * COR_ROWS; u += COR_THREADS) {
+      const int i = u >> 1;
+      if (i < rows) {
+        const __nv_bfloat16* line = p.h_prev + (size_t)(tok0 + i) * row_elems + (size_t)h * p.dv + col0 + (u & 1) * 64;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(line));
+      }
+    }
+  }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -1493,19 +1744,16 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = smem_u32(sm);
   const bool have_rows = rows > 0;
+  griddep_wait();                                  // qhat, o^0 and S_p are written
   if (tid == 0 && have_rows) {
     tma_prefetch_desc(&tm_qh);
     tma_prefetch_desc(&tm_sb);
     tma_prefetch_desc(&tm_o);
-    mbar_arrive_expect_tx(&bars[1], p.residual ? 2 * COR_TILE : COR_TILE);
-    if (p.residual) cor_load_rows(sm + COR_OFF_H, &tm_h, &bars[1], col0, h, tok0);   // an input
-  }
-  griddep_wait();                                  // qhat, o^0 and S_p are written
-  if (tid == 0 && have_rows) {
     mbar_arrive_expect_tx(&bars[0], 2 * COR_TILE);
     cor_load_rows(sm + COR_OFF_A, &tm_qh, &bars[0], 0, h, tok0);
     tma_load_2d(sm + COR_OFF_B, &tm_sb, &bars[0], col0, sb_row);
     tma_load_2d(sm + COR_OFF_B + 16384, &tm_sb, &bars[0], col0 + 64, sb_row);
+    mbar_arrive_expect_tx(&bars[1], COR_TILE);
     cor_load_rows(sm + COR_OFF_O, &tm_o, &bars[1], col0, h, tok0);
   }
   bool ok = have_rows;
@@ -1525,7 +1773,8 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
   if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[2], 0, s_abort, p.status));
   tc_fence_after();
   if (ok) {
-    // thread: token row r of the tile; the result replaces o^0 in shared memory
+    // thread: token row r of the tile; o^0 + S_p^T qhat, rounded to bf16 (the
+    // output as it would be stored), replaces o^0 in shared memory
     const int r = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 #pragma unroll 1
@@ -1536,42 +1785,35 @@ __global__ void __launch_bounds__(COR_THREADS, 1)
       const uint32_t slab = (uint32_t)(cbase >> 6) * 16384;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int col = (cbase & 63) + c * 8;
-        uint4* ov = reinterpret_cast<uint4*>(sm + COR_OFF_O + slab + sw128_offset(r, col));
+        uint4* ov = reinterpret_cast<uint4*>(sm + COR_OFF_O + slab + sw128_offset(r, (cbase & 63) + c * 8));
         const uint4 x = *ov;
-        float y[8] = {bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y),
-                      bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w)};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] += acc[c * 8 + e];
-        if (p.residual) {
-          // the loop residual on the output rounded to bf16, as loop_residual sees it
-          const uint4 hp = *reinterpret_cast<const uint4*>(sm + COR_OFF_H + slab + sw128_offset(r, col));
-          const float hv[8] = {bf16_lo(hp.x), bf16_hi(hp.x), bf16_lo(hp.y), bf16_hi(hp.y),
-                               bf16_lo(hp.z), bf16_hi(hp.z), bf16_lo(hp.w), bf16_hi(hp.w)};
-          const float4 r0 = __ldg(reinterpret_cast<const float4*>(p.rho + (size_t)h * p.dv + col0 + cbase + c * 8));
-          const float4 r1 = __ldg(reinterpret_cast<const float4*>(p.rho + (size_t)h * p.dv + col0 + cbase + c * 8 + 4));
-          const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = fmaf(rr[e], hv[e], __bfloat162float(__float2bfloat16_rn(y[e])));
-        }
         uint4 v;
-        v.x = pack_bf16x2(y[0], y[1]);
-        v.y = pack_bf16x2(y[2], y[3]);
-        v.z = pack_bf16x2(y[4], y[5]);
-        v.w = pack_bf16x2(y[6], y[7]);
+        v.x = pack_bf16x2(bf16_lo(x.x) + acc[c * 8 + 0], bf16_hi(x.x) + acc[c * 8 + 1]);
+        v.y = pack_bf16x2(bf16_lo(x.y) + acc[c * 8 + 2], bf16_hi(x.y) + acc[c * 8 + 3]);
+        v.z = pack_bf16x2(bf16_lo(x.z) + acc[c * 8 + 4], bf16_hi(x.z) + acc[c * 8 + 5]);
+        v.w = pack_bf16x2(bf16_lo(x.w) + acc[c * 8 + 6], bf16_hi(x.w) + acc[c * 8 + 7]);
         *ov = v;
       }
     }
     __syncthreads();
-    // coalesced 16-byte stores of the valid rows (a row past the segment
-    // belongs to another segment or sequence and is not touched)
+    // coalesced 16-byte rows with the loop residual; a row past the segment
+    // belongs to another segment or sequence and is not touched
 #pragma unroll 4
     for (int it = tid; it < COR_ROWS * 16; it += COR_THREADS) {
       const int i = it >> 4, chunk = it & 15;
       if (i < rows) {
-        const uint4 v = *reinterpret_cast<const uint4*>(sm + COR_OFF_O + (chunk >> 3) * 16384 +
-                                                        sw128_offset(i, (chunk & 7) * 8));
-        __stcs(reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + i) * p.H + h) * p.dv + col0 + chunk * 8), v);
+        uint4 v = *reinterpret_cast<const uint4*>(sm + COR_OFF_O + (chunk >> 3) * 16384 +
+                                                  sw128_offset(i, (chunk & 7) * 8));
+        const size_t off = (size_t)(tok0 + i) * row_elems + (size_t)h * p.dv + col0 + chunk * 8;
+        if (p.h_prev) {
+          const uint4 y = *reinterpret_cast<const uint4*>(p.h_prev + off);
+          const float* rr = s_rho + chunk * 8;
+          v.x = pack_bf16x2(fmaf(rr[0], bf16_lo(y.x), bf16_lo(v.x)), fmaf(rr[1], bf16_hi(y.x), bf16_hi(v.x)));
+          v.y = pack_bf16x2(fmaf(rr[2], bf16_lo(y.y), bf16_lo(v.y)), fmaf(rr[3], bf16_hi(y.y), bf16_hi(v.y)));
+          v.z = pack_bf16x2(fmaf(rr[4], bf16_lo(y.z), bf16_lo(v.z)), fmaf(rr[5], bf16_hi(y.z), bf16_hi(v.z)));
+          v.w = pack_bf16x2(fmaf(rr[6], bf16_lo(y.w), bf16_lo(v.w)), fmaf(rr[7], bf16_hi(y.w), bf16_hi(v.w)));
+        }
+        __stcs(reinterpret_cast<uint4*>(p.o + off), v);
       }
     }
   }
@@ -1817,9 +2059,23 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
       tc_launch(mq, mk, mv, kp, chains * (kp.n_slices + (long long)n_part * (kp.n_slices + 1)), stream);
   if (st != GDN_OK) return st;
   // combine: start states S_2 .. S_{P-1} (and S_T in the corrected schedule,
-  // with every start state also in bf16 for the correction)
+  // with every start state also in bf16 for the correction; there on the
+  // tensor cores)
   const int n_steps = plan.corrected ? (p->S_T ? P - 1 : P - 2) : P - 2;
-  if (n_steps > 0 || plan.corrected) {
+  if (plan.corrected) {
+    CUtensorMap mm;
+    if (!make_map_2d(&mm, kp.Mws, tc::DK, (long long)p->n_seq * n_part * p->H * tc::DK, 32, 128, 4))
+      return GDN_ERR_CUDA;
+    const long long cblocks = chains * (p->dv / tc::CTC_COLS);
+    if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    static std::atomic<bool> ctc_attr_set[kMaxDevices];
+    if (smem_attr_once(ctc_attr_set, tc::gdn_segment_combine_tc_kernel, tc::CTC_SMEM) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    LaunchCfg lc((unsigned)cblocks, tc::CTC_THREADS, tc::CTC_SMEM, stream, /*dependent=*/true);
+    if (cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_combine_tc_kernel, mm, (const float*)kp.Bws, kp.Sst, p->S_T,
+                           Sb, status, p->H, p->dv, P, n_part, n_steps) != cudaSuccess)
+      return GDN_ERR_CUDA;
+  } else if (n_steps > 0) {
     const long long cblocks = chains * (p->dv / tc::CMB_COLS);
     if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     static std::atomic<bool> cmb_attr_set[kMaxDevices];
@@ -1827,8 +2083,8 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
       return GDN_ERR_CUDA;
     LaunchCfg lc((unsigned)cblocks, 256, tc::CMB_SMEM, stream, /*dependent=*/true);
     if (cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_combine_kernel, (const float*)kp.Bws,
-                           (const float*)kp.Mws, kp.Sst, plan.corrected ? p->S_T : nullptr, Sb, p->H,
-                           p->dv, P, n_part, n_steps) != cudaSuccess)
+                           (const float*)kp.Mws, kp.Sst, nullptr, nullptr, p->H, p->dv, P, n_part,
+                           n_steps) != cudaSuccess)
       return GDN_ERR_CUDA;
   }
   if (!plan.corrected) {
@@ -1836,16 +2092,15 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
     return tc_launch(mq, mk, mv, kp, chains * (P - 1) * kp.n_slices, stream, /*dependent=*/true);
   }
   // correction of the outputs of segments 1 .. P-1
-  CUtensorMap mqh, msb, mo, mh;
+  CUtensorMap mqh, msb, mo;
   if (!make_map(&mqh, kp.qhat, tc::DK, p->H, p->total_tokens) ||
       !make_map_2d(&msb, Sb, p->dv, (long long)p->n_seq * (P - 1) * p->H * tc::DK, 64, 128) ||
-      !make_map(&mo, p->o, p->dv, p->H, p->total_tokens) ||
-      !make_map(&mh, p->h_prev ? p->h_prev : p->o, p->dv, p->H, p->total_tokens))
+      !make_map(&mo, p->o, p->dv, p->H, p->total_tokens))
     return GDN_ERR_CUDA;
   tc::CorParams cp;
   cp.o = kp.o;
+  cp.h_prev = kp.h_prev;
   cp.rho = kp.rho;
-  cp.residual = p->h_prev != nullptr;
   cp.status = status;
   cp.H = p->H;
   cp.dv = p->dv;
@@ -1864,7 +2119,7 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   if (smem_attr_once(cor_attr_set, tc::gdn_segment_correct_kernel, tc::COR_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
   LaunchCfg lc((unsigned)cor_blocks, tc::COR_THREADS, tc::COR_SMEM, stream, /*dependent=*/true);
-  return cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_correct_kernel, mqh, msb, mo, mh, cp) == cudaSuccess
+  return cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_correct_kernel, mqh, msb, mo, cp) == cudaSuccess
              ? GDN_OK
              : GDN_ERR_CUDA;
 }

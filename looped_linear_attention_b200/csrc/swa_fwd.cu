@@ -8,19 +8,23 @@
 // t of a sequence starting at t0, over the keys j in [max(t0, t - w + 1), t]:
 //     o_t = sum_j softmax_j(scale q_t . k_j) v_j.
 //
-// One CTA of 128 threads per (sequence, head, tile of 128 queries) walks the
+// One CTA of 256 threads per (sequence, head, tile of 128 queries) walks the
 // 128-key tiles that the tile's windows touch, flash-attention style:
 //   * Q (once), K and V tiles (double-buffered) arrive by TMA in the 128-byte
 //     swizzle; S = Q K^T and O += P V are tcgen05 MMAs (M = 128 queries,
 //     N = 128, K = 128) issued by one thread, accumulating in tensor memory
 //     (two S buffers, so S of the next tile runs while this one's softmax is
 //     computed, and O);
-//   * thread r owns query row r (tensor-memory lane r): it masks the row to
-//     its window, keeps the running maximum m and sum l in base 2, writes
-//     P = 2^(s - m) as the bf16 A operand of the next MMA, and rescales its O
-//     row in tensor memory only when the maximum grew by more than 2^8
-//     (otherwise the stale maximum keeps every P <= 2^8; the result is the
-//     same after the final division by l);
+//   * two threads own query row r (tensor-memory lane r), one per half of
+//     the 128 keys (warps w and w + 4 reach the same lanes): each loads its
+//     half of the S row into registers once, masks it to the row's window
+//     (tiles that lie inside every row's window skip the mask), and the two
+//     exchange their partial maxima through shared memory; the running
+//     maximum m is kept in base 2, each thread keeps its partial sum of
+//     P = 2^(s - m), writes its half of P as the bf16 A operand of the next
+//     MMA, and rescales its half of the O row in tensor memory only when the
+//     maximum grew by more than 2^8 (otherwise the stale maximum keeps every
+//     P <= 2^8; the result is the same after the final division by l);
 //   * K of tile t+2 is loaded once S_t is done, V of tile t+1 once O of tile
 //     t-1 is done; every wait is bounded (GDN_ERR_TIMEOUT).
 // The epilogue divides by l and stores bf16 rows, staged through shared
@@ -34,13 +38,14 @@ namespace swa {
 constexpr int D = 128;        // head width of q, k and v
 constexpr int BM = 128;       // queries per CTA
 constexpr int BN = 128;       // keys per tile
-constexpr int THREADS = 128;
+constexpr int THREADS = 256;     // two threads per query row
 constexpr uint32_t TILE_BYTES = 32768;           // 128 rows x 128 bf16, two 64-column slabs
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + TILE_BYTES;    // 2 buffers
 constexpr uint32_t OFF_V = OFF_K + 2 * TILE_BYTES;  // 2 buffers
 constexpr uint32_t OFF_P = OFF_V + 2 * TILE_BYTES;  // P (bf16 A operand); output staging
-constexpr uint32_t OFF_BAR = OFF_P + TILE_BYTES;
+constexpr uint32_t OFF_RED = OFF_P + TILE_BYTES;   // [2 halves][128 rows] fp32 partial maxima / sums
+constexpr uint32_t OFF_BAR = OFF_RED + 2 * BM * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
 // tensor-memory columns: S (two buffers) and O
@@ -170,14 +175,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   ok = !__syncthreads_or(*s_abort != 0);
 
-  const int r = tid;                               // query row of this thread
+  const int quad = warp & 3, hf = warp >> 2;      // tensor-memory lane block, key / column half
+  const int r = quad * 32 + lane;                  // query row of this thread
   const int q_tok = q0 + r;
   const bool row_valid = q_tok < seq_end;
   const int win_lo = q_tok - p.window + 1;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  float m_run = -1e30f, l_run = 0.f;               // running maximum (base 2) and sum
+  const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+  float* s_red = reinterpret_cast<float*>(sm + OFF_RED);   // [hf][row]
+  float m_run = -1e30f, l_run = 0.f;               // running maximum (base 2); this half's sum
+  // tiles that lie inside every row's window (and rows all inside the
+  // sequence) need no mask
+  const bool rows_full = q0 + BM <= seq_end;
   for (int t = 0; t < n_tiles && ok; ++t) {
     const int kt0 = key_tok(t);
+    const bool interior = rows_full && kt0 + BN - 1 <= q0 && kt0 >= q0 + BM - 1 - p.window + 1;
     // ---- S_t is in tensor memory
     if (__syncthreads_or(!mbar_wait_bounded(&bars[B_S + (t & 1)], (t >> 1) & 1, s_abort, p.status))) break;
     tc_fence_after();
@@ -195,20 +206,36 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       __syncwarp();
     }
-    // ---- pass 1: the row maximum of this tile over the row's window (base 2)
-    const uint32_t s_col = tmem + lane_off + COL_S + (t & 1) * BN;
+    // ---- this thread's half of the S row (64 keys), scaled to base 2 and masked
+    float x[64];
+    {
+      const uint32_t s_col = tmem + lane_off + COL_S + (t & 1) * BN + hf * 64;
+      float* x0 = x;
+      float* x1 = x + 32;
+      tmem_ld32(s_col, *reinterpret_cast<float(*)[32]>(x0));
+      tmem_ld32(s_col + 32, *reinterpret_cast<float(*)[32]>(x1));
+    }
     float tmax = -INFINITY;
-#pragma unroll 1
-    for (int piece = 0; piece < BN / 32; ++piece) {
-      float x[32];
-      tmem_ld32(s_col + piece * 32, x);
+    if (interior) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int j = kt0 + piece * 32 + e;
+      for (int e = 0; e < 64; ++e) {
+        x[e] *= p.scale_log2;
+        tmax = fmaxf(tmax, x[e]);
+      }
+    } else {
+      const int j0 = kt0 + hf * 64;
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const int j = j0 + e;
         const bool in = row_valid && j <= q_tok && j >= win_lo;
-        tmax = fmaxf(tmax, in ? x[e] * p.scale_log2 : -INFINITY);
+        x[e] = in ? x[e] * p.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, x[e]);
       }
     }
+    // ---- the row maximum from both halves
+    s_red[hf * BM + r] = tmax;
+    __syncthreads();
+    tmax = fmaxf(tmax, s_red[(hf ^ 1) * BM + r]);
     const float m_new = fmaxf(m_run, tmax);
     // lazy rescale: only when the maximum grew by more than 8 (in base 2)
     const bool grow = (t > 0) && (m_new > m_run + 8.f);
@@ -226,42 +253,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (__any_sync(0xffffffffu, grow)) {
         l_run *= alpha;
 #pragma unroll 1
-        for (int piece = 0; piece < D / 32; ++piece) {
+        for (int piece = 0; piece < 2; ++piece) {
           float y[32];
-          tmem_ld32(tmem + lane_off + COL_O + piece * 32, y);
+          const uint32_t oc = tmem + lane_off + COL_O + hf * 64 + piece * 32;
+          tmem_ld32(oc, y);
 #pragma unroll
           for (int e = 0; e < 32; ++e) y[e] *= alpha;
-          tmem_st32(tmem + lane_off + COL_O + piece * 32, y);
+          tmem_st32(oc, y);
         }
         tmem_wait_st();
       }
     }
-    // ---- pass 2: P = 2^(s - m) (bf16, swizzled A operand), l += sum P
-    float lsum = 0.f;
-#pragma unroll 1
-    for (int piece = 0; piece < BN / 32; ++piece) {
-      float x[32];
-      tmem_ld32(s_col + piece * 32, x);
+    // ---- P = 2^(s - m) (bf16, swizzled A operand, slab hf), l += sum P
+    {
+      float lsum = 0.f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int j = kt0 + piece * 32 + e;
-        const bool in = row_valid && j <= q_tok && j >= win_lo;
-        x[e] = in ? ex2(x[e] * p.scale_log2 - m_run) : 0.f;
+      for (int e = 0; e < 64; ++e) {
+        x[e] = ex2(x[e] - m_run);                  // masked entries: 2^-inf = 0
         lsum += x[e];
       }
-      const int c0 = piece * 32;
-      uint8_t* slab = sm + OFF_P + (c0 >> 6) * 16384;
+      l_run += lsum;
+      uint8_t* slab = sm + OFF_P + hf * 16384;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 8; ++c) {
         uint4 o;
         o.x = pack_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
         o.y = pack_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
         o.z = pack_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
         o.w = pack_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
-        *reinterpret_cast<uint4*>(slab + sw128_offset(r, (c0 & 63) + c * 8)) = o;
+        *reinterpret_cast<uint4*>(slab + sw128_offset(r, c * 8)) = o;
       }
     }
-    l_run += lsum;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -287,12 +309,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     ok = !__syncthreads_or(!mbar_wait_bounded(&bars[B_O], (n_tiles - 1) & 1, s_abort, p.status));
   tc_fence_after();
   if (ok) {
-    const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    s_red[hf * BM + r] = l_run;                    // the two halves' sums
+    __syncthreads();
+    const float l = l_run + s_red[(hf ^ 1) * BM + r];
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
     uint8_t* stage = sm + OFF_P;                   // [128 rows][256 B], 16-byte chunks XOR-swizzled
 #pragma unroll 1
-    for (int piece = 0; piece < D / 32; ++piece) {
+    for (int piece = 0; piece < 2; ++piece) {
       float y[32];
-      tmem_ld32(tmem + lane_off + COL_O + piece * 32, y);
+      tmem_ld32(tmem + lane_off + COL_O + hf * 64 + piece * 32, y);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint4 o;
@@ -300,7 +325,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         o.y = pack_bf16x2(y[c * 8 + 2] * inv, y[c * 8 + 3] * inv);
         o.z = pack_bf16x2(y[c * 8 + 4] * inv, y[c * 8 + 5] * inv);
         o.w = pack_bf16x2(y[c * 8 + 6] * inv, y[c * 8 + 7] * inv);
-        const int chunk = piece * 4 + c;
+        const int chunk = hf * 8 + piece * 4 + c;
         *reinterpret_cast<uint4*>(stage + r * 256 + ((chunk ^ (r & 15)) * 16)) = o;
       }
     }

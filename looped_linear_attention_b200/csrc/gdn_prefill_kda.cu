@@ -157,13 +157,15 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
       for (int d = 0; d < DK; ++d) row[d] = to_f32(from_f32<T>(row[d] * inv));
     }
     __syncthreads();
-    // ---- A and P, each term with its own decay e^{G_ic - G_jc}
+    // ---- A and P, each term with its own decay e^{G_ic - G_jc} (the fast
+    // exponential: a few ulp on arguments <= 0, far inside the fp32 bar)
     for (int e = tid; e < C * C; e += THREADS) {
       const int i = e / C, j = e % C;
       float kk = 0.f, qk = 0.f;
       if (j <= i) {
+#pragma unroll 8
         for (int d = 0; d < DK; ++d) {
-          const float dec = expf(sG[i * LDK + d] - sG[j * LDK + d]);
+          const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
           const float kj = sK[j * LDK + d] * dec;
           kk = fmaf(sK[i * LDK + d], kj, kk);
           qk = fmaf(sQ[i * LDK + d], kj, qk);

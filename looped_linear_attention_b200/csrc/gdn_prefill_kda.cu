@@ -159,20 +159,30 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
     __syncthreads();
     // ---- A and P, each term with its own decay e^{G_ic - G_jc} (the fast
     // exponential: a few ulp on arguments <= 0, far inside the fp32 bar)
-    for (int e = tid; e < C * C; e += THREADS) {
-      const int i = e / C, j = e % C;
+    // (only the lower triangle j <= i is enumerated; the upper one is zero)
+    for (int e = tid; e < C * (C + 1) / 2; e += THREADS) {
+      int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+      while (i * (i + 1) / 2 > e) --i;
+      while ((i + 1) * (i + 2) / 2 <= e) ++i;
+      const int j = e - i * (i + 1) / 2;
       float kk = 0.f, qk = 0.f;
-      if (j <= i) {
 #pragma unroll 8
-        for (int d = 0; d < DK; ++d) {
-          const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
-          const float kj = sK[j * LDK + d] * dec;
-          kk = fmaf(sK[i * LDK + d], kj, kk);
-          qk = fmaf(sQ[i * LDK + d], kj, qk);
-        }
+      for (int d = 0; d < DK; ++d) {
+        const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
+        const float kj = sK[j * LDK + d] * dec;
+        kk = fmaf(sK[i * LDK + d], kj, kk);
+        qk = fmaf(sQ[i * LDK + d], kj, qk);
       }
       sA[i * LDC + j] = (j < i) ? sb[i] * kk : 0.f;
-      sP[i * LDC + j] = (j <= i) ? qk : 0.f;
+      sP[i * LDC + j] = qk;
+    }
+    for (int e = tid; e < C * (C - 1) / 2; e += THREADS) {   // the strict upper triangle
+      int j = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+      while (j * (j + 1) / 2 > e) --j;
+      while ((j + 1) * (j + 2) / 2 <= e) ++j;
+      const int i = e - j * (j + 1) / 2;            // i <= j, then shifted: column j + 1 > row i
+      sA[i * LDC + j + 1] = 0.f;
+      sP[i * LDC + j + 1] = 0.f;
     }
     if (tid < DK) sgc[tid] = sG[(C - 1) * LDK + tid];   // G_C (rows past the end keep it)
     __syncthreads();

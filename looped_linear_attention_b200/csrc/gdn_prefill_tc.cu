@@ -389,10 +389,11 @@ __device__ __forceinline__ void store_res_t12(uint8_t* sm, const Gates& G, int a
   }
 }
 
-// Gate inputs of one token (threads 0-63 of the state warpgroup): a, b and the
-// output gate sigmoid(gate) (1 without one), or a = 1, b = 0 past the sequence
-// end.  Issued well before they are used so the global-memory latency is
-// hidden behind a chunk.
+// Gate inputs of one token (threads 0-63 of the state warpgroup): a, b and,
+// with the looped-block epilogue (EPI), the output gate sigmoid(gate) (1
+// without one), or a = 1, b = 0 past the sequence end.  Issued well before
+// they are used so the global-memory latency is hidden behind a chunk.
+template <bool EPI>
 __device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int valid, int h, int t,
                                                  float& a_in, float& bb, float& og) {
   a_in = 1.f;
@@ -402,7 +403,7 @@ __device__ __forceinline__ void load_gate_inputs(const Params& p, int tok0, int 
     const size_t ti = (size_t)(tok0 + t) * p.H + h;
     a_in = __ldg(p.a + ti);
     bb = __ldg(p.b + ti);
-    if (p.gate) og = 1.f / (1.f + __expf(-__ldg(p.gate + ti)));
+    if (EPI && p.gate) og = 1.f / (1.f + __expf(-__ldg(p.gate + ti)));
   }
 }
 
@@ -613,6 +614,9 @@ __device__ __forceinline__ void load_v(uint8_t* sm, uint64_t* bar, const CUtenso
   tma_load_3d(sm + OFF_V, tv, bar, col0, h, tok0);
   tma_load_3d(sm + OFF_V + 8192, tv, bar, col0 + 64, h, tok0);
 }
+// EPI: the looped-block epilogue (output gate, loop residual) is compiled in;
+// the plain mixer call runs the instance without it.
+template <bool EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -670,7 +674,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   // (zero-start outputs, or qhat from the transition slice); the loop residual
   // only where the output is final
   const bool outputs = !partial || p.mode == 3;
-  const bool residual = (p.h_prev != nullptr) && !partial;
+  const bool residual = EPI && (p.h_prev != nullptr) && !partial;
   int seq_start, seq_end;
   if (p.cu_seqlens) {
     seq_start = p.cu_seqlens[seq];
@@ -779,7 +783,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // output gate and 1/|q_i|), times 1/|k_i| on A rows with the norm; the
         // column factor f_j carries 1/|k_j| (and is 1/|k_j| alone on the
         // exponential path)
-        const float sc = (tq < C) ? (l2n ? G.b[i] * G.kn[i] : G.b[i]) : G.qn[i];
+        const float sc = (tq < C) ? (l2n ? G.b[i] * G.kn[i] : G.b[i]) : ((EPI || l2n) ? G.qn[i] : 1.f);
         const int lim = (tq < C) ? i : i + 1;           // columns j < lim are kept
         float gr[32];
         if (zero_half) {
@@ -937,8 +941,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       compute_gates<BAR_STATE>(gates_at(sm, c % 3), s_carry, min(C, seq_end - (seq_start + c * C)), jt,
                                a_in, b_in, og_in);
       if (c + 1 < n_chunks)
-        load_gate_inputs(p, seq_start + (c + 1) * C, min(C, seq_end - (seq_start + (c + 1) * C)), h, jt,
-                         a_in, b_in, og_in);
+        load_gate_inputs<EPI>(p, seq_start + (c + 1) * C, min(C, seq_end - (seq_start + (c + 1) * C)), h,
+                              jt, a_in, b_in, og_in);
       wg_sync<BAR_STATE>();
     };
     // Hands chunk c2 to the prep team once its K, Q tiles have landed: with the
@@ -972,7 +976,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       return true;
     };
     if (ok && n_chunks > 0) {
-      load_gate_inputs(p, seq_start, min(C, len), h, jt, a_in, b_in, og_in);
+      load_gate_inputs<EPI>(p, seq_start, min(C, len), h, jt, a_in, b_in, og_in);
       gates_of(0);
       if (n_chunks > 1) gates_of(1);
 #pragma unroll 1
@@ -1142,7 +1146,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(tmem + lane_off + COL_OB + 32 * hf, ob);
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 g4 = *reinterpret_cast<const float4*>(G.gq + 32 * hf + 4 * e4);
+            const float4 g4 = *reinterpret_cast<const float4*>(((EPI || l2n) ? G.gq : G.gamma) + 32 * hf + 4 * e4);
             const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -1385,242 +1389,6 @@ __global__ void __launch_bounds__(256)
     __syncthreads();                                // every read of S_pp and M_pp is done
   }
 }
-// The combine on the 5th-generation tensor cores (corrected schedule).  For
-// one (sequence, head, 64 columns of dv), S_{p+1} = M_p S_p + B_p for
-// p = 1 .. n_steps, with the product as tcgen05 MMAs of kind::tf32 in three
-// terms, M_hi S_hi + M_hi S_lo + M_lo S_hi (x = hi + lo, hi = tf32(x),
-// lo = tf32(x - hi)): fp32-level accuracy, M = 128 rows of M_p, N = 64,
-// K = 128, accumulated in tensor memory.  M_p (fp32, written by the
-// transition slice) arrives by TMA into the hi tile in the 128-byte swizzle
-// (K-major, 32 K-elements per 128-byte row) and is split in place; S_p lives
-// in shared memory as the MN-major B operand (32 columns per 128-byte row).
-// M_{p+1} is requested as soon as the product of step p has read M_p.  Every
-// start state is written in fp32 (Sst, or S_T for the last) and rounded to
-// bf16 (Sb) for the correction.
-constexpr int CTC_THREADS = 128;
-constexpr int CTC_COLS = 64;                          // columns of dv per CTA
-constexpr uint32_t CTC_A_BYTES = 65536;               // 128 x 128 fp32
-constexpr uint32_t CTC_B_BYTES = 32768;               // 128 x 64 fp32
-constexpr uint32_t CTC_OFF_AH = 0;
-constexpr uint32_t CTC_OFF_AL = CTC_OFF_AH + CTC_A_BYTES;
-constexpr uint32_t CTC_OFF_BH = CTC_OFF_AL + CTC_A_BYTES;
-constexpr uint32_t CTC_OFF_BL = CTC_OFF_BH + CTC_B_BYTES;
-constexpr uint32_t CTC_OFF_BAR = CTC_OFF_BL + CTC_B_BYTES;
-constexpr uint32_t CTC_SMEM = CTC_OFF_BAR + 64 + 1024;
-static_assert(CTC_SMEM <= 232448, "tensor-core combine exceeds shared memory");
-
-// kind::tf32 instruction descriptor: fp32 D, tf32 A (K-major) and B (MN-major).
-__host__ __device__ constexpr uint32_t idesc_tf32_kmn(int M, int N) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | (1u << 16) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-__device__ __forceinline__ void mma_tf32_tc(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ float tf32_round(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
-}
-// Byte offset of fp32 element (k, n) of the MN-major B tile: 32-column blocks
-// 16 KB apart, row k 128 bytes, 16-byte chunks XOR (k mod 8).
-__device__ __forceinline__ uint32_t ctc_b_offset(int k, int n) {
-  const int chunk = ((n & 31) >> 2) ^ (k & 7);
-  return (uint32_t)((n >> 5) * 16384 + k * 128 + chunk * 16 + (n & 3) * 4);
-}
-
-__global__ void __launch_bounds__(CTC_THREADS, 1)
-    gdn_segment_combine_tc_kernel(const __grid_constant__ CUtensorMap tm_m, const float* __restrict__ Bws,
-                                  float* __restrict__ Sst, float* __restrict__ S_T,
-                                  __nv_bfloat16* __restrict__ Sb, unsigned* status, int H, int dv,
-                                  int n_segs, int n_part, int n_steps) {
-  extern __shared__ __align__(1024) uint8_t ctc_raw[];
-  uint8_t* sm = ctc_raw;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  // launched as a programmatic dependent of the state pass: let the
-  // correction launch, then wait for the state pass before reading its results
-  griddep_launch_dependents();
-  if (smem_u32(sm) & 1023u) {
-    if (tid == 0) record_status(status, GDN_ERR_CUDA);
-    return;
-  }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CTC_OFF_BAR);    // [0] M landed, [1] MMA done
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CTC_OFF_BAR + 16);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + CTC_OFF_BAR + 20);
-  const int ncb = dv / CTC_COLS;
-  const int cb = blockIdx.x % ncb;
-  const int hh = (blockIdx.x / ncb) % H;
-  const int seq = blockIdx.x / (ncb * H);
-  const size_t sd = (size_t)DK * dv;
-  const size_t colb = (size_t)cb * CTC_COLS;
-  const int r = tid;                                   // row of the state / of M_p
-  auto sptr = [&](int pp) -> float* {                  // S_{pp+1}
-    if (pp <= n_segs - 2) return Sst + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb;
-    return S_T ? S_T + ((size_t)seq * H + hh) * sd + colb : nullptr;
-  };
-  // row of M_p (slot pp) in the [n_seq * n_part * H * dk][dk] view of the transitions
-  auto m_row = [&](int pp) { return ((seq * n_part + pp) * H + hh) * DK; };
-  auto load_m = [&](int pp) {
-    mbar_arrive_expect_tx(&bars[0], CTC_A_BYTES);
-#pragma unroll
-    for (int sl = 0; sl < 4; ++sl) {
-      asm volatile(
-          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-          " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(sm + CTC_OFF_AH + sl * 16384)),
-          "l"(reinterpret_cast<uint64_t>(&tm_m)), "r"(sl * 32), "r"(m_row(pp)), "r"(smem_u32(&bars[0]))
-          : "memory");
-    }
-  };
-
-  if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    *s_abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(s_tmem, CTC_COLS);
-    tmem_relinquish();
-  }
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *s_tmem;
-  const uint32_t sbase = smem_u32(sm);
-  griddep_wait();                                      // S_1, B and M are written
-  if (tid == 0 && n_steps > 0) {
-    tma_prefetch_desc(&tm_m);
-    load_m(0);
-  }
-  // x: this thread's row of S_{pp+1} (64 columns), starting from S_1
-  float x[CTC_COLS];
-  {
-    const float4* src = reinterpret_cast<const float4*>(sptr(0) + (size_t)r * dv);
-#pragma unroll
-    for (int c = 0; c < CTC_COLS / 4; ++c) {
-      const float4 v = __ldg(src + c);
-      x[4 * c] = v.x, x[4 * c + 1] = v.y, x[4 * c + 2] = v.z, x[4 * c + 3] = v.w;
-    }
-  }
-  bool ok = true;
-  for (int pp = 0;; ++pp) {
-    // S_{pp+1}: to Sst / S_T (unless it came from there), to Sb in bf16, and
-    // as the hi/lo B operand of the next product
-    float* dst = (pp > 0) ? sptr(pp) : nullptr;
-    if (dst) {
-      float4* d4 = reinterpret_cast<float4*>(dst + (size_t)r * dv);
-#pragma unroll
-      for (int c = 0; c < CTC_COLS / 4; ++c) d4[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
-    }
-    if (Sb && pp <= n_segs - 2) {
-      uint4* b4 = reinterpret_cast<uint4*>(Sb + (((size_t)seq * (n_segs - 1) + pp) * H + hh) * sd + colb +
-                                           (size_t)r * dv);
-#pragma unroll
-      for (int c = 0; c < CTC_COLS / 8; ++c) {
-        uint4 u;
-        u.x = pack_bf16x2(x[8 * c], x[8 * c + 1]);
-        u.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
-        u.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
-        u.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
-        b4[c] = u;
-      }
-    }
-    if (pp >= n_steps || !ok) break;
-#pragma unroll
-    for (int c = 0; c < CTC_COLS / 4; ++c) {
-      float4 hi, lo;
-      hi.x = tf32_round(x[4 * c]);
-      hi.y = tf32_round(x[4 * c + 1]);
-      hi.z = tf32_round(x[4 * c + 2]);
-      hi.w = tf32_round(x[4 * c + 3]);
-      lo.x = tf32_round(x[4 * c] - hi.x);
-      lo.y = tf32_round(x[4 * c + 1] - hi.y);
-      lo.z = tf32_round(x[4 * c + 2] - hi.z);
-      lo.w = tf32_round(x[4 * c + 3] - hi.w);
-      *reinterpret_cast<float4*>(sm + CTC_OFF_BH + ctc_b_offset(r, 4 * c)) = hi;
-      *reinterpret_cast<float4*>(sm + CTC_OFF_BL + ctc_b_offset(r, 4 * c)) = lo;
-    }
-    // B_pp of this row, needed after the product
-    const float4* bsrc = reinterpret_cast<const float4*>(
-        Bws + (((size_t)seq * n_part + pp) * H + hh) * sd + colb + (size_t)r * dv);
-#pragma unroll
-    for (int c = 0; c < CTC_COLS / 4; ++c) {
-      const float4 v = __ldg(bsrc + c);
-      x[4 * c] = v.x, x[4 * c + 1] = v.y, x[4 * c + 2] = v.z, x[4 * c + 3] = v.w;
-    }
-    // M_pp landed: split it in place into its hi (A_hi) and lo (A_lo) halves;
-    // thread r owns the 512 bytes of row r in every slab
-    if (__syncthreads_or(!mbar_wait_bounded(&bars[0], pp & 1, s_abort, status))) {
-      ok = false;
-      break;
-    }
-#pragma unroll 4
-    for (int u = 0; u < 32; ++u) {
-      const uint32_t off = (uint32_t)(u >> 3) * 16384 + (uint32_t)r * 128 + (uint32_t)(u & 7) * 16;
-      float4* ph = reinterpret_cast<float4*>(sm + CTC_OFF_AH + off);
-      const float4 v = *ph;
-      float4 hi, lo;
-      hi.x = tf32_round(v.x), hi.y = tf32_round(v.y), hi.z = tf32_round(v.z), hi.w = tf32_round(v.w);
-      lo.x = tf32_round(v.x - hi.x), lo.y = tf32_round(v.y - hi.y);
-      lo.z = tf32_round(v.z - hi.z), lo.w = tf32_round(v.w - hi.w);
-      *ph = hi;
-      *reinterpret_cast<float4*>(sm + CTC_OFF_AL + off) = lo;
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-      tc_fence_after();
-      if (elect_one()) {
-        const uint32_t idesc = idesc_tf32_kmn(128, CTC_COLS);
-#pragma unroll
-        for (int term = 0; term < 3; ++term) {
-          const uint32_t a = sbase + (term == 2 ? CTC_OFF_AL : CTC_OFF_AH);
-          const uint32_t b = sbase + (term == 1 ? CTC_OFF_BL : CTC_OFF_BH);
-#pragma unroll
-          for (int kk = 0; kk < DK / 8; ++kk)
-            mma_tf32_tc(tmem, kdesc(a + (kk >> 2) * 16384 + (kk & 3) * 32), mndesc(b + kk * 1024, 16384), idesc,
-                        (term > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars[1]);
-      }
-      __syncwarp();
-    }
-    if (__syncthreads_or(!mbar_wait_bounded(&bars[1], pp & 1, s_abort, status))) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-    if (tid == 0 && pp + 1 < n_steps) load_m(pp + 1);  // A tiles are free again
-    {
-      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-      float acc[32];
-#pragma unroll
-      for (int half = 0; half < CTC_COLS / 32; ++half) {
-        tmem_ld32(tmem + lane_off + half * 32, acc);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[half * 32 + e] += acc[e];
-      }
-    }
-    tc_fence_before();
-    __syncthreads();                                   // every B read done before it is rewritten
-  }
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, CTC_COLS);
-  }
-}
-
 // Output correction of the corrected segmented schedule.  Segment p >= 1 of a
 // chain ran from a zero state in the state pass and wrote its zero-start
 // outputs o^0 into o; its transition slice wrote qhat_i = scale og_i
@@ -1986,14 +1754,17 @@ static gdn_status tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const 
   if (blocks <= 0) return GDN_OK;
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   LaunchCfg lc((unsigned)blocks, tc::THREADS, tc::SMEM_BYTES, stream, dependent);
-  const cudaError_t e = cudaLaunchKernelEx(&lc.cfg, tc::gdn_prefill_tc_kernel, mq, mk, mv, kp);
+  const bool epi = kp.gate != nullptr || kp.h_prev != nullptr;
+  const cudaError_t e = epi ? cudaLaunchKernelEx(&lc.cfg, tc::gdn_prefill_tc_kernel<true>, mq, mk, mv, kp)
+                            : cudaLaunchKernelEx(&lc.cfg, tc::gdn_prefill_tc_kernel<false>, mq, mk, mv, kp);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const SegPlan& plan, void* ws,
                              cudaStream_t stream) {
-  static std::atomic<bool> attr_set[kMaxDevices];
-  if (smem_attr_once(attr_set, tc::gdn_prefill_tc_kernel, tc::SMEM_BYTES) != cudaSuccess)
+  static std::atomic<bool> attr_set[kMaxDevices], attr_set_epi[kMaxDevices];
+  if (smem_attr_once(attr_set, tc::gdn_prefill_tc_kernel<false>, tc::SMEM_BYTES) != cudaSuccess ||
+      smem_attr_once(attr_set_epi, tc::gdn_prefill_tc_kernel<true>, tc::SMEM_BYTES) != cudaSuccess)
     return GDN_ERR_CUDA;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, p->q, p->dk, p->H, p->total_tokens) ||
@@ -2059,23 +1830,9 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
       tc_launch(mq, mk, mv, kp, chains * (kp.n_slices + (long long)n_part * (kp.n_slices + 1)), stream);
   if (st != GDN_OK) return st;
   // combine: start states S_2 .. S_{P-1} (and S_T in the corrected schedule,
-  // with every start state also in bf16 for the correction; there on the
-  // tensor cores)
+  // with every start state also in bf16 for the correction)
   const int n_steps = plan.corrected ? (p->S_T ? P - 1 : P - 2) : P - 2;
-  if (plan.corrected) {
-    CUtensorMap mm;
-    if (!make_map_2d(&mm, kp.Mws, tc::DK, (long long)p->n_seq * n_part * p->H * tc::DK, 32, 128, 4))
-      return GDN_ERR_CUDA;
-    const long long cblocks = chains * (p->dv / tc::CTC_COLS);
-    if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
-    static std::atomic<bool> ctc_attr_set[kMaxDevices];
-    if (smem_attr_once(ctc_attr_set, tc::gdn_segment_combine_tc_kernel, tc::CTC_SMEM) != cudaSuccess)
-      return GDN_ERR_CUDA;
-    LaunchCfg lc((unsigned)cblocks, tc::CTC_THREADS, tc::CTC_SMEM, stream, /*dependent=*/true);
-    if (cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_combine_tc_kernel, mm, (const float*)kp.Bws, kp.Sst, p->S_T,
-                           Sb, status, p->H, p->dv, P, n_part, n_steps) != cudaSuccess)
-      return GDN_ERR_CUDA;
-  } else if (n_steps > 0) {
+  if (n_steps > 0 || plan.corrected) {
     const long long cblocks = chains * (p->dv / tc::CMB_COLS);
     if (cblocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     static std::atomic<bool> cmb_attr_set[kMaxDevices];
@@ -2083,8 +1840,8 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
       return GDN_ERR_CUDA;
     LaunchCfg lc((unsigned)cblocks, 256, tc::CMB_SMEM, stream, /*dependent=*/true);
     if (cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_combine_kernel, (const float*)kp.Bws,
-                           (const float*)kp.Mws, kp.Sst, nullptr, nullptr, p->H, p->dv, P, n_part,
-                           n_steps) != cudaSuccess)
+                           (const float*)kp.Mws, kp.Sst, plan.corrected ? p->S_T : nullptr, Sb, p->H,
+                           p->dv, P, n_part, n_steps) != cudaSuccess)
       return GDN_ERR_CUDA;
   }
   if (!plan.corrected) {

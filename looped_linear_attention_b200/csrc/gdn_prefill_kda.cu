@@ -31,6 +31,25 @@ constexpr int DVS = 64;
 constexpr int THREADS = 256;
 constexpr int LDC = C + 1;
 
+// T = (I + A)^{-1} for the strictly lower C x C matrix A (row stride LDC in
+// shared memory), column `col` per thread: forward substitution with the
+// column held in registers, t_i = delta_{i,col} - sum_{m<i} A_im t_m, four
+// independent partial sums per row (the entries above the diagonal come out
+// zero by themselves: t_m = 0 for m < col).
+template <int C, int LDC>
+__device__ __forceinline__ void solve_column(const float* sA, float* sT, int col) {
+  float t[C];
+#pragma unroll
+  for (int i = 0; i < C; ++i) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < i; ++m) acc[m & 3] = fmaf(sA[i * LDC + m], t[m], acc[m & 3]);
+    t[i] = ((i == col) ? 1.f : 0.f) - ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+  }
+#pragma unroll
+  for (int i = 0; i < C; ++i) sT[i * LDC + col] = t[i];
+}
+
 template <int DK>
 struct Plan {
   static constexpr int LDK = DK + 1;
@@ -189,12 +208,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
     // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
     // operands: Q o e^G over Q, K o e^G over G, K o e^{G_C - G} over K
     if (tid < C) {
-      const int col = tid;
-      for (int i = 0; i < C; ++i) {
-        float acc = (i == col) ? 1.f : 0.f;
-        for (int m = col; m < i; ++m) acc = fmaf(-sA[i * LDC + m], sT[m * LDC + col], acc);
-        sT[i * LDC + col] = (i < col) ? 0.f : acc;
-      }
+      solve_column<C, LDC>(sA, sT, tid);
     } else {
       for (int e = tid - C; e < C * DK; e += THREADS - C) {
         const int i = e / DK, d = e % DK;

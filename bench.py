@@ -857,7 +857,16 @@ def run_profile_case(args):
     if args.n_seq:
         wl = dataclasses.replace(wl, n_seq=args.n_seq)
     dev = torch.device("cuda", 0)
-    if args.profile == "swa":
+    if args.profile == "kda":
+        # the per-channel gate prefill on the looped mixer shape
+        inp = W.prefill_inputs(dataclasses.replace(W.WORKLOADS["looped_prefill"], name="kda"), dev)
+        a, b = W.channel_gates(4096, 16, 128, dev, "bench", "kda")
+        o = torch.empty(4096, 16, 128, dtype=torch.bfloat16, device=dev)
+        fl = lla.GDN_QK_L2NORM | lla.GDN_CHANNEL_GATE
+        run = lambda: lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], a, b, None, flags=fl, o=o,
+                                        return_state=False)
+        wl = W.WORKLOADS["looped_prefill"]
+    elif args.profile == "swa":
         # sliding-window attention, w = 2048, on the looped workload's shape
         q, k, v = W.qkv(4096, 16, 128, 128, torch.bfloat16, False, dev, "bench", "swa")
         o = torch.empty_like(v)
@@ -904,7 +913,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile", choices=["tiny", "looped_prefill", "long_prefill", "varlen", "decode", "swa"],
+    ap.add_argument("--profile", choices=["tiny", "looped_prefill", "long_prefill", "varlen", "decode", "swa",
+                                          "kda"],
                     default=None,
                     help="run only this workload's kernel (for profiler captures)")
     ap.add_argument("--n-seq", type=int, default=0, help="sequences (or decode slots) for --profile")

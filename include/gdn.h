@@ -181,7 +181,8 @@ gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg
  *     start state's share of each output; a second kernel chains the start
  *     states (and S_T) in fp32 (skipped when there is nothing to chain); a
  *     third adds qhat_i^T S_p to the outputs (tensor cores) and applies the
- *     loop residual.
+ *     output gate and the loop residual, to every segment: there the output
+ *     is rounded to io_dtype before the gate factor multiplies it.
  *   output pass (when o is h_prev itself, which the first launch would
  *     overwrite): the first launch computes B and M of segments 1 .. P-2
  *     without outputs, the combine chains the start states, and a third

@@ -158,10 +158,11 @@ struct Params {
   //   mode 3: the state pass of the corrected schedule: as mode 1, but for
   //           segments 1 .. n_segs-1 (B_p, M_p in slot p-1), and with
   //           outputs: the slices write each segment's zero-start output o^0
-  //           into o (gated, no residual), the transition slice its outputs
-  //           qhat_i = scale og_i M_{p,i}^T q_i (the start state's share of
+  //           into o, the transition slice its outputs
+  //           qhat_i = scale qn_i M_{p,i}^T q_i (the start state's share of
   //           o_i is then qhat_i^T S_p, added by gdn_segment_correct_kernel)
-  //           into qhat [tokens][H][dk].
+  //           into qhat [tokens][H][dk].  It runs without the output gate and
+  //           the loop residual, which the correction applies.
   int mode, n_segs, seg_tok, seg0_tok;
   const int32_t* order;  // mode 0, varlen: sequences longest first (block order), or null
   float* Bws;          // [n_seq][n_part][H][dk][dv], n_part = n_segs-2 (mode 1) or n_segs-1 (mode 3)
@@ -1391,39 +1392,49 @@ __global__ void __launch_bounds__(256)
 }
 // Output correction of the corrected segmented schedule.  Segment p >= 1 of a
 // chain ran from a zero state in the state pass and wrote its zero-start
-// outputs o^0 into o; its transition slice wrote qhat_i = scale og_i
-// M_{p,i}^T q_i (og_i: the output gate and 1/|q_i|).  The state is affine in
-// the start state, so the outputs from the true start state S_p are
+// outputs o^0 into o; its transition slice wrote qhat_i = scale qn_i
+// M_{p,i}^T q_i (qn_i = 1/|q_i| with the in-kernel norm, else 1).  The state
+// is affine in the start state, so the outputs from the true start state S_p
+// are
 //     o_i = o^0_i + S_p^T qhat_i,
 // which this kernel adds for one (sequence, head, 128-wide dv slice) and a
-// tile of up to 128 tokens of one segment, then applies the loop residual.
+// tile of up to 128 tokens of one segment.  With the looped block's epilogue
+// (output gate, loop residual) the state pass runs without it and this kernel
+// applies it to every segment, segment 0 included (whose outputs, run from
+// S0, need no correction):
+//     o_i <- round(sigmoid(gate_i) round(o_i)) (+ rho (.) h_prev_i, rounded),
+// the order in which a gated call followed by loop_residual rounds.
 // qhat (K-major A), S_p rounded to bf16 by the combine (MN-major B: rows of
 // dk, 64 columns of dv per 128-byte row) and o^0 arrive by TMA in the 128-byte
 // swizzle; the product is one tcgen05 MMA chain (M = 128 tokens, N = 128
 // columns of dv, K = dk = 128) into tensor memory.  Thread r adds row r of
 // the product to o^0 and writes the sum, rounded to bf16, over the o^0 tile;
-// the tile then leaves as coalesced 16-byte rows, each with the loop residual
-// rho (.) h_prev added (h_prev read where it is stored, after an L2 prefetch
-// issued at entry; rho staged in shared memory).  96 KB of shared memory: two
-// CTAs per SM.  Launched as a programmatic dependent: inputs are touched
-// before griddepcontrol.wait, anything the state pass or the combine wrote
-// only after it.
+// the h_prev tile (TMA, into the qhat buffer once the MMA has read it) and the
+// gate factors (shared memory) then meet it in coalesced 16-byte rows.  96 KB
+// of shared memory: two CTAs per SM.  Launched as a programmatic dependent:
+// inputs (gate, rho, and h_prev where no MMA needs the buffer) are read before
+// griddepcontrol.wait, anything the state pass or the combine wrote only
+// after it.
 constexpr int COR_THREADS = 128;
 constexpr int COR_ROWS = 128;                      // tokens per tile
 constexpr uint32_t COR_TILE = 32768;               // 128 rows x 128 bf16 in two 64-column slabs
-constexpr uint32_t COR_OFF_A = 0;                  // qhat
+constexpr uint32_t COR_OFF_A = 0;                  // qhat, then h_prev
 constexpr uint32_t COR_OFF_B = COR_OFF_A + COR_TILE;   // S_p (bf16, MN-major)
 constexpr uint32_t COR_OFF_O = COR_OFF_B + COR_TILE;   // o^0, then o^0 + S_p^T qhat
 constexpr uint32_t COR_OFF_RHO = COR_OFF_O + COR_TILE; // rho of the slice (128 fp32)
-constexpr uint32_t COR_OFF_BAR = COR_OFF_RHO + 512;    // 3 mbarriers, tmem base, abort flag
+constexpr uint32_t COR_OFF_OG = COR_OFF_RHO + 512;     // gate factor of each row (128 fp32)
+constexpr uint32_t COR_OFF_BAR = COR_OFF_OG + 512;     // 4 mbarriers, tmem base, abort flag
 constexpr uint32_t COR_SMEM = COR_OFF_BAR + 64 + 1024;
 
 struct CorParams {
   __nv_bfloat16* o;
+  const float* gate;             // output-gate logits [tokens][H] (or null)
   const __nv_bfloat16* h_prev;   // loop residual input (or null) and its rho
   const float* rho;
   unsigned* status;
-  int H, dv, n_slices, seq_len, seg0_tok, seg_tok, n_segs, tiles_mid, tiles_per_seq;
+  int H, dv, n_slices, seq_len, seg0_tok, seg_tok, n_segs;
+  int tiles_first;               // tiles of segment 0 per (sequence, head, slice): 0 without epilogue
+  int tiles_mid, tiles_per_seq;
 };
 
 // One 128-token tile of a [tokens][H][width] map (two 64-column slabs, two
@@ -1446,7 +1457,8 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 
 __global__ void __launch_bounds__(COR_THREADS, 2)
     gdn_segment_correct_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_sb,
-                               const __grid_constant__ CUtensorMap tm_o, const CorParams p) {
+                               const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_h,
+                               const CorParams p) {
   extern __shared__ __align__(1024) uint8_t csm_raw[];
   uint8_t* sm = csm_raw;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1454,12 +1466,14 @@ __global__ void __launch_bounds__(COR_THREADS, 2)
     if (tid == 0) record_status(p.status, GDN_ERR_CUDA);
     return;
   }
-  // [0] qhat and S_p landed, [1] o^0 landed, [2] MMA done
+  // [0] qhat and S_p landed, [1] o^0 landed, [2] MMA done, [3] h_prev landed
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + COR_OFF_BAR);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + COR_OFF_BAR + 24);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + COR_OFF_BAR + 28);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + COR_OFF_BAR + 32);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + COR_OFF_BAR + 36);
   float* s_rho = reinterpret_cast<float*>(sm + COR_OFF_RHO);
-  // block -> (sequence, head, slice, tile); tiles enumerate segments 1 .. n_segs-1
+  float* s_og = reinterpret_cast<float*>(sm + COR_OFF_OG);
+  // block -> (sequence, head, slice, tile); tiles enumerate segment 0 (with the
+  // epilogue only), then segments 1 .. n_segs-1
   int bid = (int)blockIdx.x;
   const int tile = bid % p.tiles_per_seq;
   bid /= p.tiles_per_seq;
@@ -1469,24 +1483,29 @@ __global__ void __launch_bounds__(COR_THREADS, 2)
   const int seq = bid / p.H;
   const int tps = (p.seg_tok + COR_ROWS - 1) / COR_ROWS;
   int part, i0;
-  if (tile < p.tiles_mid) {
-    part = 1 + tile / tps;
-    i0 = (tile % tps) * COR_ROWS;
+  if (tile < p.tiles_first) {
+    part = 0;
+    i0 = tile * COR_ROWS;
+  } else if (tile - p.tiles_first < p.tiles_mid) {
+    part = 1 + (tile - p.tiles_first) / tps;
+    i0 = ((tile - p.tiles_first) % tps) * COR_ROWS;
   } else {
     part = p.n_segs - 1;
-    i0 = (tile - p.tiles_mid) * COR_ROWS;
+    i0 = (tile - p.tiles_first - p.tiles_mid) * COR_ROWS;
   }
-  const int seg_start = p.seg0_tok + (part - 1) * p.seg_tok;
-  const int seg_len = min(p.seg_tok, p.seq_len - seg_start);
+  const int seg_start = (part == 0) ? 0 : p.seg0_tok + (part - 1) * p.seg_tok;
+  const int seg_len = (part == 0) ? p.seg0_tok : min(p.seg_tok, p.seq_len - seg_start);
   const int rows = min(COR_ROWS, seg_len - i0);
   const int tok0 = seq * p.seq_len + seg_start + i0;
   const int col0 = slice * DVS;
+  const bool corr = part > 0;                      // start-state share S_p^T qhat
+  const bool resid = p.h_prev != nullptr;
   // row of S_p in the [n_seq * (n_segs-1) * H * dk][dv] view of the bf16 start states
   const int sb_row = ((seq * (p.n_segs - 1) + (part - 1)) * p.H + h) * DK;
   const size_t row_elems = (size_t)p.H * p.dv;
 
   if (tid == 0) {
-    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -1494,17 +1513,10 @@ __global__ void __launch_bounds__(COR_THREADS, 2)
     tmem_alloc(s_tmem, 128);
     tmem_relinquish();
   }
-  // inputs first: rho into shared memory, this tile's h_prev rows into L2
-  if (p.h_prev) {
-    s_rho[tid] = __ldg(p.rho + (size_t)h * p.dv + col0 + tid);
-    for (int u = tid; u < 2 * COR_ROWS; u += COR_THREADS) {
-      const int i = u >> 1;
-      if (i < rows) {
-        const __nv_bfloat16* line = p.h_prev + (size_t)(tok0 + i) * row_elems + (size_t)h * p.dv + col0 + (u & 1) * 64;
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(line));
-      }
-    }
-  }
+  // inputs first: rho and the gate factors into shared memory
+  s_rho[tid] = resid ? __ldg(p.rho + (size_t)h * p.dv + col0 + tid) : 0.f;
+  s_og[tid] = (p.gate && tid < rows) ? 1.f / (1.f + __expf(-__ldg(p.gate + (size_t)(tok0 + tid) * p.H + h)))
+                                     : 1.f;
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -1512,20 +1524,35 @@ __global__ void __launch_bounds__(COR_THREADS, 2)
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = smem_u32(sm);
   const bool have_rows = rows > 0;
+  bool h_issued = false;                           // thread 0: the h_prev copy is in flight
+  if (tid == 0 && have_rows) {
+    tma_prefetch_desc(&tm_o);
+    if (resid) {
+      tma_prefetch_desc(&tm_h);
+      if (!corr) {                                 // the qhat buffer is free: h_prev now
+        mbar_arrive_expect_tx(&bars[3], COR_TILE);
+        cor_load_rows(sm + COR_OFF_A, &tm_h, &bars[3], col0, h, tok0);
+        h_issued = true;
+      }
+    }
+    if (corr) {
+      tma_prefetch_desc(&tm_qh);
+      tma_prefetch_desc(&tm_sb);
+    }
+  }
   griddep_wait();                                  // qhat, o^0 and S_p are written
   if (tid == 0 && have_rows) {
-    tma_prefetch_desc(&tm_qh);
-    tma_prefetch_desc(&tm_sb);
-    tma_prefetch_desc(&tm_o);
-    mbar_arrive_expect_tx(&bars[0], 2 * COR_TILE);
-    cor_load_rows(sm + COR_OFF_A, &tm_qh, &bars[0], 0, h, tok0);
-    tma_load_2d(sm + COR_OFF_B, &tm_sb, &bars[0], col0, sb_row);
-    tma_load_2d(sm + COR_OFF_B + 16384, &tm_sb, &bars[0], col0 + 64, sb_row);
+    if (corr) {
+      mbar_arrive_expect_tx(&bars[0], 2 * COR_TILE);
+      cor_load_rows(sm + COR_OFF_A, &tm_qh, &bars[0], 0, h, tok0);
+      tma_load_2d(sm + COR_OFF_B, &tm_sb, &bars[0], col0, sb_row);
+      tma_load_2d(sm + COR_OFF_B + 16384, &tm_sb, &bars[0], col0 + 64, sb_row);
+    }
     mbar_arrive_expect_tx(&bars[1], COR_TILE);
     cor_load_rows(sm + COR_OFF_O, &tm_o, &bars[1], col0, h, tok0);
   }
   bool ok = have_rows;
-  if (ok && warp == 0) {
+  if (ok && corr && warp == 0) {
     const bool okw = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[0], 0, s_abort, p.status));
     tc_fence_after();
     if (okw && elect_one()) {
@@ -1538,9 +1565,16 @@ __global__ void __launch_bounds__(COR_THREADS, 2)
     __syncwarp();
   }
   if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[1], 0, s_abort, p.status) || *s_abort != 0);
-  if (ok) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[2], 0, s_abort, p.status));
+  if (ok && corr) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[2], 0, s_abort, p.status));
   tc_fence_after();
-  if (ok) {
+  if (ok && corr && resid && tid == 0) {
+    // the MMA has read qhat: h_prev into its buffer (only the async proxy has
+    // touched the buffer, so no proxy fence is needed)
+    mbar_arrive_expect_tx(&bars[3], COR_TILE);
+    cor_load_rows(sm + COR_OFF_A, &tm_h, &bars[3], col0, h, tok0);
+    h_issued = true;
+  }
+  if (ok && corr) {
     // thread: token row r of the tile; o^0 + S_p^T qhat, rounded to bf16 (the
     // output as it would be stored), replaces o^0 in shared memory
     const int r = warp * 32 + lane;
@@ -1563,24 +1597,35 @@ __global__ void __launch_bounds__(COR_THREADS, 2)
         *ov = v;
       }
     }
+  }
+  if (ok && resid) ok = !__syncthreads_or(!mbar_wait_bounded(&bars[3], 0, s_abort, p.status));
+  if (ok) {
     __syncthreads();
-    // coalesced 16-byte rows with the loop residual; a row past the segment
-    // belongs to another segment or sequence and is not touched
+    // coalesced 16-byte rows with the gate and the loop residual; a row past
+    // the segment belongs to another segment or sequence and is not touched
+    const bool gated = p.gate != nullptr;
 #pragma unroll 4
     for (int it = tid; it < COR_ROWS * 16; it += COR_THREADS) {
       const int i = it >> 4, chunk = it & 15;
       if (i < rows) {
-        uint4 v = *reinterpret_cast<const uint4*>(sm + COR_OFF_O + (chunk >> 3) * 16384 +
-                                                  sw128_offset(i, (chunk & 7) * 8));
-        const size_t off = (size_t)(tok0 + i) * row_elems + (size_t)h * p.dv + col0 + chunk * 8;
-        if (p.h_prev) {
-          const uint4 y = *reinterpret_cast<const uint4*>(p.h_prev + off);
+        const uint32_t soff = (chunk >> 3) * 16384 + sw128_offset(i, (chunk & 7) * 8);
+        uint4 v = *reinterpret_cast<const uint4*>(sm + COR_OFF_O + soff);
+        if (gated) {
+          const float g = s_og[i];
+          v.x = pack_bf16x2(g * bf16_lo(v.x), g * bf16_hi(v.x));
+          v.y = pack_bf16x2(g * bf16_lo(v.y), g * bf16_hi(v.y));
+          v.z = pack_bf16x2(g * bf16_lo(v.z), g * bf16_hi(v.z));
+          v.w = pack_bf16x2(g * bf16_lo(v.w), g * bf16_hi(v.w));
+        }
+        if (resid) {
+          const uint4 y = *reinterpret_cast<const uint4*>(sm + COR_OFF_A + soff);
           const float* rr = s_rho + chunk * 8;
           v.x = pack_bf16x2(fmaf(rr[0], bf16_lo(y.x), bf16_lo(v.x)), fmaf(rr[1], bf16_hi(y.x), bf16_hi(v.x)));
           v.y = pack_bf16x2(fmaf(rr[2], bf16_lo(y.y), bf16_lo(v.y)), fmaf(rr[3], bf16_hi(y.y), bf16_hi(v.y)));
           v.z = pack_bf16x2(fmaf(rr[4], bf16_lo(y.z), bf16_lo(v.z)), fmaf(rr[5], bf16_hi(y.z), bf16_hi(v.z)));
           v.w = pack_bf16x2(fmaf(rr[6], bf16_lo(y.w), bf16_lo(v.w)), fmaf(rr[7], bf16_hi(y.w), bf16_hi(v.w)));
         }
+        const size_t off = (size_t)(tok0 + i) * row_elems + (size_t)h * p.dv + col0 + chunk * 8;
         __stcs(reinterpret_cast<uint4*>(p.o + off), v);
       }
     }
@@ -1590,8 +1635,9 @@ __global__ void __launch_bounds__(COR_THREADS, 2)
   __syncthreads();
   if (tid == 0 && have_rows && !ok) {
     // never leave the block with a bulk copy still landing in its shared memory
-    mbar_wait_bounded(&bars[0], 0, nullptr, p.status);
+    if (corr) mbar_wait_bounded(&bars[0], 0, nullptr, p.status);
     mbar_wait_bounded(&bars[1], 0, nullptr, p.status);
+    if (h_issued) mbar_wait_bounded(&bars[3], 0, nullptr, p.status);
   }
   if (warp == 0) {
     tc_fence_after();
@@ -1826,6 +1872,14 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   kp.seg_tok = plan.seg_tok;
   kp.seg0_tok = plan.seg0_tok;
   kp.mode = plan.corrected ? 3 : 1;
+  // corrected schedule: the output gate and the loop residual are applied by
+  // the correction kernel (to every segment), not in the state pass's chunk loop
+  const bool epilogue = kp.gate != nullptr || kp.h_prev != nullptr;
+  if (plan.corrected) {
+    kp.gate = nullptr;
+    kp.h_prev = nullptr;
+    kp.rho = nullptr;
+  }
   gdn_status st =
       tc_launch(mq, mk, mv, kp, chains * (kp.n_slices + (long long)n_part * (kp.n_slices + 1)), stream);
   if (st != GDN_OK) return st;
@@ -1848,16 +1902,18 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
     kp.mode = 2;
     return tc_launch(mq, mk, mv, kp, chains * (P - 1) * kp.n_slices, stream, /*dependent=*/true);
   }
-  // correction of the outputs of segments 1 .. P-1
-  CUtensorMap mqh, msb, mo;
+  // correction of the outputs of segments 1 .. P-1, and the epilogue of all
+  CUtensorMap mqh, msb, mo, mh;
   if (!make_map(&mqh, kp.qhat, tc::DK, p->H, p->total_tokens) ||
       !make_map_2d(&msb, Sb, p->dv, (long long)p->n_seq * (P - 1) * p->H * tc::DK, 64, 128) ||
-      !make_map(&mo, p->o, p->dv, p->H, p->total_tokens))
+      !make_map(&mo, p->o, p->dv, p->H, p->total_tokens) ||
+      !make_map(&mh, p->h_prev ? p->h_prev : p->o, p->dv, p->H, p->total_tokens))
     return GDN_ERR_CUDA;
   tc::CorParams cp;
   cp.o = kp.o;
-  cp.h_prev = kp.h_prev;
-  cp.rho = kp.rho;
+  cp.gate = p->gate;
+  cp.h_prev = static_cast<const __nv_bfloat16*>(p->h_prev);
+  cp.rho = p->rho;
   cp.status = status;
   cp.H = p->H;
   cp.dv = p->dv;
@@ -1868,15 +1924,16 @@ gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const Se
   cp.n_segs = P;
   const int tps = (plan.seg_tok + tc::COR_ROWS - 1) / tc::COR_ROWS;
   const int last_len = p->seq_len - plan.seg0_tok - (P - 2) * plan.seg_tok;
+  cp.tiles_first = epilogue ? (plan.seg0_tok + tc::COR_ROWS - 1) / tc::COR_ROWS : 0;
   cp.tiles_mid = (P - 2) * tps;
-  cp.tiles_per_seq = cp.tiles_mid + (last_len + tc::COR_ROWS - 1) / tc::COR_ROWS;
+  cp.tiles_per_seq = cp.tiles_first + cp.tiles_mid + (last_len + tc::COR_ROWS - 1) / tc::COR_ROWS;
   const long long cor_blocks = chains * kp.n_slices * cp.tiles_per_seq;
   if (cor_blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   static std::atomic<bool> cor_attr_set[kMaxDevices];
   if (smem_attr_once(cor_attr_set, tc::gdn_segment_correct_kernel, tc::COR_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
   LaunchCfg lc((unsigned)cor_blocks, tc::COR_THREADS, tc::COR_SMEM, stream, /*dependent=*/true);
-  return cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_correct_kernel, mqh, msb, mo, cp) == cudaSuccess
+  return cudaLaunchKernelEx(&lc.cfg, tc::gdn_segment_correct_kernel, mqh, msb, mo, mh, cp) == cudaSuccess
              ? GDN_OK
              : GDN_ERR_CUDA;
 }

@@ -617,9 +617,9 @@ def bench_backward(dev, args, peaks, world):
     gST = torch.randn(wl.n_seq, wl.H, wl.dk, wl.dv, generator=g, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
+    def step(flags=0):
         return lla.gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], go, inp["S0"], gST,
-                                 n_seq=wl.n_seq)
+                                 n_seq=wl.n_seq, flags=flags)
 
     for _ in range(max(1, min(args.warmup, 2))):
         step()
@@ -635,13 +635,23 @@ def bench_backward(dev, args, peaks, world):
         e1.record(stream)
         torch.cuda.synchronize()
     t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n
+    # the token-by-token path (GDN_PRECISE), one call, for comparison
+    step(lla.GDN_PRECISE)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    step(lla.GDN_PRECISE)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_tok = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
     tokens = wl.n_seq * wl.seq_len
     nbytes = tokens * wl.H * (8 * wl.dk + 12 * wl.dk + 8 + 8) + 3 * wl.n_seq * wl.H * wl.dk * wl.dv * 4
     gbs = nbytes / t / 1e9
     return {"tokens_per_s": world * tokens / t, "ms_per_call": t * 1e3, "achieved_gbs": gbs,
             "frac_of_hbm": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
             "tokens": tokens, "heads": wl.H, "dk": wl.dk, "dv": wl.dv, "clocks": clocks.summary(),
-            "kernel": "gdn_bwd_kernel (first path: fp32 CUDA cores, one CTA per chain)"}
+            "kernel": "chunkwise: gdn_bwd_prep_kernel, gdn_bwd_states_kernel, gdn_bwd_dstates_kernel, "
+                      "gdn_bwd_grads_kernel (fp32 CUDA cores)",
+            "token_path_ms_per_call": t_tok * 1e3}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -866,6 +876,16 @@ def run_profile_case(args):
         run = lambda: lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], a, b, None, flags=fl, o=o,
                                         return_state=False)
         wl = W.WORKLOADS["looped_prefill"]
+    elif args.profile == "backward":
+        # the chunkwise reverse mode on the timed backward workload (8 x 1024 tokens)
+        wl = dataclasses.replace(W.WORKLOADS["long_prefill"], name="backward", n_seq=args.n_seq or 8,
+                                 seq_len=1024, random_s0=True)
+        inp = W.prefill_inputs(wl, dev)
+        g = torch.Generator(device=dev).manual_seed(W.seed_for("bench", "backward"))
+        go = torch.randn(inp["v"].shape, generator=g, device=dev).to(wl.dtype)
+        gST = torch.randn(wl.n_seq, wl.H, wl.dk, wl.dv, generator=g, device=dev)
+        run = lambda: lla.gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], go, inp["S0"],
+                                        gST, n_seq=wl.n_seq)
     elif args.profile == "swa":
         # sliding-window attention, w = 2048, on the looped workload's shape
         q, k, v = W.qkv(4096, 16, 128, 128, torch.bfloat16, False, dev, "bench", "swa")
@@ -914,7 +934,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", choices=["tiny", "looped_prefill", "long_prefill", "varlen", "decode", "swa",
-                                          "kda"],
+                                          "kda", "backward"],
                     default=None,
                     help="run only this workload's kernel (for profiler captures)")
     ap.add_argument("--n-seq", type=int, default=0, help="sequences (or decode slots) for --profile")

@@ -250,13 +250,24 @@ gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_params *p, cudaStream_t stream);
  * Outputs, fp32, overwritten, none overlapping an input:
  *   grad_q, grad_k [total_tokens][H][dk]; grad_v [total_tokens][H][dv];
  *   grad_a, grad_b [total_tokens][H];     grad_S0 [n_seq][H][dk][dv] or NULL.
- * Supported: dk in {64, 128}; dv a multiple of 32, at most 256; flags 0 (the
- * in-kernel q/k norm has no reverse mode here: differentiate it outside).
- * This first implementation runs on the CUDA cores in fp32: one CTA per
- * (sequence, head) chain, which recomputes the forward states from checkpoints
- * it takes every 64 tokens and walks each chunk backwards.
+ * Supported: dk in {64, 128}; dv a multiple of 32, at most 256; flags 0 or
+ * GDN_PRECISE (the in-kernel q/k norm has no reverse mode here: differentiate
+ * it outside).  fp32 arithmetic on the CUDA cores throughout.
+ * flags 0, the chunkwise path: the same relations in the chunked (WY/UT) form
+ * of gdn_chunk_fwd, chunks of 64 tokens, in four launches: per chunk the
+ * solve T = (I + A)^-1 and the chunk's transition factors; the chunk start
+ * states forward and the state gradients backward (one CTA per sequence,
+ * head and 32 columns of dv); then every token gradient, one CTA per chunk.
+ * It takes log a_t with a_t clamped to 1e-30 and returns grad_a_t =
+ * (dloss/dlog a_t) / a_t, so a gate of exactly 0 gets no meaningful grad_a_t
+ * (use GDN_PRECISE there).
+ * GDN_PRECISE, token by token: one CTA per (sequence, head) chain recomputes
+ * the forward states from checkpoints taken every 64 tokens and walks each
+ * chunk backwards with the per-token relations above.
  * ws/ws_bytes: device workspace of at least gdn_chunk_bwd_workspace(p) bytes,
- * 256-byte aligned (the checkpoints, one chunk of states and the running G of
+ * 256-byte aligned (chunkwise: per chunk and head the factors W, Qh [64][dk]
+ * and U~ [64][dv], the decays, the start state and the end-state gradient;
+ * token by token: the checkpoints, one chunk of states and the running G of
  * every chain); a missing or short workspace returns GDN_ERR_WORKSPACE.
  */
 typedef struct {

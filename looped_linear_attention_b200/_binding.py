@@ -226,12 +226,13 @@ def gdn_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
                   b: torch.Tensor, grad_o: torch.Tensor, S0: Optional[torch.Tensor] = None,
                   grad_S_T: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
                   *, n_seq: Optional[int] = None, scale: float = 1.0, want_grad_S0: bool = True,
-                  stream: Optional[torch.cuda.Stream] = None) -> dict:
+                  flags: int = 0, stream: Optional[torch.cuda.Stream] = None) -> dict:
     """Reverse mode of gdn_chunk_fwd (see gdn_chunk_bwd in include/gdn.h).
 
     Inputs as gdn_chunk_fwd plus grad_o [T, H, dv] (io dtype) and grad_S_T
     [n_seq, H, dk, dv] fp32 (or None).  Returns fp32 gradients
-    {"q", "k", "v", "a", "b", "S0"} ("S0" None unless want_grad_S0)."""
+    {"q", "k", "v", "a", "b", "S0"} ("S0" None unless want_grad_S0).
+    flags: 0 (the chunkwise path) or GDN_PRECISE (token by token)."""
     if q.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {q.dtype}")
     T, H, dk = q.shape
@@ -261,7 +262,7 @@ def gdn_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     p = gdn_bwd_params(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(S0), _ptr(grad_o),
                        _ptr(grad_S_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["a"]),
                        _ptr(g["b"]), _ptr(g["S0"]), _ptr(cu_seqlens), ns, seq_len, T, H, dk, dv,
-                       _DTYPES[q.dtype], float(scale), 0)
+                       _DTYPES[q.dtype], float(scale), int(flags))
     lib = library()
     ws = lib.gdn_chunk_bwd_workspace(ctypes.byref(p))
     if ws == ctypes.c_size_t(-1).value:

@@ -23,6 +23,8 @@ cudaError_t launch_loop_residual(const void* h_tilde, const void* h_prev, const 
 gdn_status launch_swa(const swa_params* p, unsigned* status, cudaStream_t stream);
 size_t bwd_workspace(const gdn_bwd_params* p);
 gdn_status launch_bwd(const gdn_bwd_params* p, unsigned* status, void* ws, cudaStream_t stream);
+size_t bwd_chunk_workspace(const gdn_bwd_params* p);
+gdn_status launch_bwd_chunk(const gdn_bwd_params* p, unsigned* status, void* ws, cudaStream_t stream);
 }  // namespace gdn
 
 // Device status word: kernels record the first error they hit (atomicCAS from 0).
@@ -134,7 +136,7 @@ gdn_status validate_bwd(const gdn_bwd_params* p) {
   if (!p) return GDN_ERR_INVALID;
   if (!dtype_ok(p->io_dtype)) return GDN_ERR_INVALID;
   if (p->n_seq < 0 || p->H <= 0 || p->total_tokens < 0 || p->dk <= 0 || p->dv <= 0) return GDN_ERR_INVALID;
-  if (p->flags != 0) return GDN_ERR_UNSUPPORTED;
+  if ((p->flags & ~GDN_PRECISE) != 0) return GDN_ERR_UNSUPPORTED;
   if (p->dk != 64 && p->dk != 128) return GDN_ERR_UNSUPPORTED;
   if (p->dv % 32 != 0 || p->dv > 256) return GDN_ERR_UNSUPPORTED;
   if (!p->cu_seqlens) {
@@ -160,7 +162,7 @@ extern "C" {
 size_t gdn_chunk_bwd_workspace(const gdn_bwd_params* p) {
   if (validate_bwd(p) != GDN_OK) return (size_t)-1;
   if (p->n_seq == 0) return 0;
-  return gdn::bwd_workspace(p);
+  return (p->flags & GDN_PRECISE) ? gdn::bwd_workspace(p) : gdn::bwd_chunk_workspace(p);
 }
 
 gdn_status gdn_chunk_bwd(const gdn_bwd_params* p, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -168,11 +170,12 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_params* p, void* ws, size_t ws_bytes, cud
   if (v != GDN_OK) return v;
   if (p->n_seq == 0) return GDN_OK;
   if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)) return GDN_ERR_INVALID;
-  const size_t need = gdn::bwd_workspace(p);
+  const bool token = (p->flags & GDN_PRECISE) != 0;
+  const size_t need = token ? gdn::bwd_workspace(p) : gdn::bwd_chunk_workspace(p);
   if (!ws || ws_bytes < need) return GDN_ERR_WORKSPACE;
   unsigned* st = status_ptr();
   if (!st) return GDN_ERR_CUDA;
-  return gdn::launch_bwd(p, st, ws, stream);
+  return token ? gdn::launch_bwd(p, st, ws, stream) : gdn::launch_bwd_chunk(p, st, ws, stream);
 }
 
 int gdn_version(void) { return 100; }

@@ -349,11 +349,16 @@ def _bwd_case(wl, lengths=None, n_seq=None, seq_len=None, grad_ST=True):
     return inp, go, gST
 
 
-def _bwd_check(inp, go, gST, scale):
+BWD_PATHS = {"chunkwise": 0, "token": lla.GDN_PRECISE}
+
+
+def _bwd_check(inp, go, gST, scale, flags=0):
+    """Every gradient against the oracle's reverse mode: relative L2 below 1e-4
+    over the whole tensor and, for the per-token gradients, per sequence."""
     dev = lambda t: None if t is None else t.cuda()
     cu = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).cuda()
     grads = lla.gdn_chunk_bwd(*(inp[n].cuda() for n in ("q", "k", "v", "a", "b")), go.cuda(),
-                              dev(inp["S0"]), dev(gST), cu, n_seq=inp["n_seq"], scale=scale)
+                              dev(inp["S0"]), dev(gST), cu, n_seq=inp["n_seq"], scale=scale, flags=flags)
     torch.cuda.synchronize()
     _status_ok()
     cu_h = inp["cu_seqlens"]
@@ -361,31 +366,70 @@ def _bwd_check(inp, go, gST, scale):
         cu_h = np.arange(inp["n_seq"] + 1, dtype=np.int32) * inp["seq_len"]
     ref = oracle.gdn_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], go, inp["S0"], gST, cu_h, scale)
     for name, rname in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("a", "da"), ("b", "db"), ("S0", "dS0")):
-        err = rel_l2(host(grads[name]), ref[rname])
+        got = host(grads[name])
+        err = rel_l2(got, ref[rname])
         assert err < TOL_F32, (name, err)
+        if name != "S0":
+            for s in range(len(cu_h) - 1):
+                t0, t1 = int(cu_h[s]), int(cu_h[s + 1])
+                if t1 > t0 and np.linalg.norm(ref[rname][t0:t1]) > 0:
+                    e = rel_l2(got[t0:t1], ref[rname][t0:t1])
+                    assert e < TOL_F32, (name, s, e)
+    return grads
 
 
-def test_backward_fp32_fixed_length_matches_oracle():
-    """Reverse mode on the GPU (checkpoints every 64 tokens, ragged last chunk)
-    against the oracle's: two sequences of 150 tokens, random S0 and final-state
+@pytest.mark.parametrize("path", list(BWD_PATHS))
+def test_backward_fp32_fixed_length_matches_oracle(path):
+    """Reverse mode on the GPU (chunks of 64 tokens, ragged last chunk) against
+    the oracle's: two sequences of 150 tokens, random S0 and final-state
     gradient, scale 0.5, fp32 inputs; relative L2 per gradient below 1e-4."""
     wl = _wl("tiny", H=2, dk=64, dv=64, random_s0=True, normalize_qk=True)
     inp, go, gST = _bwd_case(wl, n_seq=2, seq_len=150)
-    _bwd_check(inp, go, gST, 0.5)
+    _bwd_check(inp, go, gST, 0.5, BWD_PATHS[path])
 
 
-def test_backward_bf16_varlen_matches_oracle():
+@pytest.mark.parametrize("path", list(BWD_PATHS))
+def test_backward_bf16_varlen_matches_oracle(path):
     """bf16 inputs (compared on their exact values), varlen lengths 0, 1, 64,
     65, 200, dk = dv = 128."""
     wl = _wl("varlen", H=2, dv=128, random_s0=True)
     inp, go, gST = _bwd_case(wl, lengths=[0, 1, 64, 65, 200])
-    _bwd_check(inp, go, gST, 1.0)
+    _bwd_check(inp, go, gST, 1.0, BWD_PATHS[path])
 
 
-def test_backward_dv256_without_start_state_or_state_gradient():
+@pytest.mark.parametrize("path", list(BWD_PATHS))
+def test_backward_dv256_without_start_state_or_state_gradient(path):
     wl = _wl("long_prefill", n_seq=1, H=1, dv=256, random_s0=False)
     inp, go, gST = _bwd_case(wl, n_seq=1, seq_len=100, grad_ST=False)
+    _bwd_check(inp, go, gST, 1.0, BWD_PATHS[path])
+
+
+def test_backward_chunkwise_long_chain_matches_oracle():
+    """One 1024-token chain of the timed backward workload's shape (16 chunks,
+    so the chunk start states and end-state gradients are chained 15 times),
+    2 heads, bf16, random S0 and final-state gradient."""
+    wl = _wl("long_prefill", n_seq=1, H=2, random_s0=True)
+    inp, go, gST = _bwd_case(wl, n_seq=1, seq_len=1024)
     _bwd_check(inp, go, gST, 1.0)
+
+
+def test_backward_chunkwise_equals_token_path_at_full_size():
+    """At the timed backward workload's full size (8 x 1024 tokens, 16 heads,
+    dk = dv = 128, bf16) the chunkwise path and the token-by-token path (two
+    independent kernels) agree within 1e-4 on every gradient."""
+    wl = _wl("long_prefill", n_seq=8, random_s0=True)
+    inp = W.prefill_inputs(wl, "cuda", n_seq=8, seq_len=1024)
+    g = torch.Generator(device="cuda").manual_seed(W.seed_for("test", "bwd-full"))
+    go = torch.randn(inp["v"].shape, generator=g, device="cuda").to(wl.dtype)
+    gST = torch.randn(8, wl.H, wl.dk, wl.dv, generator=g, device="cuda")
+    args = ([inp[n] for n in ("q", "k", "v", "a", "b")] + [go, inp["S0"], gST])
+    ch = lla.gdn_chunk_bwd(*args, n_seq=8)
+    tk = lla.gdn_chunk_bwd(*args, n_seq=8, flags=lla.GDN_PRECISE)
+    torch.cuda.synchronize()
+    _status_ok()
+    for name in ("q", "k", "v", "a", "b", "S0"):
+        err = float(torch.linalg.vector_norm(ch[name] - tk[name]) / torch.linalg.vector_norm(tk[name]))
+        assert err < TOL_F32, (name, err)
 
 
 def test_prefill_tc_in_place_state():

@@ -52,11 +52,12 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the prefill kernel sources: ncu traffic figures are reported only
-    while they were taken on the kernel as it stands."""
+    """Hash of the prefill kernel sources (the kernels, their shared device code
+    and their tensor-map setup): ncu traffic figures are reported only while
+    they were taken on the kernel as it stands."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "looped_linear_attention_b200", "csrc")
-    for name in ("common.cuh", "gdn_prefill_tc.cu"):
+    for name in ("common.cuh", "tma_host.h", "gdn_prefill_tc.cu"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

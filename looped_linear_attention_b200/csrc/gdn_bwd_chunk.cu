@@ -48,7 +48,8 @@ constexpr int C = 64;
 constexpr int THREADS = 256;
 constexpr int NS = 32;            // dv columns per tile (grads) and per state-pass CTA
 constexpr int LDT = NS + 1;       // row stride of [rows][NS] tiles
-constexpr int LDC = C + 1;        // row stride of C x C tiles
+constexpr int LDC = C + 4;        // row stride of C x C tiles (a multiple of 4, = 4 mod 32)
+constexpr int LDN = NS + 4;       // row stride of [C][NS] tiles (the same two properties)
 constexpr float kMinGate = 1e-30f;   // a is clamped to this before its logarithm
 
 struct KParams {
@@ -199,41 +200,70 @@ __device__ __forceinline__ void solve_column(const float* sKK, const float* sb, 
   for (int i = 0; i < C; ++i) sT[i * LDC + col] = t[i];
 }
 
-// Shared setup of the prep and grads kernels: K and Q rows, gate vectors,
-// KK = D o K K^T (strictly lower), P = scale D o Q K^T (lower, diagonal
-// included) and T.
+// Rows [0, n) of a [tokens][H][width] input into shared memory ([C][ld]
+// fp32, columns [0, cols)), zeros below: 4 elements per load and per float4
+// store (ld, width and cols multiples of 4).
+__device__ __forceinline__ float4 ld4(const float* p, size_t i) {
+  return __ldg(reinterpret_cast<const float4*>(p + i));
+}
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16* p, size_t i) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p + i);
+  return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+}
+template <typename T>
+__device__ __forceinline__ void load_rows4(float* dst, int ld, const T* src, int t0, int n, int h, int H,
+                                           int width, int cols, int tid) {
+  const int q = cols / 4;
+  for (int e = tid; e < C * q; e += THREADS) {
+    const int i = e / q, c = (e % q) * 4;
+    *reinterpret_cast<float4*>(dst + i * ld + c) =
+        (i < n) ? ld4(src, ((size_t)(t0 + i) * H + h) * width + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+}
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float f4(const float4& v, int e) {
+  return e == 0 ? v.x : (e == 1 ? v.y : (e == 2 ? v.z : v.w));
+}
+
+// Shared setup of the prep and grads kernels: K and Q rows (stride DK + 4),
+// gate vectors, KK = D o K K^T (strictly lower), P = scale D o Q K^T (lower,
+// diagonal included) and T.
 template <int DK, typename T>
 __device__ __forceinline__ void chunk_setup(const KParams& p, int t0, int n, int h, float* sK, float* sQ,
                                             float* sKK, float* sP, float* sT, Vec V, float* s_carry,
                                             int tid) {
-  constexpr int LDK = DK + 1;
-  load_rows(sK, LDK, static_cast<const T*>(p.k), t0, n, h, p.H, DK, 0, DK, tid);
-  load_rows(sQ, LDK, static_cast<const T*>(p.q), t0, n, h, p.H, DK, 0, DK, tid);
+  constexpr int LDK = DK + 4;
+  load_rows4(sK, LDK, static_cast<const T*>(p.k), t0, n, h, p.H, DK, DK, tid);
+  load_rows4(sQ, LDK, static_cast<const T*>(p.q), t0, n, h, p.H, DK, DK, tid);
   chunk_gates(p, t0, n, h, V, s_carry, tid);
   __syncthreads();
   {
-    // thread: rows r0 .. r0+3, columns cg + 16 j (interleaved: no bank conflicts)
+    // thread: rows r0 .. r0+3, columns cg + 16 j; both products read K and Q
+    // along k four at a time (the row stride DK + 4 keeps the eight rows of a
+    // quarter-warp's column reads in distinct banks)
     const int r0 = (tid >> 4) * 4, cg = tid & 15;
     float kk[4][4], qk[4][4];
     zero(kk);
     zero(qk);
-    // both products share the B operand K^T (B(k, j) = K[cg + 16 j][k])
 #pragma unroll 2
-    for (int k = 0; k < DK; ++k) {
-      float ak[4], aq[4], bv[4];
+    for (int k = 0; k < DK; k += 4) {
+      float4 ak[4], aq[4], bk[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        ak[i] = sK[(r0 + i) * LDK + k];
-        aq[i] = sQ[(r0 + i) * LDK + k];
+        ak[i] = *reinterpret_cast<const float4*>(sK + (r0 + i) * LDK + k);
+        aq[i] = *reinterpret_cast<const float4*>(sQ + (r0 + i) * LDK + k);
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) bv[j] = sK[(cg + 16 * j) * LDK + k];
+      for (int j = 0; j < 4; ++j) bk[j] = *reinterpret_cast<const float4*>(sK + (cg + 16 * j) * LDK + k);
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          kk[i][j] = fmaf(ak[i], bv[j], kk[i][j]);
-          qk[i][j] = fmaf(aq[i], bv[j], qk[i][j]);
+          kk[i][j] = dot4(ak[i], bk[j], kk[i][j]);
+          qk[i][j] = dot4(aq[i], bk[j], qk[i][j]);
         }
     }
 #pragma unroll
@@ -253,103 +283,194 @@ __device__ __forceinline__ void chunk_setup(const KParams& p, int t0, int n, int
 
 template <int DK>
 struct PrepPlan {
-  static constexpr int LDK = DK + 1;
-  static constexpr int K = 0;
-  static constexpr int Q = K + C * LDK;
-  static constexpr int W = Q + C * LDK;
-  static constexpr int KK = W + C * LDK;
-  static constexpr int P = KK + C * LDC;
-  static constexpr int T = P + C * LDC;
-  static constexpr int V = T + C * LDC;       // [C][LDT]
-  static constexpr int VEC = V + C * LDT;     // 5 x C + carry
+  static constexpr int LDK = DK + 4;
+  static constexpr int K = 0;                 // [C][LDK]
+  static constexpr int Q = K + C * LDK;       // [C][LDK]
+  static constexpr int W = Q + C * LDK;       // [C][LDK]
+  static constexpr int KK = W + C * LDK;      // [C][LDC], then T^T
+  static constexpr int P = KK + C * LDC;      // [C][LDC]
+  static constexpr int T = P + C * LDC;       // [C][LDC]
+  static constexpr int PT = T + C * LDC;      // [C][LDC] P^T
+  static constexpr int V = PT + C * LDC;      // [C][LDN]
+  static constexpr int VEC = V + C * LDN;     // 5 x C + carry
   static constexpr int FLOATS = VEC + 5 * C + 4;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
+  static_assert(BYTES <= 232448, "shared memory of one CTA");
 };
 
 // 1. Per (chunk, head): W = T diag(b gamma) K, U~ = T diag(b) V, Qh = scale
-// diag(gamma) Q - P W and g, into the workspace.
+// diag(gamma) Q - P W and g, into the workspace.  The products read k-major
+// float4 operands: T^T (over KK, free after the solve) and P^T are transposed
+// copies.  Thread map as in the gradient kernel (rows 4 rg .. 4 rg + 3;
+// C x DK columns 4 cg .. 4 cg + 3 and 64 + 4 cg ..; tile columns cg, cg + 16).
 template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_prep_kernel(const KParams p) {
-  extern __shared__ float smf[];
+  extern __shared__ __align__(16) float smf[];
   using PL = PrepPlan<DK>;
   constexpr int LDK = PL::LDK;
-  constexpr int TN = DK / 16;
+  constexpr int NV = DK / 64;
   const int tid = threadIdx.x;
   const long long slot = blockIdx.x / p.H;
   const int h = blockIdx.x % p.H;
   int s, c, t0, n;
   if (!slot_chunk(p, slot, s, c, t0, n)) return;
   float *sK = smf + PL::K, *sQ = smf + PL::Q, *sW = smf + PL::W, *sKK = smf + PL::KK, *sP = smf + PL::P,
-        *sT = smf + PL::T, *sV = smf + PL::V;
+        *sT = smf + PL::T, *sPt = smf + PL::PT, *sV = smf + PL::V;
+  float* sTt = sKK;
   Vec V{smf + PL::VEC, smf + PL::VEC + C, smf + PL::VEC + 2 * C, smf + PL::VEC + 3 * C,
         smf + PL::VEC + 4 * C};
   chunk_setup<DK, T>(p, t0, n, h, sK, sQ, sKK, sP, sT, V, smf + PL::VEC + 5 * C, tid);
+  for (int e = tid; e < C * C; e += THREADS) {
+    const int i = e / C, j = e % C;
+    sTt[j * LDC + i] = sT[i * LDC + j];
+    sPt[j * LDC + i] = sP[i * LDC + j];
+  }
   const size_t wsi = (size_t)slot * p.H + h;
-  const int r0 = (tid >> 4) * 4;
+  const int rg = tid >> 4, cg = tid & 15;
+  const int r0 = rg * 4;
+  if (tid < C) p.G[wsi * C + tid] = V.g[tid];
+  __syncthreads();
   {
-    // W [C][DK] (thread columns cg + 16 j)
-    const int cg = tid & 15;
-    float acc[4][TN];
+    // W = T diag(b gamma) K  [C][DK]
+    float acc[4][4 * NV];
     zero(acc);
-    gemm<4, TN, C>(acc, [&](int i, int k) { return sT[(r0 + i) * LDC + k]; },
-                   [&](int k, int j) { return V.b[k] * V.gam[k] * sK[k * LDK + cg + 16 * j]; });
+#pragma unroll 2
+    for (int k = 0; k < C; ++k) {
+      const float4 a4 = lds4(sTt + k * LDC + r0);
+      const float bgk = V.b[k] * V.gam[k];
+#pragma unroll
+      for (int w = 0; w < NV; ++w) {
+        const float4 b4 = lds4(sK + k * LDK + 64 * w + 4 * cg);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[i][4 * w + e] = fmaf(f4(a4, i) * bgk, f4(b4, e), acc[i][4 * w + e]);
+      }
+    }
     float* gW = p.W + wsi * C * DK;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < TN; ++j) {
-        sW[(r0 + i) * LDK + cg + 16 * j] = acc[i][j];
-        gW[(size_t)(r0 + i) * DK + cg + 16 * j] = acc[i][j];
+      for (int w = 0; w < NV; ++w) {
+        const float4 o = make_float4(acc[i][4 * w], acc[i][4 * w + 1], acc[i][4 * w + 2], acc[i][4 * w + 3]);
+        *reinterpret_cast<float4*>(sW + (r0 + i) * LDK + 64 * w + 4 * cg) = o;
+        *reinterpret_cast<float4*>(gW + (size_t)(r0 + i) * DK + 64 * w + 4 * cg) = o;
       }
   }
-  if (tid < C) p.G[wsi * C + tid] = V.g[tid];
   __syncthreads();
   {
-    // Qh [C][DK] = scale diag(gamma) Q - P W
-    const int cg = tid & 15;
-    float acc[4][TN];
+    // Qh = scale diag(gamma) Q - P W  [C][DK]
+    float acc[4][4 * NV];
     zero(acc);
-    gemm<4, TN, C>(acc, [&](int i, int k) { return sP[(r0 + i) * LDC + k]; },
-                   [&](int k, int j) { return sW[k * LDK + cg + 16 * j]; });
+#pragma unroll 2
+    for (int k = 0; k < C; ++k) {
+      const float4 a4 = lds4(sPt + k * LDC + r0);
+#pragma unroll
+      for (int w = 0; w < NV; ++w) {
+        const float4 b4 = lds4(sW + k * LDK + 64 * w + 4 * cg);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[i][4 * w + e] = fmaf(f4(a4, i), f4(b4, e), acc[i][4 * w + e]);
+      }
+    }
     float* gQ = p.Qh + wsi * C * DK;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
+      const float sg = p.scale * V.gam[r0 + i];
 #pragma unroll
-      for (int j = 0; j < TN; ++j)
-        gQ[(size_t)(r0 + i) * DK + cg + 16 * j] =
-            p.scale * V.gam[r0 + i] * sQ[(r0 + i) * LDK + cg + 16 * j] - acc[i][j];
+      for (int w = 0; w < NV; ++w) {
+        const float4 q4 = lds4(sQ + (r0 + i) * LDK + 64 * w + 4 * cg);
+        const float4 o = make_float4(sg * q4.x - acc[i][4 * w], sg * q4.y - acc[i][4 * w + 1],
+                                     sg * q4.z - acc[i][4 * w + 2], sg * q4.w - acc[i][4 * w + 3]);
+        *reinterpret_cast<float4*>(gQ + (size_t)(r0 + i) * DK + 64 * w + 4 * cg) = o;
+      }
+    }
   }
-  // U~ [C][dv], 32 columns at a time
+  // U~ = T diag(b) V  [C][dv], 32 columns at a time
   float* gU = p.Ut + wsi * C * p.dv;
   for (int col0 = 0; col0 < p.dv; col0 += NS) {
     __syncthreads();
-    load_rows(sV, LDT, static_cast<const T*>(p.v), t0, n, h, p.H, p.dv, col0, NS, tid);
+    for (int e = tid; e < C * NS; e += THREADS) {
+      const int i = e / NS, cc = e % NS;
+      sV[i * LDN + cc] = (i < n) ? V.b[i] * ldx(static_cast<const T*>(p.v), ((size_t)(t0 + i) * p.H + h) * p.dv + col0 + cc)
+                                 : 0.f;
+    }
     __syncthreads();
-    const int c0 = (tid & 15) * 2;
     float acc[4][2];
     zero(acc);
-    gemm<4, 2, C>(acc, [&](int i, int k) { return sT[(r0 + i) * LDC + k]; },
-                  [&](int k, int j) { return V.b[k] * sV[k * LDT + c0 + j]; });
+#pragma unroll 4
+    for (int k = 0; k < C; ++k) {
+      const float4 a4 = lds4(sTt + k * LDC + r0);
+      const float b0 = sV[k * LDN + cg], b1 = sV[k * LDN + cg + 16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[i][0] = fmaf(f4(a4, i), b0, acc[i][0]);
+        acc[i][1] = fmaf(f4(a4, i), b1, acc[i][1]);
+      }
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 2; ++j) gU[(size_t)(r0 + i) * p.dv + col0 + c0 + j] = acc[i][j];
+      for (int u = 0; u < 2; ++u) gU[(size_t)(r0 + i) * p.dv + col0 + cg + 16 * u] = acc[i][u];
   }
 }
 
+// Shared-memory plans of the state passes, 2 CTAs per SM.  Row strides are
+// multiples of 4 (tiles of NS columns: NS + 2, even) so that every operand
+// read of the products is one float4 (4 rows of a transposed operand) or one
+// float2 (2 columns of a tile).
+constexpr int LDX = NS + 2;        // [rows][NS] tiles
+constexpr int LDCT = C + 4;        // [DK][C] transposed operands
 template <int DK>
-struct StatePlan {
-  static constexpr int LDK = DK + 1;
-  static constexpr int S = 0;                  // [DK][LDT]
-  static constexpr int W = S + DK * LDT;       // [C][LDK]
-  static constexpr int KH = W + C * LDK;       // [C][LDK]  diag(r) K
-  static constexpr int QH = KH + C * LDK;      // [C][LDK]  (dstates only)
-  static constexpr int X = QH + C * LDK;       // [C][LDT]
-  static constexpr int DO = X + C * LDT;       // [C][LDT]  (dstates only)
-  static constexpr int VEC = DO + C * LDT;     // g, r
+struct StatesPlan {
+  static constexpr int LDK = DK + 4;
+  static constexpr int S = 0;                    // [DK][LDX]  state slice
+  static constexpr int WT = S + DK * LDX;        // [DK][LDCT] W^T
+  static constexpr int KH = WT + DK * LDCT;      // [C][LDK]   diag(r) K
+  static constexpr int X = KH + C * LDK;         // [C][LDX]
+  static constexpr int VEC = X + C * LDX;        // g, r
   static constexpr int FLOATS = VEC + 2 * C;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
+template <int DK>
+struct DStatesPlan {
+  static constexpr int LDK = DK + 4;
+  static constexpr int E = 0;                    // [DK][LDX]  gradient slice
+  static constexpr int KT = E + DK * LDX;        // [DK][LDCT] (diag(r) K)^T, then Qh [C][LDK]
+  static constexpr int KT_FLOATS = (DK * LDCT > C * LDK) ? DK * LDCT : C * LDK;
+  static constexpr int W = KT + KT_FLOATS;       // [C][LDK]
+  static constexpr int Y = W + C * LDK;          // [C][LDX]
+  static constexpr int DO = Y + C * LDX;         // [C][LDX]
+  static constexpr int VEC = DO + C * LDX;       // g, r
+  static constexpr int FLOATS = VEC + 2 * C;
+  static constexpr size_t BYTES = (size_t)FLOATS * 4;
+};
+
+// acc[i][j] += sum_k A[k * LDA + i] B[k * LDB + j] (A and B already offset to
+// the thread's rows and columns): TM / 4 float4 and one float2 read per k.
+template <int TM, int K, int LDA, int LDB>
+__device__ __forceinline__ void gemm_v(float (&acc)[TM][2], const float* A, const float* B) {
+  static_assert(TM % 4 == 0 && LDA % 4 == 0 && LDB % 2 == 0, "vector operand layout");
+#pragma unroll 4
+  for (int k = 0; k < K; ++k) {
+    float av[TM];
+#pragma unroll
+    for (int q = 0; q < TM / 4; ++q) {
+      const float4 a4 = *reinterpret_cast<const float4*>(A + k * LDA + 4 * q);
+      av[4 * q] = a4.x;
+      av[4 * q + 1] = a4.y;
+      av[4 * q + 2] = a4.z;
+      av[4 * q + 3] = a4.w;
+    }
+    const float2 b2 = *reinterpret_cast<const float2*>(B + k * LDB);
+#pragma unroll
+    for (int i = 0; i < TM; ++i) {
+      acc[i][0] = fmaf(av[i], b2.x, acc[i][0]);
+      acc[i][1] = fmaf(av[i], b2.y, acc[i][1]);
+    }
+  }
+}
 
 // Chain (sequence, head) and column slice of a state-pass block.
 __device__ __forceinline__ void state_block(const KParams& p, int& s, int& h, int& col0) {
@@ -360,46 +481,45 @@ __device__ __forceinline__ void state_block(const KParams& p, int& s, int& h, in
   h = chain % p.H;
 }
 
-// Loads of one chunk for the state passes: W (and Qh), diag(r) K, g and r.
-template <int DK, typename T>
-__device__ __forceinline__ void state_chunk_loads(const KParams& p, size_t wsi, int t0, int n, int h,
-                                                  float* sW, float* sQh, float* sKh, float* sg, float* sr,
-                                                  int tid) {
-  constexpr int LDK = DK + 1;
+// g and r = e^{g_C - g} of a chunk (two barriers inside; every thread calls it).
+__device__ __forceinline__ void state_gates(const KParams& p, size_t wsi, float* sg, float* sr, int tid) {
   if (tid < C) sg[tid] = p.G[wsi * C + tid];
-  const float4* gW = reinterpret_cast<const float4*>(p.W + wsi * C * DK);
-  const float4* gQ = reinterpret_cast<const float4*>(p.Qh + wsi * C * DK);
-  for (int e = tid; e < C * DK / 4; e += THREADS) {
-    const int i = (e * 4) / DK, d = (e * 4) % DK;
-    const float4 w = gW[e];
-    sW[i * LDK + d] = w.x;
-    sW[i * LDK + d + 1] = w.y;
-    sW[i * LDK + d + 2] = w.z;
-    sW[i * LDK + d + 3] = w.w;
-    if (sQh) {
-      const float4 x = gQ[e];
-      sQh[i * LDK + d] = x.x;
-      sQh[i * LDK + d + 1] = x.y;
-      sQh[i * LDK + d + 2] = x.z;
-      sQh[i * LDK + d + 3] = x.w;
-    }
-  }
   __syncthreads();
   if (tid < C) sr[tid] = expf(sg[C - 1] - sg[tid]);
   __syncthreads();
-  const T* k = static_cast<const T*>(p.k);
-  for (int e = tid; e < C * DK; e += THREADS) {
-    const int i = e / DK, d = e % DK;
-    sKh[i * LDK + d] = (i < n) ? sr[i] * ldx(k, ((size_t)(t0 + i) * p.H + h) * DK + d) : 0.f;
+}
+
+// dst[d * LDCT + i] = src(i, d) for a row-major [C][DK] source (rows >= n
+// zero): 4 rows per thread, read along d (coalesced), one float4 store.
+template <int DK, class F>
+__device__ __forceinline__ void store_transposed(float* dst, int n, F src, int tid) {
+  for (int e = tid; e < DK * (C / 4); e += THREADS) {
+    const int d = e % DK, i4 = (e / DK) * 4;
+    float4 x;
+    x.x = (i4 < n) ? src(i4, d) : 0.f;
+    x.y = (i4 + 1 < n) ? src(i4 + 1, d) : 0.f;
+    x.z = (i4 + 2 < n) ? src(i4 + 2, d) : 0.f;
+    x.w = (i4 + 3 < n) ? src(i4 + 3, d) : 0.f;
+    *reinterpret_cast<float4*>(dst + d * LDCT + i4) = x;
+  }
+}
+// A [C][DK] fp32 workspace array into shared memory rows of stride LDK (float4).
+template <int DK>
+__device__ __forceinline__ void load_ws_rows(float* dst, const float* src, int tid) {
+  constexpr int LDK = DK + 4;
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+  for (int e = tid; e < C * DK / 4; e += THREADS) {
+    const int i = (e * 4) / DK, d = (e * 4) % DK;
+    *reinterpret_cast<float4*>(dst + i * LDK + d) = __ldg(s4 + e);
   }
 }
 
 // 2. Chunk start states, forward: S_c[:, J] into the workspace, then
 // S <- gamma_C S + (diag(r) K)^T (U~[:, J] - W S).
 template <int DK, typename T>
-__global__ void __launch_bounds__(THREADS, 1) gdn_bwd_states_kernel(const KParams p) {
-  extern __shared__ float smf[];
-  using PL = StatePlan<DK>;
+__global__ void __launch_bounds__(THREADS, 2) gdn_bwd_states_kernel(const KParams p) {
+  extern __shared__ __align__(16) float smf[];
+  using PL = StatesPlan<DK>;
   constexpr int LDK = PL::LDK;
   constexpr int TM = DK / 16;
   const int tid = threadIdx.x;
@@ -407,16 +527,18 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_states_kernel(const KParam
   state_block(p, s, h, col0);
   int t0, t1;
   seq_range(p, s, t0, t1, tid == 0 && col0 == 0 && h == 0);
-  float *sS = smf + PL::S, *sW = smf + PL::W, *sKh = smf + PL::KH, *sX = smf + PL::X;
+  float *sS = smf + PL::S, *sWt = smf + PL::WT, *sKh = smf + PL::KH, *sX = smf + PL::X;
   float *sg = smf + PL::VEC, *sr = smf + PL::VEC + C;
   const size_t sd = (size_t)DK * p.dv;
   const size_t sb0 = ((size_t)s * p.H + h) * sd;
   for (int e = tid; e < DK * NS; e += THREADS) {
     const int d = e / NS, c = e % NS;
-    sS[d * LDT + c] = p.S0 ? p.S0[sb0 + (size_t)d * p.dv + col0 + c] : 0.f;
+    sS[d * LDX + c] = p.S0 ? p.S0[sb0 + (size_t)d * p.dv + col0 + c] : 0.f;
   }
   const int n_chunks = (t1 - t0 + C - 1) / C;
   const long long base = slot_base(s, t0);
+  const T* k = static_cast<const T*>(p.k);
+  const int rg = tid >> 4, c0 = (tid & 15) * 2;
   for (int ci = 0; ci < n_chunks; ++ci) {
     const int tc0 = t0 + ci * C, n = min(C, t1 - tc0);
     const size_t wsi = (size_t)(base + ci) * p.H + h;
@@ -424,52 +546,55 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_states_kernel(const KParam
     float* gS = p.Sst + wsi * sd;
     for (int e = tid; e < DK * NS; e += THREADS) {
       const int d = e / NS, c = e % NS;
-      gS[(size_t)d * p.dv + col0 + c] = sS[d * LDT + c];
+      gS[(size_t)d * p.dv + col0 + c] = sS[d * LDX + c];
     }
-    state_chunk_loads<DK, T>(p, wsi, tc0, n, h, sW, nullptr, sKh, sg, sr, tid);
-    const float* gU = p.Ut + wsi * C * p.dv;
-    for (int e = tid; e < C * NS; e += THREADS) {
-      const int i = e / NS, c = e % NS;
-      sX[i * LDT + c] = gU[(size_t)i * p.dv + col0 + c];
+    state_gates(p, wsi, sg, sr, tid);
+    const float* gW = p.W + wsi * C * DK;
+    store_transposed<DK>(sWt, C, [&](int i, int d) { return __ldg(gW + (size_t)i * DK + d); }, tid);
+    for (int e = tid; e < C * DK; e += THREADS) {
+      const int i = e / DK, d = e % DK;
+      sKh[i * LDK + d] = (i < n) ? sr[i] * ldx(k, ((size_t)(tc0 + i) * p.H + h) * DK + d) : 0.f;
+    }
+    const float* gU = p.Ut + wsi * C * p.dv + col0;
+    for (int e = tid; e < C * NS / 2; e += THREADS) {
+      const int i = (e * 2) / NS, c = (e * 2) % NS;
+      *reinterpret_cast<float2*>(sX + i * LDX + c) =
+          __ldg(reinterpret_cast<const float2*>(gU + (size_t)i * p.dv + c));
     }
     __syncthreads();
     {
-      // X = U~ - W S  [C][NS]
-      const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 2;
+      // X = U~ - W S  [C][NS]: rows 4 rg .. +3, columns c0, c0 + 1
       float acc[4][2];
       zero(acc);
-      gemm<4, 2, DK>(acc, [&](int i, int k) { return sW[(r0 + i) * LDK + k]; },
-                     [&](int k, int j) { return sS[k * LDT + c0 + j]; });
+      gemm_v<4, DK, LDCT, LDX>(acc, sWt + rg * 4, sS + c0);
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) sX[(r0 + i) * LDT + c0 + j] -= acc[i][j];
+        for (int j = 0; j < 2; ++j) sX[(rg * 4 + i) * LDX + c0 + j] -= acc[i][j];
     }
     __syncthreads();
     {
-      // S = gamma_C S + Kh^T X  [DK][NS]
-      const int r0 = (tid >> 4) * TM, c0 = (tid & 15) * 2;
+      // S = gamma_C S + Kh^T X  [DK][NS]: rows TM rg .. +TM-1
       float acc[TM][2];
       zero(acc);
-      gemm<TM, 2, C>(acc, [&](int i, int k) { return sKh[k * LDK + r0 + i]; },
-                     [&](int k, int j) { return sX[k * LDT + c0 + j]; });
+      gemm_v<TM, C, LDK, LDX>(acc, sKh + rg * TM, sX + c0);
       const float gC = expf(sg[C - 1]);
 #pragma unroll
       for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-          sS[(r0 + i) * LDT + c0 + j] = fmaf(gC, sS[(r0 + i) * LDT + c0 + j], acc[i][j]);
+          sS[(rg * TM + i) * LDX + c0 + j] = fmaf(gC, sS[(rg * TM + i) * LDX + c0 + j], acc[i][j]);
     }
   }
 }
 
 // 3. State gradients, backward: dE_c[:, J] (the gradient at the end of chunk
 // c) into the workspace, then dE <- gamma_C dE - W^T (Kh dE) + Qh^T dO[:, J];
-// what remains after chunk 0 is grad_S0.
+// what remains after chunk 0 is grad_S0.  Kh^T and then Qh share one buffer.
 template <int DK, typename T>
-__global__ void __launch_bounds__(THREADS, 1) gdn_bwd_dstates_kernel(const KParams p) {
-  extern __shared__ float smf[];
-  using PL = StatePlan<DK>;
+__global__ void __launch_bounds__(THREADS, 2) gdn_bwd_dstates_kernel(const KParams p) {
+  extern __shared__ __align__(16) float smf[];
+  using PL = DStatesPlan<DK>;
   constexpr int LDK = PL::LDK;
   constexpr int TM = DK / 16;
   const int tid = threadIdx.x;
@@ -477,17 +602,20 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_dstates_kernel(const KPara
   state_block(p, s, h, col0);
   int t0, t1;
   seq_range(p, s, t0, t1, false);
-  float *sE = smf + PL::S, *sW = smf + PL::W, *sKh = smf + PL::KH, *sQh = smf + PL::QH, *sY = smf + PL::X,
-        *sdO = smf + PL::DO;
+  float *sE = smf + PL::E, *sKt = smf + PL::KT, *sW = smf + PL::W, *sY = smf + PL::Y, *sdO = smf + PL::DO;
+  float* sQh = sKt;
   float *sg = smf + PL::VEC, *sr = smf + PL::VEC + C;
   const size_t sd = (size_t)DK * p.dv;
   const size_t sb0 = ((size_t)s * p.H + h) * sd;
   for (int e = tid; e < DK * NS; e += THREADS) {
     const int d = e / NS, c = e % NS;
-    sE[d * LDT + c] = p.gST ? p.gST[sb0 + (size_t)d * p.dv + col0 + c] : 0.f;
+    sE[d * LDX + c] = p.gST ? p.gST[sb0 + (size_t)d * p.dv + col0 + c] : 0.f;
   }
   const int n_chunks = (t1 - t0 + C - 1) / C;
   const long long base = slot_base(s, t0);
+  const T* k = static_cast<const T*>(p.k);
+  const T* go = static_cast<const T*>(p.go);
+  const int rg = tid >> 4, c0 = (tid & 15) * 2;
   for (int ci = n_chunks - 1; ci >= 0; --ci) {
     const int tc0 = t0 + ci * C, n = min(C, t1 - tc0);
     const size_t wsi = (size_t)(base + ci) * p.H + h;
@@ -495,83 +623,111 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_dstates_kernel(const KPara
     float* gE = p.dE + wsi * sd;
     for (int e = tid; e < DK * NS; e += THREADS) {
       const int d = e / NS, c = e % NS;
-      gE[(size_t)d * p.dv + col0 + c] = sE[d * LDT + c];
+      gE[(size_t)d * p.dv + col0 + c] = sE[d * LDX + c];
     }
-    state_chunk_loads<DK, T>(p, wsi, tc0, n, h, sW, sQh, sKh, sg, sr, tid);
-    load_rows(sdO, LDT, static_cast<const T*>(p.go), tc0, n, h, p.H, p.dv, col0, NS, tid);
+    state_gates(p, wsi, sg, sr, tid);
+    store_transposed<DK>(sKt, n, [&](int i, int d) {
+      return sr[i] * ldx(k, ((size_t)(tc0 + i) * p.H + h) * DK + d);
+    }, tid);
+    load_ws_rows<DK>(sW, p.W + wsi * C * DK, tid);
+    for (int e = tid; e < C * NS; e += THREADS) {
+      const int i = e / NS, c = e % NS;
+      sdO[i * LDX + c] = (i < n) ? ldx(go, ((size_t)(tc0 + i) * p.H + h) * p.dv + col0 + c) : 0.f;
+    }
     __syncthreads();
     {
       // Y = Kh dE  [C][NS]
-      const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 2;
       float acc[4][2];
       zero(acc);
-      gemm<4, 2, DK>(acc, [&](int i, int k) { return sKh[(r0 + i) * LDK + k]; },
-                     [&](int k, int j) { return sE[k * LDT + c0 + j]; });
+      gemm_v<4, DK, LDCT, LDX>(acc, sKt + rg * 4, sE + c0);
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) sY[(r0 + i) * LDT + c0 + j] = acc[i][j];
+        for (int j = 0; j < 2; ++j) sY[(rg * 4 + i) * LDX + c0 + j] = acc[i][j];
     }
+    __syncthreads();
+    // Qh replaces Kh^T (its loads overlap the W^T Y product)
+    load_ws_rows<DK>(sQh, p.Qh + wsi * C * DK, tid);
+    float accW[TM][2];
+    zero(accW);
+    gemm_v<TM, C, LDK, LDX>(accW, sW + rg * TM, sY + c0);
     __syncthreads();
     {
       // dE = gamma_C dE - W^T Y + Qh^T dO  [DK][NS]
-      const int r0 = (tid >> 4) * TM, c0 = (tid & 15) * 2;
-      float acc[TM][2];
-      zero(acc);
-      gemm<TM, 2, C>(acc, [&](int i, int k) { return sQh[k * LDK + r0 + i]; },
-                     [&](int k, int j) { return sdO[k * LDT + c0 + j]; });
-      gemm<TM, 2, C>(acc, [&](int i, int k) { return -sW[k * LDK + r0 + i]; },
-                     [&](int k, int j) { return sY[k * LDT + c0 + j]; });
+      float accQ[TM][2];
+      zero(accQ);
+      gemm_v<TM, C, LDK, LDX>(accQ, sQh + rg * TM, sdO + c0);
       const float gC = expf(sg[C - 1]);
 #pragma unroll
       for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-          sE[(r0 + i) * LDT + c0 + j] = fmaf(gC, sE[(r0 + i) * LDT + c0 + j], acc[i][j]);
+          sE[(rg * TM + i) * LDX + c0 + j] =
+              fmaf(gC, sE[(rg * TM + i) * LDX + c0 + j], accQ[i][j] - accW[i][j]);
     }
   }
   __syncthreads();
   if (p.gS0)
     for (int e = tid; e < DK * NS; e += THREADS) {
       const int d = e / NS, c = e % NS;
-      p.gS0[sb0 + (size_t)d * p.dv + col0 + c] = sE[d * LDT + c];
+      p.gS0[sb0 + (size_t)d * p.dv + col0 + c] = sE[d * LDX + c];
     }
 }
 
+// Shared memory of the gradient kernel.  Every product reads float4 operands
+// in one of two patterns: "rows along k" (A[i][k..k+3] and B[j][k..k+3], both
+// row-major along the contraction) or "k-major" (A[k][i..i+3] and
+// B[k][j..j+3]); each small matrix is kept in the layout its products need,
+// some in both (dO, dR and U as [C][NS] rows and as [NS][C] transposes).
+// Row strides are multiples of 4 and = 4 mod 32 (conflict-free float4 reads
+// of the 8 rows a quarter-warp touches).
 template <int DK>
 struct GradPlan {
-  static constexpr int LDK = DK + 1;
-  static constexpr int K = 0;
-  static constexpr int Q = K + C * LDK;
-  static constexpr int KK = Q + C * LDK;
-  static constexpr int P = KK + C * LDC;
-  static constexpr int T = P + C * LDC;
-  static constexpr int S = T + C * LDC;        // [DK][LDT]
-  static constexpr int E = S + DK * LDT;       // [DK][LDT]
-  static constexpr int TILES = E + DK * LDT;   // 7 x [C][LDT]: V, dO, KS, R, U, dU, dR
-  static constexpr int VEC = TILES + 7 * C * LDT;
+  static constexpr int LDK = DK + 4;
+  static constexpr int K = 0;                    // [C][LDK]
+  static constexpr int Q = K + C * LDK;          // [C][LDK]
+  static constexpr int KK = Q + C * LDK;         // [C][LDC] D o K K^T, strictly lower
+  static constexpr int P = KK + C * LDC;         // [C][LDC] scale D o Q K^T, lower
+  static constexpr int T = P + C * LDC;          // [C][LDC]
+  static constexpr int ST = T + C * LDC;         // [NS][LDK] S_J^T (tile of the start state)
+  static constexpr int ET = ST + NS * LDK;       // [NS][LDK] dE_J^T
+  static constexpr int TILES = ET + NS * LDK;
+  // tiles: dO, U, dU (then dR) as [C][LDN]; R^T, dO^T, (r U)^T, (-b gamma dR)^T as [NS][LDC]
+  static constexpr int DO = TILES;
+  static constexpr int U = DO + C * LDN;
+  static constexpr int DU = U + C * LDN;
+  static constexpr int RT = DU + C * LDN;
+  static constexpr int DOT = RT + NS * LDC;
+  static constexpr int UT = DOT + NS * LDC;
+  static constexpr int DRT = UT + NS * LDC;
+  static constexpr int VEC = DRT + NS * LDC;
   static constexpr int FLOATS = VEC + 10 * C + 4;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
-  static_assert(7 * C * LDT >= 2 * C * LDC, "dA and dP reuse the tile area");
+  static_assert(VEC - TILES >= 3 * C * LDC, "the final phase's three C x C matrices reuse the tile area");
+  static_assert(BYTES <= 232448, "shared memory of one CTA");
 };
 
-// 4. Per (chunk, head): every gradient of the chunk's tokens.
+
+// 4. Per (chunk, head): every gradient of the chunk's tokens.  Thread maps
+// (rg = tid / 16, cg = tid % 16; rows 4 rg .. 4 rg + 3 everywhere):
+//   [C][NS] tiles: columns cg, cg + 16 (two per thread);
+//   C x C:         columns cg + 16 j, j < 4;
+//   C x DK:        columns 4 cg .. 4 cg + 3 (and 64 + 4 cg .. for DK = 128).
 template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams p) {
-  extern __shared__ float smf[];
+  extern __shared__ __align__(16) float smf[];
   using PL = GradPlan<DK>;
   constexpr int LDK = PL::LDK;
-  constexpr int TN = DK / 16;
+  constexpr int NV = DK / 64;                    // float4 column groups per thread in C x DK
   const int tid = threadIdx.x;
   const long long slot = blockIdx.x / p.H;
   const int h = blockIdx.x % p.H;
   int s, c, t0, n;
   if (!slot_chunk(p, slot, s, c, t0, n)) return;
   float *sK = smf + PL::K, *sQ = smf + PL::Q, *sKK = smf + PL::KK, *sP = smf + PL::P, *sT = smf + PL::T;
-  float *sS = smf + PL::S, *sE = smf + PL::E;
-  float* tiles = smf + PL::TILES;
-  float *sV = tiles, *sdO = tiles + C * LDT, *sKS = tiles + 2 * C * LDT, *sR = tiles + 3 * C * LDT,
-        *sU = tiles + 4 * C * LDT, *sdU = tiles + 5 * C * LDT, *sdR = tiles + 6 * C * LDT;
+  float *sSt = smf + PL::ST, *sEt = smf + PL::ET;
+  float *sdO = smf + PL::DO, *sU = smf + PL::U, *sdU = smf + PL::DU, *sRt = smf + PL::RT,
+        *sdOt = smf + PL::DOT, *sUt = smf + PL::UT, *sdRt = smf + PL::DRT;
   float* vec = smf + PL::VEC;
   Vec V{vec, vec + C, vec + 2 * C, vec + 3 * C, vec + 4 * C};
   float *s_db = vec + 5 * C, *s_dg = vec + 6 * C, *s_kap = vec + 7 * C, *s_red = vec + 8 * C;
@@ -583,194 +739,233 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
   const float* gE = p.dE + wsi * sd;
   const int rg = tid >> 4, cg = tid & 15;
   const int r0 = rg * 4;
-  // register accumulators (fixed thread -> element map over all tiles)
-  float dA[4][4], dP[4][4], dq[4][TN], dk[4][TN];
+  // register accumulators (the same thread -> element map over all tiles)
+  float dA[4][4], dP[4][4], dq[4][4 * NV], dk[4][4 * NV];
   zero(dA);
   zero(dP);
   zero(dq);
   zero(dk);
   float rd_db[4] = {0.f, 0.f, 0.f, 0.f}, rd_dg[4] = {0.f, 0.f, 0.f, 0.f}, rd_kap[4] = {0.f, 0.f, 0.f, 0.f};
   float es = 0.f;   // partial <dE, S>
+  float gam[4], bb[4], rr[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    gam[i] = V.gam[r0 + i];
+    bb[i] = V.b[r0 + i];
+    rr[i] = V.r[r0 + i];
+  }
   const T* v = static_cast<const T*>(p.v);
   const T* go = static_cast<const T*>(p.go);
 
   for (int col0 = 0; col0 < p.dv; col0 += NS) {
     __syncthreads();
+    // tiles of S and dE (transposed into [NS][DK]), dO (rows and transpose), V (registers)
     for (int e = tid; e < DK * NS; e += THREADS) {
       const int d = e / NS, cc = e % NS;
       const float x = gS[(size_t)d * p.dv + col0 + cc], y = gE[(size_t)d * p.dv + col0 + cc];
-      sS[d * LDT + cc] = x;
-      sE[d * LDT + cc] = y;
+      sSt[cc * LDK + d] = x;
+      sEt[cc * LDK + d] = y;
       es = fmaf(x, y, es);
     }
-    load_rows(sV, LDT, v, t0, n, h, p.H, p.dv, col0, NS, tid);
-    load_rows(sdO, LDT, go, t0, n, h, p.H, p.dv, col0, NS, tid);
+    for (int e = tid; e < C * NS; e += THREADS) {
+      const int i = e / NS, cc = e % NS;
+      const float x = (i < n) ? ldx(go, ((size_t)(t0 + i) * p.H + h) * p.dv + col0 + cc) : 0.f;
+      sdO[i * LDN + cc] = x;
+      sdOt[cc * LDC + i] = x;
+    }
+    float vv[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        vv[i][u] = (r0 + i < n) ? ldx(v, ((size_t)(t0 + r0 + i) * p.H + h) * p.dv + col0 + cg + 16 * u) : 0.f;
     __syncthreads();
-    const int c0 = cg * 2;
+    // KS = K S_J, KdE = K dE_J (rows along k); R = diag(b) (V - diag(gamma) KS) -> R^T;
+    // the first part of dU, diag(r) KdE, stays in registers
+    float ks[4][2], du0[4][2];
     {
-      // KS = K S_J, KdE = K dE_J; R = diag(b) (V - diag(gamma) KS); dU = diag(r) KdE
-      float ks[4][2], ke[4][2];
+      float ke[4][2];
       zero(ks);
       zero(ke);
-#pragma unroll 4
-      for (int k = 0; k < DK; ++k) {
-        float av[4];
+#pragma unroll 2
+      for (int k = 0; k < DK; k += 4) {
+        float4 a[4], bs[2], be[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) av[i] = sK[(r0 + i) * LDK + k];
-        const float b0 = sS[k * LDT + c0], b1 = sS[k * LDT + c0 + 1];
-        const float e0 = sE[k * LDT + c0], e1 = sE[k * LDT + c0 + 1];
+        for (int i = 0; i < 4; ++i) a[i] = lds4(sK + (r0 + i) * LDK + k);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          bs[u] = lds4(sSt + (cg + 16 * u) * LDK + k);
+          be[u] = lds4(sEt + (cg + 16 * u) * LDK + k);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            ks[i][u] = dot4(a[i], bs[u], ks[i][u]);
+            ke[i][u] = dot4(a[i], be[u], ke[i][u]);
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          sRt[(cg + 16 * u) * LDC + r0 + i] = bb[i] * (vv[i][u] - gam[i] * ks[i][u]);
+          du0[i][u] = rr[i] * ke[i][u];
+        }
+    }
+    __syncthreads();
+    {
+      // U = T R (rows along k), into U rows and (r U)^T; kappa partials.
+      // dU = diag(r) KdE + P^T dO (k-major), into dU rows.
+      float uu[4][2], pd[4][2];
+      zero(uu);
+      zero(pd);
+#pragma unroll 2
+      for (int k = 0; k < C; k += 4) {
+        float4 a[4], b[2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = lds4(sT + (r0 + i) * LDC + k);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) b[u] = lds4(sRt + (cg + 16 * u) * LDC + k);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int u = 0; u < 2; ++u) uu[i][u] = dot4(a[i], b[u], uu[i][u]);
+      }
+#pragma unroll 4
+      for (int k = 0; k < C; ++k) {
+        const float4 a4 = lds4(sP + k * LDC + r0);
+        const float b0 = sdO[k * LDN + cg], b1 = sdO[k * LDN + cg + 16];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          ks[i][0] = fmaf(av[i], b0, ks[i][0]);
-          ks[i][1] = fmaf(av[i], b1, ks[i][1]);
-          ke[i][0] = fmaf(av[i], e0, ke[i][0]);
-          ke[i][1] = fmaf(av[i], e1, ke[i][1]);
+          pd[i][0] = fmaf(f4(a4, i), b0, pd[i][0]);
+          pd[i][1] = fmaf(f4(a4, i), b1, pd[i][1]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int cc = cg + 16 * u;
+          sU[(r0 + i) * LDN + cc] = uu[i][u];
+          sUt[cc * LDC + r0 + i] = rr[i] * uu[i][u];
+          rd_kap[i] = fmaf(uu[i][u], du0[i][u], rd_kap[i]);
+          sdU[(r0 + i) * LDN + cc] = du0[i][u] + pd[i][u];
+        }
+    }
+    __syncthreads();
+    float dr[4][2];
+    {
+      // dR = T^T dU (k-major); grad_v = diag(b) dR; db and dg row partials
+      zero(dr);
+#pragma unroll 4
+      for (int k = 0; k < C; ++k) {
+        const float4 a4 = lds4(sT + k * LDC + r0);
+        const float b0 = sdU[k * LDN + cg], b1 = sdU[k * LDN + cg + 16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dr[i][0] = fmaf(f4(a4, i), b0, dr[i][0]);
+          dr[i][1] = fmaf(f4(a4, i), b1, dr[i][1]);
         }
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = r0 + i;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          sKS[r * LDT + c0 + j] = ks[i][j];
-          sR[r * LDT + c0 + j] = V.b[r] * (sV[r * LDT + c0 + j] - V.gam[r] * ks[i][j]);
-          sdU[r * LDT + c0 + j] = V.r[r] * ke[i][j];
+        for (int u = 0; u < 2; ++u) {
+          rd_db[i] = fmaf(dr[i][u], vv[i][u] - gam[i] * ks[i][u], rd_db[i]);
+          rd_dg[i] = fmaf(-bb[i] * gam[i] * dr[i][u], ks[i][u], rd_dg[i]);
+          if (r < n) p.gv[((size_t)(t0 + r) * p.H + h) * p.dv + col0 + cg + 16 * u] = bb[i] * dr[i][u];
         }
       }
     }
-    __syncthreads();
-    {
-      // U = T R; kappa partials U_i . (diag(r) KdE)_i
-      float acc[4][2];
-      zero(acc);
-      gemm<4, 2, C>(acc, [&](int i, int k) { return sT[(r0 + i) * LDC + k]; },
-                    [&](int k, int j) { return sR[k * LDT + c0 + j]; });
+    __syncthreads();                               // every read of dU is done: dR replaces it
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          sU[(r0 + i) * LDT + c0 + j] = acc[i][j];
-          rd_kap[i] = fmaf(acc[i][j], sdU[(r0 + i) * LDT + c0 + j], rd_kap[i]);
-        }
-    }
-    __syncthreads();
-    {
-      // dU += P^T dO
-      float acc[4][2];
-      zero(acc);
-      gemm<4, 2, C>(acc, [&](int i, int k) { return sP[k * LDC + r0 + i]; },
-                    [&](int k, int j) { return sdO[k * LDT + c0 + j]; });
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) sdU[(r0 + i) * LDT + c0 + j] += acc[i][j];
-    }
-    __syncthreads();
-    {
-      // dR = T^T dU; grad_v = diag(b) dR; db and dg row partials
-      float acc[4][2];
-      zero(acc);
-      gemm<4, 2, C>(acc, [&](int i, int k) { return sT[k * LDC + r0 + i]; },
-                    [&](int k, int j) { return sdU[k * LDT + c0 + j]; });
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = r0 + i;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const float dr = acc[i][j], ksv = sKS[r * LDT + c0 + j];
-          sdR[r * LDT + c0 + j] = dr;
-          rd_db[i] = fmaf(dr, sV[r * LDT + c0 + j] - V.gam[r] * ksv, rd_db[i]);
-          rd_dg[i] = fmaf(-V.b[r] * V.gam[r] * dr, ksv, rd_dg[i]);
-        }
-        if (r < n) {
-          float* gvr = p.gv + ((size_t)(t0 + r) * p.H + h) * p.dv + col0 + c0;
-          gvr[0] = V.b[r] * acc[i][0];
-          gvr[1] = V.b[r] * acc[i][1];
-        }
+      for (int u = 0; u < 2; ++u) {
+        const int cc = cg + 16 * u;
+        sdU[(r0 + i) * LDN + cc] = dr[i][u];
+        sdRt[cc * LDC + r0 + i] = -bb[i] * gam[i] * dr[i][u];
       }
-    }
     __syncthreads();
     {
-      // dA += dR U^T, dP += dO U^T  (C x C, K = NS; columns cg + 16 j)
-#pragma unroll 4
-      for (int k = 0; k < NS; ++k) {
-        float ar[4], ao[4], bu[4];
+      // dA += dR U^T, dP += dO U^T (rows along k)
+#pragma unroll 2
+      for (int k = 0; k < NS; k += 4) {
+        float4 ar[4], ao[4], bu[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          ar[i] = sdR[(r0 + i) * LDT + k];
-          ao[i] = sdO[(r0 + i) * LDT + k];
+          ar[i] = lds4(sdU + (r0 + i) * LDN + k);
+          ao[i] = lds4(sdO + (r0 + i) * LDN + k);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) bu[j] = sU[(cg + 16 * j) * LDT + k];
+        for (int j = 0; j < 4; ++j) bu[j] = lds4(sU + (cg + 16 * j) * LDN + k);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            dA[i][j] = fmaf(ar[i], bu[j], dA[i][j]);
-            dP[i][j] = fmaf(ao[i], bu[j], dP[i][j]);
+            dA[i][j] = dot4(ar[i], bu[j], dA[i][j]);
+            dP[i][j] = dot4(ao[i], bu[j], dP[i][j]);
           }
       }
-      // dq += dO S_J^T  (C x DK, K = NS; columns cg + 16 j)
-      gemm<4, TN, NS>(dq, [&](int i, int k) { return sdO[(r0 + i) * LDT + k]; },
-                      [&](int k, int j) { return sS[(cg + 16 * j) * LDT + k]; });
-    }
-    __syncthreads();
-    // row scalings for dk: dR <- -b gamma dR, U <- r U
-    for (int e = tid; e < C * NS; e += THREADS) {
-      const int i = e / NS, cc = e % NS;
-      sdR[i * LDT + cc] *= -V.b[i] * V.gam[i];
-      sU[i * LDT + cc] *= V.r[i];
-    }
-    __syncthreads();
-    {
-      // dk += (-b gamma dR) S_J^T + (r U) dE_J^T
-      gemm<4, TN, NS>(dk, [&](int i, int k) { return sdR[(r0 + i) * LDT + k]; },
-                      [&](int k, int j) { return sS[(cg + 16 * j) * LDT + k]; });
-      gemm<4, TN, NS>(dk, [&](int i, int k) { return sU[(r0 + i) * LDT + k]; },
-                      [&](int k, int j) { return sE[(cg + 16 * j) * LDT + k]; });
+      // dq += dO S_J^T; dk += (-b gamma dR) S_J^T + (r U) dE_J^T (k-major)
+#pragma unroll 2
+      for (int k = 0; k < NS; ++k) {
+        const float4 ao = lds4(sdOt + k * LDC + r0), ar = lds4(sdRt + k * LDC + r0), au = lds4(sUt + k * LDC + r0);
+#pragma unroll
+        for (int w = 0; w < NV; ++w) {
+          const float4 bs = lds4(sSt + k * LDK + 64 * w + 4 * cg), be = lds4(sEt + k * LDK + 64 * w + 4 * cg);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              dq[i][4 * w + e] = fmaf(f4(ao, i), f4(bs, e), dq[i][4 * w + e]);
+              dk[i][4 * w + e] = fmaf(f4(ar, i), f4(bs, e), fmaf(f4(au, i), f4(be, e), dk[i][4 * w + e]));
+            }
+        }
+      }
     }
   }
+  __syncthreads();                                 // the tile area is free
 
   // ---- row partials -> per-row values (threads with cg == 0 hold the rows)
-  {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float qd = 0.f;
+  for (int i = 0; i < 4; ++i) {
+    float qd = 0.f;
 #pragma unroll
-      for (int j = 0; j < TN; ++j) qd = fmaf(sQ[(r0 + i) * LDK + cg + 16 * j], dq[i][j], qd);
-      qd = half_warp_sum(qd);
-      const float db = half_warp_sum(rd_db[i]);
-      const float dg = half_warp_sum(rd_dg[i]);
-      const float kap = half_warp_sum(rd_kap[i]);
-      if (cg == 0) {
-        const int r = r0 + i;
-        s_db[r] = db;
-        s_dg[r] = dg + p.scale * V.gam[r] * qd;
-        s_kap[r] = kap;
-      }
+    for (int w = 0; w < NV; ++w)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qd = fmaf(sQ[(r0 + i) * LDK + 64 * w + 4 * cg + e], dq[i][4 * w + e], qd);
+    qd = half_warp_sum(qd);
+    const float db = half_warp_sum(rd_db[i]);
+    const float dg = half_warp_sum(rd_dg[i]);
+    const float kap = half_warp_sum(rd_kap[i]);
+    if (cg == 0) {
+      const int r = r0 + i;
+      s_db[r] = db;
+      s_dg[r] = dg + p.scale * gam[i] * qd;
+      s_kap[r] = kap;
     }
-    // <dE, S>
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) es += __shfl_xor_sync(0xffffffffu, es, off);
-    if ((tid & 31) == 0) s_red[tid >> 5] = es;
   }
-  __syncthreads();
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) es += __shfl_xor_sync(0xffffffffu, es, off);
+  if ((tid & 31) == 0) s_red[tid >> 5] = es;
   // dA, dP (unscaled) into the tile area
-  float* sdA = tiles;
-  float* sdP = tiles + C * LDC;
-  {
+  float* sdA = smf + PL::TILES;
+  float* sdP = sdA + C * LDC;
+  float* sPbT = sdP + C * LDC;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = r0 + i, cc = cg + 16 * j;
-        sdA[r * LDC + cc] = (cc < r) ? -dA[i][j] : 0.f;
-        sdP[r * LDC + cc] = (cc <= r) ? dP[i][j] : 0.f;
-      }
-  }
+    for (int j = 0; j < 4; ++j) {
+      const int r = r0 + i, cc = cg + 16 * j;
+      sdA[r * LDC + cc] = (cc < r) ? -dA[i][j] : 0.f;
+      sdP[r * LDC + cc] = (cc <= r) ? dP[i][j] : 0.f;
+    }
   __syncthreads();
   if (tid < C) {
-    // dg and db of row i; then scale dA, dP rows into A' and dP o scale D below
+    // dg and db of row i
     const int i = tid;
     float dg = s_dg[i] - s_kap[i], db = s_db[i];
     for (int j = 0; j < C; ++j) {
@@ -800,7 +995,6 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
       const float y = __shfl_down_sync(0xffffffffu, suf, off);
       if (lane + off < 32) suf += y;
     }
-    // suf = sum over pairs lane .. 31
     const float d1 = suf - x0;     // rows 2 lane + 1 .. 63
     const float d0 = suf;          // rows 2 lane .. 63
 #pragma unroll
@@ -813,33 +1007,62 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
       }
     }
   }
-  // A'_ij = dA_ij b_i D_ij, Pb_ij = dP_ij scale D_ij (in place)
-  for (int e = tid; e < C * C; e += THREADS) {
-    const int i = e / C, j = e % C;
-    const float d = (j <= i) ? expf(V.g[i] - V.g[j]) : 0.f;
-    sdA[i * LDC + j] *= V.b[i] * d;
-    sdP[i * LDC + j] *= p.scale * d;
+  // Pb = dP o scale D (also transposed) and M = A' + A'^T, A'_ij = dA_ij b_i D_ij:
+  // computed into registers, then written over dA and dP
+  {
+    float pb[16], mm[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const int e = tid + THREADS * m, i = e / C, j = e % C;
+      const float dij = (j <= i) ? expf(V.g[i] - V.g[j]) : 0.f;
+      const float dji = (i <= j) ? expf(V.g[j] - V.g[i]) : 0.f;
+      pb[m] = sdP[i * LDC + j] * p.scale * dij;
+      mm[m] = sdA[i * LDC + j] * V.b[i] * dij + sdA[j * LDC + i] * V.b[j] * dji;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const int e = tid + THREADS * m, i = e / C, j = e % C;
+      sdP[i * LDC + j] = pb[m];
+      sPbT[j * LDC + i] = pb[m];
+      sdA[i * LDC + j] = mm[m];
+    }
   }
   __syncthreads();
   {
-    // dq = scale diag(gamma) dq + Pb K;  dk += (A' + A'^T) K + Pb^T Q
-    float acc[4][TN];
+    // dq = scale diag(gamma) dq + Pb K;  dk += M K + Pb^T Q  (k-major)
+    float acc[4][4 * NV];
     zero(acc);
-    gemm<4, TN, C>(acc, [&](int i, int k) { return sdP[(r0 + i) * LDC + k]; },
-                   [&](int k, int j) { return sK[k * LDK + cg + 16 * j]; });
-    gemm<4, TN, C>(dk, [&](int i, int k) { return sdA[(r0 + i) * LDC + k] + sdA[k * LDC + r0 + i]; },
-                   [&](int k, int j) { return sK[k * LDK + cg + 16 * j]; });
-    gemm<4, TN, C>(dk, [&](int i, int k) { return sdP[k * LDC + r0 + i]; },
-                   [&](int k, int j) { return sQ[k * LDK + cg + 16 * j]; });
+#pragma unroll 2
+    for (int k = 0; k < C; ++k) {
+      const float4 apt = lds4(sPbT + k * LDC + r0), am = lds4(sdA + k * LDC + r0), ap = lds4(sdP + k * LDC + r0);
+#pragma unroll
+      for (int w = 0; w < NV; ++w) {
+        const float4 bk = lds4(sK + k * LDK + 64 * w + 4 * cg), bq = lds4(sQ + k * LDK + 64 * w + 4 * cg);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[i][4 * w + e] = fmaf(f4(apt, i), f4(bk, e), acc[i][4 * w + e]);
+            dk[i][4 * w + e] = fmaf(f4(am, i), f4(bk, e), fmaf(f4(ap, i), f4(bq, e), dk[i][4 * w + e]));
+          }
+      }
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = r0 + i;
       if (r < n) {
-        const size_t row = ((size_t)(t0 + r) * p.H + h) * DK + cg;
+        const size_t row = ((size_t)(t0 + r) * p.H + h) * DK;
 #pragma unroll
-        for (int j = 0; j < TN; ++j) {
-          p.gq[row + 16 * j] = fmaf(p.scale * V.gam[r], dq[i][j], acc[i][j]);
-          p.gk[row + 16 * j] = dk[i][j];
+        for (int w = 0; w < NV; ++w) {
+          float4 oq, ok;
+          oq.x = fmaf(p.scale * gam[i], dq[i][4 * w + 0], acc[i][4 * w + 0]);
+          oq.y = fmaf(p.scale * gam[i], dq[i][4 * w + 1], acc[i][4 * w + 1]);
+          oq.z = fmaf(p.scale * gam[i], dq[i][4 * w + 2], acc[i][4 * w + 2]);
+          oq.w = fmaf(p.scale * gam[i], dq[i][4 * w + 3], acc[i][4 * w + 3]);
+          ok = make_float4(dk[i][4 * w + 0], dk[i][4 * w + 1], dk[i][4 * w + 2], dk[i][4 * w + 3]);
+          *reinterpret_cast<float4*>(p.gq + row + 64 * w + 4 * cg) = oq;
+          *reinterpret_cast<float4*>(p.gk + row + 64 * w + 4 * cg) = ok;
         }
       }
     }
@@ -857,16 +1080,16 @@ static gdn_status launch_all(const KParams& kp, const gdn_bwd_params* p, cudaStr
   static std::atomic<bool> set_prep[kMaxDevices], set_st[kMaxDevices], set_dst[kMaxDevices],
       set_gr[kMaxDevices];
   if (smem_attr_once(set_prep, gdn_bwd_prep_kernel<DK, T>, PrepPlan<DK>::BYTES) != cudaSuccess ||
-      smem_attr_once(set_st, gdn_bwd_states_kernel<DK, T>, StatePlan<DK>::BYTES) != cudaSuccess ||
-      smem_attr_once(set_dst, gdn_bwd_dstates_kernel<DK, T>, StatePlan<DK>::BYTES) != cudaSuccess ||
+      smem_attr_once(set_st, gdn_bwd_states_kernel<DK, T>, StatesPlan<DK>::BYTES) != cudaSuccess ||
+      smem_attr_once(set_dst, gdn_bwd_dstates_kernel<DK, T>, DStatesPlan<DK>::BYTES) != cudaSuccess ||
       smem_attr_once(set_gr, gdn_bwd_grads_kernel<DK, T>, GradPlan<DK>::BYTES) != cudaSuccess)
     return GDN_ERR_CUDA;
   const long long chunk_blocks = kp.n_slots * p->H;
   const long long chain_blocks = (long long)p->n_seq * p->H * (p->dv / NS);
   if (chunk_blocks > 0x7fffffffLL || chain_blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   gdn_bwd_prep_kernel<DK, T><<<(unsigned)chunk_blocks, THREADS, PrepPlan<DK>::BYTES, stream>>>(kp);
-  gdn_bwd_states_kernel<DK, T><<<(unsigned)chain_blocks, THREADS, StatePlan<DK>::BYTES, stream>>>(kp);
-  gdn_bwd_dstates_kernel<DK, T><<<(unsigned)chain_blocks, THREADS, StatePlan<DK>::BYTES, stream>>>(kp);
+  gdn_bwd_states_kernel<DK, T><<<(unsigned)chain_blocks, THREADS, StatesPlan<DK>::BYTES, stream>>>(kp);
+  gdn_bwd_dstates_kernel<DK, T><<<(unsigned)chain_blocks, THREADS, DStatesPlan<DK>::BYTES, stream>>>(kp);
   gdn_bwd_grads_kernel<DK, T><<<(unsigned)chunk_blocks, THREADS, GradPlan<DK>::BYTES, stream>>>(kp);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -16,11 +16,17 @@
 //     U     = T diag(b) (V - (K o e^G) Sigma_0)
 //     O     = scale ((Q o e^G) Sigma_0 + P U)
 //     Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
-// The decay of each (i, j, c) term is its own exponential (no factorisation
-// into e^{G_i} e^{-G_j}, which overflows when a channel decays hard), so every
-// exponent is <= 0.  One CTA of 256 threads per (sequence, head, 64-column dv
-// slice); the output epilogue (head-wise gate, loop residual) is the precise
-// path's.
+// When every channel's decay over the chunk is moderate (G_0c - G_{C-1,c} <=
+// kFactorRange), the decay factors split around the channel's midpoint m_c,
+// e^{G_ic - G_jc} = e^{G_ic - m_c} e^{m_c - G_jc} (each factor within
+// e^{+-kFactorRange/2}), and A and P become plain products:
+// A = diag(b) K~ K^^T and P = Q~ K^^T (lower parts) with K~ = K o e^{G-m},
+// K^ = K o e^{m-G}, Q~ = Q o e^{G-m}: two exponentials per (i, c) instead of
+// one per (i, j, c).
+// Otherwise (a channel that decays hard or resets) the decay of each (i, j, c)
+// term is its own exponential, so every exponent is <= 0.  One CTA of 256
+// threads per (sequence, head, 64-column dv slice); the output epilogue
+// (head-wise gate, loop residual) is the precise path's.
 #include "common.cuh"
 
 namespace gdn {
@@ -29,7 +35,13 @@ namespace kda {
 constexpr int C = 64;
 constexpr int DVS = 64;
 constexpr int THREADS = 256;
-constexpr int LDC = C + 1;
+constexpr int LDC = C + 4;        // C x C and [rows][DVS] tiles: float4 rows
+constexpr float kFactorRange = 80.f;   // largest per-channel log-decay range of a factored chunk
+
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+}
 
 // T = (I + A)^{-1} for the strictly lower C x C matrix A (row stride LDC in
 // shared memory), column `col` per thread: forward substitution with the
@@ -52,7 +64,7 @@ __device__ __forceinline__ void solve_column(const float* sA, float* sT, int col
 
 template <int DK>
 struct Plan {
-  static constexpr int LDK = DK + 1;
+  static constexpr int LDK = DK + 4;               // float4 rows (the factored A and P products)
   static constexpr int K = 0;                      // [C][LDK]  K, then K o e^{G_C - G}
   static constexpr int Q = K + C * LDK;            // [C][LDK]  Q, then Q o e^G
   static constexpr int G = Q + C * LDK;            // [C][LDK]  G, then K o e^G
@@ -64,7 +76,8 @@ struct Plan {
   static constexpr int U = P + C * LDC;            // [C][LDC]
   static constexpr int B = U + C * LDC;            // b: C
   static constexpr int GC = B + C;                 // e^{G_C}: DK
-  static constexpr int FLOATS = GC + DK + 4;
+  static constexpr int MID = GC + DK;              // factored chunks: m, e^m, e^{G_C - m}: 3 x DK
+  static constexpr int FLOATS = MID + 3 * DK + 4;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 static_assert(Plan<128>::BYTES <= 232448, "KDA prefill shared memory");
@@ -88,7 +101,7 @@ template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Params p) {
   using PL = Plan<DK>;
   constexpr int LDK = PL::LDK;
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   float* sK = sm + PL::K;
   float* sQ = sm + PL::Q;
   float* sG = sm + PL::G;
@@ -100,6 +113,9 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
   float* sU = sm + PL::U;
   float* sb = sm + PL::B;
   float* sgc = sm + PL::GC;
+  float* smid = sm + PL::MID;
+  float* sem = smid + DK;
+  float* sec = sem + DK;
 
   const int tid = threadIdx.x;
   const int slice = blockIdx.x % p.n_slices;
@@ -176,92 +192,257 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
       for (int d = 0; d < DK; ++d) row[d] = to_f32(from_f32<T>(row[d] * inv));
     }
     __syncthreads();
-    // ---- A and P, each term with its own decay e^{G_ic - G_jc} (the fast
-    // exponential: a few ulp on arguments <= 0, far inside the fp32 bar)
-    // (only the lower triangle j <= i is enumerated; the upper one is zero)
-    for (int e = tid; e < C * (C + 1) / 2; e += THREADS) {
-      int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-      while (i * (i + 1) / 2 > e) --i;
-      while ((i + 1) * (i + 2) / 2 <= e) ++i;
-      const int j = e - i * (i + 1) / 2;
-      float kk = 0.f, qk = 0.f;
-#pragma unroll 8
-      for (int d = 0; d < DK; ++d) {
-        const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
-        const float kj = sK[j * LDK + d] * dec;
-        kk = fmaf(sK[i * LDK + d], kj, kk);
-        qk = fmaf(sQ[i * LDK + d], kj, qk);
-      }
-      sA[i * LDC + j] = (j < i) ? sb[i] * kk : 0.f;
-      sP[i * LDC + j] = qk;
+    // ---- G_C, the channel midpoints, and whether the chunk factors
+    if (tid < DK) {
+      const float g0 = sG[tid], gc = sG[(C - 1) * LDK + tid];
+      sgc[tid] = gc;                                  // G_C (rows past the end keep it)
+      smid[tid] = 0.5f * (g0 + gc);
     }
-    for (int e = tid; e < C * (C - 1) / 2; e += THREADS) {   // the strict upper triangle
-      int j = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-      while (j * (j + 1) / 2 > e) --j;
-      while ((j + 1) * (j + 2) / 2 <= e) ++j;
-      const int i = e - j * (j + 1) / 2;            // i <= j, then shifted: column j + 1 > row i
-      sA[i * LDC + j + 1] = 0.f;
-      sP[i * LDC + j + 1] = 0.f;
-    }
-    if (tid < DK) sgc[tid] = sG[(C - 1) * LDK + tid];   // G_C (rows past the end keep it)
-    __syncthreads();
-    // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
-    // operands: Q o e^G over Q, K o e^G over G, K o e^{G_C - G} over K
-    if (tid < C) {
-      solve_column<C, LDC>(sA, sT, tid);
-    } else {
-      for (int e = tid - C; e < C * DK; e += THREADS - C) {
+    const bool factored =
+        !__syncthreads_or(tid < DK && !(sG[tid] - sG[(C - 1) * LDK + tid] <= kFactorRange));
+    if (factored) {
+      // K^ = K o e^{m - G} over K, K~ = K o e^{G - m} over G, Q~ = Q o e^{G - m} over Q
+      for (int e = tid; e < C * DK; e += THREADS) {
         const int i = e / DK, d = e % DK;
-        const float g = sG[i * LDK + d];
-        const float eg = expf(g);
+        const float g = sG[i * LDK + d] - smid[d];
+        const float ex = expf(g), fx = expf(-g);
         const float kv = sK[i * LDK + d];
-        sQ[i * LDK + d] *= eg;
-        sG[i * LDK + d] = kv * eg;
-        sK[i * LDK + d] = kv * expf(sgc[d] - g);
+        sK[i * LDK + d] = kv * fx;
+        sG[i * LDK + d] = kv * ex;
+        sQ[i * LDK + d] *= ex;
+      }
+      if (tid < DK) {
+        sem[tid] = expf(smid[tid]);
+        sec[tid] = expf(sgc[tid] - smid[tid]);
+      }
+      __syncthreads();
+      {
+        // A = diag(b) K~ K^^T (strictly lower), P = Q~ K^^T (lower): thread rows
+        // r0 .. r0 + 3, columns cg + 16 j, four channels per read
+        const int r0 = (tid >> 4) * 4, cg = tid & 15;
+        float kk[4][4], qk[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) kk[i][j] = qk[i][j] = 0.f;
+#pragma unroll 2
+        for (int d = 0; d < DK; d += 4) {
+          float4 ak[4], aq[4], bk[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            ak[i] = lds4(sG + (r0 + i) * LDK + d);
+            aq[i] = lds4(sQ + (r0 + i) * LDK + d);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) bk[j] = lds4(sK + (cg + 16 * j) * LDK + d);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              kk[i][j] = dot4(ak[i], bk[j], kk[i][j]);
+              qk[i][j] = dot4(aq[i], bk[j], qk[i][j]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = r0 + i, cc = cg + 16 * j;
+            sA[r * LDC + cc] = (cc < r) ? sb[r] * kk[i][j] : 0.f;
+            sP[r * LDC + cc] = (cc <= r) ? qk[i][j] : 0.f;
+          }
+      }
+      __syncthreads();
+      // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
+      // operands from the factored ones: Q o e^G = Q~ e^m, K o e^G = K~ e^m,
+      // K o e^{G_C - G} = K^ e^{G_C - m}
+      if (tid < C) {
+        solve_column<C, LDC>(sA, sT, tid);
+      } else {
+        for (int e = tid - C; e < C * DK; e += THREADS - C) {
+          const int i = e / DK, d = e % DK;
+          sQ[i * LDK + d] *= sem[d];
+          sG[i * LDK + d] *= sem[d];
+          sK[i * LDK + d] *= sec[d];
+        }
+      }
+    } else {
+      // ---- A and P, each term with its own decay e^{G_ic - G_jc} (the fast
+      // exponential: a few ulp on arguments <= 0, far inside the fp32 bar)
+      // (only the lower triangle j <= i is enumerated; the upper one is zero)
+      for (int e = tid; e < C * (C + 1) / 2; e += THREADS) {
+        int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+        while (i * (i + 1) / 2 > e) --i;
+        while ((i + 1) * (i + 2) / 2 <= e) ++i;
+        const int j = e - i * (i + 1) / 2;
+        float kk = 0.f, qk = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < DK; ++d) {
+          const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
+          const float kj = sK[j * LDK + d] * dec;
+          kk = fmaf(sK[i * LDK + d], kj, kk);
+          qk = fmaf(sQ[i * LDK + d], kj, qk);
+        }
+        sA[i * LDC + j] = (j < i) ? sb[i] * kk : 0.f;
+        sP[i * LDC + j] = qk;
+      }
+      for (int e = tid; e < C * (C - 1) / 2; e += THREADS) {   // the strict upper triangle
+        int j = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+        while (j * (j + 1) / 2 > e) --j;
+        while ((j + 1) * (j + 2) / 2 <= e) ++j;
+        const int i = e - j * (j + 1) / 2;            // i <= j, then shifted: column j + 1 > row i
+        sA[i * LDC + j + 1] = 0.f;
+        sP[i * LDC + j + 1] = 0.f;
+      }
+      __syncthreads();
+      // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
+      // operands: Q o e^G over Q, K o e^G over G, K o e^{G_C - G} over K
+      if (tid < C) {
+        solve_column<C, LDC>(sA, sT, tid);
+      } else {
+        for (int e = tid - C; e < C * DK; e += THREADS - C) {
+          const int i = e / DK, d = e % DK;
+          const float g = sG[i * LDK + d];
+          const float eg = expf(g);
+          const float kv = sK[i * LDK + d];
+          sQ[i * LDK + d] *= eg;
+          sG[i * LDK + d] = kv * eg;
+          sK[i * LDK + d] = kv * expf(sgc[d] - g);
+        }
       }
     }
     __syncthreads();
     if (tid < DK) sgc[tid] = expf(sgc[tid]);          // e^{G_C}, for the carry
+    // Register tiles from here on: [C][DVS] results give thread rows
+    // 4 rg .. 4 rg + 3 and columns 4 cg .. 4 cg + 3 (rg = tid / 16, cg = tid % 16);
+    // the dk x DVS carry gives it rows DK/16 rg .. and the same columns.
+    const int rg = tid >> 4, r0 = 4 * rg, c0 = 4 * (tid & 15);
     // ---- X = V - (K o e^G) Sigma_0, in place of V
-    for (int e = tid; e < C * DVS; e += THREADS) {
-      const int i = e / DVS, c = e % DVS;
-      float acc = sV[i * LDC + c];
-      for (int d = 0; d < DK; ++d) acc = fmaf(-sG[i * LDK + d], sSig[d * LDC + c], acc);
-      sV[i * LDC + c] = acc;
+    {
+      float acc[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 x = lds4(sV + (r0 + i) * LDC + c0);
+        acc[i][0] = x.x; acc[i][1] = x.y; acc[i][2] = x.z; acc[i][3] = x.w;
+      }
+#pragma unroll 4
+      for (int d = 0; d < DK; ++d) {
+        const float4 b4 = lds4(sSig + d * LDC + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float a = sG[(r0 + i) * LDK + d];
+          acc[i][0] = fmaf(-a, b4.x, acc[i][0]);
+          acc[i][1] = fmaf(-a, b4.y, acc[i][1]);
+          acc[i][2] = fmaf(-a, b4.z, acc[i][2]);
+          acc[i][3] = fmaf(-a, b4.w, acc[i][3]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4*>(sV + (r0 + i) * LDC + c0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     }
     __syncthreads();
-    // ---- U = T diag(b) X
-    for (int e = tid; e < C * DVS; e += THREADS) {
-      const int i = e / DVS, c = e % DVS;
-      float acc = 0.f;
-      for (int j = 0; j <= i; ++j) acc = fmaf(sT[i * LDC + j] * sb[j], sV[j * LDC + c], acc);
-      sU[i * LDC + c] = acc;
+    // ---- U = T diag(b) X (T is lower triangular: j <= r0 + 3)
+    {
+      float acc[4][4] = {};
+#pragma unroll 4
+      for (int j = 0; j < r0 + 4; ++j) {
+        const float4 x = lds4(sV + j * LDC + c0);
+        const float bj = sb[j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float a = sT[(r0 + i) * LDC + j] * bj;
+          acc[i][0] = fmaf(a, x.x, acc[i][0]);
+          acc[i][1] = fmaf(a, x.y, acc[i][1]);
+          acc[i][2] = fmaf(a, x.z, acc[i][2]);
+          acc[i][3] = fmaf(a, x.w, acc[i][3]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4*>(sU + (r0 + i) * LDC + c0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     }
     __syncthreads();
     // ---- O = scale ((Q o e^G) Sigma_0 + P U), then the output gate and the
     // loop residual (as the precise path)
-    for (int e = tid; e < C * DVS; e += THREADS) {
-      const int i = e / DVS, c = e % DVS;
-      if (i >= valid) continue;
-      float qs = 0.f, pu = 0.f;
-      for (int d = 0; d < DK; ++d) qs = fmaf(sQ[i * LDK + d], sSig[d * LDC + c], qs);
-      for (int j = 0; j <= i; ++j) pu = fmaf(sP[i * LDC + j], sU[j * LDC + c], pu);
-      float y = p.scale * (qs + pu);
-      const size_t off = ((size_t)(tok0 + i) * H + h) * dv + col0 + c;
-      if (p.gate) y *= 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + i) * H + h]));
-      if (p.h_prev) {
-        const float hp = to_f32(static_cast<const T*>(p.h_prev)[off]);
-        y = fmaf(p.rho[(size_t)h * dv + col0 + c], hp, to_f32(from_f32<T>(y)));
+    {
+      float acc[4][4] = {};
+#pragma unroll 4
+      for (int d = 0; d < DK; ++d) {
+        const float4 b4 = lds4(sSig + d * LDC + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float a = sQ[(r0 + i) * LDK + d];
+          acc[i][0] = fmaf(a, b4.x, acc[i][0]);
+          acc[i][1] = fmaf(a, b4.y, acc[i][1]);
+          acc[i][2] = fmaf(a, b4.z, acc[i][2]);
+          acc[i][3] = fmaf(a, b4.w, acc[i][3]);
+        }
       }
-      o[off] = from_f32<T>(y);
+#pragma unroll 4
+      for (int j = 0; j < r0 + 4; ++j) {
+        const float4 u = lds4(sU + j * LDC + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float a = sP[(r0 + i) * LDC + j];
+          acc[i][0] = fmaf(a, u.x, acc[i][0]);
+          acc[i][1] = fmaf(a, u.y, acc[i][1]);
+          acc[i][2] = fmaf(a, u.z, acc[i][2]);
+          acc[i][3] = fmaf(a, u.w, acc[i][3]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = r0 + i;
+        if (r >= valid) continue;
+        const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + r) * H + h])) : 1.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = c0 + j;
+          float y = p.scale * acc[i][j];
+          const size_t off = ((size_t)(tok0 + r) * H + h) * dv + col0 + c;
+          if (p.gate) y *= og;
+          if (p.h_prev) {
+            const float hp = to_f32(static_cast<const T*>(p.h_prev)[off]);
+            y = fmaf(p.rho[(size_t)h * dv + col0 + c], hp, to_f32(from_f32<T>(y)));
+          }
+          o[off] = from_f32<T>(y);
+        }
+      }
     }
     __syncthreads();
     // ---- Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
-    for (int e = tid; e < DK * DVS; e += THREADS) {
-      const int d = e / DVS, c = e % DVS;
-      float acc = 0.f;
-      for (int i = 0; i < C; ++i) acc = fmaf(sK[i * LDK + d], sU[i * LDC + c], acc);
-      sSig[d * LDC + c] = fmaf(sgc[d], sSig[d * LDC + c], acc);
+    {
+      constexpr int TD = DK / 16;
+      const int d0 = TD * rg;
+      float acc[TD][4] = {};
+#pragma unroll 2
+      for (int i = 0; i < C; ++i) {
+        const float4 u = lds4(sU + i * LDC + c0);
+#pragma unroll
+        for (int q4 = 0; q4 < TD / 4; ++q4) {
+          const float4 a4 = lds4(sK + i * LDK + d0 + 4 * q4);
+          const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[4 * q4 + e][0] = fmaf(a[e], u.x, acc[4 * q4 + e][0]);
+            acc[4 * q4 + e][1] = fmaf(a[e], u.y, acc[4 * q4 + e][1]);
+            acc[4 * q4 + e][2] = fmaf(a[e], u.z, acc[4 * q4 + e][2]);
+            acc[4 * q4 + e][3] = fmaf(a[e], u.w, acc[4 * q4 + e][3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < TD; ++e) {
+        const int d = d0 + e;
+        float4 sg = lds4(sSig + d * LDC + c0);
+        const float g = sgc[d];
+        sg.x = fmaf(g, sg.x, acc[e][0]);
+        sg.y = fmaf(g, sg.y, acc[e][1]);
+        sg.z = fmaf(g, sg.z, acc[e][2]);
+        sg.w = fmaf(g, sg.w, acc[e][3]);
+        *reinterpret_cast<float4*>(sSig + d * LDC + c0) = sg;
+      }
     }
   }
   __syncthreads();

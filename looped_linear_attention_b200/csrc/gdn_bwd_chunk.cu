@@ -31,10 +31,14 @@
 // dlog a_m = sum_{i >= m} dg_i and grad_a_m = dlog a_m / a_m.
 //
 // Launches (fp32 on the CUDA cores, register-tiled products from shared memory):
-//   1. gdn_bwd_prep_kernel    one CTA per (chunk, head): T, W, U~, Qh, g
+//   1. gdn_bwd_prep_kernel    one CTA per (chunk, head): T, W, U~, Qh, g, and
+//                             the state passes' operands in their shared-memory
+//                             layouts (W^T, diag(r) K and its transpose)
 //   2. gdn_bwd_states_kernel  one CTA per (sequence, head, 32 columns of dv):
 //                             the chunk start states S_c, forward in order
 //   3. gdn_bwd_dstates_kernel the same grid: dE_c backwards, and grad_S0
+//      (both stream each chunk's operands with cp.async into single buffers,
+//      each load issued as soon as the product before it has read the buffer)
 //   4. gdn_bwd_grads_kernel   one CTA per (chunk, head): every gradient of the
 //                             chunk's tokens from S_c and dE_c
 // Chunks of sequence s take workspace slots t0_s / C + 2 s + c (consecutive
@@ -61,10 +65,13 @@ struct KParams {
   float scale;
   long long n_slots;                // chunk slots per head
   float *W, *Ut, *Qh, *G;           // per (slot, head): [C][dk], [C][dv], [C][dk], [C]
+  float *Wt, *Kh, *Kht;             // per (slot, head): W^T [dk][C], diag(r) K [C][dk], its transpose
   float *Sst, *dE;                  // per (slot, head): [dk][dv]
   unsigned* status;
 };
 
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ float ldx(const float* p, size_t i) { return __ldg(p + i); }
 __device__ __forceinline__ float ldx(const __nv_bfloat16* p, size_t i) { return __bfloat162float(p[i]); }
 
@@ -329,6 +336,22 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_prep_kernel(const KParams 
   const int rg = tid >> 4, cg = tid & 15;
   const int r0 = rg * 4;
   if (tid < C) p.G[wsi * C + tid] = V.g[tid];
+  {
+    // diag(r) K, row-major and transposed, for the state passes
+    float* gKh = p.Kh + wsi * C * DK;
+    float* gKht = p.Kht + wsi * C * DK;
+    for (int e = tid; e < C * DK / 4; e += THREADS) {
+      const int i = (e * 4) / DK, d = (e * 4) % DK;
+      float4 x = lds4(sK + i * LDK + d);
+      const float ri = V.r[i];
+      x.x *= ri; x.y *= ri; x.z *= ri; x.w *= ri;
+      *reinterpret_cast<float4*>(gKh + (size_t)i * DK + d) = x;
+    }
+    for (int e = tid; e < C * DK; e += THREADS) {
+      const int d = e / C, i = e % C;
+      gKht[(size_t)d * C + i] = V.r[i] * sK[i * LDK + d];
+    }
+  }
   __syncthreads();
   {
     // W = T diag(b gamma) K  [C][DK]
@@ -358,6 +381,13 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_prep_kernel(const KParams 
       }
   }
   __syncthreads();
+  {
+    float* gWt = p.Wt + wsi * C * DK;
+    for (int e = tid; e < C * DK; e += THREADS) {
+      const int d = e / C, i = e % C;
+      gWt[(size_t)d * C + i] = sW[i * LDK + d];
+    }
+  }
   {
     // Qh = scale diag(gamma) Q - P W  [C][DK]
     float acc[4][4 * NV];
@@ -417,10 +447,10 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_prep_kernel(const KParams 
 }
 
 // Shared-memory plans of the state passes, 2 CTAs per SM.  Row strides are
-// multiples of 4 (tiles of NS columns: NS + 2, even) so that every operand
-// read of the products is one float4 (4 rows of a transposed operand) or one
-// float2 (2 columns of a tile).
-constexpr int LDX = NS + 2;        // [rows][NS] tiles
+// multiples of 4 (16-byte rows for cp.async and float4 reads; tiles of NS
+// columns: NS + 4) so that every operand read of the products is one float4
+// (4 rows of a transposed operand) or one float2 (2 columns of a tile).
+constexpr int LDX = NS + 4;        // [rows][NS] tiles
 constexpr int LDCT = C + 4;        // [DK][C] transposed operands
 template <int DK>
 struct StatesPlan {
@@ -428,9 +458,9 @@ struct StatesPlan {
   static constexpr int S = 0;                    // [DK][LDX]  state slice
   static constexpr int WT = S + DK * LDX;        // [DK][LDCT] W^T
   static constexpr int KH = WT + DK * LDCT;      // [C][LDK]   diag(r) K
-  static constexpr int X = KH + C * LDK;         // [C][LDX]
-  static constexpr int VEC = X + C * LDX;        // g, r
-  static constexpr int FLOATS = VEC + 2 * C;
+  static constexpr int X = KH + C * LDK;         // 2 x [C][LDX]: U~ of a chunk, then X, in place
+  static constexpr int G = X + 2 * C * LDX;      // [C]
+  static constexpr int FLOATS = G + C;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 template <int DK>
@@ -442,8 +472,8 @@ struct DStatesPlan {
   static constexpr int W = KT + KT_FLOATS;       // [C][LDK]
   static constexpr int Y = W + C * LDK;          // [C][LDX]
   static constexpr int DO = Y + C * LDX;         // [C][LDX]
-  static constexpr int VEC = DO + C * LDX;       // g, r
-  static constexpr int FLOATS = VEC + 2 * C;
+  static constexpr int G = DO + C * LDX;         // [C]
+  static constexpr int FLOATS = G + C;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 
@@ -472,6 +502,24 @@ __device__ __forceinline__ void gemm_v(float (&acc)[TM][2], const float* A, cons
   }
 }
 
+// Asynchronous 16-byte copies global -> shared (per thread, in commit groups).
+__device__ __forceinline__ void cp_async16(float* smem, const float* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// rows x cols fp32 (cols a multiple of 4) from global (row stride gld) into
+// shared memory (row stride sld), 16 bytes per copy.
+__device__ __forceinline__ void cp_rows(float* dst, int sld, const float* src, size_t gld, int rows, int cols,
+                                        int tid) {
+  const int q = cols / 4;
+  for (int e = tid; e < rows * q; e += THREADS) {
+    const int i = e / q, c = (e % q) * 4;
+    cp_async16(dst + i * sld + c, src + (size_t)i * gld + c);
+  }
+}
+
 // Chain (sequence, head) and column slice of a state-pass block.
 __device__ __forceinline__ void state_block(const KParams& p, int& s, int& h, int& col0) {
   const int n_cs = p.dv / NS;
@@ -481,41 +529,10 @@ __device__ __forceinline__ void state_block(const KParams& p, int& s, int& h, in
   h = chain % p.H;
 }
 
-// g and r = e^{g_C - g} of a chunk (two barriers inside; every thread calls it).
-__device__ __forceinline__ void state_gates(const KParams& p, size_t wsi, float* sg, float* sr, int tid) {
-  if (tid < C) sg[tid] = p.G[wsi * C + tid];
-  __syncthreads();
-  if (tid < C) sr[tid] = expf(sg[C - 1] - sg[tid]);
-  __syncthreads();
-}
-
-// dst[d * LDCT + i] = src(i, d) for a row-major [C][DK] source (rows >= n
-// zero): 4 rows per thread, read along d (coalesced), one float4 store.
-template <int DK, class F>
-__device__ __forceinline__ void store_transposed(float* dst, int n, F src, int tid) {
-  for (int e = tid; e < DK * (C / 4); e += THREADS) {
-    const int d = e % DK, i4 = (e / DK) * 4;
-    float4 x;
-    x.x = (i4 < n) ? src(i4, d) : 0.f;
-    x.y = (i4 + 1 < n) ? src(i4 + 1, d) : 0.f;
-    x.z = (i4 + 2 < n) ? src(i4 + 2, d) : 0.f;
-    x.w = (i4 + 3 < n) ? src(i4 + 3, d) : 0.f;
-    *reinterpret_cast<float4*>(dst + d * LDCT + i4) = x;
-  }
-}
-// A [C][DK] fp32 workspace array into shared memory rows of stride LDK (float4).
-template <int DK>
-__device__ __forceinline__ void load_ws_rows(float* dst, const float* src, int tid) {
-  constexpr int LDK = DK + 4;
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-  for (int e = tid; e < C * DK / 4; e += THREADS) {
-    const int i = (e * 4) / DK, d = (e * 4) % DK;
-    *reinterpret_cast<float4*>(dst + i * LDK + d) = __ldg(s4 + e);
-  }
-}
-
 // 2. Chunk start states, forward: S_c[:, J] into the workspace, then
-// S <- gamma_C S + (diag(r) K)^T (U~[:, J] - W S).
+// S <- gamma_C S + (diag(r) K)^T (U~[:, J] - W S).  Loads per chunk: group A
+// (g, W^T, U~ slice) issued once the previous chunk's first product has read
+// W^T, group B (diag(r) K) once its second product has read it.
 template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_states_kernel(const KParams p) {
   extern __shared__ __align__(16) float smf[];
@@ -527,8 +544,7 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_states_kernel(const KParam
   state_block(p, s, h, col0);
   int t0, t1;
   seq_range(p, s, t0, t1, tid == 0 && col0 == 0 && h == 0);
-  float *sS = smf + PL::S, *sWt = smf + PL::WT, *sKh = smf + PL::KH, *sX = smf + PL::X;
-  float *sg = smf + PL::VEC, *sr = smf + PL::VEC + C;
+  float *sS = smf + PL::S, *sWt = smf + PL::WT, *sKh = smf + PL::KH, *sg = smf + PL::G;
   const size_t sd = (size_t)DK * p.dv;
   const size_t sb0 = ((size_t)s * p.H + h) * sd;
   for (int e = tid; e < DK * NS; e += THREADS) {
@@ -537,31 +553,33 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_states_kernel(const KParam
   }
   const int n_chunks = (t1 - t0 + C - 1) / C;
   const long long base = slot_base(s, t0);
-  const T* k = static_cast<const T*>(p.k);
+  auto wsi_of = [&](int ci) { return (size_t)(base + ci) * p.H + h; };
+  auto issue_a = [&](int ci) {
+    const size_t w = wsi_of(ci);
+    if (tid < C / 4) cp_async16(sg + 4 * tid, p.G + w * C + 4 * tid);
+    cp_rows(sWt, LDCT, p.Wt + w * C * DK, C, DK, C, tid);
+    cp_rows(smf + PL::X + (ci & 1) * C * LDX, LDX, p.Ut + w * C * p.dv + col0, p.dv, C, NS, tid);
+    cp_async_commit();
+  };
+  auto issue_b = [&](int ci) {
+    cp_rows(sKh, LDK, p.Kh + wsi_of(ci) * C * DK, DK, C, DK, tid);
+    cp_async_commit();
+  };
+  if (n_chunks > 0) {
+    issue_a(0);
+    issue_b(0);
+  }
   const int rg = tid >> 4, c0 = (tid & 15) * 2;
   for (int ci = 0; ci < n_chunks; ++ci) {
-    const int tc0 = t0 + ci * C, n = min(C, t1 - tc0);
-    const size_t wsi = (size_t)(base + ci) * p.H + h;
+    float* sX = smf + PL::X + (ci & 1) * C * LDX;
+    cp_async_wait<1>();                            // group A of this chunk (B may still fly)
     __syncthreads();
-    float* gS = p.Sst + wsi * sd;
+    float* gS = p.Sst + wsi_of(ci) * sd;
     for (int e = tid; e < DK * NS; e += THREADS) {
       const int d = e / NS, c = e % NS;
       gS[(size_t)d * p.dv + col0 + c] = sS[d * LDX + c];
     }
-    state_gates(p, wsi, sg, sr, tid);
-    const float* gW = p.W + wsi * C * DK;
-    store_transposed<DK>(sWt, C, [&](int i, int d) { return __ldg(gW + (size_t)i * DK + d); }, tid);
-    for (int e = tid; e < C * DK; e += THREADS) {
-      const int i = e / DK, d = e % DK;
-      sKh[i * LDK + d] = (i < n) ? sr[i] * ldx(k, ((size_t)(tc0 + i) * p.H + h) * DK + d) : 0.f;
-    }
-    const float* gU = p.Ut + wsi * C * p.dv + col0;
-    for (int e = tid; e < C * NS / 2; e += THREADS) {
-      const int i = (e * 2) / NS, c = (e * 2) % NS;
-      *reinterpret_cast<float2*>(sX + i * LDX + c) =
-          __ldg(reinterpret_cast<const float2*>(gU + (size_t)i * p.dv + c));
-    }
-    __syncthreads();
+    const float gC = expf(sg[C - 1]);
     {
       // X = U~ - W S  [C][NS]: rows 4 rg .. +3, columns c0, c0 + 1
       float acc[4][2];
@@ -572,39 +590,51 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_states_kernel(const KParam
 #pragma unroll
         for (int j = 0; j < 2; ++j) sX[(rg * 4 + i) * LDX + c0 + j] -= acc[i][j];
     }
+    __syncthreads();                               // W^T and g are free; X complete
+    if (ci + 1 < n_chunks) {
+      issue_a(ci + 1);
+      cp_async_wait<1>();                          // group B of this chunk
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
     {
       // S = gamma_C S + Kh^T X  [DK][NS]: rows TM rg .. +TM-1
       float acc[TM][2];
       zero(acc);
       gemm_v<TM, C, LDK, LDX>(acc, sKh + rg * TM, sX + c0);
-      const float gC = expf(sg[C - 1]);
 #pragma unroll
       for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < 2; ++j)
           sS[(rg * TM + i) * LDX + c0 + j] = fmaf(gC, sS[(rg * TM + i) * LDX + c0 + j], acc[i][j]);
     }
+    __syncthreads();                               // diag(r) K is free
+    if (ci + 1 < n_chunks) issue_b(ci + 1);
   }
+  cp_async_wait<0>();
 }
 
 // 3. State gradients, backward: dE_c[:, J] (the gradient at the end of chunk
 // c) into the workspace, then dE <- gamma_C dE - W^T (Kh dE) + Qh^T dO[:, J];
 // what remains after chunk 0 is grad_S0.  Kh^T and then Qh share one buffer.
+// Loads per chunk c: Qh once Kh dE has read Kh^T; W and g of chunk c - 1 once
+// W^T Y has read W; Kh^T of chunk c - 1 once Qh^T dO has read Qh; dO of chunk
+// c - 1 through registers, requested at the top of chunk c.
 template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_dstates_kernel(const KParams p) {
   extern __shared__ __align__(16) float smf[];
   using PL = DStatesPlan<DK>;
   constexpr int LDK = PL::LDK;
   constexpr int TM = DK / 16;
+  constexpr int DO_PER_THREAD = C * NS / THREADS;
   const int tid = threadIdx.x;
   int s, h, col0;
   state_block(p, s, h, col0);
   int t0, t1;
   seq_range(p, s, t0, t1, false);
   float *sE = smf + PL::E, *sKt = smf + PL::KT, *sW = smf + PL::W, *sY = smf + PL::Y, *sdO = smf + PL::DO;
-  float* sQh = sKt;
-  float *sg = smf + PL::VEC, *sr = smf + PL::VEC + C;
+  float *sQh = sKt, *sg = smf + PL::G;
   const size_t sd = (size_t)DK * p.dv;
   const size_t sb0 = ((size_t)s * p.H + h) * sd;
   for (int e = tid; e < DK * NS; e += THREADS) {
@@ -613,28 +643,53 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_dstates_kernel(const KPara
   }
   const int n_chunks = (t1 - t0 + C - 1) / C;
   const long long base = slot_base(s, t0);
-  const T* k = static_cast<const T*>(p.k);
   const T* go = static_cast<const T*>(p.go);
+  auto wsi_of = [&](int ci) { return (size_t)(base + ci) * p.H + h; };
+  auto issue_w = [&](int ci) {                     // W and g of chunk ci
+    const size_t w = wsi_of(ci);
+    if (tid < C / 4) cp_async16(sg + 4 * tid, p.G + w * C + 4 * tid);
+    cp_rows(sW, LDK, p.W + w * C * DK, DK, C, DK, tid);
+    cp_async_commit();
+  };
+  auto issue_kt = [&](int ci) {                    // (diag(r) K)^T of chunk ci
+    cp_rows(sKt, LDCT, p.Kht + wsi_of(ci) * C * DK, C, DK, C, tid);
+    cp_async_commit();
+  };
+  T dor[DO_PER_THREAD];                            // dO of the next chunk, in flight (raw)
+  bool dov[DO_PER_THREAD];
+  auto load_do = [&](int ci) {
+    const int tc0 = t0 + ci * C, n = min(C, t1 - tc0);
+#pragma unroll
+    for (int u = 0; u < DO_PER_THREAD; ++u) {
+      const int e = tid + THREADS * u, i = e / NS, c = e % NS;
+      dov[u] = i < n;
+      if (dov[u]) dor[u] = go[((size_t)(tc0 + i) * p.H + h) * p.dv + col0 + c];
+    }
+  };
+  auto store_do = [&]() {
+#pragma unroll
+    for (int u = 0; u < DO_PER_THREAD; ++u) {
+      const int e = tid + THREADS * u, i = e / NS, c = e % NS;
+      sdO[i * LDX + c] = dov[u] ? to_float(dor[u]) : 0.f;
+    }
+  };
+  if (n_chunks > 0) {
+    issue_w(n_chunks - 1);
+    issue_kt(n_chunks - 1);
+    load_do(n_chunks - 1);
+    store_do();
+  }
   const int rg = tid >> 4, c0 = (tid & 15) * 2;
   for (int ci = n_chunks - 1; ci >= 0; --ci) {
-    const int tc0 = t0 + ci * C, n = min(C, t1 - tc0);
-    const size_t wsi = (size_t)(base + ci) * p.H + h;
+    cp_async_wait<0>();                            // W, g and Kh^T of this chunk
     __syncthreads();
-    float* gE = p.dE + wsi * sd;
+    float* gE = p.dE + wsi_of(ci) * sd;
     for (int e = tid; e < DK * NS; e += THREADS) {
       const int d = e / NS, c = e % NS;
       gE[(size_t)d * p.dv + col0 + c] = sE[d * LDX + c];
     }
-    state_gates(p, wsi, sg, sr, tid);
-    store_transposed<DK>(sKt, n, [&](int i, int d) {
-      return sr[i] * ldx(k, ((size_t)(tc0 + i) * p.H + h) * DK + d);
-    }, tid);
-    load_ws_rows<DK>(sW, p.W + wsi * C * DK, tid);
-    for (int e = tid; e < C * NS; e += THREADS) {
-      const int i = e / NS, c = e % NS;
-      sdO[i * LDX + c] = (i < n) ? ldx(go, ((size_t)(tc0 + i) * p.H + h) * p.dv + col0 + c) : 0.f;
-    }
-    __syncthreads();
+    if (ci > 0) load_do(ci - 1);                   // registers; stored after this chunk's dO is read
+    const float gC = expf(sg[C - 1]);
     {
       // Y = Kh dE  [C][NS]
       float acc[4][2];
@@ -645,19 +700,25 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_dstates_kernel(const KPara
 #pragma unroll
         for (int j = 0; j < 2; ++j) sY[(rg * 4 + i) * LDX + c0 + j] = acc[i][j];
     }
-    __syncthreads();
-    // Qh replaces Kh^T (its loads overlap the W^T Y product)
-    load_ws_rows<DK>(sQh, p.Qh + wsi * C * DK, tid);
+    __syncthreads();                               // Kh^T is free; Y complete
+    cp_rows(sQh, LDK, p.Qh + wsi_of(ci) * C * DK, DK, C, DK, tid);
+    cp_async_commit();
     float accW[TM][2];
     zero(accW);
     gemm_v<TM, C, LDK, LDX>(accW, sW + rg * TM, sY + c0);
+    __syncthreads();                               // W and g are free
+    if (ci > 0) {
+      issue_w(ci - 1);
+      cp_async_wait<1>();                          // Qh of this chunk
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
     {
       // dE = gamma_C dE - W^T Y + Qh^T dO  [DK][NS]
       float accQ[TM][2];
       zero(accQ);
       gemm_v<TM, C, LDK, LDX>(accQ, sQh + rg * TM, sdO + c0);
-      const float gC = expf(sg[C - 1]);
 #pragma unroll
       for (int i = 0; i < TM; ++i)
 #pragma unroll
@@ -665,7 +726,13 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_dstates_kernel(const KPara
           sE[(rg * TM + i) * LDX + c0 + j] =
               fmaf(gC, sE[(rg * TM + i) * LDX + c0 + j], accQ[i][j] - accW[i][j]);
     }
+    __syncthreads();                               // Qh and dO are free
+    if (ci > 0) {
+      issue_kt(ci - 1);
+      store_do();
+    }
   }
+  cp_async_wait<0>();
   __syncthreads();
   if (p.gS0)
     for (int e = tid; e < DK * NS; e += THREADS) {
@@ -1096,12 +1163,13 @@ static gdn_status launch_all(const KParams& kp, const gdn_bwd_params* p, cudaStr
 
 }  // namespace cbwd
 
-// Workspace of the chunkwise path: W, Qh [slots][H][C][dk], U~ [slots][H][C][dv],
-// g [slots][H][C], start states and end-state gradients [slots][H][dk][dv].
+// Workspace of the chunkwise path: W, Qh, W^T, diag(r) K and its transpose
+// [slots][H][C x dk], U~ [slots][H][C][dv], g [slots][H][C], start states and
+// end-state gradients [slots][H][dk][dv].
 size_t bwd_chunk_workspace(const gdn_bwd_params* p) {
   const size_t sh = (size_t)cbwd::n_slots(p) * p->H;
   const size_t C = cbwd::C;
-  return cbwd::align256(sh * C * p->dk * 4) * 2 + cbwd::align256(sh * C * p->dv * 4) +
+  return cbwd::align256(sh * C * p->dk * 4) * 5 + cbwd::align256(sh * C * p->dv * 4) +
          cbwd::align256(sh * C * 4) + cbwd::align256(sh * (size_t)p->dk * p->dv * 4) * 2;
 }
 
@@ -1137,6 +1205,12 @@ gdn_status launch_bwd_chunk(const gdn_bwd_params* p, unsigned* status, void* ws,
   kp.W = reinterpret_cast<float*>(w);
   w += cbwd::align256(sh * C * p->dk * 4);
   kp.Qh = reinterpret_cast<float*>(w);
+  w += cbwd::align256(sh * C * p->dk * 4);
+  kp.Wt = reinterpret_cast<float*>(w);
+  w += cbwd::align256(sh * C * p->dk * 4);
+  kp.Kh = reinterpret_cast<float*>(w);
+  w += cbwd::align256(sh * C * p->dk * 4);
+  kp.Kht = reinterpret_cast<float*>(w);
   w += cbwd::align256(sh * C * p->dk * 4);
   kp.Ut = reinterpret_cast<float*>(w);
   w += cbwd::align256(sh * C * p->dv * 4);

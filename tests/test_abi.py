@@ -311,8 +311,9 @@ def _bwd_params(**kw):
 def test_backward_validation_and_workspace(lib):
     """gdn_chunk_bwd: host-side rejections before any launch, and the
     workspaces.  Both paths use one chunk slot per 64 tokens (plus two per
-    sequence and one) per head.  Chunkwise (default): W, Qh [C][dk], U~ [C][dv],
-    g [C], start state and end-state gradient [dk][dv] per slot.  Token by
+    sequence and one) per head.  Chunkwise (default): W, Qh, W^T, diag(r) K and
+    its transpose (C x dk each), U~ [C][dv], g [C], start state and end-state
+    gradient [dk][dv] per slot.  Token by
     token (GDN_PRECISE): one checkpoint per slot, one chunk of 65 states and
     the running gradient per chain."""
     p = _bwd_params()
@@ -321,7 +322,7 @@ def test_backward_validation_and_workspace(lib):
     align = lambda x: (x + 255) // 256 * 256
     slots = 200 // 64 + 2 * 2 + 1
     sh = slots * 2
-    assert need == (2 * align(sh * 64 * 128 * 4) + align(sh * 64 * 128 * 4) + align(sh * 64 * 4)
+    assert need == (5 * align(sh * 64 * 128 * 4) + align(sh * 64 * 128 * 4) + align(sh * 64 * 4)
                     + 2 * align(sh * sd))
     tok = _bwd_params(flags=B.GDN_PRECISE)
     assert lib.gdn_chunk_bwd_workspace(ctypes.byref(tok)) == align(2 * slots * sd) + align(4 * 65 * sd) + align(4 * sd)

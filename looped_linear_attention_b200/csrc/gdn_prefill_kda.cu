@@ -25,7 +25,7 @@
 // one per (i, j, c).
 // Otherwise (a channel that decays hard or resets) the decay of each (i, j, c)
 // term is its own exponential, so every exponent is <= 0.  One CTA of 256
-// threads per (sequence, head, 64-column dv slice); the output epilogue
+// threads per (sequence, head, 32-column dv slice); the output epilogue
 // (head-wise gate, loop residual) is the precise path's.
 #include "common.cuh"
 
@@ -33,12 +33,28 @@ namespace gdn {
 namespace kda {
 
 constexpr int C = 64;
-constexpr int DVS = 64;
+constexpr int DVS = 32;           // dv columns per CTA (more CTAs for few chains)
 constexpr int THREADS = 256;
 constexpr int LDC = C + 4;        // C x C and [rows][DVS] tiles: float4 rows
 constexpr float kFactorRange = 80.f;   // largest per-channel log-decay range of a factored chunk
 
 __device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+// TN consecutive floats from / to shared memory (one float2 or float4 access)
+template <int TN>
+__device__ __forceinline__ void ldv(const float* p, float (&v)[TN]) {
+  if constexpr (TN == 4) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x; v[1] = x.y;
+  }
+}
+template <int TN>
+__device__ __forceinline__ void stv(float* p, const float (&v)[TN]) {
+  if constexpr (TN == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  else *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+}
 __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
   return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
 }
@@ -68,7 +84,7 @@ struct Plan {
   static constexpr int K = 0;                      // [C][LDK]  K, then K o e^{G_C - G}
   static constexpr int Q = K + C * LDK;            // [C][LDK]  Q, then Q o e^G
   static constexpr int G = Q + C * LDK;            // [C][LDK]  G, then K o e^G
-  static constexpr int SIG = G + C * LDK;          // [DK][LDC] (64 used)
+  static constexpr int SIG = G + C * LDK;          // [DK][LDC] (DVS columns used)
   static constexpr int V = SIG + DK * LDC;         // [C][LDC]  V, then V - (K o e^G) Sigma_0
   static constexpr int A = V + C * LDC;            // [C][LDC]
   static constexpr int T = A + C * LDC;            // [C][LDC]
@@ -314,81 +330,74 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
     __syncthreads();
     if (tid < DK) sgc[tid] = expf(sgc[tid]);          // e^{G_C}, for the carry
     // Register tiles from here on: [C][DVS] results give thread rows
-    // 4 rg .. 4 rg + 3 and columns 4 cg .. 4 cg + 3 (rg = tid / 16, cg = tid % 16);
-    // the dk x DVS carry gives it rows DK/16 rg .. and the same columns.
-    const int rg = tid >> 4, r0 = 4 * rg, c0 = 4 * (tid & 15);
+    // 4 rg .. 4 rg + 3 and columns TN cg .. TN cg + TN - 1 (rg = tid / 16,
+    // cg = tid % 16, TN = DVS / 16); the dk x DVS carry gives it rows DK/16 rg ..
+    // and the same columns.
+    constexpr int TN = DVS / 16;
+    const int rg = tid >> 4, r0 = 4 * rg, c0 = TN * (tid & 15);
     // ---- X = V - (K o e^G) Sigma_0, in place of V
     {
-      float acc[4][4];
+      float acc[4][TN];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 x = lds4(sV + (r0 + i) * LDC + c0);
-        acc[i][0] = x.x; acc[i][1] = x.y; acc[i][2] = x.z; acc[i][3] = x.w;
-      }
+      for (int i = 0; i < 4; ++i) ldv<TN>(sV + (r0 + i) * LDC + c0, acc[i]);
 #pragma unroll 4
       for (int d = 0; d < DK; ++d) {
-        const float4 b4 = lds4(sSig + d * LDC + c0);
+        float b[TN];
+        ldv<TN>(sSig + d * LDC + c0, b);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float a = sG[(r0 + i) * LDK + d];
-          acc[i][0] = fmaf(-a, b4.x, acc[i][0]);
-          acc[i][1] = fmaf(-a, b4.y, acc[i][1]);
-          acc[i][2] = fmaf(-a, b4.z, acc[i][2]);
-          acc[i][3] = fmaf(-a, b4.w, acc[i][3]);
+#pragma unroll
+          for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(-a, b[j], acc[i][j]);
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4*>(sV + (r0 + i) * LDC + c0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      for (int i = 0; i < 4; ++i) stv<TN>(sV + (r0 + i) * LDC + c0, acc[i]);
     }
     __syncthreads();
     // ---- U = T diag(b) X (T is lower triangular: j <= r0 + 3)
     {
-      float acc[4][4] = {};
+      float acc[4][TN] = {};
 #pragma unroll 4
       for (int j = 0; j < r0 + 4; ++j) {
-        const float4 x = lds4(sV + j * LDC + c0);
+        float x[TN];
+        ldv<TN>(sV + j * LDC + c0, x);
         const float bj = sb[j];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float a = sT[(r0 + i) * LDC + j] * bj;
-          acc[i][0] = fmaf(a, x.x, acc[i][0]);
-          acc[i][1] = fmaf(a, x.y, acc[i][1]);
-          acc[i][2] = fmaf(a, x.z, acc[i][2]);
-          acc[i][3] = fmaf(a, x.w, acc[i][3]);
+#pragma unroll
+          for (int jj = 0; jj < TN; ++jj) acc[i][jj] = fmaf(a, x[jj], acc[i][jj]);
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4*>(sU + (r0 + i) * LDC + c0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      for (int i = 0; i < 4; ++i) stv<TN>(sU + (r0 + i) * LDC + c0, acc[i]);
     }
     __syncthreads();
     // ---- O = scale ((Q o e^G) Sigma_0 + P U), then the output gate and the
     // loop residual (as the precise path)
     {
-      float acc[4][4] = {};
+      float acc[4][TN] = {};
 #pragma unroll 4
       for (int d = 0; d < DK; ++d) {
-        const float4 b4 = lds4(sSig + d * LDC + c0);
+        float b[TN];
+        ldv<TN>(sSig + d * LDC + c0, b);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float a = sQ[(r0 + i) * LDK + d];
-          acc[i][0] = fmaf(a, b4.x, acc[i][0]);
-          acc[i][1] = fmaf(a, b4.y, acc[i][1]);
-          acc[i][2] = fmaf(a, b4.z, acc[i][2]);
-          acc[i][3] = fmaf(a, b4.w, acc[i][3]);
+#pragma unroll
+          for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a, b[j], acc[i][j]);
         }
       }
 #pragma unroll 4
       for (int j = 0; j < r0 + 4; ++j) {
-        const float4 u = lds4(sU + j * LDC + c0);
+        float u[TN];
+        ldv<TN>(sU + j * LDC + c0, u);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float a = sP[(r0 + i) * LDC + j];
-          acc[i][0] = fmaf(a, u.x, acc[i][0]);
-          acc[i][1] = fmaf(a, u.y, acc[i][1]);
-          acc[i][2] = fmaf(a, u.z, acc[i][2]);
-          acc[i][3] = fmaf(a, u.w, acc[i][3]);
+#pragma unroll
+          for (int jj = 0; jj < TN; ++jj) acc[i][jj] = fmaf(a, u[jj], acc[i][jj]);
         }
       }
 #pragma unroll
@@ -397,7 +406,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
         if (r >= valid) continue;
         const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + r) * H + h])) : 1.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < TN; ++j) {
           const int c = c0 + j;
           float y = p.scale * acc[i][j];
           const size_t off = ((size_t)(tok0 + r) * H + h) * dv + col0 + c;
@@ -415,33 +424,30 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
     {
       constexpr int TD = DK / 16;
       const int d0 = TD * rg;
-      float acc[TD][4] = {};
+      float acc[TD][TN] = {};
 #pragma unroll 2
       for (int i = 0; i < C; ++i) {
-        const float4 u = lds4(sU + i * LDC + c0);
+        float u[TN];
+        ldv<TN>(sU + i * LDC + c0, u);
 #pragma unroll
         for (int q4 = 0; q4 < TD / 4; ++q4) {
           const float4 a4 = lds4(sK + i * LDK + d0 + 4 * q4);
           const float a[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            acc[4 * q4 + e][0] = fmaf(a[e], u.x, acc[4 * q4 + e][0]);
-            acc[4 * q4 + e][1] = fmaf(a[e], u.y, acc[4 * q4 + e][1]);
-            acc[4 * q4 + e][2] = fmaf(a[e], u.z, acc[4 * q4 + e][2]);
-            acc[4 * q4 + e][3] = fmaf(a[e], u.w, acc[4 * q4 + e][3]);
-          }
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[4 * q4 + e][j] = fmaf(a[e], u[j], acc[4 * q4 + e][j]);
         }
       }
 #pragma unroll
       for (int e = 0; e < TD; ++e) {
         const int d = d0 + e;
-        float4 sg = lds4(sSig + d * LDC + c0);
+        float sg[TN];
+        ldv<TN>(sSig + d * LDC + c0, sg);
         const float g = sgc[d];
-        sg.x = fmaf(g, sg.x, acc[e][0]);
-        sg.y = fmaf(g, sg.y, acc[e][1]);
-        sg.z = fmaf(g, sg.z, acc[e][2]);
-        sg.w = fmaf(g, sg.w, acc[e][3]);
-        *reinterpret_cast<float4*>(sSig + d * LDC + c0) = sg;
+#pragma unroll
+        for (int j = 0; j < TN; ++j) sg[j] = fmaf(g, sg[j], acc[e][j]);
+        stv<TN>(sSig + d * LDC + c0, sg);
       }
     }
   }

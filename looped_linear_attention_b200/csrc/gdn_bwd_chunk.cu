@@ -51,7 +51,6 @@ namespace cbwd {
 constexpr int C = 64;
 constexpr int THREADS = 256;
 constexpr int NS = 32;            // dv columns per tile (grads) and per state-pass CTA
-constexpr int LDT = NS + 1;       // row stride of [rows][NS] tiles
 constexpr int LDC = C + 4;        // row stride of C x C tiles (a multiple of 4, = 4 mod 32)
 constexpr int LDN = NS + 4;       // row stride of [C][NS] tiles (the same two properties)
 constexpr float kMinGate = 1e-30f;   // a is clamped to this before its logarithm
@@ -115,23 +114,6 @@ __device__ bool slot_chunk(const KParams& p, long long slot, int& s, int& c, int
   return true;
 }
 
-// acc[i][j] += sum_k A(i, k) B(k, j) over k < K for a thread's TM x TN tile;
-// fa(i, k) and fb(k, j) read the operands.
-template <int TM, int TN, int K, class FA, class FB>
-__device__ __forceinline__ void gemm(float (&acc)[TM][TN], FA fa, FB fb) {
-#pragma unroll 4
-  for (int k = 0; k < K; ++k) {
-    float av[TM], bv[TN];
-#pragma unroll
-    for (int i = 0; i < TM; ++i) av[i] = fa(i, k);
-#pragma unroll
-    for (int j = 0; j < TN; ++j) bv[j] = fb(k, j);
-#pragma unroll
-    for (int i = 0; i < TM; ++i)
-#pragma unroll
-      for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-  }
-}
 template <int TM, int TN>
 __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
 #pragma unroll
@@ -179,17 +161,6 @@ __device__ __forceinline__ void chunk_gates(const KParams& p, int t0, int n, int
   }
   __syncthreads();
   if (tid < C) V.r[tid] = expf(V.g[C - 1] - V.g[tid]);
-}
-
-// Rows [0, n) of a [tokens][H][width] input into shared memory ([C][ld]
-// fp32, columns [c0, c0 + cols)), zeros below.
-template <typename T>
-__device__ __forceinline__ void load_rows(float* dst, int ld, const T* src, int t0, int n, int h, int H,
-                                          int width, int c0, int cols, int tid) {
-  for (int e = tid; e < C * cols; e += THREADS) {
-    const int i = e / cols, c = e % cols;
-    dst[i * ld + c] = (i < n) ? ldx(src, ((size_t)(t0 + i) * H + h) * width + c0 + c) : 0.f;
-  }
 }
 
 // T = (I + A)^{-1} with A_ij = b_i KK_ij (i > j): column `col` by forward

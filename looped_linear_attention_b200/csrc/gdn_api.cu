@@ -12,7 +12,8 @@ size_t prefill_segment_workspace(const gdn_fwd_params* p, const SegPlan& plan);
 gdn_status launch_prefill_tc(const gdn_fwd_params* p, unsigned* status, const SegPlan& plan, void* ws,
                              cudaStream_t stream);
 gdn_status launch_prefill_simt(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
-gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream);
+gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, void* ws, cudaStream_t stream);
+size_t prefill_kda_workspace(const gdn_fwd_params* p);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* a,
                           const float* b, float* S, void* o, const float* gate, const void* h_prev,
                           const float* rho, int N, int H, int dk, int dv, gdn_dtype dt, float scale,
@@ -194,7 +195,8 @@ const char* gdn_status_string(gdn_status s) {
 
 size_t gdn_chunk_fwd_workspace(const gdn_fwd_params* p) {
   if (validate_fwd(p) != GDN_OK) return (size_t)-1;
-  if (p->total_tokens == 0) return 0;
+  if (p->total_tokens == 0 || p->n_seq == 0) return 0;
+  if (p->flags & GDN_CHANNEL_GATE) return gdn::prefill_kda_workspace(p);
   return gdn::prefill_segment_workspace(p, gdn::plan_prefill_segments(p, sm_count()));
 }
 
@@ -210,6 +212,7 @@ gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params* p, int* n_segs, int* seg
   else if (plan.corrected) n = (plan.n_segs > 2 || p->S_T) ? 3 : 2;          // state pass, combine, correction
   else if (plan.n_segs > 2) n = 3;                                          // state pass, combine, output pass
   else if (plan.n_segs == 2 || plan.lpt) n = 2;
+  else if (p->flags & GDN_CHANNEL_GATE) n = 2;                               // the chunks' operands, the chains
   if (n_segs) *n_segs = plan.n_segs;
   if (seg0_tok) *seg0_tok = plan.seg0_tok;
   if (seg_tok) *seg_tok = plan.seg_tok;
@@ -241,10 +244,13 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_params* p, void* ws, size_t ws_bytes,
     if (!ws && ws_bytes == 0) plan = gdn::SegPlan{1, 0, 0, 0, 0};   // no workspace: one pass, natural order
     else if (!ws || ws_bytes < need) return GDN_ERR_WORKSPACE;
   }
+  // per-channel gate: a workspace selects the two launches, none the one-launch kernel
+  if ((p->flags & GDN_CHANNEL_GATE) && (ws ? ws_bytes < gdn::prefill_kda_workspace(p) : ws_bytes != 0))
+    return GDN_ERR_WORKSPACE;
   unsigned* st = status_ptr();
   if (!st) return GDN_ERR_CUDA;
   if (tc) return gdn::launch_prefill_tc(p, st, plan, ws, stream);
-  if (p->flags & GDN_CHANNEL_GATE) return gdn::launch_prefill_kda(p, st, stream);
+  if (p->flags & GDN_CHANNEL_GATE) return gdn::launch_prefill_kda(p, st, ws, stream);
   return gdn::launch_prefill_simt(p, st, stream);
 }
 

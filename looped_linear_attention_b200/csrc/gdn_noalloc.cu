@@ -40,7 +40,11 @@ extern "C" {
 gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_params* p, cudaStream_t stream) {
   const size_t need = gdn_chunk_fwd_workspace(p);
   if (need == (size_t)-1) return GDN_ERR_INVALID;
-  if (need > kNoallocScratchBytes) return GDN_ERR_WORKSPACE;
+  if (need > kNoallocScratchBytes) {
+    // the per-channel gate prefill has a one-launch kernel that needs none
+    if (p->flags & GDN_CHANNEL_GATE) return gdn_chunk_fwd(p, nullptr, 0, stream);
+    return GDN_ERR_WORKSPACE;
+  }
   if (need == 0) return gdn_chunk_fwd(p, nullptr, 0, stream);
   void* scratch = nullptr;
   const gdn_status st = scratch_address(&scratch);

@@ -45,15 +45,18 @@ __device__ __forceinline__ void ldv(const float* p, float (&v)[TN]) {
   if constexpr (TN == 4) {
     const float4 x = *reinterpret_cast<const float4*>(p);
     v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-  } else {
+  } else if constexpr (TN == 2) {
     const float2 x = *reinterpret_cast<const float2*>(p);
     v[0] = x.x; v[1] = x.y;
+  } else {
+    v[0] = *p;
   }
 }
 template <int TN>
 __device__ __forceinline__ void stv(float* p, const float (&v)[TN]) {
   if constexpr (TN == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  else *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  else if constexpr (TN == 2) *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  else *p = v[0];
 }
 __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
   return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
@@ -98,6 +101,15 @@ struct Plan {
 };
 static_assert(Plan<128>::BYTES <= 232448, "KDA prefill shared memory");
 
+// Workspace of the two-launch schedule, per (chunk slot, head): the chunk's
+// decayed operands, its two C x C matrices and its decay over the chunk.
+struct Ws {
+  float *KG, *QG, *Kh;   // [slots][H][C][dk]: K o e^G, Q o e^G, K o e^{G_C - G}
+  float *TB, *P;         // [slots][H][C][C]: T diag(b), P
+  float* EGC;            // [slots][H][dk]: e^{G_C}
+  long long n_slots;
+};
+
 struct Params {
   const void *q, *k, *v;
   const float *a, *b, *S0;   // a: [tokens][H][dk]
@@ -111,7 +123,190 @@ struct Params {
   int n_seq, seq_len, total_tokens, H, dv, n_slices;
   float scale;
   unsigned flags;
+  Ws ws;
 };
+
+// The chunk's operands of the KDA form (every thread of the CTA calls it):
+// K, Q (with the q/k norm rounded to the io dtype) and the per-channel log
+// decay prefix G of the chunk starting at tok0 (valid rows, zeros below), b,
+// A and P (factored when the chunk's decay range allows), T = (I + A)^{-1},
+// and the decayed operands written over K, Q and G: K o e^{G_C - G} over K,
+// Q o e^G over Q, K o e^G over G; sgc = e^{G_C}.  Ends with the block synced.
+template <int DK, typename T, typename PL>
+__device__ __forceinline__ void kda_chunk_operands(const Params& p, int tok0, int valid, int h, float* sm, int tid) {
+  constexpr int LDK = PL::LDK;
+  float* sK = sm + PL::K;
+  float* sQ = sm + PL::Q;
+  float* sG = sm + PL::G;
+  float* sA = sm + PL::A;
+  float* sT = sm + PL::T;
+  float* sP = sm + PL::P;
+  float* sb = sm + PL::B;
+  float* sgc = sm + PL::GC;
+  float* smid = sm + PL::MID;
+  float* sem = smid + DK;
+  float* sec = sem + DK;
+  const int H = p.H;
+  const T* q = static_cast<const T*>(p.q);
+  const T* k = static_cast<const T*>(p.k);
+  // ---- load the chunk; rows past the sequence end: zero keys, queries and
+  // values, log a = 0, b = 0
+  for (int e = tid; e < C * DK; e += THREADS) {
+    const int i = e / DK, d = e % DK;
+    float kv = 0.f, qv = 0.f, la = 0.f;
+    if (i < valid) {
+      const size_t off = ((size_t)(tok0 + i) * H + h) * DK + d;
+      kv = to_f32(k[off]);
+      qv = to_f32(q[off]);
+      la = logf(p.a[off]);
+    }
+    sK[i * LDK + d] = kv;
+    sQ[i * LDK + d] = qv;
+    sG[i * LDK + d] = la;
+  }
+  if (tid < C) sb[tid] = (tid < valid) ? p.b[(size_t)(tok0 + tid) * H + h] : 0.f;
+  __syncthreads();
+  // ---- G = prefix sums of log a down each channel (one thread per channel);
+  // the q/k L2 norm (threads 128 .. 255, one row each), rounded to the io dtype
+  if (tid < DK) {
+    float acc = 0.f;
+    for (int i = 0; i < C; ++i) {
+      acc += sG[i * LDK + tid];
+      sG[i * LDK + tid] = acc;
+    }
+  }
+  if ((p.flags & GDN_QK_L2NORM) && tid >= 128 && tid < 128 + 2 * C) {
+    const int r = tid - 128;
+    float* row = (r < C) ? sK + r * LDK : sQ + (r - C) * LDK;
+    float ss = 0.f;
+    for (int d = 0; d < DK; ++d) ss = fmaf(row[d], row[d], ss);
+    const float inv = 1.0f / sqrtf(ss + kQkNormEps);
+    for (int d = 0; d < DK; ++d) row[d] = to_f32(from_f32<T>(row[d] * inv));
+  }
+  __syncthreads();
+  // ---- G_C, the channel midpoints, and whether the chunk factors
+  if (tid < DK) {
+    const float g0 = sG[tid], gc = sG[(C - 1) * LDK + tid];
+    sgc[tid] = gc;                                  // G_C (rows past the end keep it)
+    smid[tid] = 0.5f * (g0 + gc);
+  }
+  const bool factored =
+      !__syncthreads_or(tid < DK && !(sG[tid] - sG[(C - 1) * LDK + tid] <= kFactorRange));
+  if (factored) {
+    // K^ = K o e^{m - G} over K, K~ = K o e^{G - m} over G, Q~ = Q o e^{G - m} over Q
+    for (int e = tid; e < C * DK; e += THREADS) {
+      const int i = e / DK, d = e % DK;
+      const float g = sG[i * LDK + d] - smid[d];
+      const float ex = expf(g), fx = expf(-g);
+      const float kv = sK[i * LDK + d];
+      sK[i * LDK + d] = kv * fx;
+      sG[i * LDK + d] = kv * ex;
+      sQ[i * LDK + d] *= ex;
+    }
+    if (tid < DK) {
+      sem[tid] = expf(smid[tid]);
+      sec[tid] = expf(sgc[tid] - smid[tid]);
+    }
+    __syncthreads();
+    {
+      // A = diag(b) K~ K^^T (strictly lower), P = Q~ K^^T (lower): thread rows
+      // r0 .. r0 + 3, columns cg + 16 j, four channels per read
+      const int r0 = (tid >> 4) * 4, cg = tid & 15;
+      float kk[4][4], qk[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) kk[i][j] = qk[i][j] = 0.f;
+#pragma unroll 2
+      for (int d = 0; d < DK; d += 4) {
+        float4 ak[4], aq[4], bk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          ak[i] = lds4(sG + (r0 + i) * LDK + d);
+          aq[i] = lds4(sQ + (r0 + i) * LDK + d);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bk[j] = lds4(sK + (cg + 16 * j) * LDK + d);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            kk[i][j] = dot4(ak[i], bk[j], kk[i][j]);
+            qk[i][j] = dot4(aq[i], bk[j], qk[i][j]);
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = r0 + i, cc = cg + 16 * j;
+          sA[r * LDC + cc] = (cc < r) ? sb[r] * kk[i][j] : 0.f;
+          sP[r * LDC + cc] = (cc <= r) ? qk[i][j] : 0.f;
+        }
+    }
+    __syncthreads();
+    // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
+    // operands from the factored ones: Q o e^G = Q~ e^m, K o e^G = K~ e^m,
+    // K o e^{G_C - G} = K^ e^{G_C - m}
+    if (tid < C) {
+      solve_column<C, LDC>(sA, sT, tid);
+    } else {
+      for (int e = tid - C; e < C * DK; e += THREADS - C) {
+        const int i = e / DK, d = e % DK;
+        sQ[i * LDK + d] *= sem[d];
+        sG[i * LDK + d] *= sem[d];
+        sK[i * LDK + d] *= sec[d];
+      }
+    }
+  } else {
+    // ---- A and P, each term with its own decay e^{G_ic - G_jc} (the fast
+    // exponential: a few ulp on arguments <= 0, far inside the fp32 bar)
+    // (only the lower triangle j <= i is enumerated; the upper one is zero)
+    for (int e = tid; e < C * (C + 1) / 2; e += THREADS) {
+      int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+      while (i * (i + 1) / 2 > e) --i;
+      while ((i + 1) * (i + 2) / 2 <= e) ++i;
+      const int j = e - i * (i + 1) / 2;
+      float kk = 0.f, qk = 0.f;
+#pragma unroll 8
+      for (int d = 0; d < DK; ++d) {
+        const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
+        const float kj = sK[j * LDK + d] * dec;
+        kk = fmaf(sK[i * LDK + d], kj, kk);
+        qk = fmaf(sQ[i * LDK + d], kj, qk);
+      }
+      sA[i * LDC + j] = (j < i) ? sb[i] * kk : 0.f;
+      sP[i * LDC + j] = qk;
+    }
+    for (int e = tid; e < C * (C - 1) / 2; e += THREADS) {   // the strict upper triangle
+      int j = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+      while (j * (j + 1) / 2 > e) --j;
+      while ((j + 1) * (j + 2) / 2 <= e) ++j;
+      const int i = e - j * (j + 1) / 2;            // i <= j, then shifted: column j + 1 > row i
+      sA[i * LDC + j + 1] = 0.f;
+      sP[i * LDC + j + 1] = 0.f;
+    }
+    __syncthreads();
+    // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
+    // operands: Q o e^G over Q, K o e^G over G, K o e^{G_C - G} over K
+    if (tid < C) {
+      solve_column<C, LDC>(sA, sT, tid);
+    } else {
+      for (int e = tid - C; e < C * DK; e += THREADS - C) {
+        const int i = e / DK, d = e % DK;
+        const float g = sG[i * LDK + d];
+        const float eg = expf(g);
+        const float kv = sK[i * LDK + d];
+        sQ[i * LDK + d] *= eg;
+        sG[i * LDK + d] = kv * eg;
+        sK[i * LDK + d] = kv * expf(sgc[d] - g);
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < DK) sgc[tid] = expf(sgc[tid]);          // e^{G_C}, for the carry
+  __syncthreads();
+}
 
 template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Params p) {
@@ -169,166 +364,11 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
   for (int tok0 = seq_start; tok0 < seq_end; tok0 += C) {
     const int valid = min(C, seq_end - tok0);
     __syncthreads();
-    // ---- load the chunk; rows past the sequence end: zero keys, queries and
-    // values, log a = 0, b = 0
-    for (int e = tid; e < C * DK; e += THREADS) {
-      const int i = e / DK, d = e % DK;
-      float kv = 0.f, qv = 0.f, la = 0.f;
-      if (i < valid) {
-        const size_t off = ((size_t)(tok0 + i) * H + h) * DK + d;
-        kv = to_f32(k[off]);
-        qv = to_f32(q[off]);
-        la = logf(p.a[off]);
-      }
-      sK[i * LDK + d] = kv;
-      sQ[i * LDK + d] = qv;
-      sG[i * LDK + d] = la;
-    }
     for (int e = tid; e < C * DVS; e += THREADS) {
       const int i = e / DVS, c = e % DVS;
       sV[i * LDC + c] = (i < valid) ? to_f32(v[((size_t)(tok0 + i) * H + h) * dv + col0 + c]) : 0.f;
     }
-    if (tid < C) sb[tid] = (tid < valid) ? p.b[(size_t)(tok0 + tid) * H + h] : 0.f;
-    __syncthreads();
-    // ---- G = prefix sums of log a down each channel (one thread per channel);
-    // the q/k L2 norm (threads 128 .. 255, one row each), rounded to the io dtype
-    if (tid < DK) {
-      float acc = 0.f;
-      for (int i = 0; i < C; ++i) {
-        acc += sG[i * LDK + tid];
-        sG[i * LDK + tid] = acc;
-      }
-    }
-    if ((p.flags & GDN_QK_L2NORM) && tid >= 128 && tid < 128 + 2 * C) {
-      const int r = tid - 128;
-      float* row = (r < C) ? sK + r * LDK : sQ + (r - C) * LDK;
-      float ss = 0.f;
-      for (int d = 0; d < DK; ++d) ss = fmaf(row[d], row[d], ss);
-      const float inv = 1.0f / sqrtf(ss + kQkNormEps);
-      for (int d = 0; d < DK; ++d) row[d] = to_f32(from_f32<T>(row[d] * inv));
-    }
-    __syncthreads();
-    // ---- G_C, the channel midpoints, and whether the chunk factors
-    if (tid < DK) {
-      const float g0 = sG[tid], gc = sG[(C - 1) * LDK + tid];
-      sgc[tid] = gc;                                  // G_C (rows past the end keep it)
-      smid[tid] = 0.5f * (g0 + gc);
-    }
-    const bool factored =
-        !__syncthreads_or(tid < DK && !(sG[tid] - sG[(C - 1) * LDK + tid] <= kFactorRange));
-    if (factored) {
-      // K^ = K o e^{m - G} over K, K~ = K o e^{G - m} over G, Q~ = Q o e^{G - m} over Q
-      for (int e = tid; e < C * DK; e += THREADS) {
-        const int i = e / DK, d = e % DK;
-        const float g = sG[i * LDK + d] - smid[d];
-        const float ex = expf(g), fx = expf(-g);
-        const float kv = sK[i * LDK + d];
-        sK[i * LDK + d] = kv * fx;
-        sG[i * LDK + d] = kv * ex;
-        sQ[i * LDK + d] *= ex;
-      }
-      if (tid < DK) {
-        sem[tid] = expf(smid[tid]);
-        sec[tid] = expf(sgc[tid] - smid[tid]);
-      }
-      __syncthreads();
-      {
-        // A = diag(b) K~ K^^T (strictly lower), P = Q~ K^^T (lower): thread rows
-        // r0 .. r0 + 3, columns cg + 16 j, four channels per read
-        const int r0 = (tid >> 4) * 4, cg = tid & 15;
-        float kk[4][4], qk[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) kk[i][j] = qk[i][j] = 0.f;
-#pragma unroll 2
-        for (int d = 0; d < DK; d += 4) {
-          float4 ak[4], aq[4], bk[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            ak[i] = lds4(sG + (r0 + i) * LDK + d);
-            aq[i] = lds4(sQ + (r0 + i) * LDK + d);
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) bk[j] = lds4(sK + (cg + 16 * j) * LDK + d);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              kk[i][j] = dot4(ak[i], bk[j], kk[i][j]);
-              qk[i][j] = dot4(aq[i], bk[j], qk[i][j]);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = r0 + i, cc = cg + 16 * j;
-            sA[r * LDC + cc] = (cc < r) ? sb[r] * kk[i][j] : 0.f;
-            sP[r * LDC + cc] = (cc <= r) ? qk[i][j] : 0.f;
-          }
-      }
-      __syncthreads();
-      // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
-      // operands from the factored ones: Q o e^G = Q~ e^m, K o e^G = K~ e^m,
-      // K o e^{G_C - G} = K^ e^{G_C - m}
-      if (tid < C) {
-        solve_column<C, LDC>(sA, sT, tid);
-      } else {
-        for (int e = tid - C; e < C * DK; e += THREADS - C) {
-          const int i = e / DK, d = e % DK;
-          sQ[i * LDK + d] *= sem[d];
-          sG[i * LDK + d] *= sem[d];
-          sK[i * LDK + d] *= sec[d];
-        }
-      }
-    } else {
-      // ---- A and P, each term with its own decay e^{G_ic - G_jc} (the fast
-      // exponential: a few ulp on arguments <= 0, far inside the fp32 bar)
-      // (only the lower triangle j <= i is enumerated; the upper one is zero)
-      for (int e = tid; e < C * (C + 1) / 2; e += THREADS) {
-        int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-        while (i * (i + 1) / 2 > e) --i;
-        while ((i + 1) * (i + 2) / 2 <= e) ++i;
-        const int j = e - i * (i + 1) / 2;
-        float kk = 0.f, qk = 0.f;
-#pragma unroll 8
-        for (int d = 0; d < DK; ++d) {
-          const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
-          const float kj = sK[j * LDK + d] * dec;
-          kk = fmaf(sK[i * LDK + d], kj, kk);
-          qk = fmaf(sQ[i * LDK + d], kj, qk);
-        }
-        sA[i * LDC + j] = (j < i) ? sb[i] * kk : 0.f;
-        sP[i * LDC + j] = qk;
-      }
-      for (int e = tid; e < C * (C - 1) / 2; e += THREADS) {   // the strict upper triangle
-        int j = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-        while (j * (j + 1) / 2 > e) --j;
-        while ((j + 1) * (j + 2) / 2 <= e) ++j;
-        const int i = e - j * (j + 1) / 2;            // i <= j, then shifted: column j + 1 > row i
-        sA[i * LDC + j + 1] = 0.f;
-        sP[i * LDC + j + 1] = 0.f;
-      }
-      __syncthreads();
-      // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
-      // operands: Q o e^G over Q, K o e^G over G, K o e^{G_C - G} over K
-      if (tid < C) {
-        solve_column<C, LDC>(sA, sT, tid);
-      } else {
-        for (int e = tid - C; e < C * DK; e += THREADS - C) {
-          const int i = e / DK, d = e % DK;
-          const float g = sG[i * LDK + d];
-          const float eg = expf(g);
-          const float kv = sK[i * LDK + d];
-          sQ[i * LDK + d] *= eg;
-          sG[i * LDK + d] = kv * eg;
-          sK[i * LDK + d] = kv * expf(sgc[d] - g);
-        }
-      }
-    }
-    __syncthreads();
-    if (tid < DK) sgc[tid] = expf(sgc[tid]);          // e^{G_C}, for the carry
+    kda_chunk_operands<DK, T, PL>(p, tok0, valid, h, sm, tid);
     // Register tiles from here on: [C][DVS] results give thread rows
     // 4 rg .. 4 rg + 3 and columns TN cg .. TN cg + TN - 1 (rg = tid / 16,
     // cg = tid % 16, TN = DVS / 16); the dk x DVS carry gives it rows DK/16 rg ..
@@ -460,6 +500,362 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
   }
 }
 
+// ---------------------------------------------------------------- two launches
+// With a workspace the chunk-parallel part of the form (the decayed operands,
+// A, P and T) runs once per (chunk, head) in a launch of its own, and the
+// chains then walk their chunks with only the state-dependent products:
+//     X = V - (K o e^G) Sigma_0,  U = T diag(b) X,
+//     O = scale ((Q o e^G) Sigma_0 + P U),
+//     Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U.
+// Chunk c of sequence s (first token t0_s) has workspace slot
+// floor(t0_s / C) + s + c: no two chunks share one, and every slot is below
+// floor(total / C) + n_seq.
+
+template <int DK>
+struct PrepPlan {
+  static constexpr int LDK = DK + 4;
+  static constexpr int K = 0;                      // [C][LDK]
+  static constexpr int Q = K + C * LDK;            // [C][LDK]
+  static constexpr int G = Q + C * LDK;            // [C][LDK]
+  static constexpr int A = G + C * LDK;            // [C][LDC]
+  static constexpr int T = A + C * LDC;            // [C][LDC]
+  static constexpr int P = T + C * LDC;            // [C][LDC]
+  static constexpr int B = P + C * LDC;            // C
+  static constexpr int GC = B + C;                 // DK
+  static constexpr int MID = GC + DK;              // 3 x DK
+  static constexpr int FLOATS = MID + 3 * DK + 4;
+  static constexpr size_t BYTES = (size_t)FLOATS * 4;
+};
+
+// A chain's state slice of NV columns, the chunk's operands (single buffers,
+// each refilled with cp.async as soon as its last reader is done) and the V
+// rows in the io dtype.
+template <int DK, int NV, typename T>
+struct ChainPlan {
+  static constexpr int LDK = DK + 4;
+  static constexpr int LDS = NV + 4;               // [rows][NV] fp32 tiles
+  static constexpr int VROW = (NV * (int)sizeof(T) + 16) / 4;   // floats per V row
+  static constexpr int KG = 0;                     // [C][LDK]  K o e^G
+  static constexpr int QG = KG + C * LDK;          // [C][LDK]  Q o e^G
+  static constexpr int KH = QG + C * LDK;          // [C][LDK]  K o e^{G_C - G}
+  static constexpr int TB = KH + C * LDK;          // [C][LDC]  T diag(b)
+  static constexpr int P = TB + C * LDC;           // [C][LDC]
+  static constexpr int SIG = P + C * LDC;          // [DK][LDS]
+  static constexpr int X = SIG + DK * LDS;         // [C][LDS]
+  static constexpr int U = X + C * LDS;            // [C][LDS]
+  static constexpr int EGC = U + C * LDS;          // DK
+  static constexpr int V = EGC + DK;               // [C][VROW]
+  static constexpr int FLOATS = V + C * VROW;
+  static constexpr size_t BYTES = (size_t)FLOATS * 4;
+};
+static_assert(ChainPlan<128, 32, float>::BYTES <= 232448, "KDA chain shared memory");
+
+__device__ __forceinline__ void seq_range(const Params& p, int s, int& t0, int& t1, bool report) {
+  if (p.cu_seqlens) {
+    t0 = __ldg(p.cu_seqlens + s);
+    t1 = __ldg(p.cu_seqlens + s + 1);
+  } else {
+    t0 = s * p.seq_len;
+    t1 = t0 + p.seq_len;
+  }
+  const int c0 = min(max(t0, 0), p.total_tokens);
+  const int c1 = min(max(t1, c0), p.total_tokens);
+  if (report && (c0 != t0 || c1 != t1)) record_status(p.status, GDN_ERR_INVALID);
+  t0 = c0;
+  t1 = c1;
+}
+__device__ __forceinline__ long long slot_base(int s, int t0) { return t0 / C + (long long)s; }
+
+// Slot -> (sequence, chunk, first token, rows): the last sequence whose first
+// slot is <= slot; false when the slot holds no chunk.
+__device__ bool slot_chunk(const Params& p, long long slot, int& tok0, int& valid) {
+  int lo = 0, hi = p.n_seq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    int a0, a1;
+    seq_range(p, mid, a0, a1, false);
+    if (slot_base(mid, a0) <= slot) lo = mid;
+    else hi = mid - 1;
+  }
+  int s0, s1;
+  seq_range(p, lo, s0, s1, false);
+  const long long c = slot - slot_base(lo, s0);
+  if (c < 0 || c >= (s1 - s0 + C - 1) / C) return false;
+  tok0 = s0 + (int)c * C;
+  valid = min(C, s1 - tok0);
+  return true;
+}
+
+__device__ __forceinline__ void cp_async16(float* smem, const float* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+// 16 bytes, or zeros when !take (nothing is read then)
+__device__ __forceinline__ void cp_async16_or_zero(float* smem, const void* gmem, bool take) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(take ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// rows x W contiguous floats into shared rows of stride LD
+template <int ROWS, int W, int LD>
+__device__ __forceinline__ void copy_rows(float* dst, const float* src, int tid) {
+  for (int e = tid; e < ROWS * W / 4; e += THREADS) {
+    const int i = e / (W / 4), c = 4 * (e % (W / 4));
+    cp_async16(dst + i * LD + c, src + (size_t)i * W + c);
+  }
+}
+
+// One CTA per (chunk slot, head): the chunk's operands into the workspace.
+template <int DK, typename T>
+__global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const Params p) {
+  using PL = PrepPlan<DK>;
+  constexpr int LDK = PL::LDK;
+  extern __shared__ __align__(16) float sm[];
+  const int tid = threadIdx.x;
+  const long long slot = blockIdx.x / p.H;
+  const int h = blockIdx.x % p.H;
+  int tok0, valid;
+  if (!slot_chunk(p, slot, tok0, valid)) return;
+  kda_chunk_operands<DK, T, PL>(p, tok0, valid, h, sm, tid);
+  const size_t w = (size_t)slot * p.H + h;
+  float4* kg = reinterpret_cast<float4*>(p.ws.KG + w * C * DK);
+  float4* qg = reinterpret_cast<float4*>(p.ws.QG + w * C * DK);
+  float4* kh = reinterpret_cast<float4*>(p.ws.Kh + w * C * DK);
+  for (int e = tid; e < C * DK / 4; e += THREADS) {
+    const int i = e / (DK / 4), d = 4 * (e % (DK / 4));
+    kg[e] = lds4(sm + PL::G + i * LDK + d);
+    qg[e] = lds4(sm + PL::Q + i * LDK + d);
+    kh[e] = lds4(sm + PL::K + i * LDK + d);
+  }
+  float4* tb = reinterpret_cast<float4*>(p.ws.TB + w * C * C);
+  float4* pp = reinterpret_cast<float4*>(p.ws.P + w * C * C);
+  for (int e = tid; e < C * C / 4; e += THREADS) {
+    const int i = e / (C / 4), j = 4 * (e % (C / 4));
+    float4 t = lds4(sm + PL::T + i * LDC + j);
+    const float4 b = lds4(sm + PL::B + j);
+    t.x *= b.x;
+    t.y *= b.y;
+    t.z *= b.z;
+    t.w *= b.w;
+    tb[e] = t;
+    pp[e] = lds4(sm + PL::P + i * LDC + j);
+  }
+  if (tid < DK / 4) reinterpret_cast<float4*>(p.ws.EGC + w * DK)[tid] = lds4(sm + PL::GC + 4 * tid);
+}
+
+// acc[j] += a . (b[0][j], b[1][j], b[2][j], b[3][j])
+template <int TN>
+__device__ __forceinline__ void fma4(float (&acc)[TN], float4 a, const float (&b)[4][TN]) {
+#pragma unroll
+  for (int j = 0; j < TN; ++j)
+    acc[j] = fmaf(a.w, b[3][j], fmaf(a.z, b[2][j], fmaf(a.y, b[1][j], fmaf(a.x, b[0][j], acc[j]))));
+}
+
+// acc[i][:] += sum over k < n (a multiple of 4) of A[r0 + i][k] B[k][c0 .. c0 + TN - 1]
+// (A rows of stride lda read four k at a time, B rows of stride ldb)
+template <int TN>
+__device__ __forceinline__ void rows_times(float (&acc)[4][TN], const float* A, int lda, const float* B, int ldb,
+                                           int n) {
+#pragma unroll 2
+  for (int k = 0; k < n; k += 4) {
+    float4 a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = lds4(A + i * lda + k);
+    float b[4][TN];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) ldv<TN>(B + (k + kk) * ldb, b[kk]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) fma4<TN>(acc[i], a[i], b);
+  }
+}
+
+// One CTA per (sequence, head, NV-column dv slice): the chain through its
+// chunks, operands from the workspace.
+template <int DK, int NV, typename T>
+__global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const Params p) {
+  using PL = ChainPlan<DK, NV, T>;
+  constexpr int LDK = PL::LDK, LDS = PL::LDS;
+  constexpr int TN = NV / 16;                      // columns per thread
+  extern __shared__ __align__(16) float sm[];
+  float* sKG = sm + PL::KG;
+  float* sQG = sm + PL::QG;
+  float* sKh = sm + PL::KH;
+  float* sTB = sm + PL::TB;
+  float* sP = sm + PL::P;
+  float* sSig = sm + PL::SIG;
+  float* sX = sm + PL::X;
+  float* sU = sm + PL::U;
+  float* sEGC = sm + PL::EGC;
+  float* sV = sm + PL::V;
+
+  const int tid = threadIdx.x;
+  const int n_slices = p.dv / NV;
+  const int slice = blockIdx.x % n_slices;
+  const int chain = blockIdx.x / n_slices;
+  const int h = chain % p.H;
+  const int seq = chain / p.H;
+  const int H = p.H, dv = p.dv;
+  int t0, t1;
+  seq_range(p, seq, t0, t1, tid == 0);
+  const int n_chunks = (t1 - t0 + C - 1) / C;
+  const long long slot0 = slot_base(seq, t0);
+  const int col0 = slice * NV;
+  const size_t sbase = ((size_t)seq * H + h) * DK * (size_t)dv + col0;
+  const T* v = static_cast<const T*>(p.v);
+  T* o = static_cast<T*>(p.o);
+
+  // Operand groups of chunk c, one cp.async group each (empty past the last
+  // chunk): X's (K o e^G, V rows), U's (T diag(b)), O's (Q o e^G, P), the
+  // carry's (K o e^{G_C - G}, e^{G_C}).
+  auto load_x = [&](int c) {
+    if (c < n_chunks) {
+      const size_t w = (size_t)(slot0 + c) * H + h;
+      copy_rows<C, DK, LDK>(sKG, p.ws.KG + w * C * DK, tid);
+      const int tok0 = t0 + c * C, valid = min(C, t1 - tok0);
+      constexpr int PIECES = NV * (int)sizeof(T) / 16;
+      for (int e = tid; e < C * PIECES; e += THREADS) {
+        const int i = e / PIECES, q = e % PIECES;
+        const T* src = v + ((size_t)(tok0 + min(i, valid - 1)) * H + h) * dv + col0;
+        cp_async16_or_zero(sV + i * PL::VROW + 4 * q, reinterpret_cast<const char*>(src) + 16 * q, i < valid);
+      }
+    }
+    cp_async_commit();
+  };
+  auto load_u = [&](int c) {
+    if (c < n_chunks) copy_rows<C, C, LDC>(sTB, p.ws.TB + (size_t)((slot0 + c) * H + h) * C * C, tid);
+    cp_async_commit();
+  };
+  auto load_o = [&](int c) {
+    if (c < n_chunks) {
+      const size_t w = (size_t)(slot0 + c) * H + h;
+      copy_rows<C, DK, LDK>(sQG, p.ws.QG + w * C * DK, tid);
+      copy_rows<C, C, LDC>(sP, p.ws.P + w * C * C, tid);
+    }
+    cp_async_commit();
+  };
+  auto load_s = [&](int c) {
+    if (c < n_chunks) {
+      const size_t w = (size_t)(slot0 + c) * H + h;
+      copy_rows<C, DK, LDK>(sKh, p.ws.Kh + w * C * DK, tid);
+      if (tid < DK / 4) cp_async16(sEGC + 4 * tid, p.ws.EGC + w * DK + 4 * tid);
+    }
+    cp_async_commit();
+  };
+
+  load_x(0);
+  load_u(0);
+  load_o(0);
+  for (int e = tid; e < DK * NV; e += THREADS) {
+    const int d = e / NV, c = e % NV;
+    sSig[d * LDS + c] = p.S0 ? p.S0[sbase + (size_t)d * dv + c] : 0.f;
+  }
+  // Register tiles: [C][NV] results give a thread rows r0 .. r0 + 3 and
+  // columns c0 .. c0 + TN - 1; the dk x NV carry gives it rows DK/16 rg ..
+  const int rg = tid >> 4, r0 = 4 * rg, c0 = TN * (tid & 15);
+  // Each phase waits for its own group (two later groups may still be in
+  // flight), syncs, then refills the buffers of the phase before it.
+  for (int c = 0; c < n_chunks; ++c) {
+    const int tok0 = t0 + c * C, valid = min(C, t1 - tok0);
+    // ---- X = V - (K o e^G) Sigma_0
+    cp_async_wait<2>();
+    __syncthreads();
+    load_s(c);
+    {
+      float acc[4][TN] = {};
+      rows_times<TN>(acc, sKG + r0 * LDK, LDK, sSig + c0, LDS, DK);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const T* vr = reinterpret_cast<const T*>(sV + (r0 + i) * PL::VROW) + c0;
+        float x[TN];
+#pragma unroll
+        for (int j = 0; j < TN; ++j) x[j] = to_f32(vr[j]) - acc[i][j];
+        stv<TN>(sX + (r0 + i) * LDS + c0, x);
+      }
+    }
+    // ---- U = T diag(b) X (lower triangular: columns < r0 + 4)
+    cp_async_wait<2>();
+    __syncthreads();
+    load_x(c + 1);
+    {
+      float acc[4][TN] = {};
+      rows_times<TN>(acc, sTB + r0 * LDC, LDC, sX + c0, LDS, r0 + 4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) stv<TN>(sU + (r0 + i) * LDS + c0, acc[i]);
+    }
+    // ---- O = scale ((Q o e^G) Sigma_0 + P U), then the output gate and the
+    // loop residual
+    cp_async_wait<2>();
+    __syncthreads();
+    load_u(c + 1);
+    {
+      float acc[4][TN] = {};
+      rows_times<TN>(acc, sQG + r0 * LDK, LDK, sSig + c0, LDS, DK);
+      rows_times<TN>(acc, sP + r0 * LDC, LDC, sU + c0, LDS, r0 + 4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = r0 + i;
+        if (r >= valid) continue;
+        const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + r) * H + h])) : 1.f;
+#pragma unroll
+        for (int j = 0; j < TN; ++j) {
+          const int cc = c0 + j;
+          float y = p.scale * acc[i][j];
+          const size_t off = ((size_t)(tok0 + r) * H + h) * dv + col0 + cc;
+          if (p.gate) y *= og;
+          if (p.h_prev) {
+            const float hp = to_f32(static_cast<const T*>(p.h_prev)[off]);
+            y = fmaf(p.rho[(size_t)h * dv + col0 + cc], hp, to_f32(from_f32<T>(y)));
+          }
+          o[off] = from_f32<T>(y);
+        }
+      }
+    }
+    // ---- Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
+    cp_async_wait<2>();
+    __syncthreads();
+    load_o(c + 1);
+    {
+      constexpr int TD = DK / 16;
+      const int d0 = TD * rg;
+      float acc[TD][TN] = {};
+#pragma unroll 2
+      for (int i = 0; i < C; ++i) {
+        float u[TN];
+        ldv<TN>(sU + i * LDS + c0, u);
+#pragma unroll
+        for (int q4 = 0; q4 < TD / 4; ++q4) {
+          const float4 a4 = lds4(sKh + i * LDK + d0 + 4 * q4);
+          const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[4 * q4 + e][j] = fmaf(a[e], u[j], acc[4 * q4 + e][j]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < TD; ++e) {
+        const int d = d0 + e;
+        float sg[TN];
+        ldv<TN>(sSig + d * LDS + c0, sg);
+        const float g = sEGC[d];
+#pragma unroll
+        for (int j = 0; j < TN; ++j) sg[j] = fmaf(g, sg[j], acc[e][j]);
+        stv<TN>(sSig + d * LDS + c0, sg);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  if (p.S_T) {
+    for (int e = tid; e < DK * NV; e += THREADS) {
+      const int d = e / NV, c = e % NV;
+      p.S_T[sbase + (size_t)d * dv + c] = sSig[d * LDS + c];
+    }
+  }
+}
+
 template <int DK, typename T>
 static cudaError_t launch_t(const Params& kp, long long blocks, cudaStream_t stream) {
   static std::atomic<bool> attr_set[kMaxDevices];
@@ -470,9 +866,39 @@ static cudaError_t launch_t(const Params& kp, long long blocks, cudaStream_t str
   return cudaGetLastError();
 }
 
+// dv columns per chain CTA of the two-launch schedule
+constexpr int kChainCols = 16;
+
+template <int DK, typename T>
+static cudaError_t launch_two(const Params& kp, long long chunk_blocks, long long chain_blocks,
+                              cudaStream_t stream) {
+  static std::atomic<bool> set_prep[kMaxDevices], set_chain[kMaxDevices];
+  constexpr size_t prep_bytes = PrepPlan<DK>::BYTES;
+  constexpr size_t chain_bytes = ChainPlan<DK, kChainCols, T>::BYTES;
+  cudaError_t e = smem_attr_once(set_prep, gdn_prefill_kda_prep_kernel<DK, T>, prep_bytes);
+  if (e == cudaSuccess) e = smem_attr_once(set_chain, gdn_prefill_kda_chain_kernel<DK, kChainCols, T>, chain_bytes);
+  if (e != cudaSuccess) return e;
+  gdn_prefill_kda_prep_kernel<DK, T><<<(unsigned)chunk_blocks, THREADS, prep_bytes, stream>>>(kp);
+  gdn_prefill_kda_chain_kernel<DK, kChainCols, T><<<(unsigned)chain_blocks, THREADS, chain_bytes, stream>>>(kp);
+  return cudaGetLastError();
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static long long n_slots(const gdn_fwd_params* p) { return (long long)p->total_tokens / C + p->n_seq + 1; }
+
 }  // namespace kda
 
-gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, cudaStream_t stream) {
+// Bytes of the two-launch schedule's workspace: K o e^G, Q o e^G and
+// K o e^{G_C - G} ([slots][H][C][dk] fp32 each), T diag(b) and P
+// ([slots][H][C][C]) and e^{G_C} ([slots][H][dk]).
+size_t prefill_kda_workspace(const gdn_fwd_params* p) {
+  const size_t sh = (size_t)kda::n_slots(p) * p->H;
+  const size_t dk = (size_t)p->dk, c = kda::C;
+  return 3 * kda::align256(sh * c * dk * 4) + 2 * kda::align256(sh * c * c * 4) + kda::align256(sh * dk * 4);
+}
+
+gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, void* ws, cudaStream_t stream) {
   kda::Params kp;
   kp.q = p->q;
   kp.k = p->k;
@@ -495,10 +921,40 @@ gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, cudaStr
   kp.n_slices = p->dv / kda::DVS;
   kp.scale = p->scale;
   kp.flags = p->flags;
-  const long long blocks = (long long)p->n_seq * p->H * kp.n_slices;
-  if (blocks <= 0) return GDN_OK;
-  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  kp.ws = kda::Ws{};
+  const long long chains = (long long)p->n_seq * p->H;
+  if (chains <= 0) return GDN_OK;
   cudaError_t e;
+  if (ws) {
+    // two launches: the chunks' operands, then the chains
+    const long long n_slots = kda::n_slots(p);
+    const size_t sh = (size_t)n_slots * p->H;
+    const size_t dk = (size_t)p->dk, c = kda::C;
+    char* w = static_cast<char*>(ws);
+    float** arrays[] = {&kp.ws.KG, &kp.ws.QG, &kp.ws.Kh};
+    for (float** a : arrays) {
+      *a = reinterpret_cast<float*>(w);
+      w += kda::align256(sh * c * dk * 4);
+    }
+    kp.ws.TB = reinterpret_cast<float*>(w);
+    w += kda::align256(sh * c * c * 4);
+    kp.ws.P = reinterpret_cast<float*>(w);
+    w += kda::align256(sh * c * c * 4);
+    kp.ws.EGC = reinterpret_cast<float*>(w);
+    kp.ws.n_slots = n_slots;
+    const long long chunk_blocks = n_slots * p->H;
+    const long long chain_blocks = chains * (p->dv / kda::kChainCols);
+    if (chunk_blocks > 0x7fffffffLL || chain_blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (p->io_dtype == GDN_BF16)
+      e = p->dk == 128 ? kda::launch_two<128, __nv_bfloat16>(kp, chunk_blocks, chain_blocks, stream)
+                       : kda::launch_two<64, __nv_bfloat16>(kp, chunk_blocks, chain_blocks, stream);
+    else
+      e = p->dk == 128 ? kda::launch_two<128, float>(kp, chunk_blocks, chain_blocks, stream)
+                       : kda::launch_two<64, float>(kp, chunk_blocks, chain_blocks, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  }
+  const long long blocks = chains * kp.n_slices;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   if (p->io_dtype == GDN_BF16)
     e = p->dk == 128 ? kda::launch_t<128, __nv_bfloat16>(kp, blocks, stream)
                      : kda::launch_t<64, __nv_bfloat16>(kp, blocks, stream);

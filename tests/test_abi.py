@@ -412,11 +412,23 @@ def test_decode_looped_rejects_bad_epilogue_on_host(lib, args):
 
 def test_channel_gate_flag_validation(lib):
     """GDN_CHANNEL_GATE (per-channel decay, a [tokens][H][dk]) is accepted by
-    prefill and decode; the output may not overlap any of a's dk-wide rows,
-    and the prefill takes no segmented schedule (no workspace)."""
+    prefill and decode; the output may not overlap any of a's dk-wide rows.
+    The prefill takes two launches with a workspace (one slot per chunk:
+    floor(total / 64) + n_seq + 1 slots per head) and one without."""
     p = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16, flags=B.GDN_CHANNEL_GATE)
-    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == 0
-    assert _schedule(lib, p) == (1, 0, 0, 1, 0)
+
+    def al(x):
+        return (x + 255) // 256 * 256
+
+    for dk in (128, 64):
+        p.dk = dk
+        sh = (4096 // 64 + 1 + 1) * 16
+        need = 3 * al(sh * 64 * dk * 4) + 2 * al(sh * 64 * 64 * 4) + al(sh * dk * 4)
+        assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == need
+    assert _schedule(lib, p) == (1, 0, 0, 2, 0)
+    # a workspace smaller than the need, or a size without one, is refused on the host
+    assert lib.gdn_chunk_fwd(ctypes.byref(p), ctypes.c_void_p(1 << 30), 256, None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_chunk_fwd(ctypes.byref(p), None, 256, None) == B.GDN_ERR_WORKSPACE
     # a of 64 tokens x 2 heads x 128 channels x 4 B = 64 KiB: an output 32 KiB past it overlaps
     bad = _params(a=1 << 20, o=(1 << 20) + (32 << 10), flags=B.GDN_CHANNEL_GATE)
     assert lib.gdn_chunk_fwd(ctypes.byref(bad), None, 0, None) == B.GDN_ERR_INVALID

@@ -113,3 +113,45 @@ def test_noalloc_rejects_shapes_beyond_the_scratch(lib):
                          base + (4 << 36), None, base + (5 << 36), None, None, n_seq, L,
                          n_seq * L, H, 128, dv, B.GDN_BF16, 1.0, 0)
     assert lib.gdn_chunk_fwd_noalloc(ctypes.byref(p), None) == B.GDN_ERR_WORKSPACE
+
+
+def _kda_case(label, L, H):
+    wl = dataclasses.replace(W.WORKLOADS["looped_prefill"], name=label, H=H, seq_len=L)
+    inp = W.prefill_inputs(wl, "cuda")
+    inp["a"], inp["b"] = W.channel_gates(L, H, 128, "cuda", label)
+    o = torch.full((L, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    S_T = torch.full((1, H, 128, 128), float("nan"), device="cuda")
+    p = B.gdn_fwd_params(inp["q"].data_ptr(), inp["k"].data_ptr(), inp["v"].data_ptr(),
+                         inp["a"].data_ptr(), inp["b"].data_ptr(), None, o.data_ptr(), S_T.data_ptr(),
+                         None, 1, L, L, H, 128, 128, B.GDN_BF16, 1.0,
+                         B.GDN_CHANNEL_GATE | B.GDN_QK_L2NORM)
+    return inp, p, o, S_T
+
+
+def test_noalloc_channel_gate_schedules(lib):
+    """The per-channel gate prefill: a call whose two-launch workspace fits
+    the array runs the two launches out of it (equal bit for bit to
+    gdn_chunk_fwd with a workspace); one whose workspace does not (4096
+    tokens x 16 heads) runs the one-launch kernel (equal bit for bit to
+    gdn_chunk_fwd without one)."""
+    inp, p, o, S_T = _kda_case("noalloc-kda-small", 512, 2)
+    need = lib.gdn_chunk_fwd_workspace(ctypes.byref(p))
+    assert 0 < need <= SCRATCH_BYTES
+    fl = B.GDN_CHANNEL_GATE | B.GDN_QK_L2NORM
+    o_ref, S_ref = lla.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], flags=fl)
+    assert lib.gdn_chunk_fwd_noalloc(ctypes.byref(p), None) == B.GDN_OK
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(S_T, S_ref)
+
+    inp, p, o, S_T = _kda_case("noalloc-kda-large", 4096, 16)
+    assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) > SCRATCH_BYTES
+    o1 = torch.full_like(o, float("nan"))
+    S1 = torch.full_like(S_T, float("nan"))
+    p1 = B.gdn_fwd_params(*(getattr(p, f) for f, _ in B.gdn_fwd_params._fields_))
+    p1.o, p1.S_T = o1.data_ptr(), S1.data_ptr()
+    assert lib.gdn_chunk_fwd(ctypes.byref(p1), None, 0, None) == B.GDN_OK
+    assert lib.gdn_chunk_fwd_noalloc(ctypes.byref(p), None) == B.GDN_OK
+    torch.cuda.synchronize()
+    assert lla.gdn_get_device_status() == lla.GDN_OK
+    assert torch.isfinite(S1).all()
+    assert torch.equal(o, o1) and torch.equal(S_T, S1)

@@ -126,6 +126,91 @@ struct Params {
   Ws ws;
 };
 
+// A = diag(b) K~ K^^T (strictly lower) and P = Q~ K^^T (lower) of a factored
+// chunk, with K^ in the plan's K rows, K~ in its G rows, Q~ in its Q rows:
+// thread rows r0 .. r0 + 3, columns cg + 16 j, four channels per read.
+template <int DK, typename PL>
+__device__ __forceinline__ void ap_factored(float* sm, int tid) {
+  constexpr int LDK = PL::LDK;
+  const float* sK = sm + PL::K;
+  const float* sQ = sm + PL::Q;
+  const float* sG = sm + PL::G;
+  const float* sb = sm + PL::B;
+  float* sA = sm + PL::A;
+  float* sP = sm + PL::P;
+  const int r0 = (tid >> 4) * 4, cg = tid & 15;
+  float kk[4][4], qk[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) kk[i][j] = qk[i][j] = 0.f;
+#pragma unroll 2
+  for (int d = 0; d < DK; d += 4) {
+    float4 ak[4], aq[4], bk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ak[i] = lds4(sG + (r0 + i) * LDK + d);
+      aq[i] = lds4(sQ + (r0 + i) * LDK + d);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bk[j] = lds4(sK + (cg + 16 * j) * LDK + d);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        kk[i][j] = dot4(ak[i], bk[j], kk[i][j]);
+        qk[i][j] = dot4(aq[i], bk[j], qk[i][j]);
+      }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = r0 + i, cc = cg + 16 * j;
+      sA[r * LDC + cc] = (cc < r) ? sb[r] * kk[i][j] : 0.f;
+      sP[r * LDC + cc] = (cc <= r) ? qk[i][j] : 0.f;
+    }
+}
+
+// A and P with each term's own decay e^{G_ic - G_jc} (the fast exponential: a
+// few ulp on arguments <= 0, far inside the fp32 bar), from K, Q and G in the
+// plan's rows; only the lower triangle j <= i is enumerated, the upper one is
+// written as zeros.
+template <int DK, typename PL>
+__device__ __forceinline__ void ap_exact(float* sm, int tid) {
+  constexpr int LDK = PL::LDK;
+  const float* sK = sm + PL::K;
+  const float* sQ = sm + PL::Q;
+  const float* sG = sm + PL::G;
+  const float* sb = sm + PL::B;
+  float* sA = sm + PL::A;
+  float* sP = sm + PL::P;
+  for (int e = tid; e < C * (C + 1) / 2; e += THREADS) {
+    int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+    while (i * (i + 1) / 2 > e) --i;
+    while ((i + 1) * (i + 2) / 2 <= e) ++i;
+    const int j = e - i * (i + 1) / 2;
+    float kk = 0.f, qk = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < DK; ++d) {
+      const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
+      const float kj = sK[j * LDK + d] * dec;
+      kk = fmaf(sK[i * LDK + d], kj, kk);
+      qk = fmaf(sQ[i * LDK + d], kj, qk);
+    }
+    sA[i * LDC + j] = (j < i) ? sb[i] * kk : 0.f;
+    sP[i * LDC + j] = qk;
+  }
+  for (int e = tid; e < C * (C - 1) / 2; e += THREADS) {   // the strict upper triangle
+    int j = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+    while (j * (j + 1) / 2 > e) --j;
+    while ((j + 1) * (j + 2) / 2 <= e) ++j;
+    const int i = e - j * (j + 1) / 2;            // i <= j, then shifted: column j + 1 > row i
+    sA[i * LDC + j + 1] = 0.f;
+    sP[i * LDC + j + 1] = 0.f;
+  }
+}
+
 // The chunk's operands of the KDA form (every thread of the CTA calls it):
 // K, Q (with the q/k norm rounded to the io dtype) and the per-channel log
 // decay prefix G of the chunk starting at tok0 (valid rows, zeros below), b,
@@ -208,42 +293,7 @@ __device__ __forceinline__ void kda_chunk_operands(const Params& p, int tok0, in
       sec[tid] = expf(sgc[tid] - smid[tid]);
     }
     __syncthreads();
-    {
-      // A = diag(b) K~ K^^T (strictly lower), P = Q~ K^^T (lower): thread rows
-      // r0 .. r0 + 3, columns cg + 16 j, four channels per read
-      const int r0 = (tid >> 4) * 4, cg = tid & 15;
-      float kk[4][4], qk[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) kk[i][j] = qk[i][j] = 0.f;
-#pragma unroll 2
-      for (int d = 0; d < DK; d += 4) {
-        float4 ak[4], aq[4], bk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          ak[i] = lds4(sG + (r0 + i) * LDK + d);
-          aq[i] = lds4(sQ + (r0 + i) * LDK + d);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) bk[j] = lds4(sK + (cg + 16 * j) * LDK + d);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            kk[i][j] = dot4(ak[i], bk[j], kk[i][j]);
-            qk[i][j] = dot4(aq[i], bk[j], qk[i][j]);
-          }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = r0 + i, cc = cg + 16 * j;
-          sA[r * LDC + cc] = (cc < r) ? sb[r] * kk[i][j] : 0.f;
-          sP[r * LDC + cc] = (cc <= r) ? qk[i][j] : 0.f;
-        }
-    }
+    ap_factored<DK, PL>(sm, tid);
     __syncthreads();
     // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
     // operands from the factored ones: Q o e^G = Q~ e^m, K o e^G = K~ e^m,
@@ -259,33 +309,7 @@ __device__ __forceinline__ void kda_chunk_operands(const Params& p, int tok0, in
       }
     }
   } else {
-    // ---- A and P, each term with its own decay e^{G_ic - G_jc} (the fast
-    // exponential: a few ulp on arguments <= 0, far inside the fp32 bar)
-    // (only the lower triangle j <= i is enumerated; the upper one is zero)
-    for (int e = tid; e < C * (C + 1) / 2; e += THREADS) {
-      int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-      while (i * (i + 1) / 2 > e) --i;
-      while ((i + 1) * (i + 2) / 2 <= e) ++i;
-      const int j = e - i * (i + 1) / 2;
-      float kk = 0.f, qk = 0.f;
-#pragma unroll 8
-      for (int d = 0; d < DK; ++d) {
-        const float dec = __expf(sG[i * LDK + d] - sG[j * LDK + d]);
-        const float kj = sK[j * LDK + d] * dec;
-        kk = fmaf(sK[i * LDK + d], kj, kk);
-        qk = fmaf(sQ[i * LDK + d], kj, qk);
-      }
-      sA[i * LDC + j] = (j < i) ? sb[i] * kk : 0.f;
-      sP[i * LDC + j] = qk;
-    }
-    for (int e = tid; e < C * (C - 1) / 2; e += THREADS) {   // the strict upper triangle
-      int j = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-      while (j * (j + 1) / 2 > e) --j;
-      while ((j + 1) * (j + 2) / 2 <= e) ++j;
-      const int i = e - j * (j + 1) / 2;            // i <= j, then shifted: column j + 1 > row i
-      sA[i * LDC + j + 1] = 0.f;
-      sP[i * LDC + j + 1] = 0.f;
-    }
+    ap_exact<DK, PL>(sm, tid);
     __syncthreads();
     // ---- T = (I + A)^{-1}, one column per thread; meanwhile the decayed
     // operands: Q o e^G over Q, K o e^G over G, K o e^{G_C - G} over K
@@ -318,15 +342,11 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
   float* sG = sm + PL::G;
   float* sSig = sm + PL::SIG;
   float* sV = sm + PL::V;
-  float* sA = sm + PL::A;
   float* sT = sm + PL::T;
   float* sP = sm + PL::P;
   float* sU = sm + PL::U;
   float* sb = sm + PL::B;
   float* sgc = sm + PL::GC;
-  float* smid = sm + PL::MID;
-  float* sem = smid + DK;
-  float* sec = sem + DK;
 
   const int tid = threadIdx.x;
   const int slice = blockIdx.x % p.n_slices;
@@ -351,8 +371,6 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
   }
   const int col0 = slice * DVS;
   const size_t sbase = ((size_t)seq * H + h) * DK * (size_t)dv + col0;
-  const T* q = static_cast<const T*>(p.q);
-  const T* k = static_cast<const T*>(p.k);
   const T* v = static_cast<const T*>(p.v);
   T* o = static_cast<T*>(p.o);
 
@@ -607,42 +625,209 @@ __device__ __forceinline__ void copy_rows(float* dst, const float* src, int tid)
   }
 }
 
+// Four consecutive io values (8 or 16 bytes, read-only path) as floats.
+__device__ __forceinline__ void ld4(const float* p, float (&v)[4]) {
+  const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+__device__ __forceinline__ void ld4(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  v[0] = lo.x; v[1] = lo.y; v[2] = hi.x; v[3] = hi.y;
+}
+__device__ __forceinline__ void st4(float* p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+
 // One CTA per (chunk slot, head): the chunk's operands into the workspace.
+// Each thread holds four channels (4 dq .. 4 dq + 3) of RPT consecutive rows
+// in registers: the loads are all in flight at once, the decay prefix runs
+// down the thread's rows and then adds the totals of the row groups above,
+// the q/k norm is a reduction across the threads of one row group (lanes of
+// one warp), and the decayed operands go from registers to the workspace.
 template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const Params p) {
   using PL = PrepPlan<DK>;
   constexpr int LDK = PL::LDK;
+  constexpr int QPR = DK / 4;                      // channel quads per row
+  constexpr int RG = THREADS / QPR;                // row groups
+  constexpr int RPT = C / RG;                      // rows per thread
+  static_assert(QPR <= 32 && 32 % QPR == 0 && RG * RPT == C, "prep register map");
   extern __shared__ __align__(16) float sm[];
+  float* sK = sm + PL::K;
+  float* sQ = sm + PL::Q;
+  float* sG = sm + PL::G;
+  float* sT = sm + PL::T;
+  float* sb = sm + PL::B;
+  float* sTot = sm + PL::A;                        // [RG][DK] row-group sums of log a (A comes later)
+  float* sRow0 = sm + PL::GC;                      // [DK] log a of row 0
   const int tid = threadIdx.x;
   const long long slot = blockIdx.x / p.H;
   const int h = blockIdx.x % p.H;
   int tok0, valid;
   if (!slot_chunk(p, slot, tok0, valid)) return;
-  kda_chunk_operands<DK, T, PL>(p, tok0, valid, h, sm, tid);
-  const size_t w = (size_t)slot * p.H + h;
-  float4* kg = reinterpret_cast<float4*>(p.ws.KG + w * C * DK);
-  float4* qg = reinterpret_cast<float4*>(p.ws.QG + w * C * DK);
-  float4* kh = reinterpret_cast<float4*>(p.ws.Kh + w * C * DK);
-  for (int e = tid; e < C * DK / 4; e += THREADS) {
-    const int i = e / (DK / 4), d = 4 * (e % (DK / 4));
-    kg[e] = lds4(sm + PL::G + i * LDK + d);
-    qg[e] = lds4(sm + PL::Q + i * LDK + d);
-    kh[e] = lds4(sm + PL::K + i * LDK + d);
+  const int H = p.H;
+  const int d0 = 4 * (tid % QPR), rg = tid / QPR, i0 = RPT * rg;
+  const T* q = static_cast<const T*>(p.q);
+  const T* k = static_cast<const T*>(p.k);
+  // ---- loads (rows past the sequence end: zero keys and queries, a = 1, b = 0)
+  float kr[RPT][4], qr[RPT][4], g[RPT][4];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    if (i0 + r < valid) {
+      const size_t off = ((size_t)(tok0 + i0 + r) * H + h) * DK + d0;
+      ld4(k + off, kr[r]);
+      ld4(q + off, qr[r]);
+      ld4(p.a + off, g[r]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) kr[r][c] = qr[r][c] = 0.f, g[r][c] = 1.f;
+    }
   }
-  float4* tb = reinterpret_cast<float4*>(p.ws.TB + w * C * C);
+  if (tid < C) sb[tid] = (tid < valid) ? p.b[(size_t)(tok0 + tid) * H + h] : 0.f;
+  // ---- log a, summed down this thread's rows
+#pragma unroll
+  for (int r = 0; r < RPT; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) g[r][c] = logf(g[r][c]) + (r ? g[r - 1][c] : 0.f);
+  st4(sTot + rg * DK + d0, g[RPT - 1][0], g[RPT - 1][1], g[RPT - 1][2], g[RPT - 1][3]);
+  if (rg == 0) st4(sRow0 + d0, g[0][0], g[0][1], g[0][2], g[0][3]);
+  // ---- the q/k L2 norm over each row (QPR lanes), rounded to the io dtype
+  if (p.flags & GDN_QK_L2NORM) {
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      float sk = 0.f, sq = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        sk = fmaf(kr[r][c], kr[r][c], sk);
+        sq = fmaf(qr[r][c], qr[r][c], sq);
+      }
+#pragma unroll
+      for (int o = QPR / 2; o >= 1; o >>= 1) {
+        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      }
+      const float ik = 1.0f / sqrtf(sk + kQkNormEps), iq = 1.0f / sqrtf(sq + kQkNormEps);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        kr[r][c] = to_f32(from_f32<T>(kr[r][c] * ik));
+        qr[r][c] = to_f32(from_f32<T>(qr[r][c] * iq));
+      }
+    }
+  }
+  __syncthreads();
+  // ---- G = the thread's running sums plus the row groups above; G_0, G_C
+  float off[4] = {0.f, 0.f, 0.f, 0.f}, gc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < RG; ++j) {
+    const float4 t = lds4(sTot + j * DK + d0);
+    const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (j < rg) off[c] += tv[c];
+      gc[c] += tv[c];
+    }
+  }
+  float mid[4];
+  bool wide = false;
+  {
+    const float4 g0 = lds4(sRow0 + d0);
+    const float g0v[4] = {g0.x, g0.y, g0.z, g0.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      mid[c] = 0.5f * (g0v[c] + gc[c]);
+      wide |= !(g0v[c] - gc[c] <= kFactorRange);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < RPT; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) g[r][c] += off[c];
+  const bool factored = !__syncthreads_or(wide);
+  // ---- the decayed operands: factored ones to shared memory (K^ over K, K~
+  // over G, Q~ over Q) or the plain K, Q, G; K o e^G, Q o e^G and
+  // K o e^{G_C - G} to the workspace
+  const size_t w = (size_t)slot * H + h;
+  float* kg = p.ws.KG + w * C * DK;
+  float* qg = p.ws.QG + w * C * DK;
+  float* kh = p.ws.Kh + w * C * DK;
+  if (factored) {
+    float em[4], ec[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      em[c] = expf(mid[c]);
+      ec[c] = expf(gc[c] - mid[c]);
+    }
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      float kt[4], kc[4], qt[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float x = g[r][c] - mid[c];
+        const float ex = expf(x), fx = expf(-x);
+        kt[c] = kr[r][c] * ex;
+        kc[c] = kr[r][c] * fx;
+        qt[c] = qr[r][c] * ex;
+      }
+      const int i = i0 + r;
+      st4(sK + i * LDK + d0, kc[0], kc[1], kc[2], kc[3]);
+      st4(sG + i * LDK + d0, kt[0], kt[1], kt[2], kt[3]);
+      st4(sQ + i * LDK + d0, qt[0], qt[1], qt[2], qt[3]);
+      st4(kg + i * DK + d0, kt[0] * em[0], kt[1] * em[1], kt[2] * em[2], kt[3] * em[3]);
+      st4(qg + i * DK + d0, qt[0] * em[0], qt[1] * em[1], qt[2] * em[2], qt[3] * em[3]);
+      st4(kh + i * DK + d0, kc[0] * ec[0], kc[1] * ec[1], kc[2] * ec[2], kc[3] * ec[3]);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      float a1[4], a2[4], a3[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float eg = expf(g[r][c]);
+        a1[c] = kr[r][c] * eg;
+        a2[c] = qr[r][c] * eg;
+        a3[c] = kr[r][c] * expf(gc[c] - g[r][c]);
+      }
+      const int i = i0 + r;
+      st4(sK + i * LDK + d0, kr[r][0], kr[r][1], kr[r][2], kr[r][3]);
+      st4(sQ + i * LDK + d0, qr[r][0], qr[r][1], qr[r][2], qr[r][3]);
+      st4(sG + i * LDK + d0, g[r][0], g[r][1], g[r][2], g[r][3]);
+      st4(kg + i * DK + d0, a1[0], a1[1], a1[2], a1[3]);
+      st4(qg + i * DK + d0, a2[0], a2[1], a2[2], a2[3]);
+      st4(kh + i * DK + d0, a3[0], a3[1], a3[2], a3[3]);
+    }
+  }
+  if (rg == 0)
+    st4(p.ws.EGC + w * DK + d0, expf(gc[0]), expf(gc[1]), expf(gc[2]), expf(gc[3]));
+  __syncthreads();
+  // ---- A and P
+  if (factored) ap_factored<DK, PL>(sm, tid);
+  else ap_exact<DK, PL>(sm, tid);
+  __syncthreads();
+  // ---- T = (I + A)^{-1}, one column per thread; meanwhile P to the workspace
   float4* pp = reinterpret_cast<float4*>(p.ws.P + w * C * C);
+  if (tid < C) {
+    solve_column<C, LDC>(sm + PL::A, sT, tid);
+  } else {
+    for (int e = tid - C; e < C * C / 4; e += THREADS - C) {
+      const int i = e / (C / 4), j = 4 * (e % (C / 4));
+      pp[e] = lds4(sm + PL::P + i * LDC + j);
+    }
+  }
+  __syncthreads();
+  // ---- T diag(b) to the workspace
+  float4* tb = reinterpret_cast<float4*>(p.ws.TB + w * C * C);
   for (int e = tid; e < C * C / 4; e += THREADS) {
     const int i = e / (C / 4), j = 4 * (e % (C / 4));
-    float4 t = lds4(sm + PL::T + i * LDC + j);
-    const float4 b = lds4(sm + PL::B + j);
+    float4 t = lds4(sT + i * LDC + j);
+    const float4 b = lds4(sb + j);
     t.x *= b.x;
     t.y *= b.y;
     t.z *= b.z;
     t.w *= b.w;
     tb[e] = t;
-    pp[e] = lds4(sm + PL::P + i * LDC + j);
   }
-  if (tid < DK / 4) reinterpret_cast<float4*>(p.ws.EGC + w * DK)[tid] = lds4(sm + PL::GC + 4 * tid);
 }
 
 // acc[j] += a . (b[0][j], b[1][j], b[2][j], b[3][j])

@@ -545,29 +545,6 @@ struct PrepPlan {
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 
-// A chain's state slice of NV columns, the chunk's operands (single buffers,
-// each refilled with cp.async as soon as its last reader is done) and the V
-// rows in the io dtype.
-template <int DK, int NV, typename T>
-struct ChainPlan {
-  static constexpr int LDK = DK + 4;
-  static constexpr int LDS = NV + 4;               // [rows][NV] fp32 tiles
-  static constexpr int VROW = (NV * (int)sizeof(T) + 16) / 4;   // floats per V row
-  static constexpr int KG = 0;                     // [C][LDK]  K o e^G
-  static constexpr int QG = KG + C * LDK;          // [C][LDK]  Q o e^G
-  static constexpr int KH = QG + C * LDK;          // [C][LDK]  K o e^{G_C - G}
-  static constexpr int TB = KH + C * LDK;          // [C][LDC]  T diag(b)
-  static constexpr int P = TB + C * LDC;           // [C][LDC]
-  static constexpr int SIG = P + C * LDC;          // [DK][LDS]
-  static constexpr int X = SIG + DK * LDS;         // [C][LDS]
-  static constexpr int U = X + C * LDS;            // [C][LDS]
-  static constexpr int EGC = U + C * LDS;          // DK
-  static constexpr int V = EGC + DK;               // [C][VROW]
-  static constexpr int FLOATS = V + C * VROW;
-  static constexpr size_t BYTES = (size_t)FLOATS * 4;
-};
-static_assert(ChainPlan<128, 32, float>::BYTES <= 232448, "KDA chain shared memory");
-
 __device__ __forceinline__ void seq_range(const Params& p, int s, int& t0, int& t1, bool report) {
   if (p.cu_seqlens) {
     t0 = __ldg(p.cu_seqlens + s);
@@ -856,13 +833,58 @@ __device__ __forceinline__ void rows_times(float (&acc)[4][TN], const float* A, 
   }
 }
 
-// One CTA per (sequence, head, NV-column dv slice): the chain through its
-// chunks, operands from the workspace.
-template <int DK, int NV, typename T>
+// A chain's state slice of NV = 16 columns, the chunk's operands (single
+// buffers, each refilled with cp.async as soon as its last reader is done),
+// the V rows in the io dtype, and the partial sums of the split products.
+template <int DK, typename T>
+struct ChainPlan {
+  static constexpr int NV = 16;
+  static constexpr int LDK = DK + 4;
+  static constexpr int LDS = NV + 4;               // [rows][NV] fp32 tiles
+  static constexpr int VROW = (NV * (int)sizeof(T) + 16) / 4;   // floats per V row
+  static constexpr int RROWS = C + DK;             // rows of one group's partial sums
+  static constexpr int KG = 0;                     // [C][LDK]  K o e^G
+  static constexpr int QG = KG + C * LDK;          // [C][LDK]  Q o e^G
+  static constexpr int KH = QG + C * LDK;          // [C][LDK]  K o e^{G_C - G}
+  static constexpr int TB = KH + C * LDK;          // [C][LDC]  T diag(b)
+  static constexpr int P = TB + C * LDC;           // [C][LDC]
+  static constexpr int SIG = P + C * LDC;          // [DK][LDS]
+  static constexpr int X = SIG + DK * LDS;         // [C][LDS]  V - (K o e^G) Sigma_0
+  static constexpr int U = X + C * LDS;            // [C][LDS]
+  static constexpr int OQ = U + C * LDS;           // [C][LDS]  (Q o e^G) Sigma_0
+  static constexpr int RED = OQ + C * LDS;         // [4][RROWS][NV] partial sums (swizzled)
+  static constexpr int EGC = RED + 4 * RROWS * NV; // [2][DK]  e^{G_C}, by chunk parity
+  static constexpr int V = EGC + 2 * DK;           // [C][VROW]
+  static constexpr int FLOATS = V + C * VROW;
+  static constexpr size_t BYTES = (size_t)FLOATS * 4;
+};
+static_assert(ChainPlan<128, float>::BYTES <= 232448, "KDA chain shared memory");
+
+// Offset of (row, float4 column c4) in one group's partial sums: rows of 16
+// floats, the two rows of an even/odd pair swapped when bit 2 xor bit 3 of
+// the row is set, so that the tile writes (rows r and r + 4, or r and r + 8,
+// in one quarter warp) and the row-order reads are both conflict-free.
+__device__ __forceinline__ int red_off(int row, int c4) {
+  return (16 * row + 4 * c4) ^ ((((row >> 2) ^ (row >> 3)) & 1) << 4);
+}
+
+__device__ __forceinline__ void add4(float4& a, float4 b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+
+// One CTA per (sequence, head, 16-column dv slice): the chain through its
+// chunks, operands from the workspace.  The two products over dk and the two
+// over the chunk's rows each split their contraction over four groups of 64
+// threads (4 x 4 register tiles, partial sums reduced through shared memory).
+template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const Params p) {
-  using PL = ChainPlan<DK, NV, T>;
-  constexpr int LDK = PL::LDK, LDS = PL::LDS;
-  constexpr int TN = NV / 16;                      // columns per thread
+  using PL = ChainPlan<DK, T>;
+  constexpr int NV = PL::NV, LDK = PL::LDK, LDS = PL::LDS;
+  constexpr int RG_FLOATS = PL::RROWS * NV;        // one group's partial sums
+  constexpr int TD = DK / 16;                      // carry rows per thread
   extern __shared__ __align__(16) float sm[];
   float* sKG = sm + PL::KG;
   float* sQG = sm + PL::QG;
@@ -872,6 +894,8 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
   float* sSig = sm + PL::SIG;
   float* sX = sm + PL::X;
   float* sU = sm + PL::U;
+  float* sOq = sm + PL::OQ;
+  float* sRed = sm + PL::RED;
   float* sEGC = sm + PL::EGC;
   float* sV = sm + PL::V;
 
@@ -892,12 +916,13 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
   T* o = static_cast<T*>(p.o);
 
   // Operand groups of chunk c, one cp.async group each (empty past the last
-  // chunk): X's (K o e^G, V rows), U's (T diag(b)), O's (Q o e^G, P), the
-  // carry's (K o e^{G_C - G}, e^{G_C}).
-  auto load_x = [&](int c) {
+  // chunk): A, the dk products' (K o e^G, Q o e^G, V rows); B, U's
+  // (T diag(b)); C, the row products' (P, K o e^{G_C - G}, e^{G_C}).
+  auto load_a = [&](int c) {
     if (c < n_chunks) {
       const size_t w = (size_t)(slot0 + c) * H + h;
       copy_rows<C, DK, LDK>(sKG, p.ws.KG + w * C * DK, tid);
+      copy_rows<C, DK, LDK>(sQG, p.ws.QG + w * C * DK, tid);
       const int tok0 = t0 + c * C, valid = min(C, t1 - tok0);
       constexpr int PIECES = NV * (int)sizeof(T) / 16;
       for (int e = tid; e < C * PIECES; e += THREADS) {
@@ -908,126 +933,165 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
     }
     cp_async_commit();
   };
-  auto load_u = [&](int c) {
+  auto load_b = [&](int c) {
     if (c < n_chunks) copy_rows<C, C, LDC>(sTB, p.ws.TB + (size_t)((slot0 + c) * H + h) * C * C, tid);
     cp_async_commit();
   };
-  auto load_o = [&](int c) {
+  auto load_c = [&](int c) {
     if (c < n_chunks) {
       const size_t w = (size_t)(slot0 + c) * H + h;
-      copy_rows<C, DK, LDK>(sQG, p.ws.QG + w * C * DK, tid);
       copy_rows<C, C, LDC>(sP, p.ws.P + w * C * C, tid);
-    }
-    cp_async_commit();
-  };
-  auto load_s = [&](int c) {
-    if (c < n_chunks) {
-      const size_t w = (size_t)(slot0 + c) * H + h;
       copy_rows<C, DK, LDK>(sKh, p.ws.Kh + w * C * DK, tid);
-      if (tid < DK / 4) cp_async16(sEGC + 4 * tid, p.ws.EGC + w * DK + 4 * tid);
+      if (tid < DK / 4) cp_async16(sEGC + (c & 1) * DK + 4 * tid, p.ws.EGC + w * DK + 4 * tid);
     }
     cp_async_commit();
   };
 
-  load_x(0);
-  load_u(0);
-  load_o(0);
+  load_a(0);
+  load_b(0);
+  load_c(0);
   for (int e = tid; e < DK * NV; e += THREADS) {
     const int d = e / NV, c = e % NV;
     sSig[d * LDS + c] = p.S0 ? p.S0[sbase + (size_t)d * dv + c] : 0.f;
   }
-  // Register tiles: [C][NV] results give a thread rows r0 .. r0 + 3 and
-  // columns c0 .. c0 + TN - 1; the dk x NV carry gives it rows DK/16 rg ..
-  const int rg = tid >> 4, r0 = 4 * rg, c0 = TN * (tid & 15);
-  // Each phase waits for its own group (two later groups may still be in
-  // flight), syncs, then refills the buffers of the phase before it.
+  // split products: group g of 64 threads, 4 x 4 tile (rows 4 rt .., columns 4 ct ..)
+  const int g = tid >> 6, rt = (tid & 63) >> 2, ct = tid & 3;
+  const int r0 = 4 * rt, c0 = 4 * ct;
+  float* red = sRed + g * RG_FLOATS;
+  // Groups in flight at each wait, oldest first: [A c, B c, C c] before the dk
+  // products, [B c, C c] before U, [C c, A c+1] before the row products; a
+  // refill is issued only after the barrier that ends its buffer's last reader.
   for (int c = 0; c < n_chunks; ++c) {
     const int tok0 = t0 + c * C, valid = min(C, t1 - tok0);
-    // ---- X = V - (K o e^G) Sigma_0
-    cp_async_wait<2>();
+    cp_async_wait<2>();                            // the dk products' group
     __syncthreads();
-    load_s(c);
+    // ---- (K o e^G) Sigma_0 and (Q o e^G) Sigma_0, dk split four ways
     {
-      float acc[4][TN] = {};
-      rows_times<TN>(acc, sKG + r0 * LDK, LDK, sSig + c0, LDS, DK);
+      float ax[4][4] = {}, aq[4][4] = {};
+      constexpr int KR = DK / 4;
+#pragma unroll 2
+      for (int k = g * KR; k < (g + 1) * KR; k += 4) {
+        float4 kx[4], qx[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          kx[i] = lds4(sKG + (r0 + i) * LDK + k);
+          qx[i] = lds4(sQG + (r0 + i) * LDK + k);
+        }
+        float b[4][4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) ldv<4>(sSig + (k + kk) * LDS + c0, b[kk]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          fma4<4>(ax[i], kx[i], b);
+          fma4<4>(aq[i], qx[i], b);
+        }
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const T* vr = reinterpret_cast<const T*>(sV + (r0 + i) * PL::VROW) + c0;
-        float x[TN];
-#pragma unroll
-        for (int j = 0; j < TN; ++j) x[j] = to_f32(vr[j]) - acc[i][j];
-        stv<TN>(sX + (r0 + i) * LDS + c0, x);
+        stv<4>(red + red_off(r0 + i, ct), ax[i]);
+        stv<4>(red + red_off(C + r0 + i, ct), aq[i]);
       }
     }
-    // ---- U = T diag(b) X (lower triangular: columns < r0 + 4)
-    cp_async_wait<2>();
     __syncthreads();
-    load_x(c + 1);
-    {
-      float acc[4][TN] = {};
-      rows_times<TN>(acc, sTB + r0 * LDC, LDC, sX + c0, LDS, r0 + 4);
+    // ---- reduce: X = V - sum -> sX, the Q part -> sOq
 #pragma unroll
-      for (int i = 0; i < 4; ++i) stv<TN>(sU + (r0 + i) * LDS + c0, acc[i]);
+    for (int m = 0; m < 2; ++m) {
+      const int e = tid + THREADS * m;
+      const int row = e >> 2, c4 = e & 3;
+      const int off = red_off(row, c4);
+      float4 s = lds4(sRed + off);
+#pragma unroll
+      for (int gg = 1; gg < 4; ++gg) add4(s, lds4(sRed + gg * RG_FLOATS + off));
+      if (row < C) {
+        const T* vr = reinterpret_cast<const T*>(sV + row * PL::VROW) + 4 * c4;
+        s = make_float4(to_f32(vr[0]) - s.x, to_f32(vr[1]) - s.y, to_f32(vr[2]) - s.z, to_f32(vr[3]) - s.w);
+        *reinterpret_cast<float4*>(sX + row * LDS + 4 * c4) = s;
+      } else {
+        *reinterpret_cast<float4*>(sOq + (row - C) * LDS + 4 * c4) = s;
+      }
     }
-    // ---- O = scale ((Q o e^G) Sigma_0 + P U), then the output gate and the
-    // loop residual
-    cp_async_wait<2>();
+    cp_async_wait<1>();                            // U's group (the row products' may fly)
     __syncthreads();
-    load_u(c + 1);
+    load_a(c + 1);
+    // ---- U = T diag(b) X (lower triangular: columns < row + 1); rows
+    // 4 (tid / 16) .., column tid % 16
     {
-      float acc[4][TN] = {};
-      rows_times<TN>(acc, sQG + r0 * LDK, LDK, sSig + c0, LDS, DK);
-      rows_times<TN>(acc, sP + r0 * LDC, LDC, sU + c0, LDS, r0 + 4);
+      const int ur0 = 4 * (tid >> 4), uc = tid & 15;
+      float acc[4][1] = {};
+      rows_times<1>(acc, sTB + ur0 * LDC, LDC, sX + uc, LDS, ur0 + 4);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = r0 + i;
-        if (r >= valid) continue;
-        const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + r) * H + h])) : 1.f;
+      for (int i = 0; i < 4; ++i) sU[(ur0 + i) * LDS + uc] = acc[i][0];
+    }
+    cp_async_wait<1>();                            // the row products' group
+    __syncthreads();
+    load_b(c + 1);
+    // ---- P U and (K o e^{G_C - G})^T U, the chunk's rows split four ways
+    {
+      float ao[4][4] = {}, as[TD][4] = {};
+      const int d0 = TD * rt;
+#pragma unroll 1
+      for (int i = 16 * g; i < 16 * g + 16; i += 4) {
+        float4 pr[4];
 #pragma unroll
-        for (int j = 0; j < TN; ++j) {
-          const int cc = c0 + j;
-          float y = p.scale * acc[i][j];
-          const size_t off = ((size_t)(tok0 + r) * H + h) * dv + col0 + cc;
+        for (int ii = 0; ii < 4; ++ii) pr[ii] = lds4(sP + (r0 + ii) * LDC + i);
+        float u[4][4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) ldv<4>(sU + (i + x) * LDS + c0, u[x]);
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) fma4<4>(ao[ii], pr[ii], u);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+#pragma unroll
+          for (int q4 = 0; q4 < TD / 4; ++q4) {
+            const float4 kh = lds4(sKh + (i + x) * LDK + d0 + 4 * q4);
+            const float kv[4] = {kh.x, kh.y, kh.z, kh.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) as[4 * q4 + e][j] = fmaf(kv[e], u[x][j], as[4 * q4 + e][j]);
+          }
+        }
+      }
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) stv<4>(red + red_off(r0 + ii, ct), ao[ii]);
+#pragma unroll
+      for (int e = 0; e < TD; ++e) stv<4>(red + red_off(C + d0 + e, ct), as[e]);
+    }
+    __syncthreads();
+    load_c(c + 1);
+    // ---- reduce: O = scale ((Q o e^G) Sigma_0 + P U) with the output gate and
+    // the loop residual; Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
+    const float* egc = sEGC + (c & 1) * DK;
+#pragma unroll
+    for (int m = 0; m < (C + DK) / 64; ++m) {
+      const int e = tid + THREADS * m;
+      const int row = e >> 2, c4 = e & 3;
+      const int off = red_off(row, c4);
+      float4 s = lds4(sRed + off);
+#pragma unroll
+      for (int gg = 1; gg < 4; ++gg) add4(s, lds4(sRed + gg * RG_FLOATS + off));
+      if (row < C) {
+        if (row >= valid) continue;
+        add4(s, lds4(sOq + row * LDS + 4 * c4));
+        const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + row) * H + h])) : 1.f;
+        const float sv[4] = {s.x, s.y, s.z, s.w};
+        const size_t obase = ((size_t)(tok0 + row) * H + h) * dv + col0 + 4 * c4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float y = p.scale * sv[j];
           if (p.gate) y *= og;
           if (p.h_prev) {
-            const float hp = to_f32(static_cast<const T*>(p.h_prev)[off]);
-            y = fmaf(p.rho[(size_t)h * dv + col0 + cc], hp, to_f32(from_f32<T>(y)));
+            const float hp = to_f32(static_cast<const T*>(p.h_prev)[obase + j]);
+            y = fmaf(p.rho[(size_t)h * dv + col0 + 4 * c4 + j], hp, to_f32(from_f32<T>(y)));
           }
-          o[off] = from_f32<T>(y);
+          o[obase + j] = from_f32<T>(y);
         }
-      }
-    }
-    // ---- Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
-    cp_async_wait<2>();
-    __syncthreads();
-    load_o(c + 1);
-    {
-      constexpr int TD = DK / 16;
-      const int d0 = TD * rg;
-      float acc[TD][TN] = {};
-#pragma unroll 2
-      for (int i = 0; i < C; ++i) {
-        float u[TN];
-        ldv<TN>(sU + i * LDS + c0, u);
-#pragma unroll
-        for (int q4 = 0; q4 < TD / 4; ++q4) {
-          const float4 a4 = lds4(sKh + i * LDK + d0 + 4 * q4);
-          const float a[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-#pragma unroll
-            for (int j = 0; j < TN; ++j) acc[4 * q4 + e][j] = fmaf(a[e], u[j], acc[4 * q4 + e][j]);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < TD; ++e) {
-        const int d = d0 + e;
-        float sg[TN];
-        ldv<TN>(sSig + d * LDS + c0, sg);
-        const float g = sEGC[d];
-#pragma unroll
-        for (int j = 0; j < TN; ++j) sg[j] = fmaf(g, sg[j], acc[e][j]);
-        stv<TN>(sSig + d * LDS + c0, sg);
+      } else {
+        const int d = row - C;
+        float4* sg = reinterpret_cast<float4*>(sSig + d * LDS + 4 * c4);
+        const float4 old = *sg;
+        const float gd = egc[d];
+        *sg = make_float4(fmaf(gd, old.x, s.x), fmaf(gd, old.y, s.y), fmaf(gd, old.z, s.z), fmaf(gd, old.w, s.w));
       }
     }
   }
@@ -1051,20 +1115,17 @@ static cudaError_t launch_t(const Params& kp, long long blocks, cudaStream_t str
   return cudaGetLastError();
 }
 
-// dv columns per chain CTA of the two-launch schedule
-constexpr int kChainCols = 16;
-
 template <int DK, typename T>
 static cudaError_t launch_two(const Params& kp, long long chunk_blocks, long long chain_blocks,
                               cudaStream_t stream) {
   static std::atomic<bool> set_prep[kMaxDevices], set_chain[kMaxDevices];
   constexpr size_t prep_bytes = PrepPlan<DK>::BYTES;
-  constexpr size_t chain_bytes = ChainPlan<DK, kChainCols, T>::BYTES;
+  constexpr size_t chain_bytes = ChainPlan<DK, T>::BYTES;
   cudaError_t e = smem_attr_once(set_prep, gdn_prefill_kda_prep_kernel<DK, T>, prep_bytes);
-  if (e == cudaSuccess) e = smem_attr_once(set_chain, gdn_prefill_kda_chain_kernel<DK, kChainCols, T>, chain_bytes);
+  if (e == cudaSuccess) e = smem_attr_once(set_chain, gdn_prefill_kda_chain_kernel<DK, T>, chain_bytes);
   if (e != cudaSuccess) return e;
   gdn_prefill_kda_prep_kernel<DK, T><<<(unsigned)chunk_blocks, THREADS, prep_bytes, stream>>>(kp);
-  gdn_prefill_kda_chain_kernel<DK, kChainCols, T><<<(unsigned)chain_blocks, THREADS, chain_bytes, stream>>>(kp);
+  gdn_prefill_kda_chain_kernel<DK, T><<<(unsigned)chain_blocks, THREADS, chain_bytes, stream>>>(kp);
   return cudaGetLastError();
 }
 
@@ -1128,7 +1189,7 @@ gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, void* w
     kp.ws.EGC = reinterpret_cast<float*>(w);
     kp.ws.n_slots = n_slots;
     const long long chunk_blocks = n_slots * p->H;
-    const long long chain_blocks = chains * (p->dv / kda::kChainCols);
+    const long long chain_blocks = chains * (p->dv / 16);   // 16 columns per chain CTA
     if (chunk_blocks > 0x7fffffffLL || chain_blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     if (p->io_dtype == GDN_BF16)
       e = p->dk == 128 ? kda::launch_two<128, __nv_bfloat16>(kp, chunk_blocks, chain_blocks, stream)

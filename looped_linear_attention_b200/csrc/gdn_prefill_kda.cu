@@ -81,6 +81,66 @@ __device__ __forceinline__ void solve_column(const float* sA, float* sT, int col
   for (int i = 0; i < C; ++i) sT[i * LDC + col] = t[i];
 }
 
+// T = (I + A)^{-1} for the strictly lower C x C matrix A (row stride LDC) by
+// 16 x 16 blocks (every thread of the CTA calls it; ends with the block
+// synced): the four diagonal blocks by forward substitution, one column per
+// thread, then block row by block row T_RC = -T_RR sum_{C <= m < R} A_Rm T_mC,
+// the sums staged in sX (3 x 256 floats).  The same T as column-wise forward
+// substitution up to rounding order.
+__device__ __forceinline__ void solve_blocked(const float* sA, float* sT, float* sX, int tid) {
+  static_assert(C == 64, "four 16 x 16 blocks");
+  if (tid < C) {
+    const int R = tid >> 4, col = tid & 15, o = 16 * R;
+    float t[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int m = 0; m < i; ++m) acc[m & 3] = fmaf(sA[(o + i) * LDC + o + m], t[m], acc[m & 3]);
+      t[i] = ((i == col) ? 1.f : 0.f) - ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sT[(o + i) * LDC + o + col] = t[i];
+  } else {
+    // the blocks above the diagonal are zero
+    for (int e = tid - C; e < 6 * 256; e += THREADS - C) {
+      const int b = e >> 8, w = e & 255;
+      const int R = (b >= 5) ? 2 : (b >= 3) ? 1 : 0;
+      const int Cb = (b >= 5) ? 3 : (b >= 3) ? b - 1 : b + 1;
+      sT[(16 * R + (w >> 4)) * LDC + 16 * Cb + (w & 15)] = 0.f;
+    }
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int R = 1; R < 4; ++R) {
+    // X_Rc = sum_{c <= m < R} A_Rm T_mc for the R blocks c < R
+    for (int e = tid; e < R * 256; e += THREADS) {
+      const int c = e >> 8, i = (e >> 4) & 15, j = e & 15;
+      const float* arow = sA + (16 * R + i) * LDC;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int m = c; m < R; ++m) {
+        const float* tcol = sT + 16 * m * LDC + 16 * c + j;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(arow[16 * m + k], tcol[k * LDC], acc[k & 3]);
+      }
+      sX[e] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
+    __syncthreads();
+    // T_Rc = -T_RR X_Rc (T_RR is lower triangular, its upper part zero)
+    for (int e = tid; e < R * 256; e += THREADS) {
+      const int c = e >> 8, i = (e >> 4) & 15, j = e & 15;
+      const float* trow = sT + (16 * R + i) * LDC + 16 * R;
+      const float* xcol = sX + c * 256 + j;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(trow[k], xcol[16 * k], acc[k & 3]);
+      sT[(16 * R + i) * LDC + 16 * c + j] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    }
+    __syncthreads();
+  }
+}
+
 template <int DK>
 struct Plan {
   static constexpr int LDK = DK + 4;               // float4 rows (the factored A and P products)
@@ -127,8 +187,13 @@ struct Params {
 };
 
 // A = diag(b) K~ K^^T (strictly lower) and P = Q~ K^^T (lower) of a factored
-// chunk, with K^ in the plan's K rows, K~ in its G rows, Q~ in its Q rows:
-// thread rows r0 .. r0 + 3, columns cg + 16 j, four channels per read.
+// chunk, with K^ in the plan's K rows, K~ in its G rows, Q~ in its Q rows.
+// Only the ten 16 x 16 macro tiles on or below the diagonal are multiplied:
+// 16 threads each, a thread taking rows 16 R + a + 4 i and columns
+// 16 Cc + c + 4 j (i, j < 4), so that the eight lanes of a quarter warp read
+// two rows of one operand and four of the other, all in distinct banks
+// (row stride LDK = 4 mod 32 floats); the other 96 threads zero the six
+// macro tiles above the diagonal.
 template <int DK, typename PL>
 __device__ __forceinline__ void ap_factored(float* sm, int tid) {
   constexpr int LDK = PL::LDK;
@@ -138,38 +203,53 @@ __device__ __forceinline__ void ap_factored(float* sm, int tid) {
   const float* sb = sm + PL::B;
   float* sA = sm + PL::A;
   float* sP = sm + PL::P;
-  const int r0 = (tid >> 4) * 4, cg = tid & 15;
-  float kk[4][4], qk[4][4];
+  if (tid < 160) {
+    const int t = tid >> 4;                        // macro tile, row-band order
+    const int R = (t >= 6) ? 3 : (t >= 3) ? 2 : (t >= 1) ? 1 : 0;
+    const int Cc = t - R * (R + 1) / 2;
+    const int ra = 16 * R + ((tid >> 2) & 3), cb = 16 * Cc + (tid & 3);
+    float kk[4][4], qk[4][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) kk[i][j] = qk[i][j] = 0.f;
+      for (int j = 0; j < 4; ++j) kk[i][j] = qk[i][j] = 0.f;
 #pragma unroll 2
-  for (int d = 0; d < DK; d += 4) {
-    float4 ak[4], aq[4], bk[4];
+    for (int d = 0; d < DK; d += 4) {
+      float4 ak[4], aq[4], bk[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ak[i] = lds4(sG + (r0 + i) * LDK + d);
-      aq[i] = lds4(sQ + (r0 + i) * LDK + d);
+      for (int i = 0; i < 4; ++i) {
+        ak[i] = lds4(sG + (ra + 4 * i) * LDK + d);
+        aq[i] = lds4(sQ + (ra + 4 * i) * LDK + d);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bk[j] = lds4(sK + (cb + 4 * j) * LDK + d);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          kk[i][j] = dot4(ak[i], bk[j], kk[i][j]);
+          qk[i][j] = dot4(aq[i], bk[j], qk[i][j]);
+        }
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) bk[j] = lds4(sK + (cg + 16 * j) * LDK + d);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        kk[i][j] = dot4(ak[i], bk[j], kk[i][j]);
-        qk[i][j] = dot4(aq[i], bk[j], qk[i][j]);
+        const int r = ra + 4 * i, cc = cb + 4 * j;
+        sA[r * LDC + cc] = (cc < r) ? sb[r] * kk[i][j] : 0.f;
+        sP[r * LDC + cc] = (cc <= r) ? qk[i][j] : 0.f;
       }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int r = r0 + i, cc = cg + 16 * j;
-      sA[r * LDC + cc] = (cc < r) ? sb[r] * kk[i][j] : 0.f;
-      sP[r * LDC + cc] = (cc <= r) ? qk[i][j] : 0.f;
+  } else {
+    // macro tiles above the diagonal: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+    for (int e = tid - 160; e < 6 * 256; e += THREADS - 160) {
+      const int t = e >> 8, w = e & 255;
+      const int R = (t >= 5) ? 2 : (t >= 3) ? 1 : 0;
+      const int Cc = (t >= 5) ? 3 : (t >= 3) ? t - 1 : t + 1;
+      const int r = 16 * R + (w >> 4), cc = 16 * Cc + (w & 15);
+      sA[r * LDC + cc] = 0.f;
+      sP[r * LDC + cc] = 0.f;
     }
+  }
 }
 
 // A and P with each term's own decay e^{G_ic - G_jc} (the fast exponential: a
@@ -541,7 +621,8 @@ struct PrepPlan {
   static constexpr int B = P + C * LDC;            // C
   static constexpr int GC = B + C;                 // DK
   static constexpr int MID = GC + DK;              // 3 x DK
-  static constexpr int FLOATS = MID + 3 * DK + 4;
+  static constexpr int SX = MID + 3 * DK + 4;      // 3 x 256: the blocked solve's sums
+  static constexpr int FLOATS = SX + 3 * 256;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 
@@ -602,13 +683,9 @@ __device__ __forceinline__ void copy_rows(float* dst, const float* src, int tid)
   }
 }
 
-// Four consecutive io values (8 or 16 bytes, read-only path) as floats.
-__device__ __forceinline__ void ld4(const float* p, float (&v)[4]) {
-  const float4 x = __ldg(reinterpret_cast<const float4*>(p));
-  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-}
-__device__ __forceinline__ void ld4(const __nv_bfloat16* p, float (&v)[4]) {
-  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+// Four consecutive bf16 values (8 bytes of shared memory) as floats.
+__device__ __forceinline__ void lds_bf16x4(const float* p, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
   const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
   const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
   v[0] = lo.x; v[1] = lo.y; v[2] = hi.x; v[3] = hi.y;
@@ -619,7 +696,7 @@ __device__ __forceinline__ void st4(float* p, float a, float b, float c, float d
 
 // One CTA per (chunk slot, head): the chunk's operands into the workspace.
 // Each thread holds four channels (4 dq .. 4 dq + 3) of RPT consecutive rows
-// in registers: the loads are all in flight at once, the decay prefix runs
+// in registers (read from the staged rows): the decay prefix runs
 // down the thread's rows and then adds the totals of the row groups above,
 // the q/k norm is a reduction across the threads of one row group (lanes of
 // one warp), and the decayed operands go from registers to the workspace.
@@ -648,21 +725,51 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
   const int d0 = 4 * (tid % QPR), rg = tid / QPR, i0 = RPT * rg;
   const T* q = static_cast<const T*>(p.q);
   const T* k = static_cast<const T*>(p.k);
-  // ---- loads (rows past the sequence end: zero keys and queries, a = 1, b = 0)
+  // ---- the chunk's q and k rows (io dtype; fp32 ones straight into the Q and
+  // K rows, bf16 ones into the T and P areas, which are free until the
+  // products) and a rows (into G) staged with cp.async, every piece in
+  // flight at once; rows past the sequence end read nothing (zero fill)
+  constexpr bool kF32 = sizeof(T) == 4;
+  constexpr int RAW_LD = kF32 ? LDK : DK / 2;      // floats per staged q / k row
+  float* rq = kF32 ? sQ : sm + PL::T;
+  float* rk = kF32 ? sK : sm + PL::P;
+  {
+    constexpr int QP = DK * (int)sizeof(T) / 16;   // 16-byte pieces per q / k row
+    for (int e = tid; e < C * QP; e += THREADS) {
+      const int i = e / QP, c = e % QP;
+      const size_t off = ((size_t)(tok0 + min(i, valid - 1)) * H + h) * DK;
+      cp_async16_or_zero(rq + i * RAW_LD + 4 * c, reinterpret_cast<const char*>(q + off) + 16 * c, i < valid);
+      cp_async16_or_zero(rk + i * RAW_LD + 4 * c, reinterpret_cast<const char*>(k + off) + 16 * c, i < valid);
+    }
+    for (int e = tid; e < C * DK / 4; e += THREADS) {
+      const int i = e / (DK / 4), c = 4 * (e % (DK / 4));
+      const size_t off = ((size_t)(tok0 + min(i, valid - 1)) * H + h) * DK;
+      cp_async16_or_zero(sG + i * LDK + c, p.a + off + c, i < valid);
+    }
+    cp_async_commit();
+  }
+  if (tid < C) sb[tid] = (tid < valid) ? p.b[(size_t)(tok0 + tid) * H + h] : 0.f;
+  cp_async_wait<0>();
+  __syncthreads();
+  // ---- this thread's rows into registers (rows past the end: zero keys and
+  // queries, a = 1)
   float kr[RPT][4], qr[RPT][4], g[RPT][4];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
-    if (i0 + r < valid) {
-      const size_t off = ((size_t)(tok0 + i0 + r) * H + h) * DK + d0;
-      ld4(k + off, kr[r]);
-      ld4(q + off, qr[r]);
-      ld4(p.a + off, g[r]);
+    const int i = i0 + r;
+    if constexpr (kF32) {
+      ldv<4>(rk + i * RAW_LD + d0, kr[r]);
+      ldv<4>(rq + i * RAW_LD + d0, qr[r]);
     } else {
+      lds_bf16x4(rk + i * RAW_LD + d0 / 2, kr[r]);
+      lds_bf16x4(rq + i * RAW_LD + d0 / 2, qr[r]);
+    }
+    ldv<4>(sG + i * LDK + d0, g[r]);
+    if (i >= valid) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) kr[r][c] = qr[r][c] = 0.f, g[r][c] = 1.f;
+      for (int c = 0; c < 4; ++c) g[r][c] = 1.f;
     }
   }
-  if (tid < C) sb[tid] = (tid < valid) ? p.b[(size_t)(tok0 + tid) * H + h] : 0.f;
   // ---- log a, summed down this thread's rows
 #pragma unroll
   for (int r = 0; r < RPT; ++r)
@@ -685,7 +792,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
         sk += __shfl_xor_sync(0xffffffffu, sk, o);
         sq += __shfl_xor_sync(0xffffffffu, sq, o);
       }
-      const float ik = 1.0f / sqrtf(sk + kQkNormEps), iq = 1.0f / sqrtf(sq + kQkNormEps);
+      const float ik = rsqrtf(sk + kQkNormEps), iq = rsqrtf(sq + kQkNormEps);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         kr[r][c] = to_f32(from_f32<T>(kr[r][c] * ik));
@@ -782,17 +889,13 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
   if (factored) ap_factored<DK, PL>(sm, tid);
   else ap_exact<DK, PL>(sm, tid);
   __syncthreads();
-  // ---- T = (I + A)^{-1}, one column per thread; meanwhile P to the workspace
+  // ---- P to the workspace; T = (I + A)^{-1} by 16 x 16 blocks
   float4* pp = reinterpret_cast<float4*>(p.ws.P + w * C * C);
-  if (tid < C) {
-    solve_column<C, LDC>(sm + PL::A, sT, tid);
-  } else {
-    for (int e = tid - C; e < C * C / 4; e += THREADS - C) {
-      const int i = e / (C / 4), j = 4 * (e % (C / 4));
-      pp[e] = lds4(sm + PL::P + i * LDC + j);
-    }
+  for (int e = tid; e < C * C / 4; e += THREADS) {
+    const int i = e / (C / 4), j = 4 * (e % (C / 4));
+    pp[e] = lds4(sm + PL::P + i * LDC + j);
   }
-  __syncthreads();
+  solve_blocked(sm + PL::A, sT, sm + PL::SX, tid);
   // ---- T diag(b) to the workspace
   float4* tb = reinterpret_cast<float4*>(p.ws.TB + w * C * C);
   for (int e = tid; e < C * C / 4; e += THREADS) {

@@ -162,10 +162,11 @@ struct Plan {
 static_assert(Plan<128>::BYTES <= 232448, "KDA prefill shared memory");
 
 // Workspace of the two-launch schedule, per (chunk slot, head): the chunk's
-// decayed operands, its two C x C matrices and its decay over the chunk.
+// operands once the state-independent products are folded in (W, Q', U~ and
+// O~ below) and its decay over the chunk.
 struct Ws {
-  float *KG, *QG, *Kh;   // [slots][H][C][dk]: K o e^G, Q o e^G, K o e^{G_C - G}
-  float *TB, *P;         // [slots][H][C][C]: T diag(b), P
+  float *W, *Qp, *Kh;    // [slots][H][C][dk]: T diag(b) (K o e^G), Q o e^G - P W, K o e^{G_C - G}
+  float *Ut, *Ot;        // [slots][H][C][dv]: U~ = T diag(b) V, O~ = P U~
   float* EGC;            // [slots][H][dk]: e^{G_C}
   long long n_slots;
 };
@@ -599,12 +600,16 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_kernel(const Param
 }
 
 // ---------------------------------------------------------------- two launches
-// With a workspace the chunk-parallel part of the form (the decayed operands,
-// A, P and T) runs once per (chunk, head) in a launch of its own, and the
-// chains then walk their chunks with only the state-dependent products:
-//     X = V - (K o e^G) Sigma_0,  U = T diag(b) X,
-//     O = scale ((Q o e^G) Sigma_0 + P U),
-//     Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U.
+// With a workspace the chunk-parallel part of the form runs once per (chunk,
+// head) in a launch of its own: the decayed operands, A, P, T and the
+// state-independent products
+//     W = T diag(b) (K o e^G),  U~ = T diag(b) V,
+//     Q' = Q o e^G - P W,       O~ = P U~,
+// and the chains then walk their chunks with only the state-dependent ones:
+//     U = U~ - W Sigma_0,  O = scale (Q' Sigma_0 + O~),
+//     Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
+// (the same U and O as T diag(b) (V - (K o e^G) Sigma_0) and
+// scale ((Q o e^G) Sigma_0 + P U)).
 // Chunk c of sequence s (first token t0_s) has workspace slot
 // floor(t0_s / C) + s + c: no two chunks share one, and every slot is below
 // floor(total / C) + n_seq.
@@ -622,9 +627,11 @@ struct PrepPlan {
   static constexpr int GC = B + C;                 // DK
   static constexpr int MID = GC + DK;              // 3 x DK
   static constexpr int SX = MID + 3 * DK + 4;      // 3 x 256: the blocked solve's sums
-  static constexpr int FLOATS = SX + 3 * 256;
+  static constexpr int VST = SX + 3 * 256;         // 2 x [C][64] V rows as loaded (io dtype)
+  static constexpr int FLOATS = VST + 2 * C * 64;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
+static_assert(PrepPlan<128>::BYTES <= 232448, "KDA prep shared memory");
 
 __device__ __forceinline__ void seq_range(const Params& p, int s, int& t0, int& t1, bool report) {
   if (p.cu_seqlens) {
@@ -694,6 +701,39 @@ __device__ __forceinline__ void st4(float* p, float a, float b, float c, float d
   *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
 }
 
+// acc[i][4 q + x] = sum over k < kend (a multiple of 4) of A[i][k] B[k][64 q + 4 cg + x]
+// for the four rows of A (stride LDC, read four k at a time) and NQ float4
+// column groups of B (rows of stride ldb).
+template <int NQ>
+__device__ __forceinline__ void tri_times(float (&acc)[4][4 * NQ], const float* A, const float* B, int ldb, int cg,
+                                          int kend) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < 4 * NQ; ++c) acc[i][c] = 0.f;
+#pragma unroll 2
+  for (int k = 0; k < kend; k += 4) {
+    float4 a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = lds4(A + i * LDC + k);
+    float4 b[4][NQ];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) b[kk][q] = lds4(B + (k + kk) * ldb + 64 * q + 4 * cg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        float* o = acc[i] + 4 * q;
+        o[0] = fmaf(a[i].w, b[3][q].x, fmaf(a[i].z, b[2][q].x, fmaf(a[i].y, b[1][q].x, fmaf(a[i].x, b[0][q].x, o[0]))));
+        o[1] = fmaf(a[i].w, b[3][q].y, fmaf(a[i].z, b[2][q].y, fmaf(a[i].y, b[1][q].y, fmaf(a[i].x, b[0][q].y, o[1]))));
+        o[2] = fmaf(a[i].w, b[3][q].z, fmaf(a[i].z, b[2][q].z, fmaf(a[i].y, b[1][q].z, fmaf(a[i].x, b[0][q].z, o[2]))));
+        o[3] = fmaf(a[i].w, b[3][q].w, fmaf(a[i].z, b[2][q].w, fmaf(a[i].y, b[1][q].w, fmaf(a[i].x, b[0][q].w, o[3]))));
+      }
+  }
+}
+
 // One CTA per (chunk slot, head): the chunk's operands into the workspace.
 // Each thread holds four channels (4 dq .. 4 dq + 3) of RPT consecutive rows
 // in registers (read from the staged rows): the decay prefix runs
@@ -731,6 +771,18 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
   // flight at once; rows past the sequence end read nothing (zero fill)
   constexpr bool kF32 = sizeof(T) == 4;
   constexpr int RAW_LD = kF32 ? LDK : DK / 2;      // floats per staged q / k row
+  // 64 columns of the chunk's V rows (io dtype) into staging buffer `buf`
+  const T* v = static_cast<const T*>(p.v);
+  constexpr int VROW = 64 * (int)sizeof(T) / 4;    // floats per staged V row
+  auto stage_v = [&](int vb, int buf) {
+    constexpr int VP = 64 * (int)sizeof(T) / 16;   // 16-byte pieces per row
+    for (int e = tid; e < C * VP; e += THREADS) {
+      const int i = e / VP, c = e % VP;
+      const T* src = v + ((size_t)(tok0 + min(i, valid - 1)) * H + h) * p.dv + vb;
+      cp_async16_or_zero(sm + PL::VST + buf * C * 64 + i * VROW + 4 * c, reinterpret_cast<const char*>(src) + 16 * c,
+                         i < valid);
+    }
+  };
   float* rq = kF32 ? sQ : sm + PL::T;
   float* rk = kF32 ? sK : sm + PL::P;
   {
@@ -746,6 +798,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
       const size_t off = ((size_t)(tok0 + min(i, valid - 1)) * H + h) * DK;
       cp_async16_or_zero(sG + i * LDK + c, p.a + off + c, i < valid);
     }
+    stage_v(0, 0);
     cp_async_commit();
   }
   if (tid < C) sb[tid] = (tid < valid) ? p.b[(size_t)(tok0 + tid) * H + h] : 0.f;
@@ -830,12 +883,11 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
     for (int c = 0; c < 4; ++c) g[r][c] += off[c];
   const bool factored = !__syncthreads_or(wide);
   // ---- the decayed operands: factored ones to shared memory (K^ over K, K~
-  // over G, Q~ over Q) or the plain K, Q, G; K o e^G, Q o e^G and
-  // K o e^{G_C - G} to the workspace
+  // over G, Q~ over Q, e^m per channel) or the plain K, Q, G;
+  // K o e^{G_C - G} and e^{G_C} to the workspace
   const size_t w = (size_t)slot * H + h;
-  float* kg = p.ws.KG + w * C * DK;
-  float* qg = p.ws.QG + w * C * DK;
   float* kh = p.ws.Kh + w * C * DK;
+  float* sEm = sm + PL::MID;                       // [DK] e^m of a factored chunk
   if (factored) {
     float em[4], ec[4];
 #pragma unroll
@@ -843,6 +895,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
       em[c] = expf(mid[c]);
       ec[c] = expf(gc[c] - mid[c]);
     }
+    if (rg == 0) st4(sEm + d0, em[0], em[1], em[2], em[3]);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       float kt[4], kc[4], qt[4];
@@ -858,27 +911,18 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
       st4(sK + i * LDK + d0, kc[0], kc[1], kc[2], kc[3]);
       st4(sG + i * LDK + d0, kt[0], kt[1], kt[2], kt[3]);
       st4(sQ + i * LDK + d0, qt[0], qt[1], qt[2], qt[3]);
-      st4(kg + i * DK + d0, kt[0] * em[0], kt[1] * em[1], kt[2] * em[2], kt[3] * em[3]);
-      st4(qg + i * DK + d0, qt[0] * em[0], qt[1] * em[1], qt[2] * em[2], qt[3] * em[3]);
       st4(kh + i * DK + d0, kc[0] * ec[0], kc[1] * ec[1], kc[2] * ec[2], kc[3] * ec[3]);
     }
   } else {
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
-      float a1[4], a2[4], a3[4];
+      float a3[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float eg = expf(g[r][c]);
-        a1[c] = kr[r][c] * eg;
-        a2[c] = qr[r][c] * eg;
-        a3[c] = kr[r][c] * expf(gc[c] - g[r][c]);
-      }
+      for (int c = 0; c < 4; ++c) a3[c] = kr[r][c] * expf(gc[c] - g[r][c]);
       const int i = i0 + r;
       st4(sK + i * LDK + d0, kr[r][0], kr[r][1], kr[r][2], kr[r][3]);
       st4(sQ + i * LDK + d0, qr[r][0], qr[r][1], qr[r][2], qr[r][3]);
       st4(sG + i * LDK + d0, g[r][0], g[r][1], g[r][2], g[r][3]);
-      st4(kg + i * DK + d0, a1[0], a1[1], a1[2], a1[3]);
-      st4(qg + i * DK + d0, a2[0], a2[1], a2[2], a2[3]);
       st4(kh + i * DK + d0, a3[0], a3[1], a3[2], a3[3]);
     }
   }
@@ -889,24 +933,113 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
   if (factored) ap_factored<DK, PL>(sm, tid);
   else ap_exact<DK, PL>(sm, tid);
   __syncthreads();
-  // ---- P to the workspace; T = (I + A)^{-1} by 16 x 16 blocks
-  float4* pp = reinterpret_cast<float4*>(p.ws.P + w * C * C);
-  for (int e = tid; e < C * C / 4; e += THREADS) {
-    const int i = e / (C / 4), j = 4 * (e % (C / 4));
-    pp[e] = lds4(sm + PL::P + i * LDC + j);
-  }
+  // ---- T = (I + A)^{-1} by 16 x 16 blocks
   solve_blocked(sm + PL::A, sT, sm + PL::SX, tid);
-  // ---- T diag(b) to the workspace
-  float4* tb = reinterpret_cast<float4*>(p.ws.TB + w * C * C);
+  // ---- a chunk decayed term by term: K o e^G over G, Q o e^G over Q (a
+  // factored one keeps K~ and Q~, and its e^m scales W's and Q''s columns);
+  // T diag(b) over T
+  if (!factored) {
+#pragma unroll 4
+    for (int e = tid; e < C * DK / 4; e += THREADS) {
+      const int i = e / (DK / 4), d = 4 * (e % (DK / 4));
+      const float4 gg = lds4(sG + i * LDK + d), kk = lds4(sK + i * LDK + d), qq = lds4(sQ + i * LDK + d);
+      const float e0 = expf(gg.x), e1 = expf(gg.y), e2 = expf(gg.z), e3 = expf(gg.w);
+      st4(sG + i * LDK + d, kk.x * e0, kk.y * e1, kk.z * e2, kk.w * e3);
+      st4(sQ + i * LDK + d, qq.x * e0, qq.y * e1, qq.z * e2, qq.w * e3);
+    }
+  }
+#pragma unroll 4
   for (int e = tid; e < C * C / 4; e += THREADS) {
     const int i = e / (C / 4), j = 4 * (e % (C / 4));
-    float4 t = lds4(sT + i * LDC + j);
-    const float4 b = lds4(sb + j);
-    t.x *= b.x;
-    t.y *= b.y;
-    t.z *= b.z;
-    t.w *= b.w;
-    tb[e] = t;
+    const float4 t = lds4(sT + i * LDC + j), b = lds4(sb + j);
+    st4(sT + i * LDC + j, t.x * b.x, t.y * b.y, t.z * b.z, t.w * b.w);
+  }
+  __syncthreads();
+  // Products with a lower-triangular left factor (T diag(b) or P): thread rows
+  // r0 .. r0 + 3 of the 8-row band `band`, columns 64 q + 4 cg ..; warp w takes
+  // band w (w < 4) or 11 - w, so the two warps of each scheduler share out the
+  // triangle evenly.
+  const int wp = tid >> 5, lane = tid & 31;
+  const int band = (wp < 4) ? wp : 11 - wp;
+  const int r0 = 8 * band + 4 * (lane >> 4), cg = lane & 15, kend = 8 * band + 8;
+  const float* sP = sm + PL::P;
+  // ---- W = T diag(b) (K o e^G) (factored: (T diag(b) K~) e^m), over K^
+  // (its readers, the products, are done)
+  {
+    float acc[4][DK / 16];
+    tri_times<DK / 64>(acc, sT + r0 * LDC, sG, LDK, cg, kend);
+    float* gw = p.ws.W + w * C * DK;
+#pragma unroll
+    for (int q = 0; q < DK / 64; ++q) {
+      const float4 em = factored ? lds4(sEm + 64 * q + 4 * cg) : make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float* a = acc[i] + 4 * q;
+        a[0] *= em.x;
+        a[1] *= em.y;
+        a[2] *= em.z;
+        a[3] *= em.w;
+        st4(sK + (r0 + i) * LDK + 64 * q + 4 * cg, a[0], a[1], a[2], a[3]);
+        st4(gw + (r0 + i) * DK + 64 * q + 4 * cg, a[0], a[1], a[2], a[3]);
+      }
+    }
+  }
+  __syncthreads();
+  // ---- Q' = Q o e^G - P W
+  {
+    float acc[4][DK / 16];
+    tri_times<DK / 64>(acc, sP + r0 * LDC, sK, LDK, cg, kend);
+    float* gq = p.ws.Qp + w * C * DK;
+#pragma unroll
+    for (int q = 0; q < DK / 64; ++q) {
+      const float4 em = factored ? lds4(sEm + 64 * q + 4 * cg) : make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 qg = lds4(sQ + (r0 + i) * LDK + 64 * q + 4 * cg);
+        st4(gq + (r0 + i) * DK + 64 * q + 4 * cg, fmaf(qg.x, em.x, -acc[i][4 * q]),
+            fmaf(qg.y, em.y, -acc[i][4 * q + 1]), fmaf(qg.z, em.z, -acc[i][4 * q + 2]),
+            fmaf(qg.w, em.w, -acc[i][4 * q + 3]));
+      }
+    }
+  }
+  // ---- per 64 columns of v (staged two blocks deep; block 0 came with q, k
+  // and a): U~ = T diag(b) V (V as fp32 over A, U~ over G), then O~ = P U~
+  float* sVb = sm + PL::A;
+  float* sUb = sG;
+  float* gut = p.ws.Ut + w * C * (size_t)p.dv;
+  float* got = p.ws.Ot + w * C * (size_t)p.dv;
+  for (int vb = 0, buf = 0; vb < p.dv; vb += 64, buf ^= 1) {
+    if (vb + 64 < p.dv) stage_v(vb + 64, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();                            // this block's rows
+    __syncthreads();                               // and the last block's readers are done
+#pragma unroll 4
+    for (int e = tid; e < C * 16; e += THREADS) {
+      const int i = e >> 4, c = 4 * (e & 15);
+      const float* raw = sm + PL::VST + buf * C * 64 + i * VROW;
+      float x[4];
+      if constexpr (kF32) ldv<4>(raw + c, x);
+      else lds_bf16x4(raw + c / 2, x);
+      st4(sVb + i * LDC + c, x[0], x[1], x[2], x[3]);
+    }
+    __syncthreads();
+    {
+      float acc[4][4];
+      tri_times<1>(acc, sT + r0 * LDC, sVb, LDC, cg, kend);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        st4(sUb + (r0 + i) * LDC + 4 * cg, acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        st4(gut + (size_t)(r0 + i) * p.dv + vb + 4 * cg, acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      }
+    }
+    __syncthreads();
+    {
+      float acc[4][4];
+      tri_times<1>(acc, sP + r0 * LDC, sUb, LDC, cg, kend);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        st4(got + (size_t)(r0 + i) * p.dv + vb + 4 * cg, acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    }
   }
 }
 
@@ -937,31 +1070,27 @@ __device__ __forceinline__ void rows_times(float (&acc)[4][TN], const float* A, 
 }
 
 // A chain's state slice of NV = 16 columns, the chunk's operands (single
-// buffers, each refilled with cp.async as soon as its last reader is done),
-// the V rows in the io dtype, and the partial sums of the split products.
-template <int DK, typename T>
+// buffers, each refilled with cp.async as soon as its last reader is done)
+// and the partial sums of the split products.
+template <int DK>
 struct ChainPlan {
   static constexpr int NV = 16;
   static constexpr int LDK = DK + 4;
   static constexpr int LDS = NV + 4;               // [rows][NV] fp32 tiles
-  static constexpr int VROW = (NV * (int)sizeof(T) + 16) / 4;   // floats per V row
-  static constexpr int RROWS = C + DK;             // rows of one group's partial sums
-  static constexpr int KG = 0;                     // [C][LDK]  K o e^G
-  static constexpr int QG = KG + C * LDK;          // [C][LDK]  Q o e^G
-  static constexpr int KH = QG + C * LDK;          // [C][LDK]  K o e^{G_C - G}
-  static constexpr int TB = KH + C * LDK;          // [C][LDC]  T diag(b)
-  static constexpr int P = TB + C * LDC;           // [C][LDC]
-  static constexpr int SIG = P + C * LDC;          // [DK][LDS]
-  static constexpr int X = SIG + DK * LDS;         // [C][LDS]  V - (K o e^G) Sigma_0
-  static constexpr int U = X + C * LDS;            // [C][LDS]
-  static constexpr int OQ = U + C * LDS;           // [C][LDS]  (Q o e^G) Sigma_0
-  static constexpr int RED = OQ + C * LDS;         // [4][RROWS][NV] partial sums (swizzled)
+  static constexpr int RROWS = (2 * C > DK) ? 2 * C : DK;   // rows of one group's partial sums
+  static constexpr int W = 0;                      // [C][LDK]  T diag(b) (K o e^G)
+  static constexpr int QP = W + C * LDK;           // [C][LDK]  Q o e^G - P W
+  static constexpr int KH = QP + C * LDK;          // [C][LDK]  K o e^{G_C - G}
+  static constexpr int SIG = KH + C * LDK;         // [DK][LDS]
+  static constexpr int U = SIG + DK * LDS;         // [C][LDS]
+  static constexpr int UT = U + C * LDS;           // [C][LDS]  U~ slice
+  static constexpr int OT = UT + C * LDS;          // [C][LDS]  O~ slice
+  static constexpr int RED = OT + C * LDS;         // [4][RROWS][NV] partial sums (swizzled)
   static constexpr int EGC = RED + 4 * RROWS * NV; // [2][DK]  e^{G_C}, by chunk parity
-  static constexpr int V = EGC + 2 * DK;           // [C][VROW]
-  static constexpr int FLOATS = V + C * VROW;
+  static constexpr int FLOATS = EGC + 2 * DK;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
-static_assert(ChainPlan<128, float>::BYTES <= 232448, "KDA chain shared memory");
+static_assert(ChainPlan<128>::BYTES <= 232448, "KDA chain shared memory");
 
 // Offset of (row, float4 column c4) in one group's partial sums: rows of 16
 // floats, the two rows of an even/odd pair swapped when bit 2 xor bit 3 of
@@ -979,28 +1108,26 @@ __device__ __forceinline__ void add4(float4& a, float4 b) {
 }
 
 // One CTA per (sequence, head, 16-column dv slice): the chain through its
-// chunks, operands from the workspace.  The two products over dk and the two
-// over the chunk's rows each split their contraction over four groups of 64
-// threads (4 x 4 register tiles, partial sums reduced through shared memory).
+// chunks, operands from the workspace.  W Sigma_0 and Q' Sigma_0 share one
+// pass over the state, and the carry's product follows; each splits its
+// contraction over four groups of 64 threads (4 x 4 register tiles, partial
+// sums reduced through shared memory).
 template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const Params p) {
-  using PL = ChainPlan<DK, T>;
+  using PL = ChainPlan<DK>;
   constexpr int NV = PL::NV, LDK = PL::LDK, LDS = PL::LDS;
   constexpr int RG_FLOATS = PL::RROWS * NV;        // one group's partial sums
   constexpr int TD = DK / 16;                      // carry rows per thread
   extern __shared__ __align__(16) float sm[];
-  float* sKG = sm + PL::KG;
-  float* sQG = sm + PL::QG;
+  float* sW = sm + PL::W;
+  float* sQp = sm + PL::QP;
   float* sKh = sm + PL::KH;
-  float* sTB = sm + PL::TB;
-  float* sP = sm + PL::P;
   float* sSig = sm + PL::SIG;
-  float* sX = sm + PL::X;
   float* sU = sm + PL::U;
-  float* sOq = sm + PL::OQ;
+  float* sUt = sm + PL::UT;
+  float* sOt = sm + PL::OT;
   float* sRed = sm + PL::RED;
   float* sEGC = sm + PL::EGC;
-  float* sV = sm + PL::V;
 
   const int tid = threadIdx.x;
   const int n_slices = p.dv / NV;
@@ -1015,44 +1142,42 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
   const long long slot0 = slot_base(seq, t0);
   const int col0 = slice * NV;
   const size_t sbase = ((size_t)seq * H + h) * DK * (size_t)dv + col0;
-  const T* v = static_cast<const T*>(p.v);
   T* o = static_cast<T*>(p.o);
 
   // Operand groups of chunk c, one cp.async group each (empty past the last
-  // chunk): A, the dk products' (K o e^G, Q o e^G, V rows); B, U's
-  // (T diag(b)); C, the row products' (P, K o e^{G_C - G}, e^{G_C}).
-  auto load_a = [&](int c) {
+  // chunk): A1, the state pass's (W, Q'); A2, its reduction's (the U~ and O~
+  // slices); B, the carry's (K o e^{G_C - G}, e^{G_C}).
+  auto load_a1 = [&](int c) {
     if (c < n_chunks) {
       const size_t w = (size_t)(slot0 + c) * H + h;
-      copy_rows<C, DK, LDK>(sKG, p.ws.KG + w * C * DK, tid);
-      copy_rows<C, DK, LDK>(sQG, p.ws.QG + w * C * DK, tid);
-      const int tok0 = t0 + c * C, valid = min(C, t1 - tok0);
-      constexpr int PIECES = NV * (int)sizeof(T) / 16;
-      for (int e = tid; e < C * PIECES; e += THREADS) {
-        const int i = e / PIECES, q = e % PIECES;
-        const T* src = v + ((size_t)(tok0 + min(i, valid - 1)) * H + h) * dv + col0;
-        cp_async16_or_zero(sV + i * PL::VROW + 4 * q, reinterpret_cast<const char*>(src) + 16 * q, i < valid);
+      copy_rows<C, DK, LDK>(sW, p.ws.W + w * C * DK, tid);
+      copy_rows<C, DK, LDK>(sQp, p.ws.Qp + w * C * DK, tid);
+    }
+    cp_async_commit();
+  };
+  auto load_a2 = [&](int c) {
+    if (c < n_chunks) {
+      const size_t base = ((size_t)(slot0 + c) * H + h) * C * (size_t)dv + col0;
+      for (int e = tid; e < 2 * C * (NV / 4); e += THREADS) {
+        const int m = e / (C * (NV / 4)), r = e % (C * (NV / 4));
+        const int i = r / (NV / 4), q = r % (NV / 4);
+        cp_async16((m ? sOt : sUt) + i * LDS + 4 * q, (m ? p.ws.Ot : p.ws.Ut) + base + (size_t)i * dv + 4 * q);
       }
     }
     cp_async_commit();
   };
   auto load_b = [&](int c) {
-    if (c < n_chunks) copy_rows<C, C, LDC>(sTB, p.ws.TB + (size_t)((slot0 + c) * H + h) * C * C, tid);
-    cp_async_commit();
-  };
-  auto load_c = [&](int c) {
     if (c < n_chunks) {
       const size_t w = (size_t)(slot0 + c) * H + h;
-      copy_rows<C, C, LDC>(sP, p.ws.P + w * C * C, tid);
       copy_rows<C, DK, LDK>(sKh, p.ws.Kh + w * C * DK, tid);
       if (tid < DK / 4) cp_async16(sEGC + (c & 1) * DK + 4 * tid, p.ws.EGC + w * DK + 4 * tid);
     }
     cp_async_commit();
   };
 
-  load_a(0);
+  load_a1(0);
+  load_a2(0);
   load_b(0);
-  load_c(0);
   for (int e = tid; e < DK * NV; e += THREADS) {
     const int d = e / NV, c = e % NV;
     sSig[d * LDS + c] = p.S0 ? p.S0[sbase + (size_t)d * dv + c] : 0.f;
@@ -1061,31 +1186,32 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
   const int g = tid >> 6, rt = (tid & 63) >> 2, ct = tid & 3;
   const int r0 = 4 * rt, c0 = 4 * ct;
   float* red = sRed + g * RG_FLOATS;
-  // Groups in flight at each wait, oldest first: [A c, B c, C c] before the dk
-  // products, [B c, C c] before U, [C c, A c+1] before the row products; a
-  // refill is issued only after the barrier that ends its buffer's last reader.
+  // Groups in flight at each wait, oldest first: [A1 c, A2 c, B c] before the
+  // state pass, [A2 c, B c] before its reduction, [B c, A1 c+1] before the
+  // carry; a refill is issued only after the barrier that ends its buffers'
+  // last reader.
   for (int c = 0; c < n_chunks; ++c) {
     const int tok0 = t0 + c * C, valid = min(C, t1 - tok0);
-    cp_async_wait<2>();                            // the dk products' group
+    cp_async_wait<2>();                            // W and Q'
     __syncthreads();
-    // ---- (K o e^G) Sigma_0 and (Q o e^G) Sigma_0, dk split four ways
+    // ---- W Sigma_0 and Q' Sigma_0, dk split four ways
     {
       float ax[4][4] = {}, aq[4][4] = {};
       constexpr int KR = DK / 4;
 #pragma unroll 2
       for (int k = g * KR; k < (g + 1) * KR; k += 4) {
-        float4 kx[4], qx[4];
+        float4 wx[4], qx[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          kx[i] = lds4(sKG + (r0 + i) * LDK + k);
-          qx[i] = lds4(sQG + (r0 + i) * LDK + k);
+          wx[i] = lds4(sW + (r0 + i) * LDK + k);
+          qx[i] = lds4(sQp + (r0 + i) * LDK + k);
         }
         float b[4][4];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) ldv<4>(sSig + (k + kk) * LDS + c0, b[kk]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          fma4<4>(ax[i], kx[i], b);
+          fma4<4>(ax[i], wx[i], b);
           fma4<4>(aq[i], qx[i], b);
         }
       }
@@ -1095,8 +1221,11 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
         stv<4>(red + red_off(C + r0 + i, ct), aq[i]);
       }
     }
+    cp_async_wait<1>();                            // the U~ and O~ slices
     __syncthreads();
-    // ---- reduce: X = V - sum -> sX, the Q part -> sOq
+    load_a1(c + 1);
+    // ---- reduce: U = U~ - sum -> sU; O = scale (sum + O~) with the output
+    // gate and the loop residual
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int e = tid + THREADS * m;
@@ -1106,42 +1235,41 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
 #pragma unroll
       for (int gg = 1; gg < 4; ++gg) add4(s, lds4(sRed + gg * RG_FLOATS + off));
       if (row < C) {
-        const T* vr = reinterpret_cast<const T*>(sV + row * PL::VROW) + 4 * c4;
-        s = make_float4(to_f32(vr[0]) - s.x, to_f32(vr[1]) - s.y, to_f32(vr[2]) - s.z, to_f32(vr[3]) - s.w);
-        *reinterpret_cast<float4*>(sX + row * LDS + 4 * c4) = s;
+        const float4 ut = lds4(sUt + row * LDS + 4 * c4);
+        *reinterpret_cast<float4*>(sU + row * LDS + 4 * c4) =
+            make_float4(ut.x - s.x, ut.y - s.y, ut.z - s.z, ut.w - s.w);
       } else {
-        *reinterpret_cast<float4*>(sOq + (row - C) * LDS + 4 * c4) = s;
+        const int r = row - C;
+        if (r < valid) {
+          add4(s, lds4(sOt + r * LDS + 4 * c4));
+          const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + r) * H + h])) : 1.f;
+          const float sv[4] = {s.x, s.y, s.z, s.w};
+          const size_t obase = ((size_t)(tok0 + r) * H + h) * dv + col0 + 4 * c4;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float y = p.scale * sv[j];
+            if (p.gate) y *= og;
+            if (p.h_prev) {
+              const float hp = to_f32(static_cast<const T*>(p.h_prev)[obase + j]);
+              y = fmaf(p.rho[(size_t)h * dv + col0 + 4 * c4 + j], hp, to_f32(from_f32<T>(y)));
+            }
+            o[obase + j] = from_f32<T>(y);
+          }
+        }
       }
     }
-    cp_async_wait<1>();                            // U's group (the row products' may fly)
+    cp_async_wait<1>();                            // the carry's group
     __syncthreads();
-    load_a(c + 1);
-    // ---- U = T diag(b) X (lower triangular: columns < row + 1); rows
-    // 4 (tid / 16) .., column tid % 16
+    load_a2(c + 1);
+    // ---- (K o e^{G_C - G})^T U, the chunk's rows split four ways
     {
-      const int ur0 = 4 * (tid >> 4), uc = tid & 15;
-      float acc[4][1] = {};
-      rows_times<1>(acc, sTB + ur0 * LDC, LDC, sX + uc, LDS, ur0 + 4);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sU[(ur0 + i) * LDS + uc] = acc[i][0];
-    }
-    cp_async_wait<1>();                            // the row products' group
-    __syncthreads();
-    load_b(c + 1);
-    // ---- P U and (K o e^{G_C - G})^T U, the chunk's rows split four ways
-    {
-      float ao[4][4] = {}, as[TD][4] = {};
+      float as[TD][4] = {};
       const int d0 = TD * rt;
 #pragma unroll 1
       for (int i = 16 * g; i < 16 * g + 16; i += 4) {
-        float4 pr[4];
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) pr[ii] = lds4(sP + (r0 + ii) * LDC + i);
         float u[4][4];
 #pragma unroll
         for (int x = 0; x < 4; ++x) ldv<4>(sU + (i + x) * LDS + c0, u[x]);
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) fma4<4>(ao[ii], pr[ii], u);
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
 #pragma unroll
@@ -1156,46 +1284,24 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
         }
       }
 #pragma unroll
-      for (int ii = 0; ii < 4; ++ii) stv<4>(red + red_off(r0 + ii, ct), ao[ii]);
-#pragma unroll
-      for (int e = 0; e < TD; ++e) stv<4>(red + red_off(C + d0 + e, ct), as[e]);
+      for (int e = 0; e < TD; ++e) stv<4>(red + red_off(d0 + e, ct), as[e]);
     }
     __syncthreads();
-    load_c(c + 1);
-    // ---- reduce: O = scale ((Q o e^G) Sigma_0 + P U) with the output gate and
-    // the loop residual; Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
+    load_b(c + 1);
+    // ---- reduce: Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
     const float* egc = sEGC + (c & 1) * DK;
 #pragma unroll
-    for (int m = 0; m < (C + DK) / 64; ++m) {
+    for (int m = 0; m < DK / 64; ++m) {
       const int e = tid + THREADS * m;
-      const int row = e >> 2, c4 = e & 3;
-      const int off = red_off(row, c4);
+      const int d = e >> 2, c4 = e & 3;
+      const int off = red_off(d, c4);
       float4 s = lds4(sRed + off);
 #pragma unroll
       for (int gg = 1; gg < 4; ++gg) add4(s, lds4(sRed + gg * RG_FLOATS + off));
-      if (row < C) {
-        if (row >= valid) continue;
-        add4(s, lds4(sOq + row * LDS + 4 * c4));
-        const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + row) * H + h])) : 1.f;
-        const float sv[4] = {s.x, s.y, s.z, s.w};
-        const size_t obase = ((size_t)(tok0 + row) * H + h) * dv + col0 + 4 * c4;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float y = p.scale * sv[j];
-          if (p.gate) y *= og;
-          if (p.h_prev) {
-            const float hp = to_f32(static_cast<const T*>(p.h_prev)[obase + j]);
-            y = fmaf(p.rho[(size_t)h * dv + col0 + 4 * c4 + j], hp, to_f32(from_f32<T>(y)));
-          }
-          o[obase + j] = from_f32<T>(y);
-        }
-      } else {
-        const int d = row - C;
-        float4* sg = reinterpret_cast<float4*>(sSig + d * LDS + 4 * c4);
-        const float4 old = *sg;
-        const float gd = egc[d];
-        *sg = make_float4(fmaf(gd, old.x, s.x), fmaf(gd, old.y, s.y), fmaf(gd, old.z, s.z), fmaf(gd, old.w, s.w));
-      }
+      float4* sg = reinterpret_cast<float4*>(sSig + d * LDS + 4 * c4);
+      const float4 old = *sg;
+      const float gd = egc[d];
+      *sg = make_float4(fmaf(gd, old.x, s.x), fmaf(gd, old.y, s.y), fmaf(gd, old.z, s.z), fmaf(gd, old.w, s.w));
     }
   }
   cp_async_wait<0>();
@@ -1223,7 +1329,7 @@ static cudaError_t launch_two(const Params& kp, long long chunk_blocks, long lon
                               cudaStream_t stream) {
   static std::atomic<bool> set_prep[kMaxDevices], set_chain[kMaxDevices];
   constexpr size_t prep_bytes = PrepPlan<DK>::BYTES;
-  constexpr size_t chain_bytes = ChainPlan<DK, T>::BYTES;
+  constexpr size_t chain_bytes = ChainPlan<DK>::BYTES;
   cudaError_t e = smem_attr_once(set_prep, gdn_prefill_kda_prep_kernel<DK, T>, prep_bytes);
   if (e == cudaSuccess) e = smem_attr_once(set_chain, gdn_prefill_kda_chain_kernel<DK, T>, chain_bytes);
   if (e != cudaSuccess) return e;
@@ -1238,13 +1344,13 @@ static long long n_slots(const gdn_fwd_params* p) { return (long long)p->total_t
 
 }  // namespace kda
 
-// Bytes of the two-launch schedule's workspace: K o e^G, Q o e^G and
-// K o e^{G_C - G} ([slots][H][C][dk] fp32 each), T diag(b) and P
-// ([slots][H][C][C]) and e^{G_C} ([slots][H][dk]).
+// Bytes of the two-launch schedule's workspace: W, Q' and K o e^{G_C - G}
+// ([slots][H][C][dk] fp32 each), U~ and O~ ([slots][H][C][dv]) and e^{G_C}
+// ([slots][H][dk]).
 size_t prefill_kda_workspace(const gdn_fwd_params* p) {
   const size_t sh = (size_t)kda::n_slots(p) * p->H;
-  const size_t dk = (size_t)p->dk, c = kda::C;
-  return 3 * kda::align256(sh * c * dk * 4) + 2 * kda::align256(sh * c * c * 4) + kda::align256(sh * dk * 4);
+  const size_t dk = (size_t)p->dk, dv = (size_t)p->dv, c = kda::C;
+  return 3 * kda::align256(sh * c * dk * 4) + 2 * kda::align256(sh * c * dv * 4) + kda::align256(sh * dk * 4);
 }
 
 gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, void* ws, cudaStream_t stream) {
@@ -1280,15 +1386,16 @@ gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, void* w
     const size_t sh = (size_t)n_slots * p->H;
     const size_t dk = (size_t)p->dk, c = kda::C;
     char* w = static_cast<char*>(ws);
-    float** arrays[] = {&kp.ws.KG, &kp.ws.QG, &kp.ws.Kh};
-    for (float** a : arrays) {
+    float** rows_dk[] = {&kp.ws.W, &kp.ws.Qp, &kp.ws.Kh};
+    for (float** a : rows_dk) {
       *a = reinterpret_cast<float*>(w);
       w += kda::align256(sh * c * dk * 4);
     }
-    kp.ws.TB = reinterpret_cast<float*>(w);
-    w += kda::align256(sh * c * c * 4);
-    kp.ws.P = reinterpret_cast<float*>(w);
-    w += kda::align256(sh * c * c * 4);
+    float** rows_dv[] = {&kp.ws.Ut, &kp.ws.Ot};
+    for (float** a : rows_dv) {
+      *a = reinterpret_cast<float*>(w);
+      w += kda::align256(sh * c * (size_t)p->dv * 4);
+    }
     kp.ws.EGC = reinterpret_cast<float*>(w);
     kp.ws.n_slots = n_slots;
     const long long chunk_blocks = n_slots * p->H;

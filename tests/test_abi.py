@@ -414,16 +414,17 @@ def test_channel_gate_flag_validation(lib):
     """GDN_CHANNEL_GATE (per-channel decay, a [tokens][H][dk]) is accepted by
     prefill and decode; the output may not overlap any of a's dk-wide rows.
     The prefill takes two launches with a workspace (one slot per chunk:
-    floor(total / 64) + n_seq + 1 slots per head) and one without."""
+    floor(total / 64) + n_seq + 1 slots per head, each holding three
+    64 x dk and two 64 x dv fp32 arrays and dk decays) and one without."""
     p = _params(n_seq=1, seq_len=4096, total_tokens=4096, H=16, flags=B.GDN_CHANNEL_GATE)
 
     def al(x):
         return (x + 255) // 256 * 256
 
-    for dk in (128, 64):
-        p.dk = dk
+    for dk, dv in ((128, 128), (64, 256)):
+        p.dk, p.dv = dk, dv
         sh = (4096 // 64 + 1 + 1) * 16
-        need = 3 * al(sh * 64 * dk * 4) + 2 * al(sh * 64 * 64 * 4) + al(sh * dk * 4)
+        need = 3 * al(sh * 64 * dk * 4) + 2 * al(sh * 64 * dv * 4) + al(sh * dk * 4)
         assert lib.gdn_chunk_fwd_workspace(ctypes.byref(p)) == need
     assert _schedule(lib, p) == (1, 0, 0, 2, 0)
     # a workspace smaller than the need, or a size without one, is refused on the host

@@ -597,7 +597,9 @@ def bench_kda(dev, args, peaks, world, L=4096, H=16):
     return {"tokens_per_s": world * L / t, "ms_per_step": t * 1e3, "loops": loops, "tokens": L, "heads": H,
             "achieved_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
             "clocks": clocks.summary(),
-            "kernel": "gdn_prefill_kda_kernel (first path: fp32 CUDA cores, one CTA per (sequence, head, 64 columns))"}
+            "kernel": "gdn_prefill_kda_prep_kernel (one CTA per chunk and head: decayed operands, T, W, Q', "
+                      "U~, O~) + gdn_prefill_kda_chain_kernel (one CTA per (sequence, head, 16 columns)); "
+                      "fp32 CUDA cores"}
 
 
 def bench_backward(dev, args, peaks, world):

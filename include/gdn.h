@@ -148,8 +148,12 @@ typedef struct {
 
 /* Bytes of device workspace gdn_chunk_fwd needs for these parameters (may be 0).
  * Returns (size_t)-1 if the parameters are invalid.  The need is non-zero only
- * when the segmented schedule is chosen (see below); it is a function of the
- * shapes, flags and the current device's SM count. */
+ * when the segmented schedule or, with GDN_CHANNEL_GATE, the two-launch
+ * schedule is chosen (see below); it is a function of the shapes, flags and
+ * the current device's SM count.  For GDN_CHANNEL_GATE it is, with
+ * S = (floor(total_tokens / 64) + n_seq + 1) * H chunk slots and each array
+ * rounded up to 256 bytes, 3 arrays of S * 64 * dk fp32, 2 of S * 64 * dv and
+ * 1 of S * dk. */
 size_t gdn_chunk_fwd_workspace(const gdn_fwd_params *p);
 
 /* The schedule gdn_chunk_fwd takes for these parameters when it is given a
@@ -161,7 +165,7 @@ size_t gdn_chunk_fwd_workspace(const gdn_fwd_params *p);
  *   launches: stream operations the call enqueues: 0 (nothing to do), 1 (one
  *             pass, or the copy or clear of S_T when every sequence is empty),
  *             2 or 3 (see the schedules below; a varlen call with its length
- *             sort takes 2).
+ *             sort takes 2, a GDN_CHANNEL_GATE call with a workspace 2).
  *   corrected: 1 for the corrected segmented schedule, else 0.
  * Parameters gdn_chunk_fwd would reject return the same error status. */
 gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg0_tok,
@@ -194,11 +198,22 @@ gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg
  * launch sorts the sequences by length on the device (longest first, into the
  * workspace) and the blocks take them in that order, so that the longest
  * chains do not start last.  The outputs do not depend on the order.
+ * With GDN_CHANNEL_GATE (fp32 CUDA-core kernels, any io dtype) and a
+ * workspace, a first launch takes every (chunk, head) at once and writes its
+ * decayed operands, T = (I + A)^{-1} and the state-independent products
+ * W = T diag(b) (K o e^G), Q' = Q o e^G - P W, U~ = T diag(b) V and
+ * O~ = P U~ to the workspace; a second walks each (sequence, head, 16-wide
+ * dv slice) chain through its chunks with U = U~ - W S, O = scale (Q' S + O~)
+ * and the carry.  Without a workspace one launch does all of it per
+ * (sequence, head, 32-wide slice).  Both give the same outputs up to
+ * rounding.
  *
  * ws/ws_bytes: device workspace of at least gdn_chunk_fwd_workspace(p) bytes,
  * 256-byte aligned, owned by the caller and not read back afterwards.
  * ws == NULL with ws_bytes == 0 is always accepted and selects the one-pass
- * schedule; a non-NULL ws smaller than the need returns GDN_ERR_WORKSPACE. */
+ * schedule (the one-launch kernel for GDN_CHANNEL_GATE); a non-NULL ws
+ * smaller than the need returns GDN_ERR_WORKSPACE, and so does ws == NULL
+ * with ws_bytes != 0 when the chosen schedule needs a workspace. */
 gdn_status gdn_chunk_fwd(const gdn_fwd_params *p, void *ws, size_t ws_bytes,
                          cudaStream_t stream);
 
@@ -215,7 +230,9 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_params *p, void *ws, size_t ws_bytes,
  * 32 MiB (33554432 bytes) of device memory that every GPU which loads the
  * library holds until the process exits.  A call whose
  * gdn_chunk_fwd_workspace(p) exceeds that returns GDN_ERR_WORKSPACE without
- * launching anything; a call that needs no workspace runs as gdn_chunk_fwd.
+ * launching anything, except a GDN_CHANNEL_GATE call, which then runs the
+ * one-launch kernel (no workspace); a call that needs no workspace runs as
+ * gdn_chunk_fwd.
  * Nothing is allocated or freed.
  *
  * The first call on each device looks up the array's device address (with

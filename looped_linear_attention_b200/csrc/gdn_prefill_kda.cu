@@ -24,8 +24,10 @@
 // K^ = K o e^{m-G}, Q~ = Q o e^{G-m}: two exponentials per (i, c) instead of
 // one per (i, j, c).
 // Otherwise (a channel that decays hard or resets) the decay of each (i, j, c)
-// term is its own exponential, so every exponent is <= 0.  One CTA of 256
-// threads per (sequence, head, 32-column dv slice); the output epilogue
+// term is its own exponential, so every exponent is <= 0.  Without a
+// workspace one kernel (one CTA of 256 threads per (sequence, head, 32-column
+// dv slice)) does all of it; with one, a chunk-parallel launch and a chain
+// launch split it (the two-launch section below).  The output epilogue
 // (head-wise gate, loop residual) is the precise path's.
 #include "common.cuh"
 

@@ -1045,81 +1045,83 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
   }
 }
 
-// acc[j] += a . (b[0][j], b[1][j], b[2][j], b[3][j])
-template <int TN>
-__device__ __forceinline__ void fma4(float (&acc)[TN], float4 a, const float (&b)[4][TN]) {
-#pragma unroll
-  for (int j = 0; j < TN; ++j)
-    acc[j] = fmaf(a.w, b[3][j], fmaf(a.z, b[2][j], fmaf(a.y, b[1][j], fmaf(a.x, b[0][j], acc[j]))));
+// Warp-level m16n8k8 tf32 MMA (fp32 accumulate) with each operand split into
+// a tf32 high part and a tf32 remainder: a b ~= ah bh + ah bl + al bh, the
+// three partial products in separate accumulators, which keeps the products
+// close to fp32.
+__device__ __forceinline__ uint32_t tf32_hi(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
 }
-
-// acc[i][:] += sum over k < n (a multiple of 4) of A[r0 + i][k] B[k][c0 .. c0 + TN - 1]
-// (A rows of stride lda read four k at a time, B rows of stride ldb)
-template <int TN>
-__device__ __forceinline__ void rows_times(float (&acc)[4][TN], const float* A, int lda, const float* B, int ldb,
-                                           int n) {
-#pragma unroll 2
-  for (int k = 0; k < n; k += 4) {
-    float4 a[4];
+__device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
+  hi = tf32_hi(x);
+  lo = tf32_hi(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// acc[nt] += A (16 x 8, element (m, k) at A[m * lda_m + k * lda_k]) times
+// B (8 x 16, element (k, n) at B[k * LDB + n]) for k-step k0, fragments of
+// lane (g = lane / 4, q = lane % 4), both n-tiles.
+template <int LDB>
+__device__ __forceinline__ void mma_step(float (&acc)[2][3][4], const float* A, int lda_m, int lda_k, const float* B,
+                                         int k0, int g, int q) {
+  uint32_t ah[4], al[4];
+  tf32_split(A[g * lda_m + (k0 + q) * lda_k], ah[0], al[0]);
+  tf32_split(A[(g + 8) * lda_m + (k0 + q) * lda_k], ah[1], al[1]);
+  tf32_split(A[g * lda_m + (k0 + q + 4) * lda_k], ah[2], al[2]);
+  tf32_split(A[(g + 8) * lda_m + (k0 + q + 4) * lda_k], ah[3], al[3]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = lds4(A + i * lda + k);
-    float b[4][TN];
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) ldv<TN>(B + (k + kk) * ldb, b[kk]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) fma4<TN>(acc[i], a[i], b);
+  for (int nt = 0; nt < 2; ++nt) {
+    uint32_t bh[2], bl[2];
+    tf32_split(B[(k0 + q) * LDB + 8 * nt + g], bh[0], bl[0]);
+    tf32_split(B[(k0 + q + 4) * LDB + 8 * nt + g], bh[1], bl[1]);
+    mma_16x8x8(acc[nt][0], ah, bh);
+    mma_16x8x8(acc[nt][1], ah, bl);
+    mma_16x8x8(acc[nt][2], al, bh);
   }
 }
 
-// A chain's state slice of NV = 16 columns, the chunk's operands (single
-// buffers, each refilled with cp.async as soon as its last reader is done)
-// and the partial sums of the split products.
+// A chain's state slice of NV = 16 columns and the chunk's operands: W and Q'
+// by chunk parity (the next chunk's load while this one is used), the carry's
+// K o e^{G_C - G} and the U~ and O~ slices in single buffers.  Row strides
+// make every fragment read conflict-free: W and Q' rows (A, banks 4 g + q),
+// K o e^{G_C - G} rows read transposed (A, banks 8 q + g), the state and U
+// (B, banks 24 q + g).
 template <int DK>
 struct ChainPlan {
   static constexpr int NV = 16;
-  static constexpr int LDK = DK + 4;
-  static constexpr int LDS = NV + 4;               // [rows][NV] fp32 tiles
-  static constexpr int RROWS = (2 * C > DK) ? 2 * C : DK;   // rows of one group's partial sums
-  static constexpr int W = 0;                      // [C][LDK]  T diag(b) (K o e^G)
-  static constexpr int QP = W + C * LDK;           // [C][LDK]  Q o e^G - P W
-  static constexpr int KH = QP + C * LDK;          // [C][LDK]  K o e^{G_C - G}
-  static constexpr int SIG = KH + C * LDK;         // [DK][LDS]
+  static constexpr int LDA = DK + 4;
+  static constexpr int LDH = DK + 8;
+  static constexpr int LDS = NV + 8;
+  static constexpr int W = 0;                      // 2 x [C][LDA]  T diag(b) (K o e^G)
+  static constexpr int QP = W + 2 * C * LDA;       // 2 x [C][LDA]  Q o e^G - P W
+  static constexpr int KH = QP + 2 * C * LDA;      // [C][LDH]      K o e^{G_C - G}
+  static constexpr int SIG = KH + C * LDH;         // [DK][LDS]
   static constexpr int U = SIG + DK * LDS;         // [C][LDS]
-  static constexpr int UT = U + C * LDS;           // [C][LDS]  U~ slice
-  static constexpr int OT = UT + C * LDS;          // [C][LDS]  O~ slice
-  static constexpr int RED = OT + C * LDS;         // [4][RROWS][NV] partial sums (swizzled)
-  static constexpr int EGC = RED + 4 * RROWS * NV; // [2][DK]  e^{G_C}, by chunk parity
-  static constexpr int FLOATS = EGC + 2 * DK;
+  static constexpr int UT = U + C * LDS;           // [C][LDS]      U~ slice
+  static constexpr int OT = UT + C * LDS;          // [C][LDS]      O~ slice
+  static constexpr int EGC = OT + C * LDS;         // [DK]          e^{G_C}
+  static constexpr int FLOATS = EGC + DK;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 static_assert(ChainPlan<128>::BYTES <= 232448, "KDA chain shared memory");
 
-// Offset of (row, float4 column c4) in one group's partial sums: rows of 16
-// floats, the two rows of an even/odd pair swapped when bit 2 xor bit 3 of
-// the row is set, so that the tile writes (rows r and r + 4, or r and r + 8,
-// in one quarter warp) and the row-order reads are both conflict-free.
-__device__ __forceinline__ int red_off(int row, int c4) {
-  return (16 * row + 4 * c4) ^ ((((row >> 2) ^ (row >> 3)) & 1) << 4);
-}
-
-__device__ __forceinline__ void add4(float4& a, float4 b) {
-  a.x += b.x;
-  a.y += b.y;
-  a.z += b.z;
-  a.w += b.w;
-}
-
 // One CTA per (sequence, head, 16-column dv slice): the chain through its
-// chunks, operands from the workspace.  W Sigma_0 and Q' Sigma_0 share one
-// pass over the state, and the carry's product follows; each splits its
-// contraction over four groups of 64 threads (4 x 4 register tiles, partial
-// sums reduced through shared memory).
+// chunks, operands from the workspace, both products on the tensor cores
+// (3xTF32 MMAs, fp32 accumulate).  [W; Q'] Sigma_0: warp w takes 16 rows of W
+// (w < 4, giving U) or of Q' (w >= 4, giving O); the carry
+// (K o e^{G_C - G})^T U: warp w takes state rows 16 w .. 16 w + 15.  Each
+// output element belongs to one lane, so there is nothing to reduce.
 template <int DK, typename T>
 __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const Params p) {
   using PL = ChainPlan<DK>;
-  constexpr int NV = PL::NV, LDK = PL::LDK, LDS = PL::LDS;
-  constexpr int RG_FLOATS = PL::RROWS * NV;        // one group's partial sums
-  constexpr int TD = DK / 16;                      // carry rows per thread
+  constexpr int NV = PL::NV, LDA = PL::LDA, LDH = PL::LDH, LDS = PL::LDS;
   extern __shared__ __align__(16) float sm[];
   float* sW = sm + PL::W;
   float* sQp = sm + PL::QP;
@@ -1128,10 +1130,10 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
   float* sU = sm + PL::U;
   float* sUt = sm + PL::UT;
   float* sOt = sm + PL::OT;
-  float* sRed = sm + PL::RED;
   float* sEGC = sm + PL::EGC;
 
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, g = (tid & 31) >> 2, q = tid & 3;
   const int n_slices = p.dv / NV;
   const int slice = blockIdx.x % n_slices;
   const int chain = blockIdx.x / n_slices;
@@ -1147,163 +1149,108 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
   T* o = static_cast<T*>(p.o);
 
   // Operand groups of chunk c, one cp.async group each (empty past the last
-  // chunk): A1, the state pass's (W, Q'); A2, its reduction's (the U~ and O~
-  // slices); B, the carry's (K o e^{G_C - G}, e^{G_C}).
-  auto load_a1 = [&](int c) {
+  // chunk): W and Q' into buffer c & 1; the carry's K o e^{G_C - G} and
+  // e^{G_C}; the U~ and O~ slices.
+  auto load_w = [&](int c) {
     if (c < n_chunks) {
       const size_t w = (size_t)(slot0 + c) * H + h;
-      copy_rows<C, DK, LDK>(sW, p.ws.W + w * C * DK, tid);
-      copy_rows<C, DK, LDK>(sQp, p.ws.Qp + w * C * DK, tid);
+      copy_rows<C, DK, LDA>(sW + (c & 1) * C * LDA, p.ws.W + w * C * DK, tid);
+      copy_rows<C, DK, LDA>(sQp + (c & 1) * C * LDA, p.ws.Qp + w * C * DK, tid);
     }
     cp_async_commit();
   };
-  auto load_a2 = [&](int c) {
+  auto load_k = [&](int c) {
+    if (c < n_chunks) {
+      const size_t w = (size_t)(slot0 + c) * H + h;
+      copy_rows<C, DK, LDH>(sKh, p.ws.Kh + w * C * DK, tid);
+      if (tid < DK / 4) cp_async16(sEGC + 4 * tid, p.ws.EGC + w * DK + 4 * tid);
+    }
+    cp_async_commit();
+  };
+  auto load_u = [&](int c) {
     if (c < n_chunks) {
       const size_t base = ((size_t)(slot0 + c) * H + h) * C * (size_t)dv + col0;
       for (int e = tid; e < 2 * C * (NV / 4); e += THREADS) {
         const int m = e / (C * (NV / 4)), r = e % (C * (NV / 4));
-        const int i = r / (NV / 4), q = r % (NV / 4);
-        cp_async16((m ? sOt : sUt) + i * LDS + 4 * q, (m ? p.ws.Ot : p.ws.Ut) + base + (size_t)i * dv + 4 * q);
+        const int i = r / (NV / 4), c4 = r % (NV / 4);
+        cp_async16((m ? sOt : sUt) + i * LDS + 4 * c4, (m ? p.ws.Ot : p.ws.Ut) + base + (size_t)i * dv + 4 * c4);
       }
-    }
-    cp_async_commit();
-  };
-  auto load_b = [&](int c) {
-    if (c < n_chunks) {
-      const size_t w = (size_t)(slot0 + c) * H + h;
-      copy_rows<C, DK, LDK>(sKh, p.ws.Kh + w * C * DK, tid);
-      if (tid < DK / 4) cp_async16(sEGC + (c & 1) * DK + 4 * tid, p.ws.EGC + w * DK + 4 * tid);
     }
     cp_async_commit();
   };
 
-  load_a1(0);
-  load_a2(0);
-  load_b(0);
+  load_w(0);
+  load_u(0);
   for (int e = tid; e < DK * NV; e += THREADS) {
     const int d = e / NV, c = e % NV;
     sSig[d * LDS + c] = p.S0 ? p.S0[sbase + (size_t)d * dv + c] : 0.f;
   }
-  // split products: group g of 64 threads, 4 x 4 tile (rows 4 rt .., columns 4 ct ..)
-  const int g = tid >> 6, rt = (tid & 63) >> 2, ct = tid & 3;
-  const int r0 = 4 * rt, c0 = 4 * ct;
-  float* red = sRed + g * RG_FLOATS;
-  // Groups in flight at each wait, oldest first: [A1 c, A2 c, B c] before the
-  // state pass, [A2 c, B c] before its reduction, [B c, A1 c+1] before the
-  // carry; a refill is issued only after the barrier that ends its buffers'
-  // last reader.
+  // Groups in flight, oldest first: [W c, U c] at the top of chunk c (then K c
+  // and W c+1 are issued), [K c, W c+1] before the carry (then U c+1); a
+  // buffer is refilled only after the barrier that ends its last reader.
   for (int c = 0; c < n_chunks; ++c) {
     const int tok0 = t0 + c * C, valid = min(C, t1 - tok0);
-    cp_async_wait<2>();                            // W and Q'
+    cp_async_wait<0>();
     __syncthreads();
-    // ---- W Sigma_0 and Q' Sigma_0, dk split four ways
+    load_k(c);
+    load_w(c + 1);
+    // ---- U = U~ - W Sigma_0 (warps 0-3) and O = scale (Q' Sigma_0 + O~)
+    // with the output gate and the loop residual (warps 4-7)
     {
-      float ax[4][4] = {}, aq[4][4] = {};
-      constexpr int KR = DK / 4;
-#pragma unroll 2
-      for (int k = g * KR; k < (g + 1) * KR; k += 4) {
-        float4 wx[4], qx[4];
+      const int r0 = 16 * (warp & 3);
+      const float* A = ((warp < 4) ? sW : sQp) + (c & 1) * C * LDA + r0 * LDA;
+      float acc[2][3][4] = {};
+#pragma unroll 4
+      for (int k0 = 0; k0 < DK; k0 += 8) mma_step<LDS>(acc, A, LDA, 1, sSig, k0, g, q);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          wx[i] = lds4(sW + (r0 + i) * LDK + k);
-          qx[i] = lds4(sQp + (r0 + i) * LDK + k);
-        }
-        float b[4][4];
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) ldv<4>(sSig + (k + kk) * LDS + c0, b[kk]);
+        for (int hf = 0; hf < 2; ++hf) {
+          const int row = r0 + g + 8 * hf, col = 8 * nt + 2 * q;
+          const float x0 = acc[nt][0][2 * hf] + (acc[nt][1][2 * hf] + acc[nt][2][2 * hf]);
+          const float x1 = acc[nt][0][2 * hf + 1] + (acc[nt][1][2 * hf + 1] + acc[nt][2][2 * hf + 1]);
+          if (warp < 4) {
+            const float2 ut = *reinterpret_cast<const float2*>(sUt + row * LDS + col);
+            *reinterpret_cast<float2*>(sU + row * LDS + col) = make_float2(ut.x - x0, ut.y - x1);
+          } else if (row < valid) {
+            const float2 ot = *reinterpret_cast<const float2*>(sOt + row * LDS + col);
+            const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + row) * H + h])) : 1.f;
+            const float sv[2] = {x0 + ot.x, x1 + ot.y};
+            const size_t obase = ((size_t)(tok0 + row) * H + h) * dv + col0 + col;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          fma4<4>(ax[i], wx[i], b);
-          fma4<4>(aq[i], qx[i], b);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        stv<4>(red + red_off(r0 + i, ct), ax[i]);
-        stv<4>(red + red_off(C + r0 + i, ct), aq[i]);
-      }
-    }
-    cp_async_wait<1>();                            // the U~ and O~ slices
-    __syncthreads();
-    load_a1(c + 1);
-    // ---- reduce: U = U~ - sum -> sU; O = scale (sum + O~) with the output
-    // gate and the loop residual
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const int e = tid + THREADS * m;
-      const int row = e >> 2, c4 = e & 3;
-      const int off = red_off(row, c4);
-      float4 s = lds4(sRed + off);
-#pragma unroll
-      for (int gg = 1; gg < 4; ++gg) add4(s, lds4(sRed + gg * RG_FLOATS + off));
-      if (row < C) {
-        const float4 ut = lds4(sUt + row * LDS + 4 * c4);
-        *reinterpret_cast<float4*>(sU + row * LDS + 4 * c4) =
-            make_float4(ut.x - s.x, ut.y - s.y, ut.z - s.z, ut.w - s.w);
-      } else {
-        const int r = row - C;
-        if (r < valid) {
-          add4(s, lds4(sOt + r * LDS + 4 * c4));
-          const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + r) * H + h])) : 1.f;
-          const float sv[4] = {s.x, s.y, s.z, s.w};
-          const size_t obase = ((size_t)(tok0 + r) * H + h) * dv + col0 + 4 * c4;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float y = p.scale * sv[j];
-            if (p.gate) y *= og;
-            if (p.h_prev) {
-              const float hp = to_f32(static_cast<const T*>(p.h_prev)[obase + j]);
-              y = fmaf(p.rho[(size_t)h * dv + col0 + 4 * c4 + j], hp, to_f32(from_f32<T>(y)));
+            for (int j = 0; j < 2; ++j) {
+              float y = p.scale * sv[j];
+              if (p.gate) y *= og;
+              if (p.h_prev) {
+                const float hp = to_f32(static_cast<const T*>(p.h_prev)[obase + j]);
+                y = fmaf(p.rho[(size_t)h * dv + col0 + col + j], hp, to_f32(from_f32<T>(y)));
+              }
+              o[obase + j] = from_f32<T>(y);
             }
-            o[obase + j] = from_f32<T>(y);
           }
         }
-      }
     }
-    cp_async_wait<1>();                            // the carry's group
+    cp_async_wait<1>();                            // the carry's operands (W c+1 may fly)
     __syncthreads();
-    load_a2(c + 1);
-    // ---- (K o e^{G_C - G})^T U, the chunk's rows split four ways
-    {
-      float as[TD][4] = {};
-      const int d0 = TD * rt;
-#pragma unroll 1
-      for (int i = 16 * g; i < 16 * g + 16; i += 4) {
-        float u[4][4];
+    load_u(c + 1);
+    // ---- Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
+    if (16 * warp < DK) {
+      const int d0 = 16 * warp;
+      float acc[2][3][4] = {};
 #pragma unroll
-        for (int x = 0; x < 4; ++x) ldv<4>(sU + (i + x) * LDS + c0, u[x]);
+      for (int k0 = 0; k0 < C; k0 += 8) mma_step<LDS>(acc, sKh + d0, 1, LDH, sU, k0, g, q);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int q4 = 0; q4 < TD / 4; ++q4) {
-            const float4 kh = lds4(sKh + (i + x) * LDK + d0 + 4 * q4);
-            const float kv[4] = {kh.x, kh.y, kh.z, kh.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-#pragma unroll
-              for (int j = 0; j < 4; ++j) as[4 * q4 + e][j] = fmaf(kv[e], u[x][j], as[4 * q4 + e][j]);
-          }
+        for (int hf = 0; hf < 2; ++hf) {
+          const int d = d0 + g + 8 * hf, col = 8 * nt + 2 * q;
+          const float x0 = acc[nt][0][2 * hf] + (acc[nt][1][2 * hf] + acc[nt][2][2 * hf]);
+          const float x1 = acc[nt][0][2 * hf + 1] + (acc[nt][1][2 * hf + 1] + acc[nt][2][2 * hf + 1]);
+          float2* sg = reinterpret_cast<float2*>(sSig + d * LDS + col);
+          const float2 old = *sg;
+          const float gd = sEGC[d];
+          *sg = make_float2(fmaf(gd, old.x, x0), fmaf(gd, old.y, x1));
         }
-      }
-#pragma unroll
-      for (int e = 0; e < TD; ++e) stv<4>(red + red_off(d0 + e, ct), as[e]);
-    }
-    __syncthreads();
-    load_b(c + 1);
-    // ---- reduce: Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
-    const float* egc = sEGC + (c & 1) * DK;
-#pragma unroll
-    for (int m = 0; m < DK / 64; ++m) {
-      const int e = tid + THREADS * m;
-      const int d = e >> 2, c4 = e & 3;
-      const int off = red_off(d, c4);
-      float4 s = lds4(sRed + off);
-#pragma unroll
-      for (int gg = 1; gg < 4; ++gg) add4(s, lds4(sRed + gg * RG_FLOATS + off));
-      float4* sg = reinterpret_cast<float4*>(sSig + d * LDS + 4 * c4);
-      const float4 old = *sg;
-      const float gd = egc[d];
-      *sg = make_float4(fmaf(gd, old.x, s.x), fmaf(gd, old.y, s.y), fmaf(gd, old.z, s.z), fmaf(gd, old.w, s.w));
     }
   }
   cp_async_wait<0>();

@@ -598,8 +598,8 @@ def bench_kda(dev, args, peaks, world, L=4096, H=16):
             "achieved_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
             "clocks": clocks.summary(),
             "kernel": "gdn_prefill_kda_prep_kernel (one CTA per chunk and head: decayed operands, T, W, Q', "
-                      "U~, O~) + gdn_prefill_kda_chain_kernel (one CTA per (sequence, head, 16 columns)); "
-                      "fp32 CUDA cores"}
+                      "U~, O~; fp32 CUDA cores) + gdn_prefill_kda_chain_kernel (one CTA per (sequence, head, "
+                      "16 columns); 3xTF32 warp MMAs)"}
 
 
 def bench_backward(dev, args, peaks, world):

@@ -198,7 +198,8 @@ gdn_status gdn_chunk_fwd_schedule(const gdn_fwd_params *p, int *n_segs, int *seg
  * launch sorts the sequences by length on the device (longest first, into the
  * workspace) and the blocks take them in that order, so that the longest
  * chains do not start last.  The outputs do not depend on the order.
- * With GDN_CHANNEL_GATE (fp32 CUDA-core kernels, any io dtype) and a
+ * With GDN_CHANNEL_GATE (fp32 arithmetic, the chain's products as 3xTF32
+ * warp MMAs with fp32 accumulation; any io dtype) and a
  * workspace, a first launch takes every (chunk, head) at once and writes its
  * decayed operands, T = (I + A)^{-1} and the state-independent products
  * W = T diag(b) (K o e^G), Q' = Q o e^G - P W, U~ = T diag(b) V and

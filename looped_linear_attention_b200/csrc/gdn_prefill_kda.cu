@@ -1,5 +1,6 @@
-// Chunkwise prefill of the per-channel (diagonal) gate variant, KDA, with fp32
-// operands on the CUDA cores.
+// Chunkwise prefill of the per-channel (diagonal) gate variant, KDA, in fp32:
+// CUDA-core kernels, the chain launch's two products on warp-level 3xTF32
+// MMAs (fp32 accumulate).
 //
 // KDA is named among the LT2 mixers ("LT2: Linear-Time Looped Transformers",
 // Appendix C) and is the DPLR block of §2 / Appendix B.1 with a diagonal

@@ -31,6 +31,7 @@
 // launch split it (the two-launch section below).  The output epilogue
 // (head-wise gate, loop residual) is the precise path's.
 #include "common.cuh"
+#include "tma_host.h"
 
 namespace gdn {
 namespace kda {
@@ -168,7 +169,8 @@ static_assert(Plan<128>::BYTES <= 232448, "KDA prefill shared memory");
 // operands once the state-independent products are folded in (W, Q', U~ and
 // O~ below) and its decay over the chunk.
 struct Ws {
-  float *W, *Qp, *Kh;    // [slots][H][C][dk]: T diag(b) (K o e^G), Q o e^G - P W, K o e^{G_C - G}
+  float *W, *Qp;         // [slots][H][C][dk]: T diag(b) (K o e^G), Q o e^G - P W
+  float* KhT;            // [slots][H][dk][C]: (K o e^{G_C - G})^T
   float *Ut, *Ot;        // [slots][H][C][dv]: U~ = T diag(b) V, O~ = P U~
   float* EGC;            // [slots][H][dk]: e^{G_C}
   long long n_slots;
@@ -887,10 +889,12 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
   const bool factored = !__syncthreads_or(wide);
   // ---- the decayed operands: factored ones to shared memory (K^ over K, K~
   // over G, Q~ over Q, e^m per channel) or the plain K, Q, G;
-  // K o e^{G_C - G} and e^{G_C} to the workspace
+  // (K o e^{G_C - G})^T and e^{G_C} to the workspace
   const size_t w = (size_t)slot * H + h;
-  float* kh = p.ws.Kh + w * C * DK;
+  float* kht = p.ws.KhT + w * C * DK;
   float* sEm = sm + PL::MID;                       // [DK] e^m of a factored chunk
+  float* sEc = sEm + DK;                           // [DK] e^{G_C - m} of a factored chunk
+  float* sGc = sEc + DK;                           // [DK] G_C
   if (factored) {
     float em[4], ec[4];
 #pragma unroll
@@ -898,7 +902,10 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
       em[c] = expf(mid[c]);
       ec[c] = expf(gc[c] - mid[c]);
     }
-    if (rg == 0) st4(sEm + d0, em[0], em[1], em[2], em[3]);
+    if (rg == 0) {
+      st4(sEm + d0, em[0], em[1], em[2], em[3]);
+      st4(sEc + d0, ec[0], ec[1], ec[2], ec[3]);
+    }
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       float kt[4], kc[4], qt[4];
@@ -914,24 +921,28 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_prep_kernel(const 
       st4(sK + i * LDK + d0, kc[0], kc[1], kc[2], kc[3]);
       st4(sG + i * LDK + d0, kt[0], kt[1], kt[2], kt[3]);
       st4(sQ + i * LDK + d0, qt[0], qt[1], qt[2], qt[3]);
-      st4(kh + i * DK + d0, kc[0] * ec[0], kc[1] * ec[1], kc[2] * ec[2], kc[3] * ec[3]);
     }
   } else {
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
-      float a3[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) a3[c] = kr[r][c] * expf(gc[c] - g[r][c]);
       const int i = i0 + r;
       st4(sK + i * LDK + d0, kr[r][0], kr[r][1], kr[r][2], kr[r][3]);
       st4(sQ + i * LDK + d0, qr[r][0], qr[r][1], qr[r][2], qr[r][3]);
       st4(sG + i * LDK + d0, g[r][0], g[r][1], g[r][2], g[r][3]);
-      st4(kh + i * DK + d0, a3[0], a3[1], a3[2], a3[3]);
     }
   }
-  if (rg == 0)
+  if (rg == 0) {
+    st4(sGc + d0, gc[0], gc[1], gc[2], gc[3]);
     st4(p.ws.EGC + w * DK + d0, expf(gc[0]), expf(gc[1]), expf(gc[2]), expf(gc[3]));
+  }
   __syncthreads();
+  // ---- (K o e^{G_C - G})^T to the workspace ([dk][C]), stores coalesced
+  // along the chunk's rows: K^ e^{G_C - m} (factored) or K e^{G_C - G}
+  for (int e = tid; e < DK * C; e += THREADS) {
+    const int d = e / C, i = e % C;
+    const float kv = sK[i * LDK + d];
+    kht[e] = factored ? kv * sEc[d] : kv * expf(sGc[d] - sG[i * LDK + d]);
+  }
   // ---- A and P
   if (factored) ap_factored<DK, PL>(sm, tid);
   else ap_exact<DK, PL>(sm, tid);
@@ -1066,17 +1077,46 @@ __device__ __forceinline__ void mma_16x8x8(float (&d)[4], const uint32_t (&a)[4]
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// acc[nt] += A (16 x 8, element (m, k) at A[m * lda_m + k * lda_k]) times
-// B (8 x 16, element (k, n) at B[k * LDB + n]) for k-step k0, fragments of
-// lane (g = lane / 4, q = lane % 4), both n-tiles.
-template <int LDB>
-__device__ __forceinline__ void mma_step(float (&acc)[2][3][4], const float* A, int lda_m, int lda_k, const float* B,
-                                         int k0, int g, int q) {
+// A chain's state slice of NV = 16 columns and the chunk's operands.  W, Q'
+// (by chunk parity) and (K o e^{G_C - G})^T arrive as TMA boxes of 32 fp32
+// columns in the 128-byte swizzle (element (r, k) of a box at row r, 16-byte
+// chunk (k / 4) xor (r % 8)), which keeps the fragment reads conflict-free;
+// the state and U are padded rows (B fragments, banks 24 q + g).
+template <int DK>
+struct ChainPlan {
+  static constexpr int NV = 16;
+  static constexpr int LDS = NV + 8;
+  static constexpr int TILE = C * DK;              // floats of one W, Q' or K^T tile
+  static constexpr int W = 0;                      // 2 tiles, by chunk parity: DK / 32 boxes of [C][32]
+  static constexpr int QP = W + 2 * TILE;          // 2 tiles
+  static constexpr int KT = QP + 2 * TILE;         // C / 32 boxes of [DK][32]
+  static constexpr int SIG = KT + TILE;            // [DK][LDS]
+  static constexpr int U = SIG + DK * LDS;         // [C][LDS]
+  static constexpr int UT = U + C * LDS;           // [C][LDS]  U~ slice
+  static constexpr int OT = UT + C * LDS;          // [C][LDS]  O~ slice
+  static constexpr int EGC = OT + C * LDS;         // [DK]      e^{G_C}
+  static constexpr int BAR = EGC + DK;             // mbarriers: W / Q' by parity, K^T; abort flag
+  static constexpr int FLOATS = BAR + 8;
+  static constexpr size_t BYTES = (size_t)FLOATS * 4 + 1024;   // + alignment of the base to 1024 bytes
+};
+static_assert(ChainPlan<128>::BYTES <= 232448, "KDA chain shared memory");
+static_assert(ChainPlan<128>::TILE % 256 == 0 && ChainPlan<64>::TILE % 256 == 0, "1024-byte tile alignment");
+
+// Element (r, k) of a swizzled tile of boxes [rows][32] (box = k / 32).
+template <int ROWS>
+__device__ __forceinline__ float sw_at(const float* tile, int r, int k) {
+  return tile[(k >> 5) * ROWS * 32 + r * 32 + ((((k & 31) >> 2) ^ (r & 7)) << 2) + (k & 3)];
+}
+
+// acc[nt] += A (16 x 8 at rows m0.., k-step k0, A read through `a_at`) times
+// B (8 x 16, element (k, n) at B[k * LDB + n]), fragments of lane (g, q).
+template <int LDB, typename AAt>
+__device__ __forceinline__ void mma_step(float (&acc)[2][3][4], AAt a_at, const float* B, int k0, int g, int q) {
   uint32_t ah[4], al[4];
-  tf32_split(A[g * lda_m + (k0 + q) * lda_k], ah[0], al[0]);
-  tf32_split(A[(g + 8) * lda_m + (k0 + q) * lda_k], ah[1], al[1]);
-  tf32_split(A[g * lda_m + (k0 + q + 4) * lda_k], ah[2], al[2]);
-  tf32_split(A[(g + 8) * lda_m + (k0 + q + 4) * lda_k], ah[3], al[3]);
+  tf32_split(a_at(g, k0 + q), ah[0], al[0]);
+  tf32_split(a_at(g + 8, k0 + q), ah[1], al[1]);
+  tf32_split(a_at(g, k0 + q + 4), ah[2], al[2]);
+  tf32_split(a_at(g + 8, k0 + q + 4), ah[3], al[3]);
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
     uint32_t bh[2], bl[2];
@@ -1088,30 +1128,20 @@ __device__ __forceinline__ void mma_step(float (&acc)[2][3][4], const float* A, 
   }
 }
 
-// A chain's state slice of NV = 16 columns and the chunk's operands: W and Q'
-// by chunk parity (the next chunk's load while this one is used), the carry's
-// K o e^{G_C - G} and the U~ and O~ slices in single buffers.  Row strides
-// make every fragment read conflict-free: W and Q' rows (A, banks 4 g + q),
-// K o e^{G_C - G} rows read transposed (A, banks 8 q + g), the state and U
-// (B, banks 24 q + g).
-template <int DK>
-struct ChainPlan {
-  static constexpr int NV = 16;
-  static constexpr int LDA = DK + 4;
-  static constexpr int LDH = DK + 8;
-  static constexpr int LDS = NV + 8;
-  static constexpr int W = 0;                      // 2 x [C][LDA]  T diag(b) (K o e^G)
-  static constexpr int QP = W + 2 * C * LDA;       // 2 x [C][LDA]  Q o e^G - P W
-  static constexpr int KH = QP + 2 * C * LDA;      // [C][LDH]      K o e^{G_C - G}
-  static constexpr int SIG = KH + C * LDH;         // [DK][LDS]
-  static constexpr int U = SIG + DK * LDS;         // [C][LDS]
-  static constexpr int UT = U + C * LDS;           // [C][LDS]      U~ slice
-  static constexpr int OT = UT + C * LDS;          // [C][LDS]      O~ slice
-  static constexpr int EGC = OT + C * LDS;         // [DK]          e^{G_C}
-  static constexpr int FLOATS = EGC + DK;
-  static constexpr size_t BYTES = (size_t)FLOATS * 4;
-};
-static_assert(ChainPlan<128>::BYTES <= 232448, "KDA chain shared memory");
+__device__ __forceinline__ void kda_tma_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void kda_bulk(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 
 // One CTA per (sequence, head, 16-column dv slice): the chain through its
 // chunks, operands from the workspace, both products on the tensor cores
@@ -1120,21 +1150,27 @@ static_assert(ChainPlan<128>::BYTES <= 232448, "KDA chain shared memory");
 // (K o e^{G_C - G})^T U: warp w takes state rows 16 w .. 16 w + 15.  Each
 // output element belongs to one lane, so there is nothing to reduce.
 template <int DK, typename T>
-__global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const Params p) {
+__global__ void __launch_bounds__(THREADS, 1)
+    gdn_prefill_kda_chain_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
+                                 const __grid_constant__ CUtensorMap tm_kt, const Params p) {
   using PL = ChainPlan<DK>;
-  constexpr int NV = PL::NV, LDA = PL::LDA, LDH = PL::LDH, LDS = PL::LDS;
-  extern __shared__ __align__(16) float sm[];
+  constexpr int NV = PL::NV, LDS = PL::LDS, TILE = PL::TILE;
+  extern __shared__ __align__(16) unsigned char smraw[];
+  float* sm = reinterpret_cast<float*>(smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u));
   float* sW = sm + PL::W;
   float* sQp = sm + PL::QP;
-  float* sKh = sm + PL::KH;
+  float* sKt = sm + PL::KT;
   float* sSig = sm + PL::SIG;
   float* sU = sm + PL::U;
   float* sUt = sm + PL::UT;
   float* sOt = sm + PL::OT;
   float* sEGC = sm + PL::EGC;
+  uint64_t* bar_w = reinterpret_cast<uint64_t*>(sm + PL::BAR);   // [2], W and Q' by buffer
+  uint64_t* bar_k = bar_w + 2;                                    // the carry's operands
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_w + 3);
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5, g = (tid & 31) >> 2, q = tid & 3;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
   const int n_slices = p.dv / NV;
   const int slice = blockIdx.x % n_slices;
   const int chain = blockIdx.x / n_slices;
@@ -1149,24 +1185,30 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
   const size_t sbase = ((size_t)seq * H + h) * DK * (size_t)dv + col0;
   T* o = static_cast<T*>(p.o);
 
-  // Operand groups of chunk c, one cp.async group each (empty past the last
-  // chunk): W and Q' into buffer c & 1; the carry's K o e^{G_C - G} and
-  // e^{G_C}; the U~ and O~ slices.
-  auto load_w = [&](int c) {
-    if (c < n_chunks) {
-      const size_t w = (size_t)(slot0 + c) * H + h;
-      copy_rows<C, DK, LDA>(sW + (c & 1) * C * LDA, p.ws.W + w * C * DK, tid);
-      copy_rows<C, DK, LDA>(sQp + (c & 1) * C * LDA, p.ws.Qp + w * C * DK, tid);
+  // Thread 0 issues W and Q' of chunk c (into buffer c & 1) and the carry's
+  // (K o e^{G_C - G})^T and e^{G_C}, each after the barrier that ends its
+  // buffer's last reader; the U~ and O~ slices are one cp.async group per
+  // chunk (empty past the last chunk).
+  int issued_w0 = 0, issued_w1 = 0, issued_k = 0;  // thread 0's count of each barrier's phases
+  auto issue_w = [&](int c) {
+    const int y = (int)(((slot0 + c) * H + h) * C);
+    uint64_t* bar = &bar_w[c & 1];
+    mbar_arrive_expect_tx(bar, 2 * TILE * 4);
+#pragma unroll
+    for (int b = 0; b < DK / 32; ++b) {
+      kda_tma_2d(sW + (c & 1) * TILE + b * C * 32, &tm_w, bar, 32 * b, y);
+      kda_tma_2d(sQp + (c & 1) * TILE + b * C * 32, &tm_q, bar, 32 * b, y);
     }
-    cp_async_commit();
+    if (c & 1) ++issued_w1;
+    else ++issued_w0;
   };
-  auto load_k = [&](int c) {
-    if (c < n_chunks) {
-      const size_t w = (size_t)(slot0 + c) * H + h;
-      copy_rows<C, DK, LDH>(sKh, p.ws.Kh + w * C * DK, tid);
-      if (tid < DK / 4) cp_async16(sEGC + 4 * tid, p.ws.EGC + w * DK + 4 * tid);
-    }
-    cp_async_commit();
+  auto issue_k = [&](int c) {
+    const size_t w = (size_t)(slot0 + c) * H + h;
+    mbar_arrive_expect_tx(bar_k, (TILE + DK) * 4);
+#pragma unroll
+    for (int b = 0; b < C / 32; ++b) kda_tma_2d(sKt + b * DK * 32, &tm_kt, bar_k, 32 * b, (int)(w * DK));
+    kda_bulk(sEGC, p.ws.EGC + w * DK, DK * 4, bar_k);
+    ++issued_k;
   };
   auto load_u = [&](int c) {
     if (c < n_chunks) {
@@ -1180,29 +1222,41 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
     cp_async_commit();
   };
 
-  load_w(0);
+  if (tid == 0) {
+    mbar_init(&bar_w[0], 1);
+    mbar_init(&bar_w[1], 1);
+    mbar_init(bar_k, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0 && n_chunks > 0) issue_w(0);
   load_u(0);
   for (int e = tid; e < DK * NV; e += THREADS) {
     const int d = e / NV, c = e % NV;
     sSig[d * LDS + c] = p.S0 ? p.S0[sbase + (size_t)d * dv + c] : 0.f;
   }
-  // Groups in flight, oldest first: [W c, U c] at the top of chunk c (then K c
-  // and W c+1 are issued), [K c, W c+1] before the carry (then U c+1); a
-  // buffer is refilled only after the barrier that ends its last reader.
+  // Every wait is bounded: a timeout records GDN_ERR_TIMEOUT, raises the
+  // abort flag, and the block leaves the loop at the next barrier.
   for (int c = 0; c < n_chunks; ++c) {
     const int tok0 = t0 + c * C, valid = min(C, t1 - tok0);
-    cp_async_wait<0>();
-    __syncthreads();
-    load_k(c);
-    load_w(c + 1);
+    const bool okw = mbar_wait_bounded(&bar_w[c & 1], (c >> 1) & 1, abort_flag, p.status);
+    cp_async_wait<0>();                            // the U~ and O~ slices
+    if (__syncthreads_or(!okw || *abort_flag != 0)) break;
+    if (tid == 0) {
+      fence_proxy_async_smem();                    // the last generic reads of the refilled buffers come first
+      issue_k(c);
+      if (c + 1 < n_chunks) issue_w(c + 1);
+    }
     // ---- U = U~ - W Sigma_0 (warps 0-3) and O = scale (Q' Sigma_0 + O~)
     // with the output gate and the loop residual (warps 4-7)
     {
       const int r0 = 16 * (warp & 3);
-      const float* A = ((warp < 4) ? sW : sQp) + (c & 1) * C * LDA + r0 * LDA;
+      const float* At = ((warp < 4) ? sW : sQp) + (c & 1) * TILE;
+      auto a_at = [&](int m, int k) { return sw_at<C>(At, r0 + m, k); };
       float acc[2][3][4] = {};
 #pragma unroll 4
-      for (int k0 = 0; k0 < DK; k0 += 8) mma_step<LDS>(acc, A, LDA, 1, sSig, k0, g, q);
+      for (int k0 = 0; k0 < DK; k0 += 8) mma_step<LDS>(acc, a_at, sSig, k0, g, q);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -1231,15 +1285,16 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
           }
         }
     }
-    cp_async_wait<1>();                            // the carry's operands (W c+1 may fly)
-    __syncthreads();
+    const bool okk = mbar_wait_bounded(bar_k, c & 1, abort_flag, p.status);
+    if (__syncthreads_or(!okk || *abort_flag != 0)) break;
     load_u(c + 1);
     // ---- Sigma_C = Diag(e^{G_C}) Sigma_0 + (K o e^{G_C - G})^T U
     if (16 * warp < DK) {
       const int d0 = 16 * warp;
+      auto a_at = [&](int m, int k) { return sw_at<DK>(sKt, d0 + m, k); };
       float acc[2][3][4] = {};
 #pragma unroll
-      for (int k0 = 0; k0 < C; k0 += 8) mma_step<LDS>(acc, sKh + d0, 1, LDH, sU, k0, g, q);
+      for (int k0 = 0; k0 < C; k0 += 8) mma_step<LDS>(acc, a_at, sU, k0, g, q);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -1254,9 +1309,15 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_prefill_kda_chain_kernel(const
         }
     }
   }
+  // leave no copy in flight: the last phase issued on each barrier
+  if (tid == 0) {
+    if (issued_w0 > 0) mbar_wait_bounded(&bar_w[0], (issued_w0 - 1) & 1, nullptr, p.status);
+    if (issued_w1 > 0) mbar_wait_bounded(&bar_w[1], (issued_w1 - 1) & 1, nullptr, p.status);
+    if (issued_k > 0) mbar_wait_bounded(bar_k, (issued_k - 1) & 1, nullptr, p.status);
+  }
   cp_async_wait<0>();
   __syncthreads();
-  if (p.S_T) {
+  if (p.S_T && *abort_flag == 0) {
     for (int e = tid; e < DK * NV; e += THREADS) {
       const int d = e / NV, c = e % NV;
       p.S_T[sbase + (size_t)d * dv + c] = sSig[d * LDS + c];
@@ -1280,11 +1341,18 @@ static cudaError_t launch_two(const Params& kp, long long chunk_blocks, long lon
   static std::atomic<bool> set_prep[kMaxDevices], set_chain[kMaxDevices];
   constexpr size_t prep_bytes = PrepPlan<DK>::BYTES;
   constexpr size_t chain_bytes = ChainPlan<DK>::BYTES;
+  // W, Q' as [slots * H * C][dk] and (K o e^{G_C - G})^T as [slots * H * dk][C],
+  // fp32, boxes of 32 columns x C or dk rows in the 128-byte swizzle
+  const long long sh = kp.ws.n_slots * kp.H;
+  CUtensorMap mw, mq, mk;
+  if (!make_map_2d(&mw, kp.ws.W, DK, sh * C, 32, C, 4) || !make_map_2d(&mq, kp.ws.Qp, DK, sh * C, 32, C, 4) ||
+      !make_map_2d(&mk, kp.ws.KhT, C, sh * DK, 32, DK, 4))
+    return cudaErrorInvalidValue;
   cudaError_t e = smem_attr_once(set_prep, gdn_prefill_kda_prep_kernel<DK, T>, prep_bytes);
   if (e == cudaSuccess) e = smem_attr_once(set_chain, gdn_prefill_kda_chain_kernel<DK, T>, chain_bytes);
   if (e != cudaSuccess) return e;
   gdn_prefill_kda_prep_kernel<DK, T><<<(unsigned)chunk_blocks, THREADS, prep_bytes, stream>>>(kp);
-  gdn_prefill_kda_chain_kernel<DK, T><<<(unsigned)chain_blocks, THREADS, chain_bytes, stream>>>(kp);
+  gdn_prefill_kda_chain_kernel<DK, T><<<(unsigned)chain_blocks, THREADS, chain_bytes, stream>>>(mw, mq, mk, kp);
   return cudaGetLastError();
 }
 
@@ -1336,7 +1404,7 @@ gdn_status launch_prefill_kda(const gdn_fwd_params* p, unsigned* status, void* w
     const size_t sh = (size_t)n_slots * p->H;
     const size_t dk = (size_t)p->dk, c = kda::C;
     char* w = static_cast<char*>(ws);
-    float** rows_dk[] = {&kp.ws.W, &kp.ws.Qp, &kp.ws.Kh};
+    float** rows_dk[] = {&kp.ws.W, &kp.ws.Qp, &kp.ws.KhT};
     for (float** a : rows_dk) {
       *a = reinterpret_cast<float*>(w);
       w += kda::align256(sh * c * dk * 4);

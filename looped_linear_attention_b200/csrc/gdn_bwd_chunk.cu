@@ -477,6 +477,9 @@ __device__ __forceinline__ void gemm_v(float (&acc)[TM][2], const float* A, cons
 __device__ __forceinline__ void cp_async16(float* smem, const float* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
+__device__ __forceinline__ void cp_async4(float* smem, const float* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -797,14 +800,14 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
 
   for (int col0 = 0; col0 < p.dv; col0 += NS) {
     __syncthreads();
-    // tiles of S and dE (transposed into [NS][DK]), dO (rows and transpose), V (registers)
+    // tiles of S and dE (transposed into [NS][DK] by 4-byte cp.async, every
+    // element in flight at once), dO (rows and transpose), V (registers)
     for (int e = tid; e < DK * NS; e += THREADS) {
       const int d = e / NS, cc = e % NS;
-      const float x = gS[(size_t)d * p.dv + col0 + cc], y = gE[(size_t)d * p.dv + col0 + cc];
-      sSt[cc * LDK + d] = x;
-      sEt[cc * LDK + d] = y;
-      es = fmaf(x, y, es);
+      cp_async4(sSt + cc * LDK + d, gS + (size_t)d * p.dv + col0 + cc);
+      cp_async4(sEt + cc * LDK + d, gE + (size_t)d * p.dv + col0 + cc);
     }
+    cp_async_commit();
     for (int e = tid; e < C * NS; e += THREADS) {
       const int i = e / NS, cc = e % NS;
       const float x = (i < n) ? ldx(go, ((size_t)(t0 + i) * p.H + h) * p.dv + col0 + cc) : 0.f;
@@ -817,7 +820,13 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
 #pragma unroll
       for (int u = 0; u < 2; ++u)
         vv[i][u] = (r0 + i < n) ? ldx(v, ((size_t)(t0 + r0 + i) * p.H + h) * p.dv + col0 + cg + 16 * u) : 0.f;
+    cp_async_wait<0>();
     __syncthreads();
+    // partial <dE, S> over this thread's elements, in the order they were loaded
+    for (int e = tid; e < DK * NS; e += THREADS) {
+      const int d = e / NS, cc = e % NS;
+      es = fmaf(sSt[cc * LDK + d], sEt[cc * LDK + d], es);
+    }
     // KS = K S_J, KdE = K dE_J (rows along k); R = diag(b) (V - diag(gamma) KS) -> R^T;
     // the first part of dU, diag(r) KdE, stays in registers
     float ks[4][2], du0[4][2];

@@ -188,15 +188,19 @@ __device__ __forceinline__ float4 ld4(const __nv_bfloat16* p, size_t i) {
   const uint2 u = *reinterpret_cast<const uint2*>(p + i);
   return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
 }
-template <typename T>
-__device__ __forceinline__ void load_rows4(float* dst, int ld, const T* src, int t0, int n, int h, int H,
-                                           int width, int cols, int tid) {
-  const int q = cols / 4;
-  for (int e = tid; e < C * q; e += THREADS) {
-    const int i = e / q, c = (e % q) * 4;
-    *reinterpret_cast<float4*>(dst + i * ld + c) =
-        (i < n) ? ld4(src, ((size_t)(t0 + i) * H + h) * width + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+__device__ __forceinline__ void cp_async16(float* smem, const float* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(float* smem, const float* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// 16 bytes, or zeros when !take (nothing is read then)
+__device__ __forceinline__ void cp_async16z(float* smem, const void* gmem, bool take) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(take ? 16 : 0)
+               : "memory");
 }
 __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
   return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
@@ -214,10 +218,38 @@ __device__ __forceinline__ void chunk_setup(const KParams& p, int t0, int n, int
                                             float* sKK, float* sP, float* sT, Vec V, float* s_carry,
                                             int tid) {
   constexpr int LDK = DK + 4;
-  load_rows4(sK, LDK, static_cast<const T*>(p.k), t0, n, h, p.H, DK, DK, tid);
-  load_rows4(sQ, LDK, static_cast<const T*>(p.q), t0, n, h, p.H, DK, DK, tid);
+  // K and Q rows staged with 16-byte cp.async, every piece in flight (rows
+  // past the end read nothing: zero fill): fp32 rows straight into their
+  // rows, bf16 rows into the KK and P areas (written only later), then widened
+  constexpr bool kF32 = sizeof(T) == 4;
+  {
+    constexpr int PIECES = DK * (int)sizeof(T) / 16;
+    constexpr int RAW = kF32 ? LDK : DK / 2;      // floats per staged row
+    float* rk = kF32 ? sK : sKK;
+    float* rq = kF32 ? sQ : sP;
+    const T* kg = static_cast<const T*>(p.k);
+    const T* qg = static_cast<const T*>(p.q);
+    for (int e = tid; e < C * PIECES; e += THREADS) {
+      const int i = e / PIECES, c = e % PIECES;
+      const size_t off = ((size_t)(t0 + min(i, n - 1)) * p.H + h) * DK;
+      cp_async16z(rk + i * RAW + 4 * c, reinterpret_cast<const char*>(kg + off) + 16 * c, i < n);
+      cp_async16z(rq + i * RAW + 4 * c, reinterpret_cast<const char*>(qg + off) + 16 * c, i < n);
+    }
+    cp_async_commit();
+  }
   chunk_gates(p, t0, n, h, V, s_carry, tid);
+  cp_async_wait<0>();
   __syncthreads();
+  if constexpr (!kF32) {
+    for (int e = tid; e < C * DK / 4; e += THREADS) {
+      const int i = e / (DK / 4), c = 4 * (e % (DK / 4));
+      const uint2 uk = *reinterpret_cast<const uint2*>(sKK + i * (DK / 2) + c / 2);
+      const uint2 uq = *reinterpret_cast<const uint2*>(sP + i * (DK / 2) + c / 2);
+      *reinterpret_cast<float4*>(sK + i * LDK + c) = make_float4(bf16_lo(uk.x), bf16_hi(uk.x), bf16_lo(uk.y), bf16_hi(uk.y));
+      *reinterpret_cast<float4*>(sQ + i * LDK + c) = make_float4(bf16_lo(uq.x), bf16_hi(uq.x), bf16_lo(uq.y), bf16_hi(uq.y));
+    }
+    __syncthreads();
+  }
   {
     // thread: rows r0 .. r0+3, columns cg + 16 j; both products read K and Q
     // along k four at a time (the row stride DK + 4 keeps the eight rows of a
@@ -474,15 +506,6 @@ __device__ __forceinline__ void gemm_v(float (&acc)[TM][2], const float* A, cons
 }
 
 // Asynchronous 16-byte copies global -> shared (per thread, in commit groups).
-__device__ __forceinline__ void cp_async16(float* smem, const float* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async4(float* smem, const float* gmem) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 // rows x cols fp32 (cols a multiple of 4) from global (row stride gld) into
 // shared memory (row stride sld), 16 bytes per copy.
 __device__ __forceinline__ void cp_rows(float* dst, int sld, const float* src, size_t gld, int rows, int cols,

@@ -420,14 +420,34 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_prep_kernel(const KParams 
       }
     }
   }
-  // U~ = T diag(b) V  [C][dv], 32 columns at a time
+  // U~ = T diag(b) V  [C][dv], 32 columns at a time; V's rows (io dtype) are
+  // staged with cp.async one block ahead, in two buffers over T (free since
+  // its transpose; rows past the end read nothing: zero fill)
   float* gU = p.Ut + wsi * C * p.dv;
-  for (int col0 = 0; col0 < p.dv; col0 += NS) {
-    __syncthreads();
+  constexpr int VP = NS * (int)sizeof(T) / 16;     // 16-byte pieces per row of a block
+  constexpr int VROWF = NS * (int)sizeof(T) / 4;   // floats per staged row
+  float* sVraw = sT;
+  const T* vg = static_cast<const T*>(p.v);
+  auto stage_v = [&](int col0, int buf) {
+    for (int e = tid; e < C * VP; e += THREADS) {
+      const int i = e / VP, c = e % VP;
+      const size_t off = ((size_t)(t0 + min(i, n - 1)) * p.H + h) * p.dv + col0;
+      cp_async16z(sVraw + buf * C * VROWF + i * VROWF + 4 * c, reinterpret_cast<const char*>(vg + off) + 16 * c,
+                  i < n);
+    }
+    cp_async_commit();
+  };
+  stage_v(0, 0);
+  for (int col0 = 0, buf = 0; col0 < p.dv; col0 += NS, buf ^= 1) {
+    if (col0 + NS < p.dv) stage_v(col0 + NS, buf ^ 1);
+    else cp_async_commit();
+    cp_async_wait<1>();                            // this block's rows
+    __syncthreads();                               // and the last block's product is done with sV
     for (int e = tid; e < C * NS; e += THREADS) {
       const int i = e / NS, cc = e % NS;
-      sV[i * LDN + cc] = (i < n) ? V.b[i] * ldx(static_cast<const T*>(p.v), ((size_t)(t0 + i) * p.H + h) * p.dv + col0 + cc)
-                                 : 0.f;
+      const float* raw = sVraw + buf * C * VROWF + i * VROWF;
+      const float x = (sizeof(T) == 4) ? raw[cc] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(raw)[cc]);
+      sV[i * LDN + cc] = V.b[i] * x;
     }
     __syncthreads();
     float acc[4][2];
@@ -447,6 +467,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_prep_kernel(const KParams 
 #pragma unroll
       for (int u = 0; u < 2; ++u) gU[(size_t)(r0 + i) * p.dv + col0 + cg + 16 * u] = acc[i][u];
   }
+  cp_async_wait<0>();
 }
 
 // Shared-memory plans of the state passes, 2 CTAs per SM.  Row strides are
@@ -830,13 +851,16 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
       cp_async4(sSt + cc * LDK + d, gS + (size_t)d * p.dv + col0 + cc);
       cp_async4(sEt + cc * LDK + d, gE + (size_t)d * p.dv + col0 + cc);
     }
-    cp_async_commit();
-    for (int e = tid; e < C * NS; e += THREADS) {
-      const int i = e / NS, cc = e % NS;
-      const float x = (i < n) ? ldx(go, ((size_t)(t0 + i) * p.H + h) * p.dv + col0 + cc) : 0.f;
-      sdO[i * LDN + cc] = x;
-      sdOt[cc * LDC + i] = x;
+    // dO rows of the block (io dtype) staged over R^T, which this block
+    // writes only after the next barrier (rows past the end: zero fill)
+    constexpr int OP = NS * (int)sizeof(T) / 16;
+    constexpr int OROW = NS * (int)sizeof(T) / 4;
+    for (int e = tid; e < C * OP; e += THREADS) {
+      const int i = e / OP, c = e % OP;
+      const size_t off = ((size_t)(t0 + min(i, n - 1)) * p.H + h) * p.dv + col0;
+      cp_async16z(sRt + i * OROW + 4 * c, reinterpret_cast<const char*>(go + off) + 16 * c, i < n);
     }
+    cp_async_commit();
     float vv[4][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -850,6 +874,15 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
       const int d = e / NS, cc = e % NS;
       es = fmaf(sSt[cc * LDK + d], sEt[cc * LDK + d], es);
     }
+    // dO into rows and transpose
+    for (int e = tid; e < C * NS; e += THREADS) {
+      const int i = e / NS, cc = e % NS;
+      const float* raw = sRt + i * OROW;
+      const float x = (sizeof(T) == 4) ? raw[cc] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(raw)[cc]);
+      sdO[i * LDN + cc] = x;
+      sdOt[cc * LDC + i] = x;
+    }
+    __syncthreads();
     // KS = K S_J, KdE = K dE_J (rows along k); R = diag(b) (V - diag(gamma) KS) -> R^T;
     // the first part of dU, diag(r) KdE, stays in registers
     float ks[4][2], du0[4][2];

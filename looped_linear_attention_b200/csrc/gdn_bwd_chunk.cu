@@ -191,9 +191,6 @@ __device__ __forceinline__ float4 ld4(const __nv_bfloat16* p, size_t i) {
 __device__ __forceinline__ void cp_async16(float* smem, const float* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
-__device__ __forceinline__ void cp_async4(float* smem, const float* gmem) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -789,6 +786,8 @@ struct GradPlan {
   static constexpr int FLOATS = VEC + 10 * C + 4;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
   static_assert(VEC - TILES >= 3 * C * LDC, "the final phase's three C x C matrices reuse the tile area");
+  static_assert(DU - U + C * LDN >= DK * NS && DRT - UT + NS * LDC >= DK * NS,
+                "a column block's S and dE rows are staged over U / dU and U^T / dR^T");
   static_assert(BYTES <= 232448, "shared memory of one CTA");
 };
 
@@ -844,12 +843,16 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
 
   for (int col0 = 0; col0 < p.dv; col0 += NS) {
     __syncthreads();
-    // tiles of S and dE (transposed into [NS][DK] by 4-byte cp.async, every
-    // element in flight at once), dO (rows and transpose), V (registers)
-    for (int e = tid; e < DK * NS; e += THREADS) {
-      const int d = e / NS, cc = e % NS;
-      cp_async4(sSt + cc * LDK + d, gS + (size_t)d * p.dv + col0 + cc);
-      cp_async4(sEt + cc * LDK + d, gE + (size_t)d * p.dv + col0 + cc);
+    // tiles of S and dE: [DK][NS] rows by 16-byte cp.async into the U / dU
+    // and U^T / dR^T areas (this block writes them only after its first
+    // product), transposed below into [NS][DK]; dO (rows and transpose); V
+    // (registers)
+    float* stS = sU;                               // U and dU are adjacent: DK x NS floats fit
+    float* stE = sUt;                              // so are U^T and dR^T
+    for (int e = tid; e < DK * NS / 4; e += THREADS) {
+      const int d = e / (NS / 4), c4 = 4 * (e % (NS / 4));
+      cp_async16(stS + d * NS + c4, gS + (size_t)d * p.dv + col0 + c4);
+      cp_async16(stE + d * NS + c4, gE + (size_t)d * p.dv + col0 + c4);
     }
     // dO rows of the block (io dtype) staged over R^T, which this block
     // writes only after the next barrier (rows past the end: zero fill)
@@ -869,10 +872,13 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_bwd_grads_kernel(const KParams
         vv[i][u] = (r0 + i < n) ? ldx(v, ((size_t)(t0 + r0 + i) * p.H + h) * p.dv + col0 + cg + 16 * u) : 0.f;
     cp_async_wait<0>();
     __syncthreads();
-    // partial <dE, S> over this thread's elements, in the order they were loaded
+    // S and dE transposed; the partial <dE, S> over this thread's elements
     for (int e = tid; e < DK * NS; e += THREADS) {
       const int d = e / NS, cc = e % NS;
-      es = fmaf(sSt[cc * LDK + d], sEt[cc * LDK + d], es);
+      const float x = stS[e], y = stE[e];
+      sSt[cc * LDK + d] = x;
+      sEt[cc * LDK + d] = y;
+      es = fmaf(x, y, es);
     }
     // dO into rows and transpose
     for (int e = tid; e < C * NS; e += THREADS) {

@@ -1091,8 +1091,11 @@ struct ChainPlan {
   static constexpr int QP = W + 2 * TILE;          // 2 tiles
   static constexpr int KT = QP + 2 * TILE;         // C / 32 boxes of [DK][32]
   static constexpr int SIG = KT + TILE;            // [DK][LDS]
-  static constexpr int U = SIG + DK * LDS;         // [C][LDS]
-  static constexpr int UT = U + C * LDS;           // [C][LDS]  U~ slice
+  static constexpr int SIGH = SIG + DK * LDS;      // [DK][LDS] the state split once per chunk: tf32 high part
+  static constexpr int SIGL = SIGH + DK * LDS;     // [DK][LDS] and remainder (the B operand of the state pass)
+  static constexpr int U = SIGL + DK * LDS;        // [C][LDS]  U's tf32 high part (the carry's B operand)
+  static constexpr int UL = U + C * LDS;           // [C][LDS]  and remainder
+  static constexpr int UT = UL + C * LDS;          // [C][LDS]  U~ slice
   static constexpr int OT = UT + C * LDS;          // [C][LDS]  O~ slice
   static constexpr int EGC = OT + C * LDS;         // [DK]      e^{G_C}
   static constexpr int BAR = EGC + DK;             // mbarriers: W / Q' by parity, K^T; abort flag
@@ -1108,10 +1111,12 @@ __device__ __forceinline__ float sw_at(const float* tile, int r, int k) {
   return tile[(k >> 5) * ROWS * 32 + r * 32 + ((((k & 31) >> 2) ^ (r & 7)) << 2) + (k & 3)];
 }
 
-// acc[nt] += A (16 x 8 at rows m0.., k-step k0, A read through `a_at`) times
-// B (8 x 16, element (k, n) at B[k * LDB + n]), fragments of lane (g, q).
+// acc[nt] += A (16 x 8 at rows m0.., k-step k0, A read through `a_at` and
+// split here) times B (8 x 16, element (k, n) at [k * LDB + n], already split
+// into tf32 high parts BH and remainders BL), fragments of lane (g, q).
 template <int LDB, typename AAt>
-__device__ __forceinline__ void mma_step(float (&acc)[2][3][4], AAt a_at, const float* B, int k0, int g, int q) {
+__device__ __forceinline__ void mma_step_split(float (&acc)[2][3][4], AAt a_at, const uint32_t* BH, const uint32_t* BL,
+                                               int k0, int g, int q) {
   uint32_t ah[4], al[4];
   tf32_split(a_at(g, k0 + q), ah[0], al[0]);
   tf32_split(a_at(g + 8, k0 + q), ah[1], al[1]);
@@ -1119,9 +1124,8 @@ __device__ __forceinline__ void mma_step(float (&acc)[2][3][4], AAt a_at, const 
   tf32_split(a_at(g + 8, k0 + q + 4), ah[3], al[3]);
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    uint32_t bh[2], bl[2];
-    tf32_split(B[(k0 + q) * LDB + 8 * nt + g], bh[0], bl[0]);
-    tf32_split(B[(k0 + q + 4) * LDB + 8 * nt + g], bh[1], bl[1]);
+    const int o0 = (k0 + q) * LDB + 8 * nt + g, o1 = o0 + 4 * LDB;
+    const uint32_t bh[2] = {BH[o0], BH[o1]}, bl[2] = {BL[o0], BL[o1]};
     mma_16x8x8(acc[nt][0], ah, bh);
     mma_16x8x8(acc[nt][1], ah, bl);
     mma_16x8x8(acc[nt][2], al, bh);
@@ -1161,7 +1165,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   float* sQp = sm + PL::QP;
   float* sKt = sm + PL::KT;
   float* sSig = sm + PL::SIG;
-  float* sU = sm + PL::U;
+  uint32_t* sSigH = reinterpret_cast<uint32_t*>(sm + PL::SIGH);
+  uint32_t* sSigL = reinterpret_cast<uint32_t*>(sm + PL::SIGL);
+  uint32_t* sUH = reinterpret_cast<uint32_t*>(sm + PL::U);
+  uint32_t* sUL = reinterpret_cast<uint32_t*>(sm + PL::UL);
   float* sUt = sm + PL::UT;
   float* sOt = sm + PL::OT;
   float* sEGC = sm + PL::EGC;
@@ -1234,7 +1241,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   load_u(0);
   for (int e = tid; e < DK * NV; e += THREADS) {
     const int d = e / NV, c = e % NV;
-    sSig[d * LDS + c] = p.S0 ? p.S0[sbase + (size_t)d * dv + c] : 0.f;
+    const float x = p.S0 ? p.S0[sbase + (size_t)d * dv + c] : 0.f;
+    sSig[d * LDS + c] = x;
+    tf32_split(x, sSigH[d * LDS + c], sSigL[d * LDS + c]);
   }
   // Every wait is bounded: a timeout records GDN_ERR_TIMEOUT, raises the
   // abort flag, and the block leaves the loop at the next barrier.
@@ -1256,7 +1265,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       auto a_at = [&](int m, int k) { return sw_at<C>(At, r0 + m, k); };
       float acc[2][3][4] = {};
 #pragma unroll 4
-      for (int k0 = 0; k0 < DK; k0 += 8) mma_step<LDS>(acc, a_at, sSig, k0, g, q);
+      for (int k0 = 0; k0 < DK; k0 += 8) mma_step_split<LDS>(acc, a_at, sSigH, sSigL, k0, g, q);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -1266,7 +1275,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           const float x1 = acc[nt][0][2 * hf + 1] + (acc[nt][1][2 * hf + 1] + acc[nt][2][2 * hf + 1]);
           if (warp < 4) {
             const float2 ut = *reinterpret_cast<const float2*>(sUt + row * LDS + col);
-            *reinterpret_cast<float2*>(sU + row * LDS + col) = make_float2(ut.x - x0, ut.y - x1);
+            uint2 uh, ul;
+            tf32_split(ut.x - x0, uh.x, ul.x);
+            tf32_split(ut.y - x1, uh.y, ul.y);
+            *reinterpret_cast<uint2*>(sUH + row * LDS + col) = uh;
+            *reinterpret_cast<uint2*>(sUL + row * LDS + col) = ul;
           } else if (row < valid) {
             const float2 ot = *reinterpret_cast<const float2*>(sOt + row * LDS + col);
             const float og = p.gate ? 1.f / (1.f + __expf(-p.gate[(size_t)(tok0 + row) * H + h])) : 1.f;
@@ -1294,7 +1307,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       auto a_at = [&](int m, int k) { return sw_at<DK>(sKt, d0 + m, k); };
       float acc[2][3][4] = {};
 #pragma unroll
-      for (int k0 = 0; k0 < C; k0 += 8) mma_step<LDS>(acc, a_at, sU, k0, g, q);
+      for (int k0 = 0; k0 < C; k0 += 8) mma_step_split<LDS>(acc, a_at, sUH, sUL, k0, g, q);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -1305,7 +1318,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           float2* sg = reinterpret_cast<float2*>(sSig + d * LDS + col);
           const float2 old = *sg;
           const float gd = sEGC[d];
-          *sg = make_float2(fmaf(gd, old.x, x0), fmaf(gd, old.y, x1));
+          const float2 nw = make_float2(fmaf(gd, old.x, x0), fmaf(gd, old.y, x1));
+          *sg = nw;
+          uint2 sh, sl;
+          tf32_split(nw.x, sh.x, sl.x);
+          tf32_split(nw.y, sh.y, sl.y);
+          *reinterpret_cast<uint2*>(sSigH + d * LDS + col) = sh;
+          *reinterpret_cast<uint2*>(sSigL + d * LDS + col) = sl;
         }
     }
   }
